@@ -1,0 +1,157 @@
+"""fp64 oracle of the Wukong interaction-stack forward -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` import this package. It wraps the plain C reference in
+``wk_oracle.c`` (see its header for the equations and their sources on the
+Wukong page) and streams a stack one layer at a time, so that a large workload
+needs only one layer's weights in host memory.
+
+Parity status: pinned by identities (tests/test_oracle_pins.py); the page prints
+no worked example of a whole layer.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int32), ("d", ctypes.c_int32), ("k", ctypes.c_int32), ("n_f", ctypes.c_int32),
+                ("n_l", ctypes.c_int32), ("mlp_num_linear", ctypes.c_int32),
+                ("mlp_dims", ctypes.POINTER(ctypes.c_int32)), ("ln_eps", ctypes.c_double),
+                ("dtype", ctypes.c_int32)]
+
+
+class _Layer(ctypes.Structure):
+    _fields_ = [("Y", ctypes.c_void_p), ("W", ctypes.POINTER(ctypes.c_void_p)),
+                ("b", ctypes.POINTER(ctypes.c_void_p)), ("fmb_gamma", ctypes.c_void_p),
+                ("fmb_beta", ctypes.c_void_p), ("W_L", ctypes.c_void_p), ("out_gamma", ctypes.c_void_p),
+                ("out_beta", ctypes.c_void_p)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(_build.build())
+        vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        L.wko_fm.argtypes = [i32, i32, i32, vp, vp, vp, vp]
+        L.wko_layernorm.argtypes = [i64, vp, vp, vp, dbl, vp]
+        L.wko_lcb.argtypes = [i32, i32, i32, vp, vp, vp]
+        L.wko_layer_forward.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(_Layer), i64, vp, vp,
+                                        ctypes.c_int, ctypes.c_int]
+        L.wko_layer_forward.restype = ctypes.c_int
+        L.wko_linear.argtypes = [i64, i64, i64, i32, vp, vp, ctypes.c_int, vp, vp]
+        L.wko_round_bf16.argtypes = [dbl]
+        L.wko_round_bf16.restype = dbl
+        _lib = L
+    return _lib
+
+
+def _c64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def fm(X, Y):
+    """F = (X X^T) Y for one example, by pairwise dot products. X [n,d], Y [n,k]."""
+    X, Y = _c64(X), _c64(Y)
+    n, d = X.shape
+    k = Y.shape[1]
+    P = np.empty((n, n))
+    F = np.empty((n, k))
+    lib().wko_fm(n, d, k, _ptr(X), _ptr(Y), _ptr(P), _ptr(F))
+    return F
+
+
+def layernorm(x, gamma=None, beta=None, eps=1e-5):
+    x = _c64(x).reshape(-1)
+    g = None if gamma is None else _c64(gamma).reshape(-1)
+    b = None if beta is None else _c64(beta).reshape(-1)
+    y = np.empty_like(x)
+    lib().wko_layernorm(x.size, _ptr(x), _ptr(g), _ptr(b), float(eps), _ptr(y))
+    return y
+
+
+def lcb(W_L, X):
+    """G = W_L X for one example. W_L [n_l, n], X [n, d]."""
+    W_L, X = _c64(W_L), _c64(X)
+    n_l, n = W_L.shape
+    d = X.shape[1]
+    G = np.empty((n_l, d))
+    lib().wko_lcb(n, d, n_l, _ptr(W_L), _ptr(X), _ptr(G))
+    return G
+
+
+def linear(x, W, b=None, relu=False):
+    """y = act(x W^T + b) on a batch x [n_ex, in]; W float32 [out, in] or uint16 bf16 bits."""
+    x = _c64(x)
+    W = np.ascontiguousarray(W)
+    dt = 1 if W.dtype == np.uint16 else 0
+    if dt == 0:
+        W = W.astype(np.float32)
+    bb = None if b is None else np.ascontiguousarray(b, dtype=np.float32)
+    n_ex, i = x.shape
+    o = W.shape[0]
+    y = np.empty((n_ex, o))
+    lib().wko_linear(n_ex, i, o, dt, _ptr(W), _ptr(bb), int(relu), _ptr(x), _ptr(y))
+    return y
+
+
+def round_bf16(v):
+    return lib().wko_round_bf16(float(v))
+
+
+def default_threads():
+    return max(1, os.cpu_count() or 1)
+
+
+def layer_forward(cfg, weights, X, threads=None, diag=False, ln_eps=1e-5):
+    """One Wukong layer on host examples X [n_ex, n, d] (float64). ``weights`` is a
+    dict with Y, W0..W{m-1}, b0..b{m-1}, fmb_gamma, fmb_beta, W_L, out_gamma,
+    out_beta as host arrays (float32, or uint16 bf16 bits for Y / W_j / W_L)."""
+    X = _c64(X)
+    n_ex = X.shape[0]
+    dims = [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
+    m = len(dims) - 1
+    dims_c = (ctypes.c_int32 * len(dims))(*dims)
+    wdt = weights["Y"].dtype
+    dtype = 1 if wdt == np.uint16 else 0
+    keep = []
+
+    def arr(a, want):
+        a = np.ascontiguousarray(a)
+        if want == "w":
+            assert a.dtype == wdt
+        else:
+            a = np.ascontiguousarray(a, dtype=np.float32)
+        keep.append(a)
+        return a.ctypes.data
+
+    c = _Config(cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], cfg["n_l"], m, dims_c, ln_eps, dtype)
+    Wp = (ctypes.c_void_p * m)(*[arr(weights["W%d" % j], "w") for j in range(m)])
+    bp = (ctypes.c_void_p * m)(*[arr(weights["b%d" % j], "f") if weights.get("b%d" % j) is not None else None
+                                  for j in range(m)])
+    lay = _Layer(arr(weights["Y"], "w"), Wp, bp, arr(weights["fmb_gamma"], "f"), arr(weights["fmb_beta"], "f"),
+                 arr(weights["W_L"], "w"), arr(weights["out_gamma"], "f"), arr(weights["out_beta"], "f"))
+    out = np.empty_like(X)
+    rc = lib().wko_layer_forward(ctypes.byref(c), ctypes.byref(lay), n_ex, _ptr(X), _ptr(out),
+                                 threads or default_threads(), int(diag))
+    if rc:
+        raise ValueError("oracle rejected the configuration")
+    return out
+
+
+def stack_forward(cfg, layer_weights, X, threads=None, diag=False):
+    """The whole stack, one layer at a time. ``layer_weights(l)`` returns layer l's
+    host weights (so a large stack can be generated layer by layer)."""
+    h = _c64(X)
+    for layer in range(cfg["layers"]):
+        h = layer_forward(cfg, layer_weights(layer), h, threads=threads, diag=diag)
+    return h

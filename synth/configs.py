@@ -1,0 +1,168 @@
+"""The five synthetic workloads of the Wukong stack forward and their input recipes.
+
+Shapes follow the Wukong page (xdnf.cn repost of "Wukong: Towards a Scaling Law
+for Large-Scale Recommendation", section 2.3, the scaling knobs l, n_F, n_L, k
+and the FMB MLP) with sizes chosen to match its workloads: embedding dim 160
+and 720 features (section 3.2.1). Inputs are synthetic (no dataset):
+
+* X ~ N(0, 1); the wide/narrow workload scales the rows of feature i by
+  s_i ~ LogUniform(0.1, 10), one draw per feature shared by all examples.
+* Y, W_j, W_L ~ N(0, 1/fan_in) with fan_in = n for Y and W_L and h_j for W_j.
+* Biases are 0. LayerNorm gamma = 1, beta = 0, except the 2-layer bf16
+  workload, whose LayerNorm affine parameters (both gamma and beta of both
+  LayerNorms) are 1 + N(0, 0.02^2).
+* Seed 0 for every workload; each tensor has its own stream id (below).
+
+"MLP of m layers of width W" means m Linear layers h_0 = n*k -> W -> ... -> W ->
+h_m = n_F*d (m-1 hidden widths, ReLU after each hidden Linear, none after the
+last one).
+"""
+import math
+
+import numpy as np
+
+from . import BF16, F32, bf16_bits_to_f64, fill_normal_host, fill_x_logscaled_host
+
+SEED = 0
+
+# stream ids
+TID_X = 1
+TID_X_SCALE = 2
+
+
+def layer_tid(layer, what, j=0):
+    base = 1000 * (layer + 1)
+    return base + {"Y": 1, "W": 10 + j, "b": 40 + j, "fmb_gamma": 70, "fmb_beta": 71, "W_L": 80,
+                   "out_gamma": 90, "out_beta": 91}[what]
+
+
+CONFIGS = {
+    # name: (layers, batch, n, d, k, n_f, n_l, hidden widths, dtype, ln affine, x distribution)
+    "c1_fp32": dict(layers=1, batch=64, n=16, d=16, k=4, n_f=8, n_l=8, hidden=[64], dtype="f32",
+                    ln_affine="unit", x_dist="normal",
+                    about="1-layer fp32, B=64, n=16, d=16, k=4, MLP 64->64->128"),
+    "c2_bf16": dict(layers=2, batch=4096, n=64, d=128, k=16, n_f=32, n_l=32, hidden=[1024], dtype="bf16",
+                    ln_affine="1+N(0,0.02)", x_dist="normal",
+                    about="2-layer bf16, B=4096, n=64, d=128, k=16, MLP 1024->1024->4096"),
+    "c3_bf16": dict(layers=4, batch=16384, n=256, d=160, k=32, n_f=128, n_l=128, hidden=[4096, 4096],
+                    dtype="bf16", ln_affine="unit", x_dist="normal",
+                    about="4-layer bf16 (~1.14 GFLOP/example), B=16384, n=256, d=160, k=32"),
+    "c4_bf16": dict(layers=8, batch=4096, n=512, d=160, k=64, n_f=256, n_l=256, hidden=[16384, 16384],
+                    dtype="bf16", ln_affine="unit", x_dist="normal",
+                    about="8-layer bf16 (~24.1 GFLOP/example), B=4096, n=512, d=160, k=64"),
+    "c5_bf16": dict(layers=2, batch=32768, n=720, d=32, k=24, n_f=360, n_l=360, hidden=[2048], dtype="bf16",
+                    ln_affine="unit", x_dist="logscaled",
+                    about="2-layer wide-feature narrow-dim bf16, B=32768, n=720, d=32, k=24"),
+}
+
+
+def mlp_dims(cfg):
+    """[h_0, ..., h_m]: h_0 = n*k, the hidden widths, h_m = n_F*d."""
+    return [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
+
+
+def flops_per_example(cfg):
+    """Matmul FLOPs (2 per multiply-add) of one example through the stack:
+    L * (4 n d k + 2 n_L n d + 2 sum_j h_j h_{j+1})."""
+    n, d, k, n_l = cfg["n"], cfg["d"], cfg["k"], cfg["n_l"]
+    h = mlp_dims(cfg)
+    per_layer = 4 * n * d * k + 2 * n_l * n * d + 2 * sum(h[j] * h[j + 1] for j in range(len(h) - 1))
+    return cfg["layers"] * per_layer
+
+
+def storage_dtype(cfg):
+    return F32 if cfg["dtype"] == "f32" else BF16
+
+
+def tensor_specs(cfg, layer):
+    """Recipe of one layer's parameters: name -> (shape, kind, stream id, mean, std, dtype).
+    kind 'normal' draws mean + std * N(0,1); 'const' is the constant mean."""
+    n, d, k, n_f, n_l = cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], cfg["n_l"]
+    h = mlp_dims(cfg)
+    wd = "f32" if cfg["dtype"] == "f32" else "bf16"
+    specs = {
+        "Y": ((n, k), "normal", layer_tid(layer, "Y"), 0.0, 1.0 / math.sqrt(n), wd),
+        "W_L": ((n_l, n), "normal", layer_tid(layer, "W_L"), 0.0, 1.0 / math.sqrt(n), wd),
+    }
+    for j in range(len(h) - 1):
+        specs["W%d" % j] = ((h[j + 1], h[j]), "normal", layer_tid(layer, "W", j), 0.0, 1.0 / math.sqrt(h[j]), wd)
+        specs["b%d" % j] = ((h[j + 1],), "const", layer_tid(layer, "b", j), 0.0, 0.0, "f32")
+    if cfg["ln_affine"] == "unit":
+        specs["fmb_gamma"] = ((n * k,), "const", layer_tid(layer, "fmb_gamma"), 1.0, 0.0, "f32")
+        specs["fmb_beta"] = ((n * k,), "const", layer_tid(layer, "fmb_beta"), 0.0, 0.0, "f32")
+        specs["out_gamma"] = ((d,), "const", layer_tid(layer, "out_gamma"), 1.0, 0.0, "f32")
+        specs["out_beta"] = ((d,), "const", layer_tid(layer, "out_beta"), 0.0, 0.0, "f32")
+    else:  # 1 + N(0, 0.02^2) for every LayerNorm affine parameter
+        for nm, size in (("fmb_gamma", n * k), ("fmb_beta", n * k), ("out_gamma", d), ("out_beta", d)):
+            specs[nm] = ((size,), "normal", layer_tid(layer, nm), 1.0, 0.02, "f32")
+    return specs
+
+
+def make_layer_host(cfg, layer):
+    """One layer's parameters as host numpy arrays (bf16 as uint16 bit patterns)."""
+    out = {}
+    for name, (shape, kind, tid, mean, std, dt) in tensor_specs(cfg, layer).items():
+        if kind == "const":
+            out[name] = np.full(shape, mean, dtype=np.float32) if dt == "f32" else None
+            if out[name] is None:
+                raise ValueError("bf16 constants are not used")
+        else:
+            arr = np.empty(shape, dtype=np.float32 if dt == "f32" else np.uint16)
+            out[name] = fill_normal_host(arr, SEED, tid, mean, std)
+    return out
+
+
+def make_x_host(cfg, examples):
+    """Rows X[b] for the listed example indices, as a host array [len(examples), n, d]
+    (float32, or uint16 bf16 bits)."""
+    n, d = cfg["n"], cfg["d"]
+    per = n * d
+    dt = np.float32 if cfg["dtype"] == "f32" else np.uint16
+    out = np.empty((len(examples), n, d), dtype=dt)
+    for r, b in enumerate(examples):
+        row = out[r].reshape(-1)
+        if cfg["x_dist"] == "logscaled":
+            fill_x_logscaled_host(row, SEED, TID_X, TID_X_SCALE, n, d, offset=int(b) * per)
+        else:
+            fill_normal_host(row, SEED, TID_X, 0.0, 1.0, offset=int(b) * per)
+    return out
+
+
+def to_f64(arr):
+    """Exact float64 view of a host tensor (float32 or bf16 bits)."""
+    if arr.dtype == np.uint16:
+        return bf16_bits_to_f64(arr).reshape(arr.shape)
+    return arr.astype(np.float64)
+
+
+def make_layer_dev(cfg, layer, device="cuda"):
+    """One layer's parameters as device tensors, filled by the device generator
+    (bit-identical to make_layer_host)."""
+    import torch
+
+    from . import fill_normal_dev
+    out = {}
+    for name, (shape, kind, tid, mean, std, dt) in tensor_specs(cfg, layer).items():
+        tdt = torch.float32 if dt == "f32" else torch.bfloat16
+        if kind == "const":
+            out[name] = torch.full(shape, mean, dtype=tdt, device=device)
+        else:
+            t = torch.empty(shape, dtype=tdt, device=device)
+            out[name] = fill_normal_dev(t, SEED, tid, mean, std)
+    return out
+
+
+def make_x_dev(cfg, batch, device="cuda", first_example=0):
+    """X[first_example : first_example+batch] as a device tensor [batch, n, d]."""
+    import torch
+
+    from . import fill_normal_dev, fill_x_logscaled_dev
+    n, d = cfg["n"], cfg["d"]
+    tdt = torch.float32 if cfg["dtype"] == "f32" else torch.bfloat16
+    t = torch.empty((batch, n, d), dtype=tdt, device=device)
+    off = first_example * n * d
+    if cfg["x_dist"] == "logscaled":
+        fill_x_logscaled_dev(t, SEED, TID_X, TID_X_SCALE, n, d, offset=off)
+    else:
+        fill_normal_dev(t, SEED, TID_X, 0.0, 1.0, offset=off)
+    return t
