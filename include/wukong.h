@@ -1,0 +1,193 @@
+/*
+ * wukong.h -- C ABI of the B200 (sm_100a) Wukong interaction-stack forward.
+ *
+ * The method is the Wukong layer of "Wukong: Towards a Scaling Law for
+ * Large-Scale Recommendation" as summarised on the xdnf.cn repost of the Zhihu
+ * article (section 2.2 "Wukong", section 2.3 "Scale"), and the Wukong module of
+ * WHALE (gist.science summary of arXiv 2607.17017, section 2.1, item 1). Per
+ * example, layer i maps the embedding matrix X_i (n x d) to
+ *
+ *     X_{i+1} = LN_rows( concat_rows( FMB(X_i), LCB(X_i) ) + X_i )
+ *     FMB(X)  = reshape_{n_F x d}( MLP( LN( flatten( X (X^T Y) ) ) ) )
+ *     LCB(X)  = W_L X
+ *
+ * with Y (n x k) the learnable projection that compresses the features to k
+ * before the crossing (section 2.2, FMB paragraph), W_L (n_L x n) the linear
+ * compression (section 2.2, LCB paragraph) and n_F + n_L = n so that the
+ * residual needs no projection. The page's formulas were lost in extraction;
+ * the equations above are the reading the surviving sentences support.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named *_host are host memory; every other data pointer is device
+ *     memory on the current CUDA device. All device pointers must be 16-byte
+ *     aligned. Tensors are dense and row-major (last index fastest).
+ *   - dtype WK_BF16: X, out, Y, W_j, W_L are bf16; biases and LayerNorm
+ *     parameters are fp32; all products accumulate in fp32, LayerNorm
+ *     statistics are fp32. dtype WK_F32: everything is fp32.
+ *   - Calls that take a stream are asynchronous and stream-ordered: they only
+ *     validate their arguments on the host and enqueue kernels. They never
+ *     synchronise and never copy between host and device, except
+ *     wk_stack_forward_host, which is synchronous by design.
+ *   - Every call returns a wk_status and never aborts the process. A kernel
+ *     that detects a problem on the device (a pipeline wait that ran past its
+ *     limit) records it in a device status word and returns early; read it with
+ *     wk_stack_sync_status or wk_device_status.
+ *   - The stream argument is a cudaStream_t (NULL = legacy default stream).
+ */
+#ifndef WUKONG_H
+#define WUKONG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WK_API __attribute__((visibility("default")))
+#else
+#define WK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* wk_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  WK_OK = 0,
+  WK_ERR_INVALID_ARG = 1,  /* NULL / misaligned pointer, batch out of range, overlapping X and out */
+  WK_ERR_UNSUPPORTED = 2,  /* a shape or dtype this build does not implement (e.g. n_F + n_L != n) */
+  WK_ERR_OOM = 3,          /* workspace allocation failed */
+  WK_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch error, no device, ...) */
+  WK_ERR_TIMEOUT = 5,      /* a kernel gave up on a pipeline wait; its output is not valid */
+  WK_ERR_DEVICE = 6        /* the device status word holds another error flag */
+} wk_status;
+
+typedef enum { WK_F32 = 0, WK_BF16 = 1 } wk_dtype;
+
+/* Shape of the stack; every layer has the same shape (n is the same for every
+ * layer because n_F + n_L = n). Scaling knobs of section 2.3: num_layers = l,
+ * n_f = n_F, n_l = n_L, k, and the FMB MLP (mlp_num_linear Linear layers,
+ * h_0 = n*k -> mlp_hidden[0] -> ... -> h_m = n_f*d, ReLU after every Linear but
+ * the last). */
+typedef struct {
+  int32_t num_layers;          /* l >= 1 */
+  int32_t n, d, k, n_f, n_l;   /* n_f + n_l == n; d % 8 == 0 (bf16) or d % 4 == 0 (fp32) */
+  int32_t mlp_num_linear;      /* m >= 1 */
+  const int32_t* mlp_hidden;   /* m-1 widths (may be NULL when m == 1); copied at create */
+  wk_dtype dtype;
+  float ln_eps;                /* LayerNorm epsilon; 0 selects 1e-5 */
+  int64_t max_batch;           /* largest batch a forward will be given; sizes the workspace */
+} wk_stack_config;
+
+/* One layer's parameters. All DEVICE pointers, BORROWED: the caller keeps them
+ * alive and unchanged until wk_stack_destroy. Layouts:
+ *   Y            [n, k]               dtype
+ *   W[j]         [h_{j+1}, h_j]       dtype  (row-major, the torch Linear layout)
+ *   b[j]         [h_{j+1}]            fp32   (b or b[j] may be NULL: zero bias)
+ *   fmb_ln_gamma, fmb_ln_beta [n*k]   fp32   (LayerNorm of the flattened FM output)
+ *   W_L          [n_l, n]             dtype
+ *   out_ln_gamma, out_ln_beta [d]     fp32   (LayerNorm of each output embedding row) */
+typedef struct {
+  const void* Y;
+  const void* const* W;
+  const float* const* b;
+  const float* fmb_ln_gamma;
+  const float* fmb_ln_beta;
+  const void* W_L;
+  const float* out_ln_gamma;
+  const float* out_ln_beta;
+} wk_layer_weights;
+
+typedef struct wk_stack wk_stack;
+
+/* Validates cfg, records the weight pointers of cfg->num_layers layers
+ * (weights[0 .. num_layers-1]), builds the TMA descriptors of the weights and
+ * allocates the workspace for cfg->max_batch examples on the current device:
+ * A0 [max_batch, n*k], two MLP activation buffers [max_batch, max hidden], the
+ * concat buffer [max_batch, n, d] and two layer buffers [max_batch, n, d].
+ * The handle owns the workspace; *out is set only on WK_OK.
+ * Errors: WK_ERR_INVALID_ARG (NULL, misaligned, max_batch < 1),
+ * WK_ERR_UNSUPPORTED (n_f + n_l != n, unsupported d / dtype / widths),
+ * WK_ERR_OOM, WK_ERR_CUDA. */
+WK_API wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* weights, wk_stack** out);
+
+/* out[b] = stack(X[b]) for b < batch. X and out are [batch, n, d] device
+ * tensors of cfg->dtype; they must not overlap. batch == 0 is a no-op (WK_OK).
+ * Asynchronous on `stream`. One handle is not re-entrant: two forwards on one
+ * handle must be ordered (same stream, or synchronised), because they share the
+ * workspace. Errors: WK_ERR_INVALID_ARG (NULL handle or pointer, misaligned,
+ * batch < 0 or > max_batch, X/out overlap), WK_ERR_CUDA (launch failure). */
+WK_API wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t batch, wk_stream_t stream);
+
+/* Same result as wk_stack_forward with HOST input and output buffers
+ * ([batch, n, d], cfg->dtype). Splits the batch into chunks and overlaps the
+ * host-to-device copy of chunk c+1 and the device-to-host copy of chunk c-1
+ * with the forward of chunk c on internal streams ordered after `stream`.
+ * Returns when out_host holds the result. Page-locked (pinned) host buffers give
+ * the full copy bandwidth; pageable ones work but copy slower. Chunks use the
+ * handle's workspace and two staging buffers allocated on first use. */
+WK_API wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host, int64_t batch, wk_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the device status word.
+ * WK_OK, WK_ERR_TIMEOUT, WK_ERR_DEVICE or WK_ERR_CUDA. */
+WK_API wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream);
+
+/* Frees the workspace and the handle (synchronises the device first). NULL is a no-op. */
+WK_API void wk_stack_destroy(wk_stack* h);
+
+/* Static string for a status code. */
+WK_API const char* wk_status_string(wk_status s);
+
+/* ---- per-kernel timing of a handle's forwards (CUDA events on the launch stream) ---- */
+
+typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
+               WK_KERNEL_COUNT = 4 } wk_kernel_kind;
+
+/* enable != 0: every later forward records a start/stop event pair around each
+ * kernel launch on its stream (adds no synchronisation). */
+WK_API wk_status wk_stack_set_profiling(wk_stack* h, int enable);
+
+/* Waits for the recorded events, then reports, per kernel kind, the summed
+ * device time in ms and the number of launches since the last call, and clears
+ * the record. total_ms and launches are arrays of WK_KERNEL_COUNT entries. */
+WK_API wk_status wk_stack_kernel_times(wk_stack* h, double* total_ms, int64_t* launches);
+
+/* ---- the steps of one layer as stand-alone calls (no handle, no workspace) ---- */
+
+/* FMB front: A0[b] = LN( flatten( X_b (X_b^T Y) ) ) * gamma + beta, b < batch.
+ * X [batch, n, d], Y [n, k] (dtype), gamma/beta [n*k] fp32, A0 [batch, n*k] dtype.
+ * The FM runs per example on the tensor cores (bf16) with fp32 accumulation;
+ * X_b^T Y is rounded to bf16 before the second product (bf16 path only). */
+WK_API wk_status wk_fm_ln(const void* X, const void* Y, const float* gamma, const float* beta, void* A0, int64_t batch,
+                   int32_t n, int32_t d, int32_t k, wk_dtype dtype, float eps, wk_stream_t stream);
+
+/* One Linear of the FMB MLP over the batch: C[r, c] = act( sum_q A[r, q] W[c, q] + bias[c] ),
+ * r < M, c < N; act = ReLU if relu != 0. A [M, K] (row stride K), W [N, K],
+ * bias [N] fp32 or NULL, C [M, N] with row stride ldc elements (ldc >= N; the
+ * last Linear writes straight into the concat buffer with ldc = n*d).
+ * K % 8 == 0, N % 8 == 0, ldc % 8 == 0 (bf16). */
+WK_API wk_status wk_mlp_linear(const void* A, const void* W, const float* bias, void* C, int64_t M, int32_t K, int32_t N,
+                        int64_t ldc, int relu, wk_dtype dtype, wk_stream_t stream);
+
+/* LCB: concat[b, n_f + r, :] = sum_i W_L[r, i] X[b, i, :] for r < n_l, b < batch.
+ * W_L [n_l, n], X [batch, n, d], concat [batch, n_f + n_l, d] (dtype); rows
+ * 0..n_f-1 of concat are not touched. */
+WK_API wk_status wk_lcb(const void* W_L, const void* X, void* concat, int64_t batch, int32_t n, int32_t d, int32_t n_f,
+                 int32_t n_l, wk_dtype dtype, wk_stream_t stream);
+
+/* Concat + residual + LayerNorm: out[r, :] = LN( concat[r, :] + X[r, :] ) * gamma + beta
+ * over each of `rows` embedding rows of d values. concat, X, out [rows, d] (dtype),
+ * gamma/beta [d] fp32. out may alias concat. */
+WK_API wk_status wk_res_ln(const void* concat, const void* X, const float* gamma, const float* beta, void* out, int64_t rows,
+                    int32_t d, wk_dtype dtype, float eps, wk_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the device status word of the
+ * stand-alone calls above (handles have their own). */
+WK_API wk_status wk_device_status(wk_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WUKONG_H */

@@ -112,7 +112,7 @@ def default_threads():
     return max(1, os.cpu_count() or 1)
 
 
-def layer_forward(cfg, weights, X, threads=None, diag=False, ln_eps=1e-5):
+def layer_forward(cfg, weights, X, threads=None, diag=0, ln_eps=1e-5):
     """One Wukong layer on host examples X [n_ex, n, d] (float64). ``weights`` is a
     dict with Y, W0..W{m-1}, b0..b{m-1}, fmb_gamma, fmb_beta, W_L, out_gamma,
     out_beta as host arrays (float32, or uint16 bf16 bits for Y / W_j / W_L)."""
@@ -140,6 +140,7 @@ def layer_forward(cfg, weights, X, threads=None, diag=False, ln_eps=1e-5):
                                   for j in range(m)])
     lay = _Layer(arr(weights["Y"], "w"), Wp, bp, arr(weights["fmb_gamma"], "f"), arr(weights["fmb_beta"], "f"),
                  arr(weights["W_L"], "w"), arr(weights["out_gamma"], "f"), arr(weights["out_beta"], "f"))
+    diag = 15 if diag is True else int(diag)
     out = np.empty_like(X)
     rc = lib().wko_layer_forward(ctypes.byref(c), ctypes.byref(lay), n_ex, _ptr(X), _ptr(out),
                                  threads or default_threads(), int(diag))
@@ -148,7 +149,7 @@ def layer_forward(cfg, weights, X, threads=None, diag=False, ln_eps=1e-5):
     return out
 
 
-def stack_forward(cfg, layer_weights, X, threads=None, diag=False):
+def stack_forward(cfg, layer_weights, X, threads=None, diag=0):
     """The whole stack, one layer at a time. ``layer_weights(l)`` returns layer l's
     host weights (so a large stack can be generated layer by layer)."""
     h = _c64(X)

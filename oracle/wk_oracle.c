@@ -91,6 +91,9 @@ static double round_bf16_via_f32(double v) {
   return (double)f;
 }
 
+/* diagnostic rounding points (bit mask of the diag argument) */
+enum { DIAG_A0 = 1, DIAG_HIDDEN = 2, DIAG_CONCAT = 4, DIAG_XOUT = 8, DIAG_XOPS = 16 };
+
 static void maybe_round(double* v, int64_t len, int diag) {
   if (!diag) return;
   for (int64_t i = 0; i < len; ++i) v[i] = round_bf16_via_f32(v[i]);
@@ -205,15 +208,19 @@ static void fmb_front(void* c, int64_t e0, int64_t e1) {
   int32_t n = cfg->n, d = cfg->d, k = cfg->k;
   double* P = (double*)malloc(sizeof(double) * (size_t)n * n);
   double* F = (double*)malloc(sizeof(double) * (size_t)n * k);
+  double* Xr = (double*)malloc(sizeof(double) * (size_t)n * d);
   for (int64_t e = e0; e < e1; ++e) {
-    wko_fm(n, d, k, L->X_in + e * (int64_t)n * d, L->Yd, P, F);
+    memcpy(Xr, L->X_in + e * (int64_t)n * d, sizeof(double) * (size_t)n * d);
+    maybe_round(Xr, (int64_t)n * d, L->diag & DIAG_XOPS);
+    wko_fm(n, d, k, Xr, L->Yd, P, F);
     /* flatten row-major (feature i major, compressed index c minor), LayerNorm over n*k */
     double* a0 = L->h[0] + e * (int64_t)n * k;
     wko_layernorm((int64_t)n * k, F, L->g1, L->b1, cfg->ln_eps, a0);
-    maybe_round(a0, (int64_t)n * k, L->diag);
+    maybe_round(a0, (int64_t)n * k, L->diag & DIAG_A0);
   }
   free(P);
   free(F);
+  free(Xr);
 }
 
 static void mlp_rows(void* c, int64_t r0, int64_t r1) {
@@ -247,25 +254,29 @@ static void layer_back(void* c, int64_t e0, int64_t e1) {
   int m = cfg->mlp_num_linear;
   double* G = (double*)malloc(sizeof(double) * (size_t)n_l * d);
   double* cat = (double*)malloc(sizeof(double) * (size_t)n * d);
+  double* Xr = (double*)malloc(sizeof(double) * (size_t)n * d);
   for (int64_t e = e0; e < e1; ++e) {
     const double* X = L->X_in + e * (int64_t)n * d;
-    wko_lcb(n, d, n_l, L->WLd, X, G);
+    memcpy(Xr, X, sizeof(double) * (size_t)n * d);
+    maybe_round(Xr, (int64_t)n * d, L->diag & DIAG_XOPS);
+    wko_lcb(n, d, n_l, L->WLd, Xr, G);
     /* concat rows: FMB rows 0..n_f-1 (the last MLP output, reshaped row-major to n_f x d),
        then LCB rows n_f..n-1 */
     const double* fmb = L->h[m] + e * (int64_t)n_f * d;
     memcpy(cat, fmb, sizeof(double) * (size_t)n_f * d);
     memcpy(cat + (int64_t)n_f * d, G, sizeof(double) * (size_t)n_l * d);
-    maybe_round(cat, (int64_t)n * d, L->diag);
+    maybe_round(cat, (int64_t)n * d, L->diag & DIAG_CONCAT);
     double* Xo = L->X_out + e * (int64_t)n * d;
     for (int32_t r = 0; r < n; ++r) {
       double* y = cat + (int64_t)r * d;
       for (int32_t t = 0; t < d; ++t) y[t] += X[(int64_t)r * d + t]; /* residual */
       wko_layernorm(d, y, L->g2, L->b2, cfg->ln_eps, Xo + (int64_t)r * d);
     }
-    maybe_round(Xo, (int64_t)n * d, L->diag);
+    maybe_round(Xo, (int64_t)n * d, L->diag & DIAG_XOUT);
   }
   free(G);
   free(cat);
+  free(Xr);
 }
 
 static double* upcast(int32_t dtype, const void* p, int64_t len) {
@@ -280,9 +291,12 @@ static double* upcast_f32(const float* p, int64_t len) {
 }
 
 /* One Wukong layer on n_ex examples: X_out = LN_rows(concat(FMB(X_in), LCB(X_in)) + X_in).
- * diag = 1 additionally rounds to bf16 where a bf16 GPU implementation stores an
- * intermediate (the FMB LayerNorm output, each MLP activation, the concatenated
- * blocks and the layer output); diag = 0 is the exact fp64 reference.
+ * diag != 0 additionally rounds to bf16 where a GPU implementation may store an
+ * intermediate, selected by bits: 1 the FMB LayerNorm output, 2 each MLP
+ * activation, 4 the concatenated blocks, 8 the layer output, 16 the copy of the
+ * layer input that the FM and the LCB multiply (the residual keeps the unrounded
+ * input). diag = 0 is the
+ * exact fp64 reference (the one parity is graded against).
  * Returns 0, or 1 on an invalid configuration. */
 int wko_layer_forward(const wko_config* cfg, const wko_layer* w, int64_t n_ex, const double* X_in, double* X_out,
                       int threads, int diag) {
@@ -311,7 +325,7 @@ int wko_layer_forward(const wko_config* cfg, const wko_layer* w, int64_t n_ex, c
   for (int j = 0; j < m; ++j) {
     L.j = j;
     parallel_for(cfg->mlp_dims[j + 1], threads, mlp_rows, &L);
-    maybe_round(L.h[j + 1], n_ex * (int64_t)cfg->mlp_dims[j + 1], diag);
+    maybe_round(L.h[j + 1], n_ex * (int64_t)cfg->mlp_dims[j + 1], diag & DIAG_HIDDEN);
   }
   parallel_for(n_ex, threads, layer_back, &L);
 

@@ -1,0 +1,220 @@
+"""Python binding of the Wukong interaction-stack C ABI (include/wukong.h).
+
+Argument marshalling only: every function here forwards to the entry point of the
+same name in ``_lib/libwukong.so`` and raises :class:`WkError` on a non-OK
+status. Every step of the forward runs in that library's CUDA kernels; there is
+no Python or CPU implementation behind these names, and every one of them
+raises ImportError when the library is missing (build it with
+``recsys_feature_interaction_b200.build.build()``).
+
+Tensors are passed as torch tensors (device tensors for the device entry points,
+host tensors or numpy arrays for ``wk_stack_forward_host``) or as raw integer
+addresses. Streams are torch.cuda.Stream objects, raw cudaStream_t integers, or
+None (the current torch stream of the tensor's device).
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
+
+WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
+WK_F32, WK_BF16 = 0, 1
+WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_COUNT = range(5)
+KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln")
+
+
+class WkError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, wk_status_string(status), status))
+
+
+class WkStackConfig(ctypes.Structure):
+    _fields_ = [("num_layers", ctypes.c_int32), ("n", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("n_f", ctypes.c_int32), ("n_l", ctypes.c_int32),
+                ("mlp_num_linear", ctypes.c_int32), ("mlp_hidden", ctypes.POINTER(ctypes.c_int32)),
+                ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("max_batch", ctypes.c_int64)]
+
+
+class WkLayerWeights(ctypes.Structure):
+    _fields_ = [("Y", ctypes.c_void_p), ("W", ctypes.POINTER(ctypes.c_void_p)),
+                ("b", ctypes.POINTER(ctypes.c_void_p)), ("fmb_ln_gamma", ctypes.c_void_p),
+                ("fmb_ln_beta", ctypes.c_void_p), ("W_L", ctypes.c_void_p), ("out_ln_gamma", ctypes.c_void_p),
+                ("out_ln_beta", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libwukong.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libwukong.so is missing at %s; build it with "
+                              "recsys_feature_interaction_b200.build.build()" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, ci, cf = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        sig = {
+            "wk_stack_create": [ctypes.POINTER(WkStackConfig), ctypes.POINTER(WkLayerWeights), ctypes.POINTER(vp)],
+            "wk_stack_forward": [vp, vp, vp, i64, vp],
+            "wk_stack_forward_host": [vp, vp, vp, i64, vp],
+            "wk_stack_sync_status": [vp, vp],
+            "wk_stack_set_profiling": [vp, ci],
+            "wk_stack_kernel_times": [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)],
+            "wk_fm_ln": [vp, vp, vp, vp, vp, i64, i32, i32, i32, ci, cf, vp],
+            "wk_mlp_linear": [vp, vp, vp, vp, i64, i32, i32, i64, ci, ci, vp],
+            "wk_lcb": [vp, vp, vp, i64, i32, i32, i32, i32, ci, vp],
+            "wk_res_ln": [vp, vp, vp, vp, vp, i64, i32, ci, cf, vp],
+            "wk_device_status": [vp],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ci
+        L.wk_stack_destroy.argtypes = [vp]
+        L.wk_stack_destroy.restype = None
+        L.wk_status_string.argtypes = [ci]
+        L.wk_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _addr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    if hasattr(t, "ctypes"):  # numpy
+        return t.ctypes.data
+    raise TypeError("expected a tensor, an array or an address, got %r" % type(t))
+
+
+def _stream(stream, like=None):
+    if stream is None:
+        import torch
+        dev = like.device if (like is not None and hasattr(like, "device") and like.device.type == "cuda") else None
+        return torch.cuda.current_stream(dev).cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status, where):
+    if status != WK_OK:
+        raise WkError(status, where)
+
+
+def wk_status_string(status):
+    return lib().wk_status_string(int(status)).decode()
+
+
+def _dtype_code(dtype):
+    if dtype in (WK_F32, WK_BF16):
+        return dtype
+    s = str(dtype)
+    if "bfloat16" in s or s == "bf16":
+        return WK_BF16
+    if "float32" in s or s in ("f32", "fp32"):
+        return WK_F32
+    raise ValueError("unsupported dtype %r" % (dtype,))
+
+
+class StackHandle:
+    """An opaque wk_stack* plus the Python objects whose memory it borrows."""
+
+    def __init__(self, ptr, cfg, keep):
+        self.ptr = ptr
+        self.cfg = cfg
+        self._keep = keep
+
+    def __del__(self):
+        try:
+            if self.ptr:
+                wk_stack_destroy(self)
+        except Exception:
+            pass
+
+
+def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0):
+    """cfg: mapping with num_layers (or layers), n, d, k, n_f, n_l, hidden (the m-1
+    hidden widths) and dtype; layers: one mapping per layer with Y, W0..W{m-1},
+    b0..b{m-1} (or None), fmb_gamma, fmb_beta, W_L, out_gamma, out_beta."""
+    hidden = list(cfg.get("hidden", []))
+    m = len(hidden) + 1
+    hid = (ctypes.c_int32 * max(1, len(hidden)))(*hidden) if hidden else None
+    c = WkStackConfig(int(cfg.get("num_layers", cfg.get("layers"))), cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
+                      cfg["n_l"], m, hid, _dtype_code(dtype if dtype is not None else cfg["dtype"]),
+                      float(ln_eps), int(max_batch if max_batch is not None else cfg["batch"]))
+    keep = [hid, list(layers)]
+    arr = (WkLayerWeights * len(layers))()
+    for i, w in enumerate(layers):
+        Wp = (ctypes.c_void_p * m)(*[_addr(w["W%d" % j]) for j in range(m)])
+        bp = (ctypes.c_void_p * m)(*[_addr(w.get("b%d" % j)) for j in range(m)])
+        keep += [Wp, bp]
+        arr[i] = WkLayerWeights(_addr(w["Y"]), Wp, bp, _addr(w["fmb_gamma"]), _addr(w["fmb_beta"]), _addr(w["W_L"]),
+                                _addr(w["out_gamma"]), _addr(w["out_beta"]))
+    keep.append(arr)
+    h = ctypes.c_void_p()
+    _check(lib().wk_stack_create(ctypes.byref(c), arr, ctypes.byref(h)), "wk_stack_create")
+    return StackHandle(h.value, dict(cfg), keep)
+
+
+def wk_stack_forward(h, X, out, batch=None, stream=None):
+    b = X.shape[0] if batch is None else batch
+    _check(lib().wk_stack_forward(h.ptr, _addr(X), _addr(out), int(b), _stream(stream, X)), "wk_stack_forward")
+
+
+def wk_stack_forward_host(h, X_host, out_host, batch=None, stream=None):
+    b = X_host.shape[0] if batch is None else batch
+    _check(lib().wk_stack_forward_host(h.ptr, _addr(X_host), _addr(out_host), int(b), _stream(stream)),
+           "wk_stack_forward_host")
+
+
+def wk_stack_sync_status(h, stream=None):
+    return lib().wk_stack_sync_status(h.ptr, _stream(stream))
+
+
+def wk_stack_destroy(h):
+    if h.ptr:
+        lib().wk_stack_destroy(h.ptr)
+        h.ptr = None
+
+
+def wk_stack_set_profiling(h, enable=True):
+    _check(lib().wk_stack_set_profiling(h.ptr, 1 if enable else 0), "wk_stack_set_profiling")
+
+
+def wk_stack_kernel_times(h):
+    """{kernel name: (total_ms, launches)} since the previous call (waits for the events)."""
+    ms = (ctypes.c_double * WK_KERNEL_COUNT)()
+    n = (ctypes.c_int64 * WK_KERNEL_COUNT)()
+    _check(lib().wk_stack_kernel_times(h.ptr, ms, n), "wk_stack_kernel_times")
+    return {KERNEL_NAMES[i]: (ms[i], n[i]) for i in range(WK_KERNEL_COUNT)}
+
+
+def wk_fm_ln(X, Y, gamma, beta, A0, batch, n, d, k, dtype, eps=0.0, stream=None):
+    _check(lib().wk_fm_ln(_addr(X), _addr(Y), _addr(gamma), _addr(beta), _addr(A0), int(batch), n, d, k,
+                          _dtype_code(dtype), float(eps), _stream(stream, X)), "wk_fm_ln")
+
+
+def wk_mlp_linear(A, W, bias, C, M, K, N, ldc, relu, dtype, stream=None):
+    _check(lib().wk_mlp_linear(_addr(A), _addr(W), _addr(bias), _addr(C), int(M), K, N, int(ldc), int(bool(relu)),
+                               _dtype_code(dtype), _stream(stream, A)), "wk_mlp_linear")
+
+
+def wk_lcb(W_L, X, concat, batch, n, d, n_f, n_l, dtype, stream=None):
+    _check(lib().wk_lcb(_addr(W_L), _addr(X), _addr(concat), int(batch), n, d, n_f, n_l, _dtype_code(dtype),
+                        _stream(stream, X)), "wk_lcb")
+
+
+def wk_res_ln(concat, X, gamma, beta, out, rows, d, dtype, eps=0.0, stream=None):
+    _check(lib().wk_res_ln(_addr(concat), _addr(X), _addr(gamma), _addr(beta), _addr(out), int(rows), d,
+                           _dtype_code(dtype), float(eps), _stream(stream, X)), "wk_res_ln")
+
+
+def wk_device_status(stream=None):
+    return lib().wk_device_status(_stream(stream))

@@ -1,0 +1,322 @@
+// fm_mma.cuh -- the FMB front of a Wukong layer for bf16 inputs:
+//
+//   A0[b] = LN( flatten_rowmajor( X_b (X_b^T Y) ) ) * gamma + beta
+//
+// i.e. the optimised FM of the Wukong page (section 2.2, FMB paragraph: first
+// compress the features to k with Y, then cross), flattened (feature i major,
+// compressed index c minor) and normalised over all n*k values.
+//
+// One persistent CTA per SM walks the examples. A producer warp streams each
+// example's X rows (and the matching Y rows) from global memory into a ring of
+// shared-memory slots with bulk async copies (one copy per row, into rows padded
+// to an odd number of 16-byte units so ldmatrix is conflict-free), signalling an
+// mbarrier per slot. Eight consumer warps run two passes over the ring:
+//   pass A: Z = X^T Y   (d x k, reduction over the n features) with mma.sync
+//           m16n8k16 (bf16 in, fp32 accumulate), partial sums of up to AKS warps
+//           per output tile added in a fixed order, Z rounded to bf16 in smem;
+//   pass B: F = X Z     (n x k, reduction over d), F kept in registers;
+// then the LayerNorm statistics (two passes, fp32) and the bf16 store of A0. The
+// producer prefetches the next example while the current one finishes.
+#pragma once
+
+#include "common.cuh"
+
+namespace wk {
+
+constexpr int odd16(int bytes) {  // smallest odd multiple of 16 that is >= bytes
+  int u = (bytes + 15) / 16;
+  if ((u & 1) == 0) ++u;
+  return u * 16;
+}
+
+template <int N_, int D_, int KC_, int R_, int AWM_, int AWN_, int AKS_, int BWM_, int BWN_, int STAGES_>
+struct FmCfg {
+  static constexpr int N = N_, D = D_, KC = KC_, R = R_;
+  static constexpr int AWM = AWM_, AWN = AWN_, AKS = AKS_, BWM = BWM_, BWN = BWN_, STAGES = STAGES_;
+  static constexpr int SX = odd16(D * 2);     // bytes per staged X row
+  static constexpr int SY = odd16(KC * 2);    // bytes per staged Y row and per Z row
+  static constexpr int SLOT = R * SX + R * SY;
+  static constexpr int NCH = (N + R - 1) / R;
+  static constexpr int AMT = (D / 16) / AWM;  // pass A m16 tiles per warp (over d)
+  static constexpr int ANT = (KC / 8) / AWN;  // pass A n8 tiles per warp (over k)
+  static constexpr int BMT = (R / 16) / BWM;  // pass B m16 tiles per warp per chunk (over n)
+  static constexpr int BNT = (KC / 8) / BWN;  // pass B n8 tiles per warp (over k)
+  static constexpr int KS_D = D / 16;         // pass B k16 steps
+  static constexpr int ZPART_BYTES = AKS * D * KC * 4;
+  static constexpr int ZB_BYTES = D * SY;
+  static constexpr int SMEM = 128 + STAGES * SLOT + ZPART_BYTES + ZB_BYTES + 64 + 16 * STAGES + 16;
+  static_assert(D % 16 == 0 && KC % 8 == 0 && N % 16 == 0 && R % 16 == 0, "tile shape");
+  static_assert(AWM * AWN * AKS == 8 && BWM * BWN == 8, "8 consumer warps");
+  static_assert((D / 16) % AWM == 0 && (KC / 8) % AWN == 0 && (R / 16) % BWM == 0 && (KC / 8) % BWN == 0,
+                "warp split");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+constexpr int FM_THREADS = 288;  // 8 consumer warps + 1 producer warp
+
+template <class C>
+__global__ void __maxnreg__(224)
+    fm_ln_mma_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ Y,
+                     const float* __restrict__ gamma, const float* __restrict__ beta,
+                     __nv_bfloat16* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+  uint8_t* ring = smem;
+  float* zpart = reinterpret_cast<float*>(ring + C::STAGES * C::SLOT);
+  uint8_t* zb = reinterpret_cast<uint8_t*>(zpart) + C::ZPART_BYTES;
+  float* red = reinterpret_cast<float*>(zb + C::ZB_BYTES);  // [2][8]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 16);
+  uint64_t* empty = full + C::STAGES;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 8);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x) {
+      const __nv_bfloat16* xb = X + b * C::N * C::D;
+      for (int pass = 0; ok && pass < 2; ++pass) {
+        for (int c = 0; c < C::NCH; ++c) {
+          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          int waited = 1;
+          if (lane == 0) waited = mbar_wait(&empty[s], ph ^ 1u, status) ? 1 : 0;
+          waited = __shfl_sync(0xffffffffu, waited, 0);
+          if (!waited) {
+            ok = false;
+            break;
+          }
+          uint8_t* slot = ring + s * C::SLOT;
+          if (lane == 0)
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(rows * C::D * 2 + (pass == 0 ? rows * C::KC * 2 : 0)));
+          __syncwarp();
+          for (int r = lane; r < rows; r += 32) {
+            bulk_load(slot + r * C::SX, xb + static_cast<int64_t>(c * C::R + r) * C::D, C::D * 2, &full[s]);
+            if (pass == 0)
+              bulk_load(slot + C::R * C::SX + r * C::SY, Y + static_cast<int64_t>(c * C::R + r) * C::KC, C::KC * 2,
+                        &full[s]);
+          }
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) {  // let every armed slot land before the CTA exits
+      for (int i = 0; i < C::STAGES; ++i) mbar_wait(&full[i], ph ^ (i < s ? 0u : 1u), nullptr);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int tid = threadIdx.x;  // 0..255
+  const int g = lane >> 2, t4 = lane & 3;
+  // pass A warp coordinates
+  const int a_ks = warp % C::AKS;
+  const int a_wn = (warp / C::AKS) % C::AWN;
+  const int a_wm = warp / (C::AKS * C::AWN);
+  // pass B warp coordinates
+  const int b_wn = warp % C::BWN;
+  const int b_wm = warp / C::BWN;
+  // ldmatrix lane roles
+  const int lrow = lane & 7;           // row within an 8x8 matrix
+  const int lmat = lane >> 3;          // which of the 4 matrices this lane addresses
+
+  // After a failed wait (status flagged) a consumer stops waiting but keeps
+  // walking the same control flow, so every named barrier is still reached by all
+  // 256 consumer threads; the output of that launch is then not valid.
+  bool ok = true;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
+    // ------------------------------------------------ pass A: Z = X^T Y
+    float zacc[C::AMT][C::ANT][4];
+#pragma unroll
+    for (int i = 0; i < C::AMT; ++i)
+#pragma unroll
+      for (int j = 0; j < C::ANT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) zacc[i][j][e] = 0.f;
+    for (int c = 0; c < C::NCH; ++c) {
+      if (ok) ok = mbar_wait(&full[s], ph, status);
+      const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+      const uint32_t sx = smem_u32(ring + s * C::SLOT);
+      const uint32_t sy = sx + C::R * C::SX;
+      for (int ks = a_ks; ks < rows / 16; ks += C::AKS) {
+        uint32_t bf[C::ANT][2];
+#pragma unroll
+        for (int nt = 0; nt < C::ANT; ++nt) {
+          // B = Y (k = feature rows, n = compressed index): rows ks*16 + [0,16), column block
+          const int col = (a_wn * C::ANT + nt) * 8;
+          const int row = ks * 16 + (lmat & 1) * 8 + lrow;
+          ldsm_x2_t(sy + row * C::SY + col * 2, bf[nt][0], bf[nt][1]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < C::AMT; ++mt) {
+          // A = X^T (m = embedding dim t, k = feature rows): matrices (t0, i0), (t0+8, i0), (t0, i0+8), (t0+8, i0+8)
+          const int t0 = (a_wm * C::AMT + mt) * 16 + (lmat & 1) * 8;
+          const int row = ks * 16 + (lmat >> 1) * 8 + lrow;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(sx + row * C::SX + t0 * 2, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < C::ANT; ++nt) mma_bf16_16816(zacc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == C::STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    // partial Z tiles -> zpart[a_ks][t][c] (fp32)
+#pragma unroll
+    for (int mt = 0; mt < C::AMT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < C::ANT; ++nt) {
+        const int t = (a_wm * C::AMT + mt) * 16 + g;
+        const int cc = (a_wn * C::ANT + nt) * 8 + 2 * t4;
+        float* zp = zpart + a_ks * C::D * C::KC;
+        zp[t * C::KC + cc] = zacc[mt][nt][0];
+        zp[t * C::KC + cc + 1] = zacc[mt][nt][1];
+        zp[(t + 8) * C::KC + cc] = zacc[mt][nt][2];
+        zp[(t + 8) * C::KC + cc + 1] = zacc[mt][nt][3];
+      }
+    named_bar(1, 256);
+    for (int i = tid; i < C::D * C::KC; i += 256) {
+      float z = 0.f;
+#pragma unroll
+      for (int k = 0; k < C::AKS; ++k) z += zpart[k * C::D * C::KC + i];
+      const int t = i / C::KC, cc = i - t * C::KC;
+      *reinterpret_cast<__nv_bfloat16*>(zb + t * C::SY + cc * 2) = __float2bfloat16_rn(z);
+    }
+    named_bar(1, 256);
+    // Z as the B operand of pass B (k = embedding dim t, n = compressed index c)
+    uint32_t zf[C::BNT][C::KS_D][2];
+#pragma unroll
+    for (int nt = 0; nt < C::BNT; ++nt)
+#pragma unroll
+      for (int ks = 0; ks < C::KS_D; ++ks) {
+        const int col = (b_wn * C::BNT + nt) * 8;
+        const int row = ks * 16 + (lmat & 1) * 8 + lrow;
+        ldsm_x2_t(smem_u32(zb) + row * C::SY + col * 2, zf[nt][ks][0], zf[nt][ks][1]);
+      }
+
+    // ------------------------------------------------ pass B: F = X Z
+    float facc[C::NCH][C::BMT][C::BNT][4];
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c)
+#pragma unroll
+      for (int i = 0; i < C::BMT; ++i)
+#pragma unroll
+        for (int j = 0; j < C::BNT; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) facc[c][i][j][e] = 0.f;
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c) {
+      if (ok) ok = mbar_wait(&full[s], ph, status);
+      const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+      const uint32_t sx = smem_u32(ring + s * C::SLOT);
+#pragma unroll
+      for (int mt = 0; mt < C::BMT; ++mt) {
+        const int m0 = (b_wm * C::BMT + mt) * 16;
+        if (m0 < rows) {
+#pragma unroll
+          for (int ks = 0; ks < C::KS_D; ++ks) {
+            // A = X rows (m = features, k = embedding dim): matrices (m0, k0), (m0+8, k0), (m0, k0+8), (m0+8, k0+8)
+            const int row = m0 + (lmat & 1) * 8 + lrow;
+            const int col = ks * 16 + (lmat >> 1) * 8;
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(sx + row * C::SX + col * 2, a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < C::BNT; ++nt)
+              mma_bf16_16816(facc[c][mt][nt], a0, a1, a2, a3, zf[nt][ks][0], zf[nt][ks][1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == C::STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+
+    // ------------------------------------------------ LayerNorm over n*k
+    float part = 0.f;
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c)
+#pragma unroll
+      for (int mt = 0; mt < C::BMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::BNT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) part += facc[c][mt][nt][e];  // rows past n hold 0
+    part = warp_sum(part);
+    if (lane == 0) red[warp] = part;
+    named_bar(1, 256);
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float mean = tot * (1.0f / (C::N * C::KC));
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c)
+#pragma unroll
+      for (int mt = 0; mt < C::BMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::BNT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = c * C::R + (b_wm * C::BMT + mt) * 16 + g + (e >> 1) * 8;
+            const float dv = row < C::N ? facc[c][mt][nt][e] - mean : 0.f;
+            q += dv * dv;
+          }
+    q = warp_sum(q);
+    if (lane == 0) red[8 + warp] = q;
+    named_bar(1, 256);
+    float qt = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) qt += red[8 + w];
+    const float rstd = rsqrtf(qt * (1.0f / (C::N * C::KC)) + eps);
+    __nv_bfloat16* ab = A0 + b * (C::N * C::KC);
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c)
+#pragma unroll
+      for (int mt = 0; mt < C::BMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < C::BNT; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = c * C::R + (b_wm * C::BMT + mt) * 16 + g + h * 8;
+            if (row < C::N) {
+              const int col = (b_wn * C::BNT + nt) * 8 + 2 * t4;
+              const int idx = row * C::KC + col;
+              const float2 gm = __ldg(reinterpret_cast<const float2*>(gamma + idx));
+              const float2 bt = __ldg(reinterpret_cast<const float2*>(beta + idx));
+              const float v0 = (facc[c][mt][nt][2 * h] - mean) * rstd * gm.x + bt.x;
+              const float v1 = (facc[c][mt][nt][2 * h + 1] - mean) * rstd * gm.y + bt.y;
+              *reinterpret_cast<uint32_t*>(ab + idx) = pack_bf16x2(v0, v1);
+            }
+          }
+  }
+}
+
+// The instantiated shapes: (n, d, k) of the bf16 workloads.
+using FmC2 = FmCfg<64, 128, 16, 64, 4, 2, 1, 4, 2, 4>;
+using FmC3 = FmCfg<256, 160, 32, 64, 2, 4, 1, 2, 4, 4>;
+using FmC4 = FmCfg<512, 160, 64, 64, 2, 4, 1, 2, 4, 4>;
+using FmC5 = FmCfg<720, 32, 24, 128, 2, 1, 4, 8, 1, 4>;
+
+}  // namespace wk

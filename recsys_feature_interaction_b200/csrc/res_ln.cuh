@@ -1,0 +1,134 @@
+// res_ln.cuh -- concat + residual + LayerNorm of each embedding row (the end of a
+// Wukong layer: the FMB and LCB blocks are concatenated, the layer input is added
+// back and every output embedding is normalised; Wukong page, section 2.2).
+//
+//   out[r, :] = LN( cat[r, :] + x[r, :] ) * gamma + beta,   r < rows, d values per row
+//
+// HBM-bound: each element is read twice and written once or twice, so the kernel
+// moves 16-byte vectors (8 elements) with G = next_pow2(d/8) lanes per row and
+// 32/G rows per warp, keeps UNROLL row groups in flight per warp, and reduces
+// mean and variance (two passes over registers, fp32) with xor shuffles inside
+// each lane group. The grid is a multiple of the SM count.
+#pragma once
+
+#include "common.cuh"
+
+namespace wk {
+
+template <typename T>
+struct Vec8;
+
+template <>
+struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+
+template <>
+struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    v[0] = bf16_lo(a.x); v[1] = bf16_hi(a.x); v[2] = bf16_lo(a.y); v[3] = bf16_hi(a.y);
+    v[4] = bf16_lo(a.z); v[5] = bf16_hi(a.z); v[6] = bf16_lo(a.w); v[7] = bf16_hi(a.w);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 a;
+    a.x = pack_bf16x2(v[0], v[1]);
+    a.y = pack_bf16x2(v[2], v[3]);
+    a.z = pack_bf16x2(v[4], v[5]);
+    a.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = a;
+  }
+};
+
+constexpr int pow2_ceil(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// TC: concat element type, TR: residual element type, TO: main output type.
+// out32 (optional, fp32) receives the same values unrounded.
+template <int D, typename TC, typename TR, typename TO>
+__global__ void __launch_bounds__(256) res_ln_kernel(const TC* __restrict__ cat, const TR* __restrict__ x,
+                                                     const float* __restrict__ gamma,
+                                                     const float* __restrict__ beta, TO* __restrict__ out,
+                                                     float* __restrict__ out32, int64_t rows, float eps) {
+  constexpr int VPR = D / 8;           // 16-byte vectors (8 elements) per row
+  constexpr int G = pow2_ceil(VPR);    // lanes per row
+  static_assert(D % 8 == 0 && G <= 32, "d must be a multiple of 8 and at most 256");
+  constexpr int RPW = 32 / G;          // rows per warp step
+  constexpr int UNROLL = 4;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int sub = lane / G;            // row within the warp step
+  const int v = lane % G;              // vector index within the row
+  const bool vec_ok = v < VPR;
+
+  float g[8], b[8];
+  if (vec_ok) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      g[j] = gamma[v * 8 + j];
+      b[j] = beta[v * 8 + j];
+    }
+  }
+  const int64_t step = static_cast<int64_t>(gridDim.x) * nwarps * RPW * UNROLL;
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * nwarps + warp) * RPW * UNROLL; base < rows;
+       base += step) {
+    float y[UNROLL][8];
+    bool ok[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t r = base + u * RPW + sub;
+      ok[u] = vec_ok && r < rows;
+      if (ok[u]) {
+        float c8[8], x8[8];
+        Vec8<TC>::load(cat + r * D + v * 8, c8);
+        Vec8<TR>::load(x + r * D + v * 8, x8);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[u][j] = c8[j] + x8[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[u][j] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += y[u][j];
+#pragma unroll
+      for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const float mean = s * (1.0f / D);
+      float q = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float dv = ok[u] ? y[u][j] - mean : 0.f;
+        q += dv * dv;
+      }
+#pragma unroll
+      for (int o = G / 2; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      const float rstd = rsqrtf(q * (1.0f / D) + eps);
+      if (ok[u]) {
+        const int64_t r = base + u * RPW + sub;
+        float o8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o8[j] = (y[u][j] - mean) * rstd * g[j] + b[j];
+        Vec8<TO>::store(out + r * D + v * 8, o8);
+        if (out32) Vec8<float>::store(out32 + r * D + v * 8, o8);
+      }
+    }
+  }
+}
+
+}  // namespace wk

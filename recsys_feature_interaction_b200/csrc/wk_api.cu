@@ -1,0 +1,939 @@
+// wk_api.cu -- the C ABI of the Wukong interaction-stack forward (include/wukong.h):
+// argument validation, workspace, TMA descriptors, launch order and the
+// host-buffer pipeline. Every kernel it launches lives in the .cuh files next to
+// it; there is no host fallback: without a CUDA device every call that would
+// launch returns WK_ERR_CUDA.
+//
+// Layer order on the stream (Wukong page, section 2.2; per layer i):
+//   1. FM + LayerNorm      X_i -> A0                       (fm_mma.cuh / simt.cuh)
+//   2. MLP Linears         A0 -> ... -> concat rows 0..n_F-1 (gemm_tc.cuh, MODE_MLP)
+//   3. LCB                 X_i -> concat rows n_F..n-1      (gemm_tc.cuh, MODE_LCB)
+//   4. residual + LN       concat + X_i -> X_{i+1}          (res_ln.cuh)
+// bf16 stacks keep the residual stream (the layer outputs that are added back)
+// in fp32 and a bf16 copy for the tensor-core operands; the concat buffer is
+// fp32. Only the stack output is rounded to bf16.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "wukong.h"
+#include "common.cuh"
+#include "fm_mma.cuh"
+#include "gemm_tc.cuh"
+#include "res_ln.cuh"
+#include "simt.cuh"
+
+using namespace wk;
+
+namespace {
+
+__device__ unsigned g_standalone_status;
+
+typedef __nv_bfloat16 bf16;
+
+// ------------------------------------------------------------ device context
+
+struct DevInfo {
+  bool init = false;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  unsigned* standalone_status = nullptr;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+
+wk_status dev_info(DevInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return WK_ERR_CUDA;
+    }
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+      cudaGetLastError();
+      return WK_ERR_CUDA;
+    }
+    d.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    void* sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_standalone_status) != cudaSuccess) {
+      cudaGetLastError();
+      return WK_ERR_CUDA;
+    }
+    d.standalone_status = static_cast<unsigned*>(sym);
+    d.init = true;
+  }
+  *out = &d;
+  return WK_OK;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline wk_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? WK_OK : WK_ERR_CUDA;
+}
+
+// 2D/3D tiled tensor map; dims[0] is the contiguous dimension, strides in bytes
+// for dims 1..rank-1.
+bool make_map(const DevInfo* dv, CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank, const void* base,
+              const uint64_t* dims, const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
+  cuuint64_t gd[5];
+  cuuint64_t gs[4];
+  cuuint32_t bx[5];
+  cuuint32_t es[5];
+  for (uint32_t i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (uint32_t i = 0; i + 1 < rank; ++i) gs[i] = strides[i];
+  CUresult r = dv->encode(m, dt, rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------- GEMM maps
+
+struct GemmMaps {
+  CUtensorMap A, B, C;
+};
+
+// A [rows, K] bf16 row-major (K-major operand), box 64 x 128, 128B swizzle.
+bool map_kmajor(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[2] = {K, rows};
+  const uint64_t str[1] = {K * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return make_map(dv, m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Output [rows, N] with row stride ldc elements; 32 x 32 boxes (bf16: 64B swizzle, fp32: 128B).
+bool map_out(const DevInfo* dv, CUtensorMap* m, const void* p, bool f32, uint64_t N, uint64_t rows, uint64_t ldc) {
+  const uint64_t es = f32 ? 4 : 2;
+  const uint64_t dims[2] = {N, rows};
+  const uint64_t str[1] = {ldc * es};
+  const uint32_t box[2] = {32, 32};
+  return make_map(dv, m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, str,
+                  box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// X [batch, n, d] bf16 as the LCB's MN-major operand: box (32 t, 64 i, 1 b), 64B swizzle.
+bool map_lcb_x(const DevInfo* dv, CUtensorMap* m, const void* X, uint64_t n, uint64_t d, uint64_t batch) {
+  const uint64_t dims[3] = {d, n, batch};
+  const uint64_t str[2] = {d * 2, n * d * 2};
+  const uint32_t box[3] = {32, 64, 1};
+  return make_map(dv, m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// concat rows n_f..n-1 as a (t, r, b) tensor: box (32, 32, 1).
+bool map_lcb_out(const DevInfo* dv, CUtensorMap* m, const void* cat, bool f32, uint64_t n, uint64_t d, uint64_t n_f,
+                 uint64_t n_l, uint64_t batch) {
+  const uint64_t es = f32 ? 4 : 2;
+  const uint64_t dims[3] = {d, n_l, batch};
+  const uint64_t str[2] = {d * es, n * d * es};
+  const uint32_t box[3] = {32, 32, 1};
+  const uint8_t* base = static_cast<const uint8_t*>(cat) + n_f * d * es;
+  return make_map(dv, m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, str,
+                  box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+template <int MODE, typename TO>
+wk_status run_gemm_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p0, cudaStream_t st) {
+  static bool attr_done = false;
+  constexpr uint32_t smem = gemm_smem_bytes<TO>();
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<MODE, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return WK_ERR_CUDA;
+    }
+    attr_done = true;
+  }
+  GemmParams p = p0;
+  if (p.num_tiles <= 0) return WK_OK;
+  const int grid = std::min(p.num_tiles, dv->sms);
+  gemm_tc_kernel<MODE, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  return launch_status();
+}
+
+GemmParams mlp_params(int64_t M, int K, int N, const float* bias, int relu, unsigned* status) {
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = N;
+  p.K = K;
+  p.num_m_tiles = static_cast<int>((M + GEMM_BM - 1) / GEMM_BM);
+  p.num_n_tiles = (N + GEMM_BN - 1) / GEMM_BN;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  p.num_kb = (K + GEMM_BK - 1) / GEMM_BK;
+  p.group_m = 16;
+  p.mma_n = GEMM_BN;
+  p.bias = bias;
+  p.relu = relu;
+  p.status = status;
+  return p;
+}
+
+GemmParams lcb_params(int64_t batch, int n, int d, int n_l, unsigned* status) {
+  GemmParams p{};
+  p.M = n_l;
+  p.N = static_cast<int>(batch);
+  p.K = n;
+  p.d = d;
+  p.E = GEMM_BN / d;
+  p.dchunks = d / 32;
+  p.num_m_tiles = (n_l + GEMM_BM - 1) / GEMM_BM;
+  p.num_n_tiles = static_cast<int>((batch + p.E - 1) / p.E);
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  p.num_kb = (n + GEMM_BK - 1) / GEMM_BK;
+  p.mma_n = p.E * d;
+  p.status = status;
+  return p;
+}
+
+bool mlp_tc_ok(int64_t M, int K, int N, int64_t ldc) {
+  return M > 0 && K >= 8 && N >= 8 && K % 8 == 0 && N % 8 == 0 && ldc % 8 == 0 && ldc >= N && M < (1ll << 31);
+}
+
+bool lcb_tc_ok(int64_t batch, int n, int d) {
+  return d % 32 == 0 && d >= 32 && d <= GEMM_BN && n % 8 == 0 && batch < (1ll << 31);
+}
+
+// ------------------------------------------------------------------ FM + LN
+
+template <class C>
+wk_status run_fm_mma(const DevInfo* dv, const bf16* X, const bf16* Y, const float* g, const float* b, bf16* A0,
+                     int64_t batch, float eps, unsigned* status, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(fm_ln_mma_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return WK_ERR_CUDA;
+    }
+    attr_done = true;
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(batch, dv->sms));
+  fm_ln_mma_kernel<C><<<grid, FM_THREADS, C::SMEM, st>>>(X, Y, g, b, A0, batch, eps, status);
+  return launch_status();
+}
+
+size_t fm_simt_smem(int n, int d, int k) {
+  return sizeof(float) * (static_cast<size_t>(n) * d + 2ull * n * k + static_cast<size_t>(d) * k);
+}
+
+template <typename T>
+wk_status run_fm_simt(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0,
+                      int64_t batch, int n, int d, int k, float eps, cudaStream_t st) {
+  const size_t smem = fm_simt_smem(n, d, k);
+  if (smem > 200 * 1024) return WK_ERR_UNSUPPORTED;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(fm_ln_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(batch, 8ll * dv->sms));
+  fm_ln_simt<T><<<grid, 256, smem, st>>>(X, Y, g, b, A0, batch, n, d, k, eps);
+  return launch_status();
+}
+
+// bf16 FM dispatch: the tensor-core kernel for the instantiated shapes, else the CUDA-core one.
+wk_status run_fm_bf16(const DevInfo* dv, const bf16* X, const bf16* Y, const float* g, const float* b, bf16* A0,
+                      int64_t batch, int n, int d, int k, float eps, unsigned* status, cudaStream_t st) {
+  if (n == 512 && d == 160 && k == 64) return run_fm_mma<FmC4>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 256 && d == 160 && k == 32) return run_fm_mma<FmC3>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 64 && d == 128 && k == 16) return run_fm_mma<FmC2>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 720 && d == 32 && k == 24) return run_fm_mma<FmC5>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  return run_fm_simt<bf16>(dv, X, Y, g, b, A0, batch, n, d, k, eps, st);
+}
+
+bool fm_supported(int n, int d, int k, wk_dtype dt) {
+  if (dt == WK_BF16 && ((n == 512 && d == 160 && k == 64) || (n == 256 && d == 160 && k == 32) ||
+                        (n == 64 && d == 128 && k == 16) || (n == 720 && d == 32 && k == 24)))
+    return true;
+  return fm_simt_smem(n, d, k) <= 200 * 1024;
+}
+
+// ------------------------------------------------------------ residual + LN
+
+template <int D, typename TC, typename TR, typename TO>
+wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
+                       float* out32, int64_t rows, float eps, cudaStream_t st) {
+  constexpr int VPR = D / 8;
+  constexpr int G = pow2_ceil(VPR);
+  constexpr int rows_per_block = (256 / 32) * (32 / G) * 4;
+  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  const int64_t cap = static_cast<int64_t>(dv->sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  res_ln_kernel<D, TC, TR, TO><<<static_cast<int>(blocks), 256, 0, st>>>(cat, x, g, b, out, out32, rows, eps);
+  return launch_status();
+}
+
+bool res_ln_d_ok(int d) {
+  return d == 16 || d == 32 || d == 64 || d == 128 || d == 160 || d == 192 || d == 256;
+}
+
+template <typename TC, typename TR, typename TO>
+wk_status run_res_ln(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
+                     float* out32, int64_t rows, int d, float eps, cudaStream_t st) {
+  switch (d) {
+    case 16: return run_res_ln_d<16>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 32: return run_res_ln_d<32>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 64: return run_res_ln_d<64>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 128: return run_res_ln_d<128>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 160: return run_res_ln_d<160>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 192: return run_res_ln_d<192>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 256: return run_res_ln_d<256>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    default: return WK_ERR_UNSUPPORTED;
+  }
+}
+
+// ------------------------------------------------------------------- SIMT
+
+template <typename T, typename TO>
+wk_status run_gemm_simt(const T* A, const T* W, const float* bias, TO* C, int64_t M, int K, int N, int64_t ldc,
+                        int relu, cudaStream_t st) {
+  const int64_t gy = (M + 63) / 64;
+  if (gy > 65535) return WK_ERR_UNSUPPORTED;
+  dim3 grid((N + 63) / 64, static_cast<unsigned>(gy));
+  gemm_simt<T, TO><<<grid, 256, 0, st>>>(A, W, bias, C, M, K, N, ldc, relu);
+  return launch_status();
+}
+
+template <typename T, typename TO>
+wk_status run_lcb_simt(const T* WL, const T* X, TO* cat, int64_t batch, int n, int d, int n_f, int n_l,
+                       cudaStream_t st) {
+  for (int64_t b0 = 0; b0 < batch; b0 += 65535) {
+    const int64_t nb = std::min<int64_t>(65535, batch - b0);
+    dim3 grid((n_l * d + 255) / 256, static_cast<unsigned>(nb));
+    lcb_simt<T, TO><<<grid, 256, 0, st>>>(WL, X + b0 * n * d, cat + b0 * (n_f + n_l) * d, nb, n, d, n_f, n_l);
+    wk_status s = launch_status();
+    if (s != WK_OK) return s;
+  }
+  return WK_OK;
+}
+
+}  // namespace
+
+// ====================================================================== handle
+
+struct wk_stack {
+  int device = 0;
+  wk_stack_config cfg{};
+  std::vector<int32_t> dims;  // h_0 .. h_m
+  std::vector<wk_layer_weights> lw;
+  std::vector<std::vector<const void*>> W;
+  std::vector<std::vector<const float*>> b;
+  float eps = 1e-5f;
+  bool bf = true;  // bf16 storage
+  int64_t maxb = 0;
+  const DevInfo* dv = nullptr;
+  // workspace
+  uint8_t* ws = nullptr;
+  void* A0 = nullptr;
+  void* H[2] = {nullptr, nullptr};
+  void* cat = nullptr;  // fp32 (bf16 stacks) or fp32 (fp32 stacks)
+  void* X16[2] = {nullptr, nullptr};  // operand copies of the layer outputs (fp32 stacks: same as X32)
+  float* X32[2] = {nullptr, nullptr};
+  unsigned* status = nullptr;
+  // TMA descriptors of the tensor-core path
+  bool tc_mlp = false, tc_lcb = false;
+  std::vector<std::vector<GemmMaps>> mlp_maps;  // [layer][j]
+  std::vector<CUtensorMap> lcbA;                // [layer]
+  CUtensorMap lcbB_ws[2];
+  CUtensorMap lcbC;
+  // host-buffer forward
+  uint8_t* stage = nullptr;
+  int64_t stage_chunk = 0;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  // profiling
+  bool prof = false;
+  struct Rec {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+};
+
+namespace {
+
+struct ProfScope {
+  wk_stack* h;
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  ProfScope(wk_stack* h_, int k, cudaStream_t s) : h(h_), kind(k), st(s) {
+    if (!h->prof) return;
+    a = take();
+    b = take();
+    if (a && b) cudaEventRecord(a, st);
+  }
+  cudaEvent_t take() {
+    cudaEvent_t e = nullptr;
+    if (!h->pool.empty()) {
+      e = h->pool.back();
+      h->pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      e = nullptr;
+    }
+    return e;
+  }
+  ~ProfScope() {
+    if (!h->prof) return;
+    if (a && b) {
+      cudaEventRecord(b, st);
+      h->recs.push_back({kind, a, b});
+    } else {
+      if (a) h->pool.push_back(a);
+      if (b) h->pool.push_back(b);
+    }
+  }
+};
+
+void free_stack(wk_stack* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaGetLastError();
+  if (h->ws) cudaFree(h->ws);
+  if (h->stage) cudaFree(h->stage);
+  if (h->s_in) cudaStreamDestroy(h->s_in);
+  if (h->s_out) cudaStreamDestroy(h->s_out);
+  for (auto& r : h->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : h->pool) cudaEventDestroy(e);
+  cudaGetLastError();
+  delete h;
+}
+
+wk_status validate_cfg(const wk_stack_config* c) {
+  if (!c) return WK_ERR_INVALID_ARG;
+  if (c->num_layers < 1 || c->n < 1 || c->d < 1 || c->k < 1 || c->n_f < 1 || c->n_l < 1 || c->mlp_num_linear < 1 ||
+      c->max_batch < 1)
+    return WK_ERR_INVALID_ARG;
+  if (c->mlp_num_linear > 1 && !c->mlp_hidden) return WK_ERR_INVALID_ARG;
+  if (c->dtype != WK_F32 && c->dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (c->n_f + c->n_l != c->n) return WK_ERR_UNSUPPORTED;
+  if (c->dtype == WK_BF16 ? (c->d % 8 != 0) : (c->d % 8 != 0)) return WK_ERR_UNSUPPORTED;
+  if (!res_ln_d_ok(c->d)) return WK_ERR_UNSUPPORTED;
+  for (int j = 0; j + 1 < c->mlp_num_linear; ++j)
+    if (c->mlp_hidden[j] < 1 || c->mlp_hidden[j] % 8 != 0) return WK_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(c->n) * c->k) % 8 != 0) return WK_ERR_UNSUPPORTED;
+  if (!fm_supported(c->n, c->d, c->k, c->dtype)) return WK_ERR_UNSUPPORTED;
+  if (c->ln_eps < 0.f) return WK_ERR_INVALID_ARG;
+  return WK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wk_status_string(wk_status s) {
+  switch (s) {
+    case WK_OK: return "ok";
+    case WK_ERR_INVALID_ARG: return "invalid argument";
+    case WK_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case WK_ERR_OOM: return "out of device memory";
+    case WK_ERR_CUDA: return "CUDA runtime error";
+    case WK_ERR_TIMEOUT: return "a kernel gave up waiting (device pipeline timeout)";
+    case WK_ERR_DEVICE: return "device-side error flag";
+  }
+  return "unknown status";
+}
+
+wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* weights, wk_stack** out) {
+  if (!out || !weights) return WK_ERR_INVALID_ARG;
+  *out = nullptr;
+  wk_status st = validate_cfg(cfg);
+  if (st != WK_OK) return st;
+  const int L = cfg->num_layers, m = cfg->mlp_num_linear;
+  const int n = cfg->n, d = cfg->d, k = cfg->k;
+  std::vector<int32_t> dims;
+  dims.push_back(n * k);
+  for (int j = 0; j + 1 < m; ++j) dims.push_back(cfg->mlp_hidden[j]);
+  dims.push_back(cfg->n_f * d);
+  // weight pointers
+  for (int l = 0; l < L; ++l) {
+    const wk_layer_weights& w = weights[l];
+    if (!w.Y || !w.W || !w.fmb_ln_gamma || !w.fmb_ln_beta || !w.W_L || !w.out_ln_gamma || !w.out_ln_beta)
+      return WK_ERR_INVALID_ARG;
+    if (!al16(w.Y) || !al16(w.W_L) || !al16(w.fmb_ln_gamma) || !al16(w.fmb_ln_beta) || !al16(w.out_ln_gamma) ||
+        !al16(w.out_ln_beta))
+      return WK_ERR_INVALID_ARG;
+    for (int j = 0; j < m; ++j) {
+      if (!w.W[j] || !al16(w.W[j])) return WK_ERR_INVALID_ARG;
+      if (w.b && w.b[j] && !al16(w.b[j])) return WK_ERR_INVALID_ARG;
+    }
+  }
+  DevInfo* dv = nullptr;
+  st = dev_info(&dv);
+  if (st != WK_OK) return st;
+
+  wk_stack* h = new (std::nothrow) wk_stack();
+  if (!h) return WK_ERR_OOM;
+  cudaGetDevice(&h->device);
+  h->cfg = *cfg;
+  h->cfg.mlp_hidden = nullptr;
+  h->dims = dims;
+  h->eps = cfg->ln_eps > 0.f ? cfg->ln_eps : 1e-5f;
+  h->bf = cfg->dtype == WK_BF16;
+  h->maxb = cfg->max_batch;
+  h->dv = dv;
+  h->lw.assign(weights, weights + L);
+  h->W.resize(L);
+  h->b.resize(L);
+  for (int l = 0; l < L; ++l) {
+    for (int j = 0; j < m; ++j) {
+      h->W[l].push_back(weights[l].W[j]);
+      h->b[l].push_back(weights[l].b ? weights[l].b[j] : nullptr);
+    }
+  }
+
+  // workspace
+  const int64_t B = h->maxb;
+  const size_t es = h->bf ? 2 : 4;
+  int32_t hmax = 8;
+  for (int j = 1; j < m; ++j) hmax = std::max(hmax, dims[j]);
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const size_t nd = static_cast<size_t>(n) * d;
+  size_t off = 0;
+  const size_t o_a0 = off;
+  off += up(B * static_cast<size_t>(n) * k * es);
+  const size_t o_h0 = off;
+  off += up(B * static_cast<size_t>(hmax) * es);
+  const size_t o_h1 = off;
+  off += up(B * static_cast<size_t>(hmax) * es);
+  const size_t o_cat = off;
+  off += up(B * nd * 4);
+  const size_t o_x32_0 = off;
+  off += up(B * nd * 4);
+  const size_t o_x32_1 = off;
+  off += up(B * nd * 4);
+  size_t o_x16_0 = 0, o_x16_1 = 0;
+  if (h->bf) {
+    o_x16_0 = off;
+    off += up(B * nd * 2);
+    o_x16_1 = off;
+    off += up(B * nd * 2);
+  }
+  const size_t o_status = off;
+  off += 256;
+  if (cudaMalloc(&h->ws, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return WK_ERR_OOM;
+  }
+  h->A0 = h->ws + o_a0;
+  h->H[0] = h->ws + o_h0;
+  h->H[1] = h->ws + o_h1;
+  h->cat = h->ws + o_cat;
+  h->X32[0] = reinterpret_cast<float*>(h->ws + o_x32_0);
+  h->X32[1] = reinterpret_cast<float*>(h->ws + o_x32_1);
+  h->X16[0] = h->bf ? static_cast<void*>(h->ws + o_x16_0) : static_cast<void*>(h->X32[0]);
+  h->X16[1] = h->bf ? static_cast<void*>(h->ws + o_x16_1) : static_cast<void*>(h->X32[1]);
+  h->status = reinterpret_cast<unsigned*>(h->ws + o_status);
+  if (cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess) {
+    cudaGetLastError();
+    free_stack(h);
+    return WK_ERR_CUDA;
+  }
+
+  // tensor-core path descriptors
+  if (h->bf) {
+    h->tc_mlp = true;
+    for (int j = 0; j < m; ++j) {
+      const int64_t ldc = (j == m - 1) ? static_cast<int64_t>(nd) : dims[j + 1];
+      if (!mlp_tc_ok(B, dims[j], dims[j + 1], ldc)) h->tc_mlp = false;
+    }
+    h->tc_lcb = lcb_tc_ok(B, n, d);
+    if (h->tc_mlp) {
+      h->mlp_maps.resize(L);
+      for (int l = 0; l < L; ++l) {
+        h->mlp_maps[l].resize(m);
+        for (int j = 0; j < m; ++j) {
+          GemmMaps& mp = h->mlp_maps[l][j];
+          const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+          const bool last = j == m - 1;
+          bool ok = map_kmajor(dv, &mp.A, in, dims[j], B, GEMM_BM) &&
+                    map_kmajor(dv, &mp.B, h->W[l][j], dims[j], dims[j + 1], GEMM_BN) &&
+                    (last ? map_out(dv, &mp.C, h->cat, true, dims[j + 1], B, nd)
+                          : map_out(dv, &mp.C, h->H[j % 2], false, dims[j + 1], B, dims[j + 1]));
+          if (!ok) {
+            free_stack(h);
+            return WK_ERR_UNSUPPORTED;
+          }
+        }
+      }
+    }
+    if (h->tc_lcb) {
+      h->lcbA.resize(L);
+      bool ok = true;
+      for (int l = 0; l < L; ++l) ok = ok && map_kmajor(dv, &h->lcbA[l], h->lw[l].W_L, n, cfg->n_l, GEMM_BM);
+      ok = ok && map_lcb_x(dv, &h->lcbB_ws[0], h->X16[0], n, d, B) && map_lcb_x(dv, &h->lcbB_ws[1], h->X16[1], n, d, B) &&
+           map_lcb_out(dv, &h->lcbC, h->cat, true, n, d, cfg->n_f, cfg->n_l, B);
+      if (!ok) {
+        free_stack(h);
+        return WK_ERR_UNSUPPORTED;
+      }
+    }
+  }
+  *out = h;
+  return WK_OK;
+}
+
+wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t batch, wk_stream_t stream) {
+  if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X || !out || !al16(X) || !al16(out)) return WK_ERR_INVALID_ARG;
+  const wk_stack_config& c = h->cfg;
+  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers;
+  const size_t es = h->bf ? 2 : 4;
+  const size_t bytes = static_cast<size_t>(batch) * n * d * es;
+  const uint8_t* xa = static_cast<const uint8_t*>(X);
+  const uint8_t* oa = static_cast<const uint8_t*>(out);
+  if (xa < oa + bytes && oa < xa + bytes) return WK_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) {
+    cudaGetLastError();
+    return WK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const DevInfo* dv = h->dv;
+  const int64_t rows = batch * n;
+  const size_t nd = static_cast<size_t>(n) * d;
+  wk_status s = WK_OK;
+
+  CUtensorMap lcbB_user;
+  if (h->bf && h->tc_lcb && !map_lcb_x(dv, &lcbB_user, X, n, d, batch)) return WK_ERR_CUDA;
+
+  for (int l = 0; l < L && s == WK_OK; ++l) {
+    const wk_layer_weights& w = h->lw[l];
+    const bool last = l == L - 1;
+    const void* xin = (l == 0) ? X : h->X16[(l - 1) % 2];
+    // 1. FM + LN
+    {
+      ProfScope ps(h, WK_KERNEL_FM_LN, st);
+      if (h->bf)
+        s = run_fm_bf16(dv, static_cast<const bf16*>(xin), static_cast<const bf16*>(w.Y), w.fmb_ln_gamma,
+                        w.fmb_ln_beta, static_cast<bf16*>(h->A0), batch, n, d, k, h->eps, h->status, st);
+      else
+        s = run_fm_simt<float>(dv, static_cast<const float*>(xin), static_cast<const float*>(w.Y), w.fmb_ln_gamma,
+                               w.fmb_ln_beta, static_cast<float*>(h->A0), batch, n, d, k, h->eps, st);
+    }
+    // 2. MLP
+    for (int j = 0; j < m && s == WK_OK; ++j) {
+      ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+      const bool lastj = j == m - 1;
+      void* o = lastj ? h->cat : h->H[j % 2];
+      const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
+      const int relu = lastj ? 0 : 1;
+      if (h->bf && h->tc_mlp) {
+        GemmParams p = mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status);
+        s = lastj ? run_gemm_tc<MODE_MLP, float>(dv, h->mlp_maps[l][j], p, st)
+                  : run_gemm_tc<MODE_MLP, bf16>(dv, h->mlp_maps[l][j], p, st);
+      } else if (h->bf) {
+        s = lastj ? run_gemm_simt<bf16, float>(static_cast<const bf16*>(in), static_cast<const bf16*>(h->W[l][j]),
+                                               h->b[l][j], static_cast<float*>(o), batch, h->dims[j],
+                                               h->dims[j + 1], ldc, relu, st)
+                  : run_gemm_simt<bf16, bf16>(static_cast<const bf16*>(in), static_cast<const bf16*>(h->W[l][j]),
+                                              h->b[l][j], static_cast<bf16*>(o), batch, h->dims[j], h->dims[j + 1],
+                                              ldc, relu, st);
+      } else {
+        s = run_gemm_simt<float, float>(static_cast<const float*>(in), static_cast<const float*>(h->W[l][j]),
+                                        h->b[l][j], static_cast<float*>(o), batch, h->dims[j], h->dims[j + 1], ldc,
+                                        relu, st);
+      }
+    }
+    if (s != WK_OK) break;
+    // 3. LCB
+    {
+      ProfScope ps(h, WK_KERNEL_LCB, st);
+      if (h->bf && h->tc_lcb) {
+        GemmMaps mp;
+        mp.A = h->lcbA[l];
+        mp.B = (l == 0) ? lcbB_user : h->lcbB_ws[(l - 1) % 2];
+        mp.C = h->lcbC;
+        s = run_gemm_tc<MODE_LCB, float>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
+      } else if (h->bf) {
+        s = run_lcb_simt<bf16, float>(static_cast<const bf16*>(w.W_L), static_cast<const bf16*>(xin),
+                                      static_cast<float*>(h->cat), batch, n, d, c.n_f, c.n_l, st);
+      } else {
+        s = run_lcb_simt<float, float>(static_cast<const float*>(w.W_L), static_cast<const float*>(xin),
+                                       static_cast<float*>(h->cat), batch, n, d, c.n_f, c.n_l, st);
+      }
+    }
+    if (s != WK_OK) break;
+    // 4. residual + LN
+    {
+      ProfScope ps(h, WK_KERNEL_RES_LN, st);
+      const float* cat = static_cast<const float*>(h->cat);
+      if (h->bf) {
+        bf16* o16 = last ? static_cast<bf16*>(out) : static_cast<bf16*>(h->X16[l % 2]);
+        float* o32 = last ? nullptr : h->X32[l % 2];
+        if (l == 0)
+          s = run_res_ln<float, bf16, bf16>(dv, cat, static_cast<const bf16*>(X), w.out_ln_gamma, w.out_ln_beta, o16,
+                                            o32, rows, d, h->eps, st);
+        else
+          s = run_res_ln<float, float, bf16>(dv, cat, h->X32[(l - 1) % 2], w.out_ln_gamma, w.out_ln_beta, o16, o32,
+                                             rows, d, h->eps, st);
+      } else {
+        float* o = last ? static_cast<float*>(out) : h->X32[l % 2];
+        const float* resid = (l == 0) ? static_cast<const float*>(X) : h->X32[(l - 1) % 2];
+        s = run_res_ln<float, float, float>(dv, cat, resid, w.out_ln_gamma, w.out_ln_beta, o, nullptr, rows, d,
+                                            h->eps, st);
+      }
+    }
+  }
+  return s;
+}
+
+wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host, int64_t batch, wk_stream_t stream) {
+  if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X_host || !out_host) return WK_ERR_INVALID_ARG;
+  const size_t es = h->bf ? 2 : 4;
+  const size_t ex_bytes = static_cast<size_t>(h->cfg.n) * h->cfg.d * es;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Chunks of at least 1024 examples (or the whole batch): large enough that the
+  // GEMMs stay efficient, small enough that copies overlap the compute.
+  int64_t chunk = std::max<int64_t>(1024, (batch + 3) / 4);
+  chunk = std::min(chunk, batch);
+  if (!h->stage || h->stage_chunk < chunk) {
+    if (h->stage) {
+      cudaFree(h->stage);
+      h->stage = nullptr;
+    }
+    const int64_t cap = std::min<int64_t>(h->maxb, std::max<int64_t>(1024, (h->maxb + 3) / 4));
+    const int64_t want = std::max(cap, chunk);
+    if (cudaMalloc(&h->stage, 4 * static_cast<size_t>(want) * ex_bytes) != cudaSuccess) {
+      cudaGetLastError();
+      h->stage = nullptr;
+      return WK_ERR_OOM;
+    }
+    h->stage_chunk = want;
+  }
+  if (!h->s_in && cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking) != cudaSuccess) return WK_ERR_CUDA;
+  if (!h->s_out && cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking) != cudaSuccess) return WK_ERR_CUDA;
+  uint8_t* din[2] = {h->stage, h->stage + h->stage_chunk * ex_bytes};
+  uint8_t* dout[2] = {h->stage + 2 * h->stage_chunk * ex_bytes, h->stage + 3 * h->stage_chunk * ex_bytes};
+  cudaEvent_t ev_start, ev_in[2], ev_done[2], ev_out[2];
+  cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+  for (int i = 0; i < 2; ++i) {
+    cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
+    cudaEventCreateWithFlags(&ev_done[i], cudaEventDisableTiming);
+    cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming);
+  }
+  cudaEventRecord(ev_start, st);
+  cudaStreamWaitEvent(h->s_in, ev_start, 0);
+  cudaStreamWaitEvent(h->s_out, ev_start, 0);
+  wk_status s = WK_OK;
+  int c = 0;
+  for (int64_t b0 = 0; b0 < batch && s == WK_OK; b0 += chunk, ++c) {
+    const int p = c & 1;
+    const int64_t nb = std::min(chunk, batch - b0);
+    const size_t nbytes = static_cast<size_t>(nb) * ex_bytes;
+    if (c >= 2) cudaStreamWaitEvent(h->s_in, ev_done[p], 0);  // forward c-2 finished reading din[p]
+    if (cudaMemcpyAsync(din[p], static_cast<const uint8_t*>(X_host) + b0 * ex_bytes, nbytes, cudaMemcpyHostToDevice,
+                        h->s_in) != cudaSuccess) {
+      s = WK_ERR_CUDA;
+      break;
+    }
+    cudaEventRecord(ev_in[p], h->s_in);
+    cudaStreamWaitEvent(st, ev_in[p], 0);
+    if (c >= 2) cudaStreamWaitEvent(st, ev_out[p], 0);  // copy-out of c-2 finished reading dout[p]
+    s = wk_stack_forward(h, din[p], dout[p], nb, stream);
+    if (s != WK_OK) break;
+    cudaEventRecord(ev_done[p], st);
+    cudaStreamWaitEvent(h->s_out, ev_done[p], 0);
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + b0 * ex_bytes, dout[p], nbytes, cudaMemcpyDeviceToHost,
+                        h->s_out) != cudaSuccess) {
+      s = WK_ERR_CUDA;
+      break;
+    }
+    cudaEventRecord(ev_out[p], h->s_out);
+  }
+  if (cudaStreamSynchronize(h->s_out) != cudaSuccess) s = WK_ERR_CUDA;
+  if (cudaStreamSynchronize(h->s_in) != cudaSuccess) s = WK_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) s = WK_ERR_CUDA;
+  cudaEventDestroy(ev_start);
+  for (int i = 0; i < 2; ++i) {
+    cudaEventDestroy(ev_in[i]);
+    cudaEventDestroy(ev_done[i]);
+    cudaEventDestroy(ev_out[i]);
+  }
+  cudaGetLastError();
+  return s;
+}
+
+static wk_status read_status_word(unsigned* word, cudaStream_t st) {
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  unsigned v = 0;
+  if (cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  if (v) {
+    const unsigned zero = 0;
+    cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice);
+  }
+  if (v & kFlagTimeout) return WK_ERR_TIMEOUT;
+  if (v) return WK_ERR_DEVICE;
+  return WK_OK;
+}
+
+wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream) {
+  if (!h) return WK_ERR_INVALID_ARG;
+  return read_status_word(h->status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+void wk_stack_destroy(wk_stack* h) { free_stack(h); }
+
+wk_status wk_stack_set_profiling(wk_stack* h, int enable) {
+  if (!h) return WK_ERR_INVALID_ARG;
+  h->prof = enable != 0;
+  return WK_OK;
+}
+
+wk_status wk_stack_kernel_times(wk_stack* h, double* total_ms, int64_t* launches) {
+  if (!h || !total_ms || !launches) return WK_ERR_INVALID_ARG;
+  for (int i = 0; i < WK_KERNEL_COUNT; ++i) {
+    total_ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  wk_status s = WK_OK;
+  for (auto& r : h->recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();
+      s = WK_ERR_CUDA;
+    } else if (r.kind >= 0 && r.kind < WK_KERNEL_COUNT) {
+      total_ms[r.kind] += ms;
+      launches[r.kind] += 1;
+    }
+    h->pool.push_back(r.a);
+    h->pool.push_back(r.b);
+  }
+  h->recs.clear();
+  return s;
+}
+
+// ------------------------------------------------------------- stand-alone
+
+wk_status wk_fm_ln(const void* X, const void* Y, const float* gamma, const float* beta, void* A0, int64_t batch,
+                   int32_t n, int32_t d, int32_t k, wk_dtype dtype, float eps, wk_stream_t stream) {
+  if (batch < 0 || n < 1 || d < 1 || k < 1) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X || !Y || !gamma || !beta || !A0 || !al16(X) || !al16(Y) || !al16(A0) || !al16(gamma) || !al16(beta))
+    return WK_ERR_INVALID_ARG;
+  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || k % 2 != 0 || !fm_supported(n, d, k, dtype)) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  const float e = eps > 0.f ? eps : 1e-5f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WK_BF16)
+    return run_fm_bf16(dv, static_cast<const bf16*>(X), static_cast<const bf16*>(Y), gamma, beta,
+                       static_cast<bf16*>(A0), batch, n, d, k, e, dv->standalone_status, st);
+  return run_fm_simt<float>(dv, static_cast<const float*>(X), static_cast<const float*>(Y), gamma, beta,
+                            static_cast<float*>(A0), batch, n, d, k, e, st);
+}
+
+wk_status wk_mlp_linear(const void* A, const void* W, const float* bias, void* C, int64_t M, int32_t K, int32_t N,
+                        int64_t ldc, int relu, wk_dtype dtype, wk_stream_t stream) {
+  if (M < 0 || K < 1 || N < 1 || ldc < N) return WK_ERR_INVALID_ARG;
+  if (M == 0) return WK_OK;
+  if (!A || !W || !C || !al16(A) || !al16(W) || !al16(C) || (bias && !al16(bias))) return WK_ERR_INVALID_ARG;
+  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WK_BF16) {
+    if (!mlp_tc_ok(M, K, N, ldc)) return WK_ERR_UNSUPPORTED;
+    GemmMaps mp;
+    if (!map_kmajor(dv, &mp.A, A, K, M, GEMM_BM) || !map_kmajor(dv, &mp.B, W, K, N, GEMM_BN) ||
+        !map_out(dv, &mp.C, C, false, N, M, ldc))
+      return WK_ERR_UNSUPPORTED;
+    return run_gemm_tc<MODE_MLP, bf16>(dv, mp, mlp_params(M, K, N, bias, relu ? 1 : 0, dv->standalone_status), st);
+  }
+  return run_gemm_simt<float, float>(static_cast<const float*>(A), static_cast<const float*>(W), bias,
+                                     static_cast<float*>(C), M, K, N, ldc, relu ? 1 : 0, st);
+}
+
+wk_status wk_lcb(const void* W_L, const void* X, void* concat, int64_t batch, int32_t n, int32_t d, int32_t n_f,
+                 int32_t n_l, wk_dtype dtype, wk_stream_t stream) {
+  if (batch < 0 || n < 1 || d < 1 || n_f < 0 || n_l < 1) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!W_L || !X || !concat || !al16(W_L) || !al16(X) || !al16(concat)) return WK_ERR_INVALID_ARG;
+  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WK_BF16) {
+    if (!lcb_tc_ok(batch, n, d)) {
+      return run_lcb_simt<bf16, bf16>(static_cast<const bf16*>(W_L), static_cast<const bf16*>(X),
+                                      static_cast<bf16*>(concat), batch, n, d, n_f, n_l, st);
+    }
+    GemmMaps mp;
+    if (!map_kmajor(dv, &mp.A, W_L, n, n_l, GEMM_BM) || !map_lcb_x(dv, &mp.B, X, n, d, batch) ||
+        !map_lcb_out(dv, &mp.C, concat, false, n_f + n_l, d, n_f, n_l, batch))
+      return WK_ERR_UNSUPPORTED;
+    return run_gemm_tc<MODE_LCB, bf16>(dv, mp, lcb_params(batch, n, d, n_l, dv->standalone_status), st);
+  }
+  return run_lcb_simt<float, float>(static_cast<const float*>(W_L), static_cast<const float*>(X),
+                                    static_cast<float*>(concat), batch, n, d, n_f, n_l, st);
+}
+
+wk_status wk_res_ln(const void* concat, const void* X, const float* gamma, const float* beta, void* out, int64_t rows,
+                    int32_t d, wk_dtype dtype, float eps, wk_stream_t stream) {
+  if (rows < 0 || d < 1) return WK_ERR_INVALID_ARG;
+  if (rows == 0) return WK_OK;
+  if (!concat || !X || !gamma || !beta || !out || !al16(concat) || !al16(X) || !al16(out) || !al16(gamma) ||
+      !al16(beta))
+    return WK_ERR_INVALID_ARG;
+  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (!res_ln_d_ok(d)) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  const float e = eps > 0.f ? eps : 1e-5f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WK_BF16)
+    return run_res_ln<bf16, bf16, bf16>(dv, static_cast<const bf16*>(concat), static_cast<const bf16*>(X), gamma,
+                                        beta, static_cast<bf16*>(out), nullptr, rows, d, e, st);
+  return run_res_ln<float, float, float>(dv, static_cast<const float*>(concat), static_cast<const float*>(X), gamma,
+                                         beta, static_cast<float*>(out), nullptr, rows, d, e, st);
+}
+
+wk_status wk_device_status(wk_stream_t stream) {
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  return read_status_word(dv->standalone_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+"""The C ABI boundary without a GPU: the library loads, exports every entry point
+that include/wukong.h declares, and rejects invalid arguments before touching a
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import recsys_feature_interaction_b200 as wk
+from recsys_feature_interaction_b200 import build as wk_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^WK_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    wk_build.build()
+    return wk.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert len(wk.wk_status_string(s)) >= 2
+    assert wk.wk_status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    c = dict(num_layers=1, n=16, d=16, k=4, n_f=8, n_l=8, hidden=[64], dtype="f32", batch=64)
+    c.update(kw)
+    return c
+
+
+FAKE = 1 << 20  # aligned, never dereferenced by validation
+
+
+def _fake_layers(m, count=1):
+    layer = {"Y": FAKE, "W_L": FAKE, "fmb_gamma": FAKE, "fmb_beta": FAKE, "out_gamma": FAKE, "out_beta": FAKE}
+    for j in range(m):
+        layer["W%d" % j] = FAKE
+        layer["b%d" % j] = None
+    return [layer] * count
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(n_f=9), wk.WK_ERR_UNSUPPORTED),          # n_f + n_l != n: no residual projection
+    (dict(num_layers=0), wk.WK_ERR_INVALID_ARG),
+    (dict(batch=0), wk.WK_ERR_INVALID_ARG),
+    (dict(d=12), wk.WK_ERR_UNSUPPORTED),            # d % 8 != 0
+    (dict(hidden=[60]), wk.WK_ERR_UNSUPPORTED),     # hidden width % 8 != 0
+])
+def test_create_rejects_invalid_config_without_gpu(L, bad, status):
+    cfg = _cfg(**bad)
+    with pytest.raises(wk.WkError) as e:
+        wk.wk_stack_create(cfg, _fake_layers(len(cfg["hidden"]) + 1))
+    assert e.value.status == status
+
+
+def test_create_rejects_misaligned_weights(L):
+    layers = _fake_layers(2)
+    layers = [dict(layers[0], Y=FAKE + 4)]
+    with pytest.raises(wk.WkError) as e:
+        wk.wk_stack_create(_cfg(), layers)
+    assert e.value.status == wk.WK_ERR_INVALID_ARG
+
+
+def test_create_without_device_reports_cuda_error(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    with pytest.raises(wk.WkError) as e:
+        wk.wk_stack_create(_cfg(), _fake_layers(2))
+    assert e.value.status == wk.WK_ERR_CUDA
+
+
+def test_null_handle_and_stand_alone_argument_checks(L):
+    assert L.wk_stack_forward(None, FAKE, FAKE * 2, 1, None) == wk.WK_ERR_INVALID_ARG
+    assert L.wk_stack_sync_status(None, None) == wk.WK_ERR_INVALID_ARG
+    L.wk_stack_destroy(None)
+    # misaligned pointers and bad sizes are rejected before any launch
+    assert L.wk_mlp_linear(FAKE + 2, FAKE, None, FAKE, 4, 64, 64, 64, 0, 1, None) == wk.WK_ERR_INVALID_ARG
+    assert L.wk_mlp_linear(FAKE, FAKE, None, FAKE, 4, 64, 64, 32, 0, 1, None) == wk.WK_ERR_INVALID_ARG
+    assert L.wk_res_ln(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 160, 1, ctypes.c_float(0), None) == wk.WK_ERR_INVALID_ARG
+    assert L.wk_fm_ln(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 16, 16, 4, 0, ctypes.c_float(0), None) == wk.WK_OK
+    assert L.wk_lcb(FAKE, FAKE, FAKE, 3, 16, 16, 8, 8, 7, None) == wk.WK_ERR_UNSUPPORTED
