@@ -1,0 +1,287 @@
+"""Throughput of the Wukong interaction-stack forward on B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    (N > 1: python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...)
+
+One step is one forward of the whole stack (every layer: FM + LayerNorm, the FMB
+MLP, the LCB, residual + LayerNorm) over one batch of synthetic examples. The
+workload is the 8-layer bf16 stack (n=512 embeddings, d=160, k=64, n_F=n_L=256,
+FMB MLP 32768->16384->16384->40960, ~24.1 GFLOP/example) at batch 4096 per GPU.
+Several GPUs run independent replicas on disjoint batches (the examples are
+independent, so there is no collective in the forward): weak scaling.
+
+Rank 0 prints one JSON line. `value` is examples/s of the whole job with the
+inputs resident in HBM (CUDA events on the launch stream, max over ranks);
+`e2e` is the same metric through wk_stack_forward_host with pinned host buffers
+(host-to-device copy of X and device-to-host copy of the output inside the timed
+region); `roofline` reports the MLP GEMM kernel (the dominant one) against the
+measured bf16 peak; `cpu_baseline` times the fp64 oracle on a bounded sample.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "c4_bf16"
+METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack fwd, 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(cfg):
+    dims = [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
+    return ("%d-layer bf16 Wukong stack fwd: n=%d, d=%d, k=%d, n_F=n_L=%d, FMB MLP %s" %
+            (cfg["layers"], cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], "->".join(str(v) for v in dims)))
+
+
+def gemm_flops_per_example(cfg):
+    dims = [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
+    return cfg["layers"] * 2 * sum(dims[j] * dims[j + 1] for j in range(len(dims) - 1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [v for v in sm if mx is None or v > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(cfg, n_examples, threads=None):
+    """Times the fp64 oracle on n_examples examples through ONE layer (the layer's
+    weights are generated before the clock starts) and returns (examples/s of the
+    whole stack, seconds, threads)."""
+    import oracle
+    from synth import configs as C
+    w = C.make_layer_host(cfg, 0)
+    X = C.to_f64(C.make_x_host(cfg, list(range(n_examples))))
+    thr = threads or oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.layer_forward(cfg, w, X, threads=thr)
+    dt = time.perf_counter() - t0
+    return n_examples / (dt * cfg["layers"]), dt, thr
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    from synth import configs as C
+    cfg = C.CONFIGS[WORKLOAD]
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample(cfg, 2)
+    thr = None
+    for _ in range(args.steps):
+        v, dt, thr = oracle_sample(cfg, 2)
+        vals.append(v)
+    value = statistics.median(vals)
+    sample = "2 examples through 1 of the %d layers per step, scaled to the whole stack" % cfg["layers"]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD + ": " + workload_desc(cfg), "global_batch": cfg["batch"],
+                       "oracle": "plain C fp64, threads over examples / output rows"},
+            "cpu_baseline": {"value": value, "unit": "examples/s", "cores": thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "examples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import recsys_feature_interaction_b200 as wk
+    from recsys_feature_interaction_b200 import build as wk_build
+    from synth import configs as C
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    wk_build.build()
+
+    cfg = C.CONFIGS[WORKLOAD]
+    B = cfg["batch"]
+    layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
+    h = wk.wk_stack_create(cfg, layers, max_batch=B)
+    # rank r works on examples [r*B, (r+1)*B) of the synthetic stream
+    X = C.make_x_dev(cfg, B, device=dev, first_example=rank * B)
+    out = torch.empty_like(X)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        wk.wk_stack_forward(h, X, out, stream=stream)
+    torch.cuda.synchronize(dev)
+    if wk.wk_stack_sync_status(h) != wk.WK_OK:
+        raise RuntimeError("device status after warm-up")
+    wk.wk_stack_kernel_times(h)  # clear
+
+    # ---- device-resident timing
+    wk.wk_stack_set_profiling(h, True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            wk.wk_stack_forward(h, X, out, stream=stream)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    wk.wk_stack_set_profiling(h, False)
+    ms = ev0.elapsed_time(ev1)
+    status = wk.wk_stack_sync_status(h)
+    if status != wk.WK_OK:
+        raise RuntimeError("device status: " + wk.wk_status_string(status))
+    ktimes = wk.wk_stack_kernel_times(h)
+    ms_max = max_over_ranks(ms)
+    value = world * B * args.steps / (ms_max / 1e3)
+
+    # ---- end to end through the host-buffer entry point
+    xh = X.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    wk.wk_stack_forward_host(h, xh, oh)  # warm the staging buffers
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        wk.wk_stack_forward_host(h, xh, oh)
+    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    e2e_value = world * B * args.steps / e2e_s
+    step_bytes = B * cfg["n"] * cfg["d"] * 2
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops_ex = C.flops_per_example(cfg)
+        tflops = value * flops_ex / 1e12 / world
+        g_ms, g_n = ktimes["mlp_gemm"]
+        gemm_flops_launch = gemm_flops_per_example(cfg) * B / (cfg["layers"] * (len(cfg["hidden"]) + 1))
+        achieved = gemm_flops_launch / ((g_ms / g_n) / 1e3) / 1e12 if g_n else None
+        peak = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+        clocks = clk.summary()
+        launches_per_step = sum(n for _, n in ktimes.values()) // max(1, args.steps)
+        line = {
+            "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD + ": " + workload_desc(cfg), "per_gpu_batch": B,
+                       "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
+                       "l2": "inputs larger than L2 (X 671 MB, weights 23.6 GB per GPU)"},
+            "tflops_per_gpu": tflops,
+            "pct_of_bf16_peak": 100.0 * tflops / peak,
+            "peak_source": "%s bf16_tflops_sustained" % peak_src,
+            "roofline": {"kernel": "mlp_gemm (tcgen05)", "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None, "traffic": None,
+                         "peak_note": "%s sustained cuBLAS bf16" % peak_src},
+            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "examples/s", "h2d_bytes_per_step": step_bytes,
+                    "d2h_bytes_per_step": step_bytes},
+            "gpu_launches": launches_per_step * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, dt, thr = oracle_sample(cfg, 2)
+            line["cpu_baseline"] = {"value": v, "unit": "examples/s", "cores": thr, "kind": "oracle",
+                                    "sample": "2 examples through 1 of the %d layers (%.1f s), scaled to the "
+                                              "whole stack" % (cfg["layers"], dt)}
+        print(json.dumps(line), flush=True)
+    wk.wk_stack_destroy(h)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -52,10 +52,12 @@ struct FmCfg {
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-constexpr int FM_THREADS = 288;  // 8 consumer warps + 1 producer warp
+// 8 consumer warps + 1 producer warp. With 9 warps one SM sub-partition holds
+// three of them, so its 16K-register file caps the kernel at 168 registers a thread.
+constexpr int FM_THREADS = 288;
 
 template <class C>
-__global__ void __maxnreg__(224)
+__global__ void __launch_bounds__(FM_THREADS, 1)
     fm_ln_mma_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ Y,
                      const float* __restrict__ gamma, const float* __restrict__ beta,
                      __nv_bfloat16* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
