@@ -21,9 +21,16 @@
  *   - Pointers named *_host are host memory; every other data pointer is device
  *     memory on the current CUDA device. All device pointers must be 16-byte
  *     aligned. Tensors are dense and row-major (last index fastest).
- *   - dtype WK_BF16: X, out, Y, W_j, W_L are bf16; biases and LayerNorm
- *     parameters are fp32; all products accumulate in fp32, LayerNorm
- *     statistics are fp32. dtype WK_F32: everything is fp32.
+ *   - dtype WK_BF16 / WK_F16: X, out, Y, W_j, W_L are 16-bit; biases and
+ *     LayerNorm parameters are fp32; all products accumulate in fp32 and
+ *     LayerNorm statistics are fp32. The tensor-core operands and every
+ *     intermediate buffer of a stack use the 16-bit `operand_dtype` (fp16 by
+ *     default: its 10-bit mantissa keeps the 8-layer drift of the intermediate
+ *     roundings ~6x below bf16's, at the same tensor-core rate); bf16 weights are
+ *     converted to it once, at create. Intermediate values must stay within the
+ *     fp16 range (|v| < 65504) when the operand type is fp16; they are
+ *     LayerNorm outputs and Linear layers of them. dtype WK_F32: everything is
+ *     fp32 on CUDA cores.
  *   - Calls that take a stream are asynchronous and stream-ordered: they only
  *     validate their arguments on the host and enqueue kernels. They never
  *     synchronise and never copy between host and device, except
@@ -63,7 +70,7 @@ typedef enum {
   WK_ERR_DEVICE = 6        /* the device status word holds another error flag */
 } wk_status;
 
-typedef enum { WK_F32 = 0, WK_BF16 = 1 } wk_dtype;
+typedef enum { WK_F32 = 0, WK_BF16 = 1, WK_F16 = 2 } wk_dtype;
 
 /* Shape of the stack; every layer has the same shape (n is the same for every
  * layer because n_F + n_L = n). Scaling knobs of section 2.3: num_layers = l,
@@ -75,9 +82,12 @@ typedef struct {
   int32_t n, d, k, n_f, n_l;   /* n_f + n_l == n; d % 8 == 0 (bf16) or d % 4 == 0 (fp32) */
   int32_t mlp_num_linear;      /* m >= 1 */
   const int32_t* mlp_hidden;   /* m-1 widths (may be NULL when m == 1); copied at create */
-  wk_dtype dtype;
+  wk_dtype dtype;              /* storage type of X, out, Y, W_j and W_L */
   float ln_eps;                /* LayerNorm epsilon; 0 selects 1e-5 */
   int64_t max_batch;           /* largest batch a forward will be given; sizes the workspace */
+  wk_dtype operand_dtype;      /* 16-bit stacks: WK_F16 or WK_BF16 tensor-core operands and
+                                  intermediates; WK_F32 (0) selects the default, WK_F16.
+                                  Ignored when dtype is WK_F32. */
 } wk_stack_config;
 
 /* One layer's parameters. All DEVICE pointers, BORROWED: the caller keeps them
@@ -102,11 +112,13 @@ typedef struct {
 typedef struct wk_stack wk_stack;
 
 /* Validates cfg, records the weight pointers of cfg->num_layers layers
- * (weights[0 .. num_layers-1]), builds the TMA descriptors of the weights and
- * allocates the workspace for cfg->max_batch examples on the current device:
- * A0 [max_batch, n*k], two MLP activation buffers [max_batch, max hidden], the
- * concat buffer [max_batch, n, d] and two layer buffers [max_batch, n, d].
- * The handle owns the workspace; *out is set only on WK_OK.
+ * (weights[0 .. num_layers-1]), converts the weights to the operand type when it
+ * differs from dtype (a device copy the handle owns; the originals are then no
+ * longer read), builds the TMA descriptors of the weights and allocates the
+ * workspace for cfg->max_batch examples on the current device, in the operand
+ * type: A0 [max_batch, n*k], two MLP activation buffers [max_batch, max hidden],
+ * the concat buffer [max_batch, n, d] and two layer buffers [max_batch, n, d].
+ * Synchronises the device. The handle owns the workspace; *out is set only on WK_OK.
  * Errors: WK_ERR_INVALID_ARG (NULL, misaligned, max_batch < 1),
  * WK_ERR_UNSUPPORTED (n_f + n_l != n, unsupported d / dtype / widths),
  * WK_ERR_OOM, WK_ERR_CUDA. */

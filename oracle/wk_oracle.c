@@ -92,11 +92,30 @@ static double round_bf16_via_f32(double v) {
 }
 
 /* diagnostic rounding points (bit mask of the diag argument) */
-enum { DIAG_A0 = 1, DIAG_HIDDEN = 2, DIAG_CONCAT = 4, DIAG_XOUT = 8, DIAG_XOPS = 16 };
+enum { DIAG_A0 = 1, DIAG_HIDDEN = 2, DIAG_CONCAT = 4, DIAG_XOUT = 8, DIAG_XOPS = 16, DIAG_Z = 32, DIAG_F16 = 64 };
+
+/* set by wko_layer_forward from the DIAG_F16 bit: round to fp16 instead of bf16 */
+static int g_diag_f16 = 0;
+
+/* double -> fp32 (nearest-even) -> fp16 (nearest-even, subnormals kept), diagnostic only */
+static double round_f16_via_f32(double v) {
+  float f = (float)v;
+  double a = fabs((double)f);
+  if (a == 0.0 || a >= 65520.0) return a >= 65520.0 ? copysign(INFINITY, v) : (double)f;
+  int e;
+  frexp(a, &e);                          /* a = m * 2^e, m in [0.5, 1) */
+  int q = e - 11;                        /* spacing 2^(e-11) for 11 significant bits */
+  if (q < -24) q = -24;                  /* subnormal spacing */
+  double step = ldexp(1.0, q);
+  double r = nearbyint((double)f / step) * step;   /* ties to even under the default mode */
+  return r;
+}
+
+static double round_diag(double v) { return g_diag_f16 ? round_f16_via_f32(v) : round_bf16_via_f32(v); }
 
 static void maybe_round(double* v, int64_t len, int diag) {
   if (!diag) return;
-  for (int64_t i = 0; i < len; ++i) v[i] = round_bf16_via_f32(v[i]);
+  for (int64_t i = 0; i < len; ++i) v[i] = round_diag(v[i]);
 }
 
 /* ---- the steps, each on one example ------------------------------------ */
@@ -212,7 +231,23 @@ static void fmb_front(void* c, int64_t e0, int64_t e1) {
   for (int64_t e = e0; e < e1; ++e) {
     memcpy(Xr, L->X_in + e * (int64_t)n * d, sizeof(double) * (size_t)n * d);
     maybe_round(Xr, (int64_t)n * d, L->diag & DIAG_XOPS);
-    wko_fm(n, d, k, Xr, L->Yd, P, F);
+    if (L->diag & DIAG_Z) {
+      /* diagnostic only: the compressed association X (X^T Y) with X^T Y rounded to bf16 */
+      for (int32_t t = 0; t < d; ++t)
+        for (int32_t c = 0; c < k; ++c) {
+          double z = 0.0;
+          for (int32_t i = 0; i < n; ++i) z += Xr[(int64_t)i * d + t] * L->Yd[(int64_t)i * k + c];
+          P[(int64_t)t * k + c] = round_diag(z);
+        }
+      for (int32_t i = 0; i < n; ++i)
+        for (int32_t c = 0; c < k; ++c) {
+          double f = 0.0;
+          for (int32_t t = 0; t < d; ++t) f += Xr[(int64_t)i * d + t] * P[(int64_t)t * k + c];
+          F[(int64_t)i * k + c] = f;
+        }
+    } else {
+      wko_fm(n, d, k, Xr, L->Yd, P, F);
+    }
     /* flatten row-major (feature i major, compressed index c minor), LayerNorm over n*k */
     double* a0 = L->h[0] + e * (int64_t)n * k;
     wko_layernorm((int64_t)n * k, F, L->g1, L->b1, cfg->ln_eps, a0);
@@ -295,7 +330,8 @@ static double* upcast_f32(const float* p, int64_t len) {
  * intermediate, selected by bits: 1 the FMB LayerNorm output, 2 each MLP
  * activation, 4 the concatenated blocks, 8 the layer output, 16 the copy of the
  * layer input that the FM and the LCB multiply (the residual keeps the unrounded
- * input). diag = 0 is the
+ * input), 32 the FM taken as X (X^T Y) with X^T Y rounded; bit 64 rounds to fp16
+ * instead of bf16. diag = 0 is the
  * exact fp64 reference (the one parity is graded against).
  * Returns 0, or 1 on an invalid configuration. */
 int wko_layer_forward(const wko_config* cfg, const wko_layer* w, int64_t n_ex, const double* X_in, double* X_out,
@@ -306,6 +342,7 @@ int wko_layer_forward(const wko_config* cfg, const wko_layer* w, int64_t n_ex, c
   int m = cfg->mlp_num_linear;
   layer_ctx L;
   memset(&L, 0, sizeof L);
+  g_diag_f16 = (diag & DIAG_F16) != 0;
   L.cfg = cfg;
   L.w = w;
   L.n_ex = n_ex;

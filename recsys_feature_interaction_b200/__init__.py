@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
 
 WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
-WK_F32, WK_BF16 = 0, 1
+WK_F32, WK_BF16, WK_F16 = 0, 1, 2
 WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_COUNT = range(5)
 KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln")
 
@@ -34,7 +34,8 @@ class WkStackConfig(ctypes.Structure):
     _fields_ = [("num_layers", ctypes.c_int32), ("n", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("n_f", ctypes.c_int32), ("n_l", ctypes.c_int32),
                 ("mlp_num_linear", ctypes.c_int32), ("mlp_hidden", ctypes.POINTER(ctypes.c_int32)),
-                ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("max_batch", ctypes.c_int64)]
+                ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("max_batch", ctypes.c_int64),
+                ("operand_dtype", ctypes.c_int)]
 
 
 class WkLayerWeights(ctypes.Structure):
@@ -118,6 +119,8 @@ def _dtype_code(dtype):
     s = str(dtype)
     if "bfloat16" in s or s == "bf16":
         return WK_BF16
+    if "float16" in s or s in ("f16", "fp16", "half"):
+        return WK_F16
     if "float32" in s or s in ("f32", "fp32"):
         return WK_F32
     raise ValueError("unsupported dtype %r" % (dtype,))
@@ -139,7 +142,7 @@ class StackHandle:
             pass
 
 
-def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0):
+def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0, operand_dtype=None):
     """cfg: mapping with num_layers (or layers), n, d, k, n_f, n_l, hidden (the m-1
     hidden widths) and dtype; layers: one mapping per layer with Y, W0..W{m-1},
     b0..b{m-1} (or None), fmb_gamma, fmb_beta, W_L, out_gamma, out_beta."""
@@ -148,7 +151,8 @@ def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0):
     hid = (ctypes.c_int32 * max(1, len(hidden)))(*hidden) if hidden else None
     c = WkStackConfig(int(cfg.get("num_layers", cfg.get("layers"))), cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
                       cfg["n_l"], m, hid, _dtype_code(dtype if dtype is not None else cfg["dtype"]),
-                      float(ln_eps), int(max_batch if max_batch is not None else cfg["batch"]))
+                      float(ln_eps), int(max_batch if max_batch is not None else cfg["batch"]),
+                      _dtype_code(operand_dtype) if operand_dtype is not None else WK_F32)
     keep = [hid, list(layers)]
     arr = (WkLayerWeights * len(layers))()
     for i, w in enumerate(layers):

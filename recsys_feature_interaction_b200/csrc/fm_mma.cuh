@@ -1,4 +1,4 @@
-// fm_mma.cuh -- the FMB front of a Wukong layer for bf16 inputs:
+// fm_mma.cuh -- the FMB front of a Wukong layer for 16-bit operands (fp16 or bf16):
 //
 //   A0[b] = LN( flatten_rowmajor( X_b (X_b^T Y) ) ) * gamma + beta
 //
@@ -6,16 +6,17 @@
 // compress the features to k with Y, then cross), flattened (feature i major,
 // compressed index c minor) and normalised over all n*k values.
 //
-// One persistent CTA per SM walks the examples. A producer warp streams each
+// One persistent CTA per SM walks the examples. A producer thread streams each
 // example's X rows (and the matching Y rows) from global memory into a ring of
-// shared-memory slots with bulk async copies (one copy per row, into rows padded
-// to an odd number of 16-byte units so ldmatrix is conflict-free), signalling an
-// mbarrier per slot. Eight consumer warps run two passes over the ring:
+// shared-memory slots with TMA tile loads -- X as 32-column blocks with the 64-byte
+// swizzle, Y with the swizzle that matches its row width -- so that ldmatrix,
+// addressed through the same swizzle, is conflict-free; an mbarrier per slot
+// carries the transaction count. Eight consumer warps run two passes over the ring:
 //   pass A: Z = X^T Y   (d x k, reduction over the n features) with mma.sync
-//           m16n8k16 (bf16 in, fp32 accumulate), partial sums of up to AKS warps
-//           per output tile added in a fixed order, Z rounded to bf16 in smem;
+//           m16n8k16 (16-bit in, fp32 accumulate), partial sums of up to AKS warps
+//           per output tile added in a fixed order, Z rounded to the 16-bit type;
 //   pass B: F = X Z     (n x k, reduction over d), F kept in registers;
-// then the LayerNorm statistics (two passes, fp32) and the bf16 store of A0. The
+// then the LayerNorm statistics (two passes, fp32) and the 16-bit store of A0. The
 // producer prefetches the next example while the current one finishes.
 #pragma once
 
@@ -33,9 +34,12 @@ template <int N_, int D_, int KC_, int R_, int AWM_, int AWN_, int AKS_, int BWM
 struct FmCfg {
   static constexpr int N = N_, D = D_, KC = KC_, R = R_;
   static constexpr int AWM = AWM_, AWN = AWN_, AKS = AKS_, BWM = BWM_, BWN = BWN_, STAGES = STAGES_;
-  static constexpr int SX = odd16(D * 2);     // bytes per staged X row
-  static constexpr int SY = odd16(KC * 2);    // bytes per staged Y row and per Z row
-  static constexpr int SLOT = R * SX + R * SY;
+  static constexpr int XBLK = R * 64;        // one 32-column block of R X rows (64B swizzle)
+  static constexpr int XBYTES = (D / 32) * XBLK;
+  static constexpr int YROW = KC * 2;         // bytes per Y row in the slot
+  static constexpr int YSW = (YROW == 128) ? 128 : (YROW == 64) ? 64 : (YROW == 32) ? 32 : 0;  // Y swizzle span
+  static constexpr int SY = odd16(KC * 2);    // bytes per Z row (padded, conflict-free)
+  static constexpr int SLOT = XBYTES + R * YROW;
   static constexpr int NCH = (N + R - 1) / R;
   static constexpr int AMT = (D / 16) / AWM;  // pass A m16 tiles per warp (over d)
   static constexpr int ANT = (KC / 8) / AWN;  // pass A n8 tiles per warp (over k)
@@ -44,8 +48,10 @@ struct FmCfg {
   static constexpr int KS_D = D / 16;         // pass B k16 steps
   static constexpr int ZPART_BYTES = AKS * D * KC * 4;
   static constexpr int ZB_BYTES = D * SY;
-  static constexpr int SMEM = 128 + STAGES * SLOT + ZPART_BYTES + ZB_BYTES + 64 + 16 * STAGES + 16;
-  static_assert(D % 16 == 0 && KC % 8 == 0 && N % 16 == 0 && R % 16 == 0, "tile shape");
+  static constexpr int SMEM = 1024 + STAGES * SLOT + ZPART_BYTES + ZB_BYTES + 64 + 16 * STAGES + 16;
+  static_assert(D % 32 == 0 && KC % 8 == 0 && N % 16 == 0 && R % 16 == 0 && R <= 256, "tile shape");
+  static_assert(SLOT % 1024 == 0 && XBLK % 1024 == 0, "slot blocks stay aligned to the swizzle atoms");
+  static_assert(YSW != 0 || (YROW / 16) % 2 == 1, "unswizzled Y rows must be an odd number of 16-byte units");
   static_assert(AWM * AWN * AKS == 8 && BWM * BWN == 8, "8 consumer warps");
   static_assert((D / 16) % AWM == 0 && (KC / 8) % AWN == 0 && (R / 16) % BWM == 0 && (KC / 8) % BWN == 0,
                 "warp split");
@@ -56,13 +62,34 @@ struct FmCfg {
 // three of them, so its 16K-register file caps the kernel at 168 registers a thread.
 constexpr int FM_THREADS = 288;
 
+// Shared address of X element (row r, column c) of a slot, c a multiple of 8:
+// 32-column blocks of R rows x 64 B, 16-byte unit index XOR ((r >> 1) & 3).
 template <class C>
+__device__ __forceinline__ uint32_t fm_x_addr(uint32_t sx, int r, int c) {
+  const int unit = ((c & 31) >> 3) ^ ((r >> 1) & 3);
+  return sx + (c >> 5) * C::XBLK + r * 64 + unit * 16;
+}
+
+// Shared address of Y element (row r, column c), c a multiple of 8, with the
+// swizzle the TMA load applied for this row width.
+template <class C>
+__device__ __forceinline__ uint32_t fm_y_addr(uint32_t sy, int r, int c) {
+  int unit = c >> 3;
+  if (C::YSW == 128) unit ^= (r & 7);
+  else if (C::YSW == 64) unit ^= ((r >> 1) & 3);
+  else if (C::YSW == 32) unit ^= ((r >> 2) & 1);
+  return sy + r * C::YROW + unit * 16;
+}
+
+// tmX: X viewed as [batch*n rows, d] (box 32 x R, 64B swizzle);
+// tmY: Y [n, k] (box k x R, swizzle by row width). T: the 16-bit type of X, Y and A0.
+template <class C, typename T>
 __global__ void __launch_bounds__(FM_THREADS, 1)
-    fm_ln_mma_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ Y,
+    fm_ln_mma_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                      const float* __restrict__ gamma, const float* __restrict__ beta,
-                     __nv_bfloat16* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
+                     T* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* ring = smem;
   float* zpart = reinterpret_cast<float*>(ring + C::STAGES * C::SLOT);
   uint8_t* zb = reinterpret_cast<uint8_t*>(zpart) + C::ZPART_BYTES;
@@ -83,40 +110,35 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    int s = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x) {
-      const __nv_bfloat16* xb = X + b * C::N * C::D;
-      for (int pass = 0; ok && pass < 2; ++pass) {
-        for (int c = 0; c < C::NCH; ++c) {
-          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
-          int waited = 1;
-          if (lane == 0) waited = mbar_wait(&empty[s], ph ^ 1u, status) ? 1 : 0;
-          waited = __shfl_sync(0xffffffffu, waited, 0);
-          if (!waited) {
-            ok = false;
-            break;
-          }
-          uint8_t* slot = ring + s * C::SLOT;
-          if (lane == 0)
-            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(rows * C::D * 2 + (pass == 0 ? rows * C::KC * 2 : 0)));
-          __syncwarp();
-          for (int r = lane; r < rows; r += 32) {
-            bulk_load(slot + r * C::SX, xb + static_cast<int64_t>(c * C::R + r) * C::D, C::D * 2, &full[s]);
-            if (pass == 0)
-              bulk_load(slot + C::R * C::SX + r * C::SY, Y + static_cast<int64_t>(c * C::R + r) * C::KC, C::KC * 2,
-                        &full[s]);
-          }
-          if (++s == C::STAGES) {
-            s = 0;
-            ph ^= 1u;
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmY);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x) {
+        for (int pass = 0; ok && pass < 2; ++pass) {
+          for (int c = 0; c < C::NCH; ++c) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, status)) {
+              ok = false;
+              break;
+            }
+            uint8_t* slot = ring + s * C::SLOT;
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(pass == 0 ? C::SLOT : C::XBYTES));
+            const int row0 = static_cast<int>(b * C::N + c * C::R);
+#pragma unroll
+            for (int blk = 0; blk < C::D / 32; ++blk) tma_load_2d(&tmX, &full[s], slot + blk * C::XBLK, blk * 32, row0);
+            if (pass == 0) tma_load_2d(&tmY, &full[s], slot + C::XBYTES, 0, c * C::R);
+            if (++s == C::STAGES) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
         }
       }
-    }
-    if (!ok && lane == 0) {  // let every armed slot land before the CTA exits
-      for (int i = 0; i < C::STAGES; ++i) mbar_wait(&full[i], ph ^ (i < s ? 0u : 1u), nullptr);
+      if (!ok) {  // let every armed slot land before the CTA exits
+        for (int i = 0; i < C::STAGES; ++i) mbar_wait(&full[i], ph ^ (i < s ? 0u : 1u), nullptr);
+      }
     }
     return;
   }
@@ -154,7 +176,7 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
       if (ok) ok = mbar_wait(&full[s], ph, status);
       const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
       const uint32_t sx = smem_u32(ring + s * C::SLOT);
-      const uint32_t sy = sx + C::R * C::SX;
+      const uint32_t sy = sx + C::XBYTES;
       for (int ks = a_ks; ks < rows / 16; ks += C::AKS) {
         uint32_t bf[C::ANT][2];
 #pragma unroll
@@ -162,7 +184,7 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
           // B = Y (k = feature rows, n = compressed index): rows ks*16 + [0,16), column block
           const int col = (a_wn * C::ANT + nt) * 8;
           const int row = ks * 16 + (lmat & 1) * 8 + lrow;
-          ldsm_x2_t(sy + row * C::SY + col * 2, bf[nt][0], bf[nt][1]);
+          ldsm_x2_t(fm_y_addr<C>(sy, row, col), bf[nt][0], bf[nt][1]);
         }
 #pragma unroll
         for (int mt = 0; mt < C::AMT; ++mt) {
@@ -170,9 +192,9 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
           const int t0 = (a_wm * C::AMT + mt) * 16 + (lmat & 1) * 8;
           const int row = ks * 16 + (lmat >> 1) * 8 + lrow;
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(sx + row * C::SX + t0 * 2, a0, a1, a2, a3);
+          ldsm_x4_t(fm_x_addr<C>(sx, row, t0), a0, a1, a2, a3);
 #pragma unroll
-          for (int nt = 0; nt < C::ANT; ++nt) mma_bf16_16816(zacc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+          for (int nt = 0; nt < C::ANT; ++nt) mma_16816<T>(zacc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
         }
       }
       __syncwarp();
@@ -201,7 +223,7 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
 #pragma unroll
       for (int k = 0; k < C::AKS; ++k) z += zpart[k * C::D * C::KC + i];
       const int t = i / C::KC, cc = i - t * C::KC;
-      *reinterpret_cast<__nv_bfloat16*>(zb + t * C::SY + cc * 2) = __float2bfloat16_rn(z);
+      *reinterpret_cast<T*>(zb + t * C::SY + cc * 2) = Half16<T>::from(z);
     }
     named_bar(1, 256);
     // Z as the B operand of pass B (k = embedding dim t, n = compressed index c)
@@ -240,10 +262,10 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
             const int row = m0 + (lmat & 1) * 8 + lrow;
             const int col = ks * 16 + (lmat >> 1) * 8;
             uint32_t a0, a1, a2, a3;
-            ldsm_x4(sx + row * C::SX + col * 2, a0, a1, a2, a3);
+            ldsm_x4(fm_x_addr<C>(sx, row, col), a0, a1, a2, a3);
 #pragma unroll
             for (int nt = 0; nt < C::BNT; ++nt)
-              mma_bf16_16816(facc[c][mt][nt], a0, a1, a2, a3, zf[nt][ks][0], zf[nt][ks][1]);
+              mma_16816<T>(facc[c][mt][nt], a0, a1, a2, a3, zf[nt][ks][0], zf[nt][ks][1]);
           }
         }
       }
@@ -292,7 +314,7 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
 #pragma unroll
     for (int w = 0; w < 8; ++w) qt += red[8 + w];
     const float rstd = rsqrtf(qt * (1.0f / (C::N * C::KC)) + eps);
-    __nv_bfloat16* ab = A0 + b * (C::N * C::KC);
+    T* ab = A0 + b * (C::N * C::KC);
 #pragma unroll
     for (int c = 0; c < C::NCH; ++c)
 #pragma unroll
@@ -309,13 +331,13 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
               const float2 bt = __ldg(reinterpret_cast<const float2*>(beta + idx));
               const float v0 = (facc[c][mt][nt][2 * h] - mean) * rstd * gm.x + bt.x;
               const float v1 = (facc[c][mt][nt][2 * h + 1] - mean) * rstd * gm.y + bt.y;
-              *reinterpret_cast<uint32_t*>(ab + idx) = pack_bf16x2(v0, v1);
+              *reinterpret_cast<uint32_t*>(ab + idx) = Half16<T>::pack2(v0, v1);
             }
           }
   }
 }
 
-// The instantiated shapes: (n, d, k) of the bf16 workloads.
+// The instantiated shapes: (n, d, k) of the 16-bit workloads.
 using FmC2 = FmCfg<64, 128, 16, 64, 4, 2, 1, 4, 2, 4>;
 using FmC3 = FmCfg<256, 160, 32, 64, 2, 4, 1, 2, 4, 4>;
 using FmC4 = FmCfg<512, 160, 64, 64, 2, 4, 1, 2, 4, 4>;

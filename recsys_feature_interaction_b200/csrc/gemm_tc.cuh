@@ -1,6 +1,7 @@
 // gemm_tc.cuh -- the batch-wide tensor-core GEMM of the Wukong stack on sm_100a.
 //
 // Two uses (Wukong page, section 2.2):
+// Operands are fp16 or bf16 (both alike), accumulation fp32 in TMEM.
 //   MODE_MLP: one Linear of the FMB MLP over the whole batch,
 //             C[r, c] = act( sum_q A[r, q] W[c, q] + bias[c] ), A [M, K], W [N, K],
 //             both K-major; C has row stride ldc (the last Linear writes the FMB
@@ -12,7 +13,7 @@
 //
 // Design (one CTA per SM, persistent over output tiles, 192 threads):
 //   warp 0      TMA producer: fills a STAGES-deep ring of (A 128x64, B up to 256x64)
-//               bf16 tiles, 128B-swizzled (B of the LCB: 64B-swizzled 32-wide
+//               16-bit tiles, 128B-swizzled (B of the LCB: 64B-swizzled 32-wide
 //               column blocks), completion tracked by mbarrier transaction counts;
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and one
 //               thread issues tcgen05.mma (M=128, N<=256, K=16) over each stage,
@@ -80,7 +81,7 @@ __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, 
 }
 
 // Writes 32 fp32 values of one accumulator row into a 32x32 staging tile row,
-// laid out as the TMA store expects: bf16 rows of 64 B with the 64B swizzle, or
+// laid out as the TMA store expects: 16-bit rows of 64 B with the 64B swizzle, or
 // fp32 rows of 128 B with the 128B swizzle.
 template <typename TO>
 __device__ __forceinline__ void stage_row(uint8_t* buf, int row, const float (&v)[32]);
@@ -100,6 +101,20 @@ __device__ __forceinline__ void stage_row<__nv_bfloat16>(uint8_t* buf, int row, 
 }
 
 template <>
+__device__ __forceinline__ void stage_row<__half>(uint8_t* buf, int row, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 q;
+    q.x = Half16<__half>::pack2(v[8 * c + 0], v[8 * c + 1]);
+    q.y = Half16<__half>::pack2(v[8 * c + 2], v[8 * c + 3]);
+    q.z = Half16<__half>::pack2(v[8 * c + 4], v[8 * c + 5]);
+    q.w = Half16<__half>::pack2(v[8 * c + 6], v[8 * c + 7]);
+    const int pc = c ^ ((row >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + row * 64 + pc * 16) = q;
+  }
+}
+
+template <>
 __device__ __forceinline__ void stage_row<float>(uint8_t* buf, int row, const float (&v)[32]) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -109,7 +124,8 @@ __device__ __forceinline__ void stage_row<float>(uint8_t* buf, int row, const fl
   }
 }
 
-template <int MODE, typename TO>
+// T: operand type (__half or __nv_bfloat16, A and B alike); TO: output type.
+template <int MODE, typename T, typename TO>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, p.mma_n, 0, MODE == MODE_LCB ? 1 : 0);
+      const uint32_t idesc = idesc_f16kind_f32(GEMM_BM, p.mma_n, 0, MODE == MODE_LCB ? 1 : 0, Half16<T>::kBF16);
       int s = 0;
       uint32_t ph = 0;
       int acc = 0;
@@ -228,7 +244,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               bdesc = smem_desc(b_addr + kk * 32, 16, 1024, 2);
             else  // MN-major, 64B swizzle: 32-wide column blocks 4 KB apart, 8-row K groups 512 B apart
               bdesc = smem_desc(b_addr + kk * 1024, 4096, 512, 4);
-            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_f16kind(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[s]);
           issued = true;

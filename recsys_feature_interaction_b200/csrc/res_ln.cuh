@@ -49,6 +49,27 @@ struct Vec8<__nv_bfloat16> {
   }
 };
 
+template <>
+struct Vec8<__half> {
+  static __device__ __forceinline__ void load(const __half* p, float (&v)[8]) {
+    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = Half16<__half>::lo(w[i]);
+      v[2 * i + 1] = Half16<__half>::hi(w[i]);
+    }
+  }
+  static __device__ __forceinline__ void store(__half* p, const float (&v)[8]) {
+    uint4 a;
+    a.x = Half16<__half>::pack2(v[0], v[1]);
+    a.y = Half16<__half>::pack2(v[2], v[3]);
+    a.z = Half16<__half>::pack2(v[4], v[5]);
+    a.w = Half16<__half>::pack2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = a;
+  }
+};
+
 constexpr int pow2_ceil(int v) {
   int p = 1;
   while (p < v) p <<= 1;

@@ -22,8 +22,13 @@ __device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16* p, int
   return __bfloat162float(p[i]);
 }
 
+template <>
+__device__ __forceinline__ float ld_f<__half>(const __half* p, int64_t i) { return __half2float(p[i]); }
+
 template <typename T>
 __device__ __forceinline__ void st_f(T* p, int64_t i, float v);
+template <>
+__device__ __forceinline__ void st_f<__half>(__half* p, int64_t i, float v) { p[i] = __float2half_rn(v); }
 template <>
 __device__ __forceinline__ void st_f<float>(float* p, int64_t i, float v) { p[i] = v; }
 template <>

@@ -1,17 +1,18 @@
 // wk_api.cu -- the C ABI of the Wukong interaction-stack forward (include/wukong.h):
-// argument validation, workspace, TMA descriptors, launch order and the
-// host-buffer pipeline. Every kernel it launches lives in the .cuh files next to
-// it; there is no host fallback: without a CUDA device every call that would
-// launch returns WK_ERR_CUDA.
+// argument validation, workspace, weight conversion, TMA descriptors, launch order
+// and the host-buffer pipeline. Every kernel it launches lives in the .cuh files
+// next to it; there is no host fallback: without a CUDA device every call that
+// would launch returns WK_ERR_CUDA.
 //
 // Layer order on the stream (Wukong page, section 2.2; per layer i):
-//   1. FM + LayerNorm      X_i -> A0                       (fm_mma.cuh / simt.cuh)
-//   2. MLP Linears         A0 -> ... -> concat rows 0..n_F-1 (gemm_tc.cuh, MODE_MLP)
-//   3. LCB                 X_i -> concat rows n_F..n-1      (gemm_tc.cuh, MODE_LCB)
-//   4. residual + LN       concat + X_i -> X_{i+1}          (res_ln.cuh)
-// bf16 stacks keep the residual stream (the layer outputs that are added back)
-// in fp32 and a bf16 copy for the tensor-core operands; the concat buffer is
-// fp32. Only the stack output is rounded to bf16.
+//   1. FM + LayerNorm      X_i -> A0                          (fm_mma.cuh / simt.cuh)
+//   2. MLP Linears         A0 -> ... -> concat rows 0..n_F-1   (gemm_tc.cuh, MODE_MLP)
+//   3. LCB                 X_i -> concat rows n_F..n-1         (gemm_tc.cuh, MODE_LCB)
+//   4. residual + LN       concat + X_i -> X_{i+1}             (res_ln.cuh)
+// A 16-bit stack computes with 16-bit tensor-core operands T (fp16 by default,
+// bf16 on request) and fp32 accumulation; every intermediate buffer holds T. A
+// bf16 stack's weights are converted to T once, at create, and its input once per
+// forward. The stack output is written in the caller's type.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -19,10 +20,13 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <set>
+#include <utility>
 #include <vector>
 
 #include "wukong.h"
 #include "common.cuh"
+#include "convert.cuh"
 #include "fm_mma.cuh"
 #include "gemm_tc.cuh"
 #include "res_ln.cuh"
@@ -35,11 +39,13 @@ namespace {
 __device__ unsigned g_standalone_status;
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 // ------------------------------------------------------------ device context
 
 struct DevInfo {
   bool init = false;
+  int id = 0;
   int sms = 0;
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   unsigned* standalone_status = nullptr;
@@ -47,6 +53,7 @@ struct DevInfo {
 
 std::mutex g_mu;
 DevInfo g_dev[64];
+std::set<std::pair<int, const void*>> g_smem_attr;
 
 wk_status dev_info(DevInfo** out) {
   int dev = 0;
@@ -57,6 +64,7 @@ wk_status dev_info(DevInfo** out) {
   std::lock_guard<std::mutex> lk(g_mu);
   DevInfo& d = g_dev[dev];
   if (!d.init) {
+    d.id = dev;
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
       cudaGetLastError();
       return WK_ERR_CUDA;
@@ -81,6 +89,18 @@ wk_status dev_info(DevInfo** out) {
   return WK_OK;
 }
 
+// Raises the dynamic shared-memory limit of a kernel once per device.
+wk_status smem_attr(const DevInfo* dv, const void* fn, int bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_smem_attr.count({dv->id, fn})) return WK_OK;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  g_smem_attr.insert({dv->id, fn});
+  return WK_OK;
+}
+
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline wk_status launch_status() {
@@ -88,8 +108,19 @@ inline wk_status launch_status() {
   return e == cudaSuccess ? WK_OK : WK_ERR_CUDA;
 }
 
-// 2D/3D tiled tensor map; dims[0] is the contiguous dimension, strides in bytes
-// for dims 1..rank-1.
+inline size_t dtype_bytes(wk_dtype t) { return t == WK_F32 ? 4 : 2; }
+
+template <typename T>
+constexpr CUtensorMapDataType tmap_dtype() {
+  return sizeof(T) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                        : (Half16<T>::kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+}
+template <>
+constexpr CUtensorMapDataType tmap_dtype<float>() {
+  return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+}
+
+// Tiled tensor map; dims[0] is the contiguous dimension, strides in bytes for dims 1..rank-1.
 bool make_map(const DevInfo* dv, CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank, const void* base,
               const uint64_t* dims, const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
   cuuint64_t gd[5];
@@ -113,60 +144,55 @@ struct GemmMaps {
   CUtensorMap A, B, C;
 };
 
-// A [rows, K] bf16 row-major (K-major operand), box 64 x 128, 128B swizzle.
+// [rows, K] 16-bit row-major (a K-major operand): box 64 x box_rows, 128B swizzle.
+template <typename T>
 bool map_kmajor(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t K, uint64_t rows, uint32_t box_rows) {
   const uint64_t dims[2] = {K, rows};
   const uint64_t str[1] = {K * 2};
   const uint32_t box[2] = {64, box_rows};
-  return make_map(dv, m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map(dv, m, tmap_dtype<T>(), 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Output [rows, N] with row stride ldc elements; 32 x 32 boxes (bf16: 64B swizzle, fp32: 128B).
-bool map_out(const DevInfo* dv, CUtensorMap* m, const void* p, bool f32, uint64_t N, uint64_t rows, uint64_t ldc) {
-  const uint64_t es = f32 ? 4 : 2;
+// Output [rows, N], row stride ldc elements; 32 x 32 boxes (16-bit: 64B swizzle, fp32: 128B).
+template <typename TO>
+bool map_out(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t N, uint64_t rows, uint64_t ldc) {
   const uint64_t dims[2] = {N, rows};
-  const uint64_t str[1] = {ldc * es};
+  const uint64_t str[1] = {ldc * sizeof(TO)};
   const uint32_t box[2] = {32, 32};
-  return make_map(dv, m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, str,
-                  box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+  return make_map(dv, m, tmap_dtype<TO>(), 2, p, dims, str, box,
+                  sizeof(TO) == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// X [batch, n, d] bf16 as the LCB's MN-major operand: box (32 t, 64 i, 1 b), 64B swizzle.
+// X [batch, n, d] as the LCB's MN-major operand: box (32 t, 64 i, 1 b), 64B swizzle.
+template <typename T>
 bool map_lcb_x(const DevInfo* dv, CUtensorMap* m, const void* X, uint64_t n, uint64_t d, uint64_t batch) {
   const uint64_t dims[3] = {d, n, batch};
   const uint64_t str[2] = {d * 2, n * d * 2};
   const uint32_t box[3] = {32, 64, 1};
-  return make_map(dv, m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  return make_map(dv, m, tmap_dtype<T>(), 3, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// concat rows n_f..n-1 as a (t, r, b) tensor: box (32, 32, 1).
-bool map_lcb_out(const DevInfo* dv, CUtensorMap* m, const void* cat, bool f32, uint64_t n, uint64_t d, uint64_t n_f,
+// Rows n_f..n_f+n_l-1 of a [batch, rows, d] concat buffer as a (t, r, b) tensor: box (32, 32, 1).
+template <typename TO>
+bool map_lcb_out(const DevInfo* dv, CUtensorMap* m, const void* cat, uint64_t rows, uint64_t d, uint64_t n_f,
                  uint64_t n_l, uint64_t batch) {
-  const uint64_t es = f32 ? 4 : 2;
+  const uint64_t es = sizeof(TO);
   const uint64_t dims[3] = {d, n_l, batch};
-  const uint64_t str[2] = {d * es, n * d * es};
+  const uint64_t str[2] = {d * es, rows * d * es};
   const uint32_t box[3] = {32, 32, 1};
   const uint8_t* base = static_cast<const uint8_t*>(cat) + n_f * d * es;
-  return make_map(dv, m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, str,
-                  box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+  return make_map(dv, m, tmap_dtype<TO>(), 3, base, dims, str, box,
+                  es == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int MODE, typename TO>
-wk_status run_gemm_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p0, cudaStream_t st) {
-  static bool attr_done = false;
+template <int MODE, typename T, typename TO>
+wk_status run_gemm_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
   constexpr uint32_t smem = gemm_smem_bytes<TO>();
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<MODE, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return WK_ERR_CUDA;
-    }
-    attr_done = true;
-  }
-  GemmParams p = p0;
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc_kernel<MODE, T, TO>), smem);
+  if (s != WK_OK) return s;
   if (p.num_tiles <= 0) return WK_OK;
   const int grid = std::min(p.num_tiles, dv->sms);
-  gemm_tc_kernel<MODE, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  gemm_tc_kernel<MODE, T, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
 }
 
@@ -214,20 +240,31 @@ bool lcb_tc_ok(int64_t batch, int n, int d) {
 
 // ------------------------------------------------------------------ FM + LN
 
-template <class C>
-wk_status run_fm_mma(const DevInfo* dv, const bf16* X, const bf16* Y, const float* g, const float* b, bf16* A0,
-                     int64_t batch, float eps, unsigned* status, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(fm_ln_mma_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return WK_ERR_CUDA;
-    }
-    attr_done = true;
+template <class C, typename T>
+wk_status run_fm_mma(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
+                     float eps, unsigned* status, cudaStream_t st) {
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fm_ln_mma_kernel<C, T>), C::SMEM);
+  if (s != WK_OK) return s;
+  CUtensorMap tmX, tmY;
+  {  // X as [batch*n rows, d]: 32-column boxes of R rows, 64B swizzle
+    const uint64_t dims[2] = {static_cast<uint64_t>(C::D), static_cast<uint64_t>(batch) * C::N};
+    const uint64_t str[1] = {static_cast<uint64_t>(C::D) * 2};
+    const uint32_t box[2] = {32, static_cast<uint32_t>(C::R)};
+    if (!make_map(dv, &tmX, tmap_dtype<T>(), 2, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+      return WK_ERR_UNSUPPORTED;
+  }
+  {  // Y [n, k]: box k x R, swizzle by row width
+    const uint64_t dims[2] = {static_cast<uint64_t>(C::KC), static_cast<uint64_t>(C::N)};
+    const uint64_t str[1] = {static_cast<uint64_t>(C::KC) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(C::KC), static_cast<uint32_t>(C::R)};
+    const CUtensorMapSwizzle sw = C::YSW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : C::YSW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : C::YSW == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (!make_map(dv, &tmY, tmap_dtype<T>(), 2, Y, dims, str, box, sw)) return WK_ERR_UNSUPPORTED;
   }
   const int grid = static_cast<int>(std::min<int64_t>(batch, dv->sms));
-  fm_ln_mma_kernel<C><<<grid, FM_THREADS, C::SMEM, st>>>(X, Y, g, b, A0, batch, eps, status);
+  fm_ln_mma_kernel<C, T><<<grid, FM_THREADS, C::SMEM, st>>>(tmX, tmY, g, b, A0, batch, eps, status);
   return launch_status();
 }
 
@@ -240,31 +277,33 @@ wk_status run_fm_simt(const DevInfo* dv, const T* X, const T* Y, const float* g,
                       int64_t batch, int n, int d, int k, float eps, cudaStream_t st) {
   const size_t smem = fm_simt_smem(n, d, k);
   if (smem > 200 * 1024) return WK_ERR_UNSUPPORTED;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(fm_ln_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-          cudaSuccess) {
-    cudaGetLastError();
-    return WK_ERR_CUDA;
+  if (smem > 48 * 1024) {
+    wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fm_ln_simt<T>), static_cast<int>(smem));
+    if (s != WK_OK) return s;
   }
   const int grid = static_cast<int>(std::min<int64_t>(batch, 8ll * dv->sms));
   fm_ln_simt<T><<<grid, 256, smem, st>>>(X, Y, g, b, A0, batch, n, d, k, eps);
   return launch_status();
 }
 
-// bf16 FM dispatch: the tensor-core kernel for the instantiated shapes, else the CUDA-core one.
-wk_status run_fm_bf16(const DevInfo* dv, const bf16* X, const bf16* Y, const float* g, const float* b, bf16* A0,
-                      int64_t batch, int n, int d, int k, float eps, unsigned* status, cudaStream_t st) {
-  if (n == 512 && d == 160 && k == 64) return run_fm_mma<FmC4>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  if (n == 256 && d == 160 && k == 32) return run_fm_mma<FmC3>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  if (n == 64 && d == 128 && k == 16) return run_fm_mma<FmC2>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  if (n == 720 && d == 32 && k == 24) return run_fm_mma<FmC5>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  return run_fm_simt<bf16>(dv, X, Y, g, b, A0, batch, n, d, k, eps, st);
+bool fm_mma_shape(int n, int d, int k) {
+  return (n == 512 && d == 160 && k == 64) || (n == 256 && d == 160 && k == 32) || (n == 64 && d == 128 && k == 16) ||
+         (n == 720 && d == 32 && k == 24);
 }
 
-bool fm_supported(int n, int d, int k, wk_dtype dt) {
-  if (dt == WK_BF16 && ((n == 512 && d == 160 && k == 64) || (n == 256 && d == 160 && k == 32) ||
-                        (n == 64 && d == 128 && k == 16) || (n == 720 && d == 32 && k == 24)))
-    return true;
+// 16-bit FM dispatch: the tensor-core kernel for the instantiated shapes, else the CUDA-core one.
+template <typename T>
+wk_status run_fm16(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
+                   int n, int d, int k, float eps, unsigned* status, cudaStream_t st) {
+  if (n == 512 && d == 160 && k == 64) return run_fm_mma<FmC4, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 256 && d == 160 && k == 32) return run_fm_mma<FmC3, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 64 && d == 128 && k == 16) return run_fm_mma<FmC2, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 720 && d == 32 && k == 24) return run_fm_mma<FmC5, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  return run_fm_simt<T>(dv, X, Y, g, b, A0, batch, n, d, k, eps, st);
+}
+
+bool fm_supported(int n, int d, int k, bool sixteen_bit) {
+  if (sixteen_bit && fm_mma_shape(n, d, k)) return true;
   return fm_simt_smem(n, d, k) <= 200 * 1024;
 }
 
@@ -272,7 +311,7 @@ bool fm_supported(int n, int d, int k, wk_dtype dt) {
 
 template <int D, typename TC, typename TR, typename TO>
 wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
-                       float* out32, int64_t rows, float eps, cudaStream_t st) {
+                       int64_t rows, float eps, cudaStream_t st) {
   constexpr int VPR = D / 8;
   constexpr int G = pow2_ceil(VPR);
   constexpr int rows_per_block = (256 / 32) * (32 / G) * 4;
@@ -280,7 +319,7 @@ wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const floa
   const int64_t cap = static_cast<int64_t>(dv->sms) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  res_ln_kernel<D, TC, TR, TO><<<static_cast<int>(blocks), 256, 0, st>>>(cat, x, g, b, out, out32, rows, eps);
+  res_ln_kernel<D, TC, TR, TO><<<static_cast<int>(blocks), 256, 0, st>>>(cat, x, g, b, out, nullptr, rows, eps);
   return launch_status();
 }
 
@@ -290,17 +329,27 @@ bool res_ln_d_ok(int d) {
 
 template <typename TC, typename TR, typename TO>
 wk_status run_res_ln(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
-                     float* out32, int64_t rows, int d, float eps, cudaStream_t st) {
+                     int64_t rows, int d, float eps, cudaStream_t st) {
   switch (d) {
-    case 16: return run_res_ln_d<16>(dv, cat, x, g, b, out, out32, rows, eps, st);
-    case 32: return run_res_ln_d<32>(dv, cat, x, g, b, out, out32, rows, eps, st);
-    case 64: return run_res_ln_d<64>(dv, cat, x, g, b, out, out32, rows, eps, st);
-    case 128: return run_res_ln_d<128>(dv, cat, x, g, b, out, out32, rows, eps, st);
-    case 160: return run_res_ln_d<160>(dv, cat, x, g, b, out, out32, rows, eps, st);
-    case 192: return run_res_ln_d<192>(dv, cat, x, g, b, out, out32, rows, eps, st);
-    case 256: return run_res_ln_d<256>(dv, cat, x, g, b, out, out32, rows, eps, st);
+    case 16: return run_res_ln_d<16>(dv, cat, x, g, b, out, rows, eps, st);
+    case 32: return run_res_ln_d<32>(dv, cat, x, g, b, out, rows, eps, st);
+    case 64: return run_res_ln_d<64>(dv, cat, x, g, b, out, rows, eps, st);
+    case 128: return run_res_ln_d<128>(dv, cat, x, g, b, out, rows, eps, st);
+    case 160: return run_res_ln_d<160>(dv, cat, x, g, b, out, rows, eps, st);
+    case 192: return run_res_ln_d<192>(dv, cat, x, g, b, out, rows, eps, st);
+    case 256: return run_res_ln_d<256>(dv, cat, x, g, b, out, rows, eps, st);
     default: return WK_ERR_UNSUPPORTED;
   }
+}
+
+template <typename TI, typename TO>
+wk_status run_convert(const DevInfo* dv, const void* in, void* out, int64_t n, cudaStream_t st) {
+  if (n <= 0) return WK_OK;
+  int64_t blocks = (n / 8 + 255) / 256;
+  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(dv->sms) * 16));
+  convert_kernel<TI, TO><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const TI*>(in), static_cast<TO*>(out),
+                                                                    n);
+  return launch_status();
 }
 
 // ------------------------------------------------------------------- SIMT
@@ -336,20 +385,23 @@ struct wk_stack {
   int device = 0;
   wk_stack_config cfg{};
   std::vector<int32_t> dims;  // h_0 .. h_m
-  std::vector<wk_layer_weights> lw;
-  std::vector<std::vector<const void*>> W;
-  std::vector<std::vector<const float*>> b;
   float eps = 1e-5f;
-  bool bf = true;  // bf16 storage
+  wk_dtype io = WK_BF16;      // caller's storage type of X, out and the weights
+  wk_dtype op = WK_F16;       // operand / intermediate type (WK_F32 for fp32 stacks)
   int64_t maxb = 0;
   const DevInfo* dv = nullptr;
-  // workspace
+  // operand weights per layer (the caller's, or converted copies in wcopy)
+  std::vector<const void*> Y, WL;
+  std::vector<std::vector<const void*>> W;
+  std::vector<std::vector<const float*>> b;
+  std::vector<const float*> g1, b1, g2, b2;
+  uint8_t* wcopy = nullptr;
+  // workspace (operand type)
   uint8_t* ws = nullptr;
   void* A0 = nullptr;
   void* H[2] = {nullptr, nullptr};
-  void* cat = nullptr;  // fp32 (bf16 stacks) or fp32 (fp32 stacks)
-  void* X16[2] = {nullptr, nullptr};  // operand copies of the layer outputs (fp32 stacks: same as X32)
-  float* X32[2] = {nullptr, nullptr};
+  void* cat = nullptr;
+  void* Xs[2] = {nullptr, nullptr};  // layer outputs; Xs[1] also takes a converted input
   unsigned* status = nullptr;
   // TMA descriptors of the tensor-core path
   bool tc_mlp = false, tc_lcb = false;
@@ -412,6 +464,7 @@ void free_stack(wk_stack* h) {
   cudaDeviceSynchronize();
   cudaGetLastError();
   if (h->ws) cudaFree(h->ws);
+  if (h->wcopy) cudaFree(h->wcopy);
   if (h->stage) cudaFree(h->stage);
   if (h->s_in) cudaStreamDestroy(h->s_in);
   if (h->s_out) cudaStreamDestroy(h->s_out);
@@ -430,16 +483,208 @@ wk_status validate_cfg(const wk_stack_config* c) {
       c->max_batch < 1)
     return WK_ERR_INVALID_ARG;
   if (c->mlp_num_linear > 1 && !c->mlp_hidden) return WK_ERR_INVALID_ARG;
-  if (c->dtype != WK_F32 && c->dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (c->dtype != WK_F32 && c->dtype != WK_BF16 && c->dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  if (c->operand_dtype != WK_F32 && c->operand_dtype != WK_BF16 && c->operand_dtype != WK_F16)
+    return WK_ERR_UNSUPPORTED;
   if (c->n_f + c->n_l != c->n) return WK_ERR_UNSUPPORTED;
-  if (c->dtype == WK_BF16 ? (c->d % 8 != 0) : (c->d % 8 != 0)) return WK_ERR_UNSUPPORTED;
-  if (!res_ln_d_ok(c->d)) return WK_ERR_UNSUPPORTED;
+  if (c->d % 8 != 0 || !res_ln_d_ok(c->d)) return WK_ERR_UNSUPPORTED;
   for (int j = 0; j + 1 < c->mlp_num_linear; ++j)
     if (c->mlp_hidden[j] < 1 || c->mlp_hidden[j] % 8 != 0) return WK_ERR_UNSUPPORTED;
   if ((static_cast<int64_t>(c->n) * c->k) % 8 != 0) return WK_ERR_UNSUPPORTED;
-  if (!fm_supported(c->n, c->d, c->k, c->dtype)) return WK_ERR_UNSUPPORTED;
+  if (!fm_supported(c->n, c->d, c->k, c->dtype != WK_F32)) return WK_ERR_UNSUPPORTED;
   if (c->ln_eps < 0.f) return WK_ERR_INVALID_ARG;
   return WK_OK;
+}
+
+// Builds the tensor-core descriptors of a 16-bit stack (operand type T).
+template <typename T>
+wk_status build_maps(wk_stack* h) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int L = c.num_layers, m = c.mlp_num_linear, n = c.n, d = c.d;
+  const int64_t B = h->maxb;
+  const uint64_t nd = static_cast<uint64_t>(n) * d;
+  h->tc_mlp = true;
+  for (int j = 0; j < m; ++j) {
+    const int64_t ldc = (j == m - 1) ? static_cast<int64_t>(nd) : h->dims[j + 1];
+    if (!mlp_tc_ok(B, h->dims[j], h->dims[j + 1], ldc)) h->tc_mlp = false;
+  }
+  h->tc_lcb = lcb_tc_ok(B, n, d);
+  if (h->tc_mlp) {
+    h->mlp_maps.assign(L, std::vector<GemmMaps>(m));
+    for (int l = 0; l < L; ++l)
+      for (int j = 0; j < m; ++j) {
+        GemmMaps& mp = h->mlp_maps[l][j];
+        const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+        const bool last = j == m - 1;
+        const bool ok = map_kmajor<T>(dv, &mp.A, in, h->dims[j], B, GEMM_BM) &&
+                        map_kmajor<T>(dv, &mp.B, h->W[l][j], h->dims[j], h->dims[j + 1], GEMM_BN) &&
+                        (last ? map_out<T>(dv, &mp.C, h->cat, h->dims[j + 1], B, nd)
+                              : map_out<T>(dv, &mp.C, h->H[j % 2], h->dims[j + 1], B, h->dims[j + 1]));
+        if (!ok) return WK_ERR_UNSUPPORTED;
+      }
+  }
+  if (h->tc_lcb) {
+    h->lcbA.resize(L);
+    bool ok = true;
+    for (int l = 0; l < L; ++l) ok = ok && map_kmajor<T>(dv, &h->lcbA[l], h->WL[l], n, c.n_l, GEMM_BM);
+    ok = ok && map_lcb_x<T>(dv, &h->lcbB_ws[0], h->Xs[0], n, d, B) && map_lcb_x<T>(dv, &h->lcbB_ws[1], h->Xs[1], n, d, B) &&
+         map_lcb_out<T>(dv, &h->lcbC, h->cat, n, d, c.n_f, c.n_l, B);
+    if (!ok) return WK_ERR_UNSUPPORTED;
+  }
+  return WK_OK;
+}
+
+// The forward of a 16-bit stack with operand type T and caller type IO.
+template <typename T, typename IO>
+wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaStream_t st) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers;
+  const int64_t rows = batch * n;
+  const size_t nd = static_cast<size_t>(n) * d;
+  wk_status s = WK_OK;
+  const void* x0 = X;
+  CUtensorMap lcb_x0;
+  if (sizeof(IO) != sizeof(T) || Half16<IO>::kBF16 != Half16<T>::kBF16) {
+    s = run_convert<IO, T>(dv, X, h->Xs[1], rows * d, st);  // the input in the operand type
+    if (s != WK_OK) return s;
+    x0 = h->Xs[1];
+    lcb_x0 = h->lcbB_ws[1];
+  } else if (h->tc_lcb && !map_lcb_x<T>(dv, &lcb_x0, X, n, d, batch)) {
+    return WK_ERR_CUDA;
+  }
+  for (int l = 0; l < L && s == WK_OK; ++l) {
+    const bool last = l == L - 1;
+    const T* xin = static_cast<const T*>(l == 0 ? x0 : h->Xs[(l - 1) % 2]);
+    {  // 1. FM + LN
+      ProfScope ps(h, WK_KERNEL_FM_LN, st);
+      s = run_fm16<T>(dv, xin, static_cast<const T*>(h->Y[l]), h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, n, d,
+                      k, h->eps, h->status, st);
+    }
+    for (int j = 0; j < m && s == WK_OK; ++j) {  // 2. MLP
+      ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+      const bool lastj = j == m - 1;
+      void* o = lastj ? h->cat : h->H[j % 2];
+      const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
+      const int relu = lastj ? 0 : 1;
+      if (h->tc_mlp)
+        s = run_gemm_tc<MODE_MLP, T, T>(dv, h->mlp_maps[l][j],
+                                         mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
+      else
+        s = run_gemm_simt<T, T>(static_cast<const T*>(in), static_cast<const T*>(h->W[l][j]), h->b[l][j],
+                                static_cast<T*>(o), batch, h->dims[j], h->dims[j + 1], ldc, relu, st);
+    }
+    if (s != WK_OK) break;
+    {  // 3. LCB
+      ProfScope ps(h, WK_KERNEL_LCB, st);
+      if (h->tc_lcb) {
+        GemmMaps mp;
+        mp.A = h->lcbA[l];
+        mp.B = (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2];
+        mp.C = h->lcbC;
+        s = run_gemm_tc<MODE_LCB, T, T>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
+      } else {
+        s = run_lcb_simt<T, T>(static_cast<const T*>(h->WL[l]), xin, static_cast<T*>(h->cat), batch, n, d, c.n_f,
+                               c.n_l, st);
+      }
+    }
+    if (s != WK_OK) break;
+    {  // 4. residual + LN
+      ProfScope ps(h, WK_KERNEL_RES_LN, st);
+      const T* cat = static_cast<const T*>(h->cat);
+      if (last)
+        s = run_res_ln<T, T, IO>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<IO*>(out), rows, d, h->eps, st);
+      else
+        s = run_res_ln<T, T, T>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<T*>(h->Xs[l % 2]), rows, d, h->eps, st);
+    }
+  }
+  return s;
+}
+
+wk_status forward32(wk_stack* h, const float* X, float* out, int64_t batch, cudaStream_t st) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers;
+  const int64_t rows = batch * n;
+  const size_t nd = static_cast<size_t>(n) * d;
+  wk_status s = WK_OK;
+  for (int l = 0; l < L && s == WK_OK; ++l) {
+    const bool last = l == L - 1;
+    const float* xin = (l == 0) ? X : static_cast<const float*>(h->Xs[(l - 1) % 2]);
+    {
+      ProfScope ps(h, WK_KERNEL_FM_LN, st);
+      s = run_fm_simt<float>(dv, xin, static_cast<const float*>(h->Y[l]), h->g1[l], h->b1[l],
+                             static_cast<float*>(h->A0), batch, n, d, k, h->eps, st);
+    }
+    for (int j = 0; j < m && s == WK_OK; ++j) {
+      ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+      const bool lastj = j == m - 1;
+      void* o = lastj ? h->cat : h->H[j % 2];
+      const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
+      s = run_gemm_simt<float, float>(static_cast<const float*>(in), static_cast<const float*>(h->W[l][j]), h->b[l][j],
+                                      static_cast<float*>(o), batch, h->dims[j], h->dims[j + 1], ldc, lastj ? 0 : 1, st);
+    }
+    if (s != WK_OK) break;
+    {
+      ProfScope ps(h, WK_KERNEL_LCB, st);
+      s = run_lcb_simt<float, float>(static_cast<const float*>(h->WL[l]), xin, static_cast<float*>(h->cat), batch, n,
+                                     d, c.n_f, c.n_l, st);
+    }
+    if (s != WK_OK) break;
+    {
+      ProfScope ps(h, WK_KERNEL_RES_LN, st);
+      float* o = last ? out : static_cast<float*>(h->Xs[l % 2]);
+      s = run_res_ln<float, float, float>(dv, static_cast<const float*>(h->cat), xin, h->g2[l], h->b2[l], o, rows, d,
+                                          h->eps, st);
+    }
+  }
+  return s;
+}
+
+wk_status read_status_word(unsigned* word, cudaStream_t st) {
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  unsigned v = 0;
+  if (cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  if (v) {
+    const unsigned zero = 0;
+    cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice);
+  }
+  if (v & kFlagTimeout) return WK_ERR_TIMEOUT;
+  if (v) return WK_ERR_DEVICE;
+  return WK_OK;
+}
+
+template <typename T>
+wk_status mlp_linear16(const DevInfo* dv, const void* A, const void* W, const float* bias, void* C, int64_t M,
+                              int K, int N, int64_t ldc, int relu, cudaStream_t st) {
+  if (!mlp_tc_ok(M, K, N, ldc)) return WK_ERR_UNSUPPORTED;
+  GemmMaps mp;
+  if (!map_kmajor<T>(dv, &mp.A, A, K, M, GEMM_BM) || !map_kmajor<T>(dv, &mp.B, W, K, N, GEMM_BN) ||
+      !map_out<T>(dv, &mp.C, C, N, M, ldc))
+    return WK_ERR_UNSUPPORTED;
+  return run_gemm_tc<MODE_MLP, T, T>(dv, mp, mlp_params(M, K, N, bias, relu ? 1 : 0, dv->standalone_status), st);
+}
+
+template <typename T>
+wk_status lcb16(const DevInfo* dv, const void* W_L, const void* X, void* concat, int64_t batch, int n, int d,
+                       int n_f, int n_l, cudaStream_t st) {
+  if (!lcb_tc_ok(batch, n, d))
+    return run_lcb_simt<T, T>(static_cast<const T*>(W_L), static_cast<const T*>(X), static_cast<T*>(concat), batch, n,
+                              d, n_f, n_l, st);
+  GemmMaps mp;
+  if (!map_kmajor<T>(dv, &mp.A, W_L, n, n_l, GEMM_BM) || !map_lcb_x<T>(dv, &mp.B, X, n, d, batch) ||
+      !map_lcb_out<T>(dv, &mp.C, concat, n_f + n_l, d, n_f, n_l, batch))
+    return WK_ERR_UNSUPPORTED;
+  return run_gemm_tc<MODE_LCB, T, T>(dv, mp, lcb_params(batch, n, d, n_l, dv->standalone_status), st);
 }
 
 }  // namespace
@@ -470,7 +715,6 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   dims.push_back(n * k);
   for (int j = 0; j + 1 < m; ++j) dims.push_back(cfg->mlp_hidden[j]);
   dims.push_back(cfg->n_f * d);
-  // weight pointers
   for (int l = 0; l < L; ++l) {
     const wk_layer_weights& w = weights[l];
     if (!w.Y || !w.W || !w.fmb_ln_gamma || !w.fmb_ln_beta || !w.W_L || !w.out_ln_gamma || !w.out_ln_beta)
@@ -489,30 +733,68 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
 
   wk_stack* h = new (std::nothrow) wk_stack();
   if (!h) return WK_ERR_OOM;
-  cudaGetDevice(&h->device);
+  h->device = dv->id;
   h->cfg = *cfg;
   h->cfg.mlp_hidden = nullptr;
   h->dims = dims;
   h->eps = cfg->ln_eps > 0.f ? cfg->ln_eps : 1e-5f;
-  h->bf = cfg->dtype == WK_BF16;
+  h->io = cfg->dtype;
+  h->op = cfg->dtype == WK_F32 ? WK_F32 : (cfg->operand_dtype == WK_BF16 ? WK_BF16 : WK_F16);
   h->maxb = cfg->max_batch;
   h->dv = dv;
-  h->lw.assign(weights, weights + L);
   h->W.resize(L);
   h->b.resize(L);
   for (int l = 0; l < L; ++l) {
+    const wk_layer_weights& w = weights[l];
+    h->Y.push_back(w.Y);
+    h->WL.push_back(w.W_L);
     for (int j = 0; j < m; ++j) {
-      h->W[l].push_back(weights[l].W[j]);
-      h->b[l].push_back(weights[l].b ? weights[l].b[j] : nullptr);
+      h->W[l].push_back(w.W[j]);
+      h->b[l].push_back(w.b ? w.b[j] : nullptr);
+    }
+    h->g1.push_back(w.fmb_ln_gamma);
+    h->b1.push_back(w.fmb_ln_beta);
+    h->g2.push_back(w.out_ln_gamma);
+    h->b2.push_back(w.out_ln_beta);
+  }
+
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  // weights converted to the operand type once (bf16 stacks computing with fp16 operands, or the reverse)
+  if (h->io != h->op) {
+    size_t per_layer = up(static_cast<size_t>(n) * k * 2) + up(static_cast<size_t>(cfg->n_l) * n * 2);
+    for (int j = 0; j < m; ++j) per_layer += up(static_cast<size_t>(dims[j]) * dims[j + 1] * 2);
+    if (cudaMalloc(&h->wcopy, per_layer * L) != cudaSuccess) {
+      cudaGetLastError();
+      delete h;
+      return WK_ERR_OOM;
+    }
+    uint8_t* p = h->wcopy;
+    auto conv = [&](const void* src, int64_t count) -> const void* {
+      uint8_t* dst = p;
+      p += up(static_cast<size_t>(count) * 2);
+      wk_status cs = h->io == WK_BF16 ? run_convert<bf16, f16>(dv, src, dst, count, nullptr)
+                                      : run_convert<f16, bf16>(dv, src, dst, count, nullptr);
+      if (cs != WK_OK) st = cs;
+      return dst;
+    };
+    for (int l = 0; l < L; ++l) {
+      h->Y[l] = conv(h->Y[l], static_cast<int64_t>(n) * k);
+      h->WL[l] = conv(h->WL[l], static_cast<int64_t>(cfg->n_l) * n);
+      for (int j = 0; j < m; ++j) h->W[l][j] = conv(h->W[l][j], static_cast<int64_t>(dims[j]) * dims[j + 1]);
+    }
+    if (st == WK_OK && cudaDeviceSynchronize() != cudaSuccess) st = WK_ERR_CUDA;
+    if (st != WK_OK) {
+      cudaGetLastError();
+      free_stack(h);
+      return st;
     }
   }
 
   // workspace
   const int64_t B = h->maxb;
-  const size_t es = h->bf ? 2 : 4;
+  const size_t es = dtype_bytes(h->op);
   int32_t hmax = 8;
   for (int j = 1; j < m; ++j) hmax = std::max(hmax, dims[j]);
-  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
   const size_t nd = static_cast<size_t>(n) * d;
   size_t off = 0;
   const size_t o_a0 = off;
@@ -522,78 +804,37 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   const size_t o_h1 = off;
   off += up(B * static_cast<size_t>(hmax) * es);
   const size_t o_cat = off;
-  off += up(B * nd * 4);
-  const size_t o_x32_0 = off;
-  off += up(B * nd * 4);
-  const size_t o_x32_1 = off;
-  off += up(B * nd * 4);
-  size_t o_x16_0 = 0, o_x16_1 = 0;
-  if (h->bf) {
-    o_x16_0 = off;
-    off += up(B * nd * 2);
-    o_x16_1 = off;
-    off += up(B * nd * 2);
-  }
+  off += up(B * nd * es);
+  const size_t o_x0 = off;
+  off += up(B * nd * es);
+  const size_t o_x1 = off;
+  off += up(B * nd * es);
   const size_t o_status = off;
   off += 256;
   if (cudaMalloc(&h->ws, off) != cudaSuccess) {
     cudaGetLastError();
-    delete h;
+    free_stack(h);
     return WK_ERR_OOM;
   }
   h->A0 = h->ws + o_a0;
   h->H[0] = h->ws + o_h0;
   h->H[1] = h->ws + o_h1;
   h->cat = h->ws + o_cat;
-  h->X32[0] = reinterpret_cast<float*>(h->ws + o_x32_0);
-  h->X32[1] = reinterpret_cast<float*>(h->ws + o_x32_1);
-  h->X16[0] = h->bf ? static_cast<void*>(h->ws + o_x16_0) : static_cast<void*>(h->X32[0]);
-  h->X16[1] = h->bf ? static_cast<void*>(h->ws + o_x16_1) : static_cast<void*>(h->X32[1]);
+  h->Xs[0] = h->ws + o_x0;
+  h->Xs[1] = h->ws + o_x1;
   h->status = reinterpret_cast<unsigned*>(h->ws + o_status);
   if (cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess) {
     cudaGetLastError();
     free_stack(h);
     return WK_ERR_CUDA;
   }
-
-  // tensor-core path descriptors
-  if (h->bf) {
-    h->tc_mlp = true;
-    for (int j = 0; j < m; ++j) {
-      const int64_t ldc = (j == m - 1) ? static_cast<int64_t>(nd) : dims[j + 1];
-      if (!mlp_tc_ok(B, dims[j], dims[j + 1], ldc)) h->tc_mlp = false;
-    }
-    h->tc_lcb = lcb_tc_ok(B, n, d);
-    if (h->tc_mlp) {
-      h->mlp_maps.resize(L);
-      for (int l = 0; l < L; ++l) {
-        h->mlp_maps[l].resize(m);
-        for (int j = 0; j < m; ++j) {
-          GemmMaps& mp = h->mlp_maps[l][j];
-          const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
-          const bool last = j == m - 1;
-          bool ok = map_kmajor(dv, &mp.A, in, dims[j], B, GEMM_BM) &&
-                    map_kmajor(dv, &mp.B, h->W[l][j], dims[j], dims[j + 1], GEMM_BN) &&
-                    (last ? map_out(dv, &mp.C, h->cat, true, dims[j + 1], B, nd)
-                          : map_out(dv, &mp.C, h->H[j % 2], false, dims[j + 1], B, dims[j + 1]));
-          if (!ok) {
-            free_stack(h);
-            return WK_ERR_UNSUPPORTED;
-          }
-        }
-      }
-    }
-    if (h->tc_lcb) {
-      h->lcbA.resize(L);
-      bool ok = true;
-      for (int l = 0; l < L; ++l) ok = ok && map_kmajor(dv, &h->lcbA[l], h->lw[l].W_L, n, cfg->n_l, GEMM_BM);
-      ok = ok && map_lcb_x(dv, &h->lcbB_ws[0], h->X16[0], n, d, B) && map_lcb_x(dv, &h->lcbB_ws[1], h->X16[1], n, d, B) &&
-           map_lcb_out(dv, &h->lcbC, h->cat, true, n, d, cfg->n_f, cfg->n_l, B);
-      if (!ok) {
-        free_stack(h);
-        return WK_ERR_UNSUPPORTED;
-      }
-    }
+  if (h->op == WK_F16)
+    st = build_maps<f16>(h);
+  else if (h->op == WK_BF16)
+    st = build_maps<bf16>(h);
+  if (st != WK_OK) {
+    free_stack(h);
+    return st;
   }
   *out = h;
   return WK_OK;
@@ -603,10 +844,7 @@ wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t batch,
   if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
   if (batch == 0) return WK_OK;
   if (!X || !out || !al16(X) || !al16(out)) return WK_ERR_INVALID_ARG;
-  const wk_stack_config& c = h->cfg;
-  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers;
-  const size_t es = h->bf ? 2 : 4;
-  const size_t bytes = static_cast<size_t>(batch) * n * d * es;
+  const size_t bytes = static_cast<size_t>(batch) * h->cfg.n * h->cfg.d * dtype_bytes(h->io);
   const uint8_t* xa = static_cast<const uint8_t*>(X);
   const uint8_t* oa = static_cast<const uint8_t*>(out);
   if (xa < oa + bytes && oa < xa + bytes) return WK_ERR_INVALID_ARG;
@@ -616,102 +854,17 @@ wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t batch,
     return WK_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const DevInfo* dv = h->dv;
-  const int64_t rows = batch * n;
-  const size_t nd = static_cast<size_t>(n) * d;
-  wk_status s = WK_OK;
-
-  CUtensorMap lcbB_user;
-  if (h->bf && h->tc_lcb && !map_lcb_x(dv, &lcbB_user, X, n, d, batch)) return WK_ERR_CUDA;
-
-  for (int l = 0; l < L && s == WK_OK; ++l) {
-    const wk_layer_weights& w = h->lw[l];
-    const bool last = l == L - 1;
-    const void* xin = (l == 0) ? X : h->X16[(l - 1) % 2];
-    // 1. FM + LN
-    {
-      ProfScope ps(h, WK_KERNEL_FM_LN, st);
-      if (h->bf)
-        s = run_fm_bf16(dv, static_cast<const bf16*>(xin), static_cast<const bf16*>(w.Y), w.fmb_ln_gamma,
-                        w.fmb_ln_beta, static_cast<bf16*>(h->A0), batch, n, d, k, h->eps, h->status, st);
-      else
-        s = run_fm_simt<float>(dv, static_cast<const float*>(xin), static_cast<const float*>(w.Y), w.fmb_ln_gamma,
-                               w.fmb_ln_beta, static_cast<float*>(h->A0), batch, n, d, k, h->eps, st);
-    }
-    // 2. MLP
-    for (int j = 0; j < m && s == WK_OK; ++j) {
-      ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
-      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
-      const bool lastj = j == m - 1;
-      void* o = lastj ? h->cat : h->H[j % 2];
-      const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
-      const int relu = lastj ? 0 : 1;
-      if (h->bf && h->tc_mlp) {
-        GemmParams p = mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status);
-        s = lastj ? run_gemm_tc<MODE_MLP, float>(dv, h->mlp_maps[l][j], p, st)
-                  : run_gemm_tc<MODE_MLP, bf16>(dv, h->mlp_maps[l][j], p, st);
-      } else if (h->bf) {
-        s = lastj ? run_gemm_simt<bf16, float>(static_cast<const bf16*>(in), static_cast<const bf16*>(h->W[l][j]),
-                                               h->b[l][j], static_cast<float*>(o), batch, h->dims[j],
-                                               h->dims[j + 1], ldc, relu, st)
-                  : run_gemm_simt<bf16, bf16>(static_cast<const bf16*>(in), static_cast<const bf16*>(h->W[l][j]),
-                                              h->b[l][j], static_cast<bf16*>(o), batch, h->dims[j], h->dims[j + 1],
-                                              ldc, relu, st);
-      } else {
-        s = run_gemm_simt<float, float>(static_cast<const float*>(in), static_cast<const float*>(h->W[l][j]),
-                                        h->b[l][j], static_cast<float*>(o), batch, h->dims[j], h->dims[j + 1], ldc,
-                                        relu, st);
-      }
-    }
-    if (s != WK_OK) break;
-    // 3. LCB
-    {
-      ProfScope ps(h, WK_KERNEL_LCB, st);
-      if (h->bf && h->tc_lcb) {
-        GemmMaps mp;
-        mp.A = h->lcbA[l];
-        mp.B = (l == 0) ? lcbB_user : h->lcbB_ws[(l - 1) % 2];
-        mp.C = h->lcbC;
-        s = run_gemm_tc<MODE_LCB, float>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
-      } else if (h->bf) {
-        s = run_lcb_simt<bf16, float>(static_cast<const bf16*>(w.W_L), static_cast<const bf16*>(xin),
-                                      static_cast<float*>(h->cat), batch, n, d, c.n_f, c.n_l, st);
-      } else {
-        s = run_lcb_simt<float, float>(static_cast<const float*>(w.W_L), static_cast<const float*>(xin),
-                                       static_cast<float*>(h->cat), batch, n, d, c.n_f, c.n_l, st);
-      }
-    }
-    if (s != WK_OK) break;
-    // 4. residual + LN
-    {
-      ProfScope ps(h, WK_KERNEL_RES_LN, st);
-      const float* cat = static_cast<const float*>(h->cat);
-      if (h->bf) {
-        bf16* o16 = last ? static_cast<bf16*>(out) : static_cast<bf16*>(h->X16[l % 2]);
-        float* o32 = last ? nullptr : h->X32[l % 2];
-        if (l == 0)
-          s = run_res_ln<float, bf16, bf16>(dv, cat, static_cast<const bf16*>(X), w.out_ln_gamma, w.out_ln_beta, o16,
-                                            o32, rows, d, h->eps, st);
-        else
-          s = run_res_ln<float, float, bf16>(dv, cat, h->X32[(l - 1) % 2], w.out_ln_gamma, w.out_ln_beta, o16, o32,
-                                             rows, d, h->eps, st);
-      } else {
-        float* o = last ? static_cast<float*>(out) : h->X32[l % 2];
-        const float* resid = (l == 0) ? static_cast<const float*>(X) : h->X32[(l - 1) % 2];
-        s = run_res_ln<float, float, float>(dv, cat, resid, w.out_ln_gamma, w.out_ln_beta, o, nullptr, rows, d,
-                                            h->eps, st);
-      }
-    }
-  }
-  return s;
+  if (h->op == WK_F32) return forward32(h, static_cast<const float*>(X), static_cast<float*>(out), batch, st);
+  if (h->op == WK_F16)
+    return h->io == WK_BF16 ? forward16<f16, bf16>(h, X, out, batch, st) : forward16<f16, f16>(h, X, out, batch, st);
+  return h->io == WK_BF16 ? forward16<bf16, bf16>(h, X, out, batch, st) : forward16<bf16, f16>(h, X, out, batch, st);
 }
 
 wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host, int64_t batch, wk_stream_t stream) {
   if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
   if (batch == 0) return WK_OK;
   if (!X_host || !out_host) return WK_ERR_INVALID_ARG;
-  const size_t es = h->bf ? 2 : 4;
-  const size_t ex_bytes = static_cast<size_t>(h->cfg.n) * h->cfg.d * es;
+  const size_t ex_bytes = static_cast<size_t>(h->cfg.n) * h->cfg.d * dtype_bytes(h->io);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // Chunks of at least 1024 examples (or the whole batch): large enough that the
   // GEMMs stay efficient, small enough that copies overlap the compute.
@@ -784,25 +937,6 @@ wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host,
   return s;
 }
 
-static wk_status read_status_word(unsigned* word, cudaStream_t st) {
-  if (cudaStreamSynchronize(st) != cudaSuccess) {
-    cudaGetLastError();
-    return WK_ERR_CUDA;
-  }
-  unsigned v = 0;
-  if (cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) {
-    cudaGetLastError();
-    return WK_ERR_CUDA;
-  }
-  if (v) {
-    const unsigned zero = 0;
-    cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice);
-  }
-  if (v & kFlagTimeout) return WK_ERR_TIMEOUT;
-  if (v) return WK_ERR_DEVICE;
-  return WK_OK;
-}
-
 wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream) {
   if (!h) return WK_ERR_INVALID_ARG;
   return read_status_word(h->status, reinterpret_cast<cudaStream_t>(stream));
@@ -847,16 +981,19 @@ wk_status wk_fm_ln(const void* X, const void* Y, const float* gamma, const float
   if (batch == 0) return WK_OK;
   if (!X || !Y || !gamma || !beta || !A0 || !al16(X) || !al16(Y) || !al16(A0) || !al16(gamma) || !al16(beta))
     return WK_ERR_INVALID_ARG;
-  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
-  if (d % 8 != 0 || k % 2 != 0 || !fm_supported(n, d, k, dtype)) return WK_ERR_UNSUPPORTED;
+  if (dtype != WK_F32 && dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || k % 2 != 0 || !fm_supported(n, d, k, dtype != WK_F32)) return WK_ERR_UNSUPPORTED;
   DevInfo* dv = nullptr;
   wk_status s = dev_info(&dv);
   if (s != WK_OK) return s;
   const float e = eps > 0.f ? eps : 1e-5f;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == WK_BF16)
-    return run_fm_bf16(dv, static_cast<const bf16*>(X), static_cast<const bf16*>(Y), gamma, beta,
-                       static_cast<bf16*>(A0), batch, n, d, k, e, dv->standalone_status, st);
+    return run_fm16<bf16>(dv, static_cast<const bf16*>(X), static_cast<const bf16*>(Y), gamma, beta,
+                          static_cast<bf16*>(A0), batch, n, d, k, e, dv->standalone_status, st);
+  if (dtype == WK_F16)
+    return run_fm16<f16>(dv, static_cast<const f16*>(X), static_cast<const f16*>(Y), gamma, beta,
+                         static_cast<f16*>(A0), batch, n, d, k, e, dv->standalone_status, st);
   return run_fm_simt<float>(dv, static_cast<const float*>(X), static_cast<const float*>(Y), gamma, beta,
                             static_cast<float*>(A0), batch, n, d, k, e, st);
 }
@@ -866,19 +1003,13 @@ wk_status wk_mlp_linear(const void* A, const void* W, const float* bias, void* C
   if (M < 0 || K < 1 || N < 1 || ldc < N) return WK_ERR_INVALID_ARG;
   if (M == 0) return WK_OK;
   if (!A || !W || !C || !al16(A) || !al16(W) || !al16(C) || (bias && !al16(bias))) return WK_ERR_INVALID_ARG;
-  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (dtype != WK_F32 && dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
   DevInfo* dv = nullptr;
   wk_status s = dev_info(&dv);
   if (s != WK_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == WK_BF16) {
-    if (!mlp_tc_ok(M, K, N, ldc)) return WK_ERR_UNSUPPORTED;
-    GemmMaps mp;
-    if (!map_kmajor(dv, &mp.A, A, K, M, GEMM_BM) || !map_kmajor(dv, &mp.B, W, K, N, GEMM_BN) ||
-        !map_out(dv, &mp.C, C, false, N, M, ldc))
-      return WK_ERR_UNSUPPORTED;
-    return run_gemm_tc<MODE_MLP, bf16>(dv, mp, mlp_params(M, K, N, bias, relu ? 1 : 0, dv->standalone_status), st);
-  }
+  if (dtype == WK_BF16) return mlp_linear16<bf16>(dv, A, W, bias, C, M, K, N, ldc, relu, st);
+  if (dtype == WK_F16) return mlp_linear16<f16>(dv, A, W, bias, C, M, K, N, ldc, relu, st);
   return run_gemm_simt<float, float>(static_cast<const float*>(A), static_cast<const float*>(W), bias,
                                      static_cast<float*>(C), M, K, N, ldc, relu ? 1 : 0, st);
 }
@@ -888,22 +1019,13 @@ wk_status wk_lcb(const void* W_L, const void* X, void* concat, int64_t batch, in
   if (batch < 0 || n < 1 || d < 1 || n_f < 0 || n_l < 1) return WK_ERR_INVALID_ARG;
   if (batch == 0) return WK_OK;
   if (!W_L || !X || !concat || !al16(W_L) || !al16(X) || !al16(concat)) return WK_ERR_INVALID_ARG;
-  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (dtype != WK_F32 && dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
   DevInfo* dv = nullptr;
   wk_status s = dev_info(&dv);
   if (s != WK_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == WK_BF16) {
-    if (!lcb_tc_ok(batch, n, d)) {
-      return run_lcb_simt<bf16, bf16>(static_cast<const bf16*>(W_L), static_cast<const bf16*>(X),
-                                      static_cast<bf16*>(concat), batch, n, d, n_f, n_l, st);
-    }
-    GemmMaps mp;
-    if (!map_kmajor(dv, &mp.A, W_L, n, n_l, GEMM_BM) || !map_lcb_x(dv, &mp.B, X, n, d, batch) ||
-        !map_lcb_out(dv, &mp.C, concat, false, n_f + n_l, d, n_f, n_l, batch))
-      return WK_ERR_UNSUPPORTED;
-    return run_gemm_tc<MODE_LCB, bf16>(dv, mp, lcb_params(batch, n, d, n_l, dv->standalone_status), st);
-  }
+  if (dtype == WK_BF16) return lcb16<bf16>(dv, W_L, X, concat, batch, n, d, n_f, n_l, st);
+  if (dtype == WK_F16) return lcb16<f16>(dv, W_L, X, concat, batch, n, d, n_f, n_l, st);
   return run_lcb_simt<float, float>(static_cast<const float*>(W_L), static_cast<const float*>(X),
                                     static_cast<float*>(concat), batch, n, d, n_f, n_l, st);
 }
@@ -915,7 +1037,7 @@ wk_status wk_res_ln(const void* concat, const void* X, const float* gamma, const
   if (!concat || !X || !gamma || !beta || !out || !al16(concat) || !al16(X) || !al16(out) || !al16(gamma) ||
       !al16(beta))
     return WK_ERR_INVALID_ARG;
-  if (dtype != WK_F32 && dtype != WK_BF16) return WK_ERR_UNSUPPORTED;
+  if (dtype != WK_F32 && dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
   if (!res_ln_d_ok(d)) return WK_ERR_UNSUPPORTED;
   DevInfo* dv = nullptr;
   wk_status s = dev_info(&dv);
@@ -924,9 +1046,12 @@ wk_status wk_res_ln(const void* concat, const void* X, const float* gamma, const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == WK_BF16)
     return run_res_ln<bf16, bf16, bf16>(dv, static_cast<const bf16*>(concat), static_cast<const bf16*>(X), gamma,
-                                        beta, static_cast<bf16*>(out), nullptr, rows, d, e, st);
+                                        beta, static_cast<bf16*>(out), rows, d, e, st);
+  if (dtype == WK_F16)
+    return run_res_ln<f16, f16, f16>(dv, static_cast<const f16*>(concat), static_cast<const f16*>(X), gamma, beta,
+                                     static_cast<f16*>(out), rows, d, e, st);
   return run_res_ln<float, float, float>(dv, static_cast<const float*>(concat), static_cast<const float*>(X), gamma,
-                                         beta, static_cast<float*>(out), nullptr, rows, d, e, st);
+                                         beta, static_cast<float*>(out), rows, d, e, st);
 }
 
 wk_status wk_device_status(wk_stream_t stream) {

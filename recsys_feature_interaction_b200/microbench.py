@@ -1,0 +1,103 @@
+"""Times one step of the Wukong layer alone through its stand-alone C-ABI entry point.
+
+    python -m recsys_feature_interaction_b200.microbench --kernel fm_ln|mlp_gemm|lcb|res_ln
+        [--workload c4_bf16] [--batch B] [--iters K] [--dtype f16|bf16] [--layer-linear j]
+
+Inputs are synthetic (the seeded generator), on the device, in the workload's
+shapes. Prints one JSON line with the mean CUDA-event time per launch and the
+algorithmic FLOPs / bytes of one launch. Small --iters values make it a convenient
+target for a profiler capture of a single kernel.
+"""
+import argparse
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", required=True, choices=["fm_ln", "mlp_gemm", "lcb", "res_ln"])
+    ap.add_argument("--workload", default="c4_bf16")
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"])
+    ap.add_argument("--layer-linear", type=int, default=0, help="which MLP Linear (mlp_gemm)")
+    args = ap.parse_args()
+
+    import torch
+
+    import recsys_feature_interaction_b200 as wk
+    from recsys_feature_interaction_b200 import build
+    from synth import configs as C
+
+    build.build()
+    cfg = C.CONFIGS[args.workload]
+    B = args.batch or cfg["batch"]
+    n, d, k, n_f, n_l = cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], cfg["n_l"]
+    tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    w = C.make_layer_dev(cfg, 0)
+    dev = torch.device("cuda")
+    X = C.make_x_dev(cfg, B).to(tdt)
+    es = 2
+    if args.kernel == "fm_ln":
+        Y = w["Y"].to(tdt)
+        A0 = torch.empty((B, n * k), dtype=tdt, device=dev)
+
+        def run():
+            wk.wk_fm_ln(X, Y, w["fmb_gamma"], w["fmb_beta"], A0, B, n, d, k, args.dtype)
+        flops = 4 * n * d * k * B
+        bytes_ = (n * d + n * k) * es * B
+    elif args.kernel == "mlp_gemm":
+        dims = C.mlp_dims(cfg)
+        j = args.layer_linear
+        Kd, Nd = dims[j], dims[j + 1]
+        A = torch.randn((B, Kd), device=dev).to(tdt)
+        W = w["W%d" % j].to(tdt)
+        Cm = torch.empty((B, Nd), dtype=tdt, device=dev)
+
+        def run():
+            wk.wk_mlp_linear(A, W, w["b%d" % j], Cm, B, Kd, Nd, Nd, j < len(dims) - 2, args.dtype)
+        flops = 2 * B * Kd * Nd
+        bytes_ = (B * Kd + Nd * Kd + B * Nd) * es
+    elif args.kernel == "lcb":
+        WL = w["W_L"].to(tdt)
+        cat = torch.empty((B, n, d), dtype=tdt, device=dev)
+
+        def run():
+            wk.wk_lcb(WL, X, cat, B, n, d, n_f, n_l, args.dtype)
+        flops = 2 * n_l * n * d * B
+        bytes_ = (n * d + n_l * d) * es * B
+    else:
+        cat = torch.randn((B, n, d), device=dev).to(tdt)
+        out = torch.empty_like(X)
+
+        def run():
+            wk.wk_res_ln(cat, X, w["out_gamma"], w["out_beta"], out, B * n, d, args.dtype)
+        flops = 0
+        bytes_ = 3 * n * d * es * B
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.iters):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    st = wk.wk_device_status()
+    ms = e0.elapsed_time(e1) / max(1, args.iters)
+    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "batch": B, "dtype": args.dtype,
+                      "ms_per_launch": ms, "tflops": flops / (ms / 1e3) / 1e12 if flops else None,
+                      "gbs": bytes_ / (ms / 1e3) / 1e9, "flops_per_launch": flops, "bytes_per_launch": bytes_,
+                      "device_status": wk.wk_status_string(st)}))
+    if st != wk.WK_OK:
+        sys.exit(1)
+
+
+if __name__ == "__main__":
+    main()

@@ -34,10 +34,11 @@ def _sample(batch, count, seed=0):
 
 
 class DevStack:
-    def __init__(self, name, max_batch=None):
+    def __init__(self, name, max_batch=None, operand_dtype=None):
         self.cfg = C.CONFIGS[name]
         self.layers = [C.make_layer_dev(self.cfg, l) for l in range(self.cfg["layers"])]
-        self.h = wk.wk_stack_create(self.cfg, self.layers, max_batch=max_batch or self.cfg["batch"])
+        self.h = wk.wk_stack_create(self.cfg, self.layers, max_batch=max_batch or self.cfg["batch"],
+                                    operand_dtype=operand_dtype)
 
     def run(self, X):
         out = torch.empty_like(X)
@@ -56,9 +57,9 @@ def _oracle(cfg, examples):
     return oracle.stack_forward(cfg, lambda l: C.make_layer_host(cfg, l), X)
 
 
-def _parity(name, n_sample):
+def _parity(name, n_sample, operand_dtype=None):
     cfg = C.CONFIGS[name]
-    st = DevStack(name)
+    st = DevStack(name, operand_dtype=operand_dtype)
     try:
         X = C.make_x_dev(cfg, cfg["batch"])
         out = st.run(X)
@@ -67,7 +68,8 @@ def _parity(name, n_sample):
         assert np.isfinite(got).all()
         ref = _oracle(cfg, ex)
         err = max_scaled_err(got, ref)
-        print("%s: max |gpu-ref|/(1+|ref|) = %.3g over %d examples" % (name, err, len(ex)))
+        print("%s (operands %s): max |gpu-ref|/(1+|ref|) = %.3g over %d examples"
+              % (name, operand_dtype or "default", err, len(ex)))
         assert err <= TOL[cfg["dtype"]]
     finally:
         st.close()
@@ -91,6 +93,10 @@ def test_parity_c1_fp32_all_examples():
 
 def test_parity_c2_bf16():
     _parity("c2_bf16", 512)
+
+
+def test_parity_c2_bf16_with_bf16_operands():
+    _parity("c2_bf16", 512, operand_dtype="bf16")
 
 
 def test_parity_c5_bf16_wide_narrow():
