@@ -198,6 +198,40 @@ WK_API wk_status wk_res_ln(const void* concat, const void* X, const float* gamma
  * stand-alone calls above (handles have their own). */
 WK_API wk_status wk_device_status(wk_stream_t stream);
 
+/* ---- one layer without allocating: for callers that cannot call cudaMalloc ----
+ *
+ * The paper has no counterpart to this entry point; it exists for callers that
+ * must not have the library allocate device memory: a serving process that has
+ * handed all device memory to its own pool allocator, or a latency-critical loop
+ * where cudaMalloc / cudaFree (which synchronise the device) are not allowed.
+ * wk_stack_create allocates a workspace, so such callers use this instead.
+ *
+ * Runs ONE Wukong layer, out = LN_rows(concat(FMB(X), LCB(X)) + X), with the
+ * weights `w` used as given (operands in cfg->dtype; cfg->operand_dtype must be 0
+ * or equal to cfg->dtype, since converting weights would need memory). X and out
+ * are caller-owned device tensors [batch, n, d] of cfg->dtype that must not
+ * overlap; cfg->num_layers and cfg->max_batch are ignored.
+ *
+ * Intermediates live in one fixed device array of WK_NOALLOC_SCRATCH_BYTES that
+ * is part of the library image: every GPU that loads the library reserves it
+ * until the process exits. A batch needs, in bytes (each term rounded up to 256):
+ *   es * batch * (n*k + n*d + [m >= 2] * h + [m >= 3] * h),
+ * es = 2 (16-bit) or 4 (fp32), h = the widest hidden layer; a batch that needs
+ * more returns WK_ERR_INVALID_ARG before anything is launched. Nothing in the
+ * array has to start at zero: every call writes each region before reading it.
+ *
+ * No call allocates: no cudaMalloc, cudaFree or allocating library routine. The
+ * first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * which may load the library's device code on that device); make that first call
+ * before any stream capture. Every call shares the one array, so calls whose
+ * kernels can overlap on the GPU (different streams without ordering, or several
+ * host threads) race and corrupt each other's results; order them on one stream.
+ * Asynchronous on `stream`; device-side errors go to the status word that
+ * wk_device_status reads. */
+#define WK_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+WK_API wk_status wk_layer_forward_noalloc(const wk_stack_config* cfg, const wk_layer_weights* w, const void* X,
+                                          void* out, int64_t batch, wk_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -69,6 +69,8 @@ def lib():
             "wk_lcb": [vp, vp, vp, i64, i32, i32, i32, i32, ci, vp],
             "wk_res_ln": [vp, vp, vp, vp, vp, i64, i32, ci, cf, vp],
             "wk_device_status": [vp],
+            "wk_layer_forward_noalloc": [ctypes.POINTER(WkStackConfig), ctypes.POINTER(WkLayerWeights), vp, vp, i64,
+                                         vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -142,18 +144,18 @@ class StackHandle:
             pass
 
 
-def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0, operand_dtype=None):
-    """cfg: mapping with num_layers (or layers), n, d, k, n_f, n_l, hidden (the m-1
-    hidden widths) and dtype; layers: one mapping per layer with Y, W0..W{m-1},
-    b0..b{m-1} (or None), fmb_gamma, fmb_beta, W_L, out_gamma, out_beta."""
+def _config(cfg, max_batch, dtype, ln_eps, operand_dtype):
     hidden = list(cfg.get("hidden", []))
     m = len(hidden) + 1
     hid = (ctypes.c_int32 * max(1, len(hidden)))(*hidden) if hidden else None
-    c = WkStackConfig(int(cfg.get("num_layers", cfg.get("layers"))), cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
+    c = WkStackConfig(int(cfg.get("num_layers", cfg.get("layers", 1))), cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
                       cfg["n_l"], m, hid, _dtype_code(dtype if dtype is not None else cfg["dtype"]),
-                      float(ln_eps), int(max_batch if max_batch is not None else cfg["batch"]),
+                      float(ln_eps), int(max_batch if max_batch is not None else cfg.get("batch", 1)),
                       _dtype_code(operand_dtype) if operand_dtype is not None else WK_F32)
-    keep = [hid, list(layers)]
+    return c, hid, m
+
+
+def _layer_array(layers, m, keep):
     arr = (WkLayerWeights * len(layers))()
     for i, w in enumerate(layers):
         Wp = (ctypes.c_void_p * m)(*[_addr(w["W%d" % j]) for j in range(m)])
@@ -162,6 +164,16 @@ def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0, operand
         arr[i] = WkLayerWeights(_addr(w["Y"]), Wp, bp, _addr(w["fmb_gamma"]), _addr(w["fmb_beta"]), _addr(w["W_L"]),
                                 _addr(w["out_gamma"]), _addr(w["out_beta"]))
     keep.append(arr)
+    return arr
+
+
+def wk_stack_create(cfg, layers, max_batch=None, dtype=None, ln_eps=0.0, operand_dtype=None):
+    """cfg: mapping with num_layers (or layers), n, d, k, n_f, n_l, hidden (the m-1
+    hidden widths) and dtype; layers: one mapping per layer with Y, W0..W{m-1},
+    b0..b{m-1} (or None), fmb_gamma, fmb_beta, W_L, out_gamma, out_beta."""
+    c, hid, m = _config(cfg, max_batch, dtype, ln_eps, operand_dtype)
+    keep = [hid, list(layers)]
+    arr = _layer_array(layers, m, keep)
     h = ctypes.c_void_p()
     _check(lib().wk_stack_create(ctypes.byref(c), arr, ctypes.byref(h)), "wk_stack_create")
     return StackHandle(h.value, dict(cfg), keep)
@@ -222,3 +234,14 @@ def wk_res_ln(concat, X, gamma, beta, out, rows, d, dtype, eps=0.0, stream=None)
 
 def wk_device_status(stream=None):
     return lib().wk_device_status(_stream(stream))
+
+
+def wk_layer_forward_noalloc(cfg, layer, X, out, batch=None, stream=None, dtype=None, ln_eps=0.0):
+    """One Wukong layer with the intermediates in the library's fixed device array
+    (no allocation); see include/wukong.h for who needs it and its limits."""
+    c, hid, m = _config(cfg, 1, dtype, ln_eps, None)
+    keep = [hid]
+    arr = _layer_array([layer], m, keep)
+    b = X.shape[0] if batch is None else batch
+    _check(lib().wk_layer_forward_noalloc(ctypes.byref(c), arr, _addr(X), _addr(out), int(b), _stream(stream, X)),
+           "wk_layer_forward_noalloc")

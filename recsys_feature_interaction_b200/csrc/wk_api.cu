@@ -687,6 +687,93 @@ wk_status lcb16(const DevInfo* dv, const void* W_L, const void* X, void* concat,
   return run_gemm_tc<MODE_LCB, T, T>(dv, mp, lcb_params(batch, n, d, n_l, dv->standalone_status), st);
 }
 
+// ------------------------------------------------- no-allocation layer forward
+//
+// A one-layer forward whose intermediates live in a fixed device array that is
+// part of this library's image instead of memory the library allocates. The
+// array is reserved on every device that loads the library, until exit. Host
+// code must not hand the array's name to a kernel (on the host it names a
+// stand-in, not device memory); its device address is looked up once per device
+// with cudaGetSymbolAddress and cached.
+__device__ __align__(256) uint8_t g_noalloc_scratch[WK_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_addr[64];
+bool g_noalloc_init[64];
+
+wk_status noalloc_scratch(const DevInfo* dv, uint8_t** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_init[dv->id]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return WK_ERR_CUDA;
+    }
+    g_noalloc_addr[dv->id] = p;
+    g_noalloc_init[dv->id] = true;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_addr[dv->id]);
+  return WK_OK;
+}
+
+// Scratch bytes one example needs: A0, one or two MLP activation buffers, the
+// concat buffer; each region rounded up to 256 bytes for the whole batch.
+size_t noalloc_bytes(const wk_stack_config* c, const std::vector<int32_t>& dims, int64_t batch) {
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const size_t es = c->dtype == WK_F32 ? 4 : 2;
+  const int m = c->mlp_num_linear;
+  int32_t hmax = 0;
+  for (int j = 1; j < m; ++j) hmax = std::max(hmax, dims[j]);
+  size_t b = up(batch * static_cast<size_t>(c->n) * c->k * es) + up(batch * static_cast<size_t>(c->n) * c->d * es);
+  if (m >= 2) b += up(batch * static_cast<size_t>(hmax) * es);
+  if (m >= 3) b += up(batch * static_cast<size_t>(hmax) * es);
+  return b;
+}
+
+template <typename T>
+wk_status layer_noalloc16(const DevInfo* dv, const wk_stack_config* c, const std::vector<int32_t>& dims,
+                          const wk_layer_weights* w, const T* X, T* out, int64_t batch, uint8_t* scratch,
+                          float eps, cudaStream_t st) {
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const int n = c->n, d = c->d, k = c->k, m = c->mlp_num_linear;
+  const size_t nd = static_cast<size_t>(n) * d;
+  int32_t hmax = 0;
+  for (int j = 1; j < m; ++j) hmax = std::max(hmax, dims[j]);
+  uint8_t* p = scratch;
+  T* A0 = reinterpret_cast<T*>(p);
+  p += up(batch * static_cast<size_t>(n) * k * 2);
+  T* cat = reinterpret_cast<T*>(p);
+  p += up(batch * nd * 2);
+  T* H[2] = {reinterpret_cast<T*>(p), nullptr};
+  if (m >= 2) p += up(batch * static_cast<size_t>(hmax) * 2);
+  H[1] = reinterpret_cast<T*>(p);
+  unsigned* status = dv->standalone_status;
+  wk_status s = run_fm16<T>(dv, X, static_cast<const T*>(w->Y), w->fmb_ln_gamma, w->fmb_ln_beta, A0, batch, n, d, k,
+                            eps, status, st);
+  for (int j = 0; j < m && s == WK_OK; ++j) {
+    const T* in = (j == 0) ? A0 : H[(j - 1) % 2];
+    const bool lastj = j == m - 1;
+    T* o = lastj ? cat : H[j % 2];
+    const int64_t ldc = lastj ? static_cast<int64_t>(nd) : dims[j + 1];
+    const float* bias = w->b ? w->b[j] : nullptr;
+    if (mlp_tc_ok(batch, dims[j], dims[j + 1], ldc)) {
+      GemmMaps mp;
+      if (!map_kmajor<T>(dv, &mp.A, in, dims[j], batch, GEMM_BM) ||
+          !map_kmajor<T>(dv, &mp.B, w->W[j], dims[j], dims[j + 1], GEMM_BN) ||
+          !map_out<T>(dv, &mp.C, o, dims[j + 1], batch, ldc))
+        return WK_ERR_UNSUPPORTED;
+      s = run_gemm_tc<MODE_MLP, T, T>(dv, mp, mlp_params(batch, dims[j], dims[j + 1], bias, lastj ? 0 : 1, status),
+                                       st);
+    } else {
+      s = run_gemm_simt<T, T>(in, static_cast<const T*>(w->W[j]), bias, o, batch, dims[j], dims[j + 1], ldc,
+                              lastj ? 0 : 1, st);
+    }
+  }
+  if (s == WK_OK) s = lcb16<T>(dv, w->W_L, X, cat, batch, n, d, c->n_f, c->n_l, st);
+  if (s == WK_OK)
+    s = run_res_ln<T, T, T>(dv, cat, X, w->out_ln_gamma, w->out_ln_beta, out, batch * n, d, eps, st);
+  return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1059,6 +1146,80 @@ wk_status wk_device_status(wk_stream_t stream) {
   wk_status s = dev_info(&dv);
   if (s != WK_OK) return s;
   return read_status_word(dv->standalone_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+wk_status wk_layer_forward_noalloc(const wk_stack_config* cfg, const wk_layer_weights* w, const void* X, void* out,
+                                   int64_t batch, wk_stream_t stream) {
+  if (!w || batch < 0) return WK_ERR_INVALID_ARG;
+  wk_stack_config c1;
+  if (cfg) {
+    c1 = *cfg;
+    c1.num_layers = 1;
+    c1.max_batch = 1;
+  }
+  wk_status s = validate_cfg(cfg ? &c1 : nullptr);
+  if (s != WK_OK) return s;
+  if (cfg->operand_dtype != WK_F32 && cfg->operand_dtype != cfg->dtype) return WK_ERR_UNSUPPORTED;
+  if (batch == 0) return WK_OK;
+  if (!X || !out || !al16(X) || !al16(out) || !w->Y || !w->W || !w->W_L || !w->fmb_ln_gamma || !w->fmb_ln_beta ||
+      !w->out_ln_gamma || !w->out_ln_beta)
+    return WK_ERR_INVALID_ARG;
+  std::vector<int32_t> dims;
+  dims.push_back(cfg->n * cfg->k);
+  for (int j = 0; j + 1 < cfg->mlp_num_linear; ++j) dims.push_back(cfg->mlp_hidden[j]);
+  dims.push_back(cfg->n_f * cfg->d);
+  for (int j = 0; j < cfg->mlp_num_linear; ++j)
+    if (!w->W[j]) return WK_ERR_INVALID_ARG;
+  if (noalloc_bytes(cfg, dims, batch) > WK_NOALLOC_SCRATCH_BYTES) return WK_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(batch) * cfg->n * cfg->d * (cfg->dtype == WK_F32 ? 4 : 2);
+  const uint8_t* xa = static_cast<const uint8_t*>(X);
+  const uint8_t* oa = static_cast<const uint8_t*>(out);
+  if (xa < oa + bytes && oa < xa + bytes) return WK_ERR_INVALID_ARG;
+  DevInfo* dv = nullptr;
+  s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  uint8_t* scratch = nullptr;
+  s = noalloc_scratch(dv, &scratch);
+  if (s != WK_OK) return s;
+  const float eps = cfg->ln_eps > 0.f ? cfg->ln_eps : 1e-5f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == WK_BF16)
+    return layer_noalloc16<bf16>(dv, cfg, dims, w, static_cast<const bf16*>(X), static_cast<bf16*>(out), batch,
+                                 scratch, eps, st);
+  if (cfg->dtype == WK_F16)
+    return layer_noalloc16<f16>(dv, cfg, dims, w, static_cast<const f16*>(X), static_cast<f16*>(out), batch, scratch,
+                                eps, st);
+  // fp32: the CUDA-core kernels, same scratch layout
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const int n = cfg->n, d = cfg->d, k = cfg->k, m = cfg->mlp_num_linear;
+  const size_t nd = static_cast<size_t>(n) * d;
+  int32_t hmax = 0;
+  for (int j = 1; j < m; ++j) hmax = std::max(hmax, dims[j]);
+  uint8_t* p = scratch;
+  float* A0 = reinterpret_cast<float*>(p);
+  p += up(batch * static_cast<size_t>(n) * k * 4);
+  float* cat = reinterpret_cast<float*>(p);
+  p += up(batch * nd * 4);
+  float* H[2] = {reinterpret_cast<float*>(p), nullptr};
+  if (m >= 2) p += up(batch * static_cast<size_t>(hmax) * 4);
+  H[1] = reinterpret_cast<float*>(p);
+  const float* Xf = static_cast<const float*>(X);
+  s = run_fm_simt<float>(dv, Xf, static_cast<const float*>(w->Y), w->fmb_ln_gamma, w->fmb_ln_beta, A0, batch, n, d, k,
+                         eps, st);
+  for (int j = 0; j < m && s == WK_OK; ++j) {
+    const float* in = (j == 0) ? A0 : H[(j - 1) % 2];
+    const bool lastj = j == m - 1;
+    float* o = lastj ? cat : H[j % 2];
+    s = run_gemm_simt<float, float>(in, static_cast<const float*>(w->W[j]), w->b ? w->b[j] : nullptr, o, batch,
+                                    dims[j], dims[j + 1], lastj ? static_cast<int64_t>(nd) : dims[j + 1],
+                                    lastj ? 0 : 1, st);
+  }
+  if (s == WK_OK)
+    s = run_lcb_simt<float, float>(static_cast<const float*>(w->W_L), Xf, cat, batch, n, d, cfg->n_f, cfg->n_l, st);
+  if (s == WK_OK)
+    s = run_res_ln<float, float, float>(dv, cat, Xf, w->out_ln_gamma, w->out_ln_beta, static_cast<float*>(out),
+                                        batch * n, d, eps, st);
+  return s;
 }
 
 }  // extern "C"
