@@ -46,12 +46,14 @@ struct FmCfg {
   static constexpr int BMT = (R / 16) / BWM;  // pass B m16 tiles per warp per chunk (over n)
   static constexpr int BNT = (KC / 8) / BWN;  // pass B n8 tiles per warp (over k)
   static constexpr int KS_D = D / 16;         // pass B k16 steps
-  static constexpr int ZPART_BYTES = AKS * D * KC * 4;
+  static constexpr int KCP = KC + 4;         // padded fp32 row of the Z partials / LN staging
+  static constexpr int ZPART_BYTES = (AKS * D > R ? AKS * D : R) * KCP * 4;
   static constexpr int ZB_BYTES = D * SY;
   static constexpr int SMEM = 1024 + STAGES * SLOT + ZPART_BYTES + ZB_BYTES + 64 + 16 * STAGES + 16;
   static_assert(D % 32 == 0 && KC % 8 == 0 && N % 16 == 0 && R % 16 == 0 && R <= 256, "tile shape");
   static_assert(SLOT % 1024 == 0 && XBLK % 1024 == 0, "slot blocks stay aligned to the swizzle atoms");
   static_assert(YSW != 0 || (YROW / 16) % 2 == 1, "unswizzled Y rows must be an odd number of 16-byte units");
+  static_assert(KC % 4 == 0, "the staged LayerNorm epilogue moves 4 values at a time");
   static_assert(AWM * AWN * AKS == 8 && BWM * BWN == 8, "8 consumer warps");
   static_assert((D / 16) % AWM == 0 && (KC / 8) % AWN == 0 && (R / 16) % BWM == 0 && (KC / 8) % BWN == 0,
                 "warp split");
@@ -204,25 +206,24 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
         ph ^= 1u;
       }
     }
-    // partial Z tiles -> zpart[a_ks][t][c] (fp32)
+    // partial Z tiles -> zpart[a_ks][t][c] (fp32, rows padded to KCP: conflict-free float2 stores)
+    named_bar(1, 256);  // the previous example's LayerNorm staging in zpart is consumed
 #pragma unroll
     for (int mt = 0; mt < C::AMT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < C::ANT; ++nt) {
         const int t = (a_wm * C::AMT + mt) * 16 + g;
         const int cc = (a_wn * C::ANT + nt) * 8 + 2 * t4;
-        float* zp = zpart + a_ks * C::D * C::KC;
-        zp[t * C::KC + cc] = zacc[mt][nt][0];
-        zp[t * C::KC + cc + 1] = zacc[mt][nt][1];
-        zp[(t + 8) * C::KC + cc] = zacc[mt][nt][2];
-        zp[(t + 8) * C::KC + cc + 1] = zacc[mt][nt][3];
+        float* zp = zpart + a_ks * C::D * C::KCP;
+        *reinterpret_cast<float2*>(zp + t * C::KCP + cc) = make_float2(zacc[mt][nt][0], zacc[mt][nt][1]);
+        *reinterpret_cast<float2*>(zp + (t + 8) * C::KCP + cc) = make_float2(zacc[mt][nt][2], zacc[mt][nt][3]);
       }
     named_bar(1, 256);
     for (int i = tid; i < C::D * C::KC; i += 256) {
+      const int t = i / C::KC, cc = i - t * C::KC;
       float z = 0.f;
 #pragma unroll
-      for (int k = 0; k < C::AKS; ++k) z += zpart[k * C::D * C::KC + i];
-      const int t = i / C::KC, cc = i - t * C::KC;
+      for (int k = 0; k < C::AKS; ++k) z += zpart[(k * C::D + t) * C::KCP + cc];
       *reinterpret_cast<T*>(zb + t * C::SY + cc * 2) = Half16<T>::from(z);
     }
     named_bar(1, 256);
@@ -314,26 +315,38 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
 #pragma unroll
     for (int w = 0; w < 8; ++w) qt += red[8 + w];
     const float rstd = rsqrtf(qt * (1.0f / (C::N * C::KC)) + eps);
+    // Normalised values go out one chunk of R rows at a time through zpart (fp32,
+    // padded rows), so that gamma / beta are read and A0 is written with
+    // coalesced 16-byte accesses.
     T* ab = A0 + b * (C::N * C::KC);
 #pragma unroll
-    for (int c = 0; c < C::NCH; ++c)
+    for (int c = 0; c < C::NCH; ++c) {
+      named_bar(1, 256);  // zpart free (Z reduction done / previous chunk written out)
 #pragma unroll
       for (int mt = 0; mt < C::BMT; ++mt)
 #pragma unroll
         for (int nt = 0; nt < C::BNT; ++nt)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int row = c * C::R + (b_wm * C::BMT + mt) * 16 + g + h * 8;
-            if (row < C::N) {
-              const int col = (b_wn * C::BNT + nt) * 8 + 2 * t4;
-              const int idx = row * C::KC + col;
-              const float2 gm = __ldg(reinterpret_cast<const float2*>(gamma + idx));
-              const float2 bt = __ldg(reinterpret_cast<const float2*>(beta + idx));
-              const float v0 = (facc[c][mt][nt][2 * h] - mean) * rstd * gm.x + bt.x;
-              const float v1 = (facc[c][mt][nt][2 * h + 1] - mean) * rstd * gm.y + bt.y;
-              *reinterpret_cast<uint32_t*>(ab + idx) = Half16<T>::pack2(v0, v1);
-            }
+            const int r = (b_wm * C::BMT + mt) * 16 + g + h * 8;  // row within the chunk
+            const int col = (b_wn * C::BNT + nt) * 8 + 2 * t4;
+            *reinterpret_cast<float2*>(zpart + r * C::KCP + col) =
+                make_float2((facc[c][mt][nt][2 * h] - mean) * rstd, (facc[c][mt][nt][2 * h + 1] - mean) * rstd);
           }
+      named_bar(1, 256);
+      const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+      const int base = c * C::R * C::KC;  // flat index of the chunk's first value
+      for (int q4 = tid; q4 < rows * C::KC / 4; q4 += 256) {
+        const int r = (q4 * 4) / C::KC, col = (q4 * 4) - r * C::KC;
+        const float4 v = *reinterpret_cast<const float4*>(zpart + r * C::KCP + col);
+        const float4 gm = __ldg(reinterpret_cast<const float4*>(gamma + base) + q4);
+        const float4 bt = __ldg(reinterpret_cast<const float4*>(beta + base) + q4);
+        uint2 o;
+        o.x = Half16<T>::pack2(v.x * gm.x + bt.x, v.y * gm.y + bt.y);
+        o.y = Half16<T>::pack2(v.z * gm.z + bt.z, v.w * gm.w + bt.w);
+        *(reinterpret_cast<uint2*>(ab + base) + q4) = o;
+      }
+    }
   }
 }
 

@@ -313,8 +313,8 @@ template <int D, typename TC, typename TR, typename TO>
 wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
                        int64_t rows, float eps, cudaStream_t st) {
   constexpr int VPR = D / 8;
-  constexpr int G = pow2_ceil(VPR);
-  constexpr int rows_per_block = (256 / 32) * (32 / G) * 4;
+  constexpr int G = res_ln_lanes(VPR);
+  constexpr int rows_per_block = (256 / 32) * (32 / G) * ((VPR / G) >= 4 ? 2 : 4);
   int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
   const int64_t cap = static_cast<int64_t>(dv->sms) * 8;
   if (blocks > cap) blocks = cap;
