@@ -29,6 +29,7 @@
 #include "convert.cuh"
 #include "fm_mma.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "res_ln.cuh"
 #include "simt.cuh"
 
@@ -194,6 +195,44 @@ wk_status run_gemm_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p
   const int grid = std::min(p.num_tiles, dv->sms);
   gemm_tc_kernel<MODE, T, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
+}
+
+template <typename T, typename TO>
+wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
+  constexpr uint32_t smem = gemm2_smem_bytes<TO>();
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO>), smem);
+  if (s != WK_OK) return s;
+  if (p.num_tiles <= 0) return WK_OK;
+  const int pairs = std::min(p.num_tiles, dv->sms / 2);
+  gemm_tc2_kernel<T, TO><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  return launch_status();
+}
+
+// The CTA-pair GEMM (256-row tiles) serves every M above one 128-row tile unless
+// the environment sets WK_PAIR_GEMM=0.
+bool use_pair_gemm(int64_t M) {
+  static const bool enabled = [] {
+    const char* e = getenv("WK_PAIR_GEMM");
+    return !(e && e[0] == '0');
+  }();
+  return enabled && M > GEMM_BM;
+}
+
+GemmParams mlp2_params(int64_t M, int K, int N, const float* bias, int relu, unsigned* status) {
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = N;
+  p.K = K;
+  p.num_m_tiles = static_cast<int>((M + GEMM2_BM - 1) / GEMM2_BM);
+  p.num_n_tiles = (N + GEMM2_BN - 1) / GEMM2_BN;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  p.num_kb = (K + GEMM2_BK - 1) / GEMM2_BK;
+  p.group_m = 8;
+  p.mma_n = GEMM2_BN;
+  p.bias = bias;
+  p.relu = relu;
+  p.status = status;
+  return p;
 }
 
 GemmParams mlp_params(int64_t M, int K, int N, const float* bias, int relu, unsigned* status) {
@@ -405,6 +444,7 @@ struct wk_stack {
   unsigned* status = nullptr;
   // TMA descriptors of the tensor-core path
   bool tc_mlp = false, tc_lcb = false;
+  bool pair = false;                            // MLP Linears on CTA pairs (gemm_tc2.cuh)
   std::vector<std::vector<GemmMaps>> mlp_maps;  // [layer][j]
   std::vector<CUtensorMap> lcbA;                // [layer]
   CUtensorMap lcbB_ws[2];
@@ -510,6 +550,7 @@ wk_status build_maps(wk_stack* h) {
     if (!mlp_tc_ok(B, h->dims[j], h->dims[j + 1], ldc)) h->tc_mlp = false;
   }
   h->tc_lcb = lcb_tc_ok(B, n, d);
+  h->pair = use_pair_gemm(B);
   if (h->tc_mlp) {
     h->mlp_maps.assign(L, std::vector<GemmMaps>(m));
     for (int l = 0; l < L; ++l)
@@ -518,7 +559,7 @@ wk_status build_maps(wk_stack* h) {
         const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
         const bool last = j == m - 1;
         const bool ok = map_kmajor<T>(dv, &mp.A, in, h->dims[j], B, GEMM_BM) &&
-                        map_kmajor<T>(dv, &mp.B, h->W[l][j], h->dims[j], h->dims[j + 1], GEMM_BN) &&
+                        map_kmajor<T>(dv, &mp.B, h->W[l][j], h->dims[j], h->dims[j + 1], h->pair ? 128 : GEMM_BN) &&
                         (last ? map_out<T>(dv, &mp.C, h->cat, h->dims[j + 1], B, nd)
                               : map_out<T>(dv, &mp.C, h->H[j % 2], h->dims[j + 1], B, h->dims[j + 1]));
         if (!ok) return WK_ERR_UNSUPPORTED;
@@ -569,7 +610,10 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
       void* o = lastj ? h->cat : h->H[j % 2];
       const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
       const int relu = lastj ? 0 : 1;
-      if (h->tc_mlp)
+      if (h->tc_mlp && h->pair)
+        s = run_gemm_tc2<T, T>(dv, h->mlp_maps[l][j],
+                               mlp2_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
+      else if (h->tc_mlp)
         s = run_gemm_tc<MODE_MLP, T, T>(dv, h->mlp_maps[l][j],
                                          mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
       else
@@ -667,10 +711,13 @@ template <typename T>
 wk_status mlp_linear16(const DevInfo* dv, const void* A, const void* W, const float* bias, void* C, int64_t M,
                               int K, int N, int64_t ldc, int relu, cudaStream_t st) {
   if (!mlp_tc_ok(M, K, N, ldc)) return WK_ERR_UNSUPPORTED;
+  const bool pair = use_pair_gemm(M);
   GemmMaps mp;
-  if (!map_kmajor<T>(dv, &mp.A, A, K, M, GEMM_BM) || !map_kmajor<T>(dv, &mp.B, W, K, N, GEMM_BN) ||
+  if (!map_kmajor<T>(dv, &mp.A, A, K, M, GEMM_BM) || !map_kmajor<T>(dv, &mp.B, W, K, N, pair ? 128 : GEMM_BN) ||
       !map_out<T>(dv, &mp.C, C, N, M, ldc))
     return WK_ERR_UNSUPPORTED;
+  if (pair)
+    return run_gemm_tc2<T, T>(dv, mp, mlp2_params(M, K, N, bias, relu ? 1 : 0, dv->standalone_status), st);
   return run_gemm_tc<MODE_MLP, T, T>(dv, mp, mlp_params(M, K, N, bias, relu ? 1 : 0, dv->standalone_status), st);
 }
 
