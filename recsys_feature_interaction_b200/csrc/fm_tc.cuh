@@ -1,0 +1,367 @@
+// fm_tc.cuh -- the FMB front of a Wukong layer on the 5th-generation tensor cores:
+//
+//   A0[b] = LN( flatten_rowmajor( X_b (X_b^T Y) ) ) * gamma + beta
+//
+// (the optimised FM of the Wukong page, section 2.2, FMB paragraph: compress the
+// features to k with Y first, then cross; flatten feature-major; LayerNorm over
+// all n*k values). Per example, two tcgen05 products with fp32 accumulators in
+// TMEM:
+//   pass A  Z = X^T Y   M = d (128-row tiles), N = k, K = n: X is read as an
+//                       MN-major operand, Y as an MN-major operand;
+//   pass B  F = X Z     M = n (one 128-row tile per chunk), N = k, K = d: X is read
+//                       as a K-major operand (the same shared-memory tiles as pass A),
+//                       Z as an MN-major operand written to shared memory (16-bit)
+//                       by the epilogue warps from TMEM.
+// One persistent CTA per SM walks the examples (192 threads): warp 0 streams 128-row
+// chunks of X (and of Y in pass A) with TMA into a ring, warp 1 allocates TMEM and
+// one thread issues the MMAs, warps 2..5 turn Z into the pass-B operand and compute
+// the LayerNorm from TMEM (three passes: mean, variance, output) and store A0.
+// Pass A of example b+1 overlaps the LayerNorm of example b (Z and F have their
+// own TMEM columns). Every mbarrier wait is bounded.
+//
+// k is padded to KP = 32 or 64 columns (the MMA N) with zero columns of Y, which
+// the TMA fills out of bounds; F columns past k are never read. Rows of a chunk past
+// n (the last chunk, or the next example's rows) only reach accumulator rows that are
+// never read, and the Z tile rows past d read padding shared memory.
+#pragma once
+
+#include "common.cuh"
+
+namespace wk {
+
+template <int N_, int D_, int K_>
+struct FmTcCfg {
+  static constexpr int N = N_, D = D_, K = K_;
+  static constexpr int R = 128;                            // rows per chunk = MMA M
+  static constexpr int XBOXW = D >= 64 ? 64 : 32;          // columns per X box (128B or 64B swizzle)
+  static constexpr int XSW = XBOXW * 2;                    // swizzle span in bytes
+  static constexpr int XBOXES = (D + XBOXW - 1) / XBOXW;
+  static constexpr int XBOXB = R * XBOXW * 2;              // bytes per X box
+  static constexpr int KP = K <= 32 ? 32 : 64;             // MMA N (k padded)
+  static constexpr int YRB = KP * 2;                       // bytes per Y / Z row
+  static constexpr int YB = R * YRB;
+  static constexpr int SLOT = XBOXES * XBOXB + YB;
+  static constexpr int NCH = (N + R - 1) / R;              // chunks = F tiles
+  static constexpr int MTZ = (D + R - 1) / R;              // Z tiles
+  static constexpr int ZCOL = MTZ * KP;                    // first TMEM column of F
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int ZB = ((D + 15) / 16) * 16 * YRB;    // Z operand in shared memory
+  // Z tiles read (R / XBOXW) boxes each from a slot's first box; what lies past the
+  // slot's X and Y tiles must still be shared memory this CTA owns.
+  static constexpr int OVER = (MTZ * (R / XBOXW) - XBOXES) * XBOXB - YB;
+  static constexpr int PAD = OVER > 0 ? ((OVER + 1023) / 1024) * 1024 : 0;
+  static constexpr int BUDGET = 220 * 1024;
+  static constexpr int STAGES_RAW = (BUDGET - ZB - PAD - 1024 - 512) / SLOT;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int SMEM = 1024 + STAGES * SLOT + PAD + ZB + 512;
+  static_assert(ZCOL + NCH * KP <= TMEM_COLS, "TMEM columns");
+  static_assert(STAGES >= 2, "shared memory");
+  static_assert(D % 32 == 0 && N % 16 == 0 && K % 4 == 0 && K <= 64, "shape");
+  static_assert(SLOT % 1024 == 0 && XBOXB % 1024 == 0 && ZB % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+constexpr int FMTC_THREADS = 192;
+
+// Shared address of Z operand element row t, 16-byte unit j (MN-major, KP columns).
+template <class C>
+__device__ __forceinline__ uint32_t fmtc_zb_addr(uint32_t zb, int t, int j) {
+  const int pj = (C::YRB == 128) ? (j ^ (t & 7)) : (j ^ ((t >> 1) & 3));
+  return zb + t * C::YRB + pj * 16;
+}
+
+template <class C, typename T>
+__global__ void __launch_bounds__(FMTC_THREADS, 1)
+    fm_ln_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                    const float* __restrict__ gamma, const float* __restrict__ beta, T* __restrict__ A0,
+                    int64_t batch, float eps, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* ring = smem;
+  uint8_t* zb = ring + C::STAGES * C::SLOT + C::PAD;
+  float* red = reinterpret_cast<float*>(zb + C::ZB);       // [2][4] partial sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 8);
+  uint64_t* full = bars;                                    // [STAGES]
+  uint64_t* empty = bars + C::STAGES;                       // [STAGES]
+  uint64_t* zfull = bars + 2 * C::STAGES;                   // MMA -> epilogue: Z ready in TMEM
+  uint64_t* zready = zfull + 1;                             // epilogue -> MMA: Z operand in smem
+  uint64_t* ffull = zfull + 2;                              // MMA -> epilogue: F ready in TMEM
+  uint64_t* fempty = zfull + 3;                             // epilogue -> MMA: F read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zfull + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmY);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(zfull, 1);
+    mbar_init(zready, 4);
+    mbar_init(ffull, 1);
+    mbar_init(fempty, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x) {
+        for (int pass = 0; ok && pass < 2; ++pass) {
+          for (int c = 0; c < C::NCH; ++c) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, status)) {
+              ok = false;
+              break;
+            }
+            uint8_t* slot = ring + s * C::SLOT;
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(C::XBOXES * C::XBOXB + (pass == 0 ? C::YB : 0)));
+            const int row0 = static_cast<int>(b * C::N + c * C::R);
+#pragma unroll
+            for (int bx = 0; bx < C::XBOXES; ++bx)
+              tma_load_2d(&tmX, &full[s], slot + bx * C::XBOXB, bx * C::XBOXW, row0);
+            if (pass == 0) tma_load_2d(&tmY, &full[s], slot + C::XBOXES * C::XBOXB, 0, c * C::R);
+            if (++s == C::STAGES) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < C::STAGES; ++i) mbar_wait(&full[i], ph ^ (i < s ? 0u : 1u), nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const bool bf = Half16<T>::kBF16;
+      const uint32_t idA = idesc_f16kind_f32(C::R, C::KP, 1, 1, bf);  // Z = X^T Y: both MN-major
+      const uint32_t idB = idesc_f16kind_f32(C::R, C::KP, 0, 1, bf);  // F = X Z: X K-major, Z MN-major
+      const uint32_t xsw = C::XSW == 128 ? 2u : 4u;
+      const uint32_t ysw = C::YRB == 128 ? 2u : 4u;
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t eph = 0;  // per-example phase of zready / fempty / zfull / ffull
+      bool ok = true;
+      bool issued = false;
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x) {
+        // pass A: Z = X^T Y (the previous example's Z was consumed before its pass B)
+        for (int c = 0; ok && c < C::NCH; ++c) {
+          if (!mbar_wait(&full[s], ph, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          const uint32_t xs = smem_u32(ring + s * C::SLOT);
+          const uint32_t ys = xs + C::XBOXES * C::XBOXB;
+          for (int ks = 0; ks < rows / 16; ++ks) {
+            const uint64_t bdesc = smem_desc(ys + ks * 16 * C::YRB, C::YB, 8 * C::YRB, ysw);
+#pragma unroll
+            for (int mz = 0; mz < C::MTZ; ++mz) {
+              // M atoms of XBOXW columns are the X boxes (LBO), 8-row K groups are SBO apart
+              const uint32_t a0 = xs + mz * (C::R / C::XBOXW) * C::XBOXB + ks * 16 * C::XSW;
+              const uint64_t adesc = smem_desc(a0, C::XBOXB, 8 * C::XSW, xsw);
+              umma_f16kind(tmem_base + mz * C::KP, adesc, bdesc, idA, (c | ks) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty[s]);
+          issued = true;
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(zfull);
+        // pass B: F = X Z, once Z is in shared memory and the previous F has been read
+        if (!mbar_wait(zready, eph, status) || !mbar_wait(fempty, eph ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int c = 0; ok && c < C::NCH; ++c) {
+          if (!mbar_wait(&full[s], ph, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xs = smem_u32(ring + s * C::SLOT);
+#pragma unroll
+          for (int ks = 0; ks < C::D / 16; ++ks) {
+            const int bx = ks / (C::XBOXW / 16), kin = ks % (C::XBOXW / 16);
+            const uint64_t adesc = smem_desc(xs + bx * C::XBOXB + kin * 32, 16, 8 * C::XSW, xsw);
+            const uint64_t bdesc = smem_desc(smem_u32(zb) + ks * 16 * C::YRB, C::ZB, 8 * C::YRB, ysw);
+            umma_f16kind(tmem_base + C::ZCOL + c * C::KP, adesc, bdesc, idB, ks != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(ffull);
+        eph ^= 1u;
+      }
+      if (!ok && issued) {  // no MMA may still write TMEM when it is freed
+        umma_commit(zfull);
+        mbar_wait(zfull, eph, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;           // TMEM lane quarter
+    const int ew = warp - 2;          // 0..3 among the epilogue warps
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const float inv_cnt = 1.0f / static_cast<float>(C::N * C::K);
+    uint32_t eph = 0;
+    // After a failed wait (status flagged) a warp stops waiting but keeps walking
+    // the same control flow, so every named barrier still sees all four warps.
+    bool ok = true;
+    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
+      // Z (TMEM, fp32) -> 16-bit MN-major operand in shared memory
+      if (ok) ok = mbar_wait(zfull, eph, status);
+      tc_fence_after();
+#pragma unroll
+      for (int mz = 0; mz < C::MTZ; ++mz) {
+        const int t = mz * C::R + q * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < C::KP / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(mz * C::KP + h * 32), r);
+          tmem_ld_wait();
+          if (t < C::D) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 u;
+              u.x = Half16<T>::pack2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+              u.y = Half16<T>::pack2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+              u.z = Half16<T>::pack2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+              u.w = Half16<T>::pack2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(fmtc_zb_addr<C>(smem_u32(zb), t, h * 4 + j)),
+                           "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                           : "memory");
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();  // the tensor core reads these stores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(zready);
+
+      // LayerNorm over the n*k values of F (TMEM), three passes
+      if (ok) ok = mbar_wait(ffull, eph, status);
+      tc_fence_after();
+      float part = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < C::NCH; ++c) {
+        const int row = c * C::R + q * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < C::KP / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
+          tmem_ld_wait();
+          if (row < C::N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (h * 32 + j < C::K) part += __uint_as_float(r[j]);
+          }
+        }
+      }
+      part = warp_sum(part);
+      if (lane == 0) red[ew] = part;
+      named_bar(1, 128);
+      const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+      float qs = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < C::NCH; ++c) {
+        const int row = c * C::R + q * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < C::KP / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
+          tmem_ld_wait();
+          if (row < C::N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (h * 32 + j < C::K) {
+                const float dv = __uint_as_float(r[j]) - mean;
+                qs += dv * dv;
+              }
+          }
+        }
+      }
+      qs = warp_sum(qs);
+      if (lane == 0) red[4 + ew] = qs;
+      named_bar(1, 128);
+      const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
+      T* ab = A0 + b * (C::N * C::K);
+#pragma unroll 1
+      for (int c = 0; c < C::NCH; ++c) {
+        const int row = c * C::R + q * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < C::KP / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
+          tmem_ld_wait();
+          if (row < C::N) {
+            const float* g = gamma + row * C::K + h * 32;
+            const float* bt = beta + row * C::K + h * 32;
+            T* o = ab + row * C::K + h * 32;
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              if (h * 32 + j < C::K) {
+                const float4 g0 = __ldg(reinterpret_cast<const float4*>(g + j));
+                const float4 g1 = __ldg(reinterpret_cast<const float4*>(g + j + 4));
+                const float4 b0 = __ldg(reinterpret_cast<const float4*>(bt + j));
+                const float4 b1 = __ldg(reinterpret_cast<const float4*>(bt + j + 4));
+                uint4 u;
+                u.x = Half16<T>::pack2((__uint_as_float(r[j + 0]) - mean) * rstd * g0.x + b0.x,
+                                       (__uint_as_float(r[j + 1]) - mean) * rstd * g0.y + b0.y);
+                u.y = Half16<T>::pack2((__uint_as_float(r[j + 2]) - mean) * rstd * g0.z + b0.z,
+                                       (__uint_as_float(r[j + 3]) - mean) * rstd * g0.w + b0.w);
+                u.z = Half16<T>::pack2((__uint_as_float(r[j + 4]) - mean) * rstd * g1.x + b1.x,
+                                       (__uint_as_float(r[j + 5]) - mean) * rstd * g1.y + b1.y);
+                u.w = Half16<T>::pack2((__uint_as_float(r[j + 6]) - mean) * rstd * g1.z + b1.z,
+                                       (__uint_as_float(r[j + 7]) - mean) * rstd * g1.w + b1.w);
+                *reinterpret_cast<uint4*>(o + j) = u;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar(1, 128);  // every epilogue warp is past its reads of red[] and F
+      if (lane == 0) mbar_arrive(fempty);
+      eph ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+using FmTcC2 = FmTcCfg<64, 128, 16>;
+using FmTcC3 = FmTcCfg<256, 160, 32>;
+using FmTcC4 = FmTcCfg<512, 160, 64>;
+using FmTcC5 = FmTcCfg<720, 32, 24>;
+
+}  // namespace wk

@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "convert.cuh"
 #include "fm_mma.cuh"
+#include "fm_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
 #include "res_ln.cuh"
@@ -307,6 +308,43 @@ wk_status run_fm_mma(const DevInfo* dv, const T* X, const T* Y, const float* g, 
   return launch_status();
 }
 
+template <class C, typename T>
+wk_status run_fm_tc(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
+                    float eps, unsigned* status, cudaStream_t st) {
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fm_ln_tc_kernel<C, T>), C::SMEM);
+  if (s != WK_OK) return s;
+  CUtensorMap tmX, tmY;
+  {  // X as [batch*n rows, d]: boxes of XBOXW columns x 128 rows
+    const uint64_t dims[2] = {static_cast<uint64_t>(C::D), static_cast<uint64_t>(batch) * C::N};
+    const uint64_t str[1] = {static_cast<uint64_t>(C::D) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(C::XBOXW), static_cast<uint32_t>(C::R)};
+    if (!make_map(dv, &tmX, tmap_dtype<T>(), 2, X, dims, str, box,
+                  C::XSW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+      return WK_ERR_UNSUPPORTED;
+  }
+  {  // Y [n, k]: boxes of KP columns (zero-filled past k) x 128 rows
+    const uint64_t dims[2] = {static_cast<uint64_t>(C::K), static_cast<uint64_t>(C::N)};
+    const uint64_t str[1] = {static_cast<uint64_t>(C::K) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(C::KP), static_cast<uint32_t>(C::R)};
+    if (!make_map(dv, &tmY, tmap_dtype<T>(), 2, Y, dims, str, box,
+                  C::YRB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+      return WK_ERR_UNSUPPORTED;
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(batch, dv->sms));
+  fm_ln_tc_kernel<C, T><<<grid, FMTC_THREADS, C::SMEM, st>>>(tmX, tmY, g, b, A0, batch, eps, status);
+  return launch_status();
+}
+
+// The tcgen05 FM serves the instantiated shapes unless the environment sets
+// WK_FM_MMA_SYNC=1, which selects the warp-level-MMA kernel.
+bool use_fm_mma_sync() {
+  static const bool on = [] {
+    const char* e = getenv("WK_FM_MMA_SYNC");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
 size_t fm_simt_smem(int n, int d, int k) {
   return sizeof(float) * (static_cast<size_t>(n) * d + 2ull * n * k + static_cast<size_t>(d) * k);
 }
@@ -334,6 +372,12 @@ bool fm_mma_shape(int n, int d, int k) {
 template <typename T>
 wk_status run_fm16(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
                    int n, int d, int k, float eps, unsigned* status, cudaStream_t st) {
+  if (!use_fm_mma_sync()) {
+    if (n == 512 && d == 160 && k == 64) return run_fm_tc<FmTcC4, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+    if (n == 256 && d == 160 && k == 32) return run_fm_tc<FmTcC3, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+    if (n == 64 && d == 128 && k == 16) return run_fm_tc<FmTcC2, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+    if (n == 720 && d == 32 && k == 24) return run_fm_tc<FmTcC5, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  }
   if (n == 512 && d == 160 && k == 64) return run_fm_mma<FmC4, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
   if (n == 256 && d == 160 && k == 32) return run_fm_mma<FmC3, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
   if (n == 64 && d == 128 && k == 16) return run_fm_mma<FmC2, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
