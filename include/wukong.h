@@ -114,7 +114,10 @@ typedef struct wk_stack wk_stack;
 /* Validates cfg, records the weight pointers of cfg->num_layers layers
  * (weights[0 .. num_layers-1]), converts the weights to the operand type when it
  * differs from dtype (a device copy the handle owns; the originals are then no
- * longer read), builds the TMA descriptors of the weights and allocates the
+ * longer read), folds the FMB LayerNorm's gamma / beta into the first MLP Linear
+ * of 16-bit stacks (a handle-owned copy W0 diag(gamma) and bias b0 + W0 beta: the
+ * same function, without per-example reads of gamma and beta), builds the TMA
+ * descriptors of the weights and allocates the
  * workspace for cfg->max_batch examples on the current device, in the operand
  * type: A0 [max_batch, n*k], two MLP activation buffers [max_batch, max hidden],
  * the concat buffer [max_batch, n, d] and two layer buffers [max_batch, n, d].
@@ -169,6 +172,8 @@ WK_API wk_status wk_stack_kernel_times(wk_stack* h, double* total_ms, int64_t* l
 
 /* FMB front: A0[b] = LN( flatten( X_b (X_b^T Y) ) ) * gamma + beta, b < batch.
  * X [batch, n, d], Y [n, k] (dtype), gamma/beta [n*k] fp32, A0 [batch, n*k] dtype.
+ * gamma and beta may both be NULL: A0 then holds the normalised values (a stack
+ * passes NULL, having folded gamma and beta into its first MLP Linear).
  * The FM runs per example on the tensor cores (bf16) with fp32 accumulation;
  * X_b^T Y is rounded to bf16 before the second product (bf16 path only). */
 WK_API wk_status wk_fm_ln(const void* X, const void* Y, const float* gamma, const float* beta, void* A0, int64_t batch,

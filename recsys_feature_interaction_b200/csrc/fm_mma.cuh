@@ -339,8 +339,9 @@ __global__ void __launch_bounds__(FM_THREADS, 1)
       for (int q4 = tid; q4 < rows * C::KC / 4; q4 += 256) {
         const int r = (q4 * 4) / C::KC, col = (q4 * 4) - r * C::KC;
         const float4 v = *reinterpret_cast<const float4*>(zpart + r * C::KCP + col);
-        const float4 gm = __ldg(reinterpret_cast<const float4*>(gamma + base) + q4);
-        const float4 bt = __ldg(reinterpret_cast<const float4*>(beta + base) + q4);
+        // gamma == nullptr: the affine step lives in the next Linear (normalised values only)
+        const float4 gm = gamma ? __ldg(reinterpret_cast<const float4*>(gamma + base) + q4) : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 bt = gamma ? __ldg(reinterpret_cast<const float4*>(beta + base) + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
         uint2 o;
         o.x = Half16<T>::pack2(v.x * gm.x + bt.x, v.y * gm.y + bt.y);
         o.y = Half16<T>::pack2(v.z * gm.z + bt.z, v.w * gm.w + bt.w);

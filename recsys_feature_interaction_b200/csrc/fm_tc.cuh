@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
       named_bar(1, 128);
       const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
       T* ab = A0 + b * (C::N * C::K);
+      const bool affine = gamma != nullptr;
 #pragma unroll 1
       for (int c = 0; c < C::NCH; ++c) {
         const int row = c * C::R + q * 32 + lane;
@@ -319,16 +320,18 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
           tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
           tmem_ld_wait();
           if (row < C::N) {
-            const float* g = gamma + row * C::K + h * 32;
-            const float* bt = beta + row * C::K + h * 32;
+            const float* g = affine ? gamma + row * C::K + h * 32 : nullptr;
+            const float* bt = affine ? beta + row * C::K + h * 32 : nullptr;
             T* o = ab + row * C::K + h * 32;
 #pragma unroll
             for (int j = 0; j < 32; j += 8) {
               if (h * 32 + j < C::K) {
-                const float4 g0 = __ldg(reinterpret_cast<const float4*>(g + j));
-                const float4 g1 = __ldg(reinterpret_cast<const float4*>(g + j + 4));
-                const float4 b0 = __ldg(reinterpret_cast<const float4*>(bt + j));
-                const float4 b1 = __ldg(reinterpret_cast<const float4*>(bt + j + 4));
+                // gamma == nullptr: the affine step lives in the next Linear (normalised values only)
+                const float4 one = make_float4(1.f, 1.f, 1.f, 1.f), zero = make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 g0 = affine ? __ldg(reinterpret_cast<const float4*>(g + j)) : one;
+                const float4 g1 = affine ? __ldg(reinterpret_cast<const float4*>(g + j + 4)) : one;
+                const float4 b0 = affine ? __ldg(reinterpret_cast<const float4*>(bt + j)) : zero;
+                const float4 b1 = affine ? __ldg(reinterpret_cast<const float4*>(bt + j + 4)) : zero;
                 uint4 u;
                 u.x = Half16<T>::pack2((__uint_as_float(r[j + 0]) - mean) * rstd * g0.x + b0.x,
                                        (__uint_as_float(r[j + 1]) - mean) * rstd * g0.y + b0.y);

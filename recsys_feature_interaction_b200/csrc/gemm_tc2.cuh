@@ -48,8 +48,11 @@ __device__ __forceinline__ void gemm2_tile_coords(const GemmParams& p, int tile,
   nt = local / gm;
 }
 
-// p.num_m_tiles counts 256-row tiles; p.num_n_tiles 256-column tiles.
-template <typename T, typename TO>
+// p.num_m_tiles counts 256-row tiles, p.num_n_tiles tiles of p.mma_n columns
+// (256, or E = floor(256/d) whole embedding rows of the last Linear when ROWLN: then
+// the epilogue adds the bias and the residual, applies the output LayerNorm and tmC
+// addresses the layer output [M, n*d]).
+template <typename T, typename TO, bool ROWLN = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
@@ -107,13 +110,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         int mt, nt;
         gemm2_tile_coords(p, tile, mt, nt);
         const int arow = mt * GEMM2_BM + static_cast<int>(rank) * 128;
-        const int brow = nt * GEMM2_BN + static_cast<int>(rank) * 128;
+        const int brow = nt * p.mma_n + static_cast<int>(rank) * (p.mma_n / 2);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, p.status)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (GEMM2_A_STAGE + GEMM2_B_STAGE));
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (GEMM2_A_STAGE + static_cast<uint32_t>(p.mma_n / 2) * 128u));
           const uint32_t fbar = full0 + static_cast<uint32_t>(s) * 8u;
           tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow);
           tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow);
@@ -130,7 +133,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_f16kind_f32(GEMM2_BM, GEMM2_BN, 0, 0, Half16<T>::kBF16);
+      const uint32_t idesc = idesc_f16kind_f32(GEMM2_BM, p.mma_n, 0, 0, Half16<T>::kBF16);
       const uint32_t empty_own = smem_u32(empty), empty_peer = mapa_shared(smem_u32(empty), 1);
       const uint32_t tfull_own = smem_u32(tfull), tfull_peer = mapa_shared(smem_u32(tfull), 1);
       int s = 0;
@@ -193,7 +196,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       if (!mbar_wait(&tfull[acc], acc_ph, p.status)) break;
       tc_fence_after();
       const int row0 = mt * GEMM2_BM + static_cast<int>(rank) * 128 + q * 32;
-      for (int c = 0; c < GEMM2_BN / 32; ++c) {
+      if constexpr (ROWLN) {
+        const int brow = row0 + lane;  // example
+        const bool valid = brow < p.M;
+        for (int e = 0; e < p.E; ++e) {
+          const int r = nt * p.E + e;  // embedding row of the FMB block
+          if (r >= p.ln_rows) break;
+          const T* xr = static_cast<const T*>(p.resid) + (static_cast<int64_t>(brow) * p.ln_n + r) * p.d;
+          const uint32_t taddr =
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * GEMM2_BN + e * p.d);
+          row_ln_epilogue<T, TO>(taddr, p.d, valid, valid ? xr : nullptr, p.bias ? p.bias + r * p.d : nullptr, p.ln_g,
+                                 p.ln_b, p.ln_eps, bufs, EPI_BUF, buf, lane, [&](int c, uint8_t* sb) {
+                                   tma_store_2d(&tmC, sb, r * p.d + c * 32, row0);
+                                   bulk_commit();
+                                 });
+        }
+      }
+      for (int c = 0; c < (ROWLN ? 0 : GEMM2_BN / 32); ++c) {
         const int col0 = nt * GEMM2_BN + c * 32;
         if (col0 >= p.N) break;
         uint32_t r[32];

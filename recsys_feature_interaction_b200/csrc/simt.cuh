@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256) fm_ln_simt(const T* __restrict__ X, const
     }
     const float rstd = rsqrtf(block_sum_256(q, red) / static_cast<float>(nk) + eps);
     for (int o = threadIdx.x; o < nk; o += blockDim.x)
-      st_f(A0, b * nk + o, (sF[o] - mean) * rstd * gamma[o] + beta[o]);
+      st_f(A0, b * nk + o, gamma ? (sF[o] - mean) * rstd * gamma[o] + beta[o] : (sF[o] - mean) * rstd);
   }
 }
 

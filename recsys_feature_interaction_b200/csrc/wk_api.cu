@@ -187,26 +187,63 @@ bool map_lcb_out(const DevInfo* dv, CUtensorMap* m, const void* cat, uint64_t ro
                   es == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int MODE, typename T, typename TO>
+template <int MODE, typename T, typename TO, bool ROWLN = false>
 wk_status run_gemm_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
   constexpr uint32_t smem = gemm_smem_bytes<TO>();
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc_kernel<MODE, T, TO>), smem);
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc_kernel<MODE, T, TO, ROWLN>), smem);
   if (s != WK_OK) return s;
   if (p.num_tiles <= 0) return WK_OK;
   const int grid = std::min(p.num_tiles, dv->sms);
-  gemm_tc_kernel<MODE, T, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  gemm_tc_kernel<MODE, T, TO, ROWLN><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
 }
 
-template <typename T, typename TO>
+template <typename T, typename TO, bool ROWLN = false>
 wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
   constexpr uint32_t smem = gemm2_smem_bytes<TO>();
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO>), smem);
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, ROWLN>), smem);
   if (s != WK_OK) return s;
   if (p.num_tiles <= 0) return WK_OK;
   const int pairs = std::min(p.num_tiles, dv->sms / 2);
-  gemm_tc2_kernel<T, TO><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  gemm_tc2_kernel<T, TO, ROWLN><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
+}
+
+// The end of each layer (residual + output LayerNorm) runs inside the epilogues of
+// the last FMB Linear and of the LCB unless the environment sets WK_FUSED_LN=0.
+bool use_fused_ln() {
+  static const bool on = [] {
+    const char* e = getenv("WK_FUSED_LN");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Last FMB Linear tiled by E = floor(256/d) whole embedding rows, epilogue finishing
+// the layer for rows 0..n_f-1.
+GemmParams mlp2_rowln_params(int64_t M, int K, int n, int d, int n_f, const float* bias, const void* resid,
+                             const float* g, const float* b, float eps, unsigned* status) {
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = n_f * d;
+  p.K = K;
+  p.d = d;
+  p.E = GEMM2_BN / d;
+  p.mma_n = p.E * d;
+  p.num_m_tiles = static_cast<int>((M + GEMM2_BM - 1) / GEMM2_BM);
+  p.num_n_tiles = (n_f + p.E - 1) / p.E;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  p.num_kb = (K + GEMM2_BK - 1) / GEMM2_BK;
+  p.group_m = 8;
+  p.bias = bias;
+  p.status = status;
+  p.resid = resid;
+  p.ln_g = g;
+  p.ln_b = b;
+  p.ln_eps = eps;
+  p.ln_n = n;
+  p.ln_rows = n_f;
+  return p;
 }
 
 // The CTA-pair GEMM (256-row tiles) serves every M above one 128-row tile unless
@@ -489,6 +526,9 @@ struct wk_stack {
   // TMA descriptors of the tensor-core path
   bool tc_mlp = false, tc_lcb = false;
   bool pair = false;                            // MLP Linears on CTA pairs (gemm_tc2.cuh)
+  bool fused = false;                           // residual + LN in the last Linear / LCB epilogues
+  std::vector<GemmMaps> last_maps;              // [layer]: fused last Linear (B box mma_n/2 rows, C = Xs[l%2])
+  CUtensorMap lcbC_x[2];                        // LCB rows n_f.. of Xs[0] / Xs[1]
   std::vector<std::vector<GemmMaps>> mlp_maps;  // [layer][j]
   std::vector<CUtensorMap> lcbA;                // [layer]
   CUtensorMap lcbB_ws[2];
@@ -609,6 +649,23 @@ wk_status build_maps(wk_stack* h) {
         if (!ok) return WK_ERR_UNSUPPORTED;
       }
   }
+  h->fused = h->tc_mlp && h->pair && h->tc_lcb && use_fused_ln() && d <= GEMM2_BN;
+  if (h->fused) {
+    const int E = GEMM2_BN / d;
+    h->last_maps.resize(L);
+    for (int l = 0; l < L; ++l) {
+      GemmMaps& mp = h->last_maps[l];
+      const int j = m - 1;
+      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+      const bool ok = map_kmajor<T>(dv, &mp.A, in, h->dims[j], B, GEMM_BM) &&
+                      map_kmajor<T>(dv, &mp.B, h->W[l][j], h->dims[j], h->dims[j + 1], (E * d) / 2) &&
+                      map_out<T>(dv, &mp.C, h->Xs[l % 2], static_cast<uint64_t>(c.n_f) * d, B, nd);
+      if (!ok) return WK_ERR_UNSUPPORTED;
+    }
+    if (!map_lcb_out<T>(dv, &h->lcbC_x[0], h->Xs[0], n, d, c.n_f, c.n_l, B) ||
+        !map_lcb_out<T>(dv, &h->lcbC_x[1], h->Xs[1], n, d, c.n_f, c.n_l, B))
+      return WK_ERR_UNSUPPORTED;
+  }
   if (h->tc_lcb) {
     h->lcbA.resize(L);
     bool ok = true;
@@ -639,6 +696,10 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
   } else if (h->tc_lcb && !map_lcb_x<T>(dv, &lcb_x0, X, n, d, batch)) {
     return WK_ERR_CUDA;
   }
+  CUtensorMap out_last, out_lcb;  // the caller's output as the fused epilogues' destination
+  if (h->fused && (!map_out<IO>(dv, &out_last, out, static_cast<uint64_t>(c.n_f) * d, batch, nd) ||
+                   !map_lcb_out<IO>(dv, &out_lcb, out, n, d, c.n_f, c.n_l, batch)))
+    return WK_ERR_CUDA;
   for (int l = 0; l < L && s == WK_OK; ++l) {
     const bool last = l == L - 1;
     const T* xin = static_cast<const T*>(l == 0 ? x0 : h->Xs[(l - 1) % 2]);
@@ -647,7 +708,8 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
       s = run_fm16<T>(dv, xin, static_cast<const T*>(h->Y[l]), h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, n, d,
                       k, h->eps, h->status, st);
     }
-    for (int j = 0; j < m && s == WK_OK; ++j) {  // 2. MLP
+    const int m_plain = h->fused ? m - 1 : m;  // the fused path runs the last Linear below
+    for (int j = 0; j < m_plain && s == WK_OK; ++j) {  // 2. MLP
       ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
       const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
       const bool lastj = j == m - 1;
@@ -665,6 +727,44 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
                                 static_cast<T*>(o), batch, h->dims[j], h->dims[j + 1], ldc, relu, st);
     }
     if (s != WK_OK) break;
+    if (h->fused) {
+      // 2'. last Linear + residual + LN -> rows 0..n_f-1 of X_{i+1};
+      // 3'. LCB + residual + LN -> rows n_f..n-1 of X_{i+1}
+      {
+        ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+        const GemmParams p = mlp2_rowln_params(batch, h->dims[m - 1], n, d, c.n_f, h->b[l][m - 1], xin, h->g2[l],
+                                               h->b2[l], h->eps, h->status);
+        GemmMaps mp = h->last_maps[l];
+        if (last) {
+          mp.C = out_last;
+          s = run_gemm_tc2<T, IO, true>(dv, mp, p, st);
+        } else {
+          s = run_gemm_tc2<T, T, true>(dv, mp, p, st);
+        }
+      }
+      if (s != WK_OK) break;
+      {
+        ProfScope ps(h, WK_KERNEL_LCB, st);
+        GemmParams p = lcb_params(batch, n, d, c.n_l, h->status);
+        p.resid = xin;
+        p.ln_g = h->g2[l];
+        p.ln_b = h->b2[l];
+        p.ln_eps = h->eps;
+        p.ln_n = n;
+        p.ln_row0 = c.n_f;
+        GemmMaps mp;
+        mp.A = h->lcbA[l];
+        mp.B = (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2];
+        if (last) {
+          mp.C = out_lcb;
+          s = run_gemm_tc<MODE_LCB, T, IO, true>(dv, mp, p, st);
+        } else {
+          mp.C = h->lcbC_x[l % 2];
+          s = run_gemm_tc<MODE_LCB, T, T, true>(dv, mp, p, st);
+        }
+      }
+      continue;
+    }
     {  // 3. LCB
       ProfScope ps(h, WK_KERNEL_LCB, st);
       if (h->tc_lcb) {
@@ -937,10 +1037,17 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   }
 
   auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
-  // weights converted to the operand type once (bf16 stacks computing with fp16 operands, or the reverse)
-  if (h->io != h->op) {
-    size_t per_layer = up(static_cast<size_t>(n) * k * 2) + up(static_cast<size_t>(cfg->n_l) * n * 2);
-    for (int j = 0; j < m; ++j) per_layer += up(static_cast<size_t>(dims[j]) * dims[j + 1] * 2);
+  // 16-bit stacks: weights in the operand type (converted once when the caller's type
+  // differs), and the FMB LayerNorm's gamma / beta folded into the first Linear:
+  // W0' = W0 diag(gamma), b0' = b0 + W0 beta (the FM kernel then stores only the
+  // normalised values, with no per-example reads of gamma and beta).
+  if (h->op != WK_F32) {
+    const bool conv_all = h->io != h->op;
+    size_t per_layer = up(static_cast<size_t>(dims[0]) * dims[1] * 2) + up(static_cast<size_t>(dims[1]) * 4);
+    if (conv_all) {
+      per_layer += up(static_cast<size_t>(n) * k * 2) + up(static_cast<size_t>(cfg->n_l) * n * 2);
+      for (int j = 1; j < m; ++j) per_layer += up(static_cast<size_t>(dims[j]) * dims[j + 1] * 2);
+    }
     if (cudaMalloc(&h->wcopy, per_layer * L) != cudaSuccess) {
       cudaGetLastError();
       delete h;
@@ -955,10 +1062,43 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
       if (cs != WK_OK) st = cs;
       return dst;
     };
+    const int64_t nvec = static_cast<int64_t>(dims[0]) * dims[1] / 8;
+    const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nvec + 255) / 256, dv->sms * 16ll)));
+    const int bias_blocks = static_cast<int>(std::max(1, std::min(dims[1] / 8 + 1, dv->sms * 16)));
     for (int l = 0; l < L; ++l) {
-      h->Y[l] = conv(h->Y[l], static_cast<int64_t>(n) * k);
-      h->WL[l] = conv(h->WL[l], static_cast<int64_t>(cfg->n_l) * n);
-      for (int j = 0; j < m; ++j) h->W[l][j] = conv(h->W[l][j], static_cast<int64_t>(dims[j]) * dims[j + 1]);
+      if (conv_all) {
+        h->Y[l] = conv(h->Y[l], static_cast<int64_t>(n) * k);
+        h->WL[l] = conv(h->WL[l], static_cast<int64_t>(cfg->n_l) * n);
+        for (int j = 1; j < m; ++j) h->W[l][j] = conv(h->W[l][j], static_cast<int64_t>(dims[j]) * dims[j + 1]);
+      }
+      const void* w0 = h->W[l][0];
+      void* w0f = p;
+      p += up(static_cast<size_t>(dims[0]) * dims[1] * 2);
+      float* b0f = reinterpret_cast<float*>(p);
+      p += up(static_cast<size_t>(dims[1]) * 4);
+      const float* g = h->g1[l];
+      const float* be = h->b1[l];
+      if (h->io == WK_BF16 && h->op == WK_F16)
+        fold_scale_cols_kernel<bf16, f16><<<blocks, 256>>>(static_cast<const bf16*>(w0), g, static_cast<f16*>(w0f),
+                                                            dims[1], dims[0]);
+      else if (h->io == WK_F16 && h->op == WK_BF16)
+        fold_scale_cols_kernel<f16, bf16><<<blocks, 256>>>(static_cast<const f16*>(w0), g, static_cast<bf16*>(w0f),
+                                                            dims[1], dims[0]);
+      else if (h->op == WK_F16)
+        fold_scale_cols_kernel<f16, f16><<<blocks, 256>>>(static_cast<const f16*>(w0), g, static_cast<f16*>(w0f),
+                                                           dims[1], dims[0]);
+      else
+        fold_scale_cols_kernel<bf16, bf16><<<blocks, 256>>>(static_cast<const bf16*>(w0), g, static_cast<bf16*>(w0f),
+                                                             dims[1], dims[0]);
+      if (h->io == WK_BF16)
+        fold_bias_kernel<bf16><<<bias_blocks, 256>>>(static_cast<const bf16*>(w0), be, h->b[l][0], b0f, dims[1], dims[0]);
+      else
+        fold_bias_kernel<f16><<<bias_blocks, 256>>>(static_cast<const f16*>(w0), be, h->b[l][0], b0f, dims[1], dims[0]);
+      if (launch_status() != WK_OK) st = WK_ERR_CUDA;
+      h->W[l][0] = w0f;
+      h->b[l][0] = b0f;
+      h->g1[l] = nullptr;  // the FM stores the normalised values
+      h->b1[l] = nullptr;
     }
     if (st == WK_OK && cudaDeviceSynchronize() != cudaSuccess) st = WK_ERR_CUDA;
     if (st != WK_OK) {
@@ -1157,7 +1297,8 @@ wk_status wk_fm_ln(const void* X, const void* Y, const float* gamma, const float
                    int32_t n, int32_t d, int32_t k, wk_dtype dtype, float eps, wk_stream_t stream) {
   if (batch < 0 || n < 1 || d < 1 || k < 1) return WK_ERR_INVALID_ARG;
   if (batch == 0) return WK_OK;
-  if (!X || !Y || !gamma || !beta || !A0 || !al16(X) || !al16(Y) || !al16(A0) || !al16(gamma) || !al16(beta))
+  if (!X || !Y || !A0 || !al16(X) || !al16(Y) || !al16(A0) || (!gamma) != (!beta) || (gamma && !al16(gamma)) ||
+      (beta && !al16(beta)))
     return WK_ERR_INVALID_ARG;
   if (dtype != WK_F32 && dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
   if (d % 8 != 0 || k % 2 != 0 || !fm_supported(n, d, k, dtype != WK_F32)) return WK_ERR_UNSUPPORTED;

@@ -27,6 +27,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"])
     ap.add_argument("--layer-linear", type=int, default=0, help="which MLP Linear (mlp_gemm)")
+    ap.add_argument("--no-affine", action="store_true", help="fm_ln without gamma/beta (as a stack runs it)")
     args = ap.parse_args()
 
     import torch
@@ -49,7 +50,8 @@ def main():
         A0 = torch.empty((B, n * k), dtype=tdt, device=dev)
 
         def run():
-            wk.wk_fm_ln(X, Y, w["fmb_gamma"], w["fmb_beta"], A0, B, n, d, k, args.dtype)
+            wk.wk_fm_ln(X, Y, None if args.no_affine else w["fmb_gamma"], None if args.no_affine else w["fmb_beta"],
+                        A0, B, n, d, k, args.dtype)
         flops = 4 * n * d * k * B
         bytes_ = (n * d + n * k) * es * B
     elif args.kernel == "mlp_gemm":

@@ -154,3 +154,17 @@ def test_res_ln(rows, d, dt):
     tol = {"bf16": 1e-2, "f16": 2e-3, "f32": 1e-5}[dt]
     for r in range(0, rows, 7):
         assert max_scaled_err(got[r], oracle.layernorm(y[r], f64(g), f64(be))) <= tol, r
+
+
+@pytest.mark.parametrize("batch,n,d,k", [(160, 512, 160, 64), (170, 720, 32, 24)])
+def test_fm_ln_without_affine(batch, n, d, k):
+    """NULL gamma/beta: A0 holds the normalised FM values (how a stack calls it)."""
+    X = host_normal((batch, n, d), 26, dtype="f16")
+    Y = host_normal((n, k), 27, std=1.0 / np.sqrt(n), dtype="f16")
+    A0 = torch.full((batch, n * k), float("nan"), dtype=torch.float16, device="cuda")
+    wk.wk_fm_ln(to_dev(X), to_dev(Y), None, None, A0, batch, n, d, k, "f16")
+    _status_ok()
+    got = f64(A0)
+    for b in (0, batch // 2, batch - 1):
+        ref = oracle.layernorm(oracle.fm(f64(X[b]), f64(Y)).reshape(-1))
+        assert max_scaled_err(got[b], ref) <= 4e-3, b

@@ -136,8 +136,9 @@ def test_profiling_counts_launches():
         t = wk.wk_stack_kernel_times(st.h)
         m = len(cfg["hidden"]) + 1
         assert t["fm_ln"][1] == cfg["layers"] and t["mlp_gemm"][1] == cfg["layers"] * m
-        assert t["lcb"][1] == cfg["layers"] and t["res_ln"][1] == cfg["layers"]
-        assert all(ms > 0 for ms, _ in t.values())
+        # the residual + LayerNorm runs in its own kernel, or inside the last Linear and LCB epilogues
+        assert t["lcb"][1] == cfg["layers"] and t["res_ln"][1] in (0, cfg["layers"])
+        assert all(ms > 0 for ms, count in t.values() if count)
     finally:
         st.close()
 
