@@ -159,18 +159,15 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from recsys_feature_interaction_b200 import replicas
+
+    rank, world, local = replicas.rank_info()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
 
-    import datetime
-
     import torch
-    import torch.distributed as dist
 
     import recsys_feature_interaction_b200 as wk
     from recsys_feature_interaction_b200 import build as wk_build
@@ -178,29 +175,23 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    replicas.init("nccl", device=dev)
     wk_build.build()
 
     cfg = C.CONFIGS[WORKLOAD]
     B = cfg["batch"]
     layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
     h = wk.wk_stack_create(cfg, layers, max_batch=B)
-    # rank r works on examples [r*B, (r+1)*B) of the synthetic stream
-    X = C.make_x_dev(cfg, B, device=dev, first_example=rank * B)
+    # rank r works on examples [r*B, (r+1)*B) of the synthetic stream (no collective on the data path)
+    first, _ = replicas.example_range(rank, world, B)
+    X = C.make_x_dev(cfg, B, device=dev, first_example=first)
     out = torch.empty_like(X)
     stream = torch.cuda.current_stream(dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = replicas.barrier
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, device=dev)
 
     for _ in range(args.warmup):
         wk.wk_stack_forward(h, X, out, stream=stream)
@@ -255,8 +246,10 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {"workload": WORKLOAD + ": " + workload_desc(cfg), "per_gpu_batch": B,
+                       "precision": "bf16 inputs, weights and outputs; fp16 tensor-core operands and "
+                                    "intermediates; fp32 accumulation and LayerNorm statistics",
                        "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
                        "l2": "inputs larger than L2 (X 671 MB, weights 23.6 GB per GPU)"},
             "tflops_per_gpu": tflops,
@@ -278,9 +271,7 @@ def main():
                                               "whole stack" % (cfg["layers"], dt)}
         print(json.dumps(line), flush=True)
     wk.wk_stack_destroy(h)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finish()
 
 
 if __name__ == "__main__":

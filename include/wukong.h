@@ -157,7 +157,7 @@ WK_API const char* wk_status_string(wk_status s);
 /* ---- per-kernel timing of a handle's forwards (CUDA events on the launch stream) ---- */
 
 typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
-               WK_KERNEL_COUNT = 4 } wk_kernel_kind;
+               WK_KERNEL_CONVERT = 4, WK_KERNEL_COUNT = 5 } wk_kernel_kind;
 
 /* enable != 0: every later forward records a start/stop event pair around each
  * kernel launch on its stream (adds no synchronisation). */

@@ -20,8 +20,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
 
 WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
 WK_F32, WK_BF16, WK_F16 = 0, 1, 2
-WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_COUNT = range(5)
-KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln")
+WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_CONVERT, WK_KERNEL_COUNT = range(6)
+KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert")
 
 
 class WkError(RuntimeError):

@@ -689,6 +689,7 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
   const void* x0 = X;
   CUtensorMap lcb_x0;
   if (sizeof(IO) != sizeof(T) || Half16<IO>::kBF16 != Half16<T>::kBF16) {
+    ProfScope ps(h, WK_KERNEL_CONVERT, st);
     s = run_convert<IO, T>(dv, X, h->Xs[1], rows * d, st);  // the input in the operand type
     if (s != WK_OK) return s;
     x0 = h->Xs[1];
