@@ -34,6 +34,34 @@ METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack fwd, 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic of the CTA-pair MLP GEMM per launch, from one ncu capture of each of the
+# three Linears of the workload (dram__bytes_read.sum + dram__bytes_write.sum, averaged
+# over the three launches; profiles/mlp_gemm_pair_c4_shapes.md). It describes the kernel
+# sources it was taken on: when their hash differs, the bench reports null.
+GEMM_TRAFFIC = {
+    "sources": ["recsys_feature_interaction_b200/csrc/gemm_tc2.cuh", "recsys_feature_interaction_b200/csrc/common.cuh"],
+    "sha256": None,
+    "bytes_per_launch": None,
+}
+
+
+def sources_sha256(paths):
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic():
+    """DRAM bytes per MLP GEMM launch from the committed capture, or None when the
+    kernel sources have changed since."""
+    if GEMM_TRAFFIC["bytes_per_launch"] is None or GEMM_TRAFFIC["sha256"] != sources_sha256(GEMM_TRAFFIC["sources"]):
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -256,7 +284,7 @@ def main():
             "pct_of_bf16_peak": 100.0 * tflops / peak,
             "peak_source": "%s bf16_tflops_sustained" % peak_src,
             "roofline": {"kernel": "mlp_gemm (tcgen05)", "bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None, "traffic": None,
+                         "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None, "traffic": gemm_traffic(),
                          "peak_note": "%s sustained cuBLAS bf16" % peak_src},
             "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
             "clocks": clocks,

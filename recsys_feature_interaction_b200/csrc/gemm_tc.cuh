@@ -70,6 +70,9 @@ struct GemmParams {
   const float* ln_b;
   float ln_eps;
   int ln_n, ln_row0, ln_rows;
+  // CTA-pair GEMM: 1 = operand loads carry L2 hints (A, the activations, kept in L2
+  // across the waves of a raster group; B, the weights, streamed through)
+  int l2hint;
 };
 
 __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int mode, int& mt, int& nt) {

@@ -29,6 +29,8 @@ constexpr int GEMM2_BM = 256;  // rows per pair (128 per CTA)
 constexpr int GEMM2_BN = 256;
 constexpr int GEMM2_BK = 64;
 constexpr int GEMM2_STAGES = 6;
+constexpr int GEMM2_GROUP_M = 8;  // M tiles per raster group (tiles walk M fastest inside a group)
+constexpr int GEMM2_L2_HINT = 0;  // default of GemmParams::l2hint
 constexpr uint32_t GEMM2_A_STAGE = 128 * GEMM2_BK * 2;  // 16 KB: this CTA's 128 rows
 constexpr uint32_t GEMM2_B_STAGE = 128 * GEMM2_BK * 2;  // 16 KB: this CTA's half of N
 
@@ -103,6 +105,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // leader's full[0]
+      const uint64_t pol_a = l2_policy_evict_last();
+      const uint64_t pol_b = l2_policy_evict_first();
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -118,8 +122,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (GEMM2_A_STAGE + static_cast<uint32_t>(p.mma_n / 2) * 128u));
           const uint32_t fbar = full0 + static_cast<uint32_t>(s) * 8u;
-          tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow);
-          tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow);
+          if (p.l2hint) {
+            tma_load_2d_pair_hint(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow, pol_a);
+            tma_load_2d_pair_hint(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow, pol_b);
+          } else {
+            tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow);
+            tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow);
+          }
           if (++s == GEMM2_STAGES) {
             s = 0;
             ph ^= 1u;

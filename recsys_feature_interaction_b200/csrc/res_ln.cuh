@@ -35,10 +35,16 @@ struct Vec8<float> {
 
 template <>
 struct Vec8<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
-    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  static __device__ __forceinline__ void unpack(const uint4& a, float (&v)[8]) {
     v[0] = bf16_lo(a.x); v[1] = bf16_hi(a.x); v[2] = bf16_lo(a.y); v[3] = bf16_hi(a.y);
     v[4] = bf16_lo(a.z); v[5] = bf16_hi(a.z); v[6] = bf16_lo(a.w); v[7] = bf16_hi(a.w);
+  }
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), v);
+  }
+  // p: 16-byte aligned shared memory
+  static __device__ __forceinline__ void load_shared(const uint8_t* p, float (&v)[8]) {
+    unpack(*reinterpret_cast<const uint4*>(p), v);
   }
   static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
     uint4 a;
@@ -52,14 +58,20 @@ struct Vec8<__nv_bfloat16> {
 
 template <>
 struct Vec8<__half> {
-  static __device__ __forceinline__ void load(const __half* p, float (&v)[8]) {
-    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  static __device__ __forceinline__ void unpack(const uint4& a, float (&v)[8]) {
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       v[2 * i] = Half16<__half>::lo(w[i]);
       v[2 * i + 1] = Half16<__half>::hi(w[i]);
     }
+  }
+  static __device__ __forceinline__ void load(const __half* p, float (&v)[8]) {
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), v);
+  }
+  // p: 16-byte aligned shared memory
+  static __device__ __forceinline__ void load_shared(const uint8_t* p, float (&v)[8]) {
+    unpack(*reinterpret_cast<const uint4*>(p), v);
   }
   static __device__ __forceinline__ void store(__half* p, const float (&v)[8]) {
     uint4 a;

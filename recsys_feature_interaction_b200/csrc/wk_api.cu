@@ -31,7 +31,9 @@
 #include "fm_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
+#include "lcb_tc.cuh"
 #include "res_ln.cuh"
+#include "res_ln_ring.cuh"
 #include "simt.cuh"
 
 using namespace wk;
@@ -209,12 +211,15 @@ wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& 
   return launch_status();
 }
 
-// The end of each layer (residual + output LayerNorm) runs inside the epilogues of
-// the last FMB Linear and of the LCB unless the environment sets WK_FUSED_LN=0.
+// With WK_FUSED_LN=1 in the environment, the end of each layer (residual + output
+// LayerNorm) runs inside the epilogues of the last FMB Linear and of the LCB instead
+// of a separate residual + LayerNorm pass. Off by default: tiling the last Linear by
+// whole embedding rows caps its MMA width at d (160 of 256 columns on the 8-layer
+// d=160 stack), which costs more tensor time than the separate pass moves in bytes.
 bool use_fused_ln() {
   static const bool on = [] {
     const char* e = getenv("WK_FUSED_LN");
-    return !(e && e[0] == '0');
+    return e && e[0] == '1';
   }();
   return on;
 }
@@ -256,6 +261,28 @@ bool use_pair_gemm(int64_t M) {
   return enabled && M > GEMM_BM;
 }
 
+// M tiles per raster group of the CTA-pair GEMM (tiles walk M fastest inside a group
+// of group_m M tiles, so a wave shares both operand panels through L2);
+// WK_GEMM_GROUP_M overrides the default GEMM2_GROUP_M.
+int gemm2_group_m() {
+  static const int g = [] {
+    const char* e = getenv("WK_GEMM_GROUP_M");
+    const int v = e ? atoi(e) : 0;
+    return v >= 1 && v <= 64 ? v : GEMM2_GROUP_M;
+  }();
+  return g;
+}
+
+// L2 hints on the CTA-pair GEMM's operand loads (GemmParams::l2hint); WK_GEMM_L2_HINT
+// overrides the default GEMM2_L2_HINT.
+int gemm2_l2hint() {
+  static const int h = [] {
+    const char* e = getenv("WK_GEMM_L2_HINT");
+    return e ? (e[0] == '1' ? 1 : 0) : GEMM2_L2_HINT;
+  }();
+  return h;
+}
+
 GemmParams mlp2_params(int64_t M, int K, int N, const float* bias, int relu, unsigned* status) {
   GemmParams p{};
   p.M = static_cast<int>(M);
@@ -265,7 +292,8 @@ GemmParams mlp2_params(int64_t M, int K, int N, const float* bias, int relu, uns
   p.num_n_tiles = (N + GEMM2_BN - 1) / GEMM2_BN;
   p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   p.num_kb = (K + GEMM2_BK - 1) / GEMM2_BK;
-  p.group_m = 8;
+  p.group_m = gemm2_group_m();
+  p.l2hint = gemm2_l2hint();
   p.mma_n = GEMM2_BN;
   p.bias = bias;
   p.relu = relu;
@@ -305,6 +333,33 @@ GemmParams lcb_params(int64_t batch, int n, int d, int n_l, unsigned* status) {
   p.mma_n = p.E * d;
   p.status = status;
   return p;
+}
+
+// The LCB with W_L resident in shared memory (lcb_tc.cuh) wherever its K panel fits,
+// unless the environment sets WK_LCB_RESIDENT=0 (then the streaming GEMM).
+bool use_lcb_resident() {
+  static const bool on = [] {
+    const char* e = getenv("WK_LCB_RESIDENT");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+template <typename T, typename TO>
+wk_status run_lcb_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
+  const uint32_t b_stage = static_cast<uint32_t>(p.E * p.dchunks) * 4096u;
+  const int stages = lcb_tc_stages<TO>(p.num_kb, b_stage);
+  if (!use_lcb_resident() || p.num_kb > LCB_MAX_KB || stages < 2 || p.num_m_tiles > dv->sms)
+    return run_gemm_tc<MODE_LCB, T, TO>(dv, mp, p, st);
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(lcb_tc_kernel<T, TO>), static_cast<int>(LCB_SMEM_BUDGET));
+  if (s != WK_OK) return s;
+  if (p.num_tiles <= 0) return WK_OK;
+  // every CTA keeps one W_L tile: the grid is a multiple of the m-tile count
+  const int per_m = std::max(1, std::min(p.num_n_tiles, dv->sms / p.num_m_tiles));
+  const int grid = per_m * p.num_m_tiles;
+  const uint32_t smem = lcb_tc_fixed_bytes<TO>(p.num_kb) + static_cast<uint32_t>(stages) * b_stage;
+  lcb_tc_kernel<T, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p, stages);
+  return launch_status();
 }
 
 bool mlp_tc_ok(int64_t M, int K, int N, int64_t ldc) {
@@ -429,9 +484,30 @@ bool fm_supported(int n, int d, int k, bool sixteen_bit) {
 
 // ------------------------------------------------------------ residual + LN
 
+// The bulk-copy ring kernel for 16-bit inputs unless the environment sets
+// WK_RES_LN_RING=0 (then the register-only kernel, which also serves fp32).
+bool use_res_ln_ring() {
+  static const bool on = [] {
+    const char* e = getenv("WK_RES_LN_RING");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int D, typename TC, typename TR, typename TO>
 wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
-                       int64_t rows, float eps, cudaStream_t st) {
+                       int64_t rows, float eps, unsigned* status, cudaStream_t st) {
+  if constexpr (sizeof(TC) == 2 && sizeof(TR) == 2) {
+    if (use_res_ln_ring() && al16(cat) && al16(x)) {
+      using C = ResLnRing<D>;
+      wk_status s = smem_attr(dv, reinterpret_cast<const void*>(res_ln_ring_kernel<D, TC, TR, TO>), C::SMEM);
+      if (s != WK_OK) return s;
+      const int64_t tiles = (rows + C::R - 1) / C::R;
+      const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, dv->sms)));
+      res_ln_ring_kernel<D, TC, TR, TO><<<grid, C::THREADS, C::SMEM, st>>>(cat, x, g, b, out, rows, eps, status);
+      return launch_status();
+    }
+  }
   constexpr int VPR = D / 8;
   constexpr int G = res_ln_lanes(VPR);
   constexpr int rows_per_block = (256 / 32) * (32 / G) * ((VPR / G) >= 4 ? 2 : 4);
@@ -449,15 +525,15 @@ bool res_ln_d_ok(int d) {
 
 template <typename TC, typename TR, typename TO>
 wk_status run_res_ln(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
-                     int64_t rows, int d, float eps, cudaStream_t st) {
+                     int64_t rows, int d, float eps, unsigned* status, cudaStream_t st) {
   switch (d) {
-    case 16: return run_res_ln_d<16>(dv, cat, x, g, b, out, rows, eps, st);
-    case 32: return run_res_ln_d<32>(dv, cat, x, g, b, out, rows, eps, st);
-    case 64: return run_res_ln_d<64>(dv, cat, x, g, b, out, rows, eps, st);
-    case 128: return run_res_ln_d<128>(dv, cat, x, g, b, out, rows, eps, st);
-    case 160: return run_res_ln_d<160>(dv, cat, x, g, b, out, rows, eps, st);
-    case 192: return run_res_ln_d<192>(dv, cat, x, g, b, out, rows, eps, st);
-    case 256: return run_res_ln_d<256>(dv, cat, x, g, b, out, rows, eps, st);
+    case 16: return run_res_ln_d<16>(dv, cat, x, g, b, out, rows, eps, status, st);
+    case 32: return run_res_ln_d<32>(dv, cat, x, g, b, out, rows, eps, status, st);
+    case 64: return run_res_ln_d<64>(dv, cat, x, g, b, out, rows, eps, status, st);
+    case 128: return run_res_ln_d<128>(dv, cat, x, g, b, out, rows, eps, status, st);
+    case 160: return run_res_ln_d<160>(dv, cat, x, g, b, out, rows, eps, status, st);
+    case 192: return run_res_ln_d<192>(dv, cat, x, g, b, out, rows, eps, status, st);
+    case 256: return run_res_ln_d<256>(dv, cat, x, g, b, out, rows, eps, status, st);
     default: return WK_ERR_UNSUPPORTED;
   }
 }
@@ -773,7 +849,7 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
         mp.A = h->lcbA[l];
         mp.B = (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2];
         mp.C = h->lcbC;
-        s = run_gemm_tc<MODE_LCB, T, T>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
+        s = run_lcb_tc<T, T>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
       } else {
         s = run_lcb_simt<T, T>(static_cast<const T*>(h->WL[l]), xin, static_cast<T*>(h->cat), batch, n, d, c.n_f,
                                c.n_l, st);
@@ -784,9 +860,11 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
       ProfScope ps(h, WK_KERNEL_RES_LN, st);
       const T* cat = static_cast<const T*>(h->cat);
       if (last)
-        s = run_res_ln<T, T, IO>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<IO*>(out), rows, d, h->eps, st);
+        s = run_res_ln<T, T, IO>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<IO*>(out), rows, d, h->eps,
+                                h->status, st);
       else
-        s = run_res_ln<T, T, T>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<T*>(h->Xs[l % 2]), rows, d, h->eps, st);
+        s = run_res_ln<T, T, T>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<T*>(h->Xs[l % 2]), rows, d, h->eps,
+                               h->status, st);
     }
   }
   return s;
@@ -827,7 +905,7 @@ wk_status forward32(wk_stack* h, const float* X, float* out, int64_t batch, cuda
       ProfScope ps(h, WK_KERNEL_RES_LN, st);
       float* o = last ? out : static_cast<float*>(h->Xs[l % 2]);
       s = run_res_ln<float, float, float>(dv, static_cast<const float*>(h->cat), xin, h->g2[l], h->b2[l], o, rows, d,
-                                          h->eps, st);
+                                          h->eps, h->status, st);
     }
   }
   return s;
@@ -876,7 +954,7 @@ wk_status lcb16(const DevInfo* dv, const void* W_L, const void* X, void* concat,
   if (!map_kmajor<T>(dv, &mp.A, W_L, n, n_l, GEMM_BM) || !map_lcb_x<T>(dv, &mp.B, X, n, d, batch) ||
       !map_lcb_out<T>(dv, &mp.C, concat, n_f + n_l, d, n_f, n_l, batch))
     return WK_ERR_UNSUPPORTED;
-  return run_gemm_tc<MODE_LCB, T, T>(dv, mp, lcb_params(batch, n, d, n_l, dv->standalone_status), st);
+  return run_lcb_tc<T, T>(dv, mp, lcb_params(batch, n, d, n_l, dv->standalone_status), st);
 }
 
 // ------------------------------------------------- no-allocation layer forward
@@ -962,7 +1040,7 @@ wk_status layer_noalloc16(const DevInfo* dv, const wk_stack_config* c, const std
   }
   if (s == WK_OK) s = lcb16<T>(dv, w->W_L, X, cat, batch, n, d, c->n_f, c->n_l, st);
   if (s == WK_OK)
-    s = run_res_ln<T, T, T>(dv, cat, X, w->out_ln_gamma, w->out_ln_beta, out, batch * n, d, eps, st);
+    s = run_res_ln<T, T, T>(dv, cat, X, w->out_ln_gamma, w->out_ln_beta, out, batch * n, d, eps, status, st);
   return s;
 }
 
@@ -1039,15 +1117,19 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
 
   auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
   // 16-bit stacks: weights in the operand type (converted once when the caller's type
-  // differs), and the FMB LayerNorm's gamma / beta folded into the first Linear:
-  // W0' = W0 diag(gamma), b0' = b0 + W0 beta (the FM kernel then stores only the
-  // normalised values, with no per-example reads of gamma and beta).
-  if (h->op != WK_F32) {
+  // differs). With fp16 operands the FMB LayerNorm's gamma / beta are also folded
+  // into the first Linear: W0' = W0 diag(gamma), b0' = b0 + W0 beta (the FM kernel
+  // then stores only the normalised values, with no per-example reads of gamma and
+  // beta). bf16 operands keep the affine in the FM: rounding W0 diag(gamma) to bf16's
+  // 8-bit significand would add an error of the size the bf16 mode already spends.
+  const bool fold = h->op == WK_F16;
+  if (h->op != WK_F32 && (fold || h->io != h->op)) {
     const bool conv_all = h->io != h->op;
-    size_t per_layer = up(static_cast<size_t>(dims[0]) * dims[1] * 2) + up(static_cast<size_t>(dims[1]) * 4);
+    size_t per_layer = 0;
+    if (fold) per_layer += up(static_cast<size_t>(dims[0]) * dims[1] * 2) + up(static_cast<size_t>(dims[1]) * 4);
     if (conv_all) {
       per_layer += up(static_cast<size_t>(n) * k * 2) + up(static_cast<size_t>(cfg->n_l) * n * 2);
-      for (int j = 1; j < m; ++j) per_layer += up(static_cast<size_t>(dims[j]) * dims[j + 1] * 2);
+      for (int j = fold ? 1 : 0; j < m; ++j) per_layer += up(static_cast<size_t>(dims[j]) * dims[j + 1] * 2);
     }
     if (cudaMalloc(&h->wcopy, per_layer * L) != cudaSuccess) {
       cudaGetLastError();
@@ -1070,8 +1152,10 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
       if (conv_all) {
         h->Y[l] = conv(h->Y[l], static_cast<int64_t>(n) * k);
         h->WL[l] = conv(h->WL[l], static_cast<int64_t>(cfg->n_l) * n);
-        for (int j = 1; j < m; ++j) h->W[l][j] = conv(h->W[l][j], static_cast<int64_t>(dims[j]) * dims[j + 1]);
+        for (int j = fold ? 1 : 0; j < m; ++j)
+          h->W[l][j] = conv(h->W[l][j], static_cast<int64_t>(dims[j]) * dims[j + 1]);
       }
+      if (!fold) continue;
       const void* w0 = h->W[l][0];
       void* w0f = p;
       p += up(static_cast<size_t>(dims[0]) * dims[1] * 2);
@@ -1079,18 +1163,12 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
       p += up(static_cast<size_t>(dims[1]) * 4);
       const float* g = h->g1[l];
       const float* be = h->b1[l];
-      if (h->io == WK_BF16 && h->op == WK_F16)
+      if (h->io == WK_BF16)
         fold_scale_cols_kernel<bf16, f16><<<blocks, 256>>>(static_cast<const bf16*>(w0), g, static_cast<f16*>(w0f),
                                                             dims[1], dims[0]);
-      else if (h->io == WK_F16 && h->op == WK_BF16)
-        fold_scale_cols_kernel<f16, bf16><<<blocks, 256>>>(static_cast<const f16*>(w0), g, static_cast<bf16*>(w0f),
-                                                            dims[1], dims[0]);
-      else if (h->op == WK_F16)
+      else
         fold_scale_cols_kernel<f16, f16><<<blocks, 256>>>(static_cast<const f16*>(w0), g, static_cast<f16*>(w0f),
                                                            dims[1], dims[0]);
-      else
-        fold_scale_cols_kernel<bf16, bf16><<<blocks, 256>>>(static_cast<const bf16*>(w0), g, static_cast<bf16*>(w0f),
-                                                             dims[1], dims[0]);
       if (h->io == WK_BF16)
         fold_bias_kernel<bf16><<<bias_blocks, 256>>>(static_cast<const bf16*>(w0), be, h->b[l][0], b0f, dims[1], dims[0]);
       else
@@ -1366,12 +1444,12 @@ wk_status wk_res_ln(const void* concat, const void* X, const float* gamma, const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == WK_BF16)
     return run_res_ln<bf16, bf16, bf16>(dv, static_cast<const bf16*>(concat), static_cast<const bf16*>(X), gamma,
-                                        beta, static_cast<bf16*>(out), rows, d, e, st);
+                                        beta, static_cast<bf16*>(out), rows, d, e, dv->standalone_status, st);
   if (dtype == WK_F16)
     return run_res_ln<f16, f16, f16>(dv, static_cast<const f16*>(concat), static_cast<const f16*>(X), gamma, beta,
-                                     static_cast<f16*>(out), rows, d, e, st);
+                                     static_cast<f16*>(out), rows, d, e, dv->standalone_status, st);
   return run_res_ln<float, float, float>(dv, static_cast<const float*>(concat), static_cast<const float*>(X), gamma,
-                                         beta, static_cast<float*>(out), rows, d, e, st);
+                                         beta, static_cast<float*>(out), rows, d, e, dv->standalone_status, st);
 }
 
 wk_status wk_device_status(wk_stream_t stream) {
@@ -1451,7 +1529,7 @@ wk_status wk_layer_forward_noalloc(const wk_stack_config* cfg, const wk_layer_we
     s = run_lcb_simt<float, float>(static_cast<const float*>(w->W_L), Xf, cat, batch, n, d, cfg->n_f, cfg->n_l, st);
   if (s == WK_OK)
     s = run_res_ln<float, float, float>(dv, cat, Xf, w->out_ln_gamma, w->out_ln_beta, static_cast<float*>(out),
-                                        batch * n, d, eps, st);
+                                        batch * n, d, eps, dv->standalone_status, st);
   return s;
 }
 

@@ -75,6 +75,9 @@ def test_mlp_linear_f32_simt():
     (5, 512, 160, 256, 256),   # one example per tile (E = 1), two W_L tiles
     (13, 720, 32, 360, 360),   # E = 8 with a ragged group, K tail (720 = 11*64 + 16), M tail (360)
     (7, 64, 128, 32, 32),      # E = 2, ragged group
+    (301, 512, 160, 256, 256),  # resident W_L: several example groups per CTA, the X ring wraps
+    (1000, 256, 160, 128, 128),  # resident W_L, one m tile for every CTA
+    (97, 200, 160, 100, 100),  # resident W_L with a K tail (200 = 3*64 + 8) and an M tail (100 rows)
 ])
 def test_lcb_tcgen05(batch, n, d, n_f, n_l, dt):
     WL = host_normal((n_l, n), 9, std=1.0 / np.sqrt(n), dtype=dt)
@@ -139,8 +142,12 @@ def test_fm_ln_f32_simt():
         assert max_scaled_err(got[b], ref) <= 1e-4
 
 
+# Row counts: ragged against every stage size of the bulk-copy ring (R = 32..512 rows)
+# and, for the largest, several laps of the ring on every SM.
 @pytest.mark.parametrize("rows,d,dt", [(1003, 160, "bf16"), (4097, 32, "bf16"), (515, 128, "bf16"),
-                                       (333, 16, "f32"), (100, 256, "bf16"), (1003, 160, "f16")])
+                                       (333, 16, "f32"), (100, 256, "bf16"), (1003, 160, "f16"),
+                                       (40001, 160, "f16"), (2999, 192, "f16"), (777, 64, "bf16"),
+                                       (1501, 16, "f16"), (5, 160, "f16")])
 def test_res_ln(rows, d, dt):
     cat = host_normal((rows, d), 22, dtype=dt)
     X = host_normal((rows, d), 23, dtype=dt)
@@ -152,7 +159,7 @@ def test_res_ln(rows, d, dt):
     got = f64(out)
     y = f64(cat) + f64(X)
     tol = {"bf16": 1e-2, "f16": 2e-3, "f32": 1e-5}[dt]
-    for r in range(0, rows, 7):
+    for r in range(rows):
         assert max_scaled_err(got[r], oracle.layernorm(y[r], f64(g), f64(be))) <= tol, r
 
 
