@@ -1,12 +1,13 @@
 """Throughput of the Wukong interaction-stack forward on B200s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
     (N > 1: python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...)
 
 One step is one forward of the whole stack (every layer: FM + LayerNorm, the FMB
 MLP, the LCB, residual + LayerNorm) over one batch of synthetic examples. The
 workload is the 8-layer bf16 stack (n=512 embeddings, d=160, k=64, n_F=n_L=256,
-FMB MLP 32768->16384->16384->40960, ~24.1 GFLOP/example) at batch 4096 per GPU.
+FMB MLP 32768->16384->16384->40960, ~24.1 GFLOP/example) at batch 4096 per GPU;
+--workload names one of the other synthetic workloads (synth/configs.py) instead.
 Several GPUs run independent replicas on disjoint batches (the examples are
 independent, so there is no collective in the forward): weak scaling.
 
@@ -31,6 +32,8 @@ if ROOT not in sys.path:
 
 WORKLOAD = "c4_bf16"
 METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack fwd, 1 B200"
+# examples per oracle sample (one layer), sized for a few seconds of host work each
+ORACLE_SAMPLE = {"c1_fp32": 64, "c2_bf16": 4096, "c3_bf16": 128, "c4_bf16": 16, "c5_bf16": 512}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -40,8 +43,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sources it was taken on: when their hash differs, the bench reports null.
 GEMM_TRAFFIC = {
     "sources": ["recsys_feature_interaction_b200/csrc/gemm_tc2.cuh", "recsys_feature_interaction_b200/csrc/common.cuh"],
-    "sha256": None,
-    "bytes_per_launch": None,
+    "sha256": "2701460f8332c53c784aab747ba8478caa93d99d0778331507517a2bbd23aaf4",
+    "bytes_per_launch": 8557918629,
 }
 
 
@@ -73,8 +76,16 @@ def load_peaks():
 
 def workload_desc(cfg):
     dims = [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
-    return ("%d-layer bf16 Wukong stack fwd: n=%d, d=%d, k=%d, n_F=n_L=%d, FMB MLP %s" %
-            (cfg["layers"], cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], "->".join(str(v) for v in dims)))
+    return ("%d-layer %s Wukong stack fwd: n=%d, d=%d, k=%d, n_F=n_L=%d, FMB MLP %s" %
+            (cfg["layers"], cfg["dtype"], cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
+             "->".join(str(v) for v in dims)))
+
+
+def fp32_alu_peak(peaks):
+    """fp32 CUDA-core peak of the GPU (TFLOP/s): 148 SMs x 128 FMA lanes x 2 FLOP x the
+    SM clock (the measured max clock from the peaks file, else 1965 MHz)."""
+    mhz = peaks.get("sm_max_mhz") or 1965.0
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
 
 
 def gemm_flops_per_example(cfg):
@@ -156,20 +167,21 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from synth import configs as C
-    cfg = C.CONFIGS[WORKLOAD]
+    cfg = C.CONFIGS[args.workload]
     vals = []
+    ns = ORACLE_SAMPLE[args.workload]
     for _ in range(args.warmup):
-        oracle_sample(cfg, 2)
+        oracle_sample(cfg, ns)
     thr = None
     for _ in range(args.steps):
-        v, dt, thr = oracle_sample(cfg, 2)
+        v, dt, thr = oracle_sample(cfg, ns)
         vals.append(v)
     value = statistics.median(vals)
-    sample = "2 examples through 1 of the %d layers per step, scaled to the whole stack" % cfg["layers"]
+    sample = "%d examples through 1 of the %d layers per step, scaled to the whole stack" % (ns, cfg["layers"])
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD + ": " + workload_desc(cfg), "global_batch": cfg["batch"],
+            "config": {"workload": args.workload + ": " + workload_desc(cfg), "global_batch": cfg["batch"],
                        "oracle": "plain C fp64, threads over examples / output rows"},
             "cpu_baseline": {"value": value, "unit": "examples/s", "cores": thr, "kind": "oracle",
                              "sample": sample},
@@ -184,6 +196,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -206,7 +220,7 @@ def main():
     replicas.init("nccl", device=dev)
     wk_build.build()
 
-    cfg = C.CONFIGS[WORKLOAD]
+    cfg = C.CONFIGS[args.workload]
     B = cfg["batch"]
     layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
     h = wk.wk_stack_create(cfg, layers, max_batch=B)
@@ -228,20 +242,32 @@ def main():
         raise RuntimeError("device status after warm-up")
     wk.wk_stack_kernel_times(h)  # clear
 
-    # ---- device-resident timing
+    # ---- device-resident timing. A workload whose input is smaller than twice the
+    # L2 (126 MB) gets an L2 flush (a 256 MB write) before every step, outside the
+    # per-step event pairs; larger inputs stream through L2 by themselves.
+    x_bytes = X.numel() * X.element_size()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if x_bytes < (252 << 20) else None
     wk.wk_stack_set_profiling(h, True)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps if flush is not None else 1)]
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            wk.wk_stack_forward(h, X, out, stream=stream)
-        ev1.record(stream)
+        if flush is None:
+            evs[0][0].record(stream)
+            for _ in range(args.steps):
+                wk.wk_stack_forward(h, X, out, stream=stream)
+            evs[0][1].record(stream)
+        else:
+            for a, b in evs:
+                flush.fill_(1)
+                a.record(stream)
+                wk.wk_stack_forward(h, X, out, stream=stream)
+                b.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
     wk.wk_stack_set_profiling(h, False)
-    ms = ev0.elapsed_time(ev1)
+    ms = sum(a.elapsed_time(b) for a, b in evs)
     status = wk.wk_stack_sync_status(h)
     if status != wk.WK_OK:
         raise RuntimeError("device status: " + wk.wk_status_string(status))
@@ -259,7 +285,7 @@ def main():
         wk.wk_stack_forward_host(h, xh, oh)
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     e2e_value = world * B * args.steps / e2e_s
-    step_bytes = B * cfg["n"] * cfg["d"] * 2
+    step_bytes = B * cfg["n"] * cfg["d"] * X.element_size()
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -271,21 +297,33 @@ def main():
         peak = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
         clocks = clk.summary()
         launches_per_step = sum(n for _, n in ktimes.values()) // max(1, args.steps)
+        fp32 = cfg["dtype"] == "f32"
+        w_bytes = sum(t.numel() * t.element_size() for lw in layers for t in lw.values() if hasattr(t, "numel"))
+        if fp32:
+            roof = {"kernel": "mlp_gemm (fp32 CUDA cores)", "bound": "alu", "peak": fp32_alu_peak(peaks),
+                    "peak_note": "fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
+            precision = "fp32 everywhere (CUDA cores)"
+        else:
+            roof = {"kernel": "mlp_gemm (tcgen05)", "bound": "tensor", "peak": peak,
+                    "peak_note": "%s sustained cuBLAS bf16" % peak_src}
+            precision = ("bf16 inputs, weights and outputs; fp16 tensor-core operands and intermediates; "
+                         "fp32 accumulation and LayerNorm statistics")
+        roof.update({"achieved": achieved, "unit": "TFLOP/s", "frac": (achieved / roof["peak"]) if achieved else None,
+                     "traffic": gemm_traffic() if args.workload == WORKLOAD else None})
+        l2 = ("L2 flushed (256 MB write) before every step, outside the timed events" if flush is not None else
+              "inputs larger than L2 (X %.0f MB, weights %.2f GB per GPU)" % (x_bytes / 1e6, w_bytes / 1e9))
         line = {
             "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": {"workload": WORKLOAD + ": " + workload_desc(cfg), "per_gpu_batch": B,
-                       "precision": "bf16 inputs, weights and outputs; fp16 tensor-core operands and "
-                                    "intermediates; fp32 accumulation and LayerNorm statistics",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if fp32 else "f16", "data": "synthetic",
+            "config": {"workload": args.workload + ": " + workload_desc(cfg), "per_gpu_batch": B,
+                       "precision": precision,
                        "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
-                       "l2": "inputs larger than L2 (X 671 MB, weights 23.6 GB per GPU)"},
+                       "l2": l2},
             "tflops_per_gpu": tflops,
             "pct_of_bf16_peak": 100.0 * tflops / peak,
             "peak_source": "%s bf16_tflops_sustained" % peak_src,
-            "roofline": {"kernel": "mlp_gemm (tcgen05)", "bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None, "traffic": gemm_traffic(),
-                         "peak_note": "%s sustained cuBLAS bf16" % peak_src},
+            "roofline": roof,
             "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "examples/s", "h2d_bytes_per_step": step_bytes,
@@ -293,10 +331,11 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:
-            v, dt, thr = oracle_sample(cfg, 2)
+            ns = ORACLE_SAMPLE[args.workload]
+            v, dt, thr = oracle_sample(cfg, ns)
             line["cpu_baseline"] = {"value": v, "unit": "examples/s", "cores": thr, "kind": "oracle",
-                                    "sample": "2 examples through 1 of the %d layers (%.1f s), scaled to the "
-                                              "whole stack" % (cfg["layers"], dt)}
+                                    "sample": "%d examples through 1 of the %d layers (%.1f s), scaled to the "
+                                              "whole stack" % (ns, cfg["layers"], dt)}
         print(json.dumps(line), flush=True)
     wk.wk_stack_destroy(h)
     replicas.finish()
