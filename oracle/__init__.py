@@ -156,3 +156,58 @@ def stack_forward(cfg, layer_weights, X, threads=None, diag=0):
     for layer in range(cfg["layers"]):
         h = layer_forward(cfg, layer_weights(layer), h, threads=threads, diag=diag)
     return h
+
+
+# ------------------------------------------------------------------ Wukong-MoE
+#
+# Kunlun page (gist.science summary of arXiv 2602.10016), section 2.3, "Wukong Mixture
+# of Experts": the global interaction module runs several Wukong modules in parallel as
+# the experts of one layer, spreading the layer's computation over them. The page gives
+# no formula. Reading taken (the textbook dense mixture of experts): expert e is a whole
+# Wukong layer with its own weights; a softmax gate over the experts, computed per
+# example from the flattened layer input, weights their outputs:
+#   g(X)    = softmax( W_g vec(X) + b_g ),   W_g in R^{E x n d}, vec row-major
+#   MoE(X)  = sum_e g_e(X) * WukongLayer_e(X)
+# Every expert is evaluated for every example (no top-k routing: the page names none).
+
+
+def _weight_f64(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        import synth
+        return synth.bf16_bits_to_f64(a).reshape(a.shape)
+    return a.astype(np.float64)
+
+
+def gate_softmax(W_g, b_g, X):
+    """g [n_ex, E]: the softmax over experts of W_g vec(X_b) + b_g, in float64.
+    W_g [E, n*d] (float32 or bf16 bits), b_g [E] or None, X [n_ex, n, d] float64."""
+    X = _c64(X)
+    x = X.reshape(X.shape[0], -1)
+    logits = x @ _weight_f64(W_g).T
+    if b_g is not None:
+        logits = logits + np.asarray(b_g, dtype=np.float64)[None, :]
+    z = logits - logits.max(axis=1, keepdims=True)
+    w = np.exp(z)
+    return w / w.sum(axis=1, keepdims=True)
+
+
+def moe_layer_forward(cfg, expert_weights, gate, X, threads=None, ln_eps=1e-5):
+    """One Wukong-MoE layer: expert_weights is a list of E layer-weight dicts (as for
+    layer_forward), gate a dict with W_g and b_g; X [n_ex, n, d] float64."""
+    X = _c64(X)
+    g = gate_softmax(gate["W_g"], gate.get("b_g"), X)
+    out = np.zeros_like(X)
+    for e, w in enumerate(expert_weights):
+        out += g[:, e, None, None] * layer_forward(cfg, w, X, threads=threads, ln_eps=ln_eps)
+    return out
+
+
+def moe_forward(cfg, expert_weights, gate_weights, X, threads=None):
+    """The MoE stack, one layer at a time: expert_weights(l, e) and gate_weights(l)
+    return host weights of expert e and of the gate of layer l."""
+    h = _c64(X)
+    for layer in range(cfg["layers"]):
+        experts = [expert_weights(layer, e) for e in range(cfg["experts"])]
+        h = moe_layer_forward(cfg, experts, gate_weights(layer), h, threads=threads)
+    return h

@@ -166,3 +166,94 @@ def make_x_dev(cfg, batch, device="cuda", first_example=0):
     else:
         fill_normal_dev(t, SEED, TID_X, 0.0, 1.0, offset=off)
     return t
+
+
+# ---------------------------------------------------------------- Wukong-MoE
+#
+# The Kunlun page (section 2.3, "Wukong Mixture of Experts") describes a global
+# interaction module in which several Wukong modules run in parallel as the experts of
+# one layer. Workloads of that form: each MoE layer holds E experts, each a Wukong layer
+# of the shape below with its own weights, and a softmax gate over the experts computed
+# from the flattened layer input. Gate weights W_g [E, n*d] ~ N(0, 1/(n*d)) and gate
+# biases b_g [E] ~ N(0, 1) (non-zero so that the bias path is exercised); the experts'
+# tensors follow the recipe of the plain workloads, each on its own streams.
+MOE_CONFIGS = {
+    "moe3_c2": dict(layers=2, experts=3, batch=2048, n=64, d=128, k=16, n_f=32, n_l=32, hidden=[1024],
+                    dtype="bf16", ln_affine="1+N(0,0.02)", x_dist="normal",
+                    about="2 MoE layers x 3 experts of the 2-layer bf16 shape, B=2048"),
+    "moe4_c3": dict(layers=2, experts=4, batch=4096, n=256, d=160, k=32, n_f=128, n_l=128, hidden=[4096, 4096],
+                    dtype="bf16", ln_affine="unit", x_dist="normal",
+                    about="2 MoE layers x 4 experts of the 4-layer bf16 shape (n=256, d=160, k=32), B=4096"),
+}
+
+
+def expert_tid_offset(expert):
+    """Stream-id offset of expert e's tensors (layer ids stay below 100 per layer)."""
+    return 100 * (expert + 1)
+
+
+def expert_specs(cfg, layer, expert):
+    """Recipe of expert e of MoE layer `layer`: the plain layer recipe on shifted streams."""
+    out = {}
+    for name, (shape, kind, tid, mean, std, dt) in tensor_specs(cfg, layer).items():
+        out[name] = (shape, kind, tid + expert_tid_offset(expert), mean, std, dt)
+    return out
+
+
+def gate_specs(cfg, layer):
+    """Recipe of the gate of MoE layer `layer`: W_g [E, n*d], b_g [E] (fp32)."""
+    E, nd = cfg["experts"], cfg["n"] * cfg["d"]
+    wd = "f32" if cfg["dtype"] == "f32" else "bf16"
+    base = 1000 * (layer + 1)
+    return {"W_g": ((E, nd), "normal", base + 95, 0.0, 1.0 / math.sqrt(nd), wd),
+            "b_g": ((E,), "normal", base + 96, 0.0, 1.0, "f32")}
+
+
+def _host_from_specs(specs):
+    out = {}
+    for name, (shape, kind, tid, mean, std, dt) in specs.items():
+        if kind == "const":
+            if dt != "f32":
+                raise ValueError("bf16 constants are not used")
+            out[name] = np.full(shape, mean, dtype=np.float32)
+        else:
+            arr = np.empty(shape, dtype=np.float32 if dt == "f32" else np.uint16)
+            out[name] = fill_normal_host(arr, SEED, tid, mean, std)
+    return out
+
+
+def _dev_from_specs(specs, device):
+    import torch
+
+    from . import fill_normal_dev
+    out = {}
+    for name, (shape, kind, tid, mean, std, dt) in specs.items():
+        tdt = torch.float32 if dt == "f32" else torch.bfloat16
+        if kind == "const":
+            out[name] = torch.full(shape, mean, dtype=tdt, device=device)
+        else:
+            out[name] = fill_normal_dev(torch.empty(shape, dtype=tdt, device=device), SEED, tid, mean, std)
+    return out
+
+
+def make_expert_host(cfg, layer, expert):
+    return _host_from_specs(expert_specs(cfg, layer, expert))
+
+
+def make_expert_dev(cfg, layer, expert, device="cuda"):
+    return _dev_from_specs(expert_specs(cfg, layer, expert), device)
+
+
+def make_gate_host(cfg, layer):
+    return _host_from_specs(gate_specs(cfg, layer))
+
+
+def make_gate_dev(cfg, layer, device="cuda"):
+    return _dev_from_specs(gate_specs(cfg, layer), device)
+
+
+def moe_flops_per_example(cfg):
+    """Matmul FLOPs of one example through the MoE stack: every expert's layer plus the
+    gate's 2 * E * n * d per layer."""
+    per_layer = flops_per_example(dict(cfg, layers=1))
+    return cfg["layers"] * (cfg["experts"] * per_layer + 2 * cfg["experts"] * cfg["n"] * cfg["d"])
