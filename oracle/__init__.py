@@ -211,3 +211,26 @@ def moe_forward(cfg, expert_weights, gate_weights, X, threads=None):
         experts = [expert_weights(layer, e) for e in range(cfg["experts"])]
         h = moe_layer_forward(cfg, experts, gate_weights(layer), h, threads=threads)
     return h
+
+
+# --------------------------------------------------------------- prediction head
+#
+# Wukong page, section 2.2, first paragraph: the model first crosses features with the
+# stacked Wukong layers and then produces the prediction with an MLP. The page gives
+# the head no sizes. Reading taken: the last layer's embeddings are flattened
+# row-major, q Linear layers follow with ReLU after all but the last, the last has one
+# output (the logit), and the prediction is its logistic sigmoid (a click probability).
+
+
+def top_mlp_forward(weights, X):
+    """(logit [n_ex], p [n_ex]) of the prediction head on X [n_ex, n, d] (float64).
+    weights: list of (T_j [out_j, in_j] float32 or bf16 bits, c_j [out_j] float32 or
+    None), in_0 = n*d, out_{q-1} = 1."""
+    X = _c64(X)
+    z = X.reshape(X.shape[0], -1)
+    q = len(weights)
+    for j, (T, c) in enumerate(weights):
+        z = linear(z, T, c, relu=j < q - 1)
+    logit = z[:, 0]
+    p = 1.0 / (1.0 + np.exp(-logit))
+    return logit, p
