@@ -13,9 +13,9 @@ independent, so there is no collective in the forward): weak scaling.
 
 Rank 0 prints one JSON line. `value` is examples/s of the whole job with the
 inputs resident in HBM (CUDA events on the launch stream, max over ranks);
-`e2e` is the same metric through wk_stack_forward_host with pinned host buffers
+`e2e` is the same metric through the public forward with pinned host buffers
 (host-to-device copy of X and device-to-host copy of the output inside the timed
-region); `roofline` reports the MLP GEMM kernel (the dominant one) against the
+region; wk_stack_forward_host for a stack); `roofline` reports the MLP GEMM kernel (the dominant one) against the
 measured bf16 peak; `cpu_baseline` times the fp64 oracle on a bounded sample.
 """
 import argparse
@@ -33,7 +33,8 @@ if ROOT not in sys.path:
 WORKLOAD = "c4_bf16"
 METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack fwd, 1 B200"
 # examples per oracle sample (one layer), sized for a few seconds of host work each
-ORACLE_SAMPLE = {"c1_fp32": 64, "c2_bf16": 4096, "c3_bf16": 128, "c4_bf16": 16, "c5_bf16": 512}
+ORACLE_SAMPLE = {"c1_fp32": 64, "c2_bf16": 4096, "c3_bf16": 128, "c4_bf16": 16, "c5_bf16": 512, "moe3_c2": 1024,
+                 "moe4_c3": 32}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -76,8 +77,10 @@ def load_peaks():
 
 def workload_desc(cfg):
     dims = [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
-    return ("%d-layer %s Wukong stack fwd: n=%d, d=%d, k=%d, n_F=n_L=%d, FMB MLP %s" %
-            (cfg["layers"], cfg["dtype"], cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
+    kind = ("Wukong-MoE stack fwd (%d experts per layer, softmax gate)" % cfg["experts"] if "experts" in cfg
+            else "Wukong stack fwd")
+    return ("%d-layer %s %s: n=%d, d=%d, k=%d, n_F=n_L=%d, FMB MLP %s" %
+            (cfg["layers"], cfg["dtype"], kind, cfg["n"], cfg["d"], cfg["k"], cfg["n_f"],
              "->".join(str(v) for v in dims)))
 
 
@@ -157,21 +160,31 @@ def oracle_sample(cfg, n_examples, threads=None):
     whole stack, seconds, threads)."""
     import oracle
     from synth import configs as C
-    w = C.make_layer_host(cfg, 0)
     X = C.to_f64(C.make_x_host(cfg, list(range(n_examples))))
     thr = threads or oracle.default_threads()
-    t0 = time.perf_counter()
-    oracle.layer_forward(cfg, w, X, threads=thr)
+    if "experts" in cfg:
+        experts = [C.make_expert_host(cfg, 0, e) for e in range(cfg["experts"])]
+        gate = C.make_gate_host(cfg, 0)
+        t0 = time.perf_counter()
+        oracle.moe_layer_forward(cfg, experts, gate, X, threads=thr)
+    else:
+        w = C.make_layer_host(cfg, 0)
+        t0 = time.perf_counter()
+        oracle.layer_forward(cfg, w, X, threads=thr)
     dt = time.perf_counter() - t0
     return n_examples / (dt * cfg["layers"]), dt, thr
+
+
+def workload_cfg(name):
+    from synth import configs as C
+    return C.MOE_CONFIGS[name] if name in C.MOE_CONFIGS else C.CONFIGS[name]
 
 
 def run_reference(args, rank, world):
     """The reference arm: the fp64 oracle as it stands, on the host cores."""
     if rank != 0:
         return
-    from synth import configs as C
-    cfg = C.CONFIGS[args.workload]
+    cfg = workload_cfg(args.workload)
     vals = []
     ns = ORACLE_SAMPLE[args.workload]
     for _ in range(args.warmup):
@@ -201,7 +214,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16"])
+                    choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16", "moe3_c2", "moe4_c3"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -224,15 +237,44 @@ def main():
     replicas.init("nccl", device=dev)
     wk_build.build()
 
-    cfg = C.CONFIGS[args.workload]
+    cfg = workload_cfg(args.workload)
+    moe = "experts" in cfg
     B = cfg["batch"]
-    layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
-    h = wk.wk_stack_create(cfg, layers, max_batch=B)
     # rank r works on examples [r*B, (r+1)*B) of the synthetic stream (no collective on the data path)
     first, _ = replicas.example_range(rank, world, B)
     X = C.make_x_dev(cfg, B, device=dev, first_example=first)
     out = torch.empty_like(X)
     stream = torch.cuda.current_stream(dev)
+    if moe:
+        params = [[C.make_expert_dev(cfg, l, e, device=dev) for e in range(cfg["experts"])]
+                  for l in range(cfg["layers"])]
+        gates = [C.make_gate_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
+        h = wk.wk_moe_create(cfg, params, gates, max_batch=B)
+        api = dict(fwd=lambda x, o: wk.wk_moe_forward(h, x, o, stream=stream),
+                   status=lambda: wk.wk_moe_sync_status(h), prof=lambda on: wk.wk_moe_set_profiling(h, on),
+                   times=lambda: wk.wk_moe_kernel_times(h), destroy=lambda: wk.wk_moe_destroy(h))
+        w_tensors = [t for lay in params for ex in lay for t in ex.values()] + \
+                    [t for g in gates for t in g.values()]
+        flops_ex = C.moe_flops_per_example(cfg)
+
+        def fwd_host(xh, oh):  # the public forward with the step's input and result on the host
+            X.copy_(xh, non_blocking=True)
+            api["fwd"](X, out)
+            oh.copy_(out, non_blocking=True)
+            stream.synchronize()
+        e2e_api = "wk_moe_forward with a pinned host-to-device copy before and device-to-host copy after"
+    else:
+        layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
+        h = wk.wk_stack_create(cfg, layers, max_batch=B)
+        api = dict(fwd=lambda x, o: wk.wk_stack_forward(h, x, o, stream=stream),
+                   status=lambda: wk.wk_stack_sync_status(h), prof=lambda on: wk.wk_stack_set_profiling(h, on),
+                   times=lambda: wk.wk_stack_kernel_times(h), destroy=lambda: wk.wk_stack_destroy(h))
+        w_tensors = [t for lw in layers for t in lw.values()]
+        flops_ex = C.flops_per_example(cfg)
+
+        def fwd_host(xh, oh):
+            wk.wk_stack_forward_host(h, xh, oh)
+        e2e_api = "wk_stack_forward_host (chunked copies overlapped with compute)"
 
     barrier = replicas.barrier
 
@@ -240,18 +282,18 @@ def main():
         return replicas.max_over_ranks(v, device=dev)
 
     for _ in range(args.warmup):
-        wk.wk_stack_forward(h, X, out, stream=stream)
+        api["fwd"](X, out)
     torch.cuda.synchronize(dev)
-    if wk.wk_stack_sync_status(h) != wk.WK_OK:
+    if api["status"]() != wk.WK_OK:
         raise RuntimeError("device status after warm-up")
-    wk.wk_stack_kernel_times(h)  # clear
+    api["times"]()  # clear
 
     # ---- device-resident timing. A workload whose input is smaller than twice the
     # L2 (126 MB) gets an L2 flush (a 256 MB write) before every step, outside the
     # per-step event pairs; larger inputs stream through L2 by themselves.
     x_bytes = X.numel() * X.element_size()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if x_bytes < (252 << 20) else None
-    wk.wk_stack_set_profiling(h, True)
+    api["prof"](True)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps if flush is not None else 1)]
     barrier()
@@ -260,40 +302,39 @@ def main():
         if flush is None:
             evs[0][0].record(stream)
             for _ in range(args.steps):
-                wk.wk_stack_forward(h, X, out, stream=stream)
+                api["fwd"](X, out)
             evs[0][1].record(stream)
         else:
             for a, b in evs:
                 flush.fill_(1)
                 a.record(stream)
-                wk.wk_stack_forward(h, X, out, stream=stream)
+                api["fwd"](X, out)
                 b.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
-    wk.wk_stack_set_profiling(h, False)
+    api["prof"](False)
     ms = sum(a.elapsed_time(b) for a, b in evs)
-    status = wk.wk_stack_sync_status(h)
+    status = api["status"]()
     if status != wk.WK_OK:
         raise RuntimeError("device status: " + wk.wk_status_string(status))
-    ktimes = wk.wk_stack_kernel_times(h)
+    ktimes = api["times"]()
     ms_max = max_over_ranks(ms)
     value = world * B * args.steps / (ms_max / 1e3)
 
-    # ---- end to end through the host-buffer entry point
+    # ---- end to end with host buffers
     xh = X.cpu().pin_memory()
     oh = torch.empty_like(xh).pin_memory()
-    wk.wk_stack_forward_host(h, xh, oh)  # warm the staging buffers
+    fwd_host(xh, oh)  # warm the staging buffers
     barrier()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        wk.wk_stack_forward_host(h, xh, oh)
+        fwd_host(xh, oh)
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     e2e_value = world * B * args.steps / e2e_s
     step_bytes = B * cfg["n"] * cfg["d"] * X.element_size()
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        flops_ex = C.flops_per_example(cfg)
         tflops = value * flops_ex / 1e12 / world
         g_ms, g_n = ktimes["mlp_gemm"]
         gemm_flops_launch = gemm_flops_per_example(cfg) * B / (cfg["layers"] * (len(cfg["hidden"]) + 1))
@@ -302,7 +343,7 @@ def main():
         clocks = clk.summary()
         launches_per_step = sum(n for _, n in ktimes.values()) // max(1, args.steps)
         fp32 = cfg["dtype"] == "f32"
-        w_bytes = sum(t.numel() * t.element_size() for lw in layers for t in lw.values() if hasattr(t, "numel"))
+        w_bytes = sum(t.numel() * t.element_size() for t in w_tensors if hasattr(t, "numel"))
         if fp32:
             roof = {"kernel": "mlp_gemm (fp32 CUDA cores)", "bound": "alu", "peak": fp32_alu_peak(peaks),
                     "peak_note": "fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
@@ -331,7 +372,7 @@ def main():
             "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "examples/s", "h2d_bytes_per_step": step_bytes,
-                    "d2h_bytes_per_step": step_bytes},
+                    "d2h_bytes_per_step": step_bytes, "api": e2e_api},
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -341,7 +382,7 @@ def main():
                                     "sample": "%d examples through 1 of the %d layers (%.1f s), scaled to the "
                                               "whole stack" % (ns, cfg["layers"], dt)}
         print(json.dumps(line), flush=True)
-    wk.wk_stack_destroy(h)
+    api["destroy"]()
     replicas.finish()
 
 

@@ -157,7 +157,8 @@ WK_API const char* wk_status_string(wk_status s);
 /* ---- per-kernel timing of a handle's forwards (CUDA events on the launch stream) ---- */
 
 typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
-               WK_KERNEL_CONVERT = 4, WK_KERNEL_COUNT = 5 } wk_kernel_kind;
+               WK_KERNEL_CONVERT = 4, WK_KERNEL_MOE_GATE = 5, WK_KERNEL_MOE_COMBINE = 6,
+               WK_KERNEL_HEAD = 7, WK_KERNEL_COUNT = 8 } wk_kernel_kind;
 
 /* enable != 0: every later forward records a start/stop event pair around each
  * kernel launch on its stream (adds no synchronisation). */
@@ -202,6 +203,112 @@ WK_API wk_status wk_res_ln(const void* concat, const void* X, const float* gamma
 /* Waits for `stream`, then reads and clears the device status word of the
  * stand-alone calls above (handles have their own). */
 WK_API wk_status wk_device_status(wk_stream_t stream);
+
+/* ---- prediction head ----
+ *
+ * Wukong page, section 2.2, first paragraph: the model crosses features with the
+ * stacked Wukong layers and then produces the prediction with an MLP. The page gives
+ * the head no sizes; the reading implemented: the last layer's output X_L is
+ * flattened row-major (n*d values per example), q Linear layers follow with ReLU
+ * after all but the last, the last has one output (the logit), and the prediction
+ * is its logistic sigmoid:
+ *
+ *     z_0 = vec(X_L),  z_{j+1} = ReLU(T_j z_j + c_j) (j < q-1),
+ *     logit = T_{q-1} z_{q-1} + c_{q-1},  prob = 1 / (1 + exp(-logit)). */
+typedef struct {
+  int32_t num_linear;       /* q >= 1 */
+  const int32_t* hidden;    /* q-1 hidden widths, multiples of 8 (copied); NULL when q == 1 */
+  const void* const* T;     /* q weights [out_j, in_j] in the stack's dtype, row-major; in_0 = n*d,
+                               out_{q-1} = 1. Device pointers, BORROWED like the layer weights
+                               (copied at this call when dtype differs from the operand type) */
+  const float* const* c;    /* q biases [out_j] fp32; c or c[j] may be NULL (zero) */
+} wk_head;
+
+/* Attaches (or replaces) the prediction head of a 16-bit stack: converts its weights
+ * to the operand type when needed, allocates two activation buffers [max_batch,
+ * widest hidden] and builds the head's GEMM descriptors. Synchronises the device.
+ * Errors: WK_ERR_INVALID_ARG (NULL, misaligned), WK_ERR_UNSUPPORTED (fp32 stack,
+ * widths not multiples of 8), WK_ERR_OOM, WK_ERR_CUDA. */
+WK_API wk_status wk_stack_set_head(wk_stack* h, const wk_head* head);
+
+/* The stack forward on X [batch, n, d] followed by the head: logit [batch] fp32 and,
+ * when prob is not NULL, prob [batch] fp32. The last layer's output stays on the
+ * device in the operand type; the head's hidden Linears run on the tensor-core GEMM,
+ * its one-output Linear and the sigmoid in head_out_kernel. Asynchronous on
+ * `stream`; not re-entrant. WK_ERR_INVALID_ARG without a head. */
+WK_API wk_status wk_stack_predict(wk_stack* h, const void* X, float* logit, float* prob, int64_t batch,
+                                  wk_stream_t stream);
+
+/* ---- Wukong mixture of experts ----
+ *
+ * The Kunlun page (gist.science summary of arXiv 2602.10016, section 2.3, "Wukong
+ * Mixture of Experts") describes a global interaction module in which several
+ * Wukong modules run in parallel as the experts of one layer, spreading the layer's
+ * computation over them. The page gives no formula; the reading implemented is the
+ * dense mixture of experts: expert e of MoE layer l is a whole Wukong layer (its own
+ * FMB, LCB, residual and output LayerNorm), and a softmax gate computed per example
+ * from the flattened layer input weights the experts' outputs:
+ *
+ *     g(X)    = softmax( W_g vec(X) + b_g ),    W_g [E, n*d], vec row-major
+ *     MoE(X)  = sum_e g_e(X) * WukongLayer_e(X)
+ *
+ * Every expert runs on every example (the page names no routing). A stack of
+ * num_layers MoE layers maps X_0 to X_L. 16-bit dtypes only. */
+
+typedef struct {
+  const void* W_g;   /* [num_experts, n*d] dtype, row e scores expert e; BORROWED like the
+                        layer weights (copied at create when dtype differs from the operand type) */
+  const float* b_g;  /* [num_experts] fp32, or NULL for zero */
+} wk_moe_gate;
+
+typedef struct wk_moe wk_moe;
+
+#define WK_MOE_MAX_EXPERTS 8
+
+/* cfg: the shape of every expert layer and of the MoE stack (cfg->num_layers MoE
+ * layers; dtype WK_BF16 or WK_F16; operand_dtype, ln_eps and max_batch as for
+ * wk_stack_create). experts: num_layers * num_experts layer weights, layer-major
+ * (experts[l * num_experts + e] is expert e of layer l), device pointers BORROWED
+ * as for wk_stack_create. gates: num_layers gate parameters. 1 <= num_experts <=
+ * WK_MOE_MAX_EXPERTS. Allocates, per expert, the workspace of one layer's front
+ * (A0, MLP activations, concat buffer), plus the gate weights [max_batch,
+ * num_experts] fp32 and two layer buffers [max_batch, n, d] in the operand type.
+ * Synchronises the device. Errors as wk_stack_create; WK_ERR_UNSUPPORTED for fp32. */
+WK_API wk_status wk_moe_create(const wk_stack_config* cfg, int32_t num_experts, const wk_layer_weights* experts,
+                               const wk_moe_gate* gates, wk_moe** out);
+
+/* out[b] = MoE stack(X[b]) for b < batch; X and out [batch, n, d] of cfg->dtype, not
+ * overlapping. Per MoE layer on `stream`: the gate (moe_gate_kernel), each expert's
+ * FM + LayerNorm, MLP and LCB into its own concat buffer, then one kernel that
+ * applies every expert's residual + LayerNorm and mixes them with the gate
+ * (moe_combine_kernel). Asynchronous; not re-entrant (as wk_stack_forward). */
+WK_API wk_status wk_moe_forward(wk_moe* h, const void* X, void* out, int64_t batch, wk_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the experts' device status words. */
+WK_API wk_status wk_moe_sync_status(wk_moe* h, wk_stream_t stream);
+
+/* Per-kernel event timing of a handle's forwards, as wk_stack_set_profiling /
+ * wk_stack_kernel_times (the experts' kernels summed per kind, plus
+ * WK_KERNEL_MOE_GATE and WK_KERNEL_MOE_COMBINE). */
+WK_API wk_status wk_moe_set_profiling(wk_moe* h, int enable);
+WK_API wk_status wk_moe_kernel_times(wk_moe* h, double* total_ms, int64_t* launches);
+
+/* Frees the handle, its experts and workspace (synchronises the device). NULL is a no-op. */
+WK_API void wk_moe_destroy(wk_moe* h);
+
+/* Stand-alone gate: g[b, e] = softmax_e( sum_j W_g[e, j] X[b, j] + b_g[e] ), X [batch, nd]
+ * and W_g [num_experts, nd] of dtype (16-bit, nd % 8 == 0), b_g [num_experts] fp32 or
+ * NULL, g [batch, num_experts] fp32. Dot products accumulate in fp32. */
+WK_API wk_status wk_moe_gate_softmax(const void* X, const void* W_g, const float* b_g, float* g, int64_t batch,
+                                     int64_t nd, int32_t num_experts, wk_dtype dtype, wk_stream_t stream);
+
+/* Stand-alone mixture of the experts' residual + LayerNorm outputs:
+ *   out[b, i, :] = sum_e g[b, e] * ( LN( concat_e[b, i, :] + X[b, i, :] ) * gamma_e + beta_e )
+ * concats: num_experts pointers to [batch, n, d]; X, out [batch, n, d] (dtype, 16-bit);
+ * g [batch, num_experts] fp32; gammas, betas: num_experts pointers to [d] fp32. */
+WK_API wk_status wk_moe_combine(const void* const* concats, const void* X, const float* g, const float* const* gammas,
+                                const float* const* betas, void* out, int64_t batch, int32_t n, int32_t d,
+                                int32_t num_experts, wk_dtype dtype, float eps, wk_stream_t stream);
 
 /* ---- one layer without allocating: for callers that cannot call cudaMalloc ----
  *

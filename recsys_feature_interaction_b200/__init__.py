@@ -20,8 +20,10 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
 
 WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
 WK_F32, WK_BF16, WK_F16 = 0, 1, 2
-WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_CONVERT, WK_KERNEL_COUNT = range(6)
-KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert")
+(WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_CONVERT, WK_KERNEL_MOE_GATE,
+ WK_KERNEL_MOE_COMBINE, WK_KERNEL_COUNT) = range(8)
+KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert", "moe_gate", "moe_combine")
+WK_MOE_MAX_EXPERTS = 8
 
 
 class WkError(RuntimeError):
@@ -43,6 +45,10 @@ class WkLayerWeights(ctypes.Structure):
                 ("b", ctypes.POINTER(ctypes.c_void_p)), ("fmb_ln_gamma", ctypes.c_void_p),
                 ("fmb_ln_beta", ctypes.c_void_p), ("W_L", ctypes.c_void_p), ("out_ln_gamma", ctypes.c_void_p),
                 ("out_ln_beta", ctypes.c_void_p)]
+
+
+class WkMoeGate(ctypes.Structure):
+    _fields_ = [("W_g", ctypes.c_void_p), ("b_g", ctypes.c_void_p)]
 
 
 _lib = None
@@ -71,6 +77,15 @@ def lib():
             "wk_device_status": [vp],
             "wk_layer_forward_noalloc": [ctypes.POINTER(WkStackConfig), ctypes.POINTER(WkLayerWeights), vp, vp, i64,
                                          vp],
+            "wk_moe_create": [ctypes.POINTER(WkStackConfig), i32, ctypes.POINTER(WkLayerWeights),
+                              ctypes.POINTER(WkMoeGate), ctypes.POINTER(vp)],
+            "wk_moe_forward": [vp, vp, vp, i64, vp],
+            "wk_moe_sync_status": [vp, vp],
+            "wk_moe_set_profiling": [vp, ci],
+            "wk_moe_kernel_times": [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)],
+            "wk_moe_gate_softmax": [vp, vp, vp, vp, i64, i64, i32, ci, vp],
+            "wk_moe_combine": [ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, i64, i32, i32,
+                               i32, ci, cf, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -78,6 +93,8 @@ def lib():
             f.restype = ci
         L.wk_stack_destroy.argtypes = [vp]
         L.wk_stack_destroy.restype = None
+        L.wk_moe_destroy.argtypes = [vp]
+        L.wk_moe_destroy.restype = None
         L.wk_status_string.argtypes = [ci]
         L.wk_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -245,3 +262,78 @@ def wk_layer_forward_noalloc(cfg, layer, X, out, batch=None, stream=None, dtype=
     b = X.shape[0] if batch is None else batch
     _check(lib().wk_layer_forward_noalloc(ctypes.byref(c), arr, _addr(X), _addr(out), int(b), _stream(stream, X)),
            "wk_layer_forward_noalloc")
+
+
+# ------------------------------------------------------------ mixture of experts
+
+class MoeHandle:
+    """An opaque wk_moe* plus the Python objects whose memory it borrows."""
+
+    def __init__(self, ptr, cfg, keep):
+        self.ptr = ptr
+        self.cfg = cfg
+        self._keep = keep
+
+    def __del__(self):
+        try:
+            if self.ptr:
+                wk_moe_destroy(self)
+        except Exception:
+            pass
+
+
+def wk_moe_create(cfg, experts, gates, max_batch=None, dtype=None, ln_eps=0.0, operand_dtype=None):
+    """cfg as for wk_stack_create plus `experts`; experts[l][e]: the layer-weight mapping
+    of expert e of MoE layer l; gates[l]: mapping with W_g [E, n*d] and b_g [E] (or None)."""
+    c, hid, m = _config(cfg, max_batch, dtype, ln_eps, operand_dtype)
+    L = len(experts)
+    E = len(experts[0])
+    flat = [experts[l][e] for l in range(L) for e in range(E)]
+    keep = [hid, flat, list(gates)]
+    arr = _layer_array(flat, m, keep)
+    garr = (WkMoeGate * L)(*[WkMoeGate(_addr(g["W_g"]), _addr(g.get("b_g"))) for g in gates])
+    keep.append(garr)
+    h = ctypes.c_void_p()
+    _check(lib().wk_moe_create(ctypes.byref(c), E, arr, garr, ctypes.byref(h)), "wk_moe_create")
+    return MoeHandle(h.value, dict(cfg), keep)
+
+
+def wk_moe_forward(h, X, out, batch=None, stream=None):
+    b = X.shape[0] if batch is None else batch
+    _check(lib().wk_moe_forward(h.ptr, _addr(X), _addr(out), int(b), _stream(stream, X)), "wk_moe_forward")
+
+
+def wk_moe_sync_status(h, stream=None):
+    return lib().wk_moe_sync_status(h.ptr, _stream(stream))
+
+
+def wk_moe_destroy(h):
+    if h.ptr:
+        lib().wk_moe_destroy(h.ptr)
+        h.ptr = None
+
+
+def wk_moe_set_profiling(h, enable=True):
+    _check(lib().wk_moe_set_profiling(h.ptr, 1 if enable else 0), "wk_moe_set_profiling")
+
+
+def wk_moe_kernel_times(h):
+    """{kernel name: (total_ms, launches)} summed over the experts and the MoE's own kernels."""
+    ms = (ctypes.c_double * WK_KERNEL_COUNT)()
+    n = (ctypes.c_int64 * WK_KERNEL_COUNT)()
+    _check(lib().wk_moe_kernel_times(h.ptr, ms, n), "wk_moe_kernel_times")
+    return {KERNEL_NAMES[i]: (ms[i], n[i]) for i in range(WK_KERNEL_COUNT)}
+
+
+def wk_moe_gate_softmax(X, W_g, b_g, g, batch, nd, num_experts, dtype, stream=None):
+    _check(lib().wk_moe_gate_softmax(_addr(X), _addr(W_g), _addr(b_g), _addr(g), int(batch), int(nd),
+                                     int(num_experts), _dtype_code(dtype), _stream(stream, X)), "wk_moe_gate_softmax")
+
+
+def wk_moe_combine(concats, X, g, gammas, betas, out, batch, n, d, dtype, eps=0.0, stream=None):
+    E = len(concats)
+    cp = (ctypes.c_void_p * E)(*[_addr(c) for c in concats])
+    gp = (ctypes.c_void_p * E)(*[_addr(t) for t in gammas])
+    bp = (ctypes.c_void_p * E)(*[_addr(t) for t in betas])
+    _check(lib().wk_moe_combine(cp, _addr(X), _addr(g), gp, bp, _addr(out), int(batch), int(n), int(d), E,
+                                _dtype_code(dtype), float(eps), _stream(stream, X)), "wk_moe_combine")

@@ -31,7 +31,9 @@
 #include "fm_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
+#include "head.cuh"
 #include "lcb_tc.cuh"
+#include "moe.cuh"
 #include "res_ln.cuh"
 #include "res_ln_ring.cuh"
 #include "simt.cuh"
@@ -548,6 +550,55 @@ wk_status run_convert(const DevInfo* dv, const void* in, void* out, int64_t n, c
   return launch_status();
 }
 
+// ------------------------------------------------------------ prediction head
+
+template <typename T>
+wk_status run_head_out(const DevInfo* dv, const T* H, const T* w, const float* bias, float* logit, float* prob,
+                       int64_t batch, int64_t K, cudaStream_t st) {
+  const int64_t warps_needed = batch;
+  int64_t blocks = (warps_needed + 7) / 8;
+  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(dv->sms) * 16));
+  head_out_kernel<T><<<static_cast<int>(blocks), 256, 0, st>>>(H, w, bias, logit, prob, batch, K);
+  return launch_status();
+}
+
+// ------------------------------------------------------------ mixture of experts
+
+template <typename T>
+wk_status run_moe_gate(const DevInfo* dv, const T* X, const T* Wg, const float* bg, float* g, int64_t batch,
+                       int64_t nd, int E, cudaStream_t st) {
+  const int64_t need = (batch + MOE_GATE_EB - 1) / MOE_GATE_EB;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, static_cast<int64_t>(dv->sms) * 8)));
+  moe_gate_kernel<T><<<grid, 256, 0, st>>>(X, Wg, bg, g, batch, nd, E);
+  return launch_status();
+}
+
+template <int D, typename T, typename TO>
+wk_status run_moe_combine_d(const DevInfo* dv, const MoePtrs& p, const T* x, const float* g, TO* out, int64_t rows,
+                            int n, int E, float eps, cudaStream_t st) {
+  constexpr int G = res_ln_lanes(D / 8);
+  constexpr int rows_per_block = 8 * (32 / G);
+  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(dv->sms) * 8));
+  moe_combine_kernel<D, T, TO><<<static_cast<int>(blocks), 256, 0, st>>>(p, x, g, out, rows, n, E, eps);
+  return launch_status();
+}
+
+template <typename T, typename TO>
+wk_status run_moe_combine(const DevInfo* dv, const MoePtrs& p, const T* x, const float* g, TO* out, int64_t rows,
+                          int n, int d, int E, float eps, cudaStream_t st) {
+  switch (d) {
+    case 16: return run_moe_combine_d<16>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 32: return run_moe_combine_d<32>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 64: return run_moe_combine_d<64>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 128: return run_moe_combine_d<128>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 160: return run_moe_combine_d<160>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 192: return run_moe_combine_d<192>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 256: return run_moe_combine_d<256>(dv, p, x, g, out, rows, n, E, eps, st);
+    default: return WK_ERR_UNSUPPORTED;
+  }
+}
+
 // ------------------------------------------------------------------- SIMT
 
 template <typename T, typename TO>
@@ -603,12 +654,21 @@ struct wk_stack {
   bool tc_mlp = false, tc_lcb = false;
   bool pair = false;                            // MLP Linears on CTA pairs (gemm_tc2.cuh)
   bool fused = false;                           // residual + LN in the last Linear / LCB epilogues
+  bool front_only = false;                      // an expert of a wk_moe: no layer buffers, no fused path
   std::vector<GemmMaps> last_maps;              // [layer]: fused last Linear (B box mma_n/2 rows, C = Xs[l%2])
   CUtensorMap lcbC_x[2];                        // LCB rows n_f.. of Xs[0] / Xs[1]
   std::vector<std::vector<GemmMaps>> mlp_maps;  // [layer][j]
   std::vector<CUtensorMap> lcbA;                // [layer]
   CUtensorMap lcbB_ws[2];
   CUtensorMap lcbC;
+  // prediction head (wk_stack_set_head): q Linears, dims n*d -> ... -> 1
+  std::vector<int32_t> head_dims;               // empty: no head
+  std::vector<const void*> hT;                  // [q] operand type
+  std::vector<const float*> hc;                 // [q]
+  uint8_t* head_copy = nullptr;                 // weights converted to the operand type
+  uint8_t* head_ws = nullptr;                   // two activation buffers [maxb, widest hidden]
+  void* HH[2] = {nullptr, nullptr};
+  std::vector<GemmMaps> head_maps;              // [q-1] hidden Linears
   // host-buffer forward
   uint8_t* stage = nullptr;
   int64_t stage_chunk = 0;
@@ -621,6 +681,27 @@ struct wk_stack {
   };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
+};
+
+// A stack of Wukong mixture-of-experts layers: one front-only wk_stack per expert
+// (its weights, converted copies, descriptors and one layer's front workspace),
+// the gates, and the MoE's own layer buffers.
+struct wk_moe {
+  int device = 0;
+  wk_stack_config cfg{};
+  int E = 0;
+  float eps = 1e-5f;
+  wk_dtype io = WK_BF16, op = WK_F16;
+  int64_t maxb = 0;
+  const DevInfo* dv = nullptr;
+  std::vector<wk_stack*> ex;        // [E]
+  std::vector<const void*> Wg;      // [layer], operand type
+  std::vector<const float*> bg;     // [layer]
+  uint8_t* wcopy = nullptr;         // gate weights converted to the operand type
+  uint8_t* ws = nullptr;
+  float* g = nullptr;               // [maxb, E]
+  void* Xm[2] = {nullptr, nullptr}; // layer outputs; Xm[1] also takes a converted input
+  CUtensorMap lcbX[2];              // Xm[0], Xm[1] as the LCB's operand
 };
 
 namespace {
@@ -665,6 +746,8 @@ void free_stack(wk_stack* h) {
   cudaGetLastError();
   if (h->ws) cudaFree(h->ws);
   if (h->wcopy) cudaFree(h->wcopy);
+  if (h->head_copy) cudaFree(h->head_copy);
+  if (h->head_ws) cudaFree(h->head_ws);
   if (h->stage) cudaFree(h->stage);
   if (h->s_in) cudaStreamDestroy(h->s_in);
   if (h->s_out) cudaStreamDestroy(h->s_out);
@@ -725,7 +808,7 @@ wk_status build_maps(wk_stack* h) {
         if (!ok) return WK_ERR_UNSUPPORTED;
       }
   }
-  h->fused = h->tc_mlp && h->pair && h->tc_lcb && use_fused_ln() && d <= GEMM2_BN;
+  h->fused = h->tc_mlp && h->pair && h->tc_lcb && use_fused_ln() && d <= GEMM2_BN && !h->front_only;
   if (h->fused) {
     const int E = GEMM2_BN / d;
     h->last_maps.resize(L);
@@ -746,15 +829,68 @@ wk_status build_maps(wk_stack* h) {
     h->lcbA.resize(L);
     bool ok = true;
     for (int l = 0; l < L; ++l) ok = ok && map_kmajor<T>(dv, &h->lcbA[l], h->WL[l], n, c.n_l, GEMM_BM);
-    ok = ok && map_lcb_x<T>(dv, &h->lcbB_ws[0], h->Xs[0], n, d, B) && map_lcb_x<T>(dv, &h->lcbB_ws[1], h->Xs[1], n, d, B) &&
-         map_lcb_out<T>(dv, &h->lcbC, h->cat, n, d, c.n_f, c.n_l, B);
+    if (!h->front_only)
+      ok = ok && map_lcb_x<T>(dv, &h->lcbB_ws[0], h->Xs[0], n, d, B) &&
+           map_lcb_x<T>(dv, &h->lcbB_ws[1], h->Xs[1], n, d, B);
+    ok = ok && map_lcb_out<T>(dv, &h->lcbC, h->cat, n, d, c.n_f, c.n_l, B);
     if (!ok) return WK_ERR_UNSUPPORTED;
   }
   return WK_OK;
 }
 
-// The forward of a 16-bit stack with operand type T and caller type IO.
-template <typename T, typename IO>
+// The front of layer l of a 16-bit stack (operand type T): FM + LayerNorm, the MLP
+// Linears (the last one into rows 0..n_f-1 of the concat buffer) and the LCB (rows
+// n_f..n-1), reading the layer input xin; lcb_x is xin as the LCB's TMA operand.
+// Leaves the residual + LayerNorm to the caller.
+template <typename T>
+wk_status layer_front16(wk_stack* h, int l, const T* xin, const CUtensorMap& lcb_x, int64_t batch, cudaStream_t st) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear;
+  const size_t nd = static_cast<size_t>(n) * d;
+  wk_status s = WK_OK;
+  {  // 1. FM + LN
+    ProfScope ps(h, WK_KERNEL_FM_LN, st);
+    s = run_fm16<T>(dv, xin, static_cast<const T*>(h->Y[l]), h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, n, d,
+                    k, h->eps, h->status, st);
+  }
+  for (int j = 0; j < m && s == WK_OK; ++j) {  // 2. MLP
+    ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+    const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+    const bool lastj = j == m - 1;
+    void* o = lastj ? h->cat : h->H[j % 2];
+    const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
+    const int relu = lastj ? 0 : 1;
+    if (h->tc_mlp && h->pair)
+      s = run_gemm_tc2<T, T>(dv, h->mlp_maps[l][j],
+                             mlp2_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
+    else if (h->tc_mlp)
+      s = run_gemm_tc<MODE_MLP, T, T>(dv, h->mlp_maps[l][j],
+                                       mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
+    else
+      s = run_gemm_simt<T, T>(static_cast<const T*>(in), static_cast<const T*>(h->W[l][j]), h->b[l][j],
+                              static_cast<T*>(o), batch, h->dims[j], h->dims[j + 1], ldc, relu, st);
+  }
+  if (s != WK_OK) return s;
+  {  // 3. LCB
+    ProfScope ps(h, WK_KERNEL_LCB, st);
+    if (h->tc_lcb) {
+      GemmMaps mp;
+      mp.A = h->lcbA[l];
+      mp.B = lcb_x;
+      mp.C = h->lcbC;
+      s = run_lcb_tc<T, T>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
+    } else {
+      s = run_lcb_simt<T, T>(static_cast<const T*>(h->WL[l]), xin, static_cast<T*>(h->cat), batch, n, d, c.n_f,
+                             c.n_l, st);
+    }
+  }
+  return s;
+}
+
+// The forward of a 16-bit stack with operand type T, input type IO and output type
+// OUT (the caller's type, or T when the prediction head reads the output).
+template <typename T, typename IO, typename OUT = IO>
 wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaStream_t st) {
   const wk_stack_config& c = h->cfg;
   const DevInfo* dv = h->dv;
@@ -774,37 +910,27 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
     return WK_ERR_CUDA;
   }
   CUtensorMap out_last, out_lcb;  // the caller's output as the fused epilogues' destination
-  if (h->fused && (!map_out<IO>(dv, &out_last, out, static_cast<uint64_t>(c.n_f) * d, batch, nd) ||
-                   !map_lcb_out<IO>(dv, &out_lcb, out, n, d, c.n_f, c.n_l, batch)))
+  if (h->fused && (!map_out<OUT>(dv, &out_last, out, static_cast<uint64_t>(c.n_f) * d, batch, nd) ||
+                   !map_lcb_out<OUT>(dv, &out_lcb, out, n, d, c.n_f, c.n_l, batch)))
     return WK_ERR_CUDA;
   for (int l = 0; l < L && s == WK_OK; ++l) {
     const bool last = l == L - 1;
     const T* xin = static_cast<const T*>(l == 0 ? x0 : h->Xs[(l - 1) % 2]);
-    {  // 1. FM + LN
-      ProfScope ps(h, WK_KERNEL_FM_LN, st);
-      s = run_fm16<T>(dv, xin, static_cast<const T*>(h->Y[l]), h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, n, d,
-                      k, h->eps, h->status, st);
-    }
-    const int m_plain = h->fused ? m - 1 : m;  // the fused path runs the last Linear below
-    for (int j = 0; j < m_plain && s == WK_OK; ++j) {  // 2. MLP
-      ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
-      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
-      const bool lastj = j == m - 1;
-      void* o = lastj ? h->cat : h->H[j % 2];
-      const int64_t ldc = lastj ? static_cast<int64_t>(nd) : h->dims[j + 1];
-      const int relu = lastj ? 0 : 1;
-      if (h->tc_mlp && h->pair)
-        s = run_gemm_tc2<T, T>(dv, h->mlp_maps[l][j],
-                               mlp2_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
-      else if (h->tc_mlp)
-        s = run_gemm_tc<MODE_MLP, T, T>(dv, h->mlp_maps[l][j],
-                                         mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], relu, h->status), st);
-      else
-        s = run_gemm_simt<T, T>(static_cast<const T*>(in), static_cast<const T*>(h->W[l][j]), h->b[l][j],
-                                static_cast<T*>(o), batch, h->dims[j], h->dims[j + 1], ldc, relu, st);
-    }
-    if (s != WK_OK) break;
-    if (h->fused) {
+    if (!h->fused) {
+      s = layer_front16<T>(h, l, xin, (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2], batch, st);
+      if (s != WK_OK) break;
+    } else {
+      {  // 1. FM + LN
+        ProfScope ps(h, WK_KERNEL_FM_LN, st);
+        s = run_fm16<T>(dv, xin, static_cast<const T*>(h->Y[l]), h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, n,
+                        d, k, h->eps, h->status, st);
+      }
+      for (int j = 0; j < m - 1 && s == WK_OK; ++j) {  // 2. MLP Linears but the last
+        ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+        s = run_gemm_tc2<T, T>(dv, h->mlp_maps[l][j], mlp2_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], 1,
+                                                                  h->status), st);
+      }
+      if (s != WK_OK) break;
       // 2'. last Linear + residual + LN -> rows 0..n_f-1 of X_{i+1};
       // 3'. LCB + residual + LN -> rows n_f..n-1 of X_{i+1}
       {
@@ -814,7 +940,7 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
         GemmMaps mp = h->last_maps[l];
         if (last) {
           mp.C = out_last;
-          s = run_gemm_tc2<T, IO, true>(dv, mp, p, st);
+          s = run_gemm_tc2<T, OUT, true>(dv, mp, p, st);
         } else {
           s = run_gemm_tc2<T, T, true>(dv, mp, p, st);
         }
@@ -834,7 +960,7 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
         mp.B = (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2];
         if (last) {
           mp.C = out_lcb;
-          s = run_gemm_tc<MODE_LCB, T, IO, true>(dv, mp, p, st);
+          s = run_gemm_tc<MODE_LCB, T, OUT, true>(dv, mp, p, st);
         } else {
           mp.C = h->lcbC_x[l % 2];
           s = run_gemm_tc<MODE_LCB, T, T, true>(dv, mp, p, st);
@@ -842,26 +968,12 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
       }
       continue;
     }
-    {  // 3. LCB
-      ProfScope ps(h, WK_KERNEL_LCB, st);
-      if (h->tc_lcb) {
-        GemmMaps mp;
-        mp.A = h->lcbA[l];
-        mp.B = (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2];
-        mp.C = h->lcbC;
-        s = run_lcb_tc<T, T>(dv, mp, lcb_params(batch, n, d, c.n_l, h->status), st);
-      } else {
-        s = run_lcb_simt<T, T>(static_cast<const T*>(h->WL[l]), xin, static_cast<T*>(h->cat), batch, n, d, c.n_f,
-                               c.n_l, st);
-      }
-    }
-    if (s != WK_OK) break;
     {  // 4. residual + LN
       ProfScope ps(h, WK_KERNEL_RES_LN, st);
       const T* cat = static_cast<const T*>(h->cat);
       if (last)
-        s = run_res_ln<T, T, IO>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<IO*>(out), rows, d, h->eps,
-                                h->status, st);
+        s = run_res_ln<T, T, OUT>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<OUT*>(out), rows, d, h->eps,
+                                 h->status, st);
       else
         s = run_res_ln<T, T, T>(dv, cat, xin, h->g2[l], h->b2[l], static_cast<T*>(h->Xs[l % 2]), rows, d, h->eps,
                                h->status, st);
@@ -909,6 +1021,116 @@ wk_status forward32(wk_stack* h, const float* X, float* out, int64_t batch, cuda
     }
   }
   return s;
+}
+
+// Stack forward into the operand-type layer buffer, then the prediction head: the
+// hidden Linears on the tensor-core GEMM (ReLU), the one-output Linear and sigmoid.
+template <typename T, typename IO>
+wk_status predict16(wk_stack* h, const void* X, float* logit, float* prob, int64_t batch, cudaStream_t st) {
+  const DevInfo* dv = h->dv;
+  const int L = h->cfg.num_layers;
+  void* xl = h->Xs[(L - 1) % 2];
+  wk_status s = forward16<T, IO, T>(h, X, xl, batch, st);
+  if (s != WK_OK) return s;
+  const std::vector<int32_t>& dims = h->head_dims;
+  const int q = static_cast<int>(dims.size()) - 1;
+  const void* z = xl;
+  for (int j = 0; j + 1 < q && s == WK_OK; ++j) {
+    ProfScope ps(h, WK_KERNEL_HEAD, st);
+    if (h->head_maps.empty())
+      s = run_gemm_simt<T, T>(static_cast<const T*>(z), static_cast<const T*>(h->hT[j]), h->hc[j],
+                              static_cast<T*>(h->HH[j % 2]), batch, dims[j], dims[j + 1], dims[j + 1], 1, st);
+    else if (h->pair)
+      s = run_gemm_tc2<T, T>(dv, h->head_maps[j], mlp2_params(batch, dims[j], dims[j + 1], h->hc[j], 1, h->status),
+                             st);
+    else
+      s = run_gemm_tc<MODE_MLP, T, T>(dv, h->head_maps[j],
+                                       mlp_params(batch, dims[j], dims[j + 1], h->hc[j], 1, h->status), st);
+    z = h->HH[j % 2];
+  }
+  if (s != WK_OK) return s;
+  ProfScope ps(h, WK_KERNEL_HEAD, st);
+  return run_head_out<T>(dv, static_cast<const T*>(z), static_cast<const T*>(h->hT[q - 1]), h->hc[q - 1], logit, prob,
+                         batch, dims[q - 1], st);
+}
+
+template <typename T>
+wk_status build_head_maps(wk_stack* h) {
+  const std::vector<int32_t>& dims = h->head_dims;
+  const int q = static_cast<int>(dims.size()) - 1;
+  const int64_t B = h->maxb;
+  h->head_maps.clear();
+  bool tc = true;
+  for (int j = 0; j + 1 < q; ++j) tc = tc && mlp_tc_ok(B, dims[j], dims[j + 1], dims[j + 1]);
+  if (!tc || q < 2) return WK_OK;
+  h->head_maps.resize(q - 1);
+  const void* xl = h->Xs[(h->cfg.num_layers - 1) % 2];
+  for (int j = 0; j + 1 < q; ++j) {
+    GemmMaps& mp = h->head_maps[j];
+    const void* in = (j == 0) ? xl : h->HH[(j - 1) % 2];
+    if (!map_kmajor<T>(h->dv, &mp.A, in, dims[j], B, GEMM_BM) ||
+        !map_kmajor<T>(h->dv, &mp.B, h->hT[j], dims[j], dims[j + 1], h->pair ? 128 : GEMM_BN) ||
+        !map_out<T>(h->dv, &mp.C, h->HH[j % 2], dims[j + 1], B, dims[j + 1]))
+      return WK_ERR_UNSUPPORTED;
+  }
+  return WK_OK;
+}
+
+// The forward of a MoE stack with operand type T and caller type IO.
+template <typename T, typename IO>
+wk_status moe_forward16(wk_moe* h, const void* X, void* out, int64_t batch, cudaStream_t st) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int n = c.n, d = c.d, L = c.num_layers, E = h->E;
+  const int64_t rows = batch * n;
+  const int64_t nd = static_cast<int64_t>(n) * d;
+  wk_stack* p0 = h->ex[0];  // carries the MoE's own profiling records
+  wk_status s = WK_OK;
+  const void* x0 = X;
+  CUtensorMap lcb_x0;
+  if (sizeof(IO) != sizeof(T) || Half16<IO>::kBF16 != Half16<T>::kBF16) {
+    ProfScope ps(p0, WK_KERNEL_CONVERT, st);
+    s = run_convert<IO, T>(dv, X, h->Xm[1], rows * d, st);
+    if (s != WK_OK) return s;
+    x0 = h->Xm[1];
+    lcb_x0 = h->lcbX[1];
+  } else if (p0->tc_lcb && !map_lcb_x<T>(dv, &lcb_x0, X, n, d, batch)) {
+    return WK_ERR_CUDA;
+  }
+  for (int l = 0; l < L && s == WK_OK; ++l) {
+    const bool last = l == L - 1;
+    const T* xin = static_cast<const T*>(l == 0 ? x0 : h->Xm[(l - 1) % 2]);
+    const CUtensorMap& xmap = (l == 0) ? lcb_x0 : h->lcbX[(l - 1) % 2];
+    {
+      ProfScope ps(p0, WK_KERNEL_MOE_GATE, st);
+      s = run_moe_gate<T>(dv, xin, static_cast<const T*>(h->Wg[l]), h->bg[l], h->g, batch, nd, E, st);
+    }
+    for (int e = 0; e < E && s == WK_OK; ++e) s = layer_front16<T>(h->ex[e], l, xin, xmap, batch, st);
+    if (s != WK_OK) break;
+    MoePtrs mp{};
+    for (int e = 0; e < E; ++e) {
+      mp.cat[e] = h->ex[e]->cat;
+      mp.gamma[e] = h->ex[e]->g2[l];
+      mp.beta[e] = h->ex[e]->b2[l];
+    }
+    ProfScope ps(p0, WK_KERNEL_MOE_COMBINE, st);
+    if (last)
+      s = run_moe_combine<T, IO>(dv, mp, xin, h->g, static_cast<IO*>(out), rows, n, d, E, h->eps, st);
+    else
+      s = run_moe_combine<T, T>(dv, mp, xin, h->g, static_cast<T*>(h->Xm[l % 2]), rows, n, d, E, h->eps, st);
+  }
+  return s;
+}
+
+void free_moe(wk_moe* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaGetLastError();
+  for (wk_stack* e : h->ex) free_stack(e);
+  if (h->ws) cudaFree(h->ws);
+  if (h->wcopy) cudaFree(h->wcopy);
+  cudaGetLastError();
+  delete h;
 }
 
 wk_status read_status_word(unsigned* word, cudaStream_t st) {
@@ -1061,7 +1283,10 @@ const char* wk_status_string(wk_status s) {
   return "unknown status";
 }
 
-wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* weights, wk_stack** out) {
+// wk_stack_create; front_only: a stack whose layers another handle drives one front
+// at a time (an expert of a wk_moe): no layer buffers and no fused end-of-layer path.
+static wk_status stack_create_impl(const wk_stack_config* cfg, const wk_layer_weights* weights, wk_stack** out,
+                                   bool front_only) {
   if (!out || !weights) return WK_ERR_INVALID_ARG;
   *out = nullptr;
   wk_status st = validate_cfg(cfg);
@@ -1099,6 +1324,7 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   h->op = cfg->dtype == WK_F32 ? WK_F32 : (cfg->operand_dtype == WK_BF16 ? WK_BF16 : WK_F16);
   h->maxb = cfg->max_batch;
   h->dv = dv;
+  h->front_only = front_only;
   h->W.resize(L);
   h->b.resize(L);
   for (int l = 0; l < L; ++l) {
@@ -1203,9 +1429,9 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   const size_t o_cat = off;
   off += up(B * nd * es);
   const size_t o_x0 = off;
-  off += up(B * nd * es);
+  if (!front_only) off += up(B * nd * es);
   const size_t o_x1 = off;
-  off += up(B * nd * es);
+  if (!front_only) off += up(B * nd * es);
   const size_t o_status = off;
   off += 256;
   if (cudaMalloc(&h->ws, off) != cudaSuccess) {
@@ -1217,8 +1443,8 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   h->H[0] = h->ws + o_h0;
   h->H[1] = h->ws + o_h1;
   h->cat = h->ws + o_cat;
-  h->Xs[0] = h->ws + o_x0;
-  h->Xs[1] = h->ws + o_x1;
+  h->Xs[0] = front_only ? nullptr : h->ws + o_x0;
+  h->Xs[1] = front_only ? nullptr : h->ws + o_x1;
   h->status = reinterpret_cast<unsigned*>(h->ws + o_status);
   if (cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess) {
     cudaGetLastError();
@@ -1235,6 +1461,10 @@ wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* we
   }
   *out = h;
   return WK_OK;
+}
+
+wk_status wk_stack_create(const wk_stack_config* cfg, const wk_layer_weights* weights, wk_stack** out) {
+  return stack_create_impl(cfg, weights, out, false);
 }
 
 wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t batch, wk_stream_t stream) {
@@ -1531,6 +1761,302 @@ wk_status wk_layer_forward_noalloc(const wk_stack_config* cfg, const wk_layer_we
     s = run_res_ln<float, float, float>(dv, cat, Xf, w->out_ln_gamma, w->out_ln_beta, static_cast<float*>(out),
                                         batch * n, d, eps, dv->standalone_status, st);
   return s;
+}
+
+// ------------------------------------------------------------ prediction head
+
+wk_status wk_stack_set_head(wk_stack* h, const wk_head* head) {
+  if (!h || !head || h->front_only) return WK_ERR_INVALID_ARG;
+  const int q = head->num_linear;
+  if (q < 1 || !head->T || (q > 1 && !head->hidden)) return WK_ERR_INVALID_ARG;
+  if (h->op == WK_F32) return WK_ERR_UNSUPPORTED;
+  std::vector<int32_t> dims;
+  dims.push_back(h->cfg.n * h->cfg.d);
+  for (int j = 0; j + 1 < q; ++j) {
+    if (head->hidden[j] < 8 || head->hidden[j] % 8 != 0) return WK_ERR_UNSUPPORTED;
+    dims.push_back(head->hidden[j]);
+  }
+  dims.push_back(1);
+  for (int j = 0; j < q; ++j) {
+    if (!head->T[j] || !al16(head->T[j])) return WK_ERR_INVALID_ARG;
+    if (head->c && head->c[j] && !al16(head->c[j])) return WK_ERR_INVALID_ARG;
+  }
+  const DevInfo* dv = h->dv;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) {
+    cudaGetLastError();
+    return WK_ERR_INVALID_ARG;
+  }
+  cudaDeviceSynchronize();
+  if (h->head_copy) cudaFree(h->head_copy);
+  if (h->head_ws) cudaFree(h->head_ws);
+  h->head_copy = h->head_ws = nullptr;
+  h->HH[0] = h->HH[1] = nullptr;
+  h->head_dims.clear();
+  h->hT.clear();
+  h->hc.clear();
+  h->head_maps.clear();
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  wk_status st = WK_OK;
+  if (h->io != h->op) {
+    size_t total = 0;
+    for (int j = 0; j < q; ++j) total += up(static_cast<size_t>(dims[j]) * dims[j + 1] * 2);
+    if (cudaMalloc(&h->head_copy, total) != cudaSuccess) {
+      cudaGetLastError();
+      return WK_ERR_OOM;
+    }
+  }
+  uint8_t* p = h->head_copy;
+  for (int j = 0; j < q; ++j) {
+    const int64_t cnt = static_cast<int64_t>(dims[j]) * dims[j + 1];
+    if (h->io != h->op) {
+      const wk_status cs = h->io == WK_BF16 ? run_convert<bf16, f16>(dv, head->T[j], p, cnt, nullptr)
+                                            : run_convert<f16, bf16>(dv, head->T[j], p, cnt, nullptr);
+      if (cs != WK_OK) st = cs;
+      h->hT.push_back(p);
+      p += up(static_cast<size_t>(cnt) * 2);
+    } else {
+      h->hT.push_back(head->T[j]);
+    }
+    h->hc.push_back(head->c ? head->c[j] : nullptr);
+  }
+  int32_t hmax = 0;
+  for (int j = 1; j < q; ++j) hmax = std::max(hmax, dims[j]);
+  if (st == WK_OK && hmax > 0) {
+    const size_t one = up(static_cast<size_t>(h->maxb) * hmax * 2);
+    if (cudaMalloc(&h->head_ws, 2 * one) != cudaSuccess) {
+      cudaGetLastError();
+      st = WK_ERR_OOM;
+    } else {
+      h->HH[0] = h->head_ws;
+      h->HH[1] = h->head_ws + one;
+    }
+  }
+  h->head_dims = dims;
+  if (st == WK_OK) st = h->op == WK_F16 ? build_head_maps<f16>(h) : build_head_maps<bf16>(h);
+  if (st == WK_OK && cudaDeviceSynchronize() != cudaSuccess) st = WK_ERR_CUDA;
+  if (st != WK_OK) {
+    cudaGetLastError();
+    if (h->head_copy) cudaFree(h->head_copy);
+    if (h->head_ws) cudaFree(h->head_ws);
+    h->head_copy = h->head_ws = nullptr;
+    h->head_dims.clear();
+    h->hT.clear();
+    h->hc.clear();
+    h->head_maps.clear();
+  }
+  return st;
+}
+
+wk_status wk_stack_predict(wk_stack* h, const void* X, float* logit, float* prob, int64_t batch,
+                           wk_stream_t stream) {
+  if (!h || batch < 0 || batch > h->maxb || h->head_dims.empty()) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X || !logit || !al16(X)) return WK_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) {
+    cudaGetLastError();
+    return WK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (h->op == WK_F16)
+    return h->io == WK_BF16 ? predict16<f16, bf16>(h, X, logit, prob, batch, st)
+                            : predict16<f16, f16>(h, X, logit, prob, batch, st);
+  return h->io == WK_BF16 ? predict16<bf16, bf16>(h, X, logit, prob, batch, st)
+                          : predict16<bf16, f16>(h, X, logit, prob, batch, st);
+}
+
+// ------------------------------------------------------- mixture of experts
+
+wk_status wk_moe_create(const wk_stack_config* cfg, int32_t num_experts, const wk_layer_weights* experts,
+                        const wk_moe_gate* gates, wk_moe** out) {
+  if (!out || !experts || !gates || !cfg) return WK_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (num_experts < 1 || num_experts > MOE_MAX_E) return WK_ERR_INVALID_ARG;
+  wk_status st = validate_cfg(cfg);
+  if (st != WK_OK) return st;
+  if (cfg->dtype == WK_F32) return WK_ERR_UNSUPPORTED;
+  const int L = cfg->num_layers, E = num_experts;
+  for (int l = 0; l < L; ++l)
+    if (!gates[l].W_g || !al16(gates[l].W_g) || (gates[l].b_g && !al16(gates[l].b_g))) return WK_ERR_INVALID_ARG;
+  DevInfo* dv = nullptr;
+  st = dev_info(&dv);
+  if (st != WK_OK) return st;
+  wk_moe* h = new (std::nothrow) wk_moe();
+  if (!h) return WK_ERR_OOM;
+  h->device = dv->id;
+  h->cfg = *cfg;
+  h->cfg.mlp_hidden = nullptr;
+  h->E = E;
+  h->eps = cfg->ln_eps > 0.f ? cfg->ln_eps : 1e-5f;
+  h->io = cfg->dtype;
+  h->op = cfg->operand_dtype == WK_BF16 ? WK_BF16 : WK_F16;
+  h->maxb = cfg->max_batch;
+  h->dv = dv;
+  std::vector<wk_layer_weights> lw(L);
+  for (int e = 0; e < E; ++e) {
+    for (int l = 0; l < L; ++l) lw[l] = experts[static_cast<size_t>(l) * E + e];
+    wk_stack* x = nullptr;
+    st = stack_create_impl(cfg, lw.data(), &x, true);
+    if (st != WK_OK) {
+      free_moe(h);
+      return st;
+    }
+    h->ex.push_back(x);
+  }
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const size_t nd = static_cast<size_t>(cfg->n) * cfg->d;
+  const size_t gbytes = up(static_cast<size_t>(E) * nd * 2);
+  if (h->io != h->op) {
+    if (cudaMalloc(&h->wcopy, gbytes * L) != cudaSuccess) {
+      cudaGetLastError();
+      free_moe(h);
+      return WK_ERR_OOM;
+    }
+  }
+  for (int l = 0; l < L; ++l) {
+    if (h->io != h->op) {
+      uint8_t* dst = h->wcopy + gbytes * l;
+      const int64_t cnt = static_cast<int64_t>(E) * nd;
+      st = h->io == WK_BF16 ? run_convert<bf16, f16>(dv, gates[l].W_g, dst, cnt, nullptr)
+                            : run_convert<f16, bf16>(dv, gates[l].W_g, dst, cnt, nullptr);
+      h->Wg.push_back(dst);
+    } else {
+      h->Wg.push_back(gates[l].W_g);
+    }
+    h->bg.push_back(gates[l].b_g);
+  }
+  const int64_t B = h->maxb;
+  const size_t o_g = 0, o_x0 = up(static_cast<size_t>(B) * E * 4), o_x1 = o_x0 + up(B * nd * 2),
+               total = o_x1 + up(B * nd * 2);
+  if (st != WK_OK || cudaMalloc(&h->ws, total) != cudaSuccess) {
+    cudaGetLastError();
+    free_moe(h);
+    return st != WK_OK ? st : WK_ERR_OOM;
+  }
+  h->g = reinterpret_cast<float*>(h->ws + o_g);
+  h->Xm[0] = h->ws + o_x0;
+  h->Xm[1] = h->ws + o_x1;
+  if (h->ex[0]->tc_lcb) {
+    const bool ok = h->op == WK_F16 ? (map_lcb_x<f16>(dv, &h->lcbX[0], h->Xm[0], cfg->n, cfg->d, B) &&
+                                       map_lcb_x<f16>(dv, &h->lcbX[1], h->Xm[1], cfg->n, cfg->d, B))
+                                    : (map_lcb_x<bf16>(dv, &h->lcbX[0], h->Xm[0], cfg->n, cfg->d, B) &&
+                                       map_lcb_x<bf16>(dv, &h->lcbX[1], h->Xm[1], cfg->n, cfg->d, B));
+    if (!ok) {
+      free_moe(h);
+      return WK_ERR_UNSUPPORTED;
+    }
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    free_moe(h);
+    return WK_ERR_CUDA;
+  }
+  *out = h;
+  return WK_OK;
+}
+
+wk_status wk_moe_forward(wk_moe* h, const void* X, void* out, int64_t batch, wk_stream_t stream) {
+  if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X || !out || !al16(X) || !al16(out)) return WK_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(batch) * h->cfg.n * h->cfg.d * dtype_bytes(h->io);
+  const uint8_t* xa = static_cast<const uint8_t*>(X);
+  const uint8_t* oa = static_cast<const uint8_t*>(out);
+  if (xa < oa + bytes && oa < xa + bytes) return WK_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) {
+    cudaGetLastError();
+    return WK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (h->op == WK_F16)
+    return h->io == WK_BF16 ? moe_forward16<f16, bf16>(h, X, out, batch, st) : moe_forward16<f16, f16>(h, X, out, batch, st);
+  return h->io == WK_BF16 ? moe_forward16<bf16, bf16>(h, X, out, batch, st) : moe_forward16<bf16, f16>(h, X, out, batch, st);
+}
+
+wk_status wk_moe_sync_status(wk_moe* h, wk_stream_t stream) {
+  if (!h) return WK_ERR_INVALID_ARG;
+  wk_status first = WK_OK;
+  for (wk_stack* e : h->ex) {
+    const wk_status s = read_status_word(e->status, reinterpret_cast<cudaStream_t>(stream));
+    if (first == WK_OK) first = s;
+  }
+  return first;
+}
+
+wk_status wk_moe_set_profiling(wk_moe* h, int enable) {
+  if (!h) return WK_ERR_INVALID_ARG;
+  for (wk_stack* e : h->ex) e->prof = enable != 0;
+  return WK_OK;
+}
+
+wk_status wk_moe_kernel_times(wk_moe* h, double* total_ms, int64_t* launches) {
+  if (!h || !total_ms || !launches) return WK_ERR_INVALID_ARG;
+  for (int i = 0; i < WK_KERNEL_COUNT; ++i) {
+    total_ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  wk_status first = WK_OK;
+  for (wk_stack* e : h->ex) {
+    double t[WK_KERNEL_COUNT];
+    int64_t c[WK_KERNEL_COUNT];
+    const wk_status s = wk_stack_kernel_times(e, t, c);
+    if (first == WK_OK) first = s;
+    for (int i = 0; i < WK_KERNEL_COUNT; ++i) {
+      total_ms[i] += t[i];
+      launches[i] += c[i];
+    }
+  }
+  return first;
+}
+
+void wk_moe_destroy(wk_moe* h) { free_moe(h); }
+
+wk_status wk_moe_gate_softmax(const void* X, const void* W_g, const float* b_g, float* g, int64_t batch, int64_t nd,
+                              int32_t num_experts, wk_dtype dtype, wk_stream_t stream) {
+  if (batch < 0 || nd < 8 || nd % 8 != 0 || num_experts < 1 || num_experts > MOE_MAX_E) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X || !W_g || !g || !al16(X) || !al16(W_g) || (b_g && !al16(b_g))) return WK_ERR_INVALID_ARG;
+  if (dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WK_BF16)
+    return run_moe_gate<bf16>(dv, static_cast<const bf16*>(X), static_cast<const bf16*>(W_g), b_g, g, batch, nd,
+                              num_experts, st);
+  return run_moe_gate<f16>(dv, static_cast<const f16*>(X), static_cast<const f16*>(W_g), b_g, g, batch, nd,
+                           num_experts, st);
+}
+
+wk_status wk_moe_combine(const void* const* concats, const void* X, const float* g, const float* const* gammas,
+                         const float* const* betas, void* out, int64_t batch, int32_t n, int32_t d,
+                         int32_t num_experts, wk_dtype dtype, float eps, wk_stream_t stream) {
+  if (batch < 0 || n < 1 || d < 1 || num_experts < 1 || num_experts > MOE_MAX_E) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!concats || !X || !g || !gammas || !betas || !out || !al16(X) || !al16(out)) return WK_ERR_INVALID_ARG;
+  MoePtrs mp{};
+  for (int e = 0; e < num_experts; ++e) {
+    if (!concats[e] || !gammas[e] || !betas[e] || !al16(concats[e]) || !al16(gammas[e]) || !al16(betas[e]))
+      return WK_ERR_INVALID_ARG;
+    mp.cat[e] = concats[e];
+    mp.gamma[e] = gammas[e];
+    mp.beta[e] = betas[e];
+  }
+  if (dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  if (!res_ln_d_ok(d)) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  const float e = eps > 0.f ? eps : 1e-5f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t rows = batch * n;
+  if (dtype == WK_BF16)
+    return run_moe_combine<bf16, bf16>(dv, mp, static_cast<const bf16*>(X), g, static_cast<bf16*>(out), rows, n, d,
+                                       num_experts, e, st);
+  return run_moe_combine<f16, f16>(dv, mp, static_cast<const f16*>(X), g, static_cast<f16*>(out), rows, n, d,
+                                   num_experts, e, st);
 }
 
 }  // extern "C"

@@ -99,3 +99,27 @@ def test_null_handle_and_stand_alone_argument_checks(L):
     assert L.wk_res_ln(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 160, 1, ctypes.c_float(0), None) == wk.WK_ERR_INVALID_ARG
     assert L.wk_fm_ln(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 16, 16, 4, 0, ctypes.c_float(0), None) == wk.WK_OK
     assert L.wk_lcb(FAKE, FAKE, FAKE, 3, 16, 16, 8, 8, 7, None) == wk.WK_ERR_UNSUPPORTED
+
+
+def _moe_status(L, cfg, E, gate_addr=FAKE):
+    c, hid, m = wk._config(cfg, None, None, 0.0, None)
+    layers = _fake_layers(m, count=max(1, E))
+    keep = []
+    arr = wk._layer_array(layers, m, keep)
+    garr = (wk.WkMoeGate * 1)(wk.WkMoeGate(gate_addr, None))
+    h = ctypes.c_void_p()
+    return L.wk_moe_create(ctypes.byref(c), E, arr, garr, ctypes.byref(h))
+
+
+def test_moe_argument_errors_without_a_device(L):
+    assert _moe_status(L, _cfg(dtype="bf16"), 0) == wk.WK_ERR_INVALID_ARG
+    assert _moe_status(L, _cfg(dtype="bf16"), wk.WK_MOE_MAX_EXPERTS + 1) == wk.WK_ERR_INVALID_ARG
+    assert _moe_status(L, _cfg(dtype="f32"), 2) == wk.WK_ERR_UNSUPPORTED
+    assert _moe_status(L, _cfg(dtype="bf16"), 2, gate_addr=FAKE + 2) == wk.WK_ERR_INVALID_ARG
+    assert _moe_status(L, _cfg(dtype="bf16"), 2, gate_addr=0) == wk.WK_ERR_INVALID_ARG
+    with pytest.raises(wk.WkError) as ei:
+        wk.wk_moe_gate_softmax(FAKE, FAKE, None, FAKE, 4, 12, 2, "bf16", stream=0)  # nd not a multiple of 8
+    assert ei.value.status == wk.WK_ERR_INVALID_ARG
+    with pytest.raises(wk.WkError) as ei:
+        wk.wk_moe_combine([FAKE] * 9, FAKE, FAKE, [FAKE] * 9, [FAKE] * 9, FAKE, 4, 16, 16, "bf16", stream=0)
+    assert ei.value.status == wk.WK_ERR_INVALID_ARG
