@@ -213,6 +213,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head", action="store_true",
+                    help="each step also runs the prediction head (wk_stack_predict: logits and probabilities)")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16", "moe3_c2", "moe4_c3"])
     args = ap.parse_args()
@@ -263,6 +265,26 @@ def main():
             oh.copy_(out, non_blocking=True)
             stream.synchronize()
         e2e_api = "wk_moe_forward with a pinned host-to-device copy before and device-to-host copy after"
+    elif args.head:
+        layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
+        h = wk.wk_stack_create(cfg, layers, max_batch=B)
+        head = C.make_head_dev(cfg, device=dev)
+        wk.wk_stack_set_head(h, head)
+        logit = torch.empty((B,), device=dev)
+        prob = torch.empty((B,), device=dev)
+        api = dict(fwd=lambda x, o: wk.wk_stack_predict(h, x, logit, prob, stream=stream),
+                   status=lambda: wk.wk_stack_sync_status(h), prof=lambda on: wk.wk_stack_set_profiling(h, on),
+                   times=lambda: wk.wk_stack_kernel_times(h), destroy=lambda: wk.wk_stack_destroy(h))
+        w_tensors = [t for lw in layers for t in lw.values()] + list(head["T"]) + list(head["c"])
+        flops_ex = C.flops_per_example(cfg) + C.head_flops_per_example(cfg)
+        out = prob
+
+        def fwd_host(xh, oh):  # input copied in, the probabilities copied out
+            X.copy_(xh, non_blocking=True)
+            api["fwd"](X, None)
+            oh.copy_(prob, non_blocking=True)
+            stream.synchronize()
+        e2e_api = "wk_stack_predict with a pinned host-to-device copy of X and a device-to-host copy of prob"
     else:
         layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(cfg["layers"])]
         h = wk.wk_stack_create(cfg, layers, max_batch=B)
@@ -323,7 +345,7 @@ def main():
 
     # ---- end to end with host buffers
     xh = X.cpu().pin_memory()
-    oh = torch.empty_like(xh).pin_memory()
+    oh = torch.empty_like(out, device="cpu").pin_memory()
     fwd_host(xh, oh)  # warm the staging buffers
     barrier()
     t0 = time.perf_counter()
@@ -332,6 +354,7 @@ def main():
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     e2e_value = world * B * args.steps / e2e_s
     step_bytes = B * cfg["n"] * cfg["d"] * X.element_size()
+    out_bytes = oh.numel() * oh.element_size()
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -361,7 +384,10 @@ def main():
             "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32" if fp32 else "f16", "data": "synthetic",
-            "config": {"workload": args.workload + ": " + workload_desc(cfg), "per_gpu_batch": B,
+            "config": {"workload": args.workload + ": " + workload_desc(cfg) +
+                       (" + prediction head %d->%s->1, sigmoid" % (cfg["n"] * cfg["d"],
+                                                                    "->".join(str(v) for v in C.HEAD_HIDDEN))
+                        if args.head else ""), "per_gpu_batch": B,
                        "precision": precision,
                        "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
                        "l2": l2},
@@ -372,7 +398,7 @@ def main():
             "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "examples/s", "h2d_bytes_per_step": step_bytes,
-                    "d2h_bytes_per_step": step_bytes, "api": e2e_api},
+                    "d2h_bytes_per_step": out_bytes, "api": e2e_api},
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:

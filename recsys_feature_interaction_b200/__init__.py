@@ -21,8 +21,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
 WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
 WK_F32, WK_BF16, WK_F16 = 0, 1, 2
 (WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_CONVERT, WK_KERNEL_MOE_GATE,
- WK_KERNEL_MOE_COMBINE, WK_KERNEL_COUNT) = range(8)
-KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert", "moe_gate", "moe_combine")
+ WK_KERNEL_MOE_COMBINE, WK_KERNEL_HEAD, WK_KERNEL_COUNT) = range(9)
+KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert", "moe_gate", "moe_combine", "head")
 WK_MOE_MAX_EXPERTS = 8
 
 
@@ -337,3 +337,38 @@ def wk_moe_combine(concats, X, g, gammas, betas, out, batch, n, d, dtype, eps=0.
     bp = (ctypes.c_void_p * E)(*[_addr(t) for t in betas])
     _check(lib().wk_moe_combine(cp, _addr(X), _addr(g), gp, bp, _addr(out), int(batch), int(n), int(d), E,
                                 _dtype_code(dtype), float(eps), _stream(stream, X)), "wk_moe_combine")
+
+
+# ------------------------------------------------------------ prediction head
+
+class WkHead(ctypes.Structure):
+    _fields_ = [("num_linear", ctypes.c_int32), ("hidden", ctypes.POINTER(ctypes.c_int32)),
+                ("T", ctypes.POINTER(ctypes.c_void_p)), ("c", ctypes.POINTER(ctypes.c_void_p))]
+
+
+def wk_stack_set_head(h, head):
+    """head: mapping with T (list of q weights [out_j, in_j]) and c (list of q biases
+    or None entries); in_0 = n*d, out_{q-1} = 1."""
+    T = list(head["T"])
+    c = list(head.get("c") or [None] * len(T))
+    q = len(T)
+    hidden = [int(t.shape[0]) for t in T[:-1]]
+    hid = (ctypes.c_int32 * max(1, len(hidden)))(*hidden) if hidden else None
+    Tp = (ctypes.c_void_p * q)(*[_addr(t) for t in T])
+    cp = (ctypes.c_void_p * q)(*[_addr(t) for t in c])
+    hs = WkHead(q, hid, Tp, cp)
+    L = lib()
+    L.wk_stack_set_head.argtypes = [ctypes.c_void_p, ctypes.POINTER(WkHead)]
+    L.wk_stack_set_head.restype = ctypes.c_int
+    _check(L.wk_stack_set_head(h.ptr, ctypes.byref(hs)), "wk_stack_set_head")
+    h._keep.append((T, c, hid, Tp, cp))
+
+
+def wk_stack_predict(h, X, logit, prob=None, batch=None, stream=None):
+    b = X.shape[0] if batch is None else batch
+    L = lib()
+    L.wk_stack_predict.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_int64, ctypes.c_void_p]
+    L.wk_stack_predict.restype = ctypes.c_int
+    _check(L.wk_stack_predict(h.ptr, _addr(X), _addr(logit), _addr(prob), int(b), _stream(stream, X)),
+           "wk_stack_predict")

@@ -28,50 +28,60 @@ struct MoePtrs {
 // Gate logits and softmax. X [batch, nd] and W_g [E, nd] in T (nd a multiple of 8,
 // 16-byte aligned rows), b_g [E] fp32 or null, g [batch, E] fp32. A block takes EB
 // examples at a time: every thread walks 16-byte vectors of the flattened input with
-// the block's stride, reads each W_g vector once for the EB examples, and keeps EB x E
-// fp32 partial dot products; warps reduce by shuffles, then through shared memory.
-template <typename T>
+// the block's stride, two strides per step with all their loads issued before any
+// arithmetic (more bytes in flight per thread), reads each W_g vector once for the EB
+// examples and keeps EB x E fp32 partial dot products; warps reduce by shuffles, then
+// through shared memory. E is a template parameter so that the accumulators and the
+// W_g vectors in flight take exactly the registers the expert count needs.
+template <typename T, int E>
 __global__ void __launch_bounds__(256) moe_gate_kernel(const T* __restrict__ X, const T* __restrict__ Wg,
                                                       const float* __restrict__ bg, float* __restrict__ g,
-                                                      int64_t batch, int64_t nd, int E) {
+                                                      int64_t batch, int64_t nd) {
   constexpr int EB = MOE_GATE_EB;
-  __shared__ float red[8][EB][MOE_MAX_E];
+  constexpr int UNR = 2;
+  __shared__ float red[8][EB][E];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t nvec = nd / 8;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
   for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * EB; b0 < batch; b0 += static_cast<int64_t>(gridDim.x) * EB) {
-    float acc[EB][MOE_MAX_E];
+    float acc[EB][E];
 #pragma unroll
     for (int u = 0; u < EB; ++u)
 #pragma unroll
-      for (int e = 0; e < MOE_MAX_E; ++e) acc[u][e] = 0.f;
-    for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
-      float xv[EB][8];
+      for (int e = 0; e < E; ++e) acc[u][e] = 0.f;
+    for (int64_t v0 = threadIdx.x; v0 < nvec; v0 += UNR * blockDim.x) {
+      uint4 xv[UNR][EB], wv[UNR][E];
 #pragma unroll
-      for (int u = 0; u < EB; ++u) {
-        if (b0 + u < batch) {
-          Vec8<T>::load(X + (b0 + u) * nd + v * 8, xv[u]);
-        } else {
+      for (int s = 0; s < UNR; ++s) {
+        const int64_t v = v0 + s * blockDim.x;
+        const bool in = v < nvec;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) xv[u][j] = 0.f;
-        }
+        for (int u = 0; u < EB; ++u)
+          xv[s][u] = (in && b0 + u < batch) ? __ldg(reinterpret_cast<const uint4*>(X + (b0 + u) * nd + v * 8)) : zero;
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          wv[s][e] = in ? __ldg(reinterpret_cast<const uint4*>(Wg + static_cast<int64_t>(e) * nd + v * 8)) : zero;
       }
 #pragma unroll
-      for (int e = 0; e < MOE_MAX_E; ++e) {
-        if (e < E) {
-          float w[8];
-          Vec8<T>::load(Wg + static_cast<int64_t>(e) * nd + v * 8, w);
+      for (int s = 0; s < UNR; ++s)
 #pragma unroll
-          for (int u = 0; u < EB; ++u)
+        for (int u = 0; u < EB; ++u) {
+          float x8[8];
+          Vec8<T>::unpack(xv[s][u], x8);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[u][e] = fmaf(w[j], xv[u][j], acc[u][e]);
+          for (int e = 0; e < E; ++e) {
+            float w8[8];
+            Vec8<T>::unpack(wv[s][e], w8);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[u][e] = fmaf(w8[j], x8[j], acc[u][e]);
+          }
         }
-      }
     }
 #pragma unroll
     for (int u = 0; u < EB; ++u)
 #pragma unroll
-      for (int e = 0; e < MOE_MAX_E; ++e) {
+      for (int e = 0; e < E; ++e) {
         float s = acc[u][e];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -81,28 +91,24 @@ __global__ void __launch_bounds__(256) moe_gate_kernel(const T* __restrict__ X, 
     if (threadIdx.x < EB && b0 + threadIdx.x < batch) {
       const int u = threadIdx.x;
       const int nw = blockDim.x >> 5;
-      float z[MOE_MAX_E];
+      float z[E];
       float mx = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < MOE_MAX_E; ++e) {
-        if (e < E) {
-          float s = bg ? bg[e] : 0.f;
-          for (int w = 0; w < nw; ++w) s += red[w][u][e];
-          z[e] = s;
-          mx = fmaxf(mx, s);
-        }
+      for (int e = 0; e < E; ++e) {
+        float s = bg ? bg[e] : 0.f;
+        for (int w = 0; w < nw; ++w) s += red[w][u][e];
+        z[e] = s;
+        mx = fmaxf(mx, s);
       }
       float tot = 0.f;
 #pragma unroll
-      for (int e = 0; e < MOE_MAX_E; ++e)
-        if (e < E) {
-          z[e] = expf(z[e] - mx);
-          tot += z[e];
-        }
+      for (int e = 0; e < E; ++e) {
+        z[e] = expf(z[e] - mx);
+        tot += z[e];
+      }
       const float inv = 1.0f / tot;
 #pragma unroll
-      for (int e = 0; e < MOE_MAX_E; ++e)
-        if (e < E) g[(b0 + u) * E + e] = z[e] * inv;
+      for (int e = 0; e < E; ++e) g[(b0 + u) * E + e] = z[e] * inv;
     }
     __syncthreads();
   }
@@ -112,8 +118,8 @@ __global__ void __launch_bounds__(256) moe_gate_kernel(const T* __restrict__ X, 
 // d values; cat_e and x in the 16-bit type T, out in TO, g [batch, E] fp32. Lane
 // layout as in res_ln_kernel: G lanes per row (G a power of two dividing d/8), each
 // lane owning VPL 16-byte vectors. Per row the residual is loaded once and kept as
-// packed 16-bit words, each expert's concat row is loaded once (all VPL vectors
-// issued before any arithmetic) and kept packed too; each expert's statistics are two
+// packed 16-bit words, each expert's concat row is loaded once, one expert ahead of
+// the arithmetic (all VPL vectors at once), and kept packed too; each expert's statistics are two
 // fp32 passes over the unpacked values (registers: the fp32 mixture plus the packed
 // rows, which leaves room for two 256-thread blocks per SM at d = 160).
 template <int D, typename T, typename TO>
@@ -143,12 +149,21 @@ __global__ void __launch_bounds__(256, 2) moe_combine_kernel(const MoePtrs p, co
       for (int j = 0; j < 8; ++j) acc[k][j] = 0.f;
     }
     const int64_t b = ok ? r / n : 0;
+    uint4 cn[VPL];  // the next expert's concat row, loaded one expert ahead
+#pragma unroll
+    for (int k = 0; k < VPL; ++k)
+      cn[k] = ok ? __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(p.cat[0]) + r * D + (v0 + k * G) * 8))
+                 : zero;
     for (int e = 0; e < E; ++e) {
-      const T* cat = static_cast<const T*>(p.cat[e]);
       uint4 cr[VPL];
 #pragma unroll
-      for (int k = 0; k < VPL; ++k)
-        cr[k] = ok ? __ldg(reinterpret_cast<const uint4*>(cat + r * D + (v0 + k * G) * 8)) : zero;
+      for (int k = 0; k < VPL; ++k) cr[k] = cn[k];
+      if (e + 1 < E) {
+        const T* nxt = static_cast<const T*>(p.cat[e + 1]);
+#pragma unroll
+        for (int k = 0; k < VPL; ++k)
+          cn[k] = ok ? __ldg(reinterpret_cast<const uint4*>(nxt + r * D + (v0 + k * G) * 8)) : zero;
+      }
       // y = cat + x is recomputed from the packed words in each pass instead of being
       // held as fp32 (the unpack is a shift or a convert per element)
       float s = 0.f;

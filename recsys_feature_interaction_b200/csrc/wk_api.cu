@@ -564,13 +564,29 @@ wk_status run_head_out(const DevInfo* dv, const T* H, const T* w, const float* b
 
 // ------------------------------------------------------------ mixture of experts
 
+template <typename T, int E>
+wk_status run_moe_gate_e(const DevInfo* dv, const T* X, const T* Wg, const float* bg, float* g, int64_t batch,
+                         int64_t nd, cudaStream_t st) {
+  const int64_t need = (batch + MOE_GATE_EB - 1) / MOE_GATE_EB;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, static_cast<int64_t>(dv->sms) * 8)));
+  moe_gate_kernel<T, E><<<grid, 256, 0, st>>>(X, Wg, bg, g, batch, nd);
+  return launch_status();
+}
+
 template <typename T>
 wk_status run_moe_gate(const DevInfo* dv, const T* X, const T* Wg, const float* bg, float* g, int64_t batch,
                        int64_t nd, int E, cudaStream_t st) {
-  const int64_t need = (batch + MOE_GATE_EB - 1) / MOE_GATE_EB;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, static_cast<int64_t>(dv->sms) * 8)));
-  moe_gate_kernel<T><<<grid, 256, 0, st>>>(X, Wg, bg, g, batch, nd, E);
-  return launch_status();
+  switch (E) {
+    case 1: return run_moe_gate_e<T, 1>(dv, X, Wg, bg, g, batch, nd, st);
+    case 2: return run_moe_gate_e<T, 2>(dv, X, Wg, bg, g, batch, nd, st);
+    case 3: return run_moe_gate_e<T, 3>(dv, X, Wg, bg, g, batch, nd, st);
+    case 4: return run_moe_gate_e<T, 4>(dv, X, Wg, bg, g, batch, nd, st);
+    case 5: return run_moe_gate_e<T, 5>(dv, X, Wg, bg, g, batch, nd, st);
+    case 6: return run_moe_gate_e<T, 6>(dv, X, Wg, bg, g, batch, nd, st);
+    case 7: return run_moe_gate_e<T, 7>(dv, X, Wg, bg, g, batch, nd, st);
+    case 8: return run_moe_gate_e<T, 8>(dv, X, Wg, bg, g, batch, nd, st);
+    default: return WK_ERR_UNSUPPORTED;
+  }
 }
 
 template <int D, typename T, typename TO>

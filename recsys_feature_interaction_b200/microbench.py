@@ -1,7 +1,7 @@
 """Times one step of the Wukong layer alone through its stand-alone C-ABI entry point.
 
-    python -m recsys_feature_interaction_b200.microbench --kernel fm_ln|mlp_gemm|lcb|res_ln
-        [--workload c4_bf16] [--batch B] [--iters K] [--dtype f16|bf16] [--layer-linear j]
+    python -m recsys_feature_interaction_b200.microbench --kernel fm_ln|mlp_gemm|lcb|res_ln|moe_gate|moe_combine
+        [--workload c4_bf16] [--batch B] [--iters K] [--dtype f16|bf16] [--layer-linear j] [--experts E]
 
 Inputs are synthetic (the seeded generator), on the device, in the workload's
 shapes. Prints one JSON line with the mean CUDA-event time per launch and the
@@ -20,7 +20,7 @@ if ROOT not in sys.path:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", required=True, choices=["fm_ln", "mlp_gemm", "lcb", "res_ln"])
+    ap.add_argument("--kernel", required=True, choices=["fm_ln", "mlp_gemm", "lcb", "res_ln", "moe_gate", "moe_combine"])
     ap.add_argument("--workload", default="c4_bf16")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--iters", type=int, default=10)
@@ -28,6 +28,7 @@ def main():
     ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"])
     ap.add_argument("--layer-linear", type=int, default=0, help="which MLP Linear (mlp_gemm)")
     ap.add_argument("--no-affine", action="store_true", help="fm_ln without gamma/beta (as a stack runs it)")
+    ap.add_argument("--experts", type=int, default=4, help="experts (moe_gate, moe_combine)")
     args = ap.parse_args()
 
     import torch
@@ -37,7 +38,7 @@ def main():
     from synth import configs as C
 
     build.build()
-    cfg = C.CONFIGS[args.workload]
+    cfg = C.MOE_CONFIGS[args.workload] if args.workload in C.MOE_CONFIGS else C.CONFIGS[args.workload]
     B = args.batch or cfg["batch"]
     n, d, k, n_f, n_l = cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], cfg["n_l"]
     tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
@@ -74,6 +75,26 @@ def main():
             wk.wk_lcb(WL, X, cat, B, n, d, n_f, n_l, args.dtype)
         flops = 2 * n_l * n * d * B
         bytes_ = (n * d + n_l * d) * es * B
+    elif args.kernel == "moe_gate":
+        E = args.experts
+        Wg = (torch.randn((E, n * d), device=dev) / (n * d) ** 0.5).to(tdt)
+        bg = torch.randn((E,), device=dev)
+        g = torch.empty((B, E), device=dev)
+
+        def run():
+            wk.wk_moe_gate_softmax(X, Wg, bg, g, B, n * d, E, args.dtype)
+        flops = 2 * E * n * d * B
+        bytes_ = (n * d * es + E * 4) * B
+    elif args.kernel == "moe_combine":
+        E = args.experts
+        cats = [torch.randn((B, n, d), device=dev).to(tdt) for _ in range(E)]
+        g = torch.softmax(torch.randn((B, E), device=dev), dim=1)
+        out = torch.empty_like(X)
+
+        def run():
+            wk.wk_moe_combine(cats, X, g, [w["out_gamma"]] * E, [w["out_beta"]] * E, out, B, n, d, args.dtype)
+        flops = 0
+        bytes_ = (E + 2) * n * d * es * B
     else:
         cat = torch.randn((B, n, d), device=dev).to(tdt)
         out = torch.empty_like(X)

@@ -257,3 +257,40 @@ def moe_flops_per_example(cfg):
     gate's 2 * E * n * d per layer."""
     per_layer = flops_per_example(dict(cfg, layers=1))
     return cfg["layers"] * (cfg["experts"] * per_layer + 2 * cfg["experts"] * cfg["n"] * cfg["d"])
+
+
+# ------------------------------------------------------------ prediction head
+#
+# The Wukong page (section 2.2) follows the stacked layers with an MLP that produces
+# the prediction and gives it no sizes. The workloads' head: flatten (n*d) -> 1024 ->
+# 256 -> 1 with ReLU between, T_j ~ N(0, 1/in_j), c_j ~ N(0, 0.1^2) (non-zero so the
+# bias path is exercised), each tensor on its own stream.
+HEAD_HIDDEN = [1024, 256]
+
+
+def head_specs(cfg, hidden=None):
+    hidden = HEAD_HIDDEN if hidden is None else list(hidden)
+    dims = [cfg["n"] * cfg["d"]] + hidden + [1]
+    wd = "f32" if cfg["dtype"] == "f32" else "bf16"
+    specs = {}
+    for j in range(len(dims) - 1):
+        specs["T%d" % j] = ((dims[j + 1], dims[j]), "normal", 900000 + 10 * j, 0.0, 1.0 / math.sqrt(dims[j]), wd)
+        specs["c%d" % j] = ((dims[j + 1],), "normal", 900000 + 10 * j + 1, 0.0, 0.1, "f32")
+    return specs
+
+
+def make_head_host(cfg, hidden=None):
+    """[(T_j, c_j)] as host arrays (bf16 bits or float32)."""
+    h = _host_from_specs(head_specs(cfg, hidden))
+    return [(h["T%d" % j], h["c%d" % j]) for j in range(len(h) // 2)]
+
+
+def make_head_dev(cfg, hidden=None, device="cuda"):
+    h = _dev_from_specs(head_specs(cfg, hidden), device)
+    return {"T": [h["T%d" % j] for j in range(len(h) // 2)], "c": [h["c%d" % j] for j in range(len(h) // 2)]}
+
+
+def head_flops_per_example(cfg, hidden=None):
+    hidden = HEAD_HIDDEN if hidden is None else list(hidden)
+    dims = [cfg["n"] * cfg["d"]] + hidden + [1]
+    return 2 * sum(dims[j] * dims[j + 1] for j in range(len(dims) - 1))

@@ -123,3 +123,9 @@ def test_moe_argument_errors_without_a_device(L):
     with pytest.raises(wk.WkError) as ei:
         wk.wk_moe_combine([FAKE] * 9, FAKE, FAKE, [FAKE] * 9, [FAKE] * 9, FAKE, 4, 16, 16, "bf16", stream=0)
     assert ei.value.status == wk.WK_ERR_INVALID_ARG
+
+
+def test_kernel_kind_count_matches_the_header():
+    text = open(os.path.join(ROOT, "include", "wukong.h")).read()
+    m = re.search(r"WK_KERNEL_COUNT\s*=\s*(\d+)", text)
+    assert m and int(m.group(1)) == wk.WK_KERNEL_COUNT == len(wk.KERNEL_NAMES)
