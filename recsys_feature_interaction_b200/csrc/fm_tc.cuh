@@ -54,6 +54,10 @@ struct FmTcCfg {
   static constexpr int STAGES_RAW = (BUDGET - ZB - PAD - 1024 - 512) / SLOT;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int SMEM = 1024 + STAGES * SLOT + PAD + ZB + 512;
+  // LayerNorm from registers when a thread's share of F (one row per chunk, k values
+  // each) fits: the 2-, 4- and wide 2-layer shapes; the 8-layer shape (4 x 64) reads TMEM
+  // in three passes instead.
+  static constexpr bool REGLN = NCH * K <= 160 && (K == 16 || K == 24 || K == 32);
   static_assert(ZCOL + NCH * KP <= TMEM_COLS, "TMEM columns");
   static_assert(STAGES >= 2, "shared memory");
   static_assert(D % 32 == 0 && N % 16 == 0 && K % 4 == 0 && K <= 64, "shape");
@@ -61,6 +65,25 @@ struct FmTcCfg {
 };
 
 constexpr int FMTC_THREADS = 192;
+
+// 16- and 8-column TMEM loads (32 lanes x 32 bits): the register-resident LayerNorm
+// reads exactly k columns per chunk.
+__device__ __forceinline__ void fmtc_tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void fmtc_tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
 
 // Shared address of Z operand element row t, 16-byte unit j (MN-major, KP columns).
 template <class C>
@@ -263,93 +286,176 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(zready);
 
-      // LayerNorm over the n*k values of F (TMEM), three passes
-      if (ok) ok = mbar_wait(ffull, eph, status);
-      tc_fence_after();
-      float part = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < C::NCH; ++c) {
-        const int row = c * C::R + q * 32 + lane;
+      if constexpr (C::REGLN) {
+        // The LayerNorm from registers: each thread's F values (one row per chunk, k
+        // columns) are read from TMEM once, all chunks before one wait; TMEM is handed
+        // back to the MMA warp at once, and mean, variance and the output are computed
+        // from registers (two passes over them).
+        if (ok) ok = mbar_wait(ffull, eph, status);
+        tc_fence_after();
+        uint32_t fr[C::NCH][C::K];
 #pragma unroll
-        for (int h = 0; h < C::KP / 32; ++h) {
-          uint32_t r[32];
-          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
-          tmem_ld_wait();
-          if (row < C::N) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (h * 32 + j < C::K) part += __uint_as_float(r[j]);
+        for (int c = 0; c < C::NCH; ++c) {
+          const uint32_t ta = tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP);
+          if constexpr (C::K == 32) {
+            tmem_ld32(ta, reinterpret_cast<uint32_t(&)[32]>(fr[c][0]));
+          } else if constexpr (C::K == 24) {
+            fmtc_tmem_ld16(ta, reinterpret_cast<uint32_t(&)[16]>(fr[c][0]));
+            fmtc_tmem_ld8(ta + 16, reinterpret_cast<uint32_t(&)[8]>(fr[c][16]));
+          } else {
+            fmtc_tmem_ld16(ta, reinterpret_cast<uint32_t(&)[16]>(fr[c][0]));
           }
         }
-      }
-      part = warp_sum(part);
-      if (lane == 0) red[ew] = part;
-      named_bar(1, 128);
-      const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
-      float qs = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < C::NCH; ++c) {
-        const int row = c * C::R + q * 32 + lane;
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(fempty);  // F is in registers: the next pass B may overwrite it
+        float part = 0.f;
 #pragma unroll
-        for (int h = 0; h < C::KP / 32; ++h) {
-          uint32_t r[32];
-          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
-          tmem_ld_wait();
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
           if (row < C::N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (h * 32 + j < C::K) {
-                const float dv = __uint_as_float(r[j]) - mean;
-                qs += dv * dv;
+            for (int j = 0; j < C::K; ++j) part += __uint_as_float(fr[c][j]);
+          }
+        }
+        part = warp_sum(part);
+        if (lane == 0) red[ew] = part;
+        named_bar(1, 128);
+        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+        float qs = 0.f;
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+          if (row < C::N) {
+#pragma unroll
+            for (int j = 0; j < C::K; ++j) {
+              const float dv = __uint_as_float(fr[c][j]) - mean;
+              qs = fmaf(dv, dv, qs);
+            }
+          }
+        }
+        qs = warp_sum(qs);
+        if (lane == 0) red[4 + ew] = qs;
+        named_bar(1, 128);
+        const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
+        T* ab = A0 + b * (C::N * C::K);
+        const bool affine = gamma != nullptr;
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+          if (row < C::N) {
+            T* o = ab + row * C::K;
+#pragma unroll
+            for (int j = 0; j < C::K; j += 8) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = (__uint_as_float(fr[c][j + i]) - mean) * rstd;
+              if (affine) {
+                const float* gp = gamma + row * C::K + j;
+                const float* bp = beta + row * C::K + j;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = v[i] * __ldg(gp + i) + __ldg(bp + i);
               }
+              uint4 u;
+              u.x = Half16<T>::pack2(v[0], v[1]);
+              u.y = Half16<T>::pack2(v[2], v[3]);
+              u.z = Half16<T>::pack2(v[4], v[5]);
+              u.w = Half16<T>::pack2(v[6], v[7]);
+              *reinterpret_cast<uint4*>(o + j) = u;
+            }
           }
         }
-      }
-      qs = warp_sum(qs);
-      if (lane == 0) red[4 + ew] = qs;
-      named_bar(1, 128);
-      const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
-      T* ab = A0 + b * (C::N * C::K);
-      const bool affine = gamma != nullptr;
-#pragma unroll 1
-      for (int c = 0; c < C::NCH; ++c) {
-        const int row = c * C::R + q * 32 + lane;
-#pragma unroll
-        for (int h = 0; h < C::KP / 32; ++h) {
-          uint32_t r[32];
-          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
-          tmem_ld_wait();
-          if (row < C::N) {
-            const float* g = affine ? gamma + row * C::K + h * 32 : nullptr;
-            const float* bt = affine ? beta + row * C::K + h * 32 : nullptr;
-            T* o = ab + row * C::K + h * 32;
-#pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              if (h * 32 + j < C::K) {
-                // gamma == nullptr: the affine step lives in the next Linear (normalised values only)
-                const float4 one = make_float4(1.f, 1.f, 1.f, 1.f), zero = make_float4(0.f, 0.f, 0.f, 0.f);
-                const float4 g0 = affine ? __ldg(reinterpret_cast<const float4*>(g + j)) : one;
-                const float4 g1 = affine ? __ldg(reinterpret_cast<const float4*>(g + j + 4)) : one;
-                const float4 b0 = affine ? __ldg(reinterpret_cast<const float4*>(bt + j)) : zero;
-                const float4 b1 = affine ? __ldg(reinterpret_cast<const float4*>(bt + j + 4)) : zero;
-                uint4 u;
-                u.x = Half16<T>::pack2((__uint_as_float(r[j + 0]) - mean) * rstd * g0.x + b0.x,
-                                       (__uint_as_float(r[j + 1]) - mean) * rstd * g0.y + b0.y);
-                u.y = Half16<T>::pack2((__uint_as_float(r[j + 2]) - mean) * rstd * g0.z + b0.z,
-                                       (__uint_as_float(r[j + 3]) - mean) * rstd * g0.w + b0.w);
-                u.z = Half16<T>::pack2((__uint_as_float(r[j + 4]) - mean) * rstd * g1.x + b1.x,
-                                       (__uint_as_float(r[j + 5]) - mean) * rstd * g1.y + b1.y);
-                u.w = Half16<T>::pack2((__uint_as_float(r[j + 6]) - mean) * rstd * g1.z + b1.z,
-                                       (__uint_as_float(r[j + 7]) - mean) * rstd * g1.w + b1.w);
-                *reinterpret_cast<uint4*>(o + j) = u;
+        named_bar(1, 128);  // every epilogue warp is past its reads of red[]
+      } else {
+        // LayerNorm over the n*k values of F (TMEM), three passes
+        if (ok) ok = mbar_wait(ffull, eph, status);
+        tc_fence_after();
+        float part = 0.f;
+  #pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+  #pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
+            tmem_ld_wait();
+            if (row < C::N) {
+  #pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (h * 32 + j < C::K) part += __uint_as_float(r[j]);
+            }
+          }
+        }
+        part = warp_sum(part);
+        if (lane == 0) red[ew] = part;
+        named_bar(1, 128);
+        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+        float qs = 0.f;
+  #pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+  #pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
+            tmem_ld_wait();
+            if (row < C::N) {
+  #pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (h * 32 + j < C::K) {
+                  const float dv = __uint_as_float(r[j]) - mean;
+                  qs += dv * dv;
+                }
+            }
+          }
+        }
+        qs = warp_sum(qs);
+        if (lane == 0) red[4 + ew] = qs;
+        named_bar(1, 128);
+        const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
+        T* ab = A0 + b * (C::N * C::K);
+        const bool affine = gamma != nullptr;
+  #pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+  #pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::ZCOL + c * C::KP + h * 32), r);
+            tmem_ld_wait();
+            if (row < C::N) {
+              const float* g = affine ? gamma + row * C::K + h * 32 : nullptr;
+              const float* bt = affine ? beta + row * C::K + h * 32 : nullptr;
+              T* o = ab + row * C::K + h * 32;
+  #pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                if (h * 32 + j < C::K) {
+                  // gamma == nullptr: the affine step lives in the next Linear (normalised values only)
+                  const float4 one = make_float4(1.f, 1.f, 1.f, 1.f), zero = make_float4(0.f, 0.f, 0.f, 0.f);
+                  const float4 g0 = affine ? __ldg(reinterpret_cast<const float4*>(g + j)) : one;
+                  const float4 g1 = affine ? __ldg(reinterpret_cast<const float4*>(g + j + 4)) : one;
+                  const float4 b0 = affine ? __ldg(reinterpret_cast<const float4*>(bt + j)) : zero;
+                  const float4 b1 = affine ? __ldg(reinterpret_cast<const float4*>(bt + j + 4)) : zero;
+                  uint4 u;
+                  u.x = Half16<T>::pack2((__uint_as_float(r[j + 0]) - mean) * rstd * g0.x + b0.x,
+                                         (__uint_as_float(r[j + 1]) - mean) * rstd * g0.y + b0.y);
+                  u.y = Half16<T>::pack2((__uint_as_float(r[j + 2]) - mean) * rstd * g0.z + b0.z,
+                                         (__uint_as_float(r[j + 3]) - mean) * rstd * g0.w + b0.w);
+                  u.z = Half16<T>::pack2((__uint_as_float(r[j + 4]) - mean) * rstd * g1.x + b1.x,
+                                         (__uint_as_float(r[j + 5]) - mean) * rstd * g1.y + b1.y);
+                  u.w = Half16<T>::pack2((__uint_as_float(r[j + 6]) - mean) * rstd * g1.z + b1.z,
+                                         (__uint_as_float(r[j + 7]) - mean) * rstd * g1.w + b1.w);
+                  *reinterpret_cast<uint4*>(o + j) = u;
+                }
               }
             }
           }
         }
+        tc_fence_before();
+        named_bar(1, 128);  // every epilogue warp is past its reads of red[] and F
+        if (lane == 0) mbar_arrive(fempty);
       }
-      tc_fence_before();
-      named_bar(1, 128);  // every epilogue warp is past its reads of red[] and F
-      if (lane == 0) mbar_arrive(fempty);
       eph ^= 1u;
     }
   }

@@ -567,7 +567,7 @@ wk_status run_head_out(const DevInfo* dv, const T* H, const T* w, const float* b
 template <typename T, int E>
 wk_status run_moe_gate_e(const DevInfo* dv, const T* X, const T* Wg, const float* bg, float* g, int64_t batch,
                          int64_t nd, cudaStream_t st) {
-  const int64_t need = (batch + MOE_GATE_EB - 1) / MOE_GATE_EB;
+  const int64_t need = (batch + 7) / 8;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(need, static_cast<int64_t>(dv->sms) * 8)));
   moe_gate_kernel<T, E><<<grid, 256, 0, st>>>(X, Wg, bg, g, batch, nd);
   return launch_status();
@@ -589,9 +589,28 @@ wk_status run_moe_gate(const DevInfo* dv, const T* X, const T* Wg, const float* 
   }
 }
 
+// The ring-fed mixture kernel (moe_combine_ring_kernel) unless the environment sets
+// WK_MOE_RING=0 (then the register-only moe_combine_kernel).
+bool use_moe_ring() {
+  static const bool on = [] {
+    const char* e = getenv("WK_MOE_RING");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int D, typename T, typename TO>
 wk_status run_moe_combine_d(const DevInfo* dv, const MoePtrs& p, const T* x, const float* g, TO* out, int64_t rows,
-                            int n, int E, float eps, cudaStream_t st) {
+                            int n, int E, float eps, unsigned* status, cudaStream_t st) {
+  if (use_moe_ring()) {
+    using R = MoeRing<D>;
+    wk_status s = smem_attr(dv, reinterpret_cast<const void*>(moe_combine_ring_kernel<D, T, TO>), R::SMEM);
+    if (s != WK_OK) return s;
+    const int64_t tiles = (rows + R::R - 1) / R::R;
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, dv->sms)));
+    moe_combine_ring_kernel<D, T, TO><<<grid, R::THREADS, R::SMEM, st>>>(p, x, g, out, rows, n, E, eps, status);
+    return launch_status();
+  }
   constexpr int G = res_ln_lanes(D / 8);
   constexpr int rows_per_block = 8 * (32 / G);
   int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
@@ -602,15 +621,15 @@ wk_status run_moe_combine_d(const DevInfo* dv, const MoePtrs& p, const T* x, con
 
 template <typename T, typename TO>
 wk_status run_moe_combine(const DevInfo* dv, const MoePtrs& p, const T* x, const float* g, TO* out, int64_t rows,
-                          int n, int d, int E, float eps, cudaStream_t st) {
+                          int n, int d, int E, float eps, unsigned* status, cudaStream_t st) {
   switch (d) {
-    case 16: return run_moe_combine_d<16>(dv, p, x, g, out, rows, n, E, eps, st);
-    case 32: return run_moe_combine_d<32>(dv, p, x, g, out, rows, n, E, eps, st);
-    case 64: return run_moe_combine_d<64>(dv, p, x, g, out, rows, n, E, eps, st);
-    case 128: return run_moe_combine_d<128>(dv, p, x, g, out, rows, n, E, eps, st);
-    case 160: return run_moe_combine_d<160>(dv, p, x, g, out, rows, n, E, eps, st);
-    case 192: return run_moe_combine_d<192>(dv, p, x, g, out, rows, n, E, eps, st);
-    case 256: return run_moe_combine_d<256>(dv, p, x, g, out, rows, n, E, eps, st);
+    case 16: return run_moe_combine_d<16>(dv, p, x, g, out, rows, n, E, eps, status, st);
+    case 32: return run_moe_combine_d<32>(dv, p, x, g, out, rows, n, E, eps, status, st);
+    case 64: return run_moe_combine_d<64>(dv, p, x, g, out, rows, n, E, eps, status, st);
+    case 128: return run_moe_combine_d<128>(dv, p, x, g, out, rows, n, E, eps, status, st);
+    case 160: return run_moe_combine_d<160>(dv, p, x, g, out, rows, n, E, eps, status, st);
+    case 192: return run_moe_combine_d<192>(dv, p, x, g, out, rows, n, E, eps, status, st);
+    case 256: return run_moe_combine_d<256>(dv, p, x, g, out, rows, n, E, eps, status, st);
     default: return WK_ERR_UNSUPPORTED;
   }
 }
@@ -1131,9 +1150,10 @@ wk_status moe_forward16(wk_moe* h, const void* X, void* out, int64_t batch, cuda
     }
     ProfScope ps(p0, WK_KERNEL_MOE_COMBINE, st);
     if (last)
-      s = run_moe_combine<T, IO>(dv, mp, xin, h->g, static_cast<IO*>(out), rows, n, d, E, h->eps, st);
+      s = run_moe_combine<T, IO>(dv, mp, xin, h->g, static_cast<IO*>(out), rows, n, d, E, h->eps, p0->status, st);
     else
-      s = run_moe_combine<T, T>(dv, mp, xin, h->g, static_cast<T*>(h->Xm[l % 2]), rows, n, d, E, h->eps, st);
+      s = run_moe_combine<T, T>(dv, mp, xin, h->g, static_cast<T*>(h->Xm[l % 2]), rows, n, d, E, h->eps, p0->status,
+                                st);
   }
   return s;
 }
@@ -2070,9 +2090,9 @@ wk_status wk_moe_combine(const void* const* concats, const void* X, const float*
   const int64_t rows = batch * n;
   if (dtype == WK_BF16)
     return run_moe_combine<bf16, bf16>(dv, mp, static_cast<const bf16*>(X), g, static_cast<bf16*>(out), rows, n, d,
-                                       num_experts, e, st);
+                                       num_experts, e, dv->standalone_status, st);
   return run_moe_combine<f16, f16>(dv, mp, static_cast<const f16*>(X), g, static_cast<f16*>(out), rows, n, d,
-                                   num_experts, e, st);
+                                   num_experts, e, dv->standalone_status, st);
 }
 
 }  // extern "C"

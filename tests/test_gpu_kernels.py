@@ -163,7 +163,7 @@ def test_res_ln(rows, d, dt):
         assert max_scaled_err(got[r], oracle.layernorm(y[r], f64(g), f64(be))) <= tol, r
 
 
-@pytest.mark.parametrize("batch,n,d,k", [(160, 512, 160, 64), (170, 720, 32, 24)])
+@pytest.mark.parametrize("batch,n,d,k", [(160, 512, 160, 64), (170, 720, 32, 24), (150, 256, 160, 32), (200, 64, 128, 16)])
 def test_fm_ln_without_affine(batch, n, d, k):
     """NULL gamma/beta: A0 holds the normalised FM values (how a stack calls it)."""
     X = host_normal((batch, n, d), 26, dtype="f16")
