@@ -53,7 +53,20 @@ struct FmTcCfg {
   static constexpr int BUDGET = 220 * 1024;
   static constexpr int STAGES_RAW = (BUDGET - ZB - PAD - 1024 - 512) / SLOT;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int SMEM = 1024 + STAGES * SLOT + PAD + ZB + 512;
+  static constexpr int SMEM_RING = 1024 + STAGES * SLOT + PAD + ZB + 512;
+  // Example-resident mode, when two examples' X fit: a slot holds all NCH chunks of one
+  // example and Y has its own region, loaded once per CTA. Pass A and pass B read the
+  // same slot, so an example's X crosses HBM -> SM once, and the next examples' loads
+  // never wait for this example's pass B to release ring slots.
+  static constexpr int EXB = NCH * XBOXES * XBOXB;              // X bytes per example slot
+  static constexpr int YREG = NCH * YB;                         // resident Y
+  static constexpr int OVER_R = (MTZ * (R / XBOXW) - XBOXES) * XBOXB;
+  static constexpr int PAD_R = OVER_R > 0 ? ((OVER_R + 1023) / 1024) * 1024 : 0;
+  static constexpr int ES_RAW = (BUDGET - YREG - ZB - PAD_R - 1024 - 512) / EXB;
+  static constexpr bool RES = ES_RAW >= 2;
+  static constexpr int ES = ES_RAW > 4 ? 4 : (ES_RAW < 1 ? 1 : ES_RAW);
+  static constexpr int SMEM_RES = 1024 + YREG + ES * EXB + PAD_R + ZB + 512;
+  static constexpr int SMEM = RES ? SMEM_RES : SMEM_RING;
   // LayerNorm from registers when a thread's share of F (one row per chunk, k values
   // each) fits: the 2-, 4- and wide 2-layer shapes; the 8-layer shape (4 x 64) reads TMEM
   // in three passes instead.
@@ -99,27 +112,33 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
                     int64_t batch, float eps, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* ring = smem;
-  uint8_t* zb = ring + C::STAGES * C::SLOT + C::PAD;
+  // ring mode: [STAGES slots of (X chunk, Y chunk)][PAD][Z][red, barriers]
+  // resident mode: [Y region][ES example slots][PAD_R][Z][red, barriers]
+  constexpr int NSLOT = C::RES ? C::ES : C::STAGES;
+  uint8_t* yreg = smem;                                      // resident mode only
+  uint8_t* ring = C::RES ? smem + C::YREG : smem;
+  uint8_t* zb = C::RES ? ring + C::ES * C::EXB + C::PAD_R : ring + C::STAGES * C::SLOT + C::PAD;
   float* red = reinterpret_cast<float*>(zb + C::ZB);       // [2][4] partial sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(red + 8);
-  uint64_t* full = bars;                                    // [STAGES]
-  uint64_t* empty = bars + C::STAGES;                       // [STAGES]
-  uint64_t* zfull = bars + 2 * C::STAGES;                   // MMA -> epilogue: Z ready in TMEM
+  uint64_t* full = bars;                                    // [NSLOT]
+  uint64_t* empty = bars + NSLOT;                           // [NSLOT]
+  uint64_t* zfull = bars + 2 * NSLOT;                       // MMA -> epilogue: Z ready in TMEM
   uint64_t* zready = zfull + 1;                             // epilogue -> MMA: Z operand in smem
   uint64_t* ffull = zfull + 2;                              // MMA -> epilogue: F ready in TMEM
   uint64_t* fempty = zfull + 3;                             // epilogue -> MMA: F read
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zfull + 4);
+  uint64_t* yfull = zfull + 4;                              // resident Y has landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zfull + 5);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmY);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < NSLOT; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(yfull, 1);
     mbar_init(zfull, 1);
     mbar_init(zready, 4);
     mbar_init(ffull, 1);
@@ -137,7 +156,36 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && C::RES) {
+      // Y once, then one whole example per slot (both passes read it)
+      mbar_arrive_expect_tx(yfull, static_cast<uint32_t>(C::YREG));
+      for (int c = 0; c < C::NCH; ++c) tma_load_2d(&tmY, yfull, yreg + c * C::YB, 0, c * C::R);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* slot = ring + s * C::EXB;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(C::EXB));
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row0 = static_cast<int>(b * C::N + c * C::R);
+#pragma unroll
+          for (int bx = 0; bx < C::XBOXES; ++bx)
+            tma_load_2d(&tmX, &full[s], slot + (c * C::XBOXES + bx) * C::XBOXB, bx * C::XBOXW, row0);
+        }
+        if (++s == C::ES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      mbar_drain(yfull, 0u, status);
+      if (!ok) {
+        for (int i = 0; i < C::ES; ++i) mbar_wait(&full[i], ph ^ (i < s ? 0u : 1u), nullptr);
+      }
+    } else if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -168,7 +216,72 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && C::RES) {
+      const bool bf = Half16<T>::kBF16;
+      const uint32_t idA = idesc_f16kind_f32(C::R, C::KP, 1, 1, bf);  // Z = X^T Y: both MN-major
+      const uint32_t idB = idesc_f16kind_f32(C::R, C::KP, 0, 1, bf);  // F = X Z: X K-major, Z MN-major
+      const uint32_t xsw = C::XSW == 128 ? 2u : 4u;
+      const uint32_t ysw = C::YRB == 128 ? 2u : 4u;
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t eph = 0;
+      bool ok = mbar_wait(yfull, 0u, status);
+      bool issued = false;
+      tc_fence_after();
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x) {
+        if (!mbar_wait(&full[s], ph, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t slot = smem_u32(ring + s * C::EXB);
+        // pass A: Z = X^T Y over the example's chunks
+        for (int c = 0; c < C::NCH; ++c) {
+          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          const uint32_t xs = slot + c * C::XBOXES * C::XBOXB;
+          const uint32_t ys = smem_u32(yreg) + c * C::YB;
+          for (int ks = 0; ks < rows / 16; ++ks) {
+            const uint64_t bdesc = smem_desc(ys + ks * 16 * C::YRB, C::YB, 8 * C::YRB, ysw);
+#pragma unroll
+            for (int mz = 0; mz < C::MTZ; ++mz) {
+              const uint32_t a0 = xs + mz * (C::R / C::XBOXW) * C::XBOXB + ks * 16 * C::XSW;
+              const uint64_t adesc = smem_desc(a0, C::XBOXB, 8 * C::XSW, xsw);
+              umma_f16kind(tmem_base + mz * C::KP, adesc, bdesc, idA, (c | ks) != 0 ? 1u : 0u);
+            }
+          }
+        }
+        issued = true;
+        umma_commit(zfull);
+        // pass B: F = X Z from the same slot, once Z is in shared memory and the
+        // previous F has been read
+        if (!mbar_wait(zready, eph, status) || !mbar_wait(fempty, eph ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int c = 0; c < C::NCH; ++c) {
+          const uint32_t xs = slot + c * C::XBOXES * C::XBOXB;
+#pragma unroll
+          for (int ks = 0; ks < C::D / 16; ++ks) {
+            const int bx = ks / (C::XBOXW / 16), kin = ks % (C::XBOXW / 16);
+            const uint64_t adesc = smem_desc(xs + bx * C::XBOXB + kin * 32, 16, 8 * C::XSW, xsw);
+            const uint64_t bdesc = smem_desc(smem_u32(zb) + ks * 16 * C::YRB, C::ZB, 8 * C::YRB, ysw);
+            umma_f16kind(tmem_base + C::ZCOL + c * C::KP, adesc, bdesc, idB, ks != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty[s]);  // the slot is free once both passes have read it
+        umma_commit(ffull);
+        eph ^= 1u;
+        if (++s == C::ES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok && issued) {  // no MMA may still write TMEM when it is freed
+        umma_commit(zfull);
+        mbar_wait(zfull, eph, nullptr);
+      }
+    } else if (lane == 0) {
       const bool bf = Half16<T>::kBF16;
       const uint32_t idA = idesc_f16kind_f32(C::R, C::KP, 1, 1, bf);  // Z = X^T Y: both MN-major
       const uint32_t idB = idesc_f16kind_f32(C::R, C::KP, 0, 1, bf);  // F = X Z: X K-major, Z MN-major
