@@ -38,14 +38,14 @@ ORACLE_SAMPLE = {"c1_fp32": 64, "c2_bf16": 4096, "c3_bf16": 128, "c4_bf16": 16, 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM traffic of the CTA-pair MLP GEMM per launch, from one ncu capture of each of the
-# three Linears of the workload (dram__bytes_read.sum + dram__bytes_write.sum, averaged
-# over the three launches; profiles/mlp_gemm_pair_c4_shapes.md). It describes the kernel
+# DRAM traffic of the CTA-pair MLP GEMM per launch (streaming launch shape), from one ncu
+# capture of each of the three Linears of the workload (dram__bytes_read.sum +
+# dram__bytes_write.sum, averaged over the three launches; profiles/mlp_gemm_pair_c4_shapes.md). It describes the kernel
 # sources it was taken on: when their hash differs, the bench reports null.
 GEMM_TRAFFIC = {
     "sources": ["recsys_feature_interaction_b200/csrc/gemm_tc2.cuh", "recsys_feature_interaction_b200/csrc/common.cuh"],
-    "sha256": "2701460f8332c53c784aab747ba8478caa93d99d0778331507517a2bbd23aaf4",
-    "bytes_per_launch": 8557918629,
+    "sha256": "1e7902e5ecfd65ca1140976e864c705496a8ae5e69df45f56b752cf70b0f7a36",
+    "bytes_per_launch": 3183891712,
 }
 
 

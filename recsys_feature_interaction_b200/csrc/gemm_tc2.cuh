@@ -34,9 +34,27 @@ constexpr int GEMM2_L2_HINT = 0;  // default of GemmParams::l2hint
 constexpr uint32_t GEMM2_A_STAGE = 128 * GEMM2_BK * 2;  // 16 KB: this CTA's 128 rows
 constexpr uint32_t GEMM2_B_STAGE = 128 * GEMM2_BK * 2;  // 16 KB: this CTA's half of N
 
-template <typename TO>
+// Two launch shapes of the same kernel:
+//   persistent (STREAM = false): one pair per two SMs walks tiles pair, pair + pairs, ...
+//     with a 6-stage ring, two TMEM accumulators (the epilogue of tile t overlaps the
+//     main loop of tile t + 1) and double-buffered epilogue staging;
+//   streaming (STREAM = true): one pair per output tile, a 3-stage ring, one
+//     accumulator (256 TMEM columns) and single epilogue buffers, so that two pairs'
+//     CTAs share each SM (105 KB of shared memory each): the epilogue of one overlaps
+//     the main loop of the other, and the hardware block scheduler keeps the tiles in
+//     flight consecutive in raster order, which keeps their operand panels in L2.
+template <bool STREAM>
+struct Gemm2Shape {
+  static constexpr int STAGES = STREAM ? 3 : GEMM2_STAGES;
+  static constexpr int NACC = STREAM ? 1 : 2;
+  static constexpr int NBUF = STREAM ? 1 : 2;
+  static constexpr uint32_t TMEM_COLS = STREAM ? 256u : 512u;
+};
+
+template <typename TO, bool STREAM = false>
 constexpr uint32_t gemm2_smem_bytes() {
-  return 1024u + GEMM2_STAGES * (GEMM2_A_STAGE + GEMM2_B_STAGE) + 4u * 2u * gemm_epi_buf_bytes<TO>() + 256u;
+  using S = Gemm2Shape<STREAM>;
+  return 1024u + S::STAGES * (GEMM2_A_STAGE + GEMM2_B_STAGE) + 4u * S::NBUF * gemm_epi_buf_bytes<TO>() + 256u;
 }
 
 __device__ __forceinline__ void gemm2_tile_coords(const GemmParams& p, int tile, int& mt, int& nt) {
@@ -54,17 +72,20 @@ __device__ __forceinline__ void gemm2_tile_coords(const GemmParams& p, int tile,
 // (256, or E = floor(256/d) whole embedding rows of the last Linear when ROWLN: then
 // the epilogue adds the bias and the residual, applies the output LayerNorm and tmC
 // addresses the layer output [M, n*d]).
-template <typename T, typename TO, bool ROWLN = false>
+template <typename T, typename TO, bool ROWLN = false, bool STREAM = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+  using S = Gemm2Shape<STREAM>;
+  static_assert(!(STREAM && ROWLN), "the fused end-of-layer epilogue runs persistent");
+  constexpr int GEMM2_STAGES = S::STAGES;  // shadows the persistent default
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = sA + GEMM2_STAGES * GEMM2_A_STAGE;
   uint8_t* sEpi = sB + GEMM2_STAGES * GEMM2_B_STAGE;
   constexpr uint32_t EPI_BUF = gemm_epi_buf_bytes<TO>();
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 8 * EPI_BUF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 4 * S::NBUF * EPI_BUF);
   uint64_t* full = bars;                                // [STAGES]
   uint64_t* empty = bars + GEMM2_STAGES;                // [STAGES]
   uint64_t* tfull = bars + 2 * GEMM2_STAGES;            // [2]
@@ -92,7 +113,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, GEMM_TMEM_COLS);
+    tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
     tmem_relinquish_pair();
   }
   tc_fence_before();
@@ -181,7 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         if (!ok) break;
         umma_commit_pair(tfull_own + static_cast<uint32_t>(acc) * 8u);
         umma_commit_pair(tfull_peer + static_cast<uint32_t>(acc) * 8u);
-        if (++acc == 2) {
+        if (++acc == S::NACC) {
           acc = 0;
           acc_ph ^= 1u;
         }
@@ -194,7 +215,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    uint8_t* bufs = sEpi + (warp - 2) * 2 * EPI_BUF;
+    uint8_t* bufs = sEpi + (warp - 2) * S::NBUF * EPI_BUF;
     const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);  // leader's tempty[0]
     int acc = 0;
     uint32_t acc_ph = 0;
@@ -251,7 +272,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
         }
         uint8_t* sb = bufs + buf * EPI_BUF;
-        if (lane == 0) bulk_wait_read<1>();
+        if (lane == 0) {
+          if constexpr (S::NBUF == 2) bulk_wait_read<1>();
+          else bulk_wait_read<0>();
+        }
         __syncwarp();
         stage_row<TO>(sb, lane, v);
         fence_proxy_async_smem();
@@ -260,12 +284,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           tma_store_2d(&tmC, sb, col0, row0);
           bulk_commit();
         }
-        buf ^= 1;
+        if constexpr (S::NBUF == 2) buf ^= 1;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(acc) * 8u);
-      if (++acc == 2) {
+      if (++acc == S::NACC) {
         acc = 0;
         acc_ph ^= 1u;
       }
@@ -279,7 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync_all();  // no remote signal or MMA of the pair is still in flight
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
   }
 }
 

@@ -32,7 +32,7 @@ struct MoePtrs {
 // chunks of gate_chunk<E>() elements: the block stages that chunk of all E gate rows
 // in shared memory once, converted to fp32 (two planes of float4, so that consecutive
 // lanes read consecutive 16 bytes), and every warp streams its example's chunk of X
-// from HBM (16-byte loads, all of a lane's loads of the chunk issued before the
+// from HBM (16-byte loads, the next chunk's loads issued before this chunk's
 // arithmetic) and accumulates E fp32 dot products. W_g is read from L2 once per block
 // and chunk instead of once per example; X is read once. A shuffle reduction and an
 // fp32 softmax end each example.
@@ -60,7 +60,27 @@ __global__ void __launch_bounds__(256) moe_gate_kernel(const T* __restrict__ X, 
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    // X chunks are loaded one chunk ahead: chunk c + 1's loads are in flight while
+    // chunk c's W_g is staged and its products are taken
+    uint4 xn[VL];
+#pragma unroll
+    for (int i = 0; i < VL; ++i) {
+      const int v = lane + 32 * i;
+      xn[i] = (b < batch && v * 8 < nd) ? __ldg(reinterpret_cast<const uint4*>(X + b * nd + v * 8)) : zero;
+    }
     for (int64_t c0 = 0; c0 < nd; c0 += CH) {
+      uint4 xv[VL];
+#pragma unroll
+      for (int i = 0; i < VL; ++i) xv[i] = xn[i];
+      if (c0 + CH < nd) {
+#pragma unroll
+        for (int i = 0; i < VL; ++i) {
+          const int v = lane + 32 * i;
+          xn[i] = (b < batch && c0 + CH + v * 8 < nd)
+                      ? __ldg(reinterpret_cast<const uint4*>(X + b * nd + c0 + CH + v * 8))
+                      : zero;
+        }
+      }
       __syncthreads();  // the previous chunk of W_g has been read by every warp
       for (int i = threadIdx.x; i < E * VC; i += blockDim.x) {
         const int e = i / VC, v = i % VC;
@@ -75,13 +95,6 @@ __global__ void __launch_bounds__(256) moe_gate_kernel(const T* __restrict__ X, 
         ws[e][VC + v] = make_float4(w8[4], w8[5], w8[6], w8[7]);
       }
       __syncthreads();
-      uint4 xv[VL];
-#pragma unroll
-      for (int i = 0; i < VL; ++i) {
-        const int v = lane + 32 * i;
-        xv[i] = (b < batch && c0 + v * 8 < nd) ? __ldg(reinterpret_cast<const uint4*>(X + b * nd + c0 + v * 8))
-                                               : zero;
-      }
 #pragma unroll
       for (int i = 0; i < VL; ++i) {
         const int v = lane + 32 * i;

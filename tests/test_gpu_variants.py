@@ -6,6 +6,9 @@ whole-stack parity tests in a child process (the switches are read once per proc
   WK_PAIR_GEMM=0    the FMB MLP on one-CTA tcgen05 tiles instead of CTA pairs
   WK_RES_LN_RING=0  the residual + LayerNorm without the bulk-copy ring
   WK_LCB_RESIDENT=0 the LCB as a streaming GEMM instead of with W_L resident in shared memory
+  WK_GEMM_STREAM=0  the CTA-pair MLP GEMM persistent (one pair per two SMs) instead of one
+                    pair per output tile
+  WK_MOE_RING=0     the MoE mixture without the bulk-copy ring (runs the MoE tests)
 """
 import os
 import subprocess
@@ -23,14 +26,20 @@ VARIANTS = {
     "one_cta_gemm": {"WK_PAIR_GEMM": "0"},
     "res_ln_registers": {"WK_RES_LN_RING": "0"},
     "lcb_streaming": {"WK_LCB_RESIDENT": "0"},
+    "gemm_persistent": {"WK_GEMM_STREAM": "0"},
+    "moe_register_combine": {"WK_MOE_RING": "0"},
 }
 
 
 @pytest.mark.parametrize("name", sorted(VARIANTS))
 def test_variant_stack_parity(name, cuda_device):
     env = dict(os.environ, **VARIANTS[name])
-    cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_stack.py"), "-q", "-x", "-s",
-           "-m", "gpu", "-k", "c2_bf16 or c4_bf16 or c5_bf16 or batch_split or profiling"]
+    if name.startswith("moe"):
+        cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_moe.py"), "-q", "-x", "-s",
+               "-m", "gpu"]
+    else:
+        cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_stack.py"), "-q", "-x", "-s",
+               "-m", "gpu", "-k", "c2_bf16 or c4_bf16 or c5_bf16 or batch_split or profiling"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
     tail = "\n".join((r.stdout + r.stderr).splitlines()[-25:])
     print(tail)
