@@ -213,6 +213,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step from a CUDA graph of one forward (wk_*_graph_create); the "
+                         "per-kernel times then come from an eager profiled pass after the timed region")
     ap.add_argument("--head", action="store_true",
                     help="each step also runs the prediction head (wk_stack_predict: logits and probabilities)")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -315,7 +318,18 @@ def main():
     # per-step event pairs; larger inputs stream through L2 by themselves.
     x_bytes = X.numel() * X.element_size()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if x_bytes < (252 << 20) else None
-    api["prof"](True)
+    graph = None
+    step = api["fwd"]
+    if args.graph:
+        if args.head:
+            raise SystemExit("--graph captures wk_stack_forward / wk_moe_forward, not the head")
+        graph = (wk.wk_moe_graph_create if moe else wk.wk_stack_graph_create)(h, X, out)
+        wk.wk_graph_launch(graph, stream)  # warm the graph
+
+        def step(x, o):
+            wk.wk_graph_launch(graph, stream)
+    else:
+        api["prof"](True)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps if flush is not None else 1)]
     barrier()
@@ -324,13 +338,13 @@ def main():
         if flush is None:
             evs[0][0].record(stream)
             for _ in range(args.steps):
-                api["fwd"](X, out)
+                step(X, out)
             evs[0][1].record(stream)
         else:
             for a, b in evs:
                 flush.fill_(1)
                 a.record(stream)
-                api["fwd"](X, out)
+                step(X, out)
                 b.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
@@ -339,6 +353,15 @@ def main():
     status = api["status"]()
     if status != wk.WK_OK:
         raise RuntimeError("device status: " + wk.wk_status_string(status))
+    if graph is not None:  # per-kernel times of an eager profiled pass of the same steps
+        api["prof"](True)
+        for _ in range(args.steps):
+            if flush is not None:
+                flush.fill_(1)
+            api["fwd"](X, out)
+        torch.cuda.synchronize(dev)
+        api["prof"](False)
+        wk.wk_graph_destroy(graph)
     ktimes = api["times"]()
     ms_max = max_over_ranks(ms)
     value = world * B * args.steps / (ms_max / 1e3)
@@ -390,7 +413,8 @@ def main():
                         if args.head else ""), "per_gpu_batch": B,
                        "precision": precision,
                        "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
-                       "l2": l2},
+                       "l2": l2, "launch": ("one CUDA graph replay per step; per-kernel times from an eager "
+                                            "profiled pass" if args.graph else "eager, one C-ABI call per step")},
             "tflops_per_gpu": tflops,
             "pct_of_bf16_peak": 100.0 * tflops / peak,
             "peak_source": "%s bf16_tflops_sustained" % peak_src,

@@ -154,6 +154,21 @@ WK_API void wk_stack_destroy(wk_stack* h);
 /* Static string for a status code. */
 WK_API const char* wk_status_string(wk_status s);
 
+/* ---- CUDA graphs of a forward (for launch-bound batches) ----
+ *
+ * Captures one forward on FIXED device buffers X and out into a CUDA graph that
+ * wk_graph_launch replays with one launch: every kernel of the stack (or MoE stack)
+ * in order, with none of the host work of a forward call (argument checks, TMA
+ * descriptor encoding, launch overhead per kernel). The caller refills X between
+ * launches; the graph reads X and writes out at replay time. The handle must outlive
+ * the graph and must not be used by another forward while a replay runs (same
+ * workspace). Capture happens on a private stream; profiling records are not taken
+ * inside graphs. Errors: WK_ERR_INVALID_ARG (as for the forward), WK_ERR_CUDA. */
+typedef struct wk_graph wk_graph;
+WK_API wk_status wk_stack_graph_create(wk_stack* h, const void* X, void* out, int64_t batch, wk_graph** g);
+WK_API wk_status wk_graph_launch(wk_graph* g, wk_stream_t stream);
+WK_API void wk_graph_destroy(wk_graph* g);
+
 /* ---- per-kernel timing of a handle's forwards (CUDA events on the launch stream) ---- */
 
 typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
@@ -295,6 +310,10 @@ WK_API wk_status wk_moe_kernel_times(wk_moe* h, double* total_ms, int64_t* launc
 
 /* Frees the handle, its experts and workspace (synchronises the device). NULL is a no-op. */
 WK_API void wk_moe_destroy(wk_moe* h);
+
+/* A CUDA graph of one MoE forward on fixed X and out (as wk_stack_graph_create);
+ * replay with wk_graph_launch, free with wk_graph_destroy. */
+WK_API wk_status wk_moe_graph_create(wk_moe* h, const void* X, void* out, int64_t batch, wk_graph** g);
 
 /* Stand-alone gate: g[b, e] = softmax_e( sum_j W_g[e, j] X[b, j] + b_g[e] ), X [batch, nd]
  * and W_g [num_experts, nd] of dtype (16-bit, nd % 8 == 0), b_g [num_experts] fp32 or

@@ -372,3 +372,65 @@ def wk_stack_predict(h, X, logit, prob=None, batch=None, stream=None):
     L.wk_stack_predict.restype = ctypes.c_int
     _check(L.wk_stack_predict(h.ptr, _addr(X), _addr(logit), _addr(prob), int(b), _stream(stream, X)),
            "wk_stack_predict")
+
+
+# ------------------------------------------------------------------ graphs
+
+class GraphHandle:
+    """An opaque wk_graph* (one captured forward on fixed buffers) plus what it uses."""
+
+    def __init__(self, ptr, keep):
+        self.ptr = ptr
+        self._keep = keep
+
+    def __del__(self):
+        try:
+            if self.ptr:
+                wk_graph_destroy(self)
+        except Exception:
+            pass
+
+
+def _graph_sig(L):
+    vp = ctypes.c_void_p
+    for name in ("wk_stack_graph_create", "wk_moe_graph_create"):
+        f = getattr(L, name)
+        f.argtypes = [vp, vp, vp, ctypes.c_int64, ctypes.POINTER(vp)]
+        f.restype = ctypes.c_int
+    L.wk_graph_launch.argtypes = [vp, vp]
+    L.wk_graph_launch.restype = ctypes.c_int
+    L.wk_graph_destroy.argtypes = [vp]
+    L.wk_graph_destroy.restype = None
+
+
+def wk_stack_graph_create(h, X, out, batch=None):
+    L = lib()
+    _graph_sig(L)
+    g = ctypes.c_void_p()
+    b = X.shape[0] if batch is None else batch
+    _check(L.wk_stack_graph_create(h.ptr, _addr(X), _addr(out), int(b), ctypes.byref(g)), "wk_stack_graph_create")
+    return GraphHandle(g.value, [h, X, out])
+
+
+def wk_moe_graph_create(h, X, out, batch=None):
+    L = lib()
+    _graph_sig(L)
+    g = ctypes.c_void_p()
+    b = X.shape[0] if batch is None else batch
+    _check(L.wk_moe_graph_create(h.ptr, _addr(X), _addr(out), int(b), ctypes.byref(g)), "wk_moe_graph_create")
+    return GraphHandle(g.value, [h, X, out])
+
+
+def wk_graph_launch(g, stream=None):
+    L = lib()
+    _graph_sig(L)
+    like = g._keep[1] if len(g._keep) > 1 else None
+    _check(L.wk_graph_launch(g.ptr, _stream(stream, like)), "wk_graph_launch")
+
+
+def wk_graph_destroy(g):
+    if g.ptr:
+        L = lib()
+        _graph_sig(L)
+        L.wk_graph_destroy(g.ptr)
+        g.ptr = None

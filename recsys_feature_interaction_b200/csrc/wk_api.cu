@@ -761,6 +761,12 @@ struct wk_moe {
   CUtensorMap lcbX[2];              // Xm[0], Xm[1] as the LCB's operand
 };
 
+struct wk_graph {
+  int device = 0;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+
 namespace {
 
 struct ProfScope {
@@ -1324,6 +1330,44 @@ wk_status layer_noalloc16(const DevInfo* dv, const wk_stack_config* c, const std
   return s;
 }
 
+// Runs `body` (which enqueues a forward on the stream it is given) under stream
+// capture on a private stream and instantiates the graph.
+template <typename F>
+wk_status capture_graph(int device, F body, wk_graph** out) {
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  wk_graph* g = new (std::nothrow) wk_graph();
+  if (!g) {
+    cudaStreamDestroy(cs);
+    return WK_ERR_OOM;
+  }
+  g->device = device;
+  wk_status st = WK_OK;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    st = WK_ERR_CUDA;
+  } else {
+    st = body(reinterpret_cast<wk_stream_t>(cs));
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(cs, &graph);
+    if (st == WK_OK && (e != cudaSuccess || !graph)) st = WK_ERR_CUDA;
+    g->graph = graph;
+    if (st == WK_OK && cudaGraphInstantiate(&g->exec, graph, 0) != cudaSuccess) st = WK_ERR_CUDA;
+  }
+  cudaGetLastError();
+  cudaStreamDestroy(cs);
+  if (st != WK_OK) {
+    if (g->exec) cudaGraphExecDestroy(g->exec);
+    if (g->graph) cudaGraphDestroy(g->graph);
+    delete g;
+    return st;
+  }
+  *out = g;
+  return WK_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1819,6 +1863,48 @@ wk_status wk_layer_forward_noalloc(const wk_stack_config* cfg, const wk_layer_we
     s = run_res_ln<float, float, float>(dv, cat, Xf, w->out_ln_gamma, w->out_ln_beta, static_cast<float*>(out),
                                         batch * n, d, eps, dv->standalone_status, st);
   return s;
+}
+
+// ------------------------------------------------------------------ graphs
+
+wk_status wk_stack_graph_create(wk_stack* h, const void* X, void* out, int64_t batch, wk_graph** g) {
+  if (!h || !g || batch < 1) return WK_ERR_INVALID_ARG;
+  *g = nullptr;
+  const bool prof = h->prof;
+  h->prof = false;  // no event records inside a graph
+  const wk_status st = capture_graph(h->device, [&](wk_stream_t s) { return wk_stack_forward(h, X, out, batch, s); }, g);
+  h->prof = prof;
+  return st;
+}
+
+wk_status wk_moe_graph_create(wk_moe* h, const void* X, void* out, int64_t batch, wk_graph** g) {
+  if (!h || !g || batch < 1) return WK_ERR_INVALID_ARG;
+  *g = nullptr;
+  std::vector<bool> prof;
+  for (wk_stack* e : h->ex) {
+    prof.push_back(e->prof);
+    e->prof = false;
+  }
+  const wk_status st = capture_graph(h->device, [&](wk_stream_t s) { return wk_moe_forward(h, X, out, batch, s); }, g);
+  for (size_t i = 0; i < h->ex.size(); ++i) h->ex[i]->prof = prof[i];
+  return st;
+}
+
+wk_status wk_graph_launch(wk_graph* g, wk_stream_t stream) {
+  if (!g || !g->exec) return WK_ERR_INVALID_ARG;
+  if (cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  return WK_OK;
+}
+
+void wk_graph_destroy(wk_graph* g) {
+  if (!g) return;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  cudaGetLastError();
+  delete g;
 }
 
 // ------------------------------------------------------------ prediction head
