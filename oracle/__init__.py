@@ -234,3 +234,41 @@ def top_mlp_forward(weights, X):
     logit = z[:, 0]
     p = 1.0 / (1.0 + np.exp(-logit))
     return logit, p
+
+
+# ------------------------------------------------------- WHALE attention fusion
+#
+# WHALE pages (gist.science summaries of arXiv 2607.17017, Korean and French), section 2.1,
+# item 3 (attention-based fusion) and section 2.2 (shared K = V; shared-gate SwiGLU with
+# W_gate = W_up). The Wukong representation H_w (n rows of d) is the query, the sequence
+# representation H_s (L rows of d) is both key and value; the attention output is
+# concatenated with H_w, projected by a fusion MLP, and passed through a pre-norm SwiGLU
+# FFN whose gate and up projections are one matrix. The pages give no formulas. Readings
+# taken (the plainest ones the text supports): one head, no Q/K/V projections (K = V =
+# H_s), scaled dot-product scores S = H_w H_s^T / sqrt(d); the fusion MLP is one Linear
+# 2d -> d with bias; the FFN is H_f = Z + W_down (SiLU(U) * U), U = W_up LN(Z) (pre-norm:
+# LayerNorm over d, then the FFN, then the residual), no FFN biases.
+
+
+def attention_shared_kv(Hw, Hs):
+    """A [n, d] = softmax_rows(Hw Hs^T / sqrt(d)) Hs for one example, in float64."""
+    Hw, Hs = _c64(Hw), _c64(Hs)
+    d = Hw.shape[1]
+    S = (Hw @ Hs.T) / np.sqrt(d)
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P = P / P.sum(axis=1, keepdims=True)
+    return P @ Hs
+
+
+def whale_fusion(Hw, Hs, w, ln_eps=1e-5):
+    """H_f [n, d] for one example. w: W_F [d, 2d], b_F [d] (or None), ln_gamma / ln_beta [d],
+    W_up [h, d], W_down [d, h] (float32 or bf16 bits)."""
+    Hw = _c64(Hw)
+    A = attention_shared_kv(Hw, Hs)
+    C = np.concatenate([Hw, A], axis=1)
+    Z = linear(C, w["W_F"], w.get("b_F"))
+    Zn = np.stack([layernorm(z, w["ln_gamma"], w["ln_beta"], ln_eps) for z in Z])
+    U = linear(Zn, w["W_up"])
+    G = U * U / (1.0 + np.exp(-U))
+    return Z + linear(G, w["W_down"])

@@ -294,3 +294,71 @@ def head_flops_per_example(cfg, hidden=None):
     hidden = HEAD_HIDDEN if hidden is None else list(hidden)
     dims = [cfg["n"] * cfg["d"]] + hidden + [1]
     return 2 * sum(dims[j] * dims[j + 1] for j in range(len(dims) - 1))
+
+
+# ------------------------------------------------------- WHALE attention fusion
+#
+# WHALE pages (section 2.1 item 3, section 2.2): the Wukong representation H_w attends
+# over the sequence representation H_s (K = V = H_s), the result is concatenated with
+# H_w, projected by a fusion Linear and passed through a pre-norm shared-gate SwiGLU FFN.
+# Workloads of that form: H_w stands for a Wukong stack's output (n x d per example, the
+# shapes of the 2- and 8-layer workloads), H_s for an HSTU output of L positions (the
+# pages scale L up to 15k); both synthetic N(0, 1). W_F [d, 2d], W_up [h, d], W_down [d, h]
+# ~ N(0, 1/fan_in); b_F ~ N(0, 0.1^2); LayerNorm gamma = 1, beta = 0; h = 4d.
+WHALE_CONFIGS = {
+    "whale_c2": dict(batch=1024, n=64, d=128, L=2048, h=512, dtype="bf16",
+                     about="n=64 queries of d=128 over L=2048, h=512, B=1024"),
+    "whale_c4": dict(batch=256, n=512, d=160, L=4096, h=640, dtype="bf16",
+                     about="n=512 queries of d=160 over L=4096, h=640, B=256"),
+}
+
+TID_WHALE_HW = 800001
+TID_WHALE_HS = 800002
+
+
+def whale_specs(cfg):
+    d, h = cfg["d"], cfg["h"]
+    return {"W_F": ((d, 2 * d), "normal", 800010, 0.0, 1.0 / math.sqrt(2 * d), "bf16"),
+            "b_F": ((d,), "normal", 800011, 0.0, 0.1, "f32"),
+            "ln_gamma": ((d,), "const", 800012, 1.0, 0.0, "f32"),
+            "ln_beta": ((d,), "const", 800013, 0.0, 0.0, "f32"),
+            "W_up": ((h, d), "normal", 800014, 0.0, 1.0 / math.sqrt(d), "bf16"),
+            "W_down": ((d, h), "normal", 800015, 0.0, 1.0 / math.sqrt(h), "bf16")}
+
+
+def make_whale_host(cfg):
+    return _host_from_specs(whale_specs(cfg))
+
+
+def make_whale_dev(cfg, device="cuda"):
+    return _dev_from_specs(whale_specs(cfg), device)
+
+
+def make_whale_inputs_host(cfg, examples):
+    """(H_w [len, n, d], H_s [len, L, d]) as bf16 bit patterns for the listed examples."""
+    n, L, d = cfg["n"], cfg["L"], cfg["d"]
+    hw = np.empty((len(examples), n, d), dtype=np.uint16)
+    hs = np.empty((len(examples), L, d), dtype=np.uint16)
+    for r, b in enumerate(examples):
+        fill_normal_host(hw[r].reshape(-1), SEED, TID_WHALE_HW, 0.0, 1.0, offset=int(b) * n * d)
+        fill_normal_host(hs[r].reshape(-1), SEED, TID_WHALE_HS, 0.0, 1.0, offset=int(b) * L * d)
+    return hw, hs
+
+
+def make_whale_inputs_dev(cfg, batch, device="cuda", first_example=0):
+    import torch
+
+    from . import fill_normal_dev
+    n, L, d = cfg["n"], cfg["L"], cfg["d"]
+    hw = torch.empty((batch, n, d), dtype=torch.bfloat16, device=device)
+    hs = torch.empty((batch, L, d), dtype=torch.bfloat16, device=device)
+    fill_normal_dev(hw, SEED, TID_WHALE_HW, 0.0, 1.0, offset=first_example * n * d)
+    fill_normal_dev(hs, SEED, TID_WHALE_HS, 0.0, 1.0, offset=first_example * L * d)
+    return hw, hs
+
+
+def whale_flops_per_example(cfg):
+    """Matmul FLOPs of one example: 4 n L d (scores and weighted sum) + 2 n (2d) d (fusion)
+    + 4 n d h (up and down)."""
+    n, L, d, h = cfg["n"], cfg["L"], cfg["d"], cfg["h"]
+    return 4 * n * L * d + 4 * n * d * d + 4 * n * d * h
