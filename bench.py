@@ -34,7 +34,8 @@ WORKLOAD = "c4_bf16"
 METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack fwd, 1 B200"
 # examples per oracle sample (one layer), sized for a few seconds of host work each
 ORACLE_SAMPLE = {"c1_fp32": 64, "c2_bf16": 4096, "c3_bf16": 128, "c4_bf16": 16, "c5_bf16": 512, "moe3_c2": 1024,
-                 "moe4_c3": 32}
+                 "moe4_c3": 32, "whale_c2": 512, "whale_c4": 32}
+WHALE_METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), WHALE attention fusion fwd, 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -76,6 +77,10 @@ def load_peaks():
 
 
 def workload_desc(cfg):
+    if "L" in cfg:
+        return ("WHALE attention fusion fwd, %s: n=%d queries of d=%d over L=%d shared keys/values, fusion "
+                "Linear %d->%d, pre-norm shared-gate SwiGLU %d->%d->%d" %
+                (cfg["dtype"], cfg["n"], cfg["d"], cfg["L"], 2 * cfg["d"], cfg["d"], cfg["d"], cfg["h"], cfg["d"]))
     dims = [cfg["n"] * cfg["k"]] + list(cfg["hidden"]) + [cfg["n_f"] * cfg["d"]]
     kind = ("Wukong-MoE stack fwd (%d experts per layer, softmax gate)" % cfg["experts"] if "experts" in cfg
             else "Wukong stack fwd")
@@ -160,6 +165,17 @@ def oracle_sample(cfg, n_examples, threads=None):
     whole stack, seconds, threads)."""
     import oracle
     from synth import configs as C
+    if "L" in cfg:  # WHALE fusion: numpy fp64 per example (BLAS threads)
+        from threadpoolctl import threadpool_info
+        hw, hs = C.make_whale_inputs_host(cfg, list(range(n_examples)))
+        hw, hs = C.to_f64(hw), C.to_f64(hs)
+        w = C.make_whale_host(cfg)
+        t0 = time.perf_counter()
+        for b in range(n_examples):
+            oracle.whale_fusion(hw[b], hs[b], w)
+        dt = time.perf_counter() - t0
+        thr = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+        return n_examples / dt, dt, thr
     X = C.to_f64(C.make_x_host(cfg, list(range(n_examples))))
     thr = threads or oracle.default_threads()
     if "experts" in cfg:
@@ -177,6 +193,8 @@ def oracle_sample(cfg, n_examples, threads=None):
 
 def workload_cfg(name):
     from synth import configs as C
+    if name in C.WHALE_CONFIGS:
+        return C.WHALE_CONFIGS[name]
     return C.MOE_CONFIGS[name] if name in C.MOE_CONFIGS else C.CONFIGS[name]
 
 
@@ -194,16 +212,143 @@ def run_reference(args, rank, world):
         v, dt, thr = oracle_sample(cfg, ns)
         vals.append(v)
     value = statistics.median(vals)
-    sample = "%d examples through 1 of the %d layers per step, scaled to the whole stack" % (ns, cfg["layers"])
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
+    whale = "L" in cfg
+    sample = ("%d examples of the fusion per step" % ns if whale else
+              "%d examples through 1 of the %d layers per step, scaled to the whole stack" % (ns, cfg["layers"]))
+    line = {"impl": "reference", "metric": WHALE_METRIC if whale else METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload + ": " + workload_desc(cfg), "global_batch": cfg["batch"],
-                       "oracle": "plain C fp64, threads over examples / output rows"},
+                       "oracle": ("numpy fp64 (BLAS threads)" if whale else
+                                  "plain C fp64, threads over examples / output rows")},
             "cpu_baseline": {"value": value, "unit": "examples/s", "cores": thr, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "examples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_whale(args, cfg, rank, world, local, dev):
+    """One step = one WHALE fusion forward (attention with shared K = V, fusion Linear,
+    pre-norm shared-gate SwiGLU FFN) over the per-GPU batch; roofline on the attention
+    kernel (tensor-bound when 2 * L * d * n / (L * d * 2) = 2n FLOP per H_s byte is above
+    the ridge, else HBM-bound)."""
+    import torch
+
+    import recsys_feature_interaction_b200 as wk
+    from recsys_feature_interaction_b200 import replicas
+    from synth import configs as C
+
+    B, n, L, d = cfg["batch"], cfg["n"], cfg["L"], cfg["d"]
+    first, _ = replicas.example_range(rank, world, B)
+    Hw, Hs = C.make_whale_inputs_dev(cfg, B, device=dev, first_example=first)
+    Hf = torch.empty_like(Hw)
+    w = C.make_whale_dev(cfg, device=dev)
+    h = wk.wk_whale_create(cfg, w, max_batch=B)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        wk.wk_whale_forward(h, Hw, Hs, Hf, stream=stream)
+    torch.cuda.synchronize(dev)
+    if wk.wk_whale_sync_status(h) != wk.WK_OK:
+        raise RuntimeError("device status after warm-up")
+    wk.wk_whale_kernel_times(h)  # clear
+    in_bytes = (Hw.numel() + Hs.numel()) * Hw.element_size()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < (252 << 20) else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps if flush is not None else 1)]
+    wk.wk_whale_set_profiling(h, True)
+    replicas.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        if flush is None:
+            evs[0][0].record(stream)
+            for _ in range(args.steps):
+                wk.wk_whale_forward(h, Hw, Hs, Hf, stream=stream)
+            evs[0][1].record(stream)
+        else:
+            for a, b in evs:
+                flush.fill_(1)
+                a.record(stream)
+                wk.wk_whale_forward(h, Hw, Hs, Hf, stream=stream)
+                b.record(stream)
+        torch.cuda.synchronize(dev)
+    replicas.barrier()
+    wk.wk_whale_set_profiling(h, False)
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    if wk.wk_whale_sync_status(h) != wk.WK_OK:
+        raise RuntimeError("device status after the timed region")
+    ktimes = wk.wk_whale_kernel_times(h)
+    ms_max = replicas.max_over_ranks(ms, device=dev)
+    value = world * B * args.steps / (ms_max / 1e3)
+
+    # end to end: H_w and H_s copied in from pinned host memory, H_f copied out, every step
+    hwh, hsh = Hw.cpu().pin_memory(), Hs.cpu().pin_memory()
+    hfh = torch.empty_like(Hf, device="cpu").pin_memory()
+
+    def fwd_host():
+        Hw.copy_(hwh, non_blocking=True)
+        Hs.copy_(hsh, non_blocking=True)
+        wk.wk_whale_forward(h, Hw, Hs, Hf, stream=stream)
+        hfh.copy_(Hf, non_blocking=True)
+        stream.synchronize()
+    fwd_host()
+    replicas.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fwd_host()
+    e2e_s = replicas.max_over_ranks(time.perf_counter() - t0, device=dev)
+    e2e_value = world * B * args.steps / e2e_s
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops_ex = C.whale_flops_per_example(cfg)
+        tflops = value * flops_ex / 1e12 / world
+        a_ms, a_n = ktimes["whale_attn"]
+        a_s = (a_ms / a_n) / 1e3 if a_n else None
+        attn_flops = 4.0 * n * L * d * B                           # per launch: S = Q K^T and P V
+        attn_bytes = float(B) * (L * d + 2 * n * d) * 2            # H_s once, H_w in, A out
+        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if attn_flops / attn_bytes >= ridge:
+            ach = attn_flops / a_s / 1e12 if a_s else None
+            roof = {"kernel": "whale_attn_kernel (tcgen05)", "bound": "tensor", "achieved": ach,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "peak_note": "%s burst cuBLAS bf16 (a kernel of well under a second)" % peak_src}
+        else:
+            ach = attn_bytes / a_s / 1e9 if a_s else None
+            roof = {"kernel": "whale_attn_kernel (tcgen05)", "bound": "hbm", "achieved": ach,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_note": "%s copy bandwidth" % peak_src}
+        roof["frac"] = (ach / roof["peak"]) if ach else None
+        roof["traffic"] = None
+        roof["algorithmic_per_launch"] = {"flops": attn_flops, "bytes": attn_bytes}
+        l2 = ("L2 flushed (256 MB write) before every step, outside the timed events" if flush is not None else
+              "inputs larger than L2 (H_w + H_s %.0f MB per GPU)" % (in_bytes / 1e6))
+        line = {
+            "metric": WHALE_METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg["dtype"], "data": "synthetic",
+            "config": {"workload": args.workload + ": " + workload_desc(cfg), "per_gpu_batch": B,
+                       "precision": "16-bit inputs, weights, softmax weights and gated activations; fp32 "
+                                    "accumulation, softmax and LayerNorm statistics",
+                       "global_batch": B * world, "seq_len": L, "parallelism": "replicas (batch shards)",
+                       "l2": l2, "launch": "eager, one C-ABI call per step"},
+            "tflops_per_gpu": tflops,
+            "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+            "peak_source": "%s bf16_tflops (burst)" % peak_src,
+            "roofline": roof,
+            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items() if v[1]},
+            "clocks": clk.summary(),
+            "e2e": {"value": e2e_value, "unit": "examples/s",
+                    "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": Hf.numel() * Hf.element_size(),
+                    "api": "wk_whale_forward with pinned host-to-device copies of H_w and H_s before and a "
+                           "device-to-host copy of H_f after"},
+            "gpu_launches": sum(v[1] for v in ktimes.values()),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            ns = ORACLE_SAMPLE[args.workload]
+            v, dt, thr = oracle_sample(cfg, ns)
+            line["cpu_baseline"] = {"value": v, "unit": "examples/s", "cores": thr, "kind": "oracle",
+                                    "sample": "%d examples of the fusion (%.1f s)" % (ns, dt)}
+        print(json.dumps(line), flush=True)
+    wk.wk_whale_destroy(h)
 
 
 def main():
@@ -219,7 +364,8 @@ def main():
     ap.add_argument("--head", action="store_true",
                     help="each step also runs the prediction head (wk_stack_predict: logits and probabilities)")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16", "moe3_c2", "moe4_c3"])
+                    choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16", "moe3_c2", "moe4_c3",
+                             "whale_c2", "whale_c4"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -243,6 +389,10 @@ def main():
     wk_build.build()
 
     cfg = workload_cfg(args.workload)
+    if "L" in cfg:
+        run_whale(args, cfg, rank, world, local, dev)
+        replicas.finish()
+        return
     moe = "experts" in cfg
     B = cfg["batch"]
     # rank r works on examples [r*B, (r+1)*B) of the synthetic stream (no collective on the data path)

@@ -173,7 +173,8 @@ WK_API void wk_graph_destroy(wk_graph* g);
 
 typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
                WK_KERNEL_CONVERT = 4, WK_KERNEL_MOE_GATE = 5, WK_KERNEL_MOE_COMBINE = 6,
-               WK_KERNEL_HEAD = 7, WK_KERNEL_COUNT = 8 } wk_kernel_kind;
+               WK_KERNEL_HEAD = 7, WK_KERNEL_WHALE_ATTN = 8, WK_KERNEL_WHALE_FFN = 9,
+               WK_KERNEL_COUNT = 10 } wk_kernel_kind;
 
 /* enable != 0: every later forward records a start/stop event pair around each
  * kernel launch on its stream (adds no synchronisation). */
@@ -328,6 +329,84 @@ WK_API wk_status wk_moe_gate_softmax(const void* X, const void* W_g, const float
 WK_API wk_status wk_moe_combine(const void* const* concats, const void* X, const float* g, const float* const* gammas,
                                 const float* const* betas, void* out, int64_t batch, int32_t n, int32_t d,
                                 int32_t num_experts, wk_dtype dtype, float eps, wk_stream_t stream);
+
+/* ---- WHALE attention-based fusion ----
+ *
+ * The WHALE pages (gist.science summaries of arXiv 2607.17017, Korean and French),
+ * section 2.1 item 3: the Wukong interaction representation H_w is the query and the
+ * HSTU behaviour representation H_s both key and value of an attention; its output is
+ * concatenated with H_w, projected by a fusion MLP and passed through a pre-norm
+ * SwiGLU FFN, giving the fused representation H_f. Section 2.2: K = V (one tensor
+ * for both) and the gate and up projections of the SwiGLU share one matrix
+ * (W_gate = W_up). The pages give no formulas; the reading implemented (one head, no
+ * Q/K/V projections, a one-Linear fusion MLP, no FFN biases), per example:
+ *
+ *     A   = softmax_rows( H_w H_s^T / sqrt(d) ) H_s          H_w [n, d], H_s [L, d]
+ *     Z   = [H_w | A] W_F^T + b_F                            W_F [d, 2d]
+ *     U   = LN(Z) W_up^T                                     W_up [h, d], LN over d
+ *     H_f = Z + ( SiLU(U) * U ) W_down^T                     W_down [d, h]
+ *
+ * 16-bit storage (bf16 or fp16) for H_w, H_s, H_f, A and the weight matrices; fp32
+ * accumulation, softmax and LayerNorm statistics; the softmax weights and the gated
+ * activations are rounded to the 16-bit type as tensor-core operands. */
+
+typedef struct {
+  int32_t n;          /* query rows per example (rows of H_w and H_f), >= 1 */
+  int32_t d;          /* embedding width: 32, 64, 128 or 160 */
+  int32_t L;          /* key / value rows per example (rows of H_s), >= 1 */
+  int32_t h;          /* FFN width, a positive multiple of 64 */
+  wk_dtype dtype;     /* WK_BF16 or WK_F16 */
+  float ln_eps;       /* LayerNorm epsilon; 0 selects 1e-5 */
+  int64_t max_batch;  /* examples per forward, sizes the workspace */
+} wk_whale_config;
+
+typedef struct {      /* DEVICE pointers, BORROWED: the caller keeps them alive until destroy */
+  const void* W_F;    /* [d, 2d] dtype, row-major (PyTorch Linear layout) */
+  const float* b_F;   /* [d] fp32, or NULL for zero */
+  const float* ln_gamma, *ln_beta;  /* [d] fp32 */
+  const void* W_up;   /* [h, d] dtype */
+  const void* W_down; /* [d, h] dtype */
+} wk_whale_weights;
+
+typedef struct wk_whale wk_whale;
+
+/* Validates the shape (WK_ERR_UNSUPPORTED for a d, h or dtype the kernels do not
+ * handle; WK_ERR_INVALID_ARG for NULL or misaligned pointers, n, L or max_batch < 1),
+ * allocates the attention output A [max_batch, n, d] and a status word. Synchronises
+ * the device. */
+WK_API wk_status wk_whale_create(const wk_whale_config* cfg, const wk_whale_weights* w, wk_whale** out);
+
+/* Hf[b] = fusion(Hw[b], Hs[b]) for b < batch: Hw, Hf [batch, n, d], Hs [batch, L, d],
+ * all dtype, 16-byte aligned; Hf must not overlap Hw or Hs. Two kernels on `stream`:
+ * whale_attn_kernel (A) and whale_ffn_kernel (Z, LayerNorm, SwiGLU, residual).
+ * batch == 0 is a no-op; batch > max_batch is WK_ERR_INVALID_ARG. Asynchronous; not
+ * re-entrant (the handle's A buffer is shared). */
+WK_API wk_status wk_whale_forward(wk_whale* h, const void* Hw, const void* Hs, void* Hf, int64_t batch,
+                                  wk_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the handle's device status word. */
+WK_API wk_status wk_whale_sync_status(wk_whale* h, wk_stream_t stream);
+
+/* Per-kernel event timing of the handle's forwards (kinds WK_KERNEL_WHALE_ATTN and
+ * WK_KERNEL_WHALE_FFN), as wk_stack_set_profiling / wk_stack_kernel_times. */
+WK_API wk_status wk_whale_set_profiling(wk_whale* h, int enable);
+WK_API wk_status wk_whale_kernel_times(wk_whale* h, double* total_ms, int64_t* launches);
+
+/* Frees the handle and its workspace (synchronises the device). NULL is a no-op. */
+WK_API void wk_whale_destroy(wk_whale* h);
+
+/* Stand-alone attention with shared keys and values:
+ *   A[b] = softmax_rows( Hw[b] Hs[b]^T / sqrt(d) ) Hs[b]
+ * Hw, A [batch, n, d], Hs [batch, L, d] (dtype, 16-bit); d in {32, 64, 128, 160}. */
+WK_API wk_status wk_whale_attention(const void* Hw, const void* Hs, void* A, int64_t batch, int32_t n, int32_t L,
+                                    int32_t d, wk_dtype dtype, wk_stream_t stream);
+
+/* Stand-alone fusion Linear + pre-norm shared-gate SwiGLU FFN over `rows` rows:
+ *   Z = [Hw | A] W_F^T + b_F,  Hf = Z + ( SiLU(U) * U ) W_down^T,  U = LN(Z) W_up^T
+ * Hw, A, Hf [rows, d] (dtype); weights as wk_whale_weights; eps 0 selects 1e-5. */
+WK_API wk_status wk_whale_fusion_ffn(const void* Hw, const void* A, const wk_whale_weights* w, void* Hf,
+                                     int64_t rows, int32_t d, int32_t h, wk_dtype dtype, float eps,
+                                     wk_stream_t stream);
 
 /* ---- one layer without allocating: for callers that cannot call cudaMalloc ----
  *

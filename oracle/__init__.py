@@ -265,7 +265,13 @@ def whale_fusion(Hw, Hs, w, ln_eps=1e-5):
     """H_f [n, d] for one example. w: W_F [d, 2d], b_F [d] (or None), ln_gamma / ln_beta [d],
     W_up [h, d], W_down [d, h] (float32 or bf16 bits)."""
     Hw = _c64(Hw)
-    A = attention_shared_kv(Hw, Hs)
+    return fusion_ffn(Hw, attention_shared_kv(Hw, Hs), w, ln_eps)
+
+
+def fusion_ffn(Hw, A, w, ln_eps=1e-5):
+    """The part of the fusion after the attention, on rows of H_w [r, d] and A [r, d]:
+    Z = [H_w | A] W_F^T + b_F, then Z + W_down(SiLU(U) * U) with U = W_up LN(Z)."""
+    Hw, A = _c64(Hw), _c64(A)
     C = np.concatenate([Hw, A], axis=1)
     Z = linear(C, w["W_F"], w.get("b_F"))
     Zn = np.stack([layernorm(z, w["ln_gamma"], w["ln_beta"], ln_eps) for z in Z])

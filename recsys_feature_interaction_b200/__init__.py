@@ -21,8 +21,9 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
 WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
 WK_F32, WK_BF16, WK_F16 = 0, 1, 2
 (WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_CONVERT, WK_KERNEL_MOE_GATE,
- WK_KERNEL_MOE_COMBINE, WK_KERNEL_HEAD, WK_KERNEL_COUNT) = range(9)
-KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert", "moe_gate", "moe_combine", "head")
+ WK_KERNEL_MOE_COMBINE, WK_KERNEL_HEAD, WK_KERNEL_WHALE_ATTN, WK_KERNEL_WHALE_FFN, WK_KERNEL_COUNT) = range(11)
+KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert", "moe_gate", "moe_combine", "head", "whale_attn",
+                "whale_ffn")
 WK_MOE_MAX_EXPERTS = 8
 
 
@@ -49,6 +50,16 @@ class WkLayerWeights(ctypes.Structure):
 
 class WkMoeGate(ctypes.Structure):
     _fields_ = [("W_g", ctypes.c_void_p), ("b_g", ctypes.c_void_p)]
+
+
+class WkWhaleConfig(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int32), ("d", ctypes.c_int32), ("L", ctypes.c_int32), ("h", ctypes.c_int32),
+                ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("max_batch", ctypes.c_int64)]
+
+
+class WkWhaleWeights(ctypes.Structure):
+    _fields_ = [("W_F", ctypes.c_void_p), ("b_F", ctypes.c_void_p), ("ln_gamma", ctypes.c_void_p),
+                ("ln_beta", ctypes.c_void_p), ("W_up", ctypes.c_void_p), ("W_down", ctypes.c_void_p)]
 
 
 _lib = None
@@ -86,6 +97,13 @@ def lib():
             "wk_moe_gate_softmax": [vp, vp, vp, vp, i64, i64, i32, ci, vp],
             "wk_moe_combine": [ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, i64, i32, i32,
                                i32, ci, cf, vp],
+            "wk_whale_create": [ctypes.POINTER(WkWhaleConfig), ctypes.POINTER(WkWhaleWeights), ctypes.POINTER(vp)],
+            "wk_whale_forward": [vp, vp, vp, vp, i64, vp],
+            "wk_whale_sync_status": [vp, vp],
+            "wk_whale_set_profiling": [vp, ci],
+            "wk_whale_kernel_times": [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)],
+            "wk_whale_attention": [vp, vp, vp, i64, i32, i32, i32, ci, vp],
+            "wk_whale_fusion_ffn": [vp, vp, ctypes.POINTER(WkWhaleWeights), vp, i64, i32, i32, ci, cf, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -95,6 +113,8 @@ def lib():
         L.wk_stack_destroy.restype = None
         L.wk_moe_destroy.argtypes = [vp]
         L.wk_moe_destroy.restype = None
+        L.wk_whale_destroy.argtypes = [vp]
+        L.wk_whale_destroy.restype = None
         L.wk_status_string.argtypes = [ci]
         L.wk_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -434,3 +454,77 @@ def wk_graph_destroy(g):
         _graph_sig(L)
         L.wk_graph_destroy(g.ptr)
         g.ptr = None
+
+
+# ------------------------------------------------------- WHALE attention fusion
+
+class WhaleHandle:
+    """An opaque wk_whale* plus the Python objects whose memory it borrows."""
+
+    def __init__(self, ptr, cfg, keep):
+        self.ptr = ptr
+        self.cfg = cfg
+        self._keep = keep
+
+    def __del__(self):
+        try:
+            if self.ptr:
+                wk_whale_destroy(self)
+        except Exception:
+            pass
+
+
+def _whale_weights(w):
+    return WkWhaleWeights(_addr(w["W_F"]), _addr(w.get("b_F")), _addr(w["ln_gamma"]), _addr(w["ln_beta"]),
+                          _addr(w["W_up"]), _addr(w["W_down"]))
+
+
+def wk_whale_create(cfg, weights, max_batch=None, dtype=None, ln_eps=0.0):
+    """cfg: mapping with n, d, L, h and dtype (and batch, the default max_batch);
+    weights: mapping with W_F [d, 2d], b_F [d] (or None), ln_gamma, ln_beta [d],
+    W_up [h, d], W_down [d, h]."""
+    c = WkWhaleConfig(cfg["n"], cfg["d"], cfg["L"], cfg["h"], _dtype_code(dtype if dtype is not None else cfg["dtype"]),
+                      float(ln_eps), int(max_batch if max_batch is not None else cfg.get("batch", 1)))
+    ww = _whale_weights(weights)
+    h = ctypes.c_void_p()
+    _check(lib().wk_whale_create(ctypes.byref(c), ctypes.byref(ww), ctypes.byref(h)), "wk_whale_create")
+    return WhaleHandle(h.value, dict(cfg), [dict(weights), ww])
+
+
+def wk_whale_forward(h, Hw, Hs, Hf, batch=None, stream=None):
+    b = Hw.shape[0] if batch is None else batch
+    _check(lib().wk_whale_forward(h.ptr, _addr(Hw), _addr(Hs), _addr(Hf), int(b), _stream(stream, Hw)),
+           "wk_whale_forward")
+
+
+def wk_whale_sync_status(h, stream=None):
+    return lib().wk_whale_sync_status(h.ptr, _stream(stream))
+
+
+def wk_whale_destroy(h):
+    if h.ptr:
+        lib().wk_whale_destroy(h.ptr)
+        h.ptr = None
+
+
+def wk_whale_set_profiling(h, enable=True):
+    _check(lib().wk_whale_set_profiling(h.ptr, 1 if enable else 0), "wk_whale_set_profiling")
+
+
+def wk_whale_kernel_times(h):
+    """{kernel name: (total_ms, launches)} of the handle's forwards since the last call."""
+    ms = (ctypes.c_double * WK_KERNEL_COUNT)()
+    n = (ctypes.c_int64 * WK_KERNEL_COUNT)()
+    _check(lib().wk_whale_kernel_times(h.ptr, ms, n), "wk_whale_kernel_times")
+    return {KERNEL_NAMES[i]: (ms[i], n[i]) for i in range(WK_KERNEL_COUNT)}
+
+
+def wk_whale_attention(Hw, Hs, A, batch, n, L, d, dtype, stream=None):
+    _check(lib().wk_whale_attention(_addr(Hw), _addr(Hs), _addr(A), int(batch), int(n), int(L), int(d),
+                                    _dtype_code(dtype), _stream(stream, Hw)), "wk_whale_attention")
+
+
+def wk_whale_fusion_ffn(Hw, A, weights, Hf, rows, d, h, dtype, eps=0.0, stream=None):
+    ww = _whale_weights(weights)
+    _check(lib().wk_whale_fusion_ffn(_addr(Hw), _addr(A), ctypes.byref(ww), _addr(Hf), int(rows), int(d), int(h),
+                                     _dtype_code(dtype), float(eps), _stream(stream, Hw)), "wk_whale_fusion_ffn")

@@ -1,0 +1,774 @@
+// whale.cuh -- the attention-based fusion module of WHALE on the 5th-generation
+// tensor cores (WHALE pages, gist.science summaries of arXiv 2607.17017: section 2.1
+// item 3, attention-based fusion; section 2.2, shared key-value and shared-gate SwiGLU).
+//
+// Per example, with H_w (n x d) the Wukong representation and H_s (L x d) the sequence
+// representation (one head, no projections; K = V = H_s):
+//
+//   A   = softmax_rows( H_w H_s^T / sqrt(d) ) H_s                 whale_attn_kernel
+//   Z   = [H_w | A] W_F^T + b_F                 (fusion Linear)    whale_ffn_kernel
+//   U   = LN(Z) W_up^T                          (pre-norm)
+//   H_f = Z + ( SiLU(U) * U ) W_down^T          (W_gate = W_up, residual)
+//
+// whale_attn_kernel: one CTA per SM walks (example, 128-query tile) units. Warp 0 streams
+// the query tile and 128-key tiles of H_s with TMA; each key tile is loaded into shared
+// memory ONCE and read twice by the tensor core: as the K-major operand of S = Q K^T and
+// as the MN-major operand of O += P V (the page's shared K = V, which halves the key/value
+// traffic). Warp 1 issues the MMAs (S double-buffered in TMEM, S of the next block issued
+// before P V of this one). Warps 2..5 (one query row per thread) run the online softmax
+// from TMEM: P = 2^(S log2(e)/sqrt(d) - m) rounded to the operand type into shared memory,
+// row sums in fp32. The running max m is raised only when a block's max exceeds it by
+// more than 8 (P <= 2^8, exact in fp32 and in the 16-bit operand's exponent range), and
+// only then is the O row rescaled in TMEM; the result is the same softmax, with fewer
+// rescales. The last block of a ragged L is masked; query rows past n are zero rows of
+// the TMA box and are never stored.
+//
+// whale_ffn_kernel: one CTA per SM walks 128-row tiles of the batch's B*n rows. Z is
+// accumulated in TMEM from the [H_w | A] tile and W_F; the epilogue warps add b_F, take
+// the LayerNorm over d (fp32, two passes over TMEM) and write LN(Z) to shared memory;
+// the FFN then runs in chunks of 64 columns of h: U_c = LN(Z) W_up_c^T into TMEM, the
+// epilogue writes G_c = U_c^2 / (1 + exp(-U_c)) to shared memory, and the down
+// projection accumulates G_c W_down_c^T onto Z's own TMEM columns, so the residual costs
+// nothing. H_f = that sum + b_F. Weights stream through a TMA ring from L2.
+//
+// Every mbarrier wait is bounded (common.cuh); on a failed wait the threads stop waiting,
+// let issued copies land, let issued MMAs finish and free TMEM before the CTA exits.
+#pragma once
+
+#include "common.cuh"
+
+namespace wk {
+
+__device__ __forceinline__ void whale_tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void whale_tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x (the hardware's approximate base-2 exponential; 2^-inf = +0).
+__device__ __forceinline__ float whale_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Byte offset of 16-byte unit j of row r inside a K-major tile written with the TMA's
+// 128-byte (row pitch 128) or 64-byte (row pitch 64) swizzle.
+template <int SWB>
+__device__ __forceinline__ uint32_t whale_swz(int r, int j) {
+  return static_cast<uint32_t>(r * SWB + ((SWB == 128 ? (j ^ (r & 7)) : (j ^ ((r >> 1) & 3))) << 4));
+}
+
+// b_F[i], or zero when the fusion Linear has no bias.
+__device__ __forceinline__ float whale_bias(const float* __restrict__ b, int i) { return b ? __ldg(&b[i]) : 0.f; }
+
+template <typename T>
+__device__ __forceinline__ void whale_st_row32(T* dst, const uint32_t (&r)[32], float scale, const float* add) {
+  uint32_t p[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float a = __uint_as_float(r[2 * i]) * scale, b = __uint_as_float(r[2 * i + 1]) * scale;
+    if (add) {
+      a += add[2 * i];
+      b += add[2 * i + 1];
+    }
+    p[i] = Half16<T>::pack2(a, b);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+}
+
+// ----------------------------------------------------------------- attention
+
+template <int D_>
+struct WaCfg {
+  static constexpr int D = D_;
+  static constexpr int R = 128;                          // query rows per tile (MMA M)
+  static constexpr int LB = 128;                         // keys per block (N of S, K of P V)
+  static constexpr int BW = (D % 64 == 0) ? 64 : 32;     // columns per TMA box
+  static constexpr int SWB = BW * 2;                     // bytes per box row = swizzle span
+  static constexpr uint32_t SWMODE = BW == 64 ? 2u : 4u; // descriptor swizzle: 128B / 64B
+  static constexpr int NBOX = D / BW;
+  static constexpr int QBOXB = R * SWB;
+  static constexpr int KVBOXB = LB * SWB;
+  static constexpr int QB = NBOX * QBOXB;
+  static constexpr int KVB = NBOX * KVBOXB;
+  static constexpr int PBOXB = R * 128;                  // P: 64 keys per 128B-swizzled box
+  static constexpr int PB = (LB / 64) * PBOXB;
+  static constexpr int LIMIT = 227 * 1024;
+  static constexpr int FIXED = 1024 + QB + 2 * PB + 256;
+  static constexpr int STAGES_RAW = (LIMIT - FIXED) / KVB;
+  static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
+  // at least half an SM's shared memory: one CTA per SM, so that its 512 TMEM columns are free
+  static constexpr int SMEM = FIXED + STAGES * KVB > 120 * 1024 ? FIXED + STAGES * KVB : 120 * 1024;
+  static constexpr int OCOL = 2 * LB;                    // TMEM: S0 [0,128), S1 [128,256), O [256, 256+D)
+  static_assert(D % 32 == 0 && D >= 32 && D <= 256, "D");
+  static_assert(OCOL + D <= 512, "TMEM columns");
+  static_assert(STAGES >= 2, "shared memory");
+  static_assert(QB % 1024 == 0 && KVB % 1024 == 0 && PB % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+constexpr int WA_THREADS = 192;
+
+template <class C, typename T>
+__global__ void __launch_bounds__(WA_THREADS, 1)
+    whale_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+                      T* __restrict__ Aout, int64_t batch, int n, int L, float scale_log2, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + C::QB;
+  uint8_t* sP = sKV + C::STAGES * C::KVB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::PB);
+  uint64_t* kv_full = bars;                  // [STAGES] key tile landed
+  uint64_t* kv_empty = bars + C::STAGES;     // [STAGES] both products read it
+  uint64_t* s_full = bars + 2 * C::STAGES;   // [2] S in TMEM
+  uint64_t* s_empty = s_full + 2;            // [2] S read by the softmax warps
+  uint64_t* p_full = s_full + 4;             // [2] P in shared memory
+  uint64_t* q_full = s_full + 6;
+  uint64_t* q_empty = s_full + 7;
+  uint64_t* pv_done = s_full + 8;            // one phase per P V block, in order
+  uint64_t* o_empty = s_full + 9;            // O read by the softmax warps (per unit)
+  uint64_t* fin = s_full + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 11);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmKV);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(pv_done, 1);
+    mbar_init(o_empty, 4);
+    mbar_init(fin, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int qtiles = (n + C::R - 1) / C::R;
+  const int64_t units = batch * qtiles;
+  const int nb = (L + C::LB - 1) / C::LB;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, uc = 0, qn = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++uc) {
+        const int b = static_cast<int>(u / qtiles), q0 = static_cast<int>(u % qtiles) * C::R;
+        if (!mbar_wait(q_empty, (uc & 1u) ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(C::QB));
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx) tma_load_3d(&tmQ, q_full, sQ + bx * C::QBOXB, bx * C::BW, q0, b);
+        ++qn;
+        for (int j = 0; j < nb; ++j) {
+          if (!mbar_wait(&kv_empty[s], ph ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(C::KVB));
+#pragma unroll
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_3d(&tmKV, &kv_full[s], sKV + s * C::KVB + bx * C::KVBOXB, bx * C::BW, j * C::LB, b);
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {  // copies already issued must land before the CTA exits
+        for (int i = 0; i < C::STAGES; ++i) mbar_drain(&kv_full[i], ph ^ (i < s ? 0u : 1u), status);
+        if (qn > 0) mbar_drain(q_full, (qn - 1) & 1u, status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const bool bf = Half16<T>::kBF16;
+      const uint32_t idS = idesc_f16kind_f32(C::R, C::LB, 0, 0, bf);  // S = Q K^T: both K-major
+      const uint32_t idO = idesc_f16kind_f32(C::R, C::D, 0, 1, bf);   // O += P V: V MN-major
+      int ns = 0, cs = 0;  // ring slots of the next S block and of the next P V block
+      uint32_t nph = 0, g = 0, uc = 0;
+      bool ok = true;
+      auto issue_s = [&](uint32_t gb) -> bool {
+        if (!mbar_wait(&kv_full[ns], nph, status)) return false;
+        if (!mbar_wait(&s_empty[gb & 1u], ((gb >> 1) & 1u) ^ 1u, status)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sKV + ns * C::KVB);
+#pragma unroll
+        for (int ks = 0; ks < C::D / 16; ++ks) {
+          const int bx = ks / (C::BW / 16), kin = ks % (C::BW / 16);
+          const uint64_t ad = smem_desc(qa + bx * C::QBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+          const uint64_t bd = smem_desc(ka + bx * C::KVBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+          umma_f16kind(tmem + (gb & 1u) * C::LB, ad, bd, idS, ks != 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[gb & 1u]);
+        if (++ns == C::STAGES) {
+          ns = 0;
+          nph ^= 1u;
+        }
+        return true;
+      };
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++uc) {
+        if (!mbar_wait(q_full, uc & 1u, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (!issue_s(g)) {
+          ok = false;
+          break;
+        }
+        for (int j = 0; j < nb; ++j) {
+          const uint32_t gj = g + static_cast<uint32_t>(j);
+          if (j + 1 < nb) {
+            if (!issue_s(gj + 1)) {
+              ok = false;
+              break;
+            }
+          } else {
+            umma_commit(q_empty);  // the unit's last S has read Q
+          }
+          if (j == 0 && uc > 0 && !mbar_wait(o_empty, (uc - 1) & 1u, status)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&p_full[gj & 1u], (gj >> 1) & 1u, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sP + (gj & 1u) * C::PB), va = smem_u32(sKV + cs * C::KVB);
+#pragma unroll
+          for (int ks = 0; ks < C::LB / 16; ++ks) {
+            const uint64_t ad = smem_desc(pa + (ks / 4) * C::PBOXB + (ks % 4) * 32, 16, 1024, 2u);
+            // MN-major V: BW-column atoms C::KVBOXB apart, 8-key groups 8 * SWB apart
+            const uint64_t bd = smem_desc(va + ks * 16 * C::SWB, C::KVBOXB, 8 * C::SWB, C::SWMODE);
+            umma_f16kind(tmem + C::OCOL, ad, bd, idO, (j | ks) != 0 ? 1u : 0u);
+          }
+          umma_commit(pv_done);
+          umma_commit(&kv_empty[cs]);
+          if (++cs == C::STAGES) cs = 0;
+        }
+        g += static_cast<uint32_t>(nb);
+      }
+      umma_commit(fin);  // no MMA may still write TMEM when it is freed
+      mbar_drain(fin, 0u, status);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t g = 0;
+    // After a failed wait a thread stops waiting but walks the same schedule, so the
+    // warp-collective TMEM accesses stay converged.
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+      const int b = static_cast<int>(u / qtiles), q0 = static_cast<int>(u % qtiles) * C::R;
+      const bool warp_on = q0 + q * 32 < n;
+      const bool row_on = q0 + row < n;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nb; ++j) {
+        const uint32_t gj = g + static_cast<uint32_t>(j), buf = gj & 1u;
+        if (ok) ok = mbar_wait(&s_full[buf], (gj >> 1) & 1u, status);
+        tc_fence_after();
+        uint32_t sr[C::LB];
+        if (warp_on) {
+#pragma unroll
+          for (int c = 0; c < C::LB / 32; ++c)
+            tmem_ld32(tmem + lane_base + buf * C::LB + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[buf]);
+        const int kvalid = min(C::LB, L - j * C::LB);
+        float mb = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < C::LB; ++c)
+          if (c < kvalid) mb = fmaxf(mb, __uint_as_float(sr[c]));
+        const float mb2 = mb * scale_log2;
+        const bool need = warp_on && row_on && (mb2 > m + 8.f);
+        // P V of the previous block has finished: its P buffer (two blocks back) is free
+        // and O holds every earlier block.
+        if (gj > 0 && ok) ok = mbar_wait(pv_done, (gj - 1) & 1u, status);
+        tc_fence_after();
+        const float mnew = need ? mb2 : m;
+        const float factor = need ? whale_ex2(m - mnew) : 1.f;
+        if (warp_on && j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int cc = 0; cc < C::D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + C::OCOL + cc * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            whale_tmem_st32(tmem + lane_base + C::OCOL + cc * 32, o);
+          }
+          whale_tmem_st_wait();
+        }
+        l *= factor;
+        m = mnew;
+        if (warp_on) {
+          const float mm = row_on ? m : 0.f;
+          const uint32_t pb = smem_u32(sP + buf * C::PB);
+          float ls = 0.f;
+#pragma unroll
+          for (int c8 = 0; c8 < C::LB / 8; ++c8) {
+            float p[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int c = c8 * 8 + i;
+              p[i] = c < kvalid ? whale_ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -mm)) : 0.f;
+              ls += p[i];
+            }
+            const uint32_t a = pb + (c8 / 8) * C::PBOXB + whale_swz<128>(row, c8 % 8);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(Half16<T>::pack2(p[0], p[1])),
+                         "r"(Half16<T>::pack2(p[2], p[3])), "r"(Half16<T>::pack2(p[4], p[5])),
+                         "r"(Half16<T>::pack2(p[6], p[7]))
+                         : "memory");
+          }
+          l += ls;
+        }
+        fence_proxy_async_smem();  // the tensor core reads P
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[buf]);
+      }
+      // the unit's output rows: O / l
+      const uint32_t gl = g + static_cast<uint32_t>(nb) - 1u;
+      if (ok) ok = mbar_wait(pv_done, gl & 1u, status);
+      tc_fence_after();
+      if (warp_on) {
+        const float inv = row_on ? 1.f / l : 0.f;
+        T* dst = Aout + (static_cast<int64_t>(b) * n + q0 + row) * C::D;
+#pragma unroll 1
+        for (int cc = 0; cc < C::D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + C::OCOL + cc * 32, o);
+          tmem_ld_wait();
+          if (row_on && ok) whale_st_row32<T>(dst + cc * 32, o, inv, nullptr);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
+      g += static_cast<uint32_t>(nb);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------- fusion + FFN
+
+template <int D_>
+struct WfCfg {
+  static constexpr int D = D_;
+  static constexpr int R = 128;                          // rows per tile (MMA M)
+  static constexpr int HC = 64;                          // FFN columns per chunk
+  static constexpr int BW = (D % 64 == 0) ? 64 : 32;
+  static constexpr int SWB = BW * 2;
+  static constexpr uint32_t SWMODE = BW == 64 ? 2u : 4u;
+  static constexpr int NBOX = D / BW;
+  static constexpr int TBOXB = R * SWB;                  // one box of a 128-row tile
+  static constexpr int CB = 2 * NBOX * TBOXB;            // [H_w | A], 128 x 2D
+  static constexpr int ZNB = NBOX * TBOXB;               // LN(Z), 128 x D
+  static constexpr int GBOX = HC / BW;
+  static constexpr int GB = GBOX * TBOXB;                // one gated chunk, 128 x HC
+  static constexpr int WDBOXB = D * SWB;                 // W_F / W_down box: D rows x BW
+  static constexpr int WUBOXB = HC * SWB;                // W_up box: HC rows x BW
+  static constexpr int WS = 128 * D;                     // one weight chunk (D x 64 or 64 x D, 16-bit)
+  static constexpr int NKC = 2 * D / 64;                 // W_F chunks of 64 input columns
+  static constexpr int LIMIT = 227 * 1024;
+  static constexpr int FIXED = 1024 + CB + ZNB + 2 * GB + 512;
+  static constexpr int STAGES_RAW = (LIMIT - FIXED) / WS;
+  static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
+  static constexpr int SMEM = FIXED + STAGES * WS > 120 * 1024 ? FIXED + STAGES * WS : 120 * 1024;
+  static constexpr int UCOL = 2 * D;                     // TMEM: Z/out x2 [0, 2D), U x2 [2D, 2D + 128)
+  static_assert(D % 32 == 0 && D >= 32 && D <= 192, "D");
+  static_assert(UCOL + 2 * HC <= 512, "TMEM columns");
+  static_assert(STAGES >= 2, "shared memory");
+  static_assert(CB % 1024 == 0 && ZNB % 1024 == 0 && GB % 1024 == 0 && WS % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(WDBOXB % 512 == 0 && WUBOXB % 512 == 0, "swizzle atoms stay aligned");
+};
+
+constexpr int WF_THREADS = 192;
+
+template <class C, typename T>
+__global__ void __launch_bounds__(WF_THREADS, 1)
+    whale_ffn_kernel(const __grid_constant__ CUtensorMap tmHw, const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmWF, const __grid_constant__ CUtensorMap tmWU,
+                     const __grid_constant__ CUtensorMap tmWD, const float* __restrict__ bF,
+                     const float* __restrict__ gamma, const float* __restrict__ beta, T* __restrict__ Hf,
+                     int64_t rows, int h, float eps, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sC = smem;
+  uint8_t* sZn = sC + C::CB;
+  uint8_t* sG = sZn + C::ZNB;
+  uint8_t* sW = sG + 2 * C::GB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + C::STAGES * C::WS);
+  uint64_t* wfull = bars;                   // [STAGES]
+  uint64_t* wempty = bars + C::STAGES;      // [STAGES]
+  uint64_t* z_full = bars + 2 * C::STAGES;  // [2] Z in TMEM
+  uint64_t* o_full = z_full + 2;            // [2] Z + FFN in TMEM
+  uint64_t* o_empty = z_full + 4;           // [2] read by the epilogue
+  uint64_t* u_full = z_full + 6;            // [2]
+  uint64_t* u_empty = z_full + 8;           // [2]
+  uint64_t* g_full = z_full + 10;           // [2]
+  uint64_t* g_empty = z_full + 12;          // [2]
+  uint64_t* c_full = z_full + 14;
+  uint64_t* c_empty = z_full + 15;
+  uint64_t* zn_full = z_full + 16;
+  uint64_t* zn_empty = z_full + 17;
+  uint64_t* fin = z_full + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(z_full + 19);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmHw);
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmWF);
+    prefetch_tmap(&tmWU);
+    prefetch_tmap(&tmWD);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&z_full[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 4);
+      mbar_init(&u_full[i], 1);
+      mbar_init(&u_empty[i], 4);
+      mbar_init(&g_full[i], 4);
+      mbar_init(&g_empty[i], 1);
+    }
+    mbar_init(c_full, 1);
+    mbar_init(c_empty, 1);
+    mbar_init(zn_full, 4);
+    mbar_init(zn_empty, 1);
+    mbar_init(fin, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t tiles = (rows + C::R - 1) / C::R;
+  const int nh = h / C::HC;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int ws = 0;
+      uint32_t wph = 0, tl = 0, cn = 0;
+      bool ok = true;
+      auto load_w = [&](const CUtensorMap* m, int nbox, int boxb, int x0, int xstep, int y0) -> bool {
+        if (!mbar_wait(&wempty[ws], wph ^ 1u, status)) return false;
+        mbar_arrive_expect_tx(&wfull[ws], static_cast<uint32_t>(C::WS));
+        for (int i = 0; i < nbox; ++i) tma_load_2d(m, &wfull[ws], sW + ws * C::WS + i * boxb, x0 + i * xstep, y0);
+        if (++ws == C::STAGES) {
+          ws = 0;
+          wph ^= 1u;
+        }
+        return true;
+      };
+      for (int64_t t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tl) {
+        const int row0 = static_cast<int>(t * C::R);
+        if (!mbar_wait(c_empty, (tl & 1u) ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(c_full, static_cast<uint32_t>(C::CB));
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tma_load_2d(&tmHw, c_full, sC + bx * C::TBOXB, bx * C::BW, row0);
+          tma_load_2d(&tmA, c_full, sC + (C::NBOX + bx) * C::TBOXB, bx * C::BW, row0);
+        }
+        ++cn;
+        // weights in the order the MMA warp consumes them
+        for (int kc = 0; ok && kc < C::NKC; ++kc) ok = load_w(&tmWF, 64 / C::BW, C::WDBOXB, kc * 64, C::BW, 0);
+        for (int c = 0; ok && c < nh; ++c) {
+          ok = load_w(&tmWU, C::NBOX, C::WUBOXB, 0, C::BW, c * C::HC);
+          if (ok && c > 0) ok = load_w(&tmWD, C::GBOX, C::WDBOXB, (c - 1) * C::HC, C::BW, 0);
+        }
+        if (ok) ok = load_w(&tmWD, C::GBOX, C::WDBOXB, (nh - 1) * C::HC, C::BW, 0);
+      }
+      if (!ok) {  // copies already issued must land before the CTA exits
+        for (int i = 0; i < C::STAGES; ++i) mbar_drain(&wfull[i], wph ^ (i < ws ? 0u : 1u), status);
+        if (cn > 0) mbar_drain(c_full, (cn - 1) & 1u, status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const bool bf = Half16<T>::kBF16;
+      const uint32_t idZ = idesc_f16kind_f32(C::R, C::D, 0, 0, bf);
+      const uint32_t idU = idesc_f16kind_f32(C::R, C::HC, 0, 0, bf);
+      int ws = 0;
+      uint32_t wph = 0, tl = 0, uc = 0;
+      bool ok = true;
+      auto wait_w = [&]() -> bool {
+        if (!mbar_wait(&wfull[ws], wph, status)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto free_w = [&]() {
+        umma_commit(&wempty[ws]);
+        if (++ws == C::STAGES) {
+          ws = 0;
+          wph ^= 1u;
+        }
+      };
+      auto down = [&](uint32_t zc, uint32_t ucc) -> bool {
+        const uint32_t gb = ucc & 1u;
+        if (!mbar_wait(&g_full[gb], (ucc >> 1) & 1u, status) || !wait_w()) return false;
+        const uint32_t ga = smem_u32(sG + gb * C::GB), wa = smem_u32(sW + ws * C::WS);
+#pragma unroll
+        for (int ks = 0; ks < C::HC / 16; ++ks) {
+          const int bx = ks / (C::BW / 16), kin = ks % (C::BW / 16);
+          const uint64_t ad = smem_desc(ga + bx * C::TBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+          const uint64_t bd = smem_desc(wa + bx * C::WDBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+          umma_f16kind(tmem + zc, ad, bd, idZ, 1u);  // onto Z: the residual
+        }
+        free_w();
+        umma_commit(&g_empty[gb]);
+        return true;
+      };
+      for (int64_t t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tl) {
+        const uint32_t zb = tl & 1u, zc = zb * C::D;
+        if (!mbar_wait(c_full, tl & 1u, status) || !mbar_wait(&o_empty[zb], ((tl >> 1) & 1u) ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // Z = [H_w | A] W_F^T
+        const uint32_t ca = smem_u32(sC);
+        for (int kc = 0; ok && kc < C::NKC; ++kc) {
+          if (!wait_w()) {
+            ok = false;
+            break;
+          }
+          const uint32_t wa = smem_u32(sW + ws * C::WS);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const int col = (kc * 4 + ks) * 16;           // input column of [H_w | A]
+            const int part = col / C::D, cp = col % C::D;
+            const int bx = cp / C::BW, kin = (cp % C::BW) / 16;
+            const uint64_t ad =
+                smem_desc(ca + (part * C::NBOX + bx) * C::TBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+            const int lb = (ks * 16) / C::BW, lk = ((ks * 16) % C::BW) / 16;
+            const uint64_t bd = smem_desc(wa + lb * C::WDBOXB + lk * 32, 16, 8 * C::SWB, C::SWMODE);
+            umma_f16kind(tmem + zc, ad, bd, idZ, (kc | ks) != 0 ? 1u : 0u);
+          }
+          free_w();
+        }
+        if (!ok) break;
+        umma_commit(c_empty);
+        umma_commit(&z_full[zb]);
+        if (!mbar_wait(zn_full, tl & 1u, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t za = smem_u32(sZn);
+        for (int c = 0; ok && c < nh; ++c, ++uc) {
+          const uint32_t ub = uc & 1u;
+          if (!mbar_wait(&u_empty[ub], ((uc >> 1) & 1u) ^ 1u, status) || !wait_w()) {
+            ok = false;
+            break;
+          }
+          const uint32_t wa = smem_u32(sW + ws * C::WS);
+#pragma unroll
+          for (int ks = 0; ks < C::D / 16; ++ks) {
+            const int bx = ks / (C::BW / 16), kin = ks % (C::BW / 16);
+            const uint64_t ad = smem_desc(za + bx * C::TBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+            const uint64_t bd = smem_desc(wa + bx * C::WUBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
+            umma_f16kind(tmem + C::UCOL + ub * C::HC, ad, bd, idU, ks != 0 ? 1u : 0u);
+          }
+          free_w();
+          umma_commit(&u_full[ub]);
+          if (c == nh - 1) umma_commit(zn_empty);
+          if (c > 0 && !down(zc, uc - 1u)) ok = false;  // the down projection trails by one chunk
+        }
+        if (!ok || !down(zc, uc - 1u)) {
+          ok = false;
+          break;
+        }
+        umma_commit(&o_full[zb]);
+      }
+      umma_commit(fin);  // no MMA may still write TMEM when it is freed
+      mbar_drain(fin, 0u, status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const float inv_d = 1.0f / static_cast<float>(C::D);
+    uint32_t tl = 0, uc = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
+      const uint32_t zb = tl & 1u, zc = zb * C::D;
+      const int64_t grow = t * C::R + row;
+      if (ok) ok = mbar_wait(&z_full[zb], (tl >> 1) & 1u, status);
+      tc_fence_after();
+      // LayerNorm of Z + b_F over d: two passes over TMEM (mean, then centred squares)
+      float sum = 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < C::D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + zc + cc * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sum += __uint_as_float(r[i]) + whale_bias(bF, cc * 32 + i);
+      }
+      const float mean = sum * inv_d;
+      float sq = 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < C::D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + zc + cc * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float v = __uint_as_float(r[i]) + whale_bias(bF, cc * 32 + i) - mean;
+          sq += v * v;
+        }
+      }
+      const float rstd = rsqrtf(sq * inv_d + eps);
+      if (ok) ok = mbar_wait(zn_empty, (tl & 1u) ^ 1u, status);
+      const uint32_t za = smem_u32(sZn);
+#pragma unroll 1
+      for (int cc = 0; cc < C::D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + zc + cc * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t p[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c0 = cc * 32 + j * 8 + 2 * i;
+            const float a = (__uint_as_float(r[j * 8 + 2 * i]) + whale_bias(bF, c0) - mean) * rstd * __ldg(&gamma[c0]) +
+                            __ldg(&beta[c0]);
+            const float b = (__uint_as_float(r[j * 8 + 2 * i + 1]) + whale_bias(bF, c0 + 1) - mean) * rstd *
+                                __ldg(&gamma[c0 + 1]) +
+                            __ldg(&beta[c0 + 1]);
+            p[i] = Half16<T>::pack2(a, b);
+          }
+          const int col = cc * 32 + j * 8;  // first of 8 columns = one 16-byte unit
+          const uint32_t a = za + (col / C::BW) * C::TBOXB + whale_swz<C::SWB>(row, (col % C::BW) / 8);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(p[0]), "r"(p[1]), "r"(p[2]),
+                       "r"(p[3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(zn_full);
+      // gated chunks: G = U * SiLU(U) = U^2 / (1 + 2^(-U log2 e))
+      for (int c = 0; c < nh; ++c, ++uc) {
+        const uint32_t ub = uc & 1u, up = (uc >> 1) & 1u;
+        if (ok) ok = mbar_wait(&u_full[ub], up, status);
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + lane_base + C::UCOL + ub * C::HC, r0);
+        tmem_ld32(tmem + lane_base + C::UCOL + ub * C::HC + 32, r1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&u_empty[ub]);
+        if (ok) ok = mbar_wait(&g_empty[ub], up ^ 1u, status);
+        const uint32_t ga = smem_u32(sG + ub * C::GB);
+#pragma unroll
+        for (int j = 0; j < C::HC / 8; ++j) {
+          uint32_t p[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = j * 8 + 2 * i;
+            const float va = __uint_as_float(e < 32 ? r0[e] : r1[e - 32]);
+            const float vb = __uint_as_float(e + 1 < 32 ? r0[e + 1] : r1[e + 1 - 32]);
+            p[i] = Half16<T>::pack2(__fdividef(va * va, 1.f + whale_ex2(-1.4426950408889634f * va)),
+                                    __fdividef(vb * vb, 1.f + whale_ex2(-1.4426950408889634f * vb)));
+          }
+          const int col = j * 8;
+          const uint32_t a = ga + (col / C::BW) * C::TBOXB + whale_swz<C::SWB>(row, (col % C::BW) / 8);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(p[0]), "r"(p[1]), "r"(p[2]),
+                       "r"(p[3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&g_full[ub]);
+      }
+      // H_f = Z + G W_down^T (accumulated in TMEM) + b_F
+      if (ok) ok = mbar_wait(&o_full[zb], (tl >> 1) & 1u, status);
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < C::D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + zc + cc * 32, r);
+        tmem_ld_wait();
+        float bias[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) bias[i] = whale_bias(bF, cc * 32 + i);
+        if (grow < rows && ok) whale_st_row32<T>(Hf + grow * C::D + cc * 32, r, 1.f, bias);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[zb]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace wk

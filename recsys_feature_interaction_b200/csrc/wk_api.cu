@@ -16,6 +16,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -37,6 +38,7 @@
 #include "res_ln.cuh"
 #include "res_ln_ring.cuh"
 #include "simt.cuh"
+#include "whale.cuh"
 
 using namespace wk;
 
@@ -2201,6 +2203,313 @@ wk_status wk_moe_combine(const void* const* concats, const void* X, const float*
                                        num_experts, e, dv->standalone_status, st);
   return run_moe_combine<f16, f16>(dv, mp, static_cast<const f16*>(X), g, static_cast<f16*>(out), rows, n, d,
                                    num_experts, e, dv->standalone_status, st);
+}
+
+}  // extern "C"
+
+// ====================================================================== WHALE
+//
+// Attention-based fusion of the WHALE pages (section 2.1 item 3, section 2.2): the
+// attention with shared keys and values, then the fusion Linear and the pre-norm
+// shared-gate SwiGLU FFN with its residual (kernels in whale.cuh).
+
+struct wk_whale {
+  int device = 0;
+  wk_whale_config cfg{};
+  float eps = 1e-5f;
+  const DevInfo* dv = nullptr;
+  wk_whale_weights w{};
+  uint8_t* ws = nullptr;
+  void* A = nullptr;           // [max_batch, n, d] attention output
+  unsigned* status = nullptr;
+  bool prof = false;
+  struct Rec {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+};
+
+namespace {
+
+bool whale_d_ok(int d) { return d == 32 || d == 64 || d == 128 || d == 160; }
+
+// [batch, rows, d] as a 3-D map (d, rows, batch) with boxes (bw, 128, 1): rows past
+// `rows` of an example read as zeros.
+template <typename T>
+bool whale_map3(const DevInfo* dv, CUtensorMap* m, const void* base, int d, int rows, int64_t batch, int bw) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(d) * sizeof(T), static_cast<uint64_t>(rows) * d * sizeof(T)};
+  const uint32_t box[3] = {static_cast<uint32_t>(bw), 128u, 1u};
+  return make_map(dv, m, tmap_dtype<T>(), 3, base, dims, strides, box,
+                  bw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// A row-major [rows, cols] matrix with boxes (bw, box_rows).
+template <typename T>
+bool whale_map2(const DevInfo* dv, CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int bw,
+                int box_rows) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(cols) * sizeof(T)};
+  const uint32_t box[2] = {static_cast<uint32_t>(bw), static_cast<uint32_t>(box_rows)};
+  return make_map(dv, m, tmap_dtype<T>(), 2, base, dims, strides, box,
+                  bw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+template <int D, typename T>
+wk_status whale_attn_run(const DevInfo* dv, const void* Hw, const void* Hs, void* A, int64_t batch, int n, int L,
+                         unsigned* status, cudaStream_t st) {
+  using C = WaCfg<D>;
+  CUtensorMap tq, tkv;
+  if (!whale_map3<T>(dv, &tq, Hw, D, n, batch, C::BW) || !whale_map3<T>(dv, &tkv, Hs, D, L, batch, C::BW))
+    return WK_ERR_UNSUPPORTED;
+  auto fn = whale_attn_kernel<C, T>;
+  const wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fn), C::SMEM);
+  if (s != WK_OK) return s;
+  const int64_t units = batch * ((n + C::R - 1) / C::R);
+  const int grid = static_cast<int>(std::min<int64_t>(units, dv->sms));
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  fn<<<grid, WA_THREADS, C::SMEM, st>>>(tq, tkv, static_cast<T*>(A), batch, n, L, scale_log2, status);
+  return launch_status();
+}
+
+template <int D, typename T>
+wk_status whale_ffn_run(const DevInfo* dv, const void* Hw, const void* A, const wk_whale_weights& w, void* Hf,
+                        int64_t rows, int h, float eps, unsigned* status, cudaStream_t st) {
+  using C = WfCfg<D>;
+  CUtensorMap thw, ta, twf, twu, twd;
+  if (!whale_map2<T>(dv, &thw, Hw, D, rows, C::BW, C::R) || !whale_map2<T>(dv, &ta, A, D, rows, C::BW, C::R) ||
+      !whale_map2<T>(dv, &twf, w.W_F, 2 * D, D, C::BW, D) || !whale_map2<T>(dv, &twu, w.W_up, D, h, C::BW, C::HC) ||
+      !whale_map2<T>(dv, &twd, w.W_down, h, D, C::BW, D))
+    return WK_ERR_UNSUPPORTED;
+  auto fn = whale_ffn_kernel<C, T>;
+  const wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fn), C::SMEM);
+  if (s != WK_OK) return s;
+  const int64_t tiles = (rows + C::R - 1) / C::R;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, dv->sms));
+  fn<<<grid, WF_THREADS, C::SMEM, st>>>(thw, ta, twf, twu, twd, w.b_F, w.ln_gamma, w.ln_beta, static_cast<T*>(Hf),
+                                        rows, h, eps, status);
+  return launch_status();
+}
+
+template <typename T>
+wk_status whale_attn_dispatch(const DevInfo* dv, const void* Hw, const void* Hs, void* A, int64_t batch, int n,
+                              int L, int d, unsigned* status, cudaStream_t st) {
+  switch (d) {
+    case 32: return whale_attn_run<32, T>(dv, Hw, Hs, A, batch, n, L, status, st);
+    case 64: return whale_attn_run<64, T>(dv, Hw, Hs, A, batch, n, L, status, st);
+    case 128: return whale_attn_run<128, T>(dv, Hw, Hs, A, batch, n, L, status, st);
+    case 160: return whale_attn_run<160, T>(dv, Hw, Hs, A, batch, n, L, status, st);
+  }
+  return WK_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+wk_status whale_ffn_dispatch(const DevInfo* dv, const void* Hw, const void* A, const wk_whale_weights& w, void* Hf,
+                             int64_t rows, int d, int h, float eps, unsigned* status, cudaStream_t st) {
+  switch (d) {
+    case 32: return whale_ffn_run<32, T>(dv, Hw, A, w, Hf, rows, h, eps, status, st);
+    case 64: return whale_ffn_run<64, T>(dv, Hw, A, w, Hf, rows, h, eps, status, st);
+    case 128: return whale_ffn_run<128, T>(dv, Hw, A, w, Hf, rows, h, eps, status, st);
+    case 160: return whale_ffn_run<160, T>(dv, Hw, A, w, Hf, rows, h, eps, status, st);
+  }
+  return WK_ERR_UNSUPPORTED;
+}
+
+wk_status whale_check_weights(const wk_whale_weights* w) {
+  if (!w || !w->W_F || !w->ln_gamma || !w->ln_beta || !w->W_up || !w->W_down) return WK_ERR_INVALID_ARG;
+  if (!al16(w->W_F) || !al16(w->W_up) || !al16(w->W_down) || (w->b_F && !al16(w->b_F)) || !al16(w->ln_gamma) ||
+      !al16(w->ln_beta))
+    return WK_ERR_INVALID_ARG;
+  return WK_OK;
+}
+
+// Event pair around one launch of a WHALE handle (as the stack's per-kernel records).
+struct WhaleProf {
+  wk_whale* h;
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  WhaleProf(wk_whale* h_, int k, cudaStream_t s) : h(h_), kind(k), st(s) {
+    if (!h->prof) return;
+    a = take();
+    b = take();
+    if (a && b) cudaEventRecord(a, st);
+  }
+  cudaEvent_t take() {
+    cudaEvent_t e = nullptr;
+    if (!h->pool.empty()) {
+      e = h->pool.back();
+      h->pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      e = nullptr;
+    }
+    return e;
+  }
+  ~WhaleProf() {
+    if (!h->prof) return;
+    if (a && b) {
+      cudaEventRecord(b, st);
+      h->recs.push_back({kind, a, b});
+    } else {
+      if (a) h->pool.push_back(a);
+      if (b) h->pool.push_back(b);
+    }
+  }
+};
+
+void free_whale(wk_whale* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaGetLastError();
+  if (h->ws) cudaFree(h->ws);
+  for (auto& r : h->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : h->pool) cudaEventDestroy(e);
+  cudaGetLastError();
+  delete h;
+}
+
+}  // namespace
+
+extern "C" {
+
+wk_status wk_whale_create(const wk_whale_config* cfg, const wk_whale_weights* w, wk_whale** out) {
+  if (!cfg || !out) return WK_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (cfg->n < 1 || cfg->L < 1 || cfg->max_batch < 1 || cfg->ln_eps < 0.f) return WK_ERR_INVALID_ARG;
+  if (cfg->dtype != WK_BF16 && cfg->dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  if (!whale_d_ok(cfg->d) || cfg->h < 64 || cfg->h % 64 != 0) return WK_ERR_UNSUPPORTED;
+  wk_status st = whale_check_weights(w);
+  if (st != WK_OK) return st;
+  DevInfo* dv = nullptr;
+  st = dev_info(&dv);
+  if (st != WK_OK) return st;
+  wk_whale* h = new (std::nothrow) wk_whale;
+  if (!h) return WK_ERR_OOM;
+  h->device = dv->id;
+  h->cfg = *cfg;
+  h->dv = dv;
+  h->w = *w;
+  h->eps = cfg->ln_eps > 0.f ? cfg->ln_eps : 1e-5f;
+  const size_t abytes = ((static_cast<size_t>(cfg->max_batch) * cfg->n * cfg->d * 2 + 255) / 256) * 256;
+  if (cudaMalloc(&h->ws, abytes + 256) != cudaSuccess) {
+    cudaGetLastError();
+    free_whale(h);
+    return WK_ERR_OOM;
+  }
+  h->A = h->ws;
+  h->status = reinterpret_cast<unsigned*>(h->ws + abytes);
+  if (cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    free_whale(h);
+    return WK_ERR_CUDA;
+  }
+  *out = h;
+  return WK_OK;
+}
+
+wk_status wk_whale_forward(wk_whale* h, const void* Hw, const void* Hs, void* Hf, int64_t batch, wk_stream_t stream) {
+  if (!h || batch < 0 || batch > h->cfg.max_batch) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!Hw || !Hs || !Hf || !al16(Hw) || !al16(Hs) || !al16(Hf)) return WK_ERR_INVALID_ARG;
+  const wk_whale_config& c = h->cfg;
+  const size_t fb = static_cast<size_t>(batch) * c.n * c.d * 2, sb = static_cast<size_t>(batch) * c.L * c.d * 2;
+  const uint8_t* f = static_cast<const uint8_t*>(Hf);
+  const uint8_t* q = static_cast<const uint8_t*>(Hw);
+  const uint8_t* k = static_cast<const uint8_t*>(Hs);
+  if ((f < q + fb && q < f + fb) || (f < k + sb && k < f + fb)) return WK_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) {
+    cudaGetLastError();
+    return WK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t rows = batch * c.n;
+  wk_status s;
+  {
+    WhaleProf ps(h, WK_KERNEL_WHALE_ATTN, st);
+    s = c.dtype == WK_BF16 ? whale_attn_dispatch<bf16>(h->dv, Hw, Hs, h->A, batch, c.n, c.L, c.d, h->status, st)
+                           : whale_attn_dispatch<f16>(h->dv, Hw, Hs, h->A, batch, c.n, c.L, c.d, h->status, st);
+  }
+  if (s != WK_OK) return s;
+  WhaleProf ps(h, WK_KERNEL_WHALE_FFN, st);
+  return c.dtype == WK_BF16
+             ? whale_ffn_dispatch<bf16>(h->dv, Hw, h->A, h->w, Hf, rows, c.d, c.h, h->eps, h->status, st)
+             : whale_ffn_dispatch<f16>(h->dv, Hw, h->A, h->w, Hf, rows, c.d, c.h, h->eps, h->status, st);
+}
+
+wk_status wk_whale_sync_status(wk_whale* h, wk_stream_t stream) {
+  if (!h) return WK_ERR_INVALID_ARG;
+  return read_status_word(h->status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+wk_status wk_whale_set_profiling(wk_whale* h, int enable) {
+  if (!h) return WK_ERR_INVALID_ARG;
+  h->prof = enable != 0;
+  return WK_OK;
+}
+
+wk_status wk_whale_kernel_times(wk_whale* h, double* total_ms, int64_t* launches) {
+  if (!h || !total_ms || !launches) return WK_ERR_INVALID_ARG;
+  for (int i = 0; i < WK_KERNEL_COUNT; ++i) {
+    total_ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  wk_status s = WK_OK;
+  for (auto& r : h->recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();
+      s = WK_ERR_CUDA;
+    } else if (r.kind >= 0 && r.kind < WK_KERNEL_COUNT) {
+      total_ms[r.kind] += ms;
+      launches[r.kind] += 1;
+    }
+    h->pool.push_back(r.a);
+    h->pool.push_back(r.b);
+  }
+  h->recs.clear();
+  return s;
+}
+
+void wk_whale_destroy(wk_whale* h) { free_whale(h); }
+
+wk_status wk_whale_attention(const void* Hw, const void* Hs, void* A, int64_t batch, int32_t n, int32_t L, int32_t d,
+                             wk_dtype dtype, wk_stream_t stream) {
+  if (batch < 0 || n < 1 || L < 1) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!Hw || !Hs || !A || !al16(Hw) || !al16(Hs) || !al16(A)) return WK_ERR_INVALID_ARG;
+  if (dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  if (!whale_d_ok(d)) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  wk_status s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return dtype == WK_BF16 ? whale_attn_dispatch<bf16>(dv, Hw, Hs, A, batch, n, L, d, dv->standalone_status, st)
+                          : whale_attn_dispatch<f16>(dv, Hw, Hs, A, batch, n, L, d, dv->standalone_status, st);
+}
+
+wk_status wk_whale_fusion_ffn(const void* Hw, const void* A, const wk_whale_weights* w, void* Hf, int64_t rows,
+                              int32_t d, int32_t h, wk_dtype dtype, float eps, wk_stream_t stream) {
+  if (rows < 0 || eps < 0.f) return WK_ERR_INVALID_ARG;
+  if (rows == 0) return WK_OK;
+  if (!Hw || !A || !Hf || !al16(Hw) || !al16(A) || !al16(Hf)) return WK_ERR_INVALID_ARG;
+  wk_status s = whale_check_weights(w);
+  if (s != WK_OK) return s;
+  if (dtype != WK_BF16 && dtype != WK_F16) return WK_ERR_UNSUPPORTED;
+  if (!whale_d_ok(d) || h < 64 || h % 64 != 0) return WK_ERR_UNSUPPORTED;
+  DevInfo* dv = nullptr;
+  s = dev_info(&dv);
+  if (s != WK_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float e = eps > 0.f ? eps : 1e-5f;
+  return dtype == WK_BF16 ? whale_ffn_dispatch<bf16>(dv, Hw, A, *w, Hf, rows, d, h, e, dv->standalone_status, st)
+                          : whale_ffn_dispatch<f16>(dv, Hw, A, *w, Hf, rows, d, h, e, dv->standalone_status, st);
 }
 
 }  // extern "C"

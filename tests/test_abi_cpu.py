@@ -129,3 +129,35 @@ def test_kernel_kind_count_matches_the_header():
     text = open(os.path.join(ROOT, "include", "wukong.h")).read()
     m = re.search(r"WK_KERNEL_COUNT\s*=\s*(\d+)", text)
     assert m and int(m.group(1)) == wk.WK_KERNEL_COUNT == len(wk.KERNEL_NAMES)
+
+
+def _whale_status(lib, **kw):
+    cfg = dict(n=64, d=128, L=2048, h=512, dtype="bf16", batch=4)
+    cfg.update(kw)
+    w = {"W_F": FAKE, "b_F": None, "ln_gamma": FAKE, "ln_beta": FAKE, "W_up": FAKE, "W_down": FAKE}
+    c = wk.WkWhaleConfig(cfg["n"], cfg["d"], cfg["L"], cfg["h"], wk._dtype_code(cfg["dtype"]), 0.0, cfg["batch"])
+    ww = wk._whale_weights(w)
+    h = ctypes.c_void_p()
+    return lib.wk_whale_create(ctypes.byref(c), ctypes.byref(ww), ctypes.byref(h))
+
+
+def test_whale_argument_errors_without_a_device(L):
+    assert _whale_status(L, d=48) == wk.WK_ERR_UNSUPPORTED
+    assert _whale_status(L, d=256) == wk.WK_ERR_UNSUPPORTED
+    assert _whale_status(L, h=100) == wk.WK_ERR_UNSUPPORTED
+    assert _whale_status(L, dtype="f32") == wk.WK_ERR_UNSUPPORTED
+    assert _whale_status(L, n=0) == wk.WK_ERR_INVALID_ARG
+    assert _whale_status(L, L=0) == wk.WK_ERR_INVALID_ARG
+    assert _whale_status(L, batch=0) == wk.WK_ERR_INVALID_ARG
+    c = wk.WkWhaleConfig(64, 128, 2048, 512, wk.WK_BF16, 0.0, 4)
+    bad = wk.WkWhaleWeights(FAKE, None, FAKE, FAKE, FAKE + 2, FAKE)  # W_up not 16-byte aligned
+    h = ctypes.c_void_p()
+    assert L.wk_whale_create(ctypes.byref(c), ctypes.byref(bad), ctypes.byref(h)) == wk.WK_ERR_INVALID_ARG
+    assert L.wk_whale_attention(FAKE, FAKE, FAKE, 0, 64, 2048, 128, wk.WK_BF16, None) == wk.WK_OK
+    assert L.wk_whale_attention(FAKE, FAKE, FAKE, 2, 64, 2048, 96, wk.WK_BF16, None) == wk.WK_ERR_UNSUPPORTED
+    assert L.wk_whale_attention(FAKE, FAKE, FAKE, 2, 64, 0, 128, wk.WK_BF16, None) == wk.WK_ERR_INVALID_ARG
+    w = wk.WkWhaleWeights(FAKE, None, FAKE, FAKE, FAKE, FAKE)
+    assert L.wk_whale_fusion_ffn(FAKE, FAKE, ctypes.byref(w), FAKE, 5, 128, 96, wk.WK_BF16, ctypes.c_float(0),
+                                 None) == wk.WK_ERR_UNSUPPORTED
+    assert L.wk_whale_fusion_ffn(FAKE, FAKE, ctypes.byref(w), FAKE, 0, 128, 512, wk.WK_BF16, ctypes.c_float(0),
+                                 None) == wk.WK_OK
