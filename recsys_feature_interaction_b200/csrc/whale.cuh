@@ -67,6 +67,19 @@ __device__ __forceinline__ uint32_t whale_swz(int r, int j) {
   return static_cast<uint32_t>(r * SWB + ((SWB == 128 ? (j ^ (r & 7)) : (j ^ ((r >> 1) & 3))) << 4));
 }
 
+// max of 64 fp32 values held as bit patterns, as a balanced tree (short dependency chains).
+__device__ __forceinline__ float whale_max64(const uint32_t (&v)[64]) {
+  float t[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) t[i] = fmaxf(__uint_as_float(v[i]), __uint_as_float(v[i + 32]));
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  }
+  return t[0];
+}
+
 // b_F[i], or zero when the fusion Linear has no bias.
 __device__ __forceinline__ float whale_bias(const float* __restrict__ b, int i) { return b ? __ldg(&b[i]) : 0.f; }
 
@@ -105,7 +118,9 @@ struct WaCfg {
   static constexpr int PBOXB = R * 128;                  // P: 64 keys per 128B-swizzled box
   static constexpr int PB = (LB / 64) * PBOXB;
   static constexpr int LIMIT = 227 * 1024;
-  static constexpr int FIXED = 1024 + QB + 2 * PB + 256;
+  static constexpr int BARB = 256;                       // mbarriers and the TMEM address
+  static constexpr int REDB = 6 * R * 4;                 // softmax pair exchange (row maxima, row sums)
+  static constexpr int FIXED = 1024 + QB + PB + BARB + REDB;
   static constexpr int STAGES_RAW = (LIMIT - FIXED) / KVB;
   static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
   // at least half an SM's shared memory: one CTA per SM, so that its 512 TMEM columns are free
@@ -117,7 +132,7 @@ struct WaCfg {
   static_assert(QB % 1024 == 0 && KVB % 1024 == 0 && PB % 1024 == 0, "swizzle atoms stay aligned");
 };
 
-constexpr int WA_THREADS = 192;
+constexpr int WA_THREADS = 320;  // producer, MMA issuer, 8 softmax warps
 
 template <class C, typename T>
 __global__ void __launch_bounds__(WA_THREADS, 1)
@@ -128,18 +143,20 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + C::QB;
   uint8_t* sP = sKV + C::STAGES * C::KVB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::PB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::PB);
   uint64_t* kv_full = bars;                  // [STAGES] key tile landed
   uint64_t* kv_empty = bars + C::STAGES;     // [STAGES] both products read it
   uint64_t* s_full = bars + 2 * C::STAGES;   // [2] S in TMEM
   uint64_t* s_empty = s_full + 2;            // [2] S read by the softmax warps
-  uint64_t* p_full = s_full + 4;             // [2] P in shared memory
-  uint64_t* q_full = s_full + 6;
-  uint64_t* q_empty = s_full + 7;
-  uint64_t* pv_done = s_full + 8;            // one phase per P V block, in order
-  uint64_t* o_empty = s_full + 9;            // O read by the softmax warps (per unit)
-  uint64_t* fin = s_full + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 11);
+  uint64_t* p_full = s_full + 4;             // P in shared memory (one phase per block)
+  uint64_t* q_full = s_full + 5;
+  uint64_t* q_empty = s_full + 6;
+  uint64_t* pv_done = s_full + 7;            // one phase per P V block, in order
+  uint64_t* o_empty = s_full + 8;            // O read by the softmax warps (per unit)
+  uint64_t* fin = s_full + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
+  float* red_max = reinterpret_cast<float*>(sP + C::PB + C::BARB);  // [2 parities][2 halves][R]
+  float* red_sum = red_max + 4 * C::R;                                   // [2 halves][R]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -152,13 +169,13 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&s_empty[i], 8);
     }
+    mbar_init(p_full, 8);
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     mbar_init(pv_done, 1);
-    mbar_init(o_empty, 4);
+    mbar_init(o_empty, 8);
     mbar_init(fin, 1);
     fence_mbar_init();
   }
@@ -262,12 +279,12 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
             ok = false;
             break;
           }
-          if (!mbar_wait(&p_full[gj & 1u], (gj >> 1) & 1u, status)) {
+          if (!mbar_wait(p_full, gj & 1u, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t pa = smem_u32(sP + (gj & 1u) * C::PB), va = smem_u32(sKV + cs * C::KVB);
+          const uint32_t pa = smem_u32(sP), va = smem_u32(sKV + cs * C::KVB);
 #pragma unroll
           for (int ks = 0; ks < C::LB / 16; ++ks) {
             const uint64_t ad = smem_desc(pa + (ks / 4) * C::PBOXB + (ks % 4) * 32, 16, 1024, 2u);
@@ -286,48 +303,81 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int q = warp & 3;  // TMEM lane quarter of this warp
+    // Two warps per TMEM lane quarter: warp w reads rows 32 (w % 4) .. + 31 (the
+    // quarter its hardware sub-partition may access) and the key columns
+    // 64 * half .. + 63 of each S block. The pair exchanges per-row partial maxima
+    // (double-buffered by block parity) and, at the end of a unit, partial row sums,
+    // through shared memory under a 64-thread named barrier.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const int bar_id = 1 + q;
     uint32_t g = 0;
     // After a failed wait a thread stops waiting but walks the same schedule, so the
-    // warp-collective TMEM accesses stay converged.
+    // warp-collective TMEM accesses and the pair barriers stay converged.
     bool ok = true;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
       const int b = static_cast<int>(u / qtiles), q0 = static_cast<int>(u % qtiles) * C::R;
-      const bool warp_on = q0 + q * 32 < n;
+      const bool warp_on = q0 + q * 32 < n;  // the pair agrees: same rows
       const bool row_on = q0 + row < n;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nb; ++j) {
         const uint32_t gj = g + static_cast<uint32_t>(j), buf = gj & 1u;
         if (ok) ok = mbar_wait(&s_full[buf], (gj >> 1) & 1u, status);
         tc_fence_after();
-        uint32_t sr[C::LB];
+        uint32_t sr[C::LB / 2];
         if (warp_on) {
-#pragma unroll
-          for (int c = 0; c < C::LB / 32; ++c)
-            tmem_ld32(tmem + lane_base + buf * C::LB + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          const uint32_t ta = tmem + lane_base + buf * C::LB + half * (C::LB / 2);
+          tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
           tmem_ld_wait();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[buf]);
-        const int kvalid = min(C::LB, L - j * C::LB);
-        float mb = -INFINITY;
+        const int kvalid = min(C::LB, L - j * C::LB) - half * (C::LB / 2);  // valid columns of this half
+        const bool full = kvalid >= C::LB / 2;
+        float mh = -INFINITY;
+        if (full) {
+          mh = whale_max64(sr);
+        } else {
 #pragma unroll
-        for (int c = 0; c < C::LB; ++c)
-          if (c < kvalid) mb = fmaxf(mb, __uint_as_float(sr[c]));
+          for (int c = 0; c < C::LB / 2; ++c)
+            if (c < kvalid) mh = fmaxf(mh, __uint_as_float(sr[c]));
+        }
+        red_max[(buf * 2 + half) * C::R + row] = mh;
+        named_bar(bar_id, 64);
+        const float mb = fmaxf(mh, red_max[(buf * 2 + (half ^ 1)) * C::R + row]);
         const float mb2 = mb * scale_log2;
         const bool need = warp_on && row_on && (mb2 > m + 8.f);
-        // P V of the previous block has finished: its P buffer (two blocks back) is free
-        // and O holds every earlier block.
-        if (gj > 0 && ok) ok = mbar_wait(pv_done, (gj - 1) & 1u, status);
-        tc_fence_after();
         const float mnew = need ? mb2 : m;
         const float factor = need ? whale_ex2(m - mnew) : 1.f;
+        // P = 2^(S log2(e)/sqrt(d) - m), rounded to the operand type, in registers
+        uint32_t pk[C::LB / 4];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        if (warp_on) {
+          const float nm = row_on ? -mnew : 0.f;
+#pragma unroll
+          for (int c2 = 0; c2 < C::LB / 4; ++c2) {
+            float p0 = whale_ex2(fmaf(__uint_as_float(sr[2 * c2]), scale_log2, nm));
+            float p1 = whale_ex2(fmaf(__uint_as_float(sr[2 * c2 + 1]), scale_log2, nm));
+            if (!full) {
+              if (2 * c2 >= kvalid) p0 = 0.f;
+              if (2 * c2 + 1 >= kvalid) p1 = 0.f;
+            }
+            ls[(2 * c2) & 3] += p0;
+            ls[(2 * c2 + 1) & 3] += p1;
+            pk[c2] = Half16<T>::pack2(p0, p1);
+          }
+        }
+        // P V of the previous block has finished: the P buffer is free and O holds
+        // every earlier block.
+        if (gj > 0 && ok) ok = mbar_wait(pv_done, (gj - 1) & 1u, status);
+        tc_fence_after();
         if (warp_on && j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-          for (int cc = 0; cc < C::D / 32; ++cc) {
+          for (int cc = half; cc < C::D / 32; cc += 2) {
             uint32_t o[32];
             tmem_ld32(tmem + lane_base + C::OCOL + cc * 32, o);
             tmem_ld_wait();
@@ -337,43 +387,33 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
           }
           whale_tmem_st_wait();
         }
-        l *= factor;
+        l = l * factor + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         m = mnew;
         if (warp_on) {
-          const float mm = row_on ? m : 0.f;
-          const uint32_t pb = smem_u32(sP + buf * C::PB);
-          float ls = 0.f;
+          const uint32_t pb = smem_u32(sP) + half * C::PBOXB;
 #pragma unroll
-          for (int c8 = 0; c8 < C::LB / 8; ++c8) {
-            float p[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int c = c8 * 8 + i;
-              p[i] = c < kvalid ? whale_ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -mm)) : 0.f;
-              ls += p[i];
-            }
-            const uint32_t a = pb + (c8 / 8) * C::PBOXB + whale_swz<128>(row, c8 % 8);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(Half16<T>::pack2(p[0], p[1])),
-                         "r"(Half16<T>::pack2(p[2], p[3])), "r"(Half16<T>::pack2(p[4], p[5])),
-                         "r"(Half16<T>::pack2(p[6], p[7]))
+          for (int c8 = 0; c8 < C::LB / 16; ++c8)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + whale_swz<128>(row, c8)),
+                         "r"(pk[4 * c8]), "r"(pk[4 * c8 + 1]), "r"(pk[4 * c8 + 2]), "r"(pk[4 * c8 + 3])
                          : "memory");
-          }
-          l += ls;
         }
         fence_proxy_async_smem();  // the tensor core reads P
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[buf]);
+        if (lane == 0) mbar_arrive(p_full);
       }
-      // the unit's output rows: O / l
+      // the unit's output rows: O / (l of both halves)
+      red_sum[half * C::R + row] = l;
+      named_bar(bar_id, 64);
+      const float lt = l + red_sum[(half ^ 1) * C::R + row];
       const uint32_t gl = g + static_cast<uint32_t>(nb) - 1u;
       if (ok) ok = mbar_wait(pv_done, gl & 1u, status);
       tc_fence_after();
       if (warp_on) {
-        const float inv = row_on ? 1.f / l : 0.f;
+        const float inv = row_on ? 1.f / lt : 0.f;
         T* dst = Aout + (static_cast<int64_t>(b) * n + q0 + row) * C::D;
 #pragma unroll 1
-        for (int cc = 0; cc < C::D / 32; ++cc) {
+        for (int cc = half; cc < C::D / 32; cc += 2) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_base + C::OCOL + cc * 32, o);
           tmem_ld_wait();
@@ -383,6 +423,8 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty);
+      // red_sum is written again only after the next unit's first pair barrier, which
+      // the partner reaches after reading it
       g += static_cast<uint32_t>(nb);
     }
   }

@@ -2,6 +2,7 @@
 
     python -m recsys_feature_interaction_b200.microbench --kernel fm_ln|mlp_gemm|lcb|res_ln|moe_gate|moe_combine
         [--workload c4_bf16] [--batch B] [--iters K] [--dtype f16|bf16] [--layer-linear j] [--experts E]
+    python -m recsys_feature_interaction_b200.microbench --kernel whale_attn|whale_ffn [--workload whale_c4] ...
 
 Inputs are synthetic (the seeded generator), on the device, in the workload's
 shapes. Prints one JSON line with the mean CUDA-event time per launch and the
@@ -20,7 +21,8 @@ if ROOT not in sys.path:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", required=True, choices=["fm_ln", "mlp_gemm", "lcb", "res_ln", "moe_gate", "moe_combine"])
+    ap.add_argument("--kernel", required=True, choices=["fm_ln", "mlp_gemm", "lcb", "res_ln", "moe_gate", "moe_combine",
+                                                           "whale_attn", "whale_ffn"])
     ap.add_argument("--workload", default="c4_bf16")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--iters", type=int, default=10)
@@ -38,6 +40,9 @@ def main():
     from synth import configs as C
 
     build.build()
+    if args.kernel.startswith("whale"):
+        run, flops, bytes_, B = _whale_case(args)
+        return _time(args, run, flops, bytes_, B)
     cfg = C.MOE_CONFIGS[args.workload] if args.workload in C.MOE_CONFIGS else C.CONFIGS[args.workload]
     B = args.batch or cfg["batch"]
     n, d, k, n_f, n_l = cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], cfg["n_l"]
@@ -103,6 +108,41 @@ def main():
             wk.wk_res_ln(cat, X, w["out_gamma"], w["out_beta"], out, B * n, d, args.dtype)
         flops = 0
         bytes_ = 3 * n * d * es * B
+    return _time(args, run, flops, bytes_, B)
+
+
+def _whale_case(args):
+    """The WHALE attention (A from H_w, H_s) or the fusion + FFN (H_f from H_w, A) alone."""
+    import torch
+
+    import recsys_feature_interaction_b200 as wk
+    from synth import configs as C
+    cfg = C.WHALE_CONFIGS[args.workload if args.workload in C.WHALE_CONFIGS else "whale_c4"]
+    B = args.batch or cfg["batch"]
+    n, L, d, h = cfg["n"], cfg["L"], cfg["d"], cfg["h"]
+    tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    Hw, Hs = C.make_whale_inputs_dev(cfg, B)
+    Hw, Hs = Hw.to(tdt), Hs.to(tdt)
+    A = torch.empty_like(Hw)
+    es = 2
+    if args.kernel == "whale_attn":
+        def run():
+            wk.wk_whale_attention(Hw, Hs, A, B, n, L, d, args.dtype)
+        return run, 4 * n * L * d * B, (L * d + 2 * n * d) * es * B, B
+    w = {k: (v.to(tdt) if v.dtype != torch.float32 else v) for k, v in C.make_whale_dev(cfg).items()}
+    A.copy_(Hw * 0.5)
+    Hf = torch.empty_like(Hw)
+    rows = B * n
+
+    def run():
+        wk.wk_whale_fusion_ffn(Hw, A, w, Hf, rows, d, h, args.dtype)
+    return run, rows * (4 * d * d + 4 * d * h), (3 * rows * d + 2 * d * d + 2 * d * h) * es, B
+
+
+def _time(args, run, flops, bytes_, B):
+    import torch
+
+    import recsys_feature_interaction_b200 as wk
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
