@@ -35,6 +35,8 @@
 // let issued copies land, let issued MMAs finish and free TMEM before the CTA exits.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace wk {
@@ -67,17 +69,40 @@ __device__ __forceinline__ uint32_t whale_swz(int r, int j) {
   return static_cast<uint32_t>(r * SWB + ((SWB == 128 ? (j ^ (r & 7)) : (j ^ ((r >> 1) & 3))) << 4));
 }
 
-// max of 64 fp32 values held as bit patterns, as a balanced tree (short dependency chains).
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float whale_max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max of 64 fp32 values held as bit patterns: a tree of three-input maxima (32 instructions,
+// short dependency chains).
 __device__ __forceinline__ float whale_max64(const uint32_t (&v)[64]) {
-  float t[32];
+  float t[22], u[8];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) t[i] = fmaxf(__uint_as_float(v[i]), __uint_as_float(v[i + 32]));
+  for (int i = 0; i < 21; ++i)
+    t[i] = whale_max3(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
+  t[21] = __uint_as_float(v[63]);
 #pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-  }
-  return t[0];
+  for (int i = 0; i < 7; ++i) u[i] = whale_max3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+  u[7] = t[21];
+  return whale_max3(whale_max3(u[0], u[1], u[2]), whale_max3(u[3], u[4], u[5]), fmaxf(u[6], u[7]));
+}
+
+// 2^x on the FMA pipe, for some of the softmax weights, so that the special-function
+// unit (the approximate ex2 above) does not bound the softmax alone. x = j + f with j the
+// integer nearest to x (adding 1.5 * 2^23 rounds it into the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted to 2^f by relative least squares
+// on Chebyshev nodes for this kernel (max relative error 7.5e-5 in fp32, below the 16-bit
+// rounding of the weights); 2^j enters as j added to the exponent bits. x is clamped
+// below at -126 (2^-126 stands for 0).
+__device__ __forceinline__ float whale_ex2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.05517158f, f, 0.24261111f), f, 0.69326103f), f, 0.99992806f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // b_F[i], or zero when the fusion Linear has no bias.
@@ -102,6 +127,33 @@ __device__ __forceinline__ void whale_st_row32(T* dst, const uint32_t (&r)[32], 
 
 // ----------------------------------------------------------------- attention
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, issued by one thread: A is read from tensor
+// memory (row i in lane i, consecutive 16-bit K elements packed two per 32-bit column).
+__device__ __forceinline__ void whale_umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void whale_tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// NC consecutive 32-bit TMEM columns (a multiple of 8) from registers.
+template <int NC>
+__device__ __forceinline__ void whale_tmem_st_cols(uint32_t taddr, const uint32_t (&r)[NC]) {
+#pragma unroll
+  for (int c = 0; c + 32 <= NC; c += 32) whale_tmem_st32(taddr + c, *reinterpret_cast<const uint32_t(*)[32]>(&r[c]));
+#pragma unroll
+  for (int c = (NC / 32) * 32; c < NC; c += 8) whale_tmem_st8(taddr + c, &r[c]);
+}
+
 template <int D_>
 struct WaCfg {
   static constexpr int D = D_;
@@ -111,57 +163,55 @@ struct WaCfg {
   static constexpr int SWB = BW * 2;                     // bytes per box row = swizzle span
   static constexpr uint32_t SWMODE = BW == 64 ? 2u : 4u; // descriptor swizzle: 128B / 64B
   static constexpr int NBOX = D / BW;
-  static constexpr int QBOXB = R * SWB;
   static constexpr int KVBOXB = LB * SWB;
-  static constexpr int QB = NBOX * QBOXB;
-  static constexpr int KVB = NBOX * KVBOXB;
-  static constexpr int PBOXB = R * 128;                  // P: 64 keys per 128B-swizzled box
-  static constexpr int PB = (LB / 64) * PBOXB;
+  static constexpr int KVB = NBOX * KVBOXB;              // one key/value tile
   static constexpr int LIMIT = 227 * 1024;
-  static constexpr int BARB = 256;                       // mbarriers and the TMEM address
-  static constexpr int REDB = 6 * R * 4;                 // softmax pair exchange (row maxima, row sums)
-  static constexpr int FIXED = 1024 + QB + PB + BARB + REDB;
+  static constexpr int BARB = 176;                       // mbarriers and the TMEM address
+  static constexpr int REDB = 4 * R * 4;                 // softmax pair exchange [2 parities][2 halves][R]
+  // The dynamic shared memory starts 1024-byte aligned (checked at run time): no slack.
+  static constexpr int FIXED = BARB + REDB;
   static constexpr int STAGES_RAW = (LIMIT - FIXED) / KVB;
-  static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
+  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
   // at least half an SM's shared memory: one CTA per SM, so that its 512 TMEM columns are free
   static constexpr int SMEM = FIXED + STAGES * KVB > 120 * 1024 ? FIXED + STAGES * KVB : 120 * 1024;
-  static constexpr int OCOL = 2 * LB;                    // TMEM: S0 [0,128), S1 [128,256), O [256, 256+D)
-  static_assert(D % 32 == 0 && D >= 32 && D <= 256, "D");
-  static_assert(OCOL + D <= 512, "TMEM columns");
+  // TMEM: S0 [0,128), S1 [128,256) (P_j written over the first 64 columns of S_j), O [256, 256+D),
+  // Q [256+D, 256+D+D/2) (16-bit pairs)
+  static constexpr int OCOL = 2 * LB;
+  static constexpr int QCOL = OCOL + D;
+  static_assert(D % 32 == 0 && D >= 32 && D <= 160, "D");
+  static_assert(QCOL + D / 2 <= 512, "TMEM columns");
   static_assert(STAGES >= 2, "shared memory");
-  static_assert(QB % 1024 == 0 && KVB % 1024 == 0 && PB % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(KVB % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert((2 * STAGES + 9) * 8 + 4 <= BARB, "barriers");
 };
 
 constexpr int WA_THREADS = 320;  // producer, MMA issuer, 8 softmax warps
 
 template <class C, typename T>
 __global__ void __launch_bounds__(WA_THREADS, 1)
-    whale_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
-                      T* __restrict__ Aout, int64_t batch, int n, int L, float scale_log2, unsigned* status) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::QB;
-  uint8_t* sP = sKV + C::STAGES * C::KVB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::PB);
+    whale_attn_kernel(const __grid_constant__ CUtensorMap tmKV, const T* __restrict__ Hw, T* __restrict__ Aout,
+                      int64_t batch, int n, int L, float scale_log2, unsigned* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {  // the swizzled layout needs 1024-byte alignment
+    if (threadIdx.x == 0) flag_error(status, kFlagBadShape);
+    return;
+  }
+  uint8_t* sKV = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::STAGES * C::KVB);
   uint64_t* kv_full = bars;                  // [STAGES] key tile landed
   uint64_t* kv_empty = bars + C::STAGES;     // [STAGES] both products read it
   uint64_t* s_full = bars + 2 * C::STAGES;   // [2] S in TMEM
-  uint64_t* s_empty = s_full + 2;            // [2] S read by the softmax warps
-  uint64_t* p_full = s_full + 4;             // P in shared memory (one phase per block)
-  uint64_t* q_full = s_full + 5;
-  uint64_t* q_empty = s_full + 6;
-  uint64_t* pv_done = s_full + 7;            // one phase per P V block, in order
-  uint64_t* o_empty = s_full + 8;            // O read by the softmax warps (per unit)
-  uint64_t* fin = s_full + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
-  float* red_max = reinterpret_cast<float*>(sP + C::PB + C::BARB);  // [2 parities][2 halves][R]
-  float* red_sum = red_max + 4 * C::R;                                   // [2 halves][R]
+  uint64_t* p_full = s_full + 2;             // [2] P in TMEM
+  uint64_t* p_empty = s_full + 4;            // [2] P V has read it (so O holds that block)
+  uint64_t* q_full = s_full + 6;             // the unit's Q rows are in TMEM
+  uint64_t* o_empty = s_full + 7;            // O read by the softmax warps (per unit)
+  uint64_t* fin = s_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 9);
+  float* red_max = reinterpret_cast<float*>(sKV + C::STAGES * C::KVB + C::BARB);  // [2 parities][2 halves][R]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    prefetch_tmap(&tmQ);
     prefetch_tmap(&tmKV);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -169,12 +219,10 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 8);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&p_empty[i], 1);
     }
-    mbar_init(p_full, 8);
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    mbar_init(pv_done, 1);
+    mbar_init(q_full, 8);
     mbar_init(o_empty, 8);
     mbar_init(fin, 1);
     fence_mbar_init();
@@ -195,18 +243,10 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int s = 0;
-      uint32_t ph = 0, uc = 0, qn = 0;
+      uint32_t ph = 0;
       bool ok = true;
-      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++uc) {
-        const int b = static_cast<int>(u / qtiles), q0 = static_cast<int>(u % qtiles) * C::R;
-        if (!mbar_wait(q_empty, (uc & 1u) ^ 1u, status)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(C::QB));
-#pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx) tma_load_3d(&tmQ, q_full, sQ + bx * C::QBOXB, bx * C::BW, q0, b);
-        ++qn;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        const int b = static_cast<int>(u / qtiles);
         for (int j = 0; j < nb; ++j) {
           if (!mbar_wait(&kv_empty[s], ph ^ 1u, status)) {
             ok = false;
@@ -224,29 +264,29 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
       }
       if (!ok) {  // copies already issued must land before the CTA exits
         for (int i = 0; i < C::STAGES; ++i) mbar_drain(&kv_full[i], ph ^ (i < s ? 0u : 1u), status);
-        if (qn > 0) mbar_drain(q_full, (qn - 1) & 1u, status);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
+    // Both products read their A operand from TMEM (Q, then P) and only the key tile from
+    // shared memory. The MMAs of this thread run in issue order, so S_{j+2} is written
+    // into S_j's columns only after P V_j (issued before it) has read P_j from there.
     if (lane == 0) {
       const bool bf = Half16<T>::kBF16;
-      const uint32_t idS = idesc_f16kind_f32(C::R, C::LB, 0, 0, bf);  // S = Q K^T: both K-major
+      const uint32_t idS = idesc_f16kind_f32(C::R, C::LB, 0, 0, bf);  // S = Q K^T: K K-major
       const uint32_t idO = idesc_f16kind_f32(C::R, C::D, 0, 1, bf);   // O += P V: V MN-major
       int ns = 0, cs = 0;  // ring slots of the next S block and of the next P V block
       uint32_t nph = 0, g = 0, uc = 0;
       bool ok = true;
       auto issue_s = [&](uint32_t gb) -> bool {
         if (!mbar_wait(&kv_full[ns], nph, status)) return false;
-        if (!mbar_wait(&s_empty[gb & 1u], ((gb >> 1) & 1u) ^ 1u, status)) return false;
         tc_fence_after();
-        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sKV + ns * C::KVB);
+        const uint32_t ka = smem_u32(sKV + ns * C::KVB);
 #pragma unroll
         for (int ks = 0; ks < C::D / 16; ++ks) {
           const int bx = ks / (C::BW / 16), kin = ks % (C::BW / 16);
-          const uint64_t ad = smem_desc(qa + bx * C::QBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
           const uint64_t bd = smem_desc(ka + bx * C::KVBOXB + kin * 32, 16, 8 * C::SWB, C::SWMODE);
-          umma_f16kind(tmem + (gb & 1u) * C::LB, ad, bd, idS, ks != 0 ? 1u : 0u);
+          whale_umma_ts(tmem + (gb & 1u) * C::LB, tmem + C::QCOL + ks * 8, bd, idS, ks != 0 ? 1u : 0u);
         }
         umma_commit(&s_full[gb & 1u]);
         if (++ns == C::STAGES) {
@@ -267,32 +307,27 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
         }
         for (int j = 0; j < nb; ++j) {
           const uint32_t gj = g + static_cast<uint32_t>(j);
-          if (j + 1 < nb) {
-            if (!issue_s(gj + 1)) {
-              ok = false;
-              break;
-            }
-          } else {
-            umma_commit(q_empty);  // the unit's last S has read Q
+          if (j + 1 < nb && !issue_s(gj + 1)) {
+            ok = false;
+            break;
           }
           if (j == 0 && uc > 0 && !mbar_wait(o_empty, (uc - 1) & 1u, status)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(p_full, gj & 1u, status)) {
+          if (!mbar_wait(&p_full[gj & 1u], (gj >> 1) & 1u, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t pa = smem_u32(sP), va = smem_u32(sKV + cs * C::KVB);
+          const uint32_t va = smem_u32(sKV + cs * C::KVB);
 #pragma unroll
           for (int ks = 0; ks < C::LB / 16; ++ks) {
-            const uint64_t ad = smem_desc(pa + (ks / 4) * C::PBOXB + (ks % 4) * 32, 16, 1024, 2u);
             // MN-major V: BW-column atoms C::KVBOXB apart, 8-key groups 8 * SWB apart
             const uint64_t bd = smem_desc(va + ks * 16 * C::SWB, C::KVBOXB, 8 * C::SWB, C::SWMODE);
-            umma_f16kind(tmem + C::OCOL, ad, bd, idO, (j | ks) != 0 ? 1u : 0u);
+            whale_umma_ts(tmem + C::OCOL, tmem + (gj & 1u) * C::LB + ks * 8, bd, idO, (j | ks) != 0 ? 1u : 0u);
           }
-          umma_commit(pv_done);
+          umma_commit(&p_empty[gj & 1u]);
           umma_commit(&kv_empty[cs]);
           if (++cs == C::STAGES) cs = 0;
         }
@@ -321,6 +356,31 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
       const int b = static_cast<int>(u / qtiles), q0 = static_cast<int>(u % qtiles) * C::R;
       const bool warp_on = q0 + q * 32 < n;  // the pair agrees: same rows
       const bool row_on = q0 + row < n;
+      // The unit's query rows into TMEM (this half's D/2 columns, as 16-bit pairs); every
+      // S product of the previous unit has completed (its last S block was waited for).
+      {
+        uint32_t qv[C::D / 4];
+        if (row_on) {
+          const uint4* src =
+              reinterpret_cast<const uint4*>(Hw + (static_cast<int64_t>(b) * n + q0 + row) * C::D + half * (C::D / 2));
+#pragma unroll
+          for (int i = 0; i < C::D / 16; ++i) {
+            const uint4 v = __ldg(src + i);
+            qv[4 * i] = v.x;
+            qv[4 * i + 1] = v.y;
+            qv[4 * i + 2] = v.z;
+            qv[4 * i + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < C::D / 4; ++i) qv[i] = 0u;
+        }
+        whale_tmem_st_cols<C::D / 4>(tmem + lane_base + C::QCOL + half * (C::D / 4), qv);
+        whale_tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full);
+      }
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nb; ++j) {
         const uint32_t gj = g + static_cast<uint32_t>(j), buf = gj & 1u;
@@ -333,11 +393,40 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
           tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
           tmem_ld_wait();
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[buf]);
         const int kvalid = min(C::LB, L - j * C::LB) - half * (C::LB / 2);  // valid columns of this half
         const bool full = kvalid >= C::LB / 2;
+        // P = 2^(S log2(e)/sqrt(d) - mrow) for this half's columns, rounded to the operand
+        // type and packed in registers; one weight in four from the polynomial.
+        uint32_t pk[C::LB / 4];
+        float lsum = 0.f;
+        auto weights = [&](float mrow, auto full_block) {
+          constexpr bool kFull = decltype(full_block)::value;  // no column masks on a full block
+          const float nm = row_on ? -mrow : 0.f;
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c2 = 0; c2 < C::LB / 4; ++c2) {
+            const float x0 = fmaf(__uint_as_float(sr[2 * c2]), scale_log2, nm);
+            const float x1 = fmaf(__uint_as_float(sr[2 * c2 + 1]), scale_log2, nm);
+            float p0 = whale_ex2(x0);
+            float p1 = (c2 & 1) ? whale_ex2_poly(x1) : whale_ex2(x1);
+            if constexpr (!kFull) {
+              if (2 * c2 >= kvalid) p0 = 0.f;
+              if (2 * c2 + 1 >= kvalid) p1 = 0.f;
+            }
+            s4[(2 * c2) & 3] += p0;
+            s4[(2 * c2 + 1) & 3] += p1;
+            pk[c2] = Half16<T>::pack2(p0, p1);
+          }
+          lsum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        };
+        // From the second block of a row on, the weights are computed with the running max
+        // m at once, next to this block's max; they are recomputed only when the block's
+        // max exceeds m by more than 8 (then m is raised and O rescaled).
+        const bool spec = j > 0;
+        if (warp_on && spec) {
+          if (full) weights(m, std::true_type{});
+          else weights(m, std::false_type{});
+        }
         float mh = -INFINITY;
         if (full) {
           mh = whale_max64(sr);
@@ -347,35 +436,27 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
             if (c < kvalid) mh = fmaxf(mh, __uint_as_float(sr[c]));
         }
         red_max[(buf * 2 + half) * C::R + row] = mh;
+        // after this barrier both warps of the pair have read S_j: P_j may overwrite it
+        tc_fence_before();
         named_bar(bar_id, 64);
+        tc_fence_after();
         const float mb = fmaxf(mh, red_max[(buf * 2 + (half ^ 1)) * C::R + row]);
         const float mb2 = mb * scale_log2;
         const bool need = warp_on && row_on && (mb2 > m + 8.f);
         const float mnew = need ? mb2 : m;
         const float factor = need ? whale_ex2(m - mnew) : 1.f;
-        // P = 2^(S log2(e)/sqrt(d) - m), rounded to the operand type, in registers
-        uint32_t pk[C::LB / 4];
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-        if (warp_on) {
-          const float nm = row_on ? -mnew : 0.f;
-#pragma unroll
-          for (int c2 = 0; c2 < C::LB / 4; ++c2) {
-            float p0 = whale_ex2(fmaf(__uint_as_float(sr[2 * c2]), scale_log2, nm));
-            float p1 = whale_ex2(fmaf(__uint_as_float(sr[2 * c2 + 1]), scale_log2, nm));
-            if (!full) {
-              if (2 * c2 >= kvalid) p0 = 0.f;
-              if (2 * c2 + 1 >= kvalid) p1 = 0.f;
-            }
-            ls[(2 * c2) & 3] += p0;
-            ls[(2 * c2 + 1) & 3] += p1;
-            pk[c2] = Half16<T>::pack2(p0, p1);
-          }
+        const bool redo = warp_on && (!spec || __any_sync(0xffffffffu, need));
+        if (redo) {
+          if (full) weights(mnew, std::true_type{});
+          else weights(mnew, std::false_type{});
         }
-        // P V of the previous block has finished: the P buffer is free and O holds
-        // every earlier block.
-        if (gj > 0 && ok) ok = mbar_wait(pv_done, (gj - 1) & 1u, status);
-        tc_fence_after();
-        if (warp_on && j > 0 && __any_sync(0xffffffffu, need)) {
+        // P V two blocks back has completed (keeps this waiter within one phase of p_empty)
+        if (ok) ok = mbar_wait(&p_empty[buf], ((gj >> 1) & 1u) ^ 1u, status);
+        if (spec && redo) {
+          // the running max was raised: O must hold every earlier block before it is rescaled
+          const uint32_t gp = gj - 1u;
+          if (ok) ok = mbar_wait(&p_empty[gp & 1u], (gp >> 1) & 1u, status);
+          tc_fence_after();
 #pragma unroll 1
           for (int cc = half; cc < C::D / 32; cc += 2) {
             uint32_t o[32];
@@ -385,29 +466,26 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
             whale_tmem_st32(tmem + lane_base + C::OCOL + cc * 32, o);
           }
-          whale_tmem_st_wait();
         }
-        l = l * factor + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        l = l * factor + lsum;
         m = mnew;
-        if (warp_on) {
-          const uint32_t pb = smem_u32(sP) + half * C::PBOXB;
-#pragma unroll
-          for (int c8 = 0; c8 < C::LB / 16; ++c8)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + whale_swz<128>(row, c8)),
-                         "r"(pk[4 * c8]), "r"(pk[4 * c8 + 1]), "r"(pk[4 * c8 + 2]), "r"(pk[4 * c8 + 3])
-                         : "memory");
-        }
-        fence_proxy_async_smem();  // the tensor core reads P
+        // P_j over the first 64 columns of S_j: keys 64 half .. + 63 in columns 32 half .. + 31
+        if (warp_on) whale_tmem_st32(tmem + lane_base + buf * C::LB + half * 32, pk);
+        whale_tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[buf]);
       }
-      // the unit's output rows: O / (l of both halves)
+      // the unit's output rows: O / (l of both halves). The row sums go through the max
+      // exchange slot of the parity the last block did not use; the second pair barrier
+      // keeps the next unit from overwriting it before the partner has read it.
+      const uint32_t gl = g + static_cast<uint32_t>(nb) - 1u;
+      float* red_sum = red_max + ((gl + 1u) & 1u) * 2 * C::R;
       red_sum[half * C::R + row] = l;
       named_bar(bar_id, 64);
       const float lt = l + red_sum[(half ^ 1) * C::R + row];
-      const uint32_t gl = g + static_cast<uint32_t>(nb) - 1u;
-      if (ok) ok = mbar_wait(pv_done, gl & 1u, status);
+      named_bar(bar_id, 64);
+      if (ok) ok = mbar_wait(&p_empty[gl & 1u], (gl >> 1) & 1u, status);
       tc_fence_after();
       if (warp_on) {
         const float inv = row_on ? 1.f / lt : 0.f;
@@ -423,8 +501,6 @@ __global__ void __launch_bounds__(WA_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty);
-      // red_sum is written again only after the next unit's first pair barrier, which
-      // the partner reaches after reading it
       g += static_cast<uint32_t>(nb);
     }
   }

@@ -2236,7 +2236,7 @@ namespace {
 bool whale_d_ok(int d) { return d == 32 || d == 64 || d == 128 || d == 160; }
 
 // [batch, rows, d] as a 3-D map (d, rows, batch) with boxes (bw, 128, 1): rows past
-// `rows` of an example read as zeros.
+// `rows` of an example read as zeros (the last key block of a ragged L).
 template <typename T>
 bool whale_map3(const DevInfo* dv, CUtensorMap* m, const void* base, int d, int rows, int64_t batch, int bw) {
   const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)};
@@ -2261,16 +2261,16 @@ template <int D, typename T>
 wk_status whale_attn_run(const DevInfo* dv, const void* Hw, const void* Hs, void* A, int64_t batch, int n, int L,
                          unsigned* status, cudaStream_t st) {
   using C = WaCfg<D>;
-  CUtensorMap tq, tkv;
-  if (!whale_map3<T>(dv, &tq, Hw, D, n, batch, C::BW) || !whale_map3<T>(dv, &tkv, Hs, D, L, batch, C::BW))
-    return WK_ERR_UNSUPPORTED;
+  CUtensorMap tkv;
+  if (!whale_map3<T>(dv, &tkv, Hs, D, L, batch, C::BW)) return WK_ERR_UNSUPPORTED;
   auto fn = whale_attn_kernel<C, T>;
   const wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fn), C::SMEM);
   if (s != WK_OK) return s;
   const int64_t units = batch * ((n + C::R - 1) / C::R);
   const int grid = static_cast<int>(std::min<int64_t>(units, dv->sms));
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  fn<<<grid, WA_THREADS, C::SMEM, st>>>(tq, tkv, static_cast<T*>(A), batch, n, L, scale_log2, status);
+  fn<<<grid, WA_THREADS, C::SMEM, st>>>(tkv, static_cast<const T*>(Hw), static_cast<T*>(A), batch, n, L, scale_log2,
+                                        status);
   return launch_status();
 }
 

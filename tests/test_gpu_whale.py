@@ -120,3 +120,34 @@ def test_whale_forward_workloads(name, sample):
     assert wk.wk_whale_sync_status(h) == wk.WK_OK
     assert torch.equal(Hf2[:half], Hf[:half])
     wk.wk_whale_destroy(h)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_attention_planted_key(dt):
+    """A key in the last block scores far above every earlier key for query 0 (about 10 sqrt(d)
+    per unit of |q|^2 / d): the kernel's weights from the running max are discarded and
+    recomputed, and query 0 attends to that key alone."""
+    batch, n, L, d = 3, 130, 700, 128
+    Hw = host_normal((batch, n, d), 121, dtype="f32")
+    Hs = host_normal((batch, L, d), 122, dtype="f32")
+    Hs[:, L - 5, :] = 10.0 * Hw[:, 0, :]
+    cast = (lambda a: a.astype(np.float16)) if dt == "f16" else (lambda a: _to_bf16_bits(a))
+    Hw16, Hs16 = cast(Hw), cast(Hs)
+    A = torch.full((batch, n, d), float("nan"), dtype=torch_dtype(dt), device="cuda")
+    wk.wk_whale_attention(to_dev(Hw16), to_dev(Hs16), A, batch, n, L, d, dt)
+    _status_ok()
+    got = f64(A)
+    hw, hs = f64(Hw16), f64(Hs16)
+    ref = np.stack([oracle.attention_shared_kv(hw[b], hs[b]) for b in range(batch)])
+    assert np.isfinite(got).all()
+    assert np.allclose(ref[:, 0, :], hs[:, L - 5, :], rtol=0, atol=1e-9)  # the oracle: one-hot on that key
+    err = max_scaled_err(got, ref)
+    print("planted key", dt, "max scaled err %.2e" % err)
+    assert err <= TOL
+
+
+def _to_bf16_bits(a):
+    """float32 -> bf16 bit patterns, round to nearest even."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return r.astype(np.uint16)
