@@ -29,7 +29,8 @@
 // the FFN then runs in chunks of 64 columns of h: U_c = LN(Z) W_up_c^T into TMEM, the
 // epilogue writes G_c = U_c^2 / (1 + exp(-U_c)) to shared memory, and the down
 // projection accumulates G_c W_down_c^T onto Z's own TMEM columns, so the residual costs
-// nothing. H_f = that sum + b_F. Weights stream through a TMA ring from L2.
+// nothing. H_f = that sum + b_F, staged in shared memory and written with TMA stores.
+// Weights stream through a TMA ring from L2.
 //
 // Every mbarrier wait is bounded (common.cuh); on a failed wait the threads stop waiting,
 // let issued copies land, let issued MMAs finish and free TMEM before the CTA exits.
@@ -533,7 +534,9 @@ struct WfCfg {
   static constexpr int WS = 128 * D;                     // one weight chunk (D x 64 or 64 x D, 16-bit)
   static constexpr int NKC = 2 * D / 64;                 // W_F chunks of 64 input columns
   static constexpr int LIMIT = 227 * 1024;
-  static constexpr int FIXED = 1024 + CB + ZNB + 2 * GB + 512;
+  static constexpr int REDB = 4 * R * 4;                 // epilogue pair exchange [sum | squares][2 halves][R]
+  static constexpr int PRMB = 3 * D * 4;                 // b_F, gamma, beta staged once per CTA
+  static constexpr int FIXED = 1024 + CB + ZNB + 2 * GB + 512 + REDB + PRMB;
   static constexpr int STAGES_RAW = (LIMIT - FIXED) / WS;
   static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
   static constexpr int SMEM = FIXED + STAGES * WS > 120 * 1024 ? FIXED + STAGES * WS : 120 * 1024;
@@ -545,14 +548,14 @@ struct WfCfg {
   static_assert(WDBOXB % 512 == 0 && WUBOXB % 512 == 0, "swizzle atoms stay aligned");
 };
 
-constexpr int WF_THREADS = 192;
+constexpr int WF_THREADS = 320;  // producer, MMA issuer, 8 epilogue warps
 
 template <class C, typename T>
 __global__ void __launch_bounds__(WF_THREADS, 1)
     whale_ffn_kernel(const __grid_constant__ CUtensorMap tmHw, const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmWF, const __grid_constant__ CUtensorMap tmWU,
-                     const __grid_constant__ CUtensorMap tmWD, const float* __restrict__ bF,
-                     const float* __restrict__ gamma, const float* __restrict__ beta, T* __restrict__ Hf,
+                     const __grid_constant__ CUtensorMap tmWD, const __grid_constant__ CUtensorMap tmHf,
+                     const float* __restrict__ bF, const float* __restrict__ gamma, const float* __restrict__ beta,
                      int64_t rows, int h, float eps, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -576,6 +579,8 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
   uint64_t* zn_empty = z_full + 17;
   uint64_t* fin = z_full + 18;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(z_full + 19);
+  float* red = reinterpret_cast<float*>(sW + C::STAGES * C::WS + 512);
+  float* prm = red + 4 * C::R;  // [3][D]: b_F (or 0), gamma, beta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -585,6 +590,7 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
     prefetch_tmap(&tmWF);
     prefetch_tmap(&tmWU);
     prefetch_tmap(&tmWD);
+    prefetch_tmap(&tmHf);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], 1);
@@ -592,15 +598,15 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&z_full[i], 1);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 4);
+      mbar_init(&o_empty[i], 8);
       mbar_init(&u_full[i], 1);
-      mbar_init(&u_empty[i], 4);
-      mbar_init(&g_full[i], 4);
+      mbar_init(&u_empty[i], 8);
+      mbar_init(&g_full[i], 8);
       mbar_init(&g_empty[i], 1);
     }
     mbar_init(c_full, 1);
     mbar_init(c_empty, 1);
-    mbar_init(zn_full, 4);
+    mbar_init(zn_full, 8);
     mbar_init(zn_empty, 1);
     mbar_init(fin, 1);
     fence_mbar_init();
@@ -761,45 +767,65 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Two warps per TMEM lane quarter (rows 32 (warp % 4) .. + 31): for Z and the output
+    // the 32-column chunks alternate between them (LayerNorm partial sums exchanged through
+    // shared memory under a 64-thread named barrier); of each 64-column gated chunk, warp
+    // `half` takes columns 32 half .. + 31.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const int bar_id = 1 + q;
     const float inv_d = 1.0f / static_cast<float>(C::D);
+    const int et = threadIdx.x - 64;           // 0..255 among the epilogue threads
+    const bool store_thread = et == 0;         // issues the output tile's TMA stores
+    for (int i = et; i < 3 * C::D; i += 256)
+      prm[i] = i < C::D ? whale_bias(bF, i) : (i < 2 * C::D ? __ldg(&gamma[i - C::D]) : __ldg(&beta[i - 2 * C::D]));
+    named_bar(5, 256);
+    const float* pb = prm;                      // b_F
+    const float* pg = prm + C::D;               // gamma
+    const float* pbeta = prm + 2 * C::D;        // beta
     uint32_t tl = 0, uc = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
       const uint32_t zb = tl & 1u, zc = zb * C::D;
-      const int64_t grow = t * C::R + row;
       if (ok) ok = mbar_wait(&z_full[zb], (tl >> 1) & 1u, status);
       tc_fence_after();
       // LayerNorm of Z + b_F over d: two passes over TMEM (mean, then centred squares)
       float sum = 0.f;
 #pragma unroll 1
-      for (int cc = 0; cc < C::D / 32; ++cc) {
+      for (int cc = half; cc < C::D / 32; cc += 2) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + zc + cc * 32, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sum += __uint_as_float(r[i]) + whale_bias(bF, cc * 32 + i);
+        for (int i = 0; i < 32; ++i) sum += __uint_as_float(r[i]) + pb[cc * 32 + i];
       }
-      const float mean = sum * inv_d;
+      red[half * C::R + row] = sum;
+      named_bar(bar_id, 64);
+      const float mean = (sum + red[(half ^ 1) * C::R + row]) * inv_d;
       float sq = 0.f;
 #pragma unroll 1
-      for (int cc = 0; cc < C::D / 32; ++cc) {
+      for (int cc = half; cc < C::D / 32; cc += 2) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + zc + cc * 32, r);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float v = __uint_as_float(r[i]) + whale_bias(bF, cc * 32 + i) - mean;
+          const float v = __uint_as_float(r[i]) + pb[cc * 32 + i] - mean;
           sq += v * v;
         }
       }
-      const float rstd = rsqrtf(sq * inv_d + eps);
+      red[(2 + half) * C::R + row] = sq;
+      named_bar(bar_id, 64);
+      const float rstd = rsqrtf((sq + red[(2 + (half ^ 1)) * C::R + row]) * inv_d + eps);
+      // the previous tile's output, staged in the LN(Z) buffer, has been read by its TMA stores
+      if (store_thread) bulk_wait_read<0>();
+      named_bar(5, 256);
       if (ok) ok = mbar_wait(zn_empty, (tl & 1u) ^ 1u, status);
       const uint32_t za = smem_u32(sZn);
 #pragma unroll 1
-      for (int cc = 0; cc < C::D / 32; ++cc) {
+      for (int cc = half; cc < C::D / 32; cc += 2) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + zc + cc * 32, r);
         tmem_ld_wait();
@@ -809,11 +835,8 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int c0 = cc * 32 + j * 8 + 2 * i;
-            const float a = (__uint_as_float(r[j * 8 + 2 * i]) + whale_bias(bF, c0) - mean) * rstd * __ldg(&gamma[c0]) +
-                            __ldg(&beta[c0]);
-            const float b = (__uint_as_float(r[j * 8 + 2 * i + 1]) + whale_bias(bF, c0 + 1) - mean) * rstd *
-                                __ldg(&gamma[c0 + 1]) +
-                            __ldg(&beta[c0 + 1]);
+            const float a = (__uint_as_float(r[j * 8 + 2 * i]) + pb[c0] - mean) * rstd * pg[c0] + pbeta[c0];
+            const float b = (__uint_as_float(r[j * 8 + 2 * i + 1]) + pb[c0 + 1] - mean) * rstd * pg[c0 + 1] + pbeta[c0 + 1];
             p[i] = Half16<T>::pack2(a, b);
           }
           const int col = cc * 32 + j * 8;  // first of 8 columns = one 16-byte unit
@@ -827,14 +850,13 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(zn_full);
-      // gated chunks: G = U * SiLU(U) = U^2 / (1 + 2^(-U log2 e))
+      // gated chunks: G = U * SiLU(U) = U^2 / (1 + 2^(-U log2 e)), this warp's 32 columns
       for (int c = 0; c < nh; ++c, ++uc) {
         const uint32_t ub = uc & 1u, up = (uc >> 1) & 1u;
         if (ok) ok = mbar_wait(&u_full[ub], up, status);
         tc_fence_after();
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + lane_base + C::UCOL + ub * C::HC, r0);
-        tmem_ld32(tmem + lane_base + C::UCOL + ub * C::HC + 32, r1);
+        uint32_t r0[32];
+        tmem_ld32(tmem + lane_base + C::UCOL + ub * C::HC + half * 32, r0);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -842,17 +864,16 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
         if (ok) ok = mbar_wait(&g_empty[ub], up ^ 1u, status);
         const uint32_t ga = smem_u32(sG + ub * C::GB);
 #pragma unroll
-        for (int j = 0; j < C::HC / 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           uint32_t p[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int e = j * 8 + 2 * i;
-            const float va = __uint_as_float(e < 32 ? r0[e] : r1[e - 32]);
-            const float vb = __uint_as_float(e + 1 < 32 ? r0[e + 1] : r1[e + 1 - 32]);
+            const float va = __uint_as_float(r0[j * 8 + 2 * i]);
+            const float vb = __uint_as_float(r0[j * 8 + 2 * i + 1]);
             p[i] = Half16<T>::pack2(__fdividef(va * va, 1.f + whale_ex2(-1.4426950408889634f * va)),
                                     __fdividef(vb * vb, 1.f + whale_ex2(-1.4426950408889634f * vb)));
           }
-          const int col = j * 8;
+          const int col = half * 32 + j * 8;
           const uint32_t a = ga + (col / C::BW) * C::TBOXB + whale_swz<C::SWB>(row, (col % C::BW) / 8);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(p[0]), "r"(p[1]), "r"(p[2]),
                        "r"(p[3])
@@ -863,23 +884,44 @@ __global__ void __launch_bounds__(WF_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&g_full[ub]);
       }
-      // H_f = Z + G W_down^T (accumulated in TMEM) + b_F
+      // H_f = Z + G W_down^T (accumulated in TMEM) + b_F, staged in the LN(Z) buffer (every
+      // MMA of the tile has completed) and written with TMA stores (rows past `rows` clipped)
       if (ok) ok = mbar_wait(&o_full[zb], (tl >> 1) & 1u, status);
       tc_fence_after();
 #pragma unroll 1
-      for (int cc = 0; cc < C::D / 32; ++cc) {
+      for (int cc = half; cc < C::D / 32; cc += 2) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + zc + cc * 32, r);
         tmem_ld_wait();
-        float bias[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) bias[i] = whale_bias(bF, cc * 32 + i);
-        if (grow < rows && ok) whale_st_row32<T>(Hf + grow * C::D + cc * 32, r, 1.f, bias);
+        for (int j = 0; j < 4; ++j) {
+          uint32_t p[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c0 = cc * 32 + j * 8 + 2 * i;
+            p[i] = Half16<T>::pack2(__uint_as_float(r[j * 8 + 2 * i]) + pb[c0],
+                                    __uint_as_float(r[j * 8 + 2 * i + 1]) + pb[c0 + 1]);
+          }
+          const int col = cc * 32 + j * 8;
+          const uint32_t a = za + (col / C::BW) * C::TBOXB + whale_swz<C::SWB>(row, (col % C::BW) / 8);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(p[0]), "r"(p[1]), "r"(p[2]),
+                       "r"(p[3])
+                       : "memory");
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[zb]);
+      fence_proxy_async_smem();  // the TMA store reads the staged tile
+      named_bar(5, 256);
+      if (store_thread && ok) {
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_store_2d(&tmHf, sZn + bx * C::TBOXB, bx * C::BW, static_cast<int32_t>(t * C::R));
+        bulk_commit();
+      }
     }
+    if (store_thread) bulk_wait<0>();  // the stores have completed before the CTA exits
   }
   tc_fence_before();
   __syncthreads();

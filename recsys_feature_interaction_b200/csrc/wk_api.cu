@@ -2278,18 +2278,18 @@ template <int D, typename T>
 wk_status whale_ffn_run(const DevInfo* dv, const void* Hw, const void* A, const wk_whale_weights& w, void* Hf,
                         int64_t rows, int h, float eps, unsigned* status, cudaStream_t st) {
   using C = WfCfg<D>;
-  CUtensorMap thw, ta, twf, twu, twd;
+  CUtensorMap thw, ta, twf, twu, twd, thf;
   if (!whale_map2<T>(dv, &thw, Hw, D, rows, C::BW, C::R) || !whale_map2<T>(dv, &ta, A, D, rows, C::BW, C::R) ||
       !whale_map2<T>(dv, &twf, w.W_F, 2 * D, D, C::BW, D) || !whale_map2<T>(dv, &twu, w.W_up, D, h, C::BW, C::HC) ||
-      !whale_map2<T>(dv, &twd, w.W_down, h, D, C::BW, D))
+      !whale_map2<T>(dv, &twd, w.W_down, h, D, C::BW, D) || !whale_map2<T>(dv, &thf, Hf, D, rows, C::BW, C::R))
     return WK_ERR_UNSUPPORTED;
   auto fn = whale_ffn_kernel<C, T>;
   const wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fn), C::SMEM);
   if (s != WK_OK) return s;
   const int64_t tiles = (rows + C::R - 1) / C::R;
   const int grid = static_cast<int>(std::min<int64_t>(tiles, dv->sms));
-  fn<<<grid, WF_THREADS, C::SMEM, st>>>(thw, ta, twf, twu, twd, w.b_F, w.ln_gamma, w.ln_beta, static_cast<T*>(Hf),
-                                        rows, h, eps, status);
+  fn<<<grid, WF_THREADS, C::SMEM, st>>>(thw, ta, twf, twu, twd, thf, w.b_F, w.ln_gamma, w.ln_beta, rows, h, eps,
+                                        status);
   return launch_status();
 }
 
