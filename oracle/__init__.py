@@ -7,7 +7,9 @@ Wukong page) and streams a stack one layer at a time, so that a large workload
 needs only one layer's weights in host memory.
 
 Parity status: pinned by identities (tests/test_oracle_pins.py); the page prints
-no worked example of a whole layer.
+no worked example of a whole layer. The backward pass (layer_backward, numpy float64,
+derived from the forward by the chain rule) is pinned by finite differences of the
+forward (tests/test_oracle_backward_pins.py).
 """
 import ctypes
 import os
@@ -278,3 +280,87 @@ def fusion_ffn(Hw, A, w, ln_eps=1e-5):
     U = linear(Zn, w["W_up"])
     G = U * U / (1.0 + np.exp(-U))
     return Z + linear(G, w["W_down"])
+
+
+# ------------------------------------------------------------ backward pass
+#
+# The gradients of one Wukong layer (the forward of layer_forward: Wukong page, section
+# 2.2), derived from that forward by the chain rule; the pages give no backward. Written
+# in the plain association of the forward (the FM through P = X X^T, F = P Y), every step
+# in float64, vectorised over the examples with einsum. Weight gradients are summed over
+# the examples. The ReLU derivative is 1 where the pre-activation is > 0, else 0.
+
+
+def layer_forward_np(cfg, w, X, ln_eps=1e-5):
+    """The layer forward in numpy float64 (the same function as layer_forward's C code),
+    returning the output and the intermediates the backward reads."""
+    X = _c64(X)
+    E, n, d = X.shape
+    k, n_f = cfg["k"], cfg["n_f"]
+    m = len(cfg["hidden"]) + 1
+    Y = _weight_f64(w["Y"])
+    Ws = [_weight_f64(w["W%d" % j]) for j in range(m)]
+    bs = [np.zeros(Ws[j].shape[0]) if w.get("b%d" % j) is None else _c64(w["b%d" % j]) for j in range(m)]
+    g1, b1 = _c64(w["fmb_gamma"]), _c64(w["fmb_beta"])
+    W_L = _weight_f64(w["W_L"])
+    g2, b2 = _c64(w["out_gamma"]), _c64(w["out_beta"])
+    P = np.einsum("eit,ejt->eij", X, X)
+    F = np.einsum("eij,jc->eic", P, Y)
+    f = F.reshape(E, n * k)
+    mu = f.mean(axis=1, keepdims=True)
+    rs = 1.0 / np.sqrt(((f - mu) ** 2).mean(axis=1, keepdims=True) + ln_eps)
+    fh = (f - mu) * rs
+    hs, zs = [fh * g1 + b1], []
+    for j in range(m):
+        z = hs[-1] @ Ws[j].T + bs[j]
+        zs.append(z)
+        hs.append(np.maximum(z, 0.0) if j < m - 1 else z)
+    G = np.einsum("ri,eit->ert", W_L, X)
+    y = np.concatenate([hs[-1].reshape(E, n_f, d), G], axis=1) + X
+    mu2 = y.mean(axis=2, keepdims=True)
+    rs2 = 1.0 / np.sqrt(((y - mu2) ** 2).mean(axis=2, keepdims=True) + ln_eps)
+    yh = (y - mu2) * rs2
+    out = yh * g2 + b2
+    return out, dict(X=X, P=P, fh=fh, rs=rs, hs=hs, zs=zs, yh=yh, rs2=rs2, Y=Y, Ws=Ws, g1=g1, W_L=W_L, g2=g2)
+
+
+def layernorm_backward(dxh, xh, rs):
+    """d/dx of the normalisation xh = (x - mean) * rs over the last axis, given d/dxh."""
+    return rs * (dxh - dxh.mean(axis=-1, keepdims=True) - xh * (dxh * xh).mean(axis=-1, keepdims=True))
+
+
+def layer_backward(cfg, w, X, dOut, ln_eps=1e-5):
+    """(dX [E, n, d], grads) of one layer at X for the upstream gradient dOut = dL/d(output).
+    grads: Y, W0.., b0.., fmb_gamma, fmb_beta, W_L, out_gamma, out_beta (float64, summed
+    over the E examples). Weights as for layer_forward (float32 or bf16 bits)."""
+    _, c = layer_forward_np(cfg, w, X, ln_eps)
+    dOut = _c64(dOut)
+    E, n, d = c["X"].shape
+    k, n_f = cfg["k"], cfg["n_f"]
+    m = len(c["Ws"])
+    g = {}
+    # output LayerNorm per embedding row, residual, concat
+    g["out_gamma"] = (dOut * c["yh"]).sum(axis=(0, 1))
+    g["out_beta"] = dOut.sum(axis=(0, 1))
+    dy = layernorm_backward(dOut * c["g2"], c["yh"], c["rs2"])
+    dX = dy.copy()
+    # LCB: G = W_L X
+    dG = dy[:, n_f:, :]
+    g["W_L"] = np.einsum("ert,eit->ri", dG, c["X"])
+    dX += np.einsum("ri,ert->eit", c["W_L"], dG)
+    # FMB MLP, last Linear first
+    dh = dy[:, :n_f, :].reshape(E, n_f * d)
+    for j in range(m - 1, -1, -1):
+        dz = dh * (c["zs"][j] > 0.0) if j < m - 1 else dh
+        g["W%d" % j] = dz.T @ c["hs"][j]
+        g["b%d" % j] = dz.sum(axis=0)
+        dh = dz @ c["Ws"][j]
+    # FMB LayerNorm over the flattened n*k values
+    g["fmb_gamma"] = (dh * c["fh"]).sum(axis=0)
+    g["fmb_beta"] = dh.sum(axis=0)
+    dF = layernorm_backward(dh * c["g1"], c["fh"], c["rs"]).reshape(E, n, k)
+    # FM: F = P Y, P = X X^T (symmetric)
+    g["Y"] = np.einsum("eij,ejc->ic", c["P"], dF)
+    dP = np.einsum("eic,jc->eij", dF, c["Y"])
+    dX += np.einsum("eij,ejt->eit", dP + dP.transpose(0, 2, 1), c["X"])
+    return dX, g
