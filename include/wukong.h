@@ -330,6 +330,38 @@ WK_API wk_status wk_moe_combine(const void* const* concats, const void* X, const
                                 const float* const* betas, void* out, int64_t batch, int32_t n, int32_t d,
                                 int32_t num_experts, wk_dtype dtype, float eps, wk_stream_t stream);
 
+/* ---- backward pass of the stack (training) ----
+ *
+ * The pages train Wukong (Wukong page, section 3.2.1: Adam for the dense parameters)
+ * but give no backward; this is the forward of wk_stack_forward differentiated by the
+ * chain rule. Given the stack's input X and dOut = dL/d(output), it computes dX =
+ * dL/dX and, per layer, the gradients of every parameter of wk_layer_weights (the
+ * caller's W0, b0, gamma1, beta1 as given at create, though the forward runs a folded
+ * first Linear), summed over the batch. */
+typedef struct {           /* fp32 DEVICE buffers the backward overwrites, one set per layer */
+  float* Y;                /* [n, k] */
+  float* const* W;         /* m entries, [h_{j+1}, h_j] (16-byte aligned) */
+  float* const* b;         /* m entries, [h_{j+1}] */
+  float* fmb_ln_gamma, *fmb_ln_beta;   /* [n*k] */
+  float* W_L;              /* [n_l, n] */
+  float* out_ln_gamma, *out_ln_beta;   /* [d] */
+} wk_layer_grads;
+
+/* X [batch, n, d] in the stack's dtype (the input of the forward whose gradient is
+ * wanted); dOut and dX [batch, n, d] fp32; grads: num_layers gradient sets. The forward
+ * is run once with every layer's input saved, then each layer's front is recomputed and
+ * differentiated, last layer first: the output LayerNorm, the residual and the LCB per
+ * row and example; the FMB MLP's input, weight and bias gradients on the tensor-core
+ * GEMM (16-bit operands transposed where the contraction needs them, fp32 weight
+ * gradients); the FMB LayerNorm and the FM per example. Supported: 16-bit stacks with
+ * fp16 operands (the default), at most 3 MLP Linears, batch % 8 == 0, d % 32 == 0 and
+ * d <= 256; otherwise WK_ERR_UNSUPPORTED. The first call (or a larger batch) allocates
+ * the backward workspace (all layer inputs, fp32 gradients of the layer stream, the
+ * MLP gradients and their transposes). Asynchronous on `stream` apart from that
+ * allocation; not re-entrant (shares the forward's workspace). */
+WK_API wk_status wk_stack_backward(wk_stack* h, const void* X, const float* dOut, float* dX,
+                                   const wk_layer_grads* grads, int64_t batch, wk_stream_t stream);
+
 /* ---- WHALE attention-based fusion ----
  *
  * The WHALE pages (gist.science summaries of arXiv 2607.17017, Korean and French),

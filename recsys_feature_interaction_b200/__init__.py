@@ -52,6 +52,13 @@ class WkMoeGate(ctypes.Structure):
     _fields_ = [("W_g", ctypes.c_void_p), ("b_g", ctypes.c_void_p)]
 
 
+class WkLayerGrads(ctypes.Structure):
+    _fields_ = [("Y", ctypes.c_void_p), ("W", ctypes.POINTER(ctypes.c_void_p)),
+                ("b", ctypes.POINTER(ctypes.c_void_p)), ("fmb_ln_gamma", ctypes.c_void_p),
+                ("fmb_ln_beta", ctypes.c_void_p), ("W_L", ctypes.c_void_p), ("out_ln_gamma", ctypes.c_void_p),
+                ("out_ln_beta", ctypes.c_void_p)]
+
+
 class WkWhaleConfig(ctypes.Structure):
     _fields_ = [("n", ctypes.c_int32), ("d", ctypes.c_int32), ("L", ctypes.c_int32), ("h", ctypes.c_int32),
                 ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("max_batch", ctypes.c_int64)]
@@ -97,6 +104,7 @@ def lib():
             "wk_moe_gate_softmax": [vp, vp, vp, vp, i64, i64, i32, ci, vp],
             "wk_moe_combine": [ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, i64, i32, i32,
                                i32, ci, cf, vp],
+            "wk_stack_backward": [vp, vp, vp, vp, ctypes.POINTER(WkLayerGrads), i64, vp],
             "wk_whale_create": [ctypes.POINTER(WkWhaleConfig), ctypes.POINTER(WkWhaleWeights), ctypes.POINTER(vp)],
             "wk_whale_forward": [vp, vp, vp, vp, i64, vp],
             "wk_whale_sync_status": [vp, vp],
@@ -229,6 +237,22 @@ def wk_stack_forward_host(h, X_host, out_host, batch=None, stream=None):
 
 def wk_stack_sync_status(h, stream=None):
     return lib().wk_stack_sync_status(h.ptr, _stream(stream))
+
+
+def wk_stack_backward(h, X, dOut, dX, grads, batch=None, stream=None):
+    """grads: one mapping per layer with fp32 device tensors Y, W (list of m), b (list of m),
+    fmb_gamma, fmb_beta, W_L, out_gamma, out_beta (overwritten with the gradients)."""
+    b = X.shape[0] if batch is None else batch
+    arr = (WkLayerGrads * len(grads))()
+    keep = []
+    for i, g in enumerate(grads):
+        Wp = (ctypes.c_void_p * len(g["W"]))(*[_addr(t) for t in g["W"]])
+        bp = (ctypes.c_void_p * len(g["b"]))(*[_addr(t) for t in g["b"]])
+        keep += [Wp, bp]
+        arr[i] = WkLayerGrads(_addr(g["Y"]), Wp, bp, _addr(g["fmb_gamma"]), _addr(g["fmb_beta"]), _addr(g["W_L"]),
+                              _addr(g["out_gamma"]), _addr(g["out_beta"]))
+    _check(lib().wk_stack_backward(h.ptr, _addr(X), _addr(dOut), _addr(dX), arr, int(b), _stream(stream, X)),
+           "wk_stack_backward")
 
 
 def wk_stack_destroy(h):

@@ -39,6 +39,7 @@
 #include "res_ln_ring.cuh"
 #include "simt.cuh"
 #include "whale.cuh"
+#include "backward.cuh"
 
 using namespace wk;
 
@@ -740,6 +741,12 @@ struct wk_stack {
   };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
+  // backward: the caller's first Linear and FMB LayerNorm parameters (the forward uses
+  // the folded W0', b0'), and the backward workspace (allocated at the first backward)
+  std::vector<const void*> W0_in;
+  std::vector<const float*> b0_in, g1_in, b1_in;
+  uint8_t* bws = nullptr;
+  size_t bws_bytes = 0;
 };
 
 // A stack of Wukong mixture-of-experts layers: one front-only wk_stack per expert
@@ -814,6 +821,7 @@ void free_stack(wk_stack* h) {
   if (h->head_copy) cudaFree(h->head_copy);
   if (h->head_ws) cudaFree(h->head_ws);
   if (h->stage) cudaFree(h->stage);
+  if (h->bws) cudaFree(h->bws);
   if (h->s_in) cudaStreamDestroy(h->s_in);
   if (h->s_out) cudaStreamDestroy(h->s_out);
   for (auto& r : h->recs) {
@@ -1199,6 +1207,246 @@ void free_moe(wk_moe* h) {
   delete h;
 }
 
+// ---------------------------------------------------------------- backward
+
+template <typename TA, typename TB>
+wk_status run_contract(const TA* A, const TB* B, float* C, const BwContr& p, cudaStream_t st) {
+  if (p.M <= 0 || p.N <= 0 || p.Z <= 0) return WK_OK;
+  const dim3 grid((p.M + 63) / 64, (p.N + 63) / 64, p.Z * p.S);
+  bw_contract_kernel<TA, TB><<<grid, 256, 0, st>>>(A, B, C, p);
+  return launch_status();
+}
+
+BwContr contr(int M, int N, int K1, int K2, int Z, int S, int accumulate) {
+  BwContr p{};
+  p.M = M;
+  p.N = N;
+  p.K1 = K1;
+  p.K2 = K2;
+  p.Z = Z;
+  p.S = S;
+  p.accumulate = accumulate;
+  return p;
+}
+
+// Splits of K1 so that a launch has about four CTAs per SM.
+int contr_splits(const DevInfo* dv, int M, int N, int K1) {
+  const int tiles = ((M + 63) / 64) * ((N + 63) / 64);
+  return std::max(1, std::min(K1, (4 * dv->sms + tiles - 1) / tiles));
+}
+
+// C [M, N] = A [M, K] W [N, K]^T on the tensor cores (16-bit K-major operands, TO output).
+template <typename T, typename TO>
+wk_status bw_gemm(wk_stack* h, const void* A, const void* W, void* C, int64_t M, int K, int N, cudaStream_t st) {
+  const DevInfo* dv = h->dv;
+  if (!mlp_tc_ok(M, K, N, N)) return WK_ERR_UNSUPPORTED;
+  const bool pair = use_pair_gemm(M);
+  GemmMaps mp;
+  if (!map_kmajor<T>(dv, &mp.A, A, K, M, GEMM_BM) || !map_kmajor<T>(dv, &mp.B, W, K, N, pair ? 128 : GEMM_BN) ||
+      !map_out<TO>(dv, &mp.C, C, N, M, N))
+    return WK_ERR_UNSUPPORTED;
+  ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+  if (pair) return run_gemm_tc2<T, TO>(dv, mp, mlp2_params(M, K, N, nullptr, 0, h->status), st);
+  return run_gemm_tc<MODE_MLP, T, TO>(dv, mp, mlp_params(M, K, N, nullptr, 0, h->status), st);
+}
+
+template <typename T>
+wk_status bw_transpose(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32));
+  bw_transpose_kernel<T><<<grid, dim3(32, 8), 0, st>>>(static_cast<const T*>(in), static_cast<T*>(out), R, C);
+  return launch_status();
+}
+
+// The backward of a 16-bit stack with fp16 operands (the folded first Linear). X (IO) is
+// the stack's input, dOut / dX fp32 [batch, n, d]. The forward is run once with every
+// layer's input saved; each layer's front is then recomputed from its saved input
+// (A0 = LN(F) normalised, the hidden activations, the concat buffer) before its backward.
+template <typename T, typename IO>
+wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, const wk_layer_grads* gr,
+                     int64_t batch, cudaStream_t st) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers, n_f = c.n_f, n_l = c.n_l;
+  const int64_t B = batch, rows = B * n;
+  const size_t nd = static_cast<size_t>(n) * d, nk = static_cast<size_t>(n) * k;
+  const std::vector<int32_t>& dims = h->dims;
+  int64_t hmax = 0, wmax = 0;
+  for (int j = 0; j <= m; ++j) hmax = std::max<int64_t>(hmax, dims[j]);
+  for (int j = 0; j < m; ++j) wmax = std::max<int64_t>(wmax, static_cast<int64_t>(dims[j]) * dims[j + 1]);
+  auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  // workspace: saved layer inputs, fp32 dy and two dX buffers, two 16-bit MLP gradients,
+  // the transposes, the FM's Z, dZ, F and dF
+  const size_t b_sv = up(B * nd * 2), b_f = up(B * nd * 4), b_h = up(B * hmax * 2), b_w = up(wmax * 2),
+               b_z = up(B * static_cast<size_t>(d) * k * 4), b_fk = up(B * nk * 4);
+  const size_t need = L * b_sv + 3 * b_f + 4 * b_h + b_w + 2 * b_z + 2 * b_fk;
+  if (h->bws_bytes < need) {
+    if (h->bws) cudaFree(h->bws);
+    h->bws = nullptr;
+    h->bws_bytes = 0;
+    if (cudaMalloc(&h->bws, need) != cudaSuccess) {
+      cudaGetLastError();
+      return WK_ERR_OOM;
+    }
+    h->bws_bytes = need;
+  }
+  uint8_t* p = h->bws;
+  std::vector<T*> xs(L);
+  for (int l = 0; l < L; ++l, p += b_sv) xs[l] = reinterpret_cast<T*>(p);
+  float* dyf = reinterpret_cast<float*>(p);
+  p += b_f;
+  float* gx[2] = {reinterpret_cast<float*>(p), reinterpret_cast<float*>(p + b_f)};
+  p += 2 * b_f;
+  T* dz[2] = {reinterpret_cast<T*>(p), reinterpret_cast<T*>(p + b_h)};
+  p += 2 * b_h;
+  T* dzT = reinterpret_cast<T*>(p);
+  p += b_h;
+  T* hT = reinterpret_cast<T*>(p);
+  p += b_h;
+  T* wT = reinterpret_cast<T*>(p);
+  p += b_w;
+  float* Zb = reinterpret_cast<float*>(p);
+  float* dZb = reinterpret_cast<float*>(p + b_z);
+  p += 2 * b_z;
+  float* Fb = reinterpret_cast<float*>(p);
+  float* dFb = reinterpret_cast<float*>(p + b_fk);
+
+  wk_status s = WK_OK;
+  // 1. the forward, saving each layer's input
+  if (sizeof(IO) != sizeof(T) || Half16<IO>::kBF16 != Half16<T>::kBF16)
+    s = run_convert<IO, T>(dv, X, xs[0], rows * d, st);
+  else if (cudaMemcpyAsync(xs[0], X, B * nd * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    s = WK_ERR_CUDA;
+  std::vector<CUtensorMap> lcbx(L);
+  for (int l = 0; l < L && s == WK_OK; ++l)
+    if (h->tc_lcb && !map_lcb_x<T>(dv, &lcbx[l], xs[l], n, d, B)) s = WK_ERR_CUDA;
+  for (int l = 0; l + 1 < L && s == WK_OK; ++l) {
+    s = layer_front16<T>(h, l, xs[l], lcbx[l], B, st);
+    if (s == WK_OK)
+      s = run_res_ln<T, T, T>(dv, static_cast<const T*>(h->cat), xs[l], h->g2[l], h->b2[l], xs[l + 1], rows, d, h->eps,
+                              h->status, st);
+  }
+  // 2. the layers' backwards, last layer first
+  for (int l = L - 1; l >= 0 && s == WK_OK; --l) {
+    const wk_layer_grads& g = gr[l];
+    const T* xin = xs[l];
+    const float* up_grad = (l == L - 1) ? dOut : gx[(l + 1) % 2];
+    float* dxl = (l == 0) ? dX : gx[l % 2];
+    s = layer_front16<T>(h, l, xin, lcbx[l], B, st);
+    if (s != WK_OK) break;
+    cudaMemsetAsync(g.out_ln_gamma, 0, d * 4, st);
+    cudaMemsetAsync(g.out_ln_beta, 0, d * 4, st);
+    cudaMemsetAsync(g.W_L, 0, static_cast<size_t>(n_l) * n * 4, st);
+    cudaMemsetAsync(g.Y, 0, nk * 4, st);
+    cudaMemsetAsync(g.fmb_ln_gamma, 0, nk * 4, st);
+    cudaMemsetAsync(g.fmb_ln_beta, 0, nk * 4, st);
+    for (int j = 0; j < m; ++j) cudaMemsetAsync(g.b[j], 0, static_cast<size_t>(dims[j + 1]) * 4, st);
+    // output LayerNorm, residual: dy, dX = dy, the FMB rows of dy as the MLP's gradient
+    {
+      const int grid = static_cast<int>(std::min<int64_t>((rows + 7) / 8, dv->sms * 8ll));
+      bw_out_ln_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(h->cat), xin, up_grad, h->g2[l], dyf, dxl, dz[0],
+                                                 g.out_ln_gamma, g.out_ln_beta, rows, n, n_f, d, h->eps);
+      s = launch_status();
+    }
+    // LCB: dX_b += W_L^T dG_b; dW_L = sum_b dG_b X_b^T (dG = rows n_f.. of dy)
+    if (s == WK_OK) {
+      BwContr p = contr(n, d, 1, n_l, static_cast<int>(B), 1, 1);
+      p.sAm = 1, p.sAk2 = n;                                                  // W_L(r, i) at r n + i
+      p.sBz = nd, p.sBn = 1, p.sBk2 = d;                                      // dG(b, r, t)
+      p.sCz = nd, p.sCm = d, p.sCn = 1;
+      s = run_contract<T, float>(static_cast<const T*>(h->WL[l]), dyf + static_cast<size_t>(n_f) * d, dxl, p, st);
+    }
+    if (s == WK_OK) {
+      BwContr p = contr(n_l, n, static_cast<int>(B), d, 1, contr_splits(dv, n_l, n, static_cast<int>(B)), 1);
+      p.sAm = d, p.sAk1 = nd, p.sAk2 = 1;                                     // dG(b, r, t)
+      p.sBn = d, p.sBk1 = nd, p.sBk2 = 1;                                     // X(b, i, t)
+      p.sCm = n, p.sCn = 1;
+      s = run_contract<float, T>(dyf + static_cast<size_t>(n_f) * d, xin, g.W_L, p, st);
+    }
+    // FMB MLP, last Linear first: dz (16-bit) -> bias, weight and input gradients
+    int cur = 0;
+    for (int j = m - 1; j >= 0 && s == WK_OK; --j) {
+      const int64_t hin = dims[j], hout = dims[j + 1];
+      const void* hj = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+      if (j < m - 1) {  // the ReLU of Linear j: its output h_{j+1} was > 0
+        const int64_t cnt = B * hout;
+        const int grid = static_cast<int>(std::min<int64_t>((cnt / 8 + 255) / 256, dv->sms * 16ll));
+        bw_relu_mask_kernel<T><<<grid, 256, 0, st>>>(dz[cur], static_cast<const T*>(h->H[j % 2]), cnt);
+        s = launch_status();
+      }
+      if (s == WK_OK) {
+        const dim3 grid(static_cast<unsigned>((hout + 255) / 256), static_cast<unsigned>(std::min<int64_t>(B, 64)));
+        bw_colsum_kernel<T><<<grid, 256, 0, st>>>(dz[cur], g.b[j], B, static_cast<int>(hout));
+        s = launch_status();
+      }
+      // dW_j = dz^T h_j (K = batch): both operands transposed to K-major
+      if (s == WK_OK) s = bw_transpose<T>(dz[cur], dzT, B, hout, st);
+      if (s == WK_OK) s = bw_transpose<T>(hj, hT, B, hin, st);
+      if (s == WK_OK) s = bw_gemm<T, float>(h, dzT, hT, g.W[j], hout, static_cast<int>(B), static_cast<int>(hin), st);
+      // dh_j = dz W_j: W_j^T as the K-major operand
+      if (s == WK_OK) s = bw_transpose<T>(h->W[l][j], wT, hout, hin, st);
+      if (s == WK_OK)
+        s = bw_gemm<T, T>(h, dz[cur], wT, dz[1 - cur], B, static_cast<int>(hout), static_cast<int>(hin), st);
+      cur = 1 - cur;
+    }
+    // the folded first Linear: gradients of the caller's W0, gamma1, beta1 (b0 = b0')
+    if (s == WK_OK) {
+      const dim3 grid(static_cast<unsigned>((dims[0] + 255) / 256), static_cast<unsigned>(std::min(dims[1], 64)));
+      bw_unfold_kernel<IO><<<grid, 256, 0, st>>>(g.W[0], g.b[0], static_cast<const IO*>(h->W0_in[l]), h->g1_in[l],
+                                                 h->b1_in[l], g.fmb_ln_gamma, g.fmb_ln_beta, dims[1], dims[0]);
+      s = launch_status();
+    }
+    // FMB: Z = X^T Y, F = X Z, dF from the LayerNorm backward, then dZ = X^T dF,
+    // dX += dF Z^T + Y dZ^T, dY = sum_b X_b dZ_b
+    if (s == WK_OK) {
+      BwContr p = contr(d, k, 1, n, static_cast<int>(B), 1, 0);
+      p.sAz = nd, p.sAm = 1, p.sAk2 = d;     // X(b, i, t) as (m = t, k = i)
+      p.sBn = 1, p.sBk2 = k;                 // Y(i, c)
+      p.sCz = static_cast<int64_t>(d) * k, p.sCm = k, p.sCn = 1;
+      s = run_contract<T, T>(xin, static_cast<const T*>(h->Y[l]), Zb, p, st);
+    }
+    if (s == WK_OK) {
+      BwContr p = contr(n, k, 1, d, static_cast<int>(B), 1, 0);
+      p.sAz = nd, p.sAm = d, p.sAk2 = 1;     // X(b, i, t)
+      p.sBz = static_cast<int64_t>(d) * k, p.sBn = 1, p.sBk2 = k;  // Z(b, t, c)
+      p.sCz = nk, p.sCm = k, p.sCn = 1;
+      s = run_contract<T, float>(xin, Zb, Fb, p, st);
+    }
+    if (s == WK_OK) {
+      bw_fmb_ln_kernel<T><<<static_cast<unsigned>(B), 256, 0, st>>>(Fb, dz[cur], dFb, static_cast<int>(nk), h->eps);
+      s = launch_status();
+    }
+    if (s == WK_OK) {
+      BwContr p = contr(d, k, 1, n, static_cast<int>(B), 1, 0);
+      p.sAz = nd, p.sAm = 1, p.sAk2 = d;     // X(b, i, t) as (m = t, k = i)
+      p.sBz = nk, p.sBn = 1, p.sBk2 = k;     // dF(b, i, c)
+      p.sCz = static_cast<int64_t>(d) * k, p.sCm = k, p.sCn = 1;
+      s = run_contract<T, float>(xin, dFb, dZb, p, st);
+    }
+    if (s == WK_OK) {
+      BwContr p = contr(n, d, 1, k, static_cast<int>(B), 1, 1);
+      p.sAz = nk, p.sAm = k, p.sAk2 = 1;     // dF(b, i, c)
+      p.sBz = static_cast<int64_t>(d) * k, p.sBn = k, p.sBk2 = 1;  // Z(b, t, c)
+      p.sCz = nd, p.sCm = d, p.sCn = 1;
+      s = run_contract<float, float>(dFb, Zb, dxl, p, st);
+    }
+    if (s == WK_OK) {
+      BwContr p = contr(n, d, 1, k, static_cast<int>(B), 1, 1);
+      p.sAm = k, p.sAk2 = 1;                 // Y(i, c)
+      p.sBz = static_cast<int64_t>(d) * k, p.sBn = k, p.sBk2 = 1;  // dZ(b, t, c)
+      p.sCz = nd, p.sCm = d, p.sCn = 1;
+      s = run_contract<T, float>(static_cast<const T*>(h->Y[l]), dZb, dxl, p, st);
+    }
+    if (s == WK_OK) {
+      BwContr p = contr(n, k, static_cast<int>(B), d, 1, contr_splits(dv, n, k, static_cast<int>(B)), 1);
+      p.sAm = d, p.sAk1 = nd, p.sAk2 = 1;    // X(b, i, t)
+      p.sBn = 1, p.sBk1 = static_cast<int64_t>(d) * k, p.sBk2 = k;  // dZ(b, t, c)
+      p.sCm = k, p.sCn = 1;
+      s = run_contract<T, float>(xin, dZb, g.Y, p, st);
+    }
+  }
+  return s;
+}
+
 wk_status read_status_word(unsigned* word, cudaStream_t st) {
   if (cudaStreamSynchronize(st) != cudaSuccess) {
     cudaGetLastError();
@@ -1441,6 +1689,10 @@ static wk_status stack_create_impl(const wk_stack_config* cfg, const wk_layer_we
     }
     h->g1.push_back(w.fmb_ln_gamma);
     h->b1.push_back(w.fmb_ln_beta);
+    h->W0_in.push_back(w.W[0]);
+    h->b0_in.push_back(w.b ? w.b[0] : nullptr);
+    h->g1_in.push_back(w.fmb_ln_gamma);
+    h->b1_in.push_back(w.fmb_ln_beta);
     h->g2.push_back(w.out_ln_gamma);
     h->b2.push_back(w.out_ln_beta);
   }
@@ -1671,6 +1923,35 @@ wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host,
 wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream) {
   if (!h) return WK_ERR_INVALID_ARG;
   return read_status_word(h->status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+wk_status wk_stack_backward(wk_stack* h, const void* X, const float* dOut, float* dX, const wk_layer_grads* grads,
+                            int64_t batch, wk_stream_t stream) {
+  if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
+  if (batch == 0) return WK_OK;
+  if (!X || !dOut || !dX || !grads || !al16(X) || !al16(dOut) || !al16(dX)) return WK_ERR_INVALID_ARG;
+  const wk_stack_config& c = h->cfg;
+  for (int l = 0; l < c.num_layers; ++l) {
+    const wk_layer_grads& g = grads[l];
+    if (!g.Y || !g.W || !g.b || !g.fmb_ln_gamma || !g.fmb_ln_beta || !g.W_L || !g.out_ln_gamma || !g.out_ln_beta)
+      return WK_ERR_INVALID_ARG;
+    for (int j = 0; j < c.mlp_num_linear; ++j)
+      if (!g.W[j] || !g.b[j] || !al16(g.W[j])) return WK_ERR_INVALID_ARG;
+  }
+  // the fp16-operand path (first Linear folded), at most three Linears (both hidden
+  // activations stay in the workspace), a batch that is a multiple of 8 (the weight
+  // gradients' GEMMs contract over it), embedding rows of at most 256
+  if (h->op != WK_F16 || h->front_only || h->fused || c.mlp_num_linear > 3 || batch % 8 != 0 || c.d > 256 ||
+      c.d % 32 != 0)
+    return WK_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) {
+    cudaGetLastError();
+    return WK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return h->io == WK_BF16 ? backward16<f16, bf16>(h, X, dOut, dX, grads, batch, st)
+                          : backward16<f16, f16>(h, X, dOut, dX, grads, batch, st);
 }
 
 void wk_stack_destroy(wk_stack* h) { free_stack(h); }
