@@ -36,6 +36,8 @@ METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack fwd, 
 ORACLE_SAMPLE = {"c1_fp32": 64, "c2_bf16": 4096, "c3_bf16": 128, "c4_bf16": 16, "c5_bf16": 512, "moe3_c2": 1024,
                  "moe4_c3": 32, "whale_c2": 512, "whale_c4": 32}
 WHALE_METRIC = "examples/sec and achieved TFLOP/s (% of bf16 peak), WHALE attention fusion fwd, 1 B200"
+BACKWARD_METRIC = ("examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong stack training step "
+                   "(forward + backward: gradients of the input and of every parameter), 1 B200")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -351,6 +353,143 @@ def run_whale(args, cfg, rank, world, local, dev):
     wk.wk_whale_destroy(h)
 
 
+def run_backward(args, cfg, rank, world, local, dev):
+    """One step = wk_stack_backward over the per-GPU batch: the forward with every layer's
+    input saved, then each layer's front recomputed and differentiated (dX and all parameter
+    gradients). Algorithmic work: 3x the forward's matmul FLOPs. Roofline: the FMB MLP GEMM
+    (forward save, recompute, input and weight gradients), tensor-bound."""
+    import torch
+
+    import recsys_feature_interaction_b200 as wk
+    from recsys_feature_interaction_b200 import replicas
+    from synth import configs as C
+
+    B, L, n, d, k = cfg["batch"], cfg["layers"], cfg["n"], cfg["d"], cfg["k"]
+    dims = C.mlp_dims(cfg)
+    first, _ = replicas.example_range(rank, world, B)
+    X = C.make_x_dev(cfg, B, device=dev, first_example=first)
+    layers = [C.make_layer_dev(cfg, l, device=dev) for l in range(L)]
+    h = wk.wk_stack_create(cfg, layers, max_batch=B)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    dOut = torch.randn((B, n, d), generator=gen, device=dev, dtype=torch.float32)
+    dX = torch.empty_like(dOut)
+    z = lambda *sh: torch.empty(sh, dtype=torch.float32, device=dev)
+    grads = [{"Y": z(n, k), "W": [z(dims[j + 1], dims[j]) for j in range(len(dims) - 1)],
+              "b": [z(dims[j + 1]) for j in range(len(dims) - 1)], "fmb_gamma": z(n * k), "fmb_beta": z(n * k),
+              "W_L": z(cfg["n_l"], n), "out_gamma": z(d), "out_beta": z(d)} for _ in range(L)]
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+    torch.cuda.synchronize(dev)
+    if wk.wk_stack_sync_status(h) != wk.WK_OK:
+        raise RuntimeError("device status after warm-up")
+    wk.wk_stack_kernel_times(h)  # clear
+    in_bytes = X.numel() * X.element_size() + dOut.numel() * 4
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < (252 << 20) else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps if flush is not None else 1)]
+    wk.wk_stack_set_profiling(h, True)
+    replicas.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        if flush is None:
+            evs[0][0].record(stream)
+            for _ in range(args.steps):
+                wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+            evs[0][1].record(stream)
+        else:
+            for a, b in evs:
+                flush.fill_(1)
+                a.record(stream)
+                wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+                b.record(stream)
+        torch.cuda.synchronize(dev)
+    replicas.barrier()
+    wk.wk_stack_set_profiling(h, False)
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    if wk.wk_stack_sync_status(h) != wk.WK_OK:
+        raise RuntimeError("device status after the timed region")
+    ktimes = wk.wk_stack_kernel_times(h)
+    ms_max = replicas.max_over_ranks(ms, device=dev)
+    value = world * B * args.steps / (ms_max / 1e3)
+
+    # end to end: X and dOut copied in from pinned host memory, dX copied out, every step
+    xh, dh = X.cpu().pin_memory(), dOut.cpu().pin_memory()
+    dxh = torch.empty_like(dX, device="cpu").pin_memory()
+
+    def step_host():
+        X.copy_(xh, non_blocking=True)
+        dOut.copy_(dh, non_blocking=True)
+        wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+        dxh.copy_(dX, non_blocking=True)
+        stream.synchronize()
+    step_host()
+    replicas.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step_host()
+    e2e_value = world * B * args.steps / replicas.max_over_ranks(time.perf_counter() - t0, device=dev)
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        fwd = C.flops_per_example(cfg)
+        flops_ex = 3 * fwd
+        tflops = value * flops_ex / 1e12 / world
+        # executed MLP GEMM work per step: forward save (L-1 layers), recompute (L), and the
+        # input and weight gradients (2 L), each the forward's per-layer MLP FLOPs
+        mlp_layer = gemm_flops_per_example(cfg) / L * B
+        gemm_flops_step = (4 * L - 1) * mlp_layer
+        g_ms, g_n = ktimes["mlp_gemm"]
+        ach = gemm_flops_step * args.steps / (g_ms / 1e3) / 1e12 if g_ms else None
+        peak = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+        roof = {"kernel": "mlp_gemm (tcgen05 pair GEMM: forward, input and weight gradients)", "bound": "tensor",
+                "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": (ach / peak) if ach else None,
+                "traffic": None, "peak_note": "%s sustained cuBLAS bf16" % peak_src,
+                "algorithmic_per_step": {"flops": gemm_flops_step, "launches": g_n / max(1, args.steps)}}
+        l2 = ("L2 flushed (256 MB write) before every step, outside the timed events" if flush is not None else
+              "inputs larger than L2 (X and dOut %.0f MB per GPU)" % (in_bytes / 1e6))
+        line = {
+            "metric": BACKWARD_METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": args.workload + ": " + workload_desc(cfg) + ", training step", "per_gpu_batch": B,
+                       "precision": "bf16 inputs and weights; fp16 tensor-core operands, activations and MLP "
+                                    "gradients; fp32 accumulation, LayerNorm statistics, layer-stream and "
+                                    "parameter gradients",
+                       "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
+                       "l2": l2, "launch": "eager, one C-ABI call per step",
+                       "flops_per_example": "3 x forward matmul FLOPs = %.4g" % flops_ex},
+            "tflops_per_gpu": tflops,
+            "pct_of_bf16_peak": 100.0 * tflops / peak,
+            "peak_source": "%s bf16_tflops_sustained" % peak_src,
+            "roofline": roof,
+            "kernel_ms_per_step": {kk: v[0] / args.steps for kk, v in ktimes.items() if v[1]},
+            "clocks": clk.summary(),
+            "e2e": {"value": e2e_value, "unit": "examples/s", "h2d_bytes_per_step": in_bytes,
+                    "d2h_bytes_per_step": dX.numel() * 4,
+                    "api": "wk_stack_backward with pinned host-to-device copies of X and dOut before and a "
+                           "device-to-host copy of dX after (parameter gradients stay on the device)"},
+            "gpu_launches": sum(v[1] for v in ktimes.values()),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            ns = max(1, min(16, ORACLE_SAMPLE.get(args.workload, 16) // 8))
+            Xh = C.to_f64(C.make_x_host(cfg, list(range(ns))))
+            w = C.make_layer_host(cfg, 0)
+            dO = dOut[:ns].double().cpu().numpy()
+            t0 = time.perf_counter()
+            oracle.layer_backward(cfg, w, Xh, dO)
+            dt = time.perf_counter() - t0
+            from threadpoolctl import threadpool_info
+            thr = max([pp.get("num_threads", 1) for pp in threadpool_info()] or [1])
+            line["cpu_baseline"] = {"value": ns / (dt * L), "unit": "examples/s", "cores": thr, "kind": "oracle",
+                                    "sample": "%d examples through the forward and backward of 1 of the %d layers "
+                                              "(%.1f s, numpy float64), scaled to the stack" % (ns, L, dt)}
+        print(json.dumps(line), flush=True)
+    wk.wk_stack_destroy(h)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -363,6 +502,9 @@ def main():
                          "per-kernel times then come from an eager profiled pass after the timed region")
     ap.add_argument("--head", action="store_true",
                     help="each step also runs the prediction head (wk_stack_predict: logits and probabilities)")
+    ap.add_argument("--backward", action="store_true",
+                    help="each step is a training step: wk_stack_backward (forward with saved layer inputs, "
+                         "then the gradients of the input and of every parameter)")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["c1_fp32", "c2_bf16", "c3_bf16", "c4_bf16", "c5_bf16", "moe3_c2", "moe4_c3",
                              "whale_c2", "whale_c4"])
@@ -391,6 +533,10 @@ def main():
     cfg = workload_cfg(args.workload)
     if "L" in cfg:
         run_whale(args, cfg, rank, world, local, dev)
+        replicas.finish()
+        return
+    if args.backward:
+        run_backward(args, cfg, rank, world, local, dev)
         replicas.finish()
         return
     moe = "experts" in cfg

@@ -174,7 +174,7 @@ WK_API void wk_graph_destroy(wk_graph* g);
 typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
                WK_KERNEL_CONVERT = 4, WK_KERNEL_MOE_GATE = 5, WK_KERNEL_MOE_COMBINE = 6,
                WK_KERNEL_HEAD = 7, WK_KERNEL_WHALE_ATTN = 8, WK_KERNEL_WHALE_FFN = 9,
-               WK_KERNEL_COUNT = 10 } wk_kernel_kind;
+               WK_KERNEL_BW_CONTRACT = 10, WK_KERNEL_BW_ROWS = 11, WK_KERNEL_COUNT = 12 } wk_kernel_kind;
 
 /* enable != 0: every later forward records a start/stop event pair around each
  * kernel launch on its stream (adds no synchronisation). */

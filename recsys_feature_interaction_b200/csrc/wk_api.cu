@@ -1210,8 +1210,9 @@ void free_moe(wk_moe* h) {
 // ---------------------------------------------------------------- backward
 
 template <typename TA, typename TB>
-wk_status run_contract(const TA* A, const TB* B, float* C, const BwContr& p, cudaStream_t st) {
+wk_status run_contract(wk_stack* h, const TA* A, const TB* B, float* C, const BwContr& p, cudaStream_t st) {
   if (p.M <= 0 || p.N <= 0 || p.Z <= 0) return WK_OK;
+  ProfScope ps(h, WK_KERNEL_BW_CONTRACT, st);
   const dim3 grid((p.M + 63) / 64, (p.N + 63) / 64, p.Z * p.S);
   bw_contract_kernel<TA, TB><<<grid, 256, 0, st>>>(A, B, C, p);
   return launch_status();
@@ -1251,7 +1252,8 @@ wk_status bw_gemm(wk_stack* h, const void* A, const void* W, void* C, int64_t M,
 }
 
 template <typename T>
-wk_status bw_transpose(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
+wk_status bw_transpose(wk_stack* h, const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
+  ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
   const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32));
   bw_transpose_kernel<T><<<grid, dim3(32, 8), 0, st>>>(static_cast<const T*>(in), static_cast<T*>(out), R, C);
   return launch_status();
@@ -1343,6 +1345,7 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     // output LayerNorm, residual: dy, dX = dy, the FMB rows of dy as the MLP's gradient
     {
       const int grid = static_cast<int>(std::min<int64_t>((rows + 7) / 8, dv->sms * 8ll));
+      ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
       bw_out_ln_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(h->cat), xin, up_grad, h->g2[l], dyf, dxl, dz[0],
                                                  g.out_ln_gamma, g.out_ln_beta, rows, n, n_f, d, h->eps);
       s = launch_status();
@@ -1353,14 +1356,14 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
       p.sAm = 1, p.sAk2 = n;                                                  // W_L(r, i) at r n + i
       p.sBz = nd, p.sBn = 1, p.sBk2 = d;                                      // dG(b, r, t)
       p.sCz = nd, p.sCm = d, p.sCn = 1;
-      s = run_contract<T, float>(static_cast<const T*>(h->WL[l]), dyf + static_cast<size_t>(n_f) * d, dxl, p, st);
+      s = run_contract<T, float>(h, static_cast<const T*>(h->WL[l]), dyf + static_cast<size_t>(n_f) * d, dxl, p, st);
     }
     if (s == WK_OK) {
       BwContr p = contr(n_l, n, static_cast<int>(B), d, 1, contr_splits(dv, n_l, n, static_cast<int>(B)), 1);
       p.sAm = d, p.sAk1 = nd, p.sAk2 = 1;                                     // dG(b, r, t)
       p.sBn = d, p.sBk1 = nd, p.sBk2 = 1;                                     // X(b, i, t)
       p.sCm = n, p.sCn = 1;
-      s = run_contract<float, T>(dyf + static_cast<size_t>(n_f) * d, xin, g.W_L, p, st);
+      s = run_contract<float, T>(h, dyf + static_cast<size_t>(n_f) * d, xin, g.W_L, p, st);
     }
     // FMB MLP, last Linear first: dz (16-bit) -> bias, weight and input gradients
     int cur = 0;
@@ -1370,20 +1373,22 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
       if (j < m - 1) {  // the ReLU of Linear j: its output h_{j+1} was > 0
         const int64_t cnt = B * hout;
         const int grid = static_cast<int>(std::min<int64_t>((cnt / 8 + 255) / 256, dv->sms * 16ll));
+        ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
         bw_relu_mask_kernel<T><<<grid, 256, 0, st>>>(dz[cur], static_cast<const T*>(h->H[j % 2]), cnt);
         s = launch_status();
       }
       if (s == WK_OK) {
         const dim3 grid(static_cast<unsigned>((hout + 255) / 256), static_cast<unsigned>(std::min<int64_t>(B, 64)));
+        ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
         bw_colsum_kernel<T><<<grid, 256, 0, st>>>(dz[cur], g.b[j], B, static_cast<int>(hout));
         s = launch_status();
       }
       // dW_j = dz^T h_j (K = batch): both operands transposed to K-major
-      if (s == WK_OK) s = bw_transpose<T>(dz[cur], dzT, B, hout, st);
-      if (s == WK_OK) s = bw_transpose<T>(hj, hT, B, hin, st);
+      if (s == WK_OK) s = bw_transpose<T>(h, dz[cur], dzT, B, hout, st);
+      if (s == WK_OK) s = bw_transpose<T>(h, hj, hT, B, hin, st);
       if (s == WK_OK) s = bw_gemm<T, float>(h, dzT, hT, g.W[j], hout, static_cast<int>(B), static_cast<int>(hin), st);
       // dh_j = dz W_j: W_j^T as the K-major operand
-      if (s == WK_OK) s = bw_transpose<T>(h->W[l][j], wT, hout, hin, st);
+      if (s == WK_OK) s = bw_transpose<T>(h, h->W[l][j], wT, hout, hin, st);
       if (s == WK_OK)
         s = bw_gemm<T, T>(h, dz[cur], wT, dz[1 - cur], B, static_cast<int>(hout), static_cast<int>(hin), st);
       cur = 1 - cur;
@@ -1391,6 +1396,7 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     // the folded first Linear: gradients of the caller's W0, gamma1, beta1 (b0 = b0')
     if (s == WK_OK) {
       const dim3 grid(static_cast<unsigned>((dims[0] + 255) / 256), static_cast<unsigned>(std::min(dims[1], 64)));
+      ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
       bw_unfold_kernel<IO><<<grid, 256, 0, st>>>(g.W[0], g.b[0], static_cast<const IO*>(h->W0_in[l]), h->g1_in[l],
                                                  h->b1_in[l], g.fmb_ln_gamma, g.fmb_ln_beta, dims[1], dims[0]);
       s = launch_status();
@@ -1402,16 +1408,17 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
       p.sAz = nd, p.sAm = 1, p.sAk2 = d;     // X(b, i, t) as (m = t, k = i)
       p.sBn = 1, p.sBk2 = k;                 // Y(i, c)
       p.sCz = static_cast<int64_t>(d) * k, p.sCm = k, p.sCn = 1;
-      s = run_contract<T, T>(xin, static_cast<const T*>(h->Y[l]), Zb, p, st);
+      s = run_contract<T, T>(h, xin, static_cast<const T*>(h->Y[l]), Zb, p, st);
     }
     if (s == WK_OK) {
       BwContr p = contr(n, k, 1, d, static_cast<int>(B), 1, 0);
       p.sAz = nd, p.sAm = d, p.sAk2 = 1;     // X(b, i, t)
       p.sBz = static_cast<int64_t>(d) * k, p.sBn = 1, p.sBk2 = k;  // Z(b, t, c)
       p.sCz = nk, p.sCm = k, p.sCn = 1;
-      s = run_contract<T, float>(xin, Zb, Fb, p, st);
+      s = run_contract<T, float>(h, xin, Zb, Fb, p, st);
     }
     if (s == WK_OK) {
+      ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
       bw_fmb_ln_kernel<T><<<static_cast<unsigned>(B), 256, 0, st>>>(Fb, dz[cur], dFb, static_cast<int>(nk), h->eps);
       s = launch_status();
     }
@@ -1420,28 +1427,28 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
       p.sAz = nd, p.sAm = 1, p.sAk2 = d;     // X(b, i, t) as (m = t, k = i)
       p.sBz = nk, p.sBn = 1, p.sBk2 = k;     // dF(b, i, c)
       p.sCz = static_cast<int64_t>(d) * k, p.sCm = k, p.sCn = 1;
-      s = run_contract<T, float>(xin, dFb, dZb, p, st);
+      s = run_contract<T, float>(h, xin, dFb, dZb, p, st);
     }
     if (s == WK_OK) {
       BwContr p = contr(n, d, 1, k, static_cast<int>(B), 1, 1);
       p.sAz = nk, p.sAm = k, p.sAk2 = 1;     // dF(b, i, c)
       p.sBz = static_cast<int64_t>(d) * k, p.sBn = k, p.sBk2 = 1;  // Z(b, t, c)
       p.sCz = nd, p.sCm = d, p.sCn = 1;
-      s = run_contract<float, float>(dFb, Zb, dxl, p, st);
+      s = run_contract<float, float>(h, dFb, Zb, dxl, p, st);
     }
     if (s == WK_OK) {
       BwContr p = contr(n, d, 1, k, static_cast<int>(B), 1, 1);
       p.sAm = k, p.sAk2 = 1;                 // Y(i, c)
       p.sBz = static_cast<int64_t>(d) * k, p.sBn = k, p.sBk2 = 1;  // dZ(b, t, c)
       p.sCz = nd, p.sCm = d, p.sCn = 1;
-      s = run_contract<T, float>(static_cast<const T*>(h->Y[l]), dZb, dxl, p, st);
+      s = run_contract<T, float>(h, static_cast<const T*>(h->Y[l]), dZb, dxl, p, st);
     }
     if (s == WK_OK) {
       BwContr p = contr(n, k, static_cast<int>(B), d, 1, contr_splits(dv, n, k, static_cast<int>(B)), 1);
       p.sAm = d, p.sAk1 = nd, p.sAk2 = 1;    // X(b, i, t)
       p.sBn = 1, p.sBk1 = static_cast<int64_t>(d) * k, p.sBk2 = k;  // dZ(b, t, c)
       p.sCm = k, p.sCn = 1;
-      s = run_contract<T, float>(xin, dZb, g.Y, p, st);
+      s = run_contract<T, float>(h, xin, dZb, g.Y, p, st);
     }
   }
   return s;
