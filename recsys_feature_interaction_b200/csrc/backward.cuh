@@ -1,14 +1,13 @@
-// backward.cuh -- the kernels of the backward pass of a Wukong layer that are not the
-// FMB MLP's tensor-core GEMMs (those reuse gemm_tc2.cuh on transposed operands).
+// backward.cuh -- the kernels of the backward pass of a Wukong layer that are neither the
+// FMB MLP's tensor-core GEMMs (gemm_tc2.cuh on transposed operands) nor the strided
+// contractions of the FM and the LCB (bw_tc.cuh).
 //
 // Per layer, with y = concat(FMB(X), LCB(X)) + X, out = LN_d(y) gamma2 + beta2, the layer
 // of the Wukong page (section 2.2) differentiated by the chain rule:
 //   bw_out_ln_kernel     dy = LN_d'(y)^T (dOut * gamma2) per embedding row; d gamma2, d beta2;
 //                        the FMB rows of dy as the MLP's upstream gradient (16-bit)
-//   bw_contract_kernel   strided batched products on CUDA cores: the LCB's W_L^T dG and
-//                        sum_b dG_b X_b^T, the FM's X^T Y, X Z, X^T dF, dF Z^T, Y dZ^T and
-//                        sum_b X_b dZ_b
 //   bw_relu_mask_kernel  dz = dh where the ReLU output was > 0
+//   bw_to_f32_kernel     fp32 copies of the 16-bit operands of the tf32 contractions
 //   bw_colsum_kernel     bias gradients (column sums over the batch)
 //   bw_transpose_kernel  16-bit transposes feeding the K-major GEMM
 //   bw_fmb_ln_kernel     dF = LN_nk'(F)^T d fhat per example (the FMB LayerNorm)
@@ -33,6 +32,14 @@ __device__ __forceinline__ float bw_ld<__half>(const __half* p) {
 template <>
 __device__ __forceinline__ float bw_ld<__nv_bfloat16>(const __nv_bfloat16* p) {
   return __bfloat162float(*p);
+}
+
+// 16-bit -> fp32 copy of an operand of the tf32 contractions (exact)
+template <typename T>
+__global__ void __launch_bounds__(256) bw_to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, int64_t n) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = bw_ld(in + i);
 }
 
 // ------------------------------------------------ output LayerNorm, per row
@@ -92,7 +99,7 @@ __global__ void __launch_bounds__(256) bw_out_ln_kernel(const T* __restrict__ ca
       if (i < per) {
         const int c = lane + 32 * i;
         const float g = rs * (go[i] - m1 - y[i] * m2);
-        dy[r * d + c] = g;
+        dy[r * d + c] = tf32_round(g);  // read only by the tf32 contractions
         dx[r * d + c] = g;  // the residual's share of dX
         if (i_row < n_f) dh_m[(b * n_f + i_row) * d + c] = Half16<T>::from(g);
       }
@@ -118,85 +125,6 @@ __global__ void __launch_bounds__(256) bw_out_ln_kernel(const T* __restrict__ ca
   }
 }
 
-// ------------------------------------------------ strided batched contraction
-
-// C[z][m][n] (+)= sum_{k1 < K1} sum_{k2 < K2} A(z, m, k1, k2) B(z, n, k1, k2), with
-// A(z, m, k1, k2) = A[z sAz + m sAm + k1 sAk1 + k2 sAk2] (B likewise), fp32 accumulation,
-// C[z sCz + m sCm + n sCn] fp32. K1 may be split over S CTAs (atomic adds into C).
-struct BwContr {
-  int M, N, K1, K2, Z, S, accumulate;
-  int64_t sAz, sAm, sAk1, sAk2, sBz, sBn, sBk1, sBk2, sCz, sCm, sCn;
-};
-
-template <typename TA, typename TB>
-__global__ void __launch_bounds__(256) bw_contract_kernel(const TA* __restrict__ A, const TB* __restrict__ B,
-                                                          float* __restrict__ C, BwContr p) {
-  __shared__ float As[16][68], Bs[16][68];
-  const int m0 = blockIdx.x * 64, n0 = blockIdx.y * 64;
-  const int z = blockIdx.z / p.S, sp = blockIdx.z - z * p.S;
-  const int k1b = static_cast<int>(static_cast<int64_t>(p.K1) * sp / p.S);
-  const int k1e = static_cast<int>(static_cast<int64_t>(p.K1) * (sp + 1) / p.S);
-  const int K = (k1e - k1b) * p.K2;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const TA* Az = A + z * p.sAz;
-  const TB* Bz = B + z * p.sBz;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < K; k0 += 16) {
-#pragma unroll
-    for (int e = threadIdx.x; e < 1024; e += 256) {
-      const int kk = e >> 6, mm = e & 63;
-      const int k = k0 + kk;
-      float va = 0.f, vb = 0.f;
-      if (k < K) {
-        const int k1 = k1b + k / p.K2, k2 = k - (k / p.K2) * p.K2;
-        if (m0 + mm < p.M) va = bw_ld(Az + (m0 + mm) * p.sAm + k1 * p.sAk1 + k2 * p.sAk2);
-        if (n0 + mm < p.N) vb = bw_ld(Bz + (n0 + mm) * p.sBn + k1 * p.sBk1 + k2 * p.sBk2);
-      }
-      As[kk][mm] = va;
-      Bs[kk][mm] = vb;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = As[kk][ty * 4 + i];
-        b[i] = Bs[kk][tx * 4 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= p.M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int nn = n0 + tx * 4 + j;
-      if (nn >= p.N) continue;
-      float* c = C + z * p.sCz + m * p.sCm + nn * p.sCn;
-      if (p.S > 1)
-        atomicAdd(c, acc[i][j]);
-      else if (p.accumulate)
-        *c += acc[i][j];
-      else
-        *c = acc[i][j];
-    }
-  }
-}
-
-// ------------------------------------------------ MLP helpers
-
-// dz = dh where the ReLU output h is > 0, else 0 (in place); count % 8 == 0.
 template <typename T>
 __global__ void bw_relu_mask_kernel(T* __restrict__ dh, const T* __restrict__ h, int64_t count) {
   const int64_t nvec = count / 8;
@@ -285,7 +213,7 @@ __global__ void __launch_bounds__(256) bw_fmb_ln_kernel(const float* __restrict_
   const float m1 = bw_block_sum(s1, red) * inv, m2 = bw_block_sum(s2, red) * inv;
   for (int i = threadIdx.x; i < nk; i += blockDim.x) {
     const float fh = (F[base + i] - mean) * rs;
-    dF[base + i] = rs * (bw_ld(dfh + base + i) - m1 - fh * m2);
+    dF[base + i] = tf32_round(rs * (bw_ld(dfh + base + i) - m1 - fh * m2));  // a tf32 operand
   }
 }
 

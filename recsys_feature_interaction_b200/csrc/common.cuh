@@ -223,7 +223,7 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 
 // Shared-memory matrix descriptor of tcgen05 (64-bit): start address, leading
 // and stride byte offsets (all >> 4), version 1 at bits 46-47, swizzle mode at
-// bits 61-63 (2 = 128B, 4 = 64B, 6 = 32B, 0 = none).
+// bits 61-63 (2 = 128B, 1 = 128B with 32-byte atoms, 4 = 64B, 6 = 32B, 0 = none).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t swizzle_mode) {
   uint64_t d = 0;
@@ -425,6 +425,13 @@ struct Half16<__half> {
   static __device__ __forceinline__ __half from(float v) { return __float2half_rn(v); }
   static __device__ __forceinline__ float to(__half v) { return __half2float(v); }
 };
+
+// fp32 -> tf32 (the top 19 bits the tensor core reads), round to nearest, ties away from zero
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -22,6 +22,7 @@
 #include <mutex>
 #include <new>
 #include <set>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -40,6 +41,7 @@
 #include "simt.cuh"
 #include "whale.cuh"
 #include "backward.cuh"
+#include "bw_tc.cuh"
 
 using namespace wk;
 
@@ -1209,31 +1211,120 @@ void free_moe(wk_moe* h) {
 
 // ---------------------------------------------------------------- backward
 
-template <typename TA, typename TB>
-wk_status run_contract(wk_stack* h, const TA* A, const TB* B, float* C, const BwContr& p, cudaStream_t st) {
-  if (p.M <= 0 || p.N <= 0 || p.Z <= 0) return WK_OK;
-  ProfScope ps(h, WK_KERNEL_BW_CONTRACT, st);
-  const dim3 grid((p.M + 63) / 64, (p.N + 63) / 64, p.Z * p.S);
-  bw_contract_kernel<TA, TB><<<grid, 256, 0, st>>>(A, B, C, p);
-  return launch_status();
+// A term of a tensor-core contraction, strides set by the caller.
+TcTerm tc_term(const float* A, const float* B, int K1, int K2) {
+  TcTerm t{};
+  t.A = A;
+  t.B = B;
+  t.K1 = K1;
+  t.K2 = K2;
+  return t;
 }
 
-BwContr contr(int M, int N, int K1, int K2, int Z, int S, int accumulate) {
-  BwContr p{};
+TcContr tc_contr(int M, int N, int Z, int S, int mode, float* C, int64_t sCz, int64_t sCm, int64_t sCn) {
+  TcContr p{};
   p.M = M;
   p.N = N;
-  p.K1 = K1;
-  p.K2 = K2;
   p.Z = Z;
   p.S = S;
-  p.accumulate = accumulate;
+  p.mode = mode;
+  p.C = C;
+  p.sCz = sCz;
+  p.sCm = sCm;
+  p.sCn = sCn;
   return p;
 }
 
-// Splits of K1 so that a launch has about four CTAs per SM.
-int contr_splits(const DevInfo* dv, int M, int N, int K1) {
-  const int tiles = ((M + 63) / 64) * ((N + 63) / 64);
-  return std::max(1, std::min(K1, (4 * dv->sms + tiles - 1) / tiles));
+int tc_bn(int N) { return N <= 64 ? 64 : N <= 128 ? 128 : N <= 160 ? 160 : 128; }
+
+// The 4-D TMA tensor of one fp32 operand with `rows` rows (m or n), K2 x K1 values of k and
+// Z of z; strides in elements. K-major where k2 is contiguous (dims k2, row, k1, z; box 32 x
+// box_rows, 128-byte swizzle), else MN-major where the row index is (dims row, k2, k1, z; box
+// 32 x 32, 128-byte swizzle with 32-byte atoms). A stride of 0 along z (an operand shared by
+// every z) becomes a dimension of size 1 read at coordinate 0.
+bool tc_map(const DevInfo* dv, CUtensorMap* m, const float* ptr, int64_t rows, int64_t K2, int64_t K1, int64_t Z,
+            int64_t s_row, int64_t s_k2, int64_t s_k1, int64_t s_z, uint32_t box_rows, int* mn, int* z0) {
+  if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return false;
+  *z0 = s_z == 0 ? 1 : 0;
+  uint64_t dims[4], str[3];
+  uint32_t box[4] = {32, box_rows, 1, 1};
+  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (s_k2 == 1) {
+    *mn = 0;
+    dims[0] = K2, dims[1] = rows, str[0] = s_row * 4;
+  } else if (s_row == 1) {
+    *mn = 1;
+    dims[0] = rows, dims[1] = K2, str[0] = s_k2 * 4;
+    box[1] = 32;
+    sw = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+  } else {
+    return false;
+  }
+  dims[2] = K1, dims[3] = *z0 ? 1 : Z;
+  str[1] = K1 > 1 ? s_k1 * 4 : str[0] * dims[1];  // a size-1 dimension takes any valid stride
+  str[2] = dims[3] > 1 ? s_z * 4 : str[1] * dims[2];
+  for (int i = 0; i < 3; ++i)
+    if (str[i] == 0 || str[i] % 16 != 0 || str[i] >= (1ull << 40)) return false;
+  return make_map(dv, m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, str, box, sw);
+}
+
+template <int BN>
+wk_status launch_tc_contract(const DevInfo* dv, const TcMaps& mp, const TcContr& p, cudaStream_t st) {
+  using Cfg = TcCfg<BN>;
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(bw_tc_contract_kernel<BN>), Cfg::SMEM);
+  if (s != WK_OK) return s;
+  const int grid = std::min(p.num_tiles, dv->sms);
+  bw_tc_contract_kernel<BN><<<grid, TC_THREADS, Cfg::SMEM, st>>>(mp, p);
+  return launch_status();
+}
+
+// The strided contraction on the tensor cores (tf32 operands, fp32 accumulation).
+wk_status run_tc_contract(wk_stack* h, TcContr p, cudaStream_t st) {
+  if (p.M <= 0 || p.N <= 0 || p.Z <= 0 || p.nterms <= 0) return WK_OK;
+  if (p.nterms > 3 || p.S < 1 || (p.S > 1 && p.mode != TC_ATOMIC)) return WK_ERR_UNSUPPORTED;
+  const int bn = tc_bn(p.N);
+  TcMaps mp;
+  for (int t = 0; t < p.nterms; ++t) {
+    TcTerm& q = p.t[t];
+    if (q.K1 < p.S || q.K2 < 1) return WK_ERR_UNSUPPORTED;  // every split of every term has a k1
+    if (!tc_map(h->dv, &mp.m[2 * t], q.A, p.M, q.K2, q.K1, p.Z, q.sAm, q.sAk2, q.sAk1, q.sAz, 128, &q.a_mn, &q.a_z0) ||
+        !tc_map(h->dv, &mp.m[2 * t + 1], q.B, p.N, q.K2, q.K1, p.Z, q.sBn, q.sBk2, q.sBk1, q.sBz,
+                static_cast<uint32_t>(bn), &q.b_mn, &q.b_z0))
+      return WK_ERR_UNSUPPORTED;
+    q.k1q = q.K1 / p.S;
+    q.k1r = q.K1 % p.S;
+    q.nk2 = (q.K2 + TC_BK - 1) / TC_BK;
+  }
+  p.mt = (p.M + 127) / 128;
+  p.nt = (p.N + bn - 1) / bn;
+  const int64_t tiles = static_cast<int64_t>(p.Z) * p.S * p.mt * p.nt;
+  if (tiles > 0x7FFFFFFFll) return WK_ERR_UNSUPPORTED;
+  p.num_tiles = static_cast<int>(tiles);
+  p.c_vec = p.sCn == 1 && reinterpret_cast<uintptr_t>(p.C) % 16 == 0 && p.sCm % 4 == 0 && p.sCz % 4 == 0;
+  p.status = h->status;
+  ProfScope ps(h, WK_KERNEL_BW_CONTRACT, st);
+  switch (bn) {
+    case 64: return launch_tc_contract<64>(h->dv, mp, p, st);
+    case 160: return launch_tc_contract<160>(h->dv, mp, p, st);
+    default: return launch_tc_contract<128>(h->dv, mp, p, st);
+  }
+}
+
+// Splits of the k1 range so that a launch has one tile per SM (rounded down: an SM with a
+// second tile would double the launch's time).
+int tc_splits(const DevInfo* dv, int M, int N, int K1) {
+  const int bn = tc_bn(N);
+  const int tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
+  return std::max(1, std::min(K1, dv->sms / tiles));
+}
+
+template <typename T>
+wk_status to_f32(wk_stack* h, const void* in, float* out, int64_t n, cudaStream_t st) {
+  if (n <= 0) return WK_OK;
+  ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
+  const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, h->dv->sms * 16ll));
+  bw_to_f32_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(in), out, n);
+  return launch_status();
 }
 
 // C [M, N] = A [M, K] W [N, K]^T on the tensor cores (16-bit K-major operands, TO output).
@@ -1279,8 +1370,9 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
   // workspace: saved layer inputs, fp32 dy and two dX buffers, two 16-bit MLP gradients,
   // the transposes, the FM's Z, dZ, F and dF
   const size_t b_sv = up(B * nd * 2), b_f = up(B * nd * 4), b_h = up(B * hmax * 2), b_w = up(wmax * 2),
-               b_z = up(B * static_cast<size_t>(d) * k * 4), b_fk = up(B * nk * 4);
-  const size_t need = L * b_sv + 3 * b_f + 4 * b_h + b_w + 2 * b_z + 2 * b_fk;
+               b_z = up(B * static_cast<size_t>(d) * k * 4), b_fk = up(B * nk * 4),
+               b_wl = up(static_cast<size_t>(n_l) * n * 4), b_y = up(nk * 4);
+  const size_t need = L * b_sv + 4 * b_f + 4 * b_h + b_w + 2 * b_z + 2 * b_fk + b_wl + b_y;
   if (h->bws_bytes < need) {
     if (h->bws) cudaFree(h->bws);
     h->bws = nullptr;
@@ -1311,6 +1403,10 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
   p += 2 * b_z;
   float* Fb = reinterpret_cast<float*>(p);
   float* dFb = reinterpret_cast<float*>(p + b_fk);
+  p += 2 * b_fk;
+  float* Xf = reinterpret_cast<float*>(p);  // fp32 copies of the layer's X, W_L and Y
+  float* WLf = reinterpret_cast<float*>(p + b_f);
+  float* Yf = reinterpret_cast<float*>(p + b_f + b_wl);
 
   wk_status s = WK_OK;
   // 1. the forward, saving each layer's input
@@ -1334,6 +1430,9 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     const float* up_grad = (l == L - 1) ? dOut : gx[(l + 1) % 2];
     float* dxl = (l == 0) ? dX : gx[l % 2];
     s = layer_front16<T>(h, l, xin, lcbx[l], B, st);
+    if (s == WK_OK) s = to_f32<T>(h, xin, Xf, B * static_cast<int64_t>(nd), st);
+    if (s == WK_OK) s = to_f32<T>(h, h->WL[l], WLf, static_cast<int64_t>(n_l) * n, st);
+    if (s == WK_OK) s = to_f32<T>(h, h->Y[l], Yf, static_cast<int64_t>(nk), st);
     if (s != WK_OK) break;
     cudaMemsetAsync(g.out_ln_gamma, 0, d * 4, st);
     cudaMemsetAsync(g.out_ln_beta, 0, d * 4, st);
@@ -1350,20 +1449,15 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
                                                  g.out_ln_gamma, g.out_ln_beta, rows, n, n_f, d, h->eps);
       s = launch_status();
     }
-    // LCB: dX_b += W_L^T dG_b; dW_L = sum_b dG_b X_b^T (dG = rows n_f.. of dy)
+    // LCB: dW_L = sum_b dG_b X_b^T (dG = rows n_f.. of dy; W_L^T dG_b joins dX below)
+    const float* dG = dyf + static_cast<size_t>(n_f) * d;
     if (s == WK_OK) {
-      BwContr p = contr(n, d, 1, n_l, static_cast<int>(B), 1, 1);
-      p.sAm = 1, p.sAk2 = n;                                                  // W_L(r, i) at r n + i
-      p.sBz = nd, p.sBn = 1, p.sBk2 = d;                                      // dG(b, r, t)
-      p.sCz = nd, p.sCm = d, p.sCn = 1;
-      s = run_contract<T, float>(h, static_cast<const T*>(h->WL[l]), dyf + static_cast<size_t>(n_f) * d, dxl, p, st);
-    }
-    if (s == WK_OK) {
-      BwContr p = contr(n_l, n, static_cast<int>(B), d, 1, contr_splits(dv, n_l, n, static_cast<int>(B)), 1);
-      p.sAm = d, p.sAk1 = nd, p.sAk2 = 1;                                     // dG(b, r, t)
-      p.sBn = d, p.sBk1 = nd, p.sBk2 = 1;                                     // X(b, i, t)
-      p.sCm = n, p.sCn = 1;
-      s = run_contract<float, T>(h, dyf + static_cast<size_t>(n_f) * d, xin, g.W_L, p, st);
+      TcContr p = tc_contr(n_l, n, 1, tc_splits(dv, n_l, n, static_cast<int>(B)), TC_ATOMIC, g.W_L, 0, n, 1);
+      p.nterms = 1;
+      p.t[0] = tc_term(dG, Xf, static_cast<int>(B), d);
+      p.t[0].sAm = d, p.t[0].sAk1 = nd, p.t[0].sAk2 = 1;  // dG(b, r, t)
+      p.t[0].sBn = d, p.t[0].sBk1 = nd, p.t[0].sBk2 = 1;  // X(b, i, t)
+      s = run_tc_contract(h, p, st);
     }
     // FMB MLP, last Linear first: dz (16-bit) -> bias, weight and input gradients
     int cur = 0;
@@ -1401,21 +1495,26 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
                                                  h->b1_in[l], g.fmb_ln_gamma, g.fmb_ln_beta, dims[1], dims[0]);
       s = launch_status();
     }
-    // FMB: Z = X^T Y, F = X Z, dF from the LayerNorm backward, then dZ = X^T dF,
-    // dX += dF Z^T + Y dZ^T, dY = sum_b X_b dZ_b
+    // FMB: Z = X^T Y, F = X Z, dF from the LayerNorm backward, then dZ = X^T dF;
+    // dX += W_L^T dG + dF Z^T + Y dZ^T in one launch; dY = sum_b X_b dZ_b
+    const int64_t dk = static_cast<int64_t>(d) * k;
+    const int Bi = static_cast<int>(B);
     if (s == WK_OK) {
-      BwContr p = contr(d, k, 1, n, static_cast<int>(B), 1, 0);
-      p.sAz = nd, p.sAm = 1, p.sAk2 = d;     // X(b, i, t) as (m = t, k = i)
-      p.sBn = 1, p.sBk2 = k;                 // Y(i, c)
-      p.sCz = static_cast<int64_t>(d) * k, p.sCm = k, p.sCn = 1;
-      s = run_contract<T, T>(h, xin, static_cast<const T*>(h->Y[l]), Zb, p, st);
+      TcContr p = tc_contr(d, k, Bi, 1, TC_STORE, Zb, dk, k, 1);
+      p.nterms = 1;
+      p.round_c = 1;  // Z is read only by the tf32 contractions
+      p.t[0] = tc_term(Xf, Yf, 1, n);
+      p.t[0].sAz = nd, p.t[0].sAm = 1, p.t[0].sAk2 = d;  // X(b, i, t) as (m = t, k = i)
+      p.t[0].sBn = 1, p.t[0].sBk2 = k;                   // Y(i, c)
+      s = run_tc_contract(h, p, st);
     }
     if (s == WK_OK) {
-      BwContr p = contr(n, k, 1, d, static_cast<int>(B), 1, 0);
-      p.sAz = nd, p.sAm = d, p.sAk2 = 1;     // X(b, i, t)
-      p.sBz = static_cast<int64_t>(d) * k, p.sBn = 1, p.sBk2 = k;  // Z(b, t, c)
-      p.sCz = nk, p.sCm = k, p.sCn = 1;
-      s = run_contract<T, float>(h, xin, Zb, Fb, p, st);
+      TcContr p = tc_contr(n, k, Bi, 1, TC_STORE, Fb, nk, k, 1);
+      p.nterms = 1;
+      p.t[0] = tc_term(Xf, Zb, 1, d);
+      p.t[0].sAz = nd, p.t[0].sAm = d, p.t[0].sAk2 = 1;  // X(b, i, t)
+      p.t[0].sBz = dk, p.t[0].sBn = 1, p.t[0].sBk2 = k;  // Z(b, t, c)
+      s = run_tc_contract(h, p, st);
     }
     if (s == WK_OK) {
       ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
@@ -1423,32 +1522,35 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
       s = launch_status();
     }
     if (s == WK_OK) {
-      BwContr p = contr(d, k, 1, n, static_cast<int>(B), 1, 0);
-      p.sAz = nd, p.sAm = 1, p.sAk2 = d;     // X(b, i, t) as (m = t, k = i)
-      p.sBz = nk, p.sBn = 1, p.sBk2 = k;     // dF(b, i, c)
-      p.sCz = static_cast<int64_t>(d) * k, p.sCm = k, p.sCn = 1;
-      s = run_contract<T, float>(h, xin, dFb, dZb, p, st);
+      TcContr p = tc_contr(d, k, Bi, 1, TC_STORE, dZb, dk, k, 1);
+      p.nterms = 1;
+      p.round_c = 1;  // so is dZ
+      p.t[0] = tc_term(Xf, dFb, 1, n);
+      p.t[0].sAz = nd, p.t[0].sAm = 1, p.t[0].sAk2 = d;  // X(b, i, t) as (m = t, k = i)
+      p.t[0].sBz = nk, p.t[0].sBn = 1, p.t[0].sBk2 = k;  // dF(b, i, c)
+      s = run_tc_contract(h, p, st);
     }
     if (s == WK_OK) {
-      BwContr p = contr(n, d, 1, k, static_cast<int>(B), 1, 1);
-      p.sAz = nk, p.sAm = k, p.sAk2 = 1;     // dF(b, i, c)
-      p.sBz = static_cast<int64_t>(d) * k, p.sBn = k, p.sBk2 = 1;  // Z(b, t, c)
-      p.sCz = nd, p.sCm = d, p.sCn = 1;
-      s = run_contract<float, float>(h, dFb, Zb, dxl, p, st);
+      TcContr p = tc_contr(n, d, Bi, 1, TC_ACCUM, dxl, nd, d, 1);
+      p.nterms = 3;
+      p.t[0] = tc_term(WLf, dG, 1, n_l);
+      p.t[0].sAm = 1, p.t[0].sAk2 = n;                   // W_L(r, i) at r n + i
+      p.t[0].sBz = nd, p.t[0].sBn = 1, p.t[0].sBk2 = d;  // dG(b, r, t)
+      p.t[1] = tc_term(dFb, Zb, 1, k);
+      p.t[1].sAz = nk, p.t[1].sAm = k, p.t[1].sAk2 = 1;  // dF(b, i, c)
+      p.t[1].sBz = dk, p.t[1].sBn = k, p.t[1].sBk2 = 1;  // Z(b, t, c)
+      p.t[2] = tc_term(Yf, dZb, 1, k);
+      p.t[2].sAm = k, p.t[2].sAk2 = 1;                   // Y(i, c)
+      p.t[2].sBz = dk, p.t[2].sBn = k, p.t[2].sBk2 = 1;  // dZ(b, t, c)
+      s = run_tc_contract(h, p, st);
     }
     if (s == WK_OK) {
-      BwContr p = contr(n, d, 1, k, static_cast<int>(B), 1, 1);
-      p.sAm = k, p.sAk2 = 1;                 // Y(i, c)
-      p.sBz = static_cast<int64_t>(d) * k, p.sBn = k, p.sBk2 = 1;  // dZ(b, t, c)
-      p.sCz = nd, p.sCm = d, p.sCn = 1;
-      s = run_contract<T, float>(h, static_cast<const T*>(h->Y[l]), dZb, dxl, p, st);
-    }
-    if (s == WK_OK) {
-      BwContr p = contr(n, k, static_cast<int>(B), d, 1, contr_splits(dv, n, k, static_cast<int>(B)), 1);
-      p.sAm = d, p.sAk1 = nd, p.sAk2 = 1;    // X(b, i, t)
-      p.sBn = 1, p.sBk1 = static_cast<int64_t>(d) * k, p.sBk2 = k;  // dZ(b, t, c)
-      p.sCm = k, p.sCn = 1;
-      s = run_contract<T, float>(h, xin, dZb, g.Y, p, st);
+      TcContr p = tc_contr(n, k, 1, tc_splits(dv, n, k, Bi), TC_ATOMIC, g.Y, 0, k, 1);
+      p.nterms = 1;
+      p.t[0] = tc_term(Xf, dZb, Bi, d);
+      p.t[0].sAm = d, p.t[0].sAk1 = nd, p.t[0].sAk2 = 1;  // X(b, i, t)
+      p.t[0].sBn = 1, p.t[0].sBk1 = dk, p.t[0].sBk2 = k;  // dZ(b, t, c)
+      s = run_tc_contract(h, p, st);
     }
   }
   return s;
