@@ -72,12 +72,18 @@ __device__ __forceinline__ void gemm2_tile_coords(const GemmParams& p, int tile,
 // (256, or E = floor(256/d) whole embedding rows of the last Linear when ROWLN: then
 // the epilogue adds the bias and the residual, applies the output LayerNorm and tmC
 // addresses the layer output [M, n*d]).
-template <typename T, typename TO, bool ROWLN = false, bool STREAM = false>
+//
+// A_MN / B_MN: the operand is stored MN-major, as A^T [K, M] (W^T [K, N]) row-major with the
+// tensor map's dims (M, K) (N, K): each CTA's 128 rows then arrive as two 64-row x 64-k boxes
+// (128-byte swizzle) 8 KB apart and are read MN-major (the backward's weight gradients
+// dz^T h and input gradients dz W need no transposed copies).
+template <typename T, typename TO, bool ROWLN = false, bool STREAM = false, bool A_MN = false, bool B_MN = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using S = Gemm2Shape<STREAM>;
   static_assert(!(STREAM && ROWLN), "the fused end-of-layer epilogue runs persistent");
+  static_assert(!(ROWLN && (A_MN || B_MN)), "MN-major operands only with the plain epilogue (mma_n = 256)");
   constexpr int GEMM2_STAGES = S::STAGES;  // shadows the persistent default
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -143,11 +149,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (GEMM2_A_STAGE + static_cast<uint32_t>(p.mma_n / 2) * 128u));
           const uint32_t fbar = full0 + static_cast<uint32_t>(s) * 8u;
-          if (p.l2hint) {
+          if constexpr (A_MN) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE + j * 8192, arow + 64 * j, kb * GEMM2_BK);
+          } else if (p.l2hint) {
             tma_load_2d_pair_hint(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow, pol_a);
-            tma_load_2d_pair_hint(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow, pol_b);
           } else {
             tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE + j * 8192, brow + 64 * j, kb * GEMM2_BK);
+          } else if (p.l2hint) {
+            tma_load_2d_pair_hint(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow, pol_b);
+          } else {
             tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow);
           }
           if (++s == GEMM2_STAGES) {
@@ -163,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_f16kind_f32(GEMM2_BM, p.mma_n, 0, 0, Half16<T>::kBF16);
+      const uint32_t idesc = idesc_f16kind_f32(GEMM2_BM, p.mma_n, A_MN ? 1 : 0, B_MN ? 1 : 0, Half16<T>::kBF16);
       const uint32_t empty_own = smem_u32(empty), empty_peer = mapa_shared(smem_u32(empty), 1);
       const uint32_t tfull_own = smem_u32(tfull), tfull_peer = mapa_shared(smem_u32(tfull), 1);
       int s = 0;
@@ -188,9 +205,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t a_addr = smem_u32(sA + s * GEMM2_A_STAGE);
           const uint32_t b_addr = smem_u32(sB + s * GEMM2_B_STAGE);
 #pragma unroll
-          for (int kk = 0; kk < GEMM2_BK / 16; ++kk)
-            umma_f16kind_pair(d_tmem, smem_desc(a_addr + kk * 32, 16, 1024, 2), smem_desc(b_addr + kk * 32, 16, 1024, 2),
-                              idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < GEMM2_BK / 16; ++kk) {
+            // K-major: the 16-k slice 32 bytes into each 128-byte row; MN-major: 16 k rows
+            // (2048 bytes) on, 64-row boxes 8 KB apart, 8-row k groups 1 KB apart
+            const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, 2) : smem_desc(a_addr + kk * 32, 16, 1024, 2);
+            const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 8192, 1024, 2) : smem_desc(b_addr + kk * 32, 16, 1024, 2);
+            umma_f16kind_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
           umma_commit_pair(empty_own + static_cast<uint32_t>(s) * 8u);
           umma_commit_pair(empty_peer + static_cast<uint32_t>(s) * 8u);
           issued = true;

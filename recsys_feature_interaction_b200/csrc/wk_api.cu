@@ -164,6 +164,16 @@ bool map_kmajor(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t K, ui
   return make_map(dv, m, tmap_dtype<T>(), 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// The transpose of a K-major operand: [K, rows] 16-bit row-major with row stride ld
+// elements, read MN-major: box 64 rows x 64 k, 128B swizzle.
+template <typename T>
+bool map_mnmajor(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t K, uint64_t rows, uint64_t ld) {
+  const uint64_t dims[2] = {rows, K};
+  const uint64_t str[1] = {ld * 2};
+  const uint32_t box[2] = {64, 64};
+  return make_map(dv, m, tmap_dtype<T>(), 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // Output [rows, N], row stride ldc elements; 32 x 32 boxes (16-bit: 64B swizzle, fp32: 128B).
 template <typename TO>
 bool map_out(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t N, uint64_t rows, uint64_t ldc) {
@@ -220,23 +230,24 @@ bool gemm2_stream() {
   return on;
 }
 
-template <typename T, typename TO, bool ROWLN = false>
+template <typename T, typename TO, bool ROWLN = false, bool A_MN = false, bool B_MN = false>
 wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
   if (p.num_tiles <= 0) return WK_OK;
   if constexpr (!ROWLN) {
     if (gemm2_stream()) {
       constexpr uint32_t smem = gemm2_smem_bytes<TO, true>();
-      wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, false, true>), smem);
+      wk_status s =
+          smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, false, true, A_MN, B_MN>), smem);
       if (s != WK_OK) return s;
-      gemm_tc2_kernel<T, TO, false, true><<<2 * p.num_tiles, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+      gemm_tc2_kernel<T, TO, false, true, A_MN, B_MN><<<2 * p.num_tiles, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
       return launch_status();
     }
   }
   constexpr uint32_t smem = gemm2_smem_bytes<TO>();
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, ROWLN>), smem);
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, ROWLN, false, A_MN, B_MN>), smem);
   if (s != WK_OK) return s;
   const int pairs = std::min(p.num_tiles, dv->sms / 2);
-  gemm_tc2_kernel<T, TO, ROWLN><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  gemm_tc2_kernel<T, TO, ROWLN, false, A_MN, B_MN><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
 }
 
@@ -1342,6 +1353,22 @@ wk_status bw_gemm(wk_stack* h, const void* A, const void* W, void* C, int64_t M,
   return run_gemm_tc<MODE_MLP, T, TO>(dv, mp, mlp_params(M, K, N, nullptr, 0, h->status), st);
 }
 
+// C [M, N] = A [M, K] W [N, K]^T on the CTA-pair GEMM with A (A_MN) and W (B_MN) given as
+// their transposes A^T [K, M], W^T [K, N] (row strides lda, ldb) and read MN-major.
+template <typename T, typename TO, bool A_MN, bool B_MN>
+wk_status bw_gemm_mn(wk_stack* h, const void* A, int64_t lda, const void* W, int64_t ldb, void* C, int64_t M, int K,
+                     int N, cudaStream_t st) {
+  const DevInfo* dv = h->dv;
+  if (!mlp_tc_ok(M, K, N, N) || (A_MN && lda % 8 != 0) || (B_MN && ldb % 8 != 0)) return WK_ERR_UNSUPPORTED;
+  GemmMaps mp;
+  const bool ok = (A_MN ? map_mnmajor<T>(dv, &mp.A, A, K, M, lda) : map_kmajor<T>(dv, &mp.A, A, K, M, GEMM_BM)) &&
+                  (B_MN ? map_mnmajor<T>(dv, &mp.B, W, K, N, ldb) : map_kmajor<T>(dv, &mp.B, W, K, N, 128)) &&
+                  map_out<TO>(dv, &mp.C, C, N, M, N);
+  if (!ok) return WK_ERR_UNSUPPORTED;
+  ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+  return run_gemm_tc2<T, TO, false, A_MN, B_MN>(dv, mp, mlp2_params(M, K, N, nullptr, 0, h->status), st);
+}
+
 template <typename T>
 wk_status bw_transpose(wk_stack* h, const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
   ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
@@ -1477,14 +1504,26 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
         bw_colsum_kernel<T><<<grid, 256, 0, st>>>(dz[cur], g.b[j], B, static_cast<int>(hout));
         s = launch_status();
       }
-      // dW_j = dz^T h_j (K = batch): both operands transposed to K-major
-      if (s == WK_OK) s = bw_transpose<T>(h, dz[cur], dzT, B, hout, st);
-      if (s == WK_OK) s = bw_transpose<T>(h, hj, hT, B, hin, st);
-      if (s == WK_OK) s = bw_gemm<T, float>(h, dzT, hT, g.W[j], hout, static_cast<int>(B), static_cast<int>(hin), st);
-      // dh_j = dz W_j: W_j^T as the K-major operand
-      if (s == WK_OK) s = bw_transpose<T>(h, h->W[l][j], wT, hout, hin, st);
-      if (s == WK_OK)
-        s = bw_gemm<T, T>(h, dz[cur], wT, dz[1 - cur], B, static_cast<int>(hout), static_cast<int>(hin), st);
+      // dW_j = dz^T h_j (K = batch): on the pair GEMM both read MN-major, else transposed
+      // to K-major for the one-CTA GEMM
+      if (s == WK_OK && use_pair_gemm(hout)) {
+        s = bw_gemm_mn<T, float, true, true>(h, dz[cur], hout, hj, hin, g.W[j], hout, static_cast<int>(B),
+                                             static_cast<int>(hin), st);
+      } else if (s == WK_OK) {
+        s = bw_transpose<T>(h, dz[cur], dzT, B, hout, st);
+        if (s == WK_OK) s = bw_transpose<T>(h, hj, hT, B, hin, st);
+        if (s == WK_OK)
+          s = bw_gemm<T, float>(h, dzT, hT, g.W[j], hout, static_cast<int>(B), static_cast<int>(hin), st);
+      }
+      // dh_j = dz W_j: W_j (= (W_j^T)^T) read MN-major on the pair GEMM, else transposed
+      if (s == WK_OK && use_pair_gemm(B)) {
+        s = bw_gemm_mn<T, T, false, true>(h, dz[cur], 0, h->W[l][j], hin, dz[1 - cur], B, static_cast<int>(hout),
+                                          static_cast<int>(hin), st);
+      } else if (s == WK_OK) {
+        s = bw_transpose<T>(h, h->W[l][j], wT, hout, hin, st);
+        if (s == WK_OK)
+          s = bw_gemm<T, T>(h, dz[cur], wT, dz[1 - cur], B, static_cast<int>(hout), static_cast<int>(hin), st);
+      }
       cur = 1 - cur;
     }
     // the folded first Linear: gradients of the caller's W0, gamma1, beta1 (b0 = b0')

@@ -16,8 +16,11 @@ it). Only the GPU's fp32 summation order then separates the two, so a gate can s
 where a pre-activation is within about 1e-4 of zero, and on a small batch such a difference
 moves the upstream gradients by percents (both are valid subgradients). Two cases therefore:
 the workload's own weights (deeper layers: units with |z| < 2e-3 rms(z) in some example are
-left out of their own W_j rows and b_j, and must be few), and the 4-layer shape with its hidden
-biases at +-4, where no pre-activation is near 0 (asserted) and everything is compared in full.
+left out of their own W_j rows and b_j, and must be few), and one layer with its hidden biases
+moved to +-5 times the spread of its pre-activations, where no pre-activation is near 0
+(asserted) and everything is compared in full: the 4-layer shape on 8 examples, and the 2-layer
+shape on 256 examples, where both MLP gradient GEMMs (batch and hidden width above 128) run on
+the CTA-pair kernel with operands read MN-major instead of transposed.
 """
 import numpy as np
 import pytest
@@ -84,7 +87,8 @@ def _shift_hidden_biases(cfg, host_w, dev_w, X, seed):
         dev_w[0]["b%d" % j] = to_dev(b)
 
 
-@pytest.mark.parametrize("name,batch,layers,shift", [("c2_bf16", 16, 2, False), ("c3_bf16", 8, 1, True)])
+@pytest.mark.parametrize("name,batch,layers,shift", [("c2_bf16", 16, 2, False), ("c3_bf16", 8, 1, True),
+                                                     ("c2_bf16", 256, 1, True)])
 def test_stack_backward_against_oracle(name, batch, layers, shift):
     cfg = dict(C.CONFIGS[name], layers=layers)
     dims = C.mlp_dims(cfg)
