@@ -355,9 +355,9 @@ def run_whale(args, cfg, rank, world, local, dev):
 
 def run_backward(args, cfg, rank, world, local, dev):
     """One step = wk_stack_backward over the per-GPU batch: the forward with every layer's
-    input saved, then each layer's front recomputed and differentiated (dX and all parameter
+    input and activations saved, then each layer differentiated (dX and all parameter
     gradients). Algorithmic work: 3x the forward's matmul FLOPs. Roofline: the FMB MLP GEMM
-    (forward save, recompute, input and weight gradients), tensor-bound."""
+    (forward, input and weight gradients), tensor-bound."""
     import torch
 
     import recsys_feature_interaction_b200 as wk
@@ -436,14 +436,15 @@ def run_backward(args, cfg, rank, world, local, dev):
         fwd = C.flops_per_example(cfg)
         flops_ex = 3 * fwd
         tflops = value * flops_ex / 1e12 / world
-        # executed MLP GEMM work per step: forward save (L-1 layers), recompute (L), and the
-        # input and weight gradients (2 L), each the forward's per-layer MLP FLOPs
+        # executed MLP GEMM work per step: the forward (L layers, activations saved, none
+        # recomputed) and the input and weight gradients (2 L), each the forward's per-layer
+        # MLP FLOPs
         mlp_layer = gemm_flops_per_example(cfg) / L * B
-        gemm_flops_step = (4 * L - 1) * mlp_layer
+        gemm_flops_step = 3 * L * mlp_layer
         g_ms, g_n = ktimes["mlp_gemm"]
         ach = gemm_flops_step * args.steps / (g_ms / 1e3) / 1e12 if g_ms else None
         peak = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
-        roof = {"kernel": "mlp_gemm (tcgen05 pair GEMM: forward, input and weight gradients)", "bound": "tensor",
+        roof = {"kernel": "mlp_gemm (tcgen05 pair GEMM: forward, input and weight gradients, the gradients reading MN-major operands)", "bound": "tensor",
                 "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": (ach / peak) if ach else None,
                 "traffic": None, "peak_note": "%s sustained cuBLAS bf16" % peak_src,
                 "algorithmic_per_step": {"flops": gemm_flops_step, "launches": g_n / max(1, args.steps)}}

@@ -1394,12 +1394,21 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
   for (int j = 0; j <= m; ++j) hmax = std::max<int64_t>(hmax, dims[j]);
   for (int j = 0; j < m; ++j) wmax = std::max<int64_t>(wmax, static_cast<int64_t>(dims[j]) * dims[j + 1]);
   auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
-  // workspace: saved layer inputs, fp32 dy and two dX buffers, two 16-bit MLP gradients,
-  // the transposes, the FM's Z, dZ, F and dF
+  // the MLP gradient GEMMs read their operands MN-major on the pair kernel; the one-CTA
+  // kernel (batch or a hidden width of at most 128) needs transposed copies
+  bool transposes = !use_pair_gemm(B);
+  for (int j = 0; j < m; ++j) transposes = transposes || !use_pair_gemm(dims[j + 1]);
+  // workspace: saved layer inputs; the saved activations of every layer but the last (its
+  // FMB LayerNorm output A0, the hidden ReLU outputs, the concat buffer); fp32 dy and two dX
+  // buffers; two 16-bit MLP gradients; the transposes if needed; the FM's Z, dZ, F and dF;
+  // fp32 copies of X, W_L and Y
   const size_t b_sv = up(B * nd * 2), b_f = up(B * nd * 4), b_h = up(B * hmax * 2), b_w = up(wmax * 2),
                b_z = up(B * static_cast<size_t>(d) * k * 4), b_fk = up(B * nk * 4),
                b_wl = up(static_cast<size_t>(n_l) * n * 4), b_y = up(nk * 4);
-  const size_t need = L * b_sv + 4 * b_f + 4 * b_h + b_w + 2 * b_z + 2 * b_fk + b_wl + b_y;
+  size_t b_act = up(B * static_cast<size_t>(dims[0]) * 2) + b_sv;
+  for (int j = 0; j + 1 < m; ++j) b_act += up(B * static_cast<size_t>(dims[j + 1]) * 2);
+  const size_t need = L * b_sv + (L - 1) * b_act + 4 * b_f + 2 * b_h + (transposes ? 2 * b_h + b_w : 0) + 2 * b_z +
+                      2 * b_fk + b_wl + b_y;
   if (h->bws_bytes < need) {
     if (h->bws) cudaFree(h->bws);
     h->bws = nullptr;
@@ -1413,18 +1422,33 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
   uint8_t* p = h->bws;
   std::vector<T*> xs(L);
   for (int l = 0; l < L; ++l, p += b_sv) xs[l] = reinterpret_cast<T*>(p);
+  struct Acts {
+    const void* A0;
+    const void* H[2];
+    const void* cat;
+  };
+  std::vector<Acts> acts(L);  // layer L - 1 keeps its activations in the stack's buffers
+  acts[L - 1] = Acts{h->A0, {h->H[0], h->H[1]}, h->cat};
+  for (int l = 0; l + 1 < L; ++l) {
+    acts[l].A0 = p;
+    p += up(B * static_cast<size_t>(dims[0]) * 2);
+    for (int j = 0; j + 1 < m; ++j) {
+      acts[l].H[j] = p;
+      p += up(B * static_cast<size_t>(dims[j + 1]) * 2);
+    }
+    acts[l].cat = p;
+    p += b_sv;
+  }
   float* dyf = reinterpret_cast<float*>(p);
   p += b_f;
   float* gx[2] = {reinterpret_cast<float*>(p), reinterpret_cast<float*>(p + b_f)};
   p += 2 * b_f;
   T* dz[2] = {reinterpret_cast<T*>(p), reinterpret_cast<T*>(p + b_h)};
   p += 2 * b_h;
-  T* dzT = reinterpret_cast<T*>(p);
-  p += b_h;
-  T* hT = reinterpret_cast<T*>(p);
-  p += b_h;
-  T* wT = reinterpret_cast<T*>(p);
-  p += b_w;
+  T* dzT = transposes ? reinterpret_cast<T*>(p) : nullptr;
+  T* hT = transposes ? reinterpret_cast<T*>(p + b_h) : nullptr;
+  T* wT = transposes ? reinterpret_cast<T*>(p + 2 * b_h) : nullptr;
+  if (transposes) p += 2 * b_h + b_w;
   float* Zb = reinterpret_cast<float*>(p);
   float* dZb = reinterpret_cast<float*>(p + b_z);
   p += 2 * b_z;
@@ -1436,7 +1460,7 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
   float* Yf = reinterpret_cast<float*>(p + b_f + b_wl);
 
   wk_status s = WK_OK;
-  // 1. the forward, saving each layer's input
+  // 1. the forward, saving each layer's input and activations
   if (sizeof(IO) != sizeof(T) || Half16<IO>::kBF16 != Half16<T>::kBF16)
     s = run_convert<IO, T>(dv, X, xs[0], rows * d, st);
   else if (cudaMemcpyAsync(xs[0], X, B * nd * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -1444,8 +1468,16 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
   std::vector<CUtensorMap> lcbx(L);
   for (int l = 0; l < L && s == WK_OK; ++l)
     if (h->tc_lcb && !map_lcb_x<T>(dv, &lcbx[l], xs[l], n, d, B)) s = WK_ERR_CUDA;
+  auto save = [&](const void* src, const void* dst, size_t bytes) {
+    if (s == WK_OK &&
+        cudaMemcpyAsync(const_cast<void*>(dst), src, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      s = WK_ERR_CUDA;
+  };
   for (int l = 0; l + 1 < L && s == WK_OK; ++l) {
     s = layer_front16<T>(h, l, xs[l], lcbx[l], B, st);
+    save(h->A0, acts[l].A0, B * static_cast<size_t>(dims[0]) * 2);
+    for (int j = 0; j + 1 < m; ++j) save(h->H[j % 2], acts[l].H[j], B * static_cast<size_t>(dims[j + 1]) * 2);
+    save(h->cat, acts[l].cat, B * nd * 2);
     if (s == WK_OK)
       s = run_res_ln<T, T, T>(dv, static_cast<const T*>(h->cat), xs[l], h->g2[l], h->b2[l], xs[l + 1], rows, d, h->eps,
                               h->status, st);
@@ -1456,7 +1488,8 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     const T* xin = xs[l];
     const float* up_grad = (l == L - 1) ? dOut : gx[(l + 1) % 2];
     float* dxl = (l == 0) ? dX : gx[l % 2];
-    s = layer_front16<T>(h, l, xin, lcbx[l], B, st);
+    if (l == L - 1) s = layer_front16<T>(h, l, xin, lcbx[l], B, st);  // the others were saved
+    const Acts& act = acts[l];
     if (s == WK_OK) s = to_f32<T>(h, xin, Xf, B * static_cast<int64_t>(nd), st);
     if (s == WK_OK) s = to_f32<T>(h, h->WL[l], WLf, static_cast<int64_t>(n_l) * n, st);
     if (s == WK_OK) s = to_f32<T>(h, h->Y[l], Yf, static_cast<int64_t>(nk), st);
@@ -1472,7 +1505,7 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     {
       const int grid = static_cast<int>(std::min<int64_t>((rows + 7) / 8, dv->sms * 8ll));
       ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
-      bw_out_ln_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(h->cat), xin, up_grad, h->g2[l], dyf, dxl, dz[0],
+      bw_out_ln_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(act.cat), xin, up_grad, h->g2[l], dyf, dxl, dz[0],
                                                  g.out_ln_gamma, g.out_ln_beta, rows, n, n_f, d, h->eps);
       s = launch_status();
     }
@@ -1490,12 +1523,12 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     int cur = 0;
     for (int j = m - 1; j >= 0 && s == WK_OK; --j) {
       const int64_t hin = dims[j], hout = dims[j + 1];
-      const void* hj = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
+      const void* hj = (j == 0) ? act.A0 : act.H[j - 1];
       if (j < m - 1) {  // the ReLU of Linear j: its output h_{j+1} was > 0
         const int64_t cnt = B * hout;
         const int grid = static_cast<int>(std::min<int64_t>((cnt / 8 + 255) / 256, dv->sms * 16ll));
         ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
-        bw_relu_mask_kernel<T><<<grid, 256, 0, st>>>(dz[cur], static_cast<const T*>(h->H[j % 2]), cnt);
+        bw_relu_mask_kernel<T><<<grid, 256, 0, st>>>(dz[cur], static_cast<const T*>(act.H[j]), cnt);
         s = launch_status();
       }
       if (s == WK_OK) {
