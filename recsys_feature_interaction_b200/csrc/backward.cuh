@@ -44,84 +44,102 @@ __global__ void __launch_bounds__(256) bw_to_f32_kernel(const T* __restrict__ in
 
 // ------------------------------------------------ output LayerNorm, per row
 
-// One warp per embedding row of d (a multiple of 32, at most 256) values.
+// One warp per embedding row of d (even, at most 256) values, lane l holding the column pairs
+// l + 32 i; every load of a row (cat, X, dOut, gamma2) is issued before its first reduction,
+// so a row costs one memory round trip. Rows r = b n + i; the FMB rows i < n_f also give the
+// MLP's upstream gradient (16-bit, [b][i][c] of the last Linear's output).
 template <typename T>
-__global__ void __launch_bounds__(256) bw_out_ln_kernel(const T* __restrict__ cat, const T* __restrict__ X,
-                                                        const float* __restrict__ dOut, const float* __restrict__ g2,
-                                                        float* __restrict__ dy, float* __restrict__ dx,
-                                                        T* __restrict__ dh_m, float* __restrict__ dg2,
-                                                        float* __restrict__ db2, int64_t rows, int n, int n_f, int d,
-                                                        float eps) {
-  __shared__ float sg[8][256], sb[8][256];
+__global__ void __launch_bounds__(256, 4) bw_out_ln_kernel(const T* __restrict__ cat, const T* __restrict__ X,
+                                                           const float* __restrict__ dOut,
+                                                           const float* __restrict__ g2, float* __restrict__ dy,
+                                                           float* __restrict__ dx, T* __restrict__ dh_m,
+                                                           float* __restrict__ dg2, float* __restrict__ db2,
+                                                           int rows, int n, int n_f, int d, float eps) {
+  __shared__ float2 sg[8][128], sb[8][128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = d >> 5;  // values per lane, columns lane + 32 i
-  float ag[8], ab[8];
+  const int pairs = d >> 1;
+  float2 ag[4], ab[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ag[i] = ab[i] = 0.f;
+  for (int i = 0; i < 4; ++i) ag[i] = ab[i] = make_float2(0.f, 0.f);
   const float inv_d = 1.f / static_cast<float>(d);
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp; r < rows; r += static_cast<int64_t>(gridDim.x) * 8) {
-    float y[8], go[8];
+  for (int r = blockIdx.x * 8 + warp; r < rows; r += gridDim.x * 8) {
+    const int64_t o = static_cast<int64_t>(r) * d;
+    float2 y[4], go[4];
     float s = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      y[i] = 0.f;
-      if (i < per) {
-        const int64_t o = r * d + lane + 32 * i;
-        y[i] = bw_ld(cat + o) + bw_ld(X + o);
-        s += y[i];
+    for (int i = 0; i < 4; ++i) {
+      const int q = lane + 32 * i;
+      y[i] = go[i] = make_float2(0.f, 0.f);
+      if (q < pairs) {
+        const uint32_t c2 = __ldg(reinterpret_cast<const unsigned int*>(cat + o) + q);
+        const uint32_t x2 = __ldg(reinterpret_cast<const unsigned int*>(X + o) + q);
+        go[i] = __ldg(reinterpret_cast<const float2*>(dOut + o) + q);
+        y[i].x = Half16<T>::lo(c2) + Half16<T>::lo(x2);
+        y[i].y = Half16<T>::hi(c2) + Half16<T>::hi(x2);
+        s += y[i].x + y[i].y;
       }
     }
     const float mean = warp_sum(s) * inv_d;
     float v = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (i < per) v += (y[i] - mean) * (y[i] - mean);
+    for (int i = 0; i < 4; ++i)
+      if (lane + 32 * i < pairs) {
+        const float a = y[i].x - mean, b = y[i].y - mean;
+        v += a * a + b * b;
+      }
     const float rs = rsqrtf(warp_sum(v) * inv_d + eps);
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i < per) {
-        const int c = lane + 32 * i;
-        const float dO = __ldg(dOut + r * d + c);
-        y[i] = (y[i] - mean) * rs;  // yhat
-        ag[i] += dO * y[i];
-        ab[i] += dO;
-        go[i] = dO * __ldg(g2 + c);
-        s1 += go[i];
-        s2 += go[i] * y[i];
+    for (int i = 0; i < 4; ++i) {
+      const int q = lane + 32 * i;
+      if (q < pairs) {
+        const float2 g = __ldg(reinterpret_cast<const float2*>(g2) + q);
+        y[i].x = (y[i].x - mean) * rs;  // yhat
+        y[i].y = (y[i].y - mean) * rs;
+        ag[i].x += go[i].x * y[i].x;
+        ag[i].y += go[i].y * y[i].y;
+        ab[i].x += go[i].x;
+        ab[i].y += go[i].y;
+        go[i].x *= g.x;
+        go[i].y *= g.y;
+        s1 += go[i].x + go[i].y;
+        s2 += go[i].x * y[i].x + go[i].y * y[i].y;
       }
     }
     const float m1 = warp_sum(s1) * inv_d, m2 = warp_sum(s2) * inv_d;
-    const int64_t b = r / n;
-    const int i_row = static_cast<int>(r - b * n);
+    const int b = r / n, i_row = r - b * n;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i < per) {
-        const int c = lane + 32 * i;
-        const float g = rs * (go[i] - m1 - y[i] * m2);
-        dy[r * d + c] = tf32_round(g);  // read only by the tf32 contractions
-        dx[r * d + c] = g;  // the residual's share of dX
-        if (i_row < n_f) dh_m[(b * n_f + i_row) * d + c] = Half16<T>::from(g);
+    for (int i = 0; i < 4; ++i) {
+      const int q = lane + 32 * i;
+      if (q < pairs) {
+        const float gx = rs * (go[i].x - m1 - y[i].x * m2), gy = rs * (go[i].y - m1 - y[i].y * m2);
+        reinterpret_cast<float2*>(dy + o)[q] = make_float2(tf32_round(gx), tf32_round(gy));  // tf32 operand
+        reinterpret_cast<float2*>(dx + o)[q] = make_float2(gx, gy);  // the residual's share of dX
+        if (i_row < n_f)
+          reinterpret_cast<unsigned int*>(dh_m + (static_cast<int64_t>(b) * n_f + i_row) * d)[q] =
+              Half16<T>::pack2(gx, gy);
       }
     }
   }
   // this CTA's partial d gamma2, d beta2
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (i < per) {
+  for (int i = 0; i < 4; ++i)
+    if (lane + 32 * i < pairs) {
       sg[warp][lane + 32 * i] = ag[i];
       sb[warp][lane + 32 * i] = ab[i];
     }
   __syncthreads();
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float a = 0.f, bsum = 0.f;
+  for (int q = threadIdx.x; q < pairs; q += blockDim.x) {
+    float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-      a += sg[w][c];
-      bsum += sb[w][c];
+      a.x += sg[w][q].x, a.y += sg[w][q].y;
+      c.x += sb[w][q].x, c.y += sb[w][q].y;
     }
-    atomicAdd(dg2 + c, a);
-    atomicAdd(db2 + c, bsum);
+    atomicAdd(dg2 + 2 * q, a.x);
+    atomicAdd(dg2 + 2 * q + 1, a.y);
+    atomicAdd(db2 + 2 * q, c.x);
+    atomicAdd(db2 + 2 * q + 1, c.y);
   }
 }
 
@@ -214,6 +232,67 @@ __global__ void __launch_bounds__(256) bw_fmb_ln_kernel(const float* __restrict_
   for (int i = threadIdx.x; i < nk; i += blockDim.x) {
     const float fh = (F[base + i] - mean) * rs;
     dF[base + i] = tf32_round(rs * (bw_ld(dfh + base + i) - m1 - fh * m2));  // a tf32 operand
+  }
+}
+
+// The same with the example in registers (nk a multiple of 4, at most 2048 V): 512 threads,
+// V / 4 float4 of F and 4-value groups of dfh per thread, read once; the statistics are
+// two-pass over the registers.
+template <typename T, int V>
+__global__ void __launch_bounds__(512, 1) bw_fmb_ln_reg_kernel(const float* __restrict__ F,
+                                                               const T* __restrict__ dfh, float* __restrict__ dF,
+                                                               int nk, float eps) {
+  __shared__ float red[16];
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * nk;
+  const float inv = 1.f / static_cast<float>(nk);
+  float4 f[V / 4];
+  uint2 g[V / 4];
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < V / 4; ++j) {
+    const int e = (j * 512 + static_cast<int>(threadIdx.x)) * 4;
+    f[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    g[j] = make_uint2(0u, 0u);
+    if (e < nk) {
+      f[j] = __ldg(reinterpret_cast<const float4*>(F + base + e));
+      g[j] = __ldg(reinterpret_cast<const uint2*>(dfh + base + e));
+      s += f[j].x + f[j].y + f[j].z + f[j].w;
+    }
+  }
+  const float mean = bw_block_sum(s, red) * inv;
+  float v = 0.f;
+#pragma unroll
+  for (int j = 0; j < V / 4; ++j) {
+    if ((j * 512 + static_cast<int>(threadIdx.x)) * 4 < nk) {
+      f[j].x -= mean, f[j].y -= mean, f[j].z -= mean, f[j].w -= mean;
+      v += f[j].x * f[j].x + f[j].y * f[j].y + f[j].z * f[j].z + f[j].w * f[j].w;
+    }
+  }
+  const float rs = rsqrtf(bw_block_sum(v, red) * inv + eps);
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int j = 0; j < V / 4; ++j) {
+    if ((j * 512 + static_cast<int>(threadIdx.x)) * 4 < nk) {
+      f[j].x *= rs, f[j].y *= rs, f[j].z *= rs, f[j].w *= rs;  // fhat
+      const float g0 = Half16<T>::lo(g[j].x), g1 = Half16<T>::hi(g[j].x), g2 = Half16<T>::lo(g[j].y),
+                  g3 = Half16<T>::hi(g[j].y);
+      s1 += g0 + g1 + g2 + g3;
+      s2 += g0 * f[j].x + g1 * f[j].y + g2 * f[j].z + g3 * f[j].w;
+    }
+  }
+  const float m1 = bw_block_sum(s1, red) * inv, m2 = bw_block_sum(s2, red) * inv;
+#pragma unroll
+  for (int j = 0; j < V / 4; ++j) {
+    const int e = (j * 512 + static_cast<int>(threadIdx.x)) * 4;
+    if (e < nk) {
+      const float g0 = Half16<T>::lo(g[j].x), g1 = Half16<T>::hi(g[j].x), g2 = Half16<T>::lo(g[j].y),
+                  g3 = Half16<T>::hi(g[j].y);
+      // tf32 operands of the contractions
+      *reinterpret_cast<float4*>(dF + base + e) = make_float4(tf32_round(rs * (g0 - m1 - f[j].x * m2)),
+                                                              tf32_round(rs * (g1 - m1 - f[j].y * m2)),
+                                                              tf32_round(rs * (g2 - m1 - f[j].z * m2)),
+                                                              tf32_round(rs * (g3 - m1 - f[j].w * m2)));
+    }
   }
 }
 

@@ -53,25 +53,29 @@ struct TcContr {
 };
 
 struct TcMaps {
-  CUtensorMap m[6];  // A and B of each term
+  CUtensorMap m[7];  // A and B of each term; C (fp32, 32-column x 128-row boxes) when read by TMA
 };
 
 constexpr int TC_BK = 32;  // k per block: one 128-byte row of fp32
 constexpr int TC_THREADS = 192;
 constexpr int TC_ABYTES = 128 * TC_BK * 4;
 
-template <int BN>
+// CIN: C is read (TC_ACCUM) through a TMA prefetch of the tile into shared memory, issued
+// when the epilogue starts waiting for the tile's accumulator, instead of by the epilogue's
+// own global loads (which stalled it); the ring gives up stages for the buffer.
+template <int BN, bool CIN = false>
 struct TcCfg {
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 160, "BN: 64..160, whole 32-row boxes");
   static constexpr int BBYTES = BN * TC_BK * 4;
   static constexpr int STAGE = TC_ABYTES + BBYTES;
-  static constexpr int STAGES = (196 * 1024) / STAGE;
+  static constexpr int CBYTES = CIN ? 128 * BN * 4 : 0;  // BN / 32 boxes of 32 columns x 128 rows
+  static constexpr int STAGES = (196 * 1024 - CBYTES) / STAGE;
   static constexpr int TCOLS = BN <= 64 ? 64 : BN <= 128 ? 128 : 256;  // per accumulator
   static constexpr int BARB = 256;
-  static constexpr int SMEM = STAGES * STAGE + BARB + 1024;  // and 1024 bytes of alignment slack
+  static constexpr int SMEM = STAGES * STAGE + CBYTES + BARB + 1024;  // and 1024 bytes of alignment slack
   static constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                                     (static_cast<uint32_t>(128 >> 4) << 24);
-  static_assert(2 * TCOLS <= 512 && SMEM <= 232448 && (2 * STAGES + 4) * 8 + 4 <= BARB, "resources");
+  static_assert(STAGES >= 3 && 2 * TCOLS <= 512 && SMEM <= 232448 && (2 * STAGES + 6) * 8 + 4 <= BARB, "resources");
 };
 
 __device__ __forceinline__ void tma_load_4d(const CUtensorMap* m, uint64_t* bar, uint32_t dst, int32_t c0, int32_t c1,
@@ -133,8 +137,9 @@ __device__ __forceinline__ void tc_load_operand(const CUtensorMap* m, uint64_t* 
   }
 }
 
-template <int BN>
-__device__ __forceinline__ void tc_epilogue(const TcContr& p, const TcTile& tl, uint32_t taddr, int q, int lane) {
+template <int BN, bool CIN>
+__device__ __forceinline__ void tc_epilogue(const TcContr& p, const TcTile& tl, uint32_t taddr, int q, int lane,
+                                            const uint8_t* cbuf) {
   const int r = 32 * q + lane, n0 = tl.ni * BN;
   const int rows_a = min(128, p.M - tl.m0), rows_b = min(BN, p.N - n0);
   float* crow = p.C + tl.z * p.sCz + (tl.m0 + r) * p.sCm;
@@ -160,7 +165,9 @@ __device__ __forceinline__ void tc_epilogue(const TcContr& p, const TcTile& tl, 
           atomicAdd(dst + j, x);
         } else {
           if (p.mode == TC_ACCUM) {
-            const float4 o = dst[j];
+            // CIN: the prefetched tile, box ch, row r at r * 128, chunk j at (j ^ (r & 7)) * 16
+            const float4 o = CIN ? *reinterpret_cast<const float4*>(cbuf + ch * 16384 + r * 128 + ((j ^ (r & 7)) << 4))
+                                 : dst[j];
             x.x += o.x, x.y += o.y, x.z += o.z, x.w += o.w;
           }
           dst[j] = x;
@@ -172,32 +179,43 @@ __device__ __forceinline__ void tc_epilogue(const TcContr& p, const TcTile& tl, 
         if (32 * ch + j >= rows_b) break;
         float* dst = crow + (nb + j) * p.sCn;
         const float x = __uint_as_float(v[j]);
-        if (p.mode == TC_ATOMIC)
+        if (p.mode == TC_ATOMIC) {
           atomicAdd(dst, x);
-        else
-          *dst = (p.mode == TC_ACCUM) ? *dst + x : x;
+        } else if (p.mode == TC_ACCUM) {
+          const int cj = j >> 2;
+          *dst = x + (CIN ? reinterpret_cast<const float*>(cbuf + ch * 16384 + r * 128 + ((cj ^ (r & 7)) << 4))[j & 3]
+                          : *dst);
+        } else {
+          *dst = x;
+        }
       }
     }
   }
 }
 
-template <int BN>
+template <int BN, bool CIN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     bw_tc_contract_kernel(const __grid_constant__ TcMaps mp, const __grid_constant__ TcContr p) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, CIN>;
   extern __shared__ uint8_t tc_smem_raw[];
   const uint32_t sbase = (smem_u32(tc_smem_raw) + 1023u) & ~1023u;
   uint8_t* gbase = tc_smem_raw + (sbase - smem_u32(tc_smem_raw));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + C::STAGES * C::STAGE);
+  uint8_t* cbuf = gbase + C::STAGES * C::STAGE;  // CIN: the prefetched C tile
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cbuf + C::CBYTES);
   uint64_t* full = bars;                        // [STAGES] TMA -> MMA
   uint64_t* empty = bars + C::STAGES;           // [STAGES] MMA -> TMA
   uint64_t* tfull = bars + 2 * C::STAGES;       // [2] MMA -> epilogue
   uint64_t* tempty = bars + 2 * C::STAGES + 2;  // [2] epilogue -> MMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 4);
+  uint64_t* cfull = bars + 2 * C::STAGES + 4;    // CIN: C tile landed
+  uint64_t* cempty = bars + 2 * C::STAGES + 5;   // CIN: the 4 epilogue warps are done with it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 6);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * p.nterms; ++i) prefetch_tmap(&mp.m[i]);
+    if (CIN) prefetch_tmap(&mp.m[6]);
+    mbar_init(cfull, 1);
+    mbar_init(cempty, 4);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -312,22 +330,45 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quarter this warp may access
-    int acc = 0;
+    const bool c_issuer = CIN && warp == 2 && lane == 0;
+    int acc = 0, nt = 0;
     uint32_t acc_ph = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    bool c_owed = false;  // a C prefetch this thread issued has not been waited for
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++nt) {
       const TcTile tl = tc_tile(p, tile);
-      if (!mbar_wait(&tfull[acc], acc_ph, p.status)) break;
+      // the lanes of a warp leave together (the TMEM loads below are warp-collective)
+      bool ok = true;
+      if (c_issuer) {  // the tile's C, once every epilogue warp is done with the previous one
+        ok = nt == 0 || mbar_wait(cempty, static_cast<uint32_t>((nt - 1) & 1), p.status);
+        if (ok) {
+          mbar_arrive_expect_tx(cfull, C::CBYTES);
+          for (int ch = 0; ch < BN / 32; ++ch)
+            tma_load_3d(&mp.m[6], cfull, cbuf + ch * 16384, tl.ni * BN + 32 * ch, tl.m0, tl.z);
+          c_owed = true;
+        }
+      }
+      ok = ok && mbar_wait(&tfull[acc], acc_ph, p.status);
+      if (CIN && ok) {
+        ok = mbar_wait(cfull, static_cast<uint32_t>(nt & 1), p.status);
+        if (ok) c_owed = false;
+      }
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      tc_epilogue<BN>(p, tl, tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * C::TCOLS),
-                      q, lane);
+      tc_epilogue<BN, CIN>(p, tl,
+                           tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * C::TCOLS),
+                           q, lane, cbuf);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        mbar_arrive(&tempty[acc]);
+        if (CIN) mbar_arrive(cempty);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_ph ^= 1u;
       }
     }
+    if (c_owed) mbar_drain(cfull, static_cast<uint32_t>(nt & 1), p.status);  // lands before exit
   }
   tc_fence_before();
   __syncthreads();

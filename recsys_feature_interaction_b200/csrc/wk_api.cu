@@ -1279,14 +1279,19 @@ bool tc_map(const DevInfo* dv, CUtensorMap* m, const float* ptr, int64_t rows, i
   return make_map(dv, m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, str, box, sw);
 }
 
-template <int BN>
+template <int BN, bool CIN>
 wk_status launch_tc_contract(const DevInfo* dv, const TcMaps& mp, const TcContr& p, cudaStream_t st) {
-  using Cfg = TcCfg<BN>;
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(bw_tc_contract_kernel<BN>), Cfg::SMEM);
+  using Cfg = TcCfg<BN, CIN>;
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(bw_tc_contract_kernel<BN, CIN>), Cfg::SMEM);
   if (s != WK_OK) return s;
   const int grid = std::min(p.num_tiles, dv->sms);
-  bw_tc_contract_kernel<BN><<<grid, TC_THREADS, Cfg::SMEM, st>>>(mp, p);
+  bw_tc_contract_kernel<BN, CIN><<<grid, TC_THREADS, Cfg::SMEM, st>>>(mp, p);
   return launch_status();
+}
+
+template <int BN>
+wk_status launch_tc_contract(const DevInfo* dv, const TcMaps& mp, const TcContr& p, bool cin, cudaStream_t st) {
+  return cin ? launch_tc_contract<BN, true>(dv, mp, p, st) : launch_tc_contract<BN, false>(dv, mp, p, st);
 }
 
 // The strided contraction on the tensor cores (tf32 operands, fp32 accumulation).
@@ -1313,11 +1318,22 @@ wk_status run_tc_contract(wk_stack* h, TcContr p, cudaStream_t st) {
   p.num_tiles = static_cast<int>(tiles);
   p.c_vec = p.sCn == 1 && reinterpret_cast<uintptr_t>(p.C) % 16 == 0 && p.sCm % 4 == 0 && p.sCz % 4 == 0;
   p.status = h->status;
+  // C read by a TMA prefetch of each tile (accumulating launches): C [Z][M][N] with the
+  // 128B-swizzled boxes of 32 columns x 128 rows the epilogue reads
+  bool cin = false;
+  if (p.mode == TC_ACCUM && p.c_vec) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.M), static_cast<uint64_t>(p.Z)};
+    const uint64_t str[2] = {static_cast<uint64_t>(p.sCm) * 4,
+                             p.Z > 1 ? static_cast<uint64_t>(p.sCz) * 4 : static_cast<uint64_t>(p.sCm) * 4 * p.M};
+    const uint32_t box[3] = {32, 128, 1};
+    cin = str[0] > 0 && str[1] > 0 && str[1] % 16 == 0 &&
+          make_map(h->dv, &mp.m[6], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.C, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
   ProfScope ps(h, WK_KERNEL_BW_CONTRACT, st);
   switch (bn) {
-    case 64: return launch_tc_contract<64>(h->dv, mp, p, st);
-    case 160: return launch_tc_contract<160>(h->dv, mp, p, st);
-    default: return launch_tc_contract<128>(h->dv, mp, p, st);
+    case 64: return launch_tc_contract<64>(h->dv, mp, p, cin, st);
+    case 160: return launch_tc_contract<160>(h->dv, mp, p, cin, st);
+    default: return launch_tc_contract<128>(h->dv, mp, p, cin, st);
   }
 }
 
@@ -1503,10 +1519,11 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     for (int j = 0; j < m; ++j) cudaMemsetAsync(g.b[j], 0, static_cast<size_t>(dims[j + 1]) * 4, st);
     // output LayerNorm, residual: dy, dX = dy, the FMB rows of dy as the MLP's gradient
     {
-      const int grid = static_cast<int>(std::min<int64_t>((rows + 7) / 8, dv->sms * 8ll));
+      const int grid = static_cast<int>(std::min<int64_t>((rows + 7) / 8, dv->sms * 4ll));
       ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
       bw_out_ln_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(act.cat), xin, up_grad, h->g2[l], dyf, dxl, dz[0],
-                                                 g.out_ln_gamma, g.out_ln_beta, rows, n, n_f, d, h->eps);
+                                                 g.out_ln_gamma, g.out_ln_beta, static_cast<int>(rows), n, n_f, d,
+                                                 h->eps);
       s = launch_status();
     }
     // LCB: dW_L = sum_b dG_b X_b^T (dG = rows n_f.. of dy; W_L^T dG_b joins dX below)
@@ -1590,7 +1607,18 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     }
     if (s == WK_OK) {
       ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
-      bw_fmb_ln_kernel<T><<<static_cast<unsigned>(B), 256, 0, st>>>(Fb, dz[cur], dFb, static_cast<int>(nk), h->eps);
+      const unsigned grid = static_cast<unsigned>(B);
+      const int nki = static_cast<int>(nk);
+      if (nk % 4 != 0 || nk > 32768)
+        bw_fmb_ln_kernel<T><<<grid, 256, 0, st>>>(Fb, dz[cur], dFb, nki, h->eps);
+      else if (nk <= 4096)
+        bw_fmb_ln_reg_kernel<T, 8><<<grid, 512, 0, st>>>(Fb, dz[cur], dFb, nki, h->eps);
+      else if (nk <= 8192)
+        bw_fmb_ln_reg_kernel<T, 16><<<grid, 512, 0, st>>>(Fb, dz[cur], dFb, nki, h->eps);
+      else if (nk <= 16384)
+        bw_fmb_ln_reg_kernel<T, 32><<<grid, 512, 0, st>>>(Fb, dz[cur], dFb, nki, h->eps);
+      else
+        bw_fmb_ln_reg_kernel<T, 64><<<grid, 512, 0, st>>>(Fb, dz[cur], dFb, nki, h->eps);
       s = launch_status();
     }
     if (s == WK_OK) {
