@@ -164,6 +164,48 @@ __global__ void bw_relu_mask_kernel(T* __restrict__ dh, const T* __restrict__ h,
   }
 }
 
+// The bias gradient of a Linear, with the ReLU derivative of its output applied first when h
+// (the Linear's forward output) is given: z[r, c] = 0 where h[r, c] <= 0 (written back), then
+// out[c] += sum over rows [r0, r1) of z[r, c]. Eight columns per thread (cols % 8 == 0),
+// gridDim.x column blocks of 2048, gridDim.y row chunks.
+template <typename T>
+__global__ void __launch_bounds__(256) bw_mask_colsum_kernel(T* __restrict__ z, const T* __restrict__ h,
+                                                             float* __restrict__ out, int64_t rows, int cols) {
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (c >= cols) return;
+  const int64_t chunk = (rows + gridDim.y - 1) / gridDim.y;
+  const int64_t r0 = blockIdx.y * chunk, r1 = min(rows, r0 + chunk);
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int64_t r = r0; r < r1; ++r) {
+    uint4* zp = reinterpret_cast<uint4*>(z + r * cols + c);
+    uint4 g = *zp;
+    uint32_t* gw = reinterpret_cast<uint32_t*>(&g);
+    if (h) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(h + r * cols + c));
+      const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t mask = 0u;
+        if (Half16<T>::lo(aw[j]) > 0.f) mask |= 0x0000FFFFu;
+        if (Half16<T>::hi(aw[j]) > 0.f) mask |= 0xFFFF0000u;
+        gw[j] &= mask;
+      }
+      *zp = g;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[2 * j] += Half16<T>::lo(gw[j]);
+      acc[2 * j + 1] += Half16<T>::hi(gw[j]);
+    }
+  }
+  if (r1 > r0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) atomicAdd(out + c + j, acc[j]);
+  }
+}
+
 // out[c] += sum over rows [r0, r1) of z[r, c]; blockDim 256 columns, gridDim.y row chunks.
 template <typename T>
 __global__ void bw_colsum_kernel(const T* __restrict__ z, float* __restrict__ out, int64_t rows, int cols) {
@@ -322,6 +364,38 @@ __global__ void bw_unfold_kernel(float* __restrict__ dW0, const float* __restric
   if (r1 > r0) {
     atomicAdd(dg1 + c, sg);
     atomicAdd(db1 + c, sb);
+  }
+}
+
+// The same, four columns per thread (cols % 4 == 0), rows unrolled by two.
+template <typename TW>
+__global__ void __launch_bounds__(256) bw_unfold4_kernel(float* __restrict__ dW0, const float* __restrict__ db0,
+                                                         const TW* __restrict__ W0, const float* __restrict__ g1,
+                                                         const float* __restrict__ b1, float* __restrict__ dg1,
+                                                         float* __restrict__ db1, int rows, int cols) {
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (c >= cols) return;
+  const int chunk = (rows + gridDim.y - 1) / gridDim.y;
+  const int r0 = blockIdx.y * chunk, r1 = min(rows, r0 + chunk);
+  const float4 gc = g1 ? __ldg(reinterpret_cast<const float4*>(g1 + c)) : make_float4(1.f, 1.f, 1.f, 1.f);
+  const float4 bc = b1 ? __ldg(reinterpret_cast<const float4*>(b1 + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 sg = make_float4(0.f, 0.f, 0.f, 0.f), sb = sg;
+#pragma unroll 2
+  for (int r = r0; r < r1; ++r) {
+    const int64_t o = static_cast<int64_t>(r) * cols + c;
+    const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(W0 + o));
+    const float w0 = Half16<TW>::lo(w2.x), w1 = Half16<TW>::hi(w2.x), w2f = Half16<TW>::lo(w2.y),
+                w3 = Half16<TW>::hi(w2.y);
+    float4* gp = reinterpret_cast<float4*>(dW0 + o);
+    const float4 gw = *gp;
+    const float gb = __ldg(db0 + r);
+    sg.x += gw.x * w0, sg.y += gw.y * w1, sg.z += gw.z * w2f, sg.w += gw.w * w3;
+    sb.x += gb * w0, sb.y += gb * w1, sb.z += gb * w2f, sb.w += gb * w3;
+    *gp = make_float4(gw.x * gc.x + gb * bc.x, gw.y * gc.y + gb * bc.y, gw.z * gc.z + gb * bc.z, gw.w * gc.w + gb * bc.w);
+  }
+  if (r1 > r0) {
+    atomicAdd(dg1 + c, sg.x), atomicAdd(dg1 + c + 1, sg.y), atomicAdd(dg1 + c + 2, sg.z), atomicAdd(dg1 + c + 3, sg.w);
+    atomicAdd(db1 + c, sb.x), atomicAdd(db1 + c + 1, sb.y), atomicAdd(db1 + c + 2, sb.z), atomicAdd(db1 + c + 3, sb.w);
   }
 }
 

@@ -155,10 +155,11 @@ __device__ __forceinline__ void tc_epilogue(const TcContr& p, const TcTile& tl, 
       for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(tf32_round(__uint_as_float(v[j])));
     }
     const int nb = n0 + 32 * ch;
-    if (p.c_vec && 32 * ch + 32 <= rows_b) {
+    if (p.c_vec && (32 * ch + 32 <= rows_b || rows_b % 4 == 0)) {  // whole float4s up to rows_b
       float4* dst = reinterpret_cast<float4*>(crow + nb);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        if (32 * ch + 4 * j >= rows_b) break;
         float4 x = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
                                __uint_as_float(v[4 * j + 3]));
         if (p.mode == TC_ATOMIC) {

@@ -1541,18 +1541,30 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     for (int j = m - 1; j >= 0 && s == WK_OK; --j) {
       const int64_t hin = dims[j], hout = dims[j + 1];
       const void* hj = (j == 0) ? act.A0 : act.H[j - 1];
-      if (j < m - 1) {  // the ReLU of Linear j: its output h_{j+1} was > 0
-        const int64_t cnt = B * hout;
-        const int grid = static_cast<int>(std::min<int64_t>((cnt / 8 + 255) / 256, dv->sms * 16ll));
+      // the ReLU of Linear j (j < m - 1: its output h_{j+1} was > 0) applied to dz, then the
+      // bias gradient (column sums over the batch), in one pass
+      const T* relu_out = (j < m - 1) ? static_cast<const T*>(act.H[j]) : nullptr;
+      if (hout % 8 == 0) {
+        const unsigned gx = static_cast<unsigned>((hout + 2047) / 2048);
+        // at most 64 row chunks: every chunk adds into each column of the bias gradient
+        const unsigned gy = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>({B, 64ll, 4ll * dv->sms / gx})));
         ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
-        bw_relu_mask_kernel<T><<<grid, 256, 0, st>>>(dz[cur], static_cast<const T*>(act.H[j]), cnt);
+        bw_mask_colsum_kernel<T><<<dim3(gx, gy), 256, 0, st>>>(dz[cur], relu_out, g.b[j], B, static_cast<int>(hout));
         s = launch_status();
-      }
-      if (s == WK_OK) {
-        const dim3 grid(static_cast<unsigned>((hout + 255) / 256), static_cast<unsigned>(std::min<int64_t>(B, 64)));
-        ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
-        bw_colsum_kernel<T><<<grid, 256, 0, st>>>(dz[cur], g.b[j], B, static_cast<int>(hout));
-        s = launch_status();
+      } else {
+        if (relu_out) {
+          const int64_t cnt = B * hout;
+          const int grid = static_cast<int>(std::min<int64_t>((cnt / 8 + 255) / 256, dv->sms * 16ll));
+          ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
+          bw_relu_mask_kernel<T><<<grid, 256, 0, st>>>(dz[cur], relu_out, cnt);
+          s = launch_status();
+        }
+        if (s == WK_OK) {
+          const dim3 grid(static_cast<unsigned>((hout + 255) / 256), static_cast<unsigned>(std::min<int64_t>(B, 64)));
+          ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
+          bw_colsum_kernel<T><<<grid, 256, 0, st>>>(dz[cur], g.b[j], B, static_cast<int>(hout));
+          s = launch_status();
+        }
       }
       // dW_j = dz^T h_j (K = batch): on the pair GEMM both read MN-major, else transposed
       // to K-major for the one-CTA GEMM
@@ -1578,10 +1590,20 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
     }
     // the folded first Linear: gradients of the caller's W0, gamma1, beta1 (b0 = b0')
     if (s == WK_OK) {
-      const dim3 grid(static_cast<unsigned>((dims[0] + 255) / 256), static_cast<unsigned>(std::min(dims[1], 64)));
       ProfScope ps(h, WK_KERNEL_BW_ROWS, st);
-      bw_unfold_kernel<IO><<<grid, 256, 0, st>>>(g.W[0], g.b[0], static_cast<const IO*>(h->W0_in[l]), h->g1_in[l],
-                                                 h->b1_in[l], g.fmb_ln_gamma, g.fmb_ln_beta, dims[1], dims[0]);
+      auto al = [](const void* q, uintptr_t a) { return reinterpret_cast<uintptr_t>(q) % a == 0; };
+      if (dims[0] % 4 == 0 && al(g.W[0], 16) && al(h->W0_in[l], 8) && al(h->g1_in[l], 16) && al(h->b1_in[l], 16)) {
+        const unsigned gx = static_cast<unsigned>((dims[0] / 4 + 255) / 256);
+        const unsigned gy =
+            static_cast<unsigned>(std::max(1, std::min({dims[1], 64, static_cast<int>(4 * dv->sms / gx)})));
+        bw_unfold4_kernel<IO><<<dim3(gx, gy), 256, 0, st>>>(g.W[0], g.b[0], static_cast<const IO*>(h->W0_in[l]),
+                                                            h->g1_in[l], h->b1_in[l], g.fmb_ln_gamma, g.fmb_ln_beta,
+                                                            dims[1], dims[0]);
+      } else {
+        const dim3 grid(static_cast<unsigned>((dims[0] + 255) / 256), static_cast<unsigned>(std::min(dims[1], 64)));
+        bw_unfold_kernel<IO><<<grid, 256, 0, st>>>(g.W[0], g.b[0], static_cast<const IO*>(h->W0_in[l]), h->g1_in[l],
+                                                   h->b1_in[l], g.fmb_ln_gamma, g.fmb_ln_beta, dims[1], dims[0]);
+      }
       s = launch_status();
     }
     // FMB: Z = X^T Y, F = X Z, dF from the LayerNorm backward, then dZ = X^T dF;
