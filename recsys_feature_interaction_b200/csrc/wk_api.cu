@@ -230,11 +230,12 @@ bool gemm2_stream() {
   return on;
 }
 
+// stream: the launch shape (streaming or persistent, see gemm_tc2.cuh); -1 = gemm2_stream().
 template <typename T, typename TO, bool ROWLN = false, bool A_MN = false, bool B_MN = false>
-wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
+wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st, int stream = -1) {
   if (p.num_tiles <= 0) return WK_OK;
   if constexpr (!ROWLN) {
-    if (gemm2_stream()) {
+    if (stream < 0 ? gemm2_stream() : stream != 0) {
       constexpr uint32_t smem = gemm2_smem_bytes<TO, true>();
       wk_status s =
           smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, false, true, A_MN, B_MN>), smem);
@@ -1382,7 +1383,15 @@ wk_status bw_gemm_mn(wk_stack* h, const void* A, int64_t lda, const void* W, int
                   map_out<TO>(dv, &mp.C, C, N, M, N);
   if (!ok) return WK_ERR_UNSUPPORTED;
   ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
-  return run_gemm_tc2<T, TO, false, A_MN, B_MN>(dv, mp, mlp2_params(M, K, N, nullptr, 0, h->status), st);
+  // The weight gradient (K = the batch, fp32 tiles) runs persistent: its two TMEM accumulators
+  // overlap a tile's epilogue with the next tile's main loop, which a short K leaves exposed in
+  // the streaming shape's one accumulator. WK_WGRAD_STREAM=1 in the environment streams it.
+  static const int wgrad_stream = [] {
+    const char* e = getenv("WK_WGRAD_STREAM");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  return run_gemm_tc2<T, TO, false, A_MN, B_MN>(dv, mp, mlp2_params(M, K, N, nullptr, 0, h->status), st,
+                                                (A_MN && B_MN) ? wgrad_stream : -1);
 }
 
 template <typename T>
