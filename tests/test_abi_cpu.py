@@ -92,6 +92,7 @@ def test_create_without_device_reports_cuda_error(L):
 def test_null_handle_and_stand_alone_argument_checks(L):
     assert L.wk_stack_forward(None, FAKE, FAKE * 2, 1, None) == wk.WK_ERR_INVALID_ARG
     assert L.wk_stack_sync_status(None, None) == wk.WK_ERR_INVALID_ARG
+    assert L.wk_stack_backward(None, FAKE, FAKE, FAKE, None, 8, None) == wk.WK_ERR_INVALID_ARG
     L.wk_stack_destroy(None)
     # misaligned pointers and bad sizes are rejected before any launch
     assert L.wk_mlp_linear(FAKE + 2, FAKE, None, FAKE, 4, 64, 64, 64, 0, 1, None) == wk.WK_ERR_INVALID_ARG
