@@ -349,16 +349,19 @@ typedef struct {           /* fp32 DEVICE buffers the backward overwrites, one s
 
 /* X [batch, n, d] in the stack's dtype (the input of the forward whose gradient is
  * wanted); dOut and dX [batch, n, d] fp32; grads: num_layers gradient sets. The forward
- * is run once with every layer's input saved, then each layer's front is recomputed and
- * differentiated, last layer first: the output LayerNorm, the residual and the LCB per
- * row and example; the FMB MLP's input, weight and bias gradients on the tensor-core
- * GEMM (16-bit operands transposed where the contraction needs them, fp32 weight
- * gradients); the FMB LayerNorm and the FM per example. Supported: 16-bit stacks with
- * fp16 operands (the default), at most 3 MLP Linears, batch % 8 == 0, d % 32 == 0 and
- * d <= 256; otherwise WK_ERR_UNSUPPORTED. The first call (or a larger batch) allocates
- * the backward workspace (all layer inputs, fp32 gradients of the layer stream, the
- * MLP gradients and their transposes). Asynchronous on `stream` apart from that
- * allocation; not re-entrant (shares the forward's workspace). */
+ * is run once with every layer's input and activations saved (the FMB LayerNorm output,
+ * the hidden ReLU outputs, the concat buffer), then each layer is differentiated, last
+ * layer first: the output LayerNorm and the residual per row; the FMB MLP's input,
+ * weight and bias gradients on the tensor-core GEMM (16-bit operands read MN-major where
+ * the contraction needs their transposes, fp32 weight gradients); the FMB LayerNorm per
+ * example; the FM's and the LCB's products on the tf32 tensor cores (fp32 accumulation).
+ * Supported: 16-bit stacks with fp16 operands (the default), at most 3 MLP Linears,
+ * batch % 8 == 0, d % 32 == 0 and d <= 256; otherwise WK_ERR_UNSUPPORTED. The first call
+ * (or a larger batch) allocates the backward workspace (all layer inputs and
+ * activations, fp32 gradients of the layer stream, the MLP gradients, fp32 copies of X,
+ * W_L and Y; transposed copies only when batch or a hidden width is at most 128).
+ * Asynchronous on `stream` apart from that allocation; not re-entrant (shares the
+ * forward's workspace). */
 WK_API wk_status wk_stack_backward(wk_stack* h, const void* X, const float* dOut, float* dX,
                                    const wk_layer_grads* grads, int64_t batch, wk_stream_t stream);
 
