@@ -374,13 +374,22 @@ def run_backward(args, cfg, rank, world, local, dev):
     gen.manual_seed(1234 + rank)
     dOut = torch.randn((B, n, d), generator=gen, device=dev, dtype=torch.float32)
     dX = torch.empty_like(dOut)
-    z = lambda *sh: torch.empty(sh, dtype=torch.float32, device=dev)
-    grads = [{"Y": z(n, k), "W": [z(dims[j + 1], dims[j]) for j in range(len(dims) - 1)],
-              "b": [z(dims[j + 1]) for j in range(len(dims) - 1)], "fmb_gamma": z(n * k), "fmb_beta": z(n * k),
-              "W_L": z(cfg["n_l"], n), "out_gamma": z(d), "out_beta": z(d)} for _ in range(L)]
+    # the gradients in one flat buffer per layer; with several ranks every step ends with
+    # their average over the ranks (NCCL), layer l's all-reduce on a side stream as soon as
+    # the backward has recorded layer l's event
+    buckets = replicas.GradBuckets(n, d, k, cfg["n_l"], dims, L, device=dev)
+    grads = buckets.grads
     stream = torch.cuda.current_stream(dev)
+    comm = torch.cuda.Stream(dev) if world > 1 else None
+    layer_ev = [torch.cuda.Event() for _ in range(L)] if world > 1 else None
+
+    def train_step():
+        wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream, layer_events=layer_ev)
+        if world > 1:
+            replicas.average_gradients(buckets.flats, layer_ev, comm)
+
     for _ in range(args.warmup):
-        wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+        train_step()
     torch.cuda.synchronize(dev)
     if wk.wk_stack_sync_status(h) != wk.WK_OK:
         raise RuntimeError("device status after warm-up")
@@ -396,13 +405,13 @@ def run_backward(args, cfg, rank, world, local, dev):
         if flush is None:
             evs[0][0].record(stream)
             for _ in range(args.steps):
-                wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+                train_step()
             evs[0][1].record(stream)
         else:
             for a, b in evs:
                 flush.fill_(1)
                 a.record(stream)
-                wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+                train_step()
                 b.record(stream)
         torch.cuda.synchronize(dev)
     replicas.barrier()
@@ -421,7 +430,7 @@ def run_backward(args, cfg, rank, world, local, dev):
     def step_host():
         X.copy_(xh, non_blocking=True)
         dOut.copy_(dh, non_blocking=True)
-        wk.wk_stack_backward(h, X, dOut, dX, grads, stream=stream)
+        train_step()
         dxh.copy_(dX, non_blocking=True)
         stream.synchronize()
     step_host()
@@ -458,7 +467,10 @@ def run_backward(args, cfg, rank, world, local, dev):
                        "precision": "bf16 inputs and weights; fp16 tensor-core operands, activations and MLP "
                                     "gradients; fp32 accumulation, LayerNorm statistics, layer-stream and "
                                     "parameter gradients",
-                       "global_batch": B * world, "seq_len": None, "parallelism": "replicas (batch shards)",
+                       "global_batch": B * world, "seq_len": None,
+                       "parallelism": ("dp%d: batch shards, parameter gradients averaged over the ranks (NCCL "
+                                       "all-reduce per layer, overlapped with the backward of the layers below)"
+                                       % world) if world > 1 else "one GPU",
                        "l2": l2, "launch": "eager, one C-ABI call per step",
                        "flops_per_example": "3 x forward matmul FLOPs = %.4g" % flops_ex},
             "tflops_per_gpu": tflops,

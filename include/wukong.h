@@ -365,6 +365,15 @@ typedef struct {           /* fp32 DEVICE buffers the backward overwrites, one s
 WK_API wk_status wk_stack_backward(wk_stack* h, const void* X, const float* dOut, float* dX,
                                    const wk_layer_grads* grads, int64_t batch, wk_stream_t stream);
 
+/* The same, recording layer_done[l] (a cudaEvent_t created by the caller, or NULL to skip
+ * it; the array itself may be NULL) on `stream` as soon as layer l's parameter gradients
+ * are written. Layers finish last first, so a data-parallel caller can start reducing
+ * layer l's gradients across ranks (on another stream, after that event) while the
+ * layers below it are still being differentiated. Errors as wk_stack_backward. */
+WK_API wk_status wk_stack_backward_events(wk_stack* h, const void* X, const float* dOut, float* dX,
+                                          const wk_layer_grads* grads, int64_t batch, wk_stream_t stream,
+                                          void* const* layer_done);
+
 /* ---- WHALE attention-based fusion ----
  *
  * The WHALE pages (gist.science summaries of arXiv 2607.17017, Korean and French),

@@ -106,6 +106,8 @@ def lib():
             "wk_moe_combine": [ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, i64, i32, i32,
                                i32, ci, cf, vp],
             "wk_stack_backward": [vp, vp, vp, vp, ctypes.POINTER(WkLayerGrads), i64, vp],
+            "wk_stack_backward_events": [vp, vp, vp, vp, ctypes.POINTER(WkLayerGrads), i64, vp,
+                                         ctypes.POINTER(vp)],
             "wk_whale_create": [ctypes.POINTER(WkWhaleConfig), ctypes.POINTER(WkWhaleWeights), ctypes.POINTER(vp)],
             "wk_whale_forward": [vp, vp, vp, vp, i64, vp],
             "wk_whale_sync_status": [vp, vp],
@@ -240,9 +242,11 @@ def wk_stack_sync_status(h, stream=None):
     return lib().wk_stack_sync_status(h.ptr, _stream(stream))
 
 
-def wk_stack_backward(h, X, dOut, dX, grads, batch=None, stream=None):
+def wk_stack_backward(h, X, dOut, dX, grads, batch=None, stream=None, layer_events=None):
     """grads: one mapping per layer with fp32 device tensors Y, W (list of m), b (list of m),
-    fmb_gamma, fmb_beta, W_L, out_gamma, out_beta (overwritten with the gradients)."""
+    fmb_gamma, fmb_beta, W_L, out_gamma, out_beta (overwritten with the gradients).
+    layer_events: optional list of torch.cuda.Event, one per layer (None entries skipped);
+    event l is recorded on the stream once layer l's gradients are written."""
     b = X.shape[0] if batch is None else batch
     arr = (WkLayerGrads * len(grads))()
     keep = []
@@ -252,8 +256,20 @@ def wk_stack_backward(h, X, dOut, dX, grads, batch=None, stream=None):
         keep += [Wp, bp]
         arr[i] = WkLayerGrads(_addr(g["Y"]), Wp, bp, _addr(g["fmb_gamma"]), _addr(g["fmb_beta"]), _addr(g["W_L"]),
                               _addr(g["out_gamma"]), _addr(g["out_beta"]))
-    _check(lib().wk_stack_backward(h.ptr, _addr(X), _addr(dOut), _addr(dX), arr, int(b), _stream(stream, X)),
-           "wk_stack_backward")
+    if layer_events is None:
+        _check(lib().wk_stack_backward(h.ptr, _addr(X), _addr(dOut), _addr(dX), arr, int(b), _stream(stream, X)),
+               "wk_stack_backward")
+        return
+    if len(layer_events) != len(grads):
+        raise ValueError("one event (or None) per layer")
+    import torch
+
+    for e in layer_events:
+        if e is not None and not e.cuda_event:  # torch creates the CUDA event at its first record
+            e.record(stream if stream is not None else torch.cuda.current_stream(X.device))
+    evp = (ctypes.c_void_p * len(layer_events))(*[e.cuda_event if e is not None else None for e in layer_events])
+    _check(lib().wk_stack_backward_events(h.ptr, _addr(X), _addr(dOut), _addr(dX), arr, int(b), _stream(stream, X),
+                                          evp), "wk_stack_backward_events")
 
 
 def wk_stack_destroy(h):

@@ -1408,7 +1408,7 @@ wk_status bw_transpose(wk_stack* h, const void* in, void* out, int64_t R, int64_
 // (A0 = LN(F) normalised, the hidden activations, the concat buffer) before its backward.
 template <typename T, typename IO>
 wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, const wk_layer_grads* gr,
-                     int64_t batch, cudaStream_t st) {
+                     int64_t batch, cudaStream_t st, void* const* layer_done) {
   const wk_stack_config& c = h->cfg;
   const DevInfo* dv = h->dv;
   const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers, n_f = c.n_f, n_l = c.n_l;
@@ -1682,6 +1682,13 @@ wk_status backward16(wk_stack* h, const void* X, const float* dOut, float* dX, c
       p.t[0].sAm = d, p.t[0].sAk1 = nd, p.t[0].sAk2 = 1;  // X(b, i, t)
       p.t[0].sBn = 1, p.t[0].sBk1 = dk, p.t[0].sBk2 = k;  // dZ(b, t, c)
       s = run_tc_contract(h, p, st);
+    }
+    // layer l's parameter gradients are final: a caller may reduce them across ranks while
+    // the layers below are differentiated
+    if (s == WK_OK && layer_done && layer_done[l] &&
+        cudaEventRecord(reinterpret_cast<cudaEvent_t>(layer_done[l]), st) != cudaSuccess) {
+      cudaGetLastError();
+      s = WK_ERR_CUDA;
     }
   }
   return s;
@@ -2167,6 +2174,12 @@ wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream) {
 
 wk_status wk_stack_backward(wk_stack* h, const void* X, const float* dOut, float* dX, const wk_layer_grads* grads,
                             int64_t batch, wk_stream_t stream) {
+  return wk_stack_backward_events(h, X, dOut, dX, grads, batch, stream, nullptr);
+}
+
+wk_status wk_stack_backward_events(wk_stack* h, const void* X, const float* dOut, float* dX,
+                                   const wk_layer_grads* grads, int64_t batch, wk_stream_t stream,
+                                   void* const* layer_done) {
   if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
   if (batch == 0) return WK_OK;
   if (!X || !dOut || !dX || !grads || !al16(X) || !al16(dOut) || !al16(dX)) return WK_ERR_INVALID_ARG;
@@ -2190,8 +2203,8 @@ wk_status wk_stack_backward(wk_stack* h, const void* X, const float* dOut, float
     return WK_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return h->io == WK_BF16 ? backward16<f16, bf16>(h, X, dOut, dX, grads, batch, st)
-                          : backward16<f16, f16>(h, X, dOut, dX, grads, batch, st);
+  return h->io == WK_BF16 ? backward16<f16, bf16>(h, X, dOut, dX, grads, batch, st, layer_done)
+                          : backward16<f16, f16>(h, X, dOut, dX, grads, batch, st, layer_done);
 }
 
 void wk_stack_destroy(wk_stack* h) { free_stack(h); }

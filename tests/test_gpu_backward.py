@@ -150,3 +150,44 @@ def test_backward_rejects_unsupported_batches():
         wk.wk_stack_backward(h, X, dOut, torch.empty_like(dOut), _grads_dev(cfg, dims), batch=12)
     assert ei.value.status == wk.WK_ERR_UNSUPPORTED
     wk.wk_stack_destroy(h)
+
+
+def test_layer_events_mark_final_gradients():
+    """wk_stack_backward with per-layer events: the gradients (written into the flat per-layer
+    buffers a data-parallel step all-reduces) match those of the call without events (bit
+    for bit for dX; the batch sums use atomic adds, whose order varies, so those to 1e-5),
+    and a second stream that waits on layer l's event copies exactly layer l's final
+    gradients while the backward of the layers below runs."""
+    from recsys_feature_interaction_b200 import replicas
+
+    cfg = dict(C.CONFIGS["c2_bf16"], layers=2)
+    dims = C.mlp_dims(cfg)
+    L, batch = cfg["layers"], 16
+    h = wk.wk_stack_create(cfg, [C.make_layer_dev(cfg, l) for l in range(L)], max_batch=batch)
+    X = C.make_x_dev(cfg, batch)
+    dOut = to_dev(host_normal((batch, cfg["n"], cfg["d"]), 133, dtype="f32"))
+    dX0, dX1 = torch.empty_like(dOut), torch.empty_like(dOut)
+    ref = replicas.GradBuckets(cfg["n"], cfg["d"], cfg["k"], cfg["n_l"], dims, L, device="cuda")
+    wk.wk_stack_backward(h, X, dOut, dX0, ref.grads)
+    got = replicas.GradBuckets(cfg["n"], cfg["d"], cfg["k"], cfg["n_l"], dims, L, device="cuda")
+    evs = [torch.cuda.Event() for _ in range(L)]
+    side = torch.cuda.Stream()
+    copies = [torch.empty_like(f) for f in got.flats]
+    main = torch.cuda.current_stream()
+    wk.wk_stack_backward(h, X, dOut, dX1, got.grads, layer_events=evs, stream=main)
+    for l in range(L - 1, -1, -1):
+        side.wait_event(evs[l])
+        with torch.cuda.stream(side):
+            copies[l].copy_(got.flats[l])
+    torch.cuda.synchronize()
+    assert wk.wk_stack_sync_status(h) == wk.WK_OK
+    assert all(e.query() for e in evs)
+    assert torch.equal(dX0, dX1)
+    for l in range(L):
+        assert torch.isfinite(ref.flats[l]).all()
+        scale = float(ref.flats[l].abs().max())
+        assert torch.allclose(got.flats[l], ref.flats[l], rtol=1e-5, atol=1e-6 * scale), l
+        assert torch.equal(copies[l], got.flats[l]), l
+    with pytest.raises(ValueError):
+        wk.wk_stack_backward(h, X, dOut, dX1, got.grads, layer_events=evs[:1])
+    wk.wk_stack_destroy(h)
