@@ -133,3 +133,27 @@ def test_fp16_gates_agree_with_exact_gates_away_from_zero():
     a = oracle.layer_backward(cfg, w, X, dOut)
     b = oracle.layer_backward(cfg, w, X, dOut, gates=exact)
     assert np.array_equal(a[0], b[0]) and all(np.array_equal(a[1][k], b[1][k]) for k in a[1])
+
+
+def test_layernorm_backward_invariants():
+    """The LayerNorm's normalisation is unchanged when a constant is added to its input row,
+    and (with eps = 0) when the row is scaled by a positive factor: the exact input gradient
+    therefore sums to zero over the row and is orthogonal to the centred row, whatever the
+    upstream gradient. A dropped mean term fails the first, a dropped variance term the
+    second. Also, against the Jacobian dxhat_i / dx_j = rs (delta_ij - 1/N - xhat_i xhat_j / N)
+    built as a matrix."""
+    rng = np.random.RandomState(11)
+    N = 37
+    x = rng.randn(5, N) * 3.0 + 2.0
+    g = rng.randn(5, N)
+    mu = x.mean(axis=1, keepdims=True)
+    for eps in (0.0, 1e-5):
+        rs = 1.0 / np.sqrt(((x - mu) ** 2).mean(axis=1, keepdims=True) + eps)
+        xh = (x - mu) * rs
+        dx = oracle.layernorm_backward(g, xh, rs)
+        assert np.allclose(dx.sum(axis=1), 0.0, atol=1e-12)
+        if eps == 0.0:
+            assert np.allclose((dx * (x - mu)).sum(axis=1), 0.0, atol=1e-11)
+        for r in range(5):
+            J = rs[r, 0] * (np.eye(N) - 1.0 / N - np.outer(xh[r], xh[r]) / N)
+            assert np.allclose(dx[r], J.T @ g[r], rtol=0, atol=1e-12)
