@@ -193,6 +193,30 @@ def oracle_sample(cfg, n_examples, threads=None):
     return n_examples / (dt * cfg["layers"]), dt, thr
 
 
+def backward_oracle_sample(cfg, n_examples, dO=None):
+    """Times the fp64 oracle's forward and backward of ONE layer on n_examples examples
+    (weights, inputs and the upstream gradient made before the clock starts) and returns
+    (examples/s of the whole stack's training step, seconds, threads)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle
+    from synth import configs as C
+    Xh = C.to_f64(C.make_x_host(cfg, list(range(n_examples))))
+    w = C.make_layer_host(cfg, 0)
+    if dO is None:
+        dO = np.random.RandomState(1234).standard_normal(Xh.shape)
+    t0 = time.perf_counter()
+    oracle.layer_backward(cfg, w, Xh, dO)
+    dt = time.perf_counter() - t0
+    thr = max([pp.get("num_threads", 1) for pp in threadpool_info()] or [1])
+    return n_examples / (dt * cfg["layers"]), dt, thr
+
+
+def backward_sample_size(workload):
+    return max(1, min(16, ORACLE_SAMPLE.get(workload, 16) // 8))
+
+
 def workload_cfg(name):
     from synth import configs as C
     if name in C.WHALE_CONFIGS:
@@ -205,23 +229,32 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     cfg = workload_cfg(args.workload)
+    whale = "L" in cfg
+    backward = args.backward and not whale and "experts" not in cfg
     vals = []
-    ns = ORACLE_SAMPLE[args.workload]
+    ns = backward_sample_size(args.workload) if backward else ORACLE_SAMPLE[args.workload]
+    sample_fn = backward_oracle_sample if backward else oracle_sample
     for _ in range(args.warmup):
-        oracle_sample(cfg, ns)
+        sample_fn(cfg, ns)
     thr = None
     for _ in range(args.steps):
-        v, dt, thr = oracle_sample(cfg, ns)
+        v, dt, thr = sample_fn(cfg, ns)
         vals.append(v)
     value = statistics.median(vals)
-    whale = "L" in cfg
-    sample = ("%d examples of the fusion per step" % ns if whale else
-              "%d examples through 1 of the %d layers per step, scaled to the whole stack" % (ns, cfg["layers"]))
-    line = {"impl": "reference", "metric": WHALE_METRIC if whale else METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
+    if whale:
+        sample = "%d examples of the fusion per step" % ns
+    elif backward:
+        sample = ("%d examples through the forward and backward of 1 of the %d layers per step (numpy "
+                  "float64), scaled to the whole stack" % (ns, cfg["layers"]))
+    else:
+        sample = "%d examples through 1 of the %d layers per step, scaled to the whole stack" % (ns, cfg["layers"])
+    metric = WHALE_METRIC if whale else (BACKWARD_METRIC if backward else METRIC)
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload + ": " + workload_desc(cfg), "global_batch": cfg["batch"],
-                       "oracle": ("numpy fp64 (BLAS threads)" if whale else
+            "config": {"workload": args.workload + ": " + workload_desc(cfg) + (", training step" if backward else ""),
+                       "global_batch": cfg["batch"],
+                       "oracle": ("numpy fp64 (BLAS threads)" if whale or backward else
                                   "plain C fp64, threads over examples / output rows")},
             "cpu_baseline": {"value": value, "unit": "examples/s", "cores": thr, "kind": "oracle",
                              "sample": sample},
@@ -486,17 +519,9 @@ def run_backward(args, cfg, rank, world, local, dev):
             "gpu_launches": sum(v[1] for v in ktimes.values()),
         }
         if world == 1 and not args.no_cpu_baseline:
-            import oracle
-            ns = max(1, min(16, ORACLE_SAMPLE.get(args.workload, 16) // 8))
-            Xh = C.to_f64(C.make_x_host(cfg, list(range(ns))))
-            w = C.make_layer_host(cfg, 0)
-            dO = dOut[:ns].double().cpu().numpy()
-            t0 = time.perf_counter()
-            oracle.layer_backward(cfg, w, Xh, dO)
-            dt = time.perf_counter() - t0
-            from threadpoolctl import threadpool_info
-            thr = max([pp.get("num_threads", 1) for pp in threadpool_info()] or [1])
-            line["cpu_baseline"] = {"value": ns / (dt * L), "unit": "examples/s", "cores": thr, "kind": "oracle",
+            ns = backward_sample_size(args.workload)
+            v, dt, thr = backward_oracle_sample(cfg, ns, dOut[:ns].double().cpu().numpy())
+            line["cpu_baseline"] = {"value": v, "unit": "examples/s", "cores": thr, "kind": "oracle",
                                     "sample": "%d examples through the forward and backward of 1 of the %d layers "
                                               "(%.1f s, numpy float64), scaled to the stack" % (ns, L, dt)}
         print(json.dumps(line), flush=True)
