@@ -155,7 +155,7 @@ def test_backward_rejects_unsupported_batches():
 def test_layer_events_mark_final_gradients():
     """wk_stack_backward with per-layer events: the gradients (written into the flat per-layer
     buffers a data-parallel step all-reduces) match those of the call without events (bit
-    for bit for dX; the batch sums use atomic adds, whose order varies, so those to 1e-5),
+    for bit for dX; the batch sums use atomic adds, whose order varies, so those to 1e-4),
     and a second stream that waits on layer l's event copies exactly layer l's final
     gradients while the backward of the layers below runs."""
     from recsys_feature_interaction_b200 import replicas
@@ -186,7 +186,7 @@ def test_layer_events_mark_final_gradients():
     for l in range(L):
         assert torch.isfinite(ref.flats[l]).all()
         scale = float(ref.flats[l].abs().max())
-        assert torch.allclose(got.flats[l], ref.flats[l], rtol=1e-5, atol=1e-6 * scale), l
+        assert torch.allclose(got.flats[l], ref.flats[l], rtol=1e-4, atol=1e-5 * scale), l
         assert torch.equal(copies[l], got.flats[l]), l
     with pytest.raises(ValueError):
         wk.wk_stack_backward(h, X, dOut, dX1, got.grads, layer_events=evs[:1])
