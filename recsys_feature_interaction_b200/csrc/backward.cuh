@@ -1,18 +1,21 @@
 // backward.cuh -- the kernels of the backward pass of a Wukong layer that are neither the
-// FMB MLP's tensor-core GEMMs (gemm_tc2.cuh on transposed operands) nor the strided
+// FMB MLP's tensor-core GEMMs (gemm_tc2.cuh, operands read MN-major) nor the strided
 // contractions of the FM and the LCB (bw_tc.cuh).
 //
 // Per layer, with y = concat(FMB(X), LCB(X)) + X, out = LN_d(y) gamma2 + beta2, the layer
 // of the Wukong page (section 2.2) differentiated by the chain rule:
-//   bw_out_ln_kernel     dy = LN_d'(y)^T (dOut * gamma2) per embedding row; d gamma2, d beta2;
-//                        the FMB rows of dy as the MLP's upstream gradient (16-bit)
-//   bw_relu_mask_kernel  dz = dh where the ReLU output was > 0
-//   bw_to_f32_kernel     fp32 copies of the 16-bit operands of the tf32 contractions
-//   bw_colsum_kernel     bias gradients (column sums over the batch)
-//   bw_transpose_kernel  16-bit transposes feeding the K-major GEMM
-//   bw_fmb_ln_kernel     dF = LN_nk'(F)^T d fhat per example (the FMB LayerNorm)
-//   bw_unfold_kernel     gradients of W0, gamma1, beta1 from those of the folded first Linear
-//                        W0' = W0 diag(gamma1), b0' = b0 + W0 beta1
+//   bw_out_ln_kernel       dy = LN_d'(y)^T (dOut * gamma2) per embedding row; d gamma2,
+//                          d beta2; the FMB rows of dy as the MLP's upstream gradient (16-bit)
+//   bw_mask_colsum_kernel  dz = dh where the ReLU output was > 0, and the bias gradient
+//                          (column sums over the batch), in one pass
+//   bw_to_f32_kernel       fp32 copies of the 16-bit operands of the tf32 contractions
+//   bw_fmb_ln_reg_kernel   dF = LN_nk'(F)^T d fhat per example (the FMB LayerNorm), the
+//                          example held in registers
+//   bw_unfold4_kernel      gradients of W0, gamma1, beta1 from those of the folded first
+//                          Linear W0' = W0 diag(gamma1), b0' = b0 + W0 beta1
+// and the general forms the launcher falls back to for shapes the fast ones do not take
+// (bw_relu_mask_kernel + bw_colsum_kernel, bw_fmb_ln_kernel, bw_unfold_kernel), with
+// bw_transpose_kernel for the one-CTA GEMM, which reads only K-major operands.
 #pragma once
 
 #include "common.cuh"
