@@ -7,9 +7,11 @@ Wukong page) and streams a stack one layer at a time, so that a large workload
 needs only one layer's weights in host memory.
 
 Parity status: pinned by identities (tests/test_oracle_pins.py); the page prints
-no worked example of a whole layer. The backward pass (layer_backward, numpy float64,
+no worked example of a whole layer. The chaining of layers (stack_forward, moe_forward)
+is pinned by closed-form multi-layer stacks (tests/test_oracle_stack_pins.py). The backward pass (layer_backward, numpy float64,
 derived from the forward by the chain rule) is pinned by finite differences of the
-forward (tests/test_oracle_backward_pins.py).
+forward (tests/test_oracle_backward_pins.py); its ReLU gates are its own float64
+decisions (pre-activation > 0), nothing here models a kernel's precision.
 """
 import ctypes
 import os
@@ -329,44 +331,11 @@ def layernorm_backward(dxh, xh, rs):
     return rs * (dxh - dxh.mean(axis=-1, keepdims=True) - xh * (dxh * xh).mean(axis=-1, keepdims=True))
 
 
-def relu_gates_fp16(cfg, w, X, ln_eps=1e-5):
-    """The ReLU gates (pre-activation > 0) of the hidden Linears of one layer, decided on the
-    forward as the fp16 tensor-core path stores it: X and Z = X^T Y rounded to fp16, the FMB
-    LayerNorm output rounded to fp16, the first Linear with the LayerNorm affine folded in
-    (W0 diag(gamma1) rounded to fp16, b0 + W0 beta1), hidden activations and weights in fp16;
-    every sum exact. A ReLU gate is a decision taken in floating point: a comparison of the
-    GPU's gradients with the oracle takes it in the kernels' precision through this function
-    (the gradient arithmetic itself stays float64 in layer_backward)."""
-    r16 = lambda a: np.asarray(a, dtype=np.float64).astype(np.float16).astype(np.float64)
-    X = r16(X)
-    E, n, d = X.shape
-    k = cfg["k"]
-    m = len(cfg["hidden"]) + 1
-    Y = r16(_weight_f64(w["Y"]))
-    Z = r16(np.einsum("eit,ic->etc", X, Y))
-    f = np.einsum("eit,etc->eic", X, Z).reshape(E, n * k)
-    mu = f.mean(axis=1, keepdims=True)
-    fh = r16((f - mu) / np.sqrt(((f - mu) ** 2).mean(axis=1, keepdims=True) + ln_eps))
-    W0 = _weight_f64(w["W0"])
-    b0 = np.zeros(W0.shape[0]) if w.get("b0") is None else _c64(w["b0"])
-    h = fh
-    Wj, bj = r16(W0 * _c64(w["fmb_gamma"])[None, :]), b0 + W0 @ _c64(w["fmb_beta"])
-    gates = []
-    for j in range(m - 1):
-        z = h @ Wj.T + bj
-        gates.append(z > 0.0)
-        h = r16(np.maximum(z, 0.0))
-        Wj = r16(_weight_f64(w["W%d" % (j + 1)]))
-        bj = np.zeros(Wj.shape[0]) if w.get("b%d" % (j + 1)) is None else _c64(w["b%d" % (j + 1)])
-    return gates
-
-
-def layer_backward(cfg, w, X, dOut, ln_eps=1e-5, gates=None):
+def layer_backward(cfg, w, X, dOut, ln_eps=1e-5):
     """(dX [E, n, d], grads) of one layer at X for the upstream gradient dOut = dL/d(output).
     grads: Y, W0.., b0.., fmb_gamma, fmb_beta, W_L, out_gamma, out_beta (float64, summed
-    over the E examples). Weights as for layer_forward (float32 or bf16 bits). gates: None
-    (the ReLU derivative is pre-activation > 0) or one boolean [E, h_{j+1}] array per hidden
-    Linear that decides it instead (relu_gates_fp16)."""
+    over the E examples). Weights as for layer_forward (float32 or bf16 bits). The ReLU
+    derivative is 1 where the float64 pre-activation is > 0, else 0."""
     _, c = layer_forward_np(cfg, w, X, ln_eps)
     dOut = _c64(dOut)
     E, n, d = c["X"].shape
@@ -386,7 +355,7 @@ def layer_backward(cfg, w, X, dOut, ln_eps=1e-5, gates=None):
     dh = dy[:, :n_f, :].reshape(E, n_f * d)
     for j in range(m - 1, -1, -1):
         if j < m - 1:
-            dz = dh * (gates[j] if gates is not None else (c["zs"][j] > 0.0))
+            dz = dh * (c["zs"][j] > 0.0)
         else:
             dz = dh
         g["W%d" % j] = dz.T @ c["hs"][j]

@@ -117,24 +117,6 @@ def test_closed_relu_gate_gets_no_weight_gradient():
     assert np.abs(g["W0"]).sum() > 0.0
 
 
-def test_fp16_gates_agree_with_exact_gates_away_from_zero():
-    cfg = CASES[2][0]
-    w = _layer(cfg, 3)
-    X = np.random.RandomState(8).randn(4, cfg["n"], cfg["d"])
-    dOut = np.random.RandomState(9).randn(4, cfg["n"], cfg["d"])
-    _, c = oracle.layer_forward_np(cfg, w, X)
-    gates = oracle.relu_gates_fp16(cfg, w, X)
-    assert len(gates) == len(cfg["hidden"])
-    for z, g in zip(c["zs"], gates):
-        away = np.abs(z) > 1e-2 * np.sqrt(np.mean(z * z))
-        assert np.array_equal(g[away], (z > 0)[away])
-    # passing the exact gates explicitly reproduces the default
-    exact = [z > 0 for z in c["zs"][:-1]]
-    a = oracle.layer_backward(cfg, w, X, dOut)
-    b = oracle.layer_backward(cfg, w, X, dOut, gates=exact)
-    assert np.array_equal(a[0], b[0]) and all(np.array_equal(a[1][k], b[1][k]) for k in a[1])
-
-
 def test_layernorm_backward_invariants():
     """The LayerNorm's normalisation is unchanged when a constant is added to its input row,
     and (with eps = 0) when the row is scaled by a positive factor: the exact input gradient
