@@ -67,7 +67,10 @@ typedef enum {
   WK_ERR_OOM = 3,          /* workspace allocation failed */
   WK_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch error, no device, ...) */
   WK_ERR_TIMEOUT = 5,      /* a kernel gave up on a pipeline wait; its output is not valid */
-  WK_ERR_DEVICE = 6        /* the device status word holds another error flag */
+  WK_ERR_DEVICE = 6,       /* the device status word holds another error flag */
+  WK_ERR_NONFINITE = 7     /* a LayerNorm met a non-finite row: a value left the range of its
+                              16-bit storage (fp16: |v| > 65504) or an input held inf / NaN;
+                              the output is not valid */
 } wk_status;
 
 typedef enum { WK_F32 = 0, WK_BF16 = 1, WK_F16 = 2 } wk_dtype;
@@ -145,7 +148,11 @@ WK_API wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t
 WK_API wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host, int64_t batch, wk_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the device status word.
- * WK_OK, WK_ERR_TIMEOUT, WK_ERR_DEVICE or WK_ERR_CUDA. */
+ * WK_OK, WK_ERR_TIMEOUT, WK_ERR_NONFINITE, WK_ERR_DEVICE or WK_ERR_CUDA.
+ * WK_ERR_NONFINITE: a 16-bit stack stores its intermediates in fp16 by default (see
+ * wk_stack_config.operand_dtype); every LayerNorm of the forward (the FMB LayerNorm, each
+ * layer's output LayerNorm) checks its row statistics, so a value that overflowed fp16
+ * anywhere upstream is reported here instead of leaving inf / NaN silently in `out`. */
 WK_API wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream);
 
 /* Frees the workspace and the handle (synchronises the device first). NULL is a no-op. */
@@ -174,7 +181,8 @@ WK_API void wk_graph_destroy(wk_graph* g);
 typedef enum { WK_KERNEL_FM_LN = 0, WK_KERNEL_MLP_GEMM = 1, WK_KERNEL_LCB = 2, WK_KERNEL_RES_LN = 3,
                WK_KERNEL_CONVERT = 4, WK_KERNEL_MOE_GATE = 5, WK_KERNEL_MOE_COMBINE = 6,
                WK_KERNEL_HEAD = 7, WK_KERNEL_WHALE_ATTN = 8, WK_KERNEL_WHALE_FFN = 9,
-               WK_KERNEL_BW_CONTRACT = 10, WK_KERNEL_BW_ROWS = 11, WK_KERNEL_COUNT = 12 } wk_kernel_kind;
+               WK_KERNEL_BW_CONTRACT = 10, WK_KERNEL_BW_ROWS = 11, WK_KERNEL_FRONT = 12,
+               WK_KERNEL_COUNT = 13 } wk_kernel_kind;
 
 /* enable != 0: every later forward records a start/stop event pair around each
  * kernel launch on its stream (adds no synchronisation). */
@@ -464,7 +472,11 @@ WK_API wk_status wk_whale_fusion_ffn(const void* Hw, const void* A, const wk_wha
  * weights `w` used as given (operands in cfg->dtype; cfg->operand_dtype must be 0
  * or equal to cfg->dtype, since converting weights would need memory). X and out
  * are caller-owned device tensors [batch, n, d] of cfg->dtype that must not
- * overlap; cfg->num_layers and cfg->max_batch are ignored.
+ * overlap; cfg->num_layers and cfg->max_batch are ignored. Every pointer (X, out,
+ * and each weight, bias and LayerNorm vector in `w`) must be 16-byte aligned, as
+ * for wk_stack_create; a misaligned one returns WK_ERR_INVALID_ARG before
+ * anything is launched. The FMB LayerNorm affine is applied in the FM's
+ * epilogue here (nothing is folded into a weight copy).
  *
  * Intermediates live in one fixed device array of WK_NOALLOC_SCRATCH_BYTES that
  * is part of the library image: every GPU that loads the library reserves it

@@ -1,8 +1,8 @@
 """Times one step of the Wukong layer alone through its stand-alone C-ABI entry point.
 
-    python -m recsys_feature_interaction_b200.microbench --kernel fm_ln|mlp_gemm|lcb|res_ln|moe_gate|moe_combine
+    python microbench.py --kernel front|fm_ln|mlp_gemm|lcb|res_ln|moe_gate|moe_combine
         [--workload c4_bf16] [--batch B] [--iters K] [--dtype f16|bf16] [--layer-linear j] [--experts E]
-    python -m recsys_feature_interaction_b200.microbench --kernel whale_attn|whale_ffn [--workload whale_c4] ...
+    python microbench.py --kernel whale_attn|whale_ffn [--workload whale_c4] ...
 
 Inputs are synthetic (the seeded generator), on the device, in the workload's
 shapes. Prints one JSON line with the mean CUDA-event time per launch and the
@@ -14,15 +14,15 @@ import json
 import os
 import sys
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", required=True, choices=["fm_ln", "mlp_gemm", "lcb", "res_ln", "moe_gate", "moe_combine",
-                                                           "whale_attn", "whale_ffn"])
+    ap.add_argument("--kernel", required=True, choices=["front", "fm_ln", "mlp_gemm", "lcb", "res_ln", "moe_gate",
+                                                           "moe_combine", "whale_attn", "whale_ffn"])
     ap.add_argument("--workload", default="c4_bf16")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--iters", type=int, default=10)
@@ -43,6 +43,8 @@ def main():
     if args.kernel.startswith("whale"):
         run, flops, bytes_, B = _whale_case(args)
         return _time(args, run, flops, bytes_, B)
+    if args.kernel == "front":
+        return _front_case(args)
     cfg = C.MOE_CONFIGS[args.workload] if args.workload in C.MOE_CONFIGS else C.CONFIGS[args.workload]
     B = args.batch or cfg["batch"]
     n, d, k, n_f, n_l = cfg["n"], cfg["d"], cfg["k"], cfg["n_f"], cfg["n_l"]
@@ -109,6 +111,47 @@ def main():
         flops = 0
         bytes_ = 3 * n * d * es * B
     return _time(args, run, flops, bytes_, B)
+
+
+def _front_case(args):
+    """The one-kernel layer front (input LayerNorm, FM + LayerNorm, LCB, residual) of the
+    workload's layer shape, inside a 2-layer stack whose FMB MLP is cut to one hidden width
+    of 64 (the front does not depend on the MLP): layer 0's front converts the input, layer
+    1's normalises the previous layer's output. Reports the mean of both layers' front
+    launches from the stack's own per-kernel events; the workload's batch unless --batch."""
+    import torch
+
+    import recsys_feature_interaction_b200 as wk
+    from synth import configs as C
+    cfg = dict(C.CONFIGS[args.workload], layers=2, hidden=[64])
+    B = args.batch or cfg["batch"]
+    n, d, k = cfg["n"], cfg["d"], cfg["k"]
+    layers = [C.make_layer_dev(cfg, l) for l in range(2)]
+    h = wk.wk_stack_create(cfg, layers, max_batch=B)
+    X = C.make_x_dev(cfg, B)
+    out = torch.empty_like(X)
+    for _ in range(args.warmup):
+        wk.wk_stack_forward(h, X, out)
+    torch.cuda.synchronize()
+    wk.wk_stack_kernel_times(h)
+    wk.wk_stack_set_profiling(h, True)
+    for _ in range(args.iters):
+        wk.wk_stack_forward(h, X, out)
+    torch.cuda.synchronize()
+    wk.wk_stack_set_profiling(h, False)
+    t = wk.wk_stack_kernel_times(h)
+    st = wk.wk_stack_sync_status(h)
+    wk.wk_stack_destroy(h)
+    ms_total, launches = t["front"]
+    ms = ms_total / max(1, launches)
+    flops = (4 * n * d * k + 2 * cfg["n_l"] * n * d) * B
+    bytes_ = (2 * n * d + n * k) * 2 * B  # layer input in, layer output and A0 out (16-bit)
+    print(json.dumps({"kernel": "front", "workload": args.workload, "batch": B, "dtype": "f16",
+                      "ms_per_launch": ms, "launches": launches, "tflops": flops / (ms / 1e3) / 1e12,
+                      "gbs": bytes_ / (ms / 1e3) / 1e9, "flops_per_launch": flops, "bytes_per_launch": bytes_,
+                      "device_status": wk.wk_status_string(st)}))
+    if st != wk.WK_OK:
+        sys.exit(1)
 
 
 def _whale_case(args):

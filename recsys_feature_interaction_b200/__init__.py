@@ -18,13 +18,13 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libwukong.so")
 
-WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE = range(7)
+WK_OK, WK_ERR_INVALID_ARG, WK_ERR_UNSUPPORTED, WK_ERR_OOM, WK_ERR_CUDA, WK_ERR_TIMEOUT, WK_ERR_DEVICE, WK_ERR_NONFINITE = range(8)
 WK_F32, WK_BF16, WK_F16 = 0, 1, 2
 (WK_KERNEL_FM_LN, WK_KERNEL_MLP_GEMM, WK_KERNEL_LCB, WK_KERNEL_RES_LN, WK_KERNEL_CONVERT, WK_KERNEL_MOE_GATE,
  WK_KERNEL_MOE_COMBINE, WK_KERNEL_HEAD, WK_KERNEL_WHALE_ATTN, WK_KERNEL_WHALE_FFN, WK_KERNEL_BW_CONTRACT,
- WK_KERNEL_BW_ROWS, WK_KERNEL_COUNT) = range(13)
+ WK_KERNEL_BW_ROWS, WK_KERNEL_FRONT, WK_KERNEL_COUNT) = range(14)
 KERNEL_NAMES = ("fm_ln", "mlp_gemm", "lcb", "res_ln", "convert", "moe_gate", "moe_combine", "head", "whale_attn",
-                "whale_ffn", "bw_contract", "bw_rows")
+                "whale_ffn", "bw_contract", "bw_rows", "front")
 WK_MOE_MAX_EXPERTS = 8
 
 

@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "_lib", "libwukong.so")
 SOURCES = ["wk_api.cu"]
-HEADERS = ["common.cuh", "gemm_tc.cuh", "gemm_tc2.cuh", "lcb_tc.cuh", "fm_mma.cuh", "fm_tc.cuh", "res_ln.cuh", "res_ln_ring.cuh", "simt.cuh", "convert.cuh", "row_ln_epi.cuh", "moe.cuh", "head.cuh", "whale.cuh", "backward.cuh", "bw_tc.cuh"]
+HEADERS = ["common.cuh", "gemm_tc.cuh", "gemm_tc2.cuh", "lcb_tc.cuh", "fm_tc.cuh", "front_tc.cuh", "res_ln.cuh", "res_ln_ring.cuh", "simt.cuh", "convert.cuh", "moe.cuh", "head.cuh", "whale.cuh", "backward.cuh", "bw_tc.cuh"]
 
 
 def _stale():

@@ -19,6 +19,7 @@ namespace wk {
 // device status word flags
 constexpr unsigned kFlagTimeout = 1u;   // a pipeline wait ran past its limit
 constexpr unsigned kFlagBadShape = 2u;  // a kernel met a shape it was not built for
+constexpr unsigned kFlagNonFinite = 4u; // a LayerNorm met a row with non-finite statistics
 
 // ~2^31 SM cycles: about one second at the B200's clocks, far above any
 // legitimate wait inside one launch.
@@ -133,6 +134,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
                "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// Tiled TMA reduce-add of a shared-memory tile into global memory: each element of the
+// box is added to the element it lands on (in the tensor map's element type).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* src, int32_t c0, int32_t c1) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
                : "memory");
 }
 
@@ -277,29 +287,6 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* m, uint32_t 
       "%4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
       : "memory");
-}
-
-// The same load with an L2 eviction-priority hint (a policy from createpolicy).
-__device__ __forceinline__ void tma_load_2d_pair_hint(const CUtensorMap* m, uint32_t bar_cluster_addr, void* dst,
-                                                      int32_t c0, int32_t c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
-      "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "l"(policy)
-      : "memory");
-}
-
-// L2 policies: lines kept in preference to others / evicted before others.
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
 }
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {

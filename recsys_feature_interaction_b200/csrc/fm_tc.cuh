@@ -451,7 +451,9 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
         qs = warp_sum(qs);
         if (lane == 0) red[4 + ew] = qs;
         named_bar(1, 128);
-        const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
+        const float var = (red[4] + red[5] + red[6] + red[7]) * inv_cnt;
+        const float rstd = rsqrtf(var + eps);
+        if (threadIdx.x == 64 && !(isfinite(mean) && isfinite(var))) flag_error(status, kFlagNonFinite);
         T* ab = A0 + b * (C::N * C::K);
         const bool affine = gamma != nullptr;
 #pragma unroll
@@ -526,7 +528,9 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
         qs = warp_sum(qs);
         if (lane == 0) red[4 + ew] = qs;
         named_bar(1, 128);
-        const float rstd = rsqrtf((red[4] + red[5] + red[6] + red[7]) * inv_cnt + eps);
+        const float var = (red[4] + red[5] + red[6] + red[7]) * inv_cnt;
+        const float rstd = rsqrtf(var + eps);
+        if (threadIdx.x == 64 && !(isfinite(mean) && isfinite(var))) flag_error(status, kFlagNonFinite);
         T* ab = A0 + b * (C::N * C::K);
         const bool affine = gamma != nullptr;
   #pragma unroll 1

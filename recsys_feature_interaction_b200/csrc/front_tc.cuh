@@ -1,0 +1,787 @@
+// front_tc.cuh -- everything of a Wukong layer but the FMB MLP, one example at a time
+// per CTA, reading each example's layer input from HBM once (Wukong page, section 2.2:
+// the layer is LN(concat(FMB(X), LCB(X)) + X); FMB(X) = MLP(LN(flatten(X (X^T Y))));
+// LCB(X) = W_L X):
+//
+//   X      = LN_rows(y_in) * g_in + b_in    (the previous layer's output LayerNorm;
+//            for the first layer X is the caller's input, converted to the operand type)
+//   A0     = LN(flatten(X (X^T Y)))         (the FM and the FMB LayerNorm; its affine is
+//            either applied here or folded into the first Linear by the caller)
+//   y_out[rows n_f..n-1] = W_L X + X[n_f..n-1]     (the LCB rows with their residual)
+//   y_out[rows 0..n_f-1] = X[0..n_f-1]              (the residual of the FMB rows; the
+//            last MLP Linear adds its output into them with a TMA reduce-add)
+//
+// so a layer's output y_out = concat(FMB, LCB) + X, before the output LayerNorm, which
+// the next layer's front (or the stack's final LayerNorm) applies as it reads y_out.
+//
+// Per example, in shared memory: the n x d layer input in 128-row chunks, each one contiguous
+// range of the input brought in by one bulk copy and rewritten in place by the normalising
+// warps as the MMA operand layout (32-column boxes, 64-byte swizzle), read by three tcgen05
+// products:
+//   pass A  Z = X^T Y       M = d (128-row tiles), N = k (padded to KP), K = n;
+//   LCB     D_m = W_L,m X   M = 128 rows of W_L, N = d, K = n (W_L and Y stream through a
+//                           small ring of 16 KB stages from L2);
+//   pass B  F = X Z         M = n (one tile per chunk), N = KP, K = d (Z written back to
+//                           shared memory as a 16-bit operand by the epilogue warps).
+// TMEM holds Z at column 0 and, from column LCOL, first the LCB accumulators and then F.
+//
+// Warps (480 threads): 0 loads input chunks; 1 allocates TMEM and issues the MMAs; 2 streams
+// Y and W_L; 3..6 are the epilogue (one TMEM lane quarter each: Z to shared memory, the LCB
+// rows plus residual out through TMA stores, the FMB LayerNorm of F into A0); 7..14
+// normalise each chunk as it lands (two threads per row) and store the FMB-row residual.
+// Every mbarrier wait is bounded; after a failed wait each role stops, every copy in flight
+// lands and TMEM is freed before the CTA exits.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "res_ln.cuh"
+
+namespace wk {
+
+constexpr int FRONT_THREADS = 480;
+constexpr int FRONT_EPI_WARP0 = 3;    // warps 3..6: the epilogue (TMEM lane quarter = warp & 3)
+constexpr int FRONT_NORM_WARP0 = 7;   // warps 7..14: normalisation
+constexpr int FRONT_NORM_THREADS = 256;
+constexpr int FRONT_SMEM_LIMIT = 232448;
+
+template <int N_, int D_, int K_, int NF_>
+struct FrontCfg {
+  static constexpr int N = N_, D = D_, K = K_, NF = NF_, NL = N_ - NF_;
+  static constexpr int R = 128;                              // rows per chunk = MMA M
+  static constexpr int NCH = (N + R - 1) / R;
+  static constexpr int XBOXES = D / 32;                      // 32-column boxes per chunk
+  static constexpr int XBOXB = R * 64;                       // 8 KB per box
+  static constexpr int CHB = XBOXES * XBOXB;                 // bytes per chunk
+  static constexpr int KP = K <= 32 ? 32 : 64;               // MMA N of the FM (k padded)
+  static constexpr int YRB = KP * 2;                         // bytes per Y / Z row
+  static constexpr int YB = R * YRB;                         // one Y box (128 rows)
+  static constexpr int MTZ = (D + R - 1) / R;                // Z tiles
+  static constexpr int MTL = (NL + R - 1) / R;               // LCB tiles
+  static constexpr int LCOL = MTZ * KP;                      // first TMEM column of the LCB / F
+  static constexpr int LCOLS = MTL * D;
+  static constexpr int FCOLS = NCH * KP;
+  static constexpr int UCOLS = LCOLS > FCOLS ? LCOLS : FCOLS;
+  static constexpr int TCOLS = LCOL + UCOLS;
+  static constexpr int TMEM_COLS = TCOLS <= 32 ? 32 : TCOLS <= 64 ? 64 : TCOLS <= 128 ? 128 : TCOLS <= 256 ? 256 : 512;
+  static constexpr int ZB = ((D + 15) / 16) * 16 * YRB;      // Z operand
+  static constexpr int WB = R * 64 * 2;                      // one W_L box (128 rows x 64 k)
+  static constexpr int STG = WB > YB ? WB : YB;              // ring stage
+  static constexpr int EPI = 4 * 2048;                       // a 32 x 32 16-bit staging tile per epilogue warp
+  static constexpr int TAIL = 2 * D * 4 + 1024;              // input LN affine, partial sums, barriers
+  static constexpr int FIXED = 1024 + NCH * CHB + ZB + EPI + TAIL;
+  static constexpr int NSTG_RAW = (FRONT_SMEM_LIMIT - FIXED) / STG;
+  static constexpr int NSTG = NSTG_RAW > 4 ? 4 : NSTG_RAW;
+  // pass A's last Z tile reads 4 * MTZ boxes from a chunk's base: past the last chunk that
+  // is OVER bytes, which must stay inside this CTA's shared memory (rows of Z past d are
+  // never read, so what they read does not matter)
+  static constexpr int OVER = (4 * MTZ - XBOXES) * XBOXB;
+  static constexpr int AFTER = ZB + NSTG * STG + EPI;
+  static constexpr int PAD = OVER > AFTER ? ((OVER - AFTER + 1023) / 1024) * 1024 : 0;
+  static constexpr int SMEM = FIXED + NSTG * STG + PAD;
+  // LayerNorm of F from registers when a thread's share (one row per chunk, k values) fits
+  static constexpr bool REGLN = NCH * K <= 96 && (K == 16 || K == 24 || K == 32);
+  // staging tiles (32 x 32, 2 KB) per epilogue warp for the LCB rows: its own tile plus a
+  // quarter of the Y / W_L ring, which is idle while the LCB accumulators are read out
+  static constexpr int NBUF_RAW = 1 + (NSTG * STG) / (4 * 2048);
+  static constexpr int NBUF = NBUF_RAW > 8 ? 8 : NBUF_RAW;
+  // A0 leaves through TMA stores of 32 x 32 tiles in the three-pass LayerNorm (k = 64, whole
+  // chunks), staged in three 2 KB tiles per epilogue warp: its own and two in the Z region
+  static constexpr bool A0_TMA = !REGLN && K == 64 && N % R == 0 && ZB >= 4 * 4096;
+  static_assert(D % 32 == 0 && D <= 256 && N % 16 == 0 && K % 4 == 0 && K <= 64, "shape");
+  static_assert(NSTG >= 2 && SMEM <= FRONT_SMEM_LIMIT, "shared memory");
+  static_assert(TCOLS <= 512, "TMEM columns");
+  static_assert(CHB % 1024 == 0 && ZB % 1024 == 0 && STG % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+// 16-byte unit u (0..3) of row r in a 64-byte-swizzled box of 64-byte rows.
+__device__ __forceinline__ uint32_t sw64_off(int r, int u) {
+  return static_cast<uint32_t>(r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
+}
+
+// Shared address of Z operand element row t, 16-byte unit j (MN-major, KP columns).
+template <class C>
+__device__ __forceinline__ uint32_t front_zb_addr(uint32_t zb, int t, int j) {
+  const int pj = (C::YRB == 128) ? (j ^ (t & 7)) : (j ^ ((t >> 1) & 3));
+  return zb + t * C::YRB + pj * 16;
+}
+
+__device__ __forceinline__ void front_tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void front_tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+
+// Eight 16-bit values of type TI (one 16-byte unit) as floats.
+template <typename TI>
+__device__ __forceinline__ void front_unpack8(const uint4& a, float (&v)[8]) {
+  Vec8<TI>::unpack(a, v);
+}
+
+template <typename TO>
+__device__ __forceinline__ uint4 front_pack8(const float (&v)[8]) {
+  uint4 a;
+  a.x = Half16<TO>::pack2(v[0], v[1]);
+  a.y = Half16<TO>::pack2(v[2], v[3]);
+  a.z = Half16<TO>::pack2(v[4], v[5]);
+  a.w = Half16<TO>::pack2(v[6], v[7]);
+  return a;
+}
+
+// xin: the layer input [batch, n, d] of type TIN (16-byte aligned). Tensor maps:
+//   tmY  Y [n, k] (T): boxes of KP columns (zero past k) x 128 rows, 128B (KP = 64) or 64B swizzle;
+//   tmW  W_L [n_l, n] (T): boxes of 64 columns x 128 rows, 128B swizzle;
+//   tmR  rows 0..n_f-1 of y_out as a (d, n_f, batch) tensor (T): boxes (32, 128, 1), 64B swizzle;
+//   tmL  rows n_f..n-1 of y_out as a (d, n_l, batch) tensor (T): boxes (32, 32, 1), 64B swizzle;
+//   tmA  A0 as [batch*n rows, k] (T): boxes (32, 32), 64B swizzle (used only when k = 64 and n is
+//        a multiple of 128: the output pass then stages A0 and stores it by TMA).
+// in_g / in_b: the input LayerNorm's affine [d] (null: the first layer, no LayerNorm);
+// fg / fb: the FMB LayerNorm's affine [n*k] (null: folded into the first Linear).
+template <class C, typename TIN, typename T>
+__global__ void __launch_bounds__(FRONT_THREADS, 1)
+    front_tc_kernel(const TIN* __restrict__ xin, const __grid_constant__ CUtensorMap tmY,
+                    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,
+                    const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmA,
+                    const float* __restrict__ in_g,
+                    const float* __restrict__ in_b, const float* __restrict__ fg, const float* __restrict__ fb,
+                    T* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* slots = smem;                                     // [NCH] chunks of the layer input
+  uint8_t* zb = slots + C::NCH * C::CHB;                     // Z operand
+  uint8_t* ring = zb + C::ZB;                                // [NSTG] Y / W_L stages
+  uint8_t* epi = ring + C::NSTG * C::STG;                    // [4] staging tiles
+  float* sg = reinterpret_cast<float*>(epi + C::EPI + C::PAD);
+  float* sb = sg + C::D;
+  float* red = sb + C::D;                                    // [8] FMB LayerNorm partial sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 8);
+  uint64_t* full = bars;                                     // [NCH] chunk landed
+  uint64_t* xready = full + C::NCH;                          // [NCH] chunk normalised
+  uint64_t* empty = xready + C::NCH;                         // [NCH] chunk slot free (2 arrivals)
+  uint64_t* wfull = empty + C::NCH;                          // [NSTG]
+  uint64_t* wempty = wfull + C::NSTG;                        // [NSTG]
+  uint64_t* zfull = wempty + C::NSTG;                        // MMA -> epilogue: Z in TMEM
+  uint64_t* ffull = zfull + 1;                               // MMA -> epilogue: F in TMEM
+  uint64_t* zready = zfull + 2;                              // epilogue -> MMA: Z operand written
+  uint64_t* ldone = zfull + 3;                               // epilogue -> MMA, ring: LCB columns read
+  uint64_t* fempty = zfull + 4;                              // epilogue -> MMA: F read
+  uint64_t* fin = zfull + 5;                                 // MMA: its last operations completed
+  uint64_t* lfull = zfull + 6;                               // [MTL] MMA -> epilogue: LCB tile m in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + C::MTL);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool ln_in = in_g != nullptr;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmY);
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmR);
+    prefetch_tmap(&tmL);
+    prefetch_tmap(&tmA);
+    for (int c = 0; c < C::NCH; ++c) {
+      mbar_init(&full[c], 1);
+      mbar_init(&xready[c], 1);
+      mbar_init(&empty[c], 2);
+    }
+    for (int s = 0; s < C::NSTG; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);
+    }
+    mbar_init(zfull, 1);
+    for (int m = 0; m < C::MTL; ++m) mbar_init(&lfull[m], 1);
+    mbar_init(ffull, 1);
+    mbar_init(zready, 4);
+    mbar_init(ldone, 4);
+    mbar_init(fempty, 4);
+    mbar_init(fin, 1);
+    fence_mbar_init();
+  }
+  if (ln_in && threadIdx.x >= 32 * FRONT_NORM_WARP0) {
+    for (int i = threadIdx.x - 32 * FRONT_NORM_WARP0; i < C::D; i += FRONT_NORM_THREADS) {
+      sg[i] = __ldg(in_g + i);
+      sb[i] = __ldg(in_b + i);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- input chunks
+    if (lane == 0) {
+      uint32_t issued = 0, lastpar = 0;
+      int64_t i = 0;
+      bool ok = true;
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x, ++i) {
+        const uint32_t par = static_cast<uint32_t>(i & 1);
+        for (int c = 0; c < C::NCH; ++c) {
+          if (!mbar_wait(&empty[c], par ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          // the chunk's rows are one contiguous range of the input: one bulk copy
+          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          const uint32_t bytes = static_cast<uint32_t>(rows * C::D * 2);
+          mbar_arrive_expect_tx(&full[c], bytes);
+          bulk_load(slots + c * C::CHB, xin + (b * C::N + c * C::R) * C::D, bytes, &full[c]);
+          issued |= 1u << c;
+          lastpar = (lastpar & ~(1u << c)) | (par << c);
+        }
+      }
+      // every copy issued lands before the CTA's shared memory is released
+      for (int c = 0; c < C::NCH; ++c)
+        if (issued & (1u << c)) mbar_drain(&full[c], (lastpar >> c) & 1u, status);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ Y / W_L ring
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, lastpar = 0;
+      int64_t i = 0;
+      bool ok = true;
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x, ++i) {
+        // the epilogue stages the previous example's LCB rows in the ring: wait until it is done
+        if (i > 0 && !mbar_wait(ldone, static_cast<uint32_t>((i - 1) & 1), status)) {
+          ok = false;
+          break;
+        }
+        // per chunk: its Y box, then its W_L boxes of every LCB tile (the MMA order)
+        for (int c = 0; ok && c < C::NCH; ++c) {
+          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          const int nkb = (rows + 63) / 64;
+          for (int t = -1; ok && t < C::MTL * nkb; ++t) {
+            if (!mbar_wait(&wempty[s], ph ^ 1u, status)) {
+              ok = false;
+              break;
+            }
+            if (t < 0) {
+              mbar_arrive_expect_tx(&wfull[s], static_cast<uint32_t>(C::YB));
+              tma_load_2d(&tmY, &wfull[s], ring + s * C::STG, 0, c * C::R);
+            } else {
+              mbar_arrive_expect_tx(&wfull[s], static_cast<uint32_t>(C::WB));
+              tma_load_2d(&tmW, &wfull[s], ring + s * C::STG, c * C::R + (t % nkb) * 64, (t / nkb) * C::R);
+            }
+            issued |= 1u << s;
+            lastpar = (lastpar & ~(1u << s)) | (ph << s);
+            if (++s == C::NSTG) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+      }
+      for (int t = 0; t < C::NSTG; ++t)
+        if (issued & (1u << t)) mbar_drain(&wfull[t], (lastpar >> t) & 1u, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const bool bf = Half16<T>::kBF16;
+      const uint32_t idA = idesc_f16kind_f32(C::R, C::KP, 1, 1, bf);  // Z = X^T Y: both MN-major
+      const uint32_t idL = idesc_f16kind_f32(C::R, C::D, 0, 1, bf);   // D = W_L X: X MN-major
+      const uint32_t idB = idesc_f16kind_f32(C::R, C::KP, 0, 1, bf);  // F = X Z: Z MN-major
+      const uint32_t ysw = C::YRB == 128 ? 2u : 4u;
+      const uint32_t slot0 = smem_u32(slots);
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t i = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x, ++i) {
+        const uint32_t par = static_cast<uint32_t>(i & 1);
+        // Chunk by chunk as they are normalised: pass A, Z += X_c^T Y_c (the previous example's Z
+        // has been turned into its pass-B operand first), and the LCB, D_m += W_L[m, c] X_c for
+        // every tile m (once the previous example's F, which shares D's TMEM columns, is read),
+        // so W_L streams in while the example's chunks arrive.
+        if (i > 0 && !mbar_wait(zready, par ^ 1u, status)) {
+          ok = false;
+          break;
+        }
+        for (int c = 0; ok && c < C::NCH; ++c) {
+          if (!mbar_wait(&xready[c], par, status) || !mbar_wait(&wfull[s], ph, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          const int nkb = (rows + 63) / 64;
+          const uint32_t xs = slot0 + c * C::CHB;
+          const uint32_t ys = smem_u32(ring + s * C::STG);
+          for (int ks = 0; ks < rows / 16; ++ks) {
+            const uint64_t bdesc = smem_desc(ys + ks * 16 * C::YRB, C::YB, 8 * C::YRB, ysw);
+#pragma unroll
+            for (int mz = 0; mz < C::MTZ; ++mz) {
+              // MN atoms of 32 columns are the boxes (LBO), 8-row k groups 512 bytes apart
+              const uint64_t adesc = smem_desc(xs + mz * 4 * C::XBOXB + ks * 16 * 64, C::XBOXB, 512, 4);
+              umma_f16kind(tmem_base + mz * C::KP, adesc, bdesc, idA, (c | ks) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&wempty[s]);
+          issued = true;
+          if (++s == C::NSTG) {
+            s = 0;
+            ph ^= 1u;
+          }
+          if (c == C::NCH - 1) umma_commit(zfull);
+          if (c == 0 && i > 0 && !mbar_wait(fempty, par ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          for (int t = 0; ok && t < C::MTL * nkb; ++t) {
+            const int m = t / nkb, kb = t % nkb;
+            if (!mbar_wait(&wfull[s], ph, status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t ws = smem_u32(ring + s * C::STG);
+            const int left = (rows - kb * 64) / 16;
+            const int nk = left < 4 ? left : 4;
+            for (int kk = 0; kk < nk; ++kk) {
+              const uint64_t adesc = smem_desc(ws + kk * 32, 16, 1024, 2);
+              const uint64_t bdesc = smem_desc(xs + (kb * 64 + kk * 16) * 64, C::XBOXB, 512, 4);
+              umma_f16kind(tmem_base + C::LCOL + m * C::D, adesc, bdesc, idL, (c | kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit(&wempty[s]);
+            if (++s == C::NSTG) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        for (int m = 0; m < C::MTL; ++m) umma_commit(&lfull[m]);
+        // pass B: F = X Z into the LCB's columns, once Z is in shared memory and the LCB
+        // accumulators have been read
+        if (!mbar_wait(zready, par, status) || !mbar_wait(ldone, par, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int c = 0; c < C::NCH; ++c) {
+          const uint32_t xs = slot0 + c * C::CHB;
+#pragma unroll
+          for (int ks = 0; ks < C::D / 16; ++ks) {
+            const uint64_t adesc = smem_desc(xs + (ks >> 1) * C::XBOXB + (ks & 1) * 32, 16, 512, 4);
+            const uint64_t bdesc = smem_desc(smem_u32(zb) + ks * 16 * C::YRB, C::ZB, 8 * C::YRB, ysw);
+            umma_f16kind(tmem_base + C::LCOL + c * C::KP, adesc, bdesc, idB, ks != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[c]);  // the chunk's slot is free once pass B has read it
+        }
+        umma_commit(ffull);
+      }
+      if (issued) {  // no MMA may still read shared memory or write TMEM when the CTA exits
+        umma_commit(fin);
+        mbar_drain(fin, 0u, status);
+      }
+    }
+  } else if (warp < FRONT_NORM_WARP0) {
+    // --------------------------------------------------------------- epilogue
+    const int q = warp & 3;                  // TMEM lane quarter
+    const int ew = warp - FRONT_EPI_WARP0;   // 0..3
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const float inv_cnt = 1.0f / static_cast<float>(C::N * C::K);
+    int64_t i = 0;
+    // After a failed wait a warp stops waiting but keeps walking the same control flow,
+    // so every named barrier still sees all four warps.
+    bool ok = true;
+    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x, ++i) {
+      const uint32_t par = static_cast<uint32_t>(i & 1);
+      // Z (TMEM, fp32) -> 16-bit MN-major operand in shared memory (once the previous
+      // example's A0 stores staged there have read it)
+      if (C::A0_TMA && lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      if (ok) ok = mbar_wait(zfull, par, status);
+      tc_fence_after();
+#pragma unroll
+      for (int mz = 0; mz < C::MTZ; ++mz) {
+        const int t = mz * C::R + q * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < C::KP / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(mz * C::KP + h * 32), r);
+          tmem_ld_wait();
+          if (t < C::D) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 u;
+              u.x = Half16<T>::pack2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+              u.y = Half16<T>::pack2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+              u.z = Half16<T>::pack2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+              u.w = Half16<T>::pack2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(front_zb_addr<C>(smem_u32(zb), t, h * 4 + j)),
+                           "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                           : "memory");
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();  // the tensor core reads these stores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(zready);
+
+      // LCB rows: accumulator + the residual X row (from the chunk in shared memory), staged
+      // 32 columns at a time and stored by TMA (rows past n_l are clipped), through this warp's
+      // own staging tile and its quarter of the Y / W_L ring, idle until the drain is done
+      for (int c = C::NF / C::R; ok && c < C::NCH; ++c) ok = mbar_wait(&xready[c], par, status);
+#pragma unroll 1
+      for (int m = 0; m < C::MTL; ++m) {
+        if (ok) ok = mbar_wait(&lfull[m], par, status);
+        tc_fence_after();
+        const int r = m * C::R + q * 32 + lane;   // LCB row
+        const bool valid = r < C::NL;
+        const bool any = m * C::R + q * 32 < C::NL;
+        const int rho = C::NF + r;                // its residual row
+        const uint8_t* xres = slots + (rho / C::R) * C::CHB;
+        const int rl = rho % C::R;
+#pragma unroll 1
+        for (int j = 0; j < C::XBOXES; ++j) {
+          uint32_t acc[32];
+          tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + m * C::D + j * 32), acc);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(acc[e]);
+          if (valid) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 xr = *reinterpret_cast<const uint4*>(xres + j * C::XBOXB + sw64_off(rl, u));
+              float x8[8];
+              front_unpack8<T>(xr, x8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[8 * u + e] += x8[e];
+            }
+          }
+          const int nb = (m * C::XBOXES + j) % C::NBUF;
+          uint8_t* stage = nb == 0 ? epi + ew * 2048 : ring + ew * (C::NBUF - 1) * 2048 + (nb - 1) * 2048;
+          if (lane == 0 && nb == 0) bulk_wait_read<0>();  // the tiles' last stores have read them
+          __syncwarp();
+          stage_row<T>(stage, lane, v);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && any) {
+            tma_store_3d(&tmL, stage, 32 * j, m * C::R + q * 32, static_cast<int32_t>(b));
+            bulk_commit();
+          }
+        }
+      }
+      tc_fence_before();
+      if (lane == 0) bulk_wait_read<0>();  // the ring is the producer's again
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ldone);
+
+      // the FMB LayerNorm over the n*k values of F
+      T* ab = A0 + b * (C::N * C::K);
+      const bool affine = fg != nullptr;
+      if constexpr (C::REGLN) {
+        // F read from TMEM once (all chunks before one wait), TMEM handed back, then mean,
+        // variance and the output from registers
+        if (ok) ok = mbar_wait(ffull, par, status);
+        tc_fence_after();
+        uint32_t fr[C::NCH][C::K];
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const uint32_t ta = tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP);
+          if constexpr (C::K == 32) {
+            tmem_ld32(ta, reinterpret_cast<uint32_t(&)[32]>(fr[c][0]));
+          } else if constexpr (C::K == 24) {
+            front_tmem_ld16(ta, reinterpret_cast<uint32_t(&)[16]>(fr[c][0]));
+            front_tmem_ld8(ta + 16, reinterpret_cast<uint32_t(&)[8]>(fr[c][16]));
+          } else {
+            front_tmem_ld16(ta, reinterpret_cast<uint32_t(&)[16]>(fr[c][0]));
+          }
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(fempty);
+        float part = 0.f;
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+          if (row < C::N) {
+#pragma unroll
+            for (int j = 0; j < C::K; ++j) part += __uint_as_float(fr[c][j]);
+          }
+        }
+        part = warp_sum(part);
+        if (lane == 0) red[ew] = part;
+        named_bar(1, 128);
+        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+        float qs = 0.f;
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+          if (row < C::N) {
+#pragma unroll
+            for (int j = 0; j < C::K; ++j) {
+              const float dv = __uint_as_float(fr[c][j]) - mean;
+              qs = fmaf(dv, dv, qs);
+            }
+          }
+        }
+        qs = warp_sum(qs);
+        if (lane == 0) red[4 + ew] = qs;
+        named_bar(1, 128);
+        const float var = (red[4] + red[5] + red[6] + red[7]) * inv_cnt;
+        const float rstd = rsqrtf(var + eps);
+        if (threadIdx.x == 32 * FRONT_EPI_WARP0 && !(isfinite(mean) && isfinite(var))) flag_error(status, kFlagNonFinite);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+          if (row < C::N) {
+            T* o = ab + row * C::K;
+#pragma unroll
+            for (int j = 0; j < C::K; j += 8) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = (__uint_as_float(fr[c][j + e]) - mean) * rstd;
+              if (affine) {
+                const float* gp = fg + row * C::K + j;
+                const float* bp = fb + row * C::K + j;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = v[e] * __ldg(gp + e) + __ldg(bp + e);
+              }
+              *reinterpret_cast<uint4*>(o + j) = front_pack8<T>(v);
+            }
+          }
+        }
+        named_bar(1, 128);  // every epilogue warp is past its reads of red[]
+      } else {
+        // three passes over F in TMEM: mean, variance, output
+        if (ok) ok = mbar_wait(ffull, par, status);
+        tc_fence_after();
+        float part = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+#pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r);
+            tmem_ld_wait();
+            if (row < C::N) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (h * 32 + j < C::K) part += __uint_as_float(r[j]);
+            }
+          }
+        }
+        part = warp_sum(part);
+        if (lane == 0) red[ew] = part;
+        named_bar(1, 128);
+        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+        float qs = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+#pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r);
+            tmem_ld_wait();
+            if (row < C::N) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (h * 32 + j < C::K) {
+                  const float dv = __uint_as_float(r[j]) - mean;
+                  qs = fmaf(dv, dv, qs);
+                }
+            }
+          }
+        }
+        qs = warp_sum(qs);
+        if (lane == 0) red[4 + ew] = qs;
+        named_bar(1, 128);
+        const float var = (red[4] + red[5] + red[6] + red[7]) * inv_cnt;
+        const float rstd = rsqrtf(var + eps);
+        if (threadIdx.x == 32 * FRONT_EPI_WARP0 && !(isfinite(mean) && isfinite(var))) flag_error(status, kFlagNonFinite);
+#pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+#pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r);
+            tmem_ld_wait();
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = (__uint_as_float(r[e]) - mean) * rstd;
+            if (affine && row < C::N) {
+              const float* gp = fg + row * C::K + h * 32;
+              const float* bp = fb + row * C::K + h * 32;
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (h * 32 + e < C::K) v[e] = v[e] * __ldg(gp + e) + __ldg(bp + e);
+            }
+            if constexpr (C::A0_TMA) {
+              const int t = c * 2 + h;  // tile, three staging buffers in turn
+              uint8_t* buf = (t % 3 == 0) ? epi + ew * 2048 : zb + ew * 4096 + (t % 3 - 1) * 2048;
+              if (lane == 0) bulk_wait_read<2>();  // the store that last used this buffer has read it
+              __syncwarp();
+              stage_row<T>(buf, lane, v);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmA, buf, 32 * h, static_cast<int32_t>(b * C::N + c * C::R + q * 32));
+                bulk_commit();
+              }
+            } else if (row < C::N) {
+              T* o = ab + row * C::K + h * 32;
+#pragma unroll
+              for (int j = 0; j < 32; j += 8)
+                if (h * 32 + j < C::K)
+                  *reinterpret_cast<uint4*>(o + j) = front_pack8<T>(reinterpret_cast<const float(&)[8]>(v[j]));
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar(1, 128);  // every epilogue warp is past its reads of red[] and F
+        if (lane == 0) mbar_arrive(fempty);
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- normalisation
+    // Two threads per row (adjacent lanes), each with half of the row's 16-byte units:
+    // the layer input's LayerNorm (two-pass fp32 statistics from registers) or, for the
+    // first layer, the conversion to the operand type, written back in place.
+    constexpr int UPR = C::D / 8;     // 16-byte units per row (of 16-bit values)
+    constexpr int UPT = UPR / 2;      // per thread
+    const int tid = threadIdx.x - 32 * FRONT_NORM_WARP0;
+    const int row = tid >> 1;
+    const int half = tid & 1;
+    int pending = -1;  // tid 0: the chunk whose residual stores are the last still reading their slot
+    int64_t i = 0;
+    bool ok = true;
+    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x, ++i) {
+      const uint32_t par = static_cast<uint32_t>(i & 1);
+      for (int c = 0; c < C::NCH; ++c) {
+        if (ok) ok = mbar_wait(&full[c], par, status);
+        const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+        uint8_t* base = slots + c * C::CHB;
+        const bool act = ok && row < rows;
+        // the row as loaded (row-major, d values), into registers; every thread reads before
+        // any thread writes the operand layout over the same bytes
+        uint4 w[UPT];
+#pragma unroll
+        for (int k = 0; k < UPT; ++k) {
+          const int g = half * UPT + k;  // unit within the row
+          w[k] = act ? *reinterpret_cast<const uint4*>(base + row * (C::D * 2) + g * 16) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        named_bar(2, FRONT_NORM_THREADS);
+        if (ln_in) {
+          float s = 0.f;
+#pragma unroll
+          for (int k = 0; k < UPT; ++k) {
+            float v[8];
+            front_unpack8<TIN>(w[k], v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += v[e];
+          }
+          s += __shfl_xor_sync(0xffffffffu, s, 1);
+          const float mean = s * (1.0f / C::D);
+          float qv = 0.f;
+#pragma unroll
+          for (int k = 0; k < UPT; ++k) {
+            float v[8];
+            front_unpack8<TIN>(w[k], v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float dv = v[e] - mean;
+              qv = fmaf(dv, dv, qv);
+            }
+          }
+          qv += __shfl_xor_sync(0xffffffffu, qv, 1);
+          const float rstd = rsqrtf(qv * (1.0f / C::D) + eps);
+          if (act && half == 0 && !(isfinite(mean) && isfinite(qv))) flag_error(status, kFlagNonFinite);
+          if (act) {
+#pragma unroll
+            for (int k = 0; k < UPT; ++k) {
+              const int g = half * UPT + k;
+              float v[8];
+              front_unpack8<TIN>(w[k], v);
+              const float4 g0 = reinterpret_cast<const float4*>(sg)[2 * g], g1 = reinterpret_cast<const float4*>(sg)[2 * g + 1];
+              const float4 b0 = reinterpret_cast<const float4*>(sb)[2 * g], b1 = reinterpret_cast<const float4*>(sb)[2 * g + 1];
+              const float ga[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+              const float be[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = (v[e] - mean) * rstd * ga[e] + be[e];
+              *reinterpret_cast<uint4*>(base + (g >> 2) * C::XBOXB + sw64_off(row, g & 3)) = front_pack8<T>(v);
+            }
+          }
+        } else if (act) {  // the first layer: the input in the operand type, in the operand layout
+#pragma unroll
+          for (int k = 0; k < UPT; ++k) {
+            const int g = half * UPT + k;
+            uint4 o = w[k];
+            if (sizeof(TIN) != sizeof(T) || Half16<TIN>::kBF16 != Half16<T>::kBF16) {
+              float v[8];
+              front_unpack8<TIN>(w[k], v);
+              o = front_pack8<T>(v);
+            }
+            *reinterpret_cast<uint4*>(base + (g >> 2) * C::XBOXB + sw64_off(row, g & 3)) = o;
+          }
+        }
+        fence_proxy_async_smem();  // the tensor core and the TMA store read the chunk
+        named_bar(2, FRONT_NORM_THREADS);
+        if (tid == 0) {
+          mbar_arrive(&xready[c]);
+          // The FMB rows' residual (rows past n_f are clipped). The slot is released (one of
+          // its two arrivals) once its stores have read it: the previous chunk's is released
+          // here, after this chunk's stores are issued, so no chunk waits for its own.
+          const bool st = ok && c * C::R < C::NF;
+          if (st) {
+#pragma unroll
+            for (int j = 0; j < C::XBOXES; ++j) tma_store_3d(&tmR, base + j * C::XBOXB, 32 * j, c * C::R,
+                                                             static_cast<int32_t>(b));
+            bulk_commit();
+          }
+          if (pending >= 0) {
+            if (st) bulk_wait_read<1>();
+            else bulk_wait_read<0>();
+            mbar_arrive(&empty[pending]);
+          }
+          pending = c;
+        }
+      }
+      if (tid == 0 && pending >= 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(&empty[pending]);
+        pending = -1;
+      }
+    }
+    if (tid == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+using FrontC2 = FrontCfg<64, 128, 16, 32>;
+using FrontC3 = FrontCfg<256, 160, 32, 128>;
+using FrontC4 = FrontCfg<512, 160, 64, 256>;
+
+}  // namespace wk

@@ -26,7 +26,8 @@
 // the CTA drains and frees TMEM, and the status word carries the flag.
 #pragma once
 
-#include "row_ln_epi.cuh"
+#include "common.cuh"
+#include "res_ln.cuh"
 
 namespace wk {
 
@@ -50,6 +51,50 @@ constexpr uint32_t gemm_smem_bytes() {
          4u * 2u * gemm_epi_buf_bytes<TO>() + 256u /* barriers + tmem slot */;
 }
 
+// Writes 32 fp32 values of one accumulator row into a 32x32 staging tile row,
+// laid out as the TMA store expects: 16-bit rows of 64 B with the 64B swizzle, or
+// fp32 rows of 128 B with the 128B swizzle.
+template <typename TO>
+__device__ __forceinline__ void stage_row(uint8_t* buf, int row, const float (&v)[32]);
+
+template <>
+__device__ __forceinline__ void stage_row<__nv_bfloat16>(uint8_t* buf, int row, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 q;
+    q.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    q.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    q.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    q.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+    const int pc = c ^ ((row >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + row * 64 + pc * 16) = q;
+  }
+}
+
+template <>
+__device__ __forceinline__ void stage_row<__half>(uint8_t* buf, int row, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 q;
+    q.x = Half16<__half>::pack2(v[8 * c + 0], v[8 * c + 1]);
+    q.y = Half16<__half>::pack2(v[8 * c + 2], v[8 * c + 3]);
+    q.z = Half16<__half>::pack2(v[8 * c + 4], v[8 * c + 5]);
+    q.w = Half16<__half>::pack2(v[8 * c + 6], v[8 * c + 7]);
+    const int pc = c ^ ((row >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + row * 64 + pc * 16) = q;
+  }
+}
+
+template <>
+__device__ __forceinline__ void stage_row<float>(uint8_t* buf, int row, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const int pc = c ^ (row & 7);
+    *reinterpret_cast<float4*>(buf + row * 128 + pc * 16) =
+        make_float4(v[4 * c + 0], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  }
+}
+
 struct GemmParams {
   int M, N, K;           // MLP: C is M x N, reduction K.  LCB: M = n_l, N = batch, K = n.
   int num_m_tiles;       // ceil(M / 128)
@@ -62,17 +107,9 @@ struct GemmParams {
   int relu;              // MLP
   int d, E, dchunks;     // LCB: embedding dim, examples per tile, d / 32
   unsigned* status;
-  // fused residual + LayerNorm epilogue (row_ln_epi.cuh): the layer input, the output
-  // LayerNorm's affine parameters, rows per example, and (LCB) the first output row
-  // or (last MLP Linear) the number of valid embedding rows.
-  const void* resid;
-  const float* ln_g;
-  const float* ln_b;
-  float ln_eps;
-  int ln_n, ln_row0, ln_rows;
-  // CTA-pair GEMM: 1 = operand loads carry L2 hints (A, the activations, kept in L2
-  // across the waves of a raster group; B, the weights, streamed through)
-  int l2hint;
+  // MLP: 1 = the epilogue adds C into what the output already holds (TMA reduce-add)
+  // instead of overwriting it
+  int reduce_out;
 };
 
 __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int mode, int& mt, int& nt) {
@@ -92,9 +129,7 @@ __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, 
 }
 
 // T: operand type (__half or __nv_bfloat16, A and B alike); TO: output type.
-// ROWLN (MODE_LCB): the epilogue finishes the layer for the LCB rows (residual +
-// LayerNorm) and tmC addresses the layer output instead of the concat buffer.
-template <int MODE, typename T, typename TO, bool ROWLN = false>
+template <int MODE, typename T, typename TO>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
@@ -247,23 +282,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       gemm_tile_coords(p, tile, MODE, mt, nt);
       if (!mbar_wait(&tfull[acc], acc_ph, p.status)) break;
       tc_fence_after();
-      if constexpr (ROWLN && MODE == MODE_LCB) {
-        const int m = mt * GEMM_BM + q * 32 + lane;  // W_L row = output row n_f + m
-        for (int e = 0; e < p.E; ++e) {
-          const int b = nt * p.E + e;
-          if (b >= p.N) break;
-          const bool valid = m < p.M;
-          const T* xr = static_cast<const T*>(p.resid) + (static_cast<int64_t>(b) * p.ln_n + p.ln_row0 + m) * p.d;
-          const uint32_t taddr =
-              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * GEMM_BN + e * p.d);
-          row_ln_epilogue<T, TO>(taddr, p.d, valid, valid ? xr : nullptr, nullptr, p.ln_g, p.ln_b, p.ln_eps, bufs,
-                                 EPI_BUF, buf, lane, [&](int c, uint8_t* sb) {
-                                   tma_store_3d(&tmC, sb, c * 32, mt * GEMM_BM + q * 32, b);
-                                   bulk_commit();
-                                 });
-        }
-      }
-      const int nchunks = ROWLN ? 0 : ((MODE == MODE_MLP) ? GEMM_BN / 32 : p.E * p.dchunks);
+      const int nchunks = (MODE == MODE_MLP) ? GEMM_BN / 32 : p.E * p.dchunks;
       for (int c = 0; c < nchunks; ++c) {
         int col0 = 0;
         if (MODE == MODE_MLP) {
@@ -309,7 +328,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         __syncwarp();
         if (lane == 0) {
           if (MODE == MODE_MLP) {
-            tma_store_2d(&tmC, sb, col0, mt * GEMM_BM + q * 32);
+            if (p.reduce_out)
+              tma_reduce_add_2d(&tmC, sb, col0, mt * GEMM_BM + q * 32);
+            else
+              tma_store_2d(&tmC, sb, col0, mt * GEMM_BM + q * 32);
           } else {
             const int e = c / p.dchunks;
             const int tc = c - e * p.dchunks;

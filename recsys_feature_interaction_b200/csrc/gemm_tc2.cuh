@@ -30,7 +30,6 @@ constexpr int GEMM2_BN = 256;
 constexpr int GEMM2_BK = 64;
 constexpr int GEMM2_STAGES = 6;
 constexpr int GEMM2_GROUP_M = 8;  // M tiles per raster group (tiles walk M fastest inside a group)
-constexpr int GEMM2_L2_HINT = 0;  // default of GemmParams::l2hint
 constexpr uint32_t GEMM2_A_STAGE = 128 * GEMM2_BK * 2;  // 16 KB: this CTA's 128 rows
 constexpr uint32_t GEMM2_B_STAGE = 128 * GEMM2_BK * 2;  // 16 KB: this CTA's half of N
 
@@ -68,22 +67,17 @@ __device__ __forceinline__ void gemm2_tile_coords(const GemmParams& p, int tile,
   nt = local / gm;
 }
 
-// p.num_m_tiles counts 256-row tiles, p.num_n_tiles tiles of p.mma_n columns
-// (256, or E = floor(256/d) whole embedding rows of the last Linear when ROWLN: then
-// the epilogue adds the bias and the residual, applies the output LayerNorm and tmC
-// addresses the layer output [M, n*d]).
+// p.num_m_tiles counts 256-row tiles, p.num_n_tiles tiles of p.mma_n = 256 columns.
 //
 // A_MN / B_MN: the operand is stored MN-major, as A^T [K, M] (W^T [K, N]) row-major with the
 // tensor map's dims (M, K) (N, K): each CTA's 128 rows then arrive as two 64-row x 64-k boxes
 // (128-byte swizzle) 8 KB apart and are read MN-major (the backward's weight gradients
 // dz^T h and input gradients dz W need no transposed copies).
-template <typename T, typename TO, bool ROWLN = false, bool STREAM = false, bool A_MN = false, bool B_MN = false>
+template <typename T, typename TO, bool STREAM = false, bool A_MN = false, bool B_MN = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using S = Gemm2Shape<STREAM>;
-  static_assert(!(STREAM && ROWLN), "the fused end-of-layer epilogue runs persistent");
-  static_assert(!(ROWLN && (A_MN || B_MN)), "MN-major operands only with the plain epilogue (mma_n = 256)");
   constexpr int GEMM2_STAGES = S::STAGES;  // shadows the persistent default
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -132,8 +126,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // leader's full[0]
-      const uint64_t pol_a = l2_policy_evict_last();
-      const uint64_t pol_b = l2_policy_evict_first();
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -153,8 +145,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 2; ++j)
               tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE + j * 8192, arow + 64 * j, kb * GEMM2_BK);
-          } else if (p.l2hint) {
-            tma_load_2d_pair_hint(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow, pol_a);
           } else {
             tma_load_2d_pair(&tmA, fbar, sA + s * GEMM2_A_STAGE, kb * GEMM2_BK, arow);
           }
@@ -162,8 +152,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 2; ++j)
               tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE + j * 8192, brow + 64 * j, kb * GEMM2_BK);
-          } else if (p.l2hint) {
-            tma_load_2d_pair_hint(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow, pol_b);
           } else {
             tma_load_2d_pair(&tmB, fbar, sB + s * GEMM2_B_STAGE, kb * GEMM2_BK, brow);
           }
@@ -247,23 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       if (!mbar_wait(&tfull[acc], acc_ph, p.status)) break;
       tc_fence_after();
       const int row0 = mt * GEMM2_BM + static_cast<int>(rank) * 128 + q * 32;
-      if constexpr (ROWLN) {
-        const int brow = row0 + lane;  // example
-        const bool valid = brow < p.M;
-        for (int e = 0; e < p.E; ++e) {
-          const int r = nt * p.E + e;  // embedding row of the FMB block
-          if (r >= p.ln_rows) break;
-          const T* xr = static_cast<const T*>(p.resid) + (static_cast<int64_t>(brow) * p.ln_n + r) * p.d;
-          const uint32_t taddr =
-              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * GEMM2_BN + e * p.d);
-          row_ln_epilogue<T, TO>(taddr, p.d, valid, valid ? xr : nullptr, p.bias ? p.bias + r * p.d : nullptr, p.ln_g,
-                                 p.ln_b, p.ln_eps, bufs, EPI_BUF, buf, lane, [&](int c, uint8_t* sb) {
-                                   tma_store_2d(&tmC, sb, r * p.d + c * 32, row0);
-                                   bulk_commit();
-                                 });
-        }
-      }
-      for (int c = 0; c < (ROWLN ? 0 : GEMM2_BN / 32); ++c) {
+      for (int c = 0; c < GEMM2_BN / 32; ++c) {
         const int col0 = nt * GEMM2_BN + c * 32;
         if (col0 >= p.N) break;
         uint32_t r[32];
@@ -302,7 +274,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmC, sb, col0, row0);
+          if (p.reduce_out)
+            tma_reduce_add_2d(&tmC, sb, col0, row0);
+          else
+            tma_store_2d(&tmC, sb, col0, row0);
           bulk_commit();
         }
         if constexpr (S::NBUF == 2) buf ^= 1;

@@ -5,7 +5,7 @@
 //
 //   g[b, :]    = softmax( W_g vec(X_b) + b_g )                      (moe_gate_kernel)
 //   out[b, i]  = sum_e g[b, e] * ( LN( cat_e[b, i] + X_b[i] ) * gamma_e + beta_e )
-//                                                                  (moe_combine_kernel)
+//                                                                  (moe_combine_ring_kernel)
 //
 // for every example b and embedding row i: each expert's own residual + LayerNorm,
 // mixed by the gate, in one pass that reads every expert's concat buffer and the layer
@@ -138,113 +138,9 @@ __global__ void __launch_bounds__(256) moe_gate_kernel(const T* __restrict__ X, 
   }
 }
 
-// The mixture of the experts' residual + LayerNorm outputs. rows = batch * n rows of
-// d values; cat_e and x in the 16-bit type T, out in TO, g [batch, E] fp32. Lane
-// layout as in res_ln_kernel: G lanes per row (G a power of two dividing d/8), each
-// lane owning VPL 16-byte vectors. Per row the residual is loaded once and kept as
-// packed 16-bit words, each expert's concat row is loaded once, one expert ahead of
-// the arithmetic (all VPL vectors at once), and kept packed too; each expert's statistics are two
-// fp32 passes over the unpacked values (registers: the fp32 mixture plus the packed
-// rows, which leaves room for two 256-thread blocks per SM at d = 160).
-template <int D, typename T, typename TO>
-__global__ void __launch_bounds__(256, 2) moe_combine_kernel(const MoePtrs p, const T* __restrict__ x,
-                                                         const float* __restrict__ g, TO* __restrict__ out,
-                                                         int64_t rows, int n, int E, float eps) {
-  static_assert(sizeof(T) == 2, "16-bit operands");
-  constexpr int VPR = D / 8;
-  constexpr int G = res_ln_lanes(VPR);
-  constexpr int VPL = VPR / G;
-  constexpr int RPW = 32 / G;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  const int sub = lane / G;
-  const int v0 = lane % G;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  const int64_t step = static_cast<int64_t>(gridDim.x) * nwarps * RPW;
-  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * nwarps + warp) * RPW + sub; r - sub < rows; r += step) {
-    const bool ok = r < rows;
-    uint4 xr[VPL];
-    float acc[VPL][8];
-#pragma unroll
-    for (int k = 0; k < VPL; ++k) {
-      xr[k] = ok ? __ldg(reinterpret_cast<const uint4*>(x + r * D + (v0 + k * G) * 8)) : zero;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[k][j] = 0.f;
-    }
-    const int64_t b = ok ? r / n : 0;
-    uint4 cn[VPL];  // the next expert's concat row, loaded one expert ahead
-#pragma unroll
-    for (int k = 0; k < VPL; ++k)
-      cn[k] = ok ? __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(p.cat[0]) + r * D + (v0 + k * G) * 8))
-                 : zero;
-    for (int e = 0; e < E; ++e) {
-      uint4 cr[VPL];
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) cr[k] = cn[k];
-      if (e + 1 < E) {
-        const T* nxt = static_cast<const T*>(p.cat[e + 1]);
-#pragma unroll
-        for (int k = 0; k < VPL; ++k)
-          cn[k] = ok ? __ldg(reinterpret_cast<const uint4*>(nxt + r * D + (v0 + k * G) * 8)) : zero;
-      }
-      // y = cat + x is recomputed from the packed words in each pass instead of being
-      // held as fp32 (the unpack is a shift or a convert per element)
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) {
-        float c8[8], x8[8];
-        Vec8<T>::unpack(cr[k], c8);
-        Vec8<T>::unpack(xr[k], x8);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s += c8[j] + x8[j];
-      }
-#pragma unroll
-      for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const float mean = s * (1.0f / D);
-      float q = 0.f;
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) {
-        float c8[8], x8[8];
-        Vec8<T>::unpack(cr[k], c8);
-        Vec8<T>::unpack(xr[k], x8);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float dv = (c8[j] + x8[j]) - mean;
-          q += dv * dv;
-        }
-      }
-#pragma unroll
-      for (int o = G / 2; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-      const float rstd = rsqrtf(q * (1.0f / D) + eps);
-      const float ge = ok ? __ldg(g + b * E + e) : 0.f;
-      const float* gam = p.gamma[e];
-      const float* bet = p.beta[e];
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) {
-        const int c = (v0 + k * G) * 8;
-        float c8[8], x8[8];
-        Vec8<T>::unpack(cr[k], c8);
-        Vec8<T>::unpack(xr[k], x8);
-        const float4 g0 = __ldg(reinterpret_cast<const float4*>(gam + c));
-        const float4 g1 = __ldg(reinterpret_cast<const float4*>(gam + c) + 1);
-        const float4 b0 = __ldg(reinterpret_cast<const float4*>(bet + c));
-        const float4 b1 = __ldg(reinterpret_cast<const float4*>(bet + c) + 1);
-        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[k][j] = fmaf(ge, ((c8[j] + x8[j]) - mean) * rstd * gg[j] + bb[j], acc[k][j]);
-      }
-    }
-    if (ok) {
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) Vec8<TO>::store(out + r * D + (v0 + k * G) * 8, acc[k]);
-    }
-  }
-}
-
-// The same mixture fed by bulk copies (the design of res_ln_ring_kernel): the rows
-// are walked in blocks of R rows, and for each block the producer thread streams E + 1
+// The mixture of the experts' residual + LayerNorm outputs, rows = batch * n rows of d
+// values (cat_e and x in the 16-bit type T, out in TO, g [batch, E] fp32), fed by bulk
+// copies (the design of res_ln_ring_kernel): the rows are walked in blocks of R rows, and for each block the producer thread streams E + 1
 // contiguous byte ranges -- the layer input's rows, then every expert's concat rows --
 // into consecutive slots of a ring in shared memory (untiled cp.async.bulk, one
 // mbarrier per slot). Eight consumer warps move the input rows into registers and

@@ -5,6 +5,9 @@
 //
 //   out[r, :] = LN( cat[r, :] + x[r, :] ) * gamma + beta,   r < rows, d values per row
 //
+// (x may be null: then out = LN(cat) * gamma + beta, the output LayerNorm of a stack whose
+// last layer has already added its residual into cat).
+//
 // HBM-bound (each element read twice, written once). A block of R consecutive rows
 // is one contiguous byte range in both inputs, so one persistent CTA per SM keeps a
 // ring of STAGES such blocks in flight with untiled bulk copies (cp.async.bulk, one
@@ -78,9 +81,9 @@ __global__ void __launch_bounds__(ResLnRing<D>::THREADS, 1)
         const int64_t nr = rows - r0 < C::R ? rows - r0 : C::R;
         const uint32_t bytes = static_cast<uint32_t>(nr) * C::ROW_B;
         uint8_t* dst = smem + slot * 2 * C::TILE_B;
-        mbar_arrive_expect_tx(&full[slot], 2u * bytes);
+        mbar_arrive_expect_tx(&full[slot], (x ? 2u : 1u) * bytes);
         bulk_load(dst, cat + r0 * D, bytes, &full[slot]);
-        bulk_load(dst + C::TILE_B, x + r0 * D, bytes, &full[slot]);
+        if (x) bulk_load(dst + C::TILE_B, x + r0 * D, bytes, &full[slot]);
         if (++slot == C::STAGES) {
           slot = 0;
           phase ^= 1u;
@@ -126,9 +129,9 @@ __global__ void __launch_bounds__(ResLnRing<D>::THREADS, 1)
 #pragma unroll
       for (int k = 0; k < C::VPL; ++k) {
         const int off = lr * C::ROW_B + (v0 + k * C::G) * 16;
-        float c8[8], x8[8];
+        float c8[8], x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         Vec8<TC>::load_shared(tc + off, c8);
-        Vec8<TR>::load_shared(tx + off, x8);
+        if (x) Vec8<TR>::load_shared(tx + off, x8);
 #pragma unroll
         for (int j = 0; j < 8; ++j) y[k][j] = ok ? c8[j] + x8[j] : 0.f;
       }
@@ -151,6 +154,8 @@ __global__ void __launch_bounds__(ResLnRing<D>::THREADS, 1)
 #pragma unroll
       for (int o = C::G / 2; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
       const float rstd = rsqrtf(q * (1.0f / D) + eps);
+      // an inf / NaN anywhere in the row (a 16-bit intermediate that overflowed upstream)
+      if (ok && v0 == 0 && !(isfinite(mean) && isfinite(q))) flag_error(status, kFlagNonFinite);
       if (ok) {
         TO* orow = out + (r0 + lr) * D;
 #pragma unroll

@@ -5,7 +5,7 @@
 // would launch returns WK_ERR_CUDA.
 //
 // Layer order on the stream (Wukong page, section 2.2; per layer i):
-//   1. FM + LayerNorm      X_i -> A0                          (fm_mma.cuh / simt.cuh)
+//   1. FM + LayerNorm      X_i -> A0                          (fm_tc.cuh / simt.cuh)
 //   2. MLP Linears         A0 -> ... -> concat rows 0..n_F-1   (gemm_tc.cuh, MODE_MLP)
 //   3. LCB                 X_i -> concat rows n_F..n-1         (gemm_tc.cuh, MODE_LCB)
 //   4. residual + LN       concat + X_i -> X_{i+1}             (res_ln.cuh)
@@ -29,8 +29,8 @@
 #include "wukong.h"
 #include "common.cuh"
 #include "convert.cuh"
-#include "fm_mma.cuh"
 #include "fm_tc.cuh"
+#include "front_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
 #include "head.cuh"
@@ -206,123 +206,56 @@ bool map_lcb_out(const DevInfo* dv, CUtensorMap* m, const void* cat, uint64_t ro
                   es == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int MODE, typename T, typename TO, bool ROWLN = false>
+// Rows [r0, r0 + nr) of each example of a [batch, n, d] 16-bit tensor as a (d, nr, batch)
+// tensor: boxes (32, box_rows, 1), 64B swizzle (stores past row nr are clipped).
+template <typename T>
+bool map_rows3(const DevInfo* dv, CUtensorMap* m, const void* base, uint64_t n, uint64_t d, uint64_t r0, uint64_t nr,
+               uint64_t batch, uint32_t box_rows) {
+  const uint64_t dims[3] = {d, nr, batch};
+  const uint64_t str[2] = {d * 2, n * d * 2};
+  const uint32_t box[3] = {32, box_rows, 1};
+  const uint8_t* b = static_cast<const uint8_t*>(base) + r0 * d * 2;
+  return make_map(dv, m, tmap_dtype<T>(), 3, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+template <int MODE, typename T, typename TO>
 wk_status run_gemm_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
   constexpr uint32_t smem = gemm_smem_bytes<TO>();
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc_kernel<MODE, T, TO, ROWLN>), smem);
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc_kernel<MODE, T, TO>), smem);
   if (s != WK_OK) return s;
   if (p.num_tiles <= 0) return WK_OK;
   const int grid = std::min(p.num_tiles, dv->sms);
-  gemm_tc_kernel<MODE, T, TO, ROWLN><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  gemm_tc_kernel<MODE, T, TO><<<grid, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
 }
 
-// The CTA-pair GEMM's launch shape: streaming (one pair per output tile, two pairs'
-// CTAs per SM; gemm_tc2.cuh) unless the environment sets WK_GEMM_STREAM=0, which
-// selects the persistent shape (one pair per two SMs). Measured on the 8-layer stack:
-// streaming reads 2.3-2.9x fewer DRAM bytes per Linear and runs the step ~5 % faster
-// under the power cap.
-bool gemm2_stream() {
-  static const bool on = [] {
-    const char* e = getenv("WK_GEMM_STREAM");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
-// stream: the launch shape (streaming or persistent, see gemm_tc2.cuh); -1 = gemm2_stream().
-template <typename T, typename TO, bool ROWLN = false, bool A_MN = false, bool B_MN = false>
-wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st, int stream = -1) {
+// The CTA-pair GEMM in one of its two launch shapes (gemm_tc2.cuh): streaming (one pair
+// per output tile, two pairs' CTAs per SM; the forward's Linears: measured on the 8-layer
+// stack it reads 2.3-2.9x fewer DRAM bytes per Linear than the persistent shape and runs
+// the step ~5 % faster under the power cap) or persistent (one pair per two SMs, two TMEM
+// accumulators: the backward's weight gradients, whose short K leaves the streaming
+// shape's single accumulator exposed).
+template <typename T, typename TO, bool A_MN = false, bool B_MN = false>
+wk_status run_gemm_tc2(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st,
+                       bool stream = true) {
   if (p.num_tiles <= 0) return WK_OK;
-  if constexpr (!ROWLN) {
-    if (stream < 0 ? gemm2_stream() : stream != 0) {
-      constexpr uint32_t smem = gemm2_smem_bytes<TO, true>();
-      wk_status s =
-          smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, false, true, A_MN, B_MN>), smem);
-      if (s != WK_OK) return s;
-      gemm_tc2_kernel<T, TO, false, true, A_MN, B_MN><<<2 * p.num_tiles, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
-      return launch_status();
-    }
+  if (stream) {
+    constexpr uint32_t smem = gemm2_smem_bytes<TO, true>();
+    wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, true, A_MN, B_MN>), smem);
+    if (s != WK_OK) return s;
+    gemm_tc2_kernel<T, TO, true, A_MN, B_MN><<<2 * p.num_tiles, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+    return launch_status();
   }
   constexpr uint32_t smem = gemm2_smem_bytes<TO>();
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, ROWLN, false, A_MN, B_MN>), smem);
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(gemm_tc2_kernel<T, TO, false, A_MN, B_MN>), smem);
   if (s != WK_OK) return s;
   const int pairs = std::min(p.num_tiles, dv->sms / 2);
-  gemm_tc2_kernel<T, TO, ROWLN, false, A_MN, B_MN><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
+  gemm_tc2_kernel<T, TO, false, A_MN, B_MN><<<2 * pairs, GEMM_THREADS, smem, st>>>(mp.A, mp.B, mp.C, p);
   return launch_status();
 }
 
-// With WK_FUSED_LN=1 in the environment, the end of each layer (residual + output
-// LayerNorm) runs inside the epilogues of the last FMB Linear and of the LCB instead
-// of a separate residual + LayerNorm pass. Off by default: tiling the last Linear by
-// whole embedding rows caps its MMA width at d (160 of 256 columns on the 8-layer
-// d=160 stack), which costs more tensor time than the separate pass moves in bytes.
-bool use_fused_ln() {
-  static const bool on = [] {
-    const char* e = getenv("WK_FUSED_LN");
-    return e && e[0] == '1';
-  }();
-  return on;
-}
-
-// Last FMB Linear tiled by E = floor(256/d) whole embedding rows, epilogue finishing
-// the layer for rows 0..n_f-1.
-GemmParams mlp2_rowln_params(int64_t M, int K, int n, int d, int n_f, const float* bias, const void* resid,
-                             const float* g, const float* b, float eps, unsigned* status) {
-  GemmParams p{};
-  p.M = static_cast<int>(M);
-  p.N = n_f * d;
-  p.K = K;
-  p.d = d;
-  p.E = GEMM2_BN / d;
-  p.mma_n = p.E * d;
-  p.num_m_tiles = static_cast<int>((M + GEMM2_BM - 1) / GEMM2_BM);
-  p.num_n_tiles = (n_f + p.E - 1) / p.E;
-  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
-  p.num_kb = (K + GEMM2_BK - 1) / GEMM2_BK;
-  p.group_m = 8;
-  p.bias = bias;
-  p.status = status;
-  p.resid = resid;
-  p.ln_g = g;
-  p.ln_b = b;
-  p.ln_eps = eps;
-  p.ln_n = n;
-  p.ln_rows = n_f;
-  return p;
-}
-
-// The CTA-pair GEMM (256-row tiles) serves every M above one 128-row tile unless
-// the environment sets WK_PAIR_GEMM=0.
-bool use_pair_gemm(int64_t M) {
-  static const bool enabled = [] {
-    const char* e = getenv("WK_PAIR_GEMM");
-    return !(e && e[0] == '0');
-  }();
-  return enabled && M > GEMM_BM;
-}
-
-// M tiles per raster group of the CTA-pair GEMM (tiles walk M fastest inside a group
-// of group_m M tiles, so a wave shares both operand panels through L2);
-// WK_GEMM_GROUP_M overrides the default GEMM2_GROUP_M.
-int gemm2_group_m() {
-  static const int g = [] {
-    const char* e = getenv("WK_GEMM_GROUP_M");
-    const int v = e ? atoi(e) : 0;
-    return v >= 1 && v <= 64 ? v : GEMM2_GROUP_M;
-  }();
-  return g;
-}
-
-// L2 hints on the CTA-pair GEMM's operand loads (GemmParams::l2hint); WK_GEMM_L2_HINT
-// overrides the default GEMM2_L2_HINT.
-int gemm2_l2hint() {
-  static const int h = [] {
-    const char* e = getenv("WK_GEMM_L2_HINT");
-    return e ? (e[0] == '1' ? 1 : 0) : GEMM2_L2_HINT;
-  }();
-  return h;
-}
+// The CTA-pair GEMM (256-row tiles) serves every M above one 128-row tile.
+bool use_pair_gemm(int64_t M) { return M > GEMM_BM; }
 
 GemmParams mlp2_params(int64_t M, int K, int N, const float* bias, int relu, unsigned* status) {
   GemmParams p{};
@@ -333,8 +266,7 @@ GemmParams mlp2_params(int64_t M, int K, int N, const float* bias, int relu, uns
   p.num_n_tiles = (N + GEMM2_BN - 1) / GEMM2_BN;
   p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   p.num_kb = (K + GEMM2_BK - 1) / GEMM2_BK;
-  p.group_m = gemm2_group_m();
-  p.l2hint = gemm2_l2hint();
+  p.group_m = GEMM2_GROUP_M;
   p.mma_n = GEMM2_BN;
   p.bias = bias;
   p.relu = relu;
@@ -377,20 +309,12 @@ GemmParams lcb_params(int64_t batch, int n, int d, int n_l, unsigned* status) {
 }
 
 // The LCB with W_L resident in shared memory (lcb_tc.cuh) wherever its K panel fits,
-// unless the environment sets WK_LCB_RESIDENT=0 (then the streaming GEMM).
-bool use_lcb_resident() {
-  static const bool on = [] {
-    const char* e = getenv("WK_LCB_RESIDENT");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
+// else the streaming GEMM (MODE_LCB).
 template <typename T, typename TO>
 wk_status run_lcb_tc(const DevInfo* dv, const GemmMaps& mp, const GemmParams& p, cudaStream_t st) {
   const uint32_t b_stage = static_cast<uint32_t>(p.E * p.dchunks) * 4096u;
   const int stages = lcb_tc_stages<TO>(p.num_kb, b_stage);
-  if (!use_lcb_resident() || p.num_kb > LCB_MAX_KB || stages < 2 || p.num_m_tiles > dv->sms)
+  if (p.num_kb > LCB_MAX_KB || stages < 2 || p.num_m_tiles > dv->sms)
     return run_gemm_tc<MODE_LCB, T, TO>(dv, mp, p, st);
   wk_status s = smem_attr(dv, reinterpret_cast<const void*>(lcb_tc_kernel<T, TO>), static_cast<int>(LCB_SMEM_BUDGET));
   if (s != WK_OK) return s;
@@ -412,34 +336,6 @@ bool lcb_tc_ok(int64_t batch, int n, int d) {
 }
 
 // ------------------------------------------------------------------ FM + LN
-
-template <class C, typename T>
-wk_status run_fm_mma(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
-                     float eps, unsigned* status, cudaStream_t st) {
-  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(fm_ln_mma_kernel<C, T>), C::SMEM);
-  if (s != WK_OK) return s;
-  CUtensorMap tmX, tmY;
-  {  // X as [batch*n rows, d]: 32-column boxes of R rows, 64B swizzle
-    const uint64_t dims[2] = {static_cast<uint64_t>(C::D), static_cast<uint64_t>(batch) * C::N};
-    const uint64_t str[1] = {static_cast<uint64_t>(C::D) * 2};
-    const uint32_t box[2] = {32, static_cast<uint32_t>(C::R)};
-    if (!make_map(dv, &tmX, tmap_dtype<T>(), 2, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
-      return WK_ERR_UNSUPPORTED;
-  }
-  {  // Y [n, k]: box k x R, swizzle by row width
-    const uint64_t dims[2] = {static_cast<uint64_t>(C::KC), static_cast<uint64_t>(C::N)};
-    const uint64_t str[1] = {static_cast<uint64_t>(C::KC) * 2};
-    const uint32_t box[2] = {static_cast<uint32_t>(C::KC), static_cast<uint32_t>(C::R)};
-    const CUtensorMapSwizzle sw = C::YSW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                                  : C::YSW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                  : C::YSW == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
-    if (!make_map(dv, &tmY, tmap_dtype<T>(), 2, Y, dims, str, box, sw)) return WK_ERR_UNSUPPORTED;
-  }
-  const int grid = static_cast<int>(std::min<int64_t>(batch, dv->sms));
-  fm_ln_mma_kernel<C, T><<<grid, FM_THREADS, C::SMEM, st>>>(tmX, tmY, g, b, A0, batch, eps, status);
-  return launch_status();
-}
 
 template <class C, typename T>
 wk_status run_fm_tc(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
@@ -468,16 +364,6 @@ wk_status run_fm_tc(const DevInfo* dv, const T* X, const T* Y, const float* g, c
   return launch_status();
 }
 
-// The tcgen05 FM serves the instantiated shapes unless the environment sets
-// WK_FM_MMA_SYNC=1, which selects the warp-level-MMA kernel.
-bool use_fm_mma_sync() {
-  static const bool on = [] {
-    const char* e = getenv("WK_FM_MMA_SYNC");
-    return e && e[0] == '1';
-  }();
-  return on;
-}
-
 size_t fm_simt_smem(int n, int d, int k) {
   return sizeof(float) * (static_cast<size_t>(n) * d + 2ull * n * k + static_cast<size_t>(d) * k);
 }
@@ -496,7 +382,7 @@ wk_status run_fm_simt(const DevInfo* dv, const T* X, const T* Y, const float* g,
   return launch_status();
 }
 
-bool fm_mma_shape(int n, int d, int k) {
+bool fm_tc_shape(int n, int d, int k) {
   return (n == 512 && d == 160 && k == 64) || (n == 256 && d == 160 && k == 32) || (n == 64 && d == 128 && k == 16) ||
          (n == 720 && d == 32 && k == 24);
 }
@@ -505,41 +391,66 @@ bool fm_mma_shape(int n, int d, int k) {
 template <typename T>
 wk_status run_fm16(const DevInfo* dv, const T* X, const T* Y, const float* g, const float* b, T* A0, int64_t batch,
                    int n, int d, int k, float eps, unsigned* status, cudaStream_t st) {
-  if (!use_fm_mma_sync()) {
-    if (n == 512 && d == 160 && k == 64) return run_fm_tc<FmTcC4, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-    if (n == 256 && d == 160 && k == 32) return run_fm_tc<FmTcC3, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-    if (n == 64 && d == 128 && k == 16) return run_fm_tc<FmTcC2, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-    if (n == 720 && d == 32 && k == 24) return run_fm_tc<FmTcC5, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  }
-  if (n == 512 && d == 160 && k == 64) return run_fm_mma<FmC4, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  if (n == 256 && d == 160 && k == 32) return run_fm_mma<FmC3, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  if (n == 64 && d == 128 && k == 16) return run_fm_mma<FmC2, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
-  if (n == 720 && d == 32 && k == 24) return run_fm_mma<FmC5, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 512 && d == 160 && k == 64) return run_fm_tc<FmTcC4, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 256 && d == 160 && k == 32) return run_fm_tc<FmTcC3, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 64 && d == 128 && k == 16) return run_fm_tc<FmTcC2, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
+  if (n == 720 && d == 32 && k == 24) return run_fm_tc<FmTcC5, T>(dv, X, Y, g, b, A0, batch, eps, status, st);
   return run_fm_simt<T>(dv, X, Y, g, b, A0, batch, n, d, k, eps, st);
 }
 
+// ------------------------------------------------------------- layer front
+
+// The shapes the front kernel is instantiated for (FrontC2..C4): 0..2, or -1.
+int front_shape(int n, int d, int k, int n_f) {
+  if (n == 64 && d == 128 && k == 16 && n_f == 32) return 0;
+  if (n == 256 && d == 160 && k == 32 && n_f == 128) return 1;
+  if (n == 512 && d == 160 && k == 64 && n_f == 256) return 2;
+  return -1;
+}
+
+struct FrontMaps {
+  CUtensorMap Y, W, R, L, A;
+};
+
+template <class C, typename TIN, typename T>
+wk_status run_front_c(const DevInfo* dv, const FrontMaps& mp, const TIN* xin, const float* in_g, const float* in_b,
+                      const float* fg, const float* fb, T* A0, int64_t batch, float eps, unsigned* status,
+                      cudaStream_t st) {
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(front_tc_kernel<C, TIN, T>), C::SMEM);
+  if (s != WK_OK) return s;
+  const int grid = static_cast<int>(std::min<int64_t>(batch, dv->sms));
+  front_tc_kernel<C, TIN, T><<<grid, FRONT_THREADS, C::SMEM, st>>>(xin, mp.Y, mp.W, mp.R, mp.L, mp.A, in_g, in_b, fg,
+                                                                   fb, A0, batch, eps, status);
+  return launch_status();
+}
+
+template <typename TIN, typename T>
+wk_status run_front(const DevInfo* dv, int shape, const FrontMaps& mp, const TIN* xin, const float* in_g,
+                    const float* in_b, const float* fg, const float* fb, T* A0, int64_t batch, float eps,
+                    unsigned* status, cudaStream_t st) {
+  switch (shape) {
+    case 0: return run_front_c<FrontC2, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, batch, eps, status, st);
+    case 1: return run_front_c<FrontC3, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, batch, eps, status, st);
+    case 2: return run_front_c<FrontC4, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, batch, eps, status, st);
+    default: return WK_ERR_UNSUPPORTED;
+  }
+}
+
 bool fm_supported(int n, int d, int k, bool sixteen_bit) {
-  if (sixteen_bit && fm_mma_shape(n, d, k)) return true;
+  if (sixteen_bit && fm_tc_shape(n, d, k)) return true;
   return fm_simt_smem(n, d, k) <= 200 * 1024;
 }
 
 // ------------------------------------------------------------ residual + LN
 
-// The bulk-copy ring kernel for 16-bit inputs unless the environment sets
-// WK_RES_LN_RING=0 (then the register-only kernel, which also serves fp32).
-bool use_res_ln_ring() {
-  static const bool on = [] {
-    const char* e = getenv("WK_RES_LN_RING");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
+// The bulk-copy ring kernel for 16-bit inputs (16-byte aligned), else the register-only
+// kernel (fp32, and the stand-alone call's unaligned 16-bit inputs); a null residual x
+// (the output LayerNorm alone) only on the ring.
 template <int D, typename TC, typename TR, typename TO>
 wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const float* g, const float* b, TO* out,
                        int64_t rows, float eps, unsigned* status, cudaStream_t st) {
   if constexpr (sizeof(TC) == 2 && sizeof(TR) == 2) {
-    if (use_res_ln_ring() && al16(cat) && al16(x)) {
+    if (al16(cat) && al16(x)) {
       using C = ResLnRing<D>;
       wk_status s = smem_attr(dv, reinterpret_cast<const void*>(res_ln_ring_kernel<D, TC, TR, TO>), C::SMEM);
       if (s != WK_OK) return s;
@@ -628,33 +539,15 @@ wk_status run_moe_gate(const DevInfo* dv, const T* X, const T* Wg, const float* 
   }
 }
 
-// The ring-fed mixture kernel (moe_combine_ring_kernel) unless the environment sets
-// WK_MOE_RING=0 (then the register-only moe_combine_kernel).
-bool use_moe_ring() {
-  static const bool on = [] {
-    const char* e = getenv("WK_MOE_RING");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
 template <int D, typename T, typename TO>
 wk_status run_moe_combine_d(const DevInfo* dv, const MoePtrs& p, const T* x, const float* g, TO* out, int64_t rows,
                             int n, int E, float eps, unsigned* status, cudaStream_t st) {
-  if (use_moe_ring()) {
-    using R = MoeRing<D>;
-    wk_status s = smem_attr(dv, reinterpret_cast<const void*>(moe_combine_ring_kernel<D, T, TO>), R::SMEM);
-    if (s != WK_OK) return s;
-    const int64_t tiles = (rows + R::R - 1) / R::R;
-    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, dv->sms)));
-    moe_combine_ring_kernel<D, T, TO><<<grid, R::THREADS, R::SMEM, st>>>(p, x, g, out, rows, n, E, eps, status);
-    return launch_status();
-  }
-  constexpr int G = res_ln_lanes(D / 8);
-  constexpr int rows_per_block = 8 * (32 / G);
-  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(dv->sms) * 8));
-  moe_combine_kernel<D, T, TO><<<static_cast<int>(blocks), 256, 0, st>>>(p, x, g, out, rows, n, E, eps);
+  using R = MoeRing<D>;
+  wk_status s = smem_attr(dv, reinterpret_cast<const void*>(moe_combine_ring_kernel<D, T, TO>), R::SMEM);
+  if (s != WK_OK) return s;
+  const int64_t tiles = (rows + R::R - 1) / R::R;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, dv->sms)));
+  moe_combine_ring_kernel<D, T, TO><<<grid, R::THREADS, R::SMEM, st>>>(p, x, g, out, rows, n, E, eps, status);
   return launch_status();
 }
 
@@ -727,14 +620,17 @@ struct wk_stack {
   // TMA descriptors of the tensor-core path
   bool tc_mlp = false, tc_lcb = false;
   bool pair = false;                            // MLP Linears on CTA pairs (gemm_tc2.cuh)
-  bool fused = false;                           // residual + LN in the last Linear / LCB epilogues
   bool front_only = false;                      // an expert of a wk_moe: no layer buffers, no fused path
-  std::vector<GemmMaps> last_maps;              // [layer]: fused last Linear (B box mma_n/2 rows, C = Xs[l%2])
-  CUtensorMap lcbC_x[2];                        // LCB rows n_f.. of Xs[0] / Xs[1]
   std::vector<std::vector<GemmMaps>> mlp_maps;  // [layer][j]
   std::vector<CUtensorMap> lcbA;                // [layer]
   CUtensorMap lcbB_ws[2];
   CUtensorMap lcbC;
+  // the layer front in one kernel (front_tc.cuh): its shape (-1: not used), Y, W_L and A0
+  // per layer, and the layer buffers Xs[0] / Xs[1] as a front's residual and LCB outputs
+  // (R, L) and as the last Linear's reduce-add target (C)
+  int front = -1;
+  std::vector<FrontMaps> fmaps;                 // [layer]: Y, W, A
+  CUtensorMap frontR[2], frontL[2], frontC[2];
   // prediction head (wk_stack_set_head): q Linears, dims n*d -> ... -> 1
   std::vector<int32_t> head_dims;               // empty: no head
   std::vector<const void*> hT;                  // [q] operand type
@@ -895,22 +791,46 @@ wk_status build_maps(wk_stack* h) {
         if (!ok) return WK_ERR_UNSUPPORTED;
       }
   }
-  h->fused = h->tc_mlp && h->pair && h->tc_lcb && use_fused_ln() && d <= GEMM2_BN && !h->front_only;
-  if (h->fused) {
-    const int E = GEMM2_BN / d;
-    h->last_maps.resize(L);
+  const int shape = front_shape(n, d, c.k, c.n_f);
+  // fp16 operands only: the front keeps each layer's output before its LayerNorm in the
+  // operand type (the last Linear adds into it), one rounding more than the separate
+  // residual + LayerNorm pass, which bf16's 8-bit significand cannot spare on the 2-layer
+  // workload (0.0211 against 0.0161 with the four-kernel layer, tolerance 0.02)
+  const bool front_types = h->op == WK_F16;
+  // The front streams W_L from L2 once per example: worth it while W_L's rows per example
+  // (n_l x n) stay within twice the example's own n x d (the wide/narrow workload, n_l = 360
+  // against d = 32, reads 11x its input's bytes of W_L and keeps the four-kernel layer, whose
+  // LCB shares each W_L load among several examples)
+  const bool front_lcb = c.n_l <= 2 * d;
+  if (h->tc_mlp && !h->front_only && shape >= 0 && front_types && front_lcb) {
+    const int KP = c.k <= 32 ? 32 : 64;
+    h->fmaps.resize(L);
+    bool ok = true;
     for (int l = 0; l < L; ++l) {
-      GemmMaps& mp = h->last_maps[l];
-      const int j = m - 1;
-      const void* in = (j == 0) ? h->A0 : h->H[(j - 1) % 2];
-      const bool ok = map_kmajor<T>(dv, &mp.A, in, h->dims[j], B, GEMM_BM) &&
-                      map_kmajor<T>(dv, &mp.B, h->W[l][j], h->dims[j], h->dims[j + 1], (E * d) / 2) &&
-                      map_out<T>(dv, &mp.C, h->Xs[l % 2], static_cast<uint64_t>(c.n_f) * d, B, nd);
-      if (!ok) return WK_ERR_UNSUPPORTED;
+      // Y [n, k]: boxes of KP columns (zero past k) x 128 rows
+      const uint64_t ydims[2] = {static_cast<uint64_t>(c.k), static_cast<uint64_t>(n)};
+      const uint64_t ystr[1] = {static_cast<uint64_t>(c.k) * 2};
+      const uint32_t ybox[2] = {static_cast<uint32_t>(KP), 128};
+      ok = ok && make_map(dv, &h->fmaps[l].Y, tmap_dtype<T>(), 2, h->Y[l], ydims, ystr, ybox,
+                          KP == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+      ok = ok && map_kmajor<T>(dv, &h->fmaps[l].W, h->WL[l], n, c.n_l, 128);
     }
-    if (!map_lcb_out<T>(dv, &h->lcbC_x[0], h->Xs[0], n, d, c.n_f, c.n_l, B) ||
-        !map_lcb_out<T>(dv, &h->lcbC_x[1], h->Xs[1], n, d, c.n_f, c.n_l, B))
-      return WK_ERR_UNSUPPORTED;
+    {  // A0 [B*n rows, k]: boxes of (up to) 32 columns x 32 rows
+      const uint64_t adims[2] = {static_cast<uint64_t>(c.k), static_cast<uint64_t>(B) * n};
+      const uint64_t astr[1] = {static_cast<uint64_t>(c.k) * 2};
+      const uint32_t abox[2] = {static_cast<uint32_t>(std::min(c.k, 32)), 32};
+      const CUtensorMapSwizzle asw = c.k >= 32   ? CU_TENSOR_MAP_SWIZZLE_64B
+                                     : c.k == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
+      for (int l = 0; l < L; ++l)
+        ok = ok && make_map(dv, &h->fmaps[l].A, tmap_dtype<T>(), 2, h->A0, adims, astr, abox, asw);
+    }
+    for (int i = 0; i < 2; ++i)
+      ok = ok && map_rows3<T>(dv, &h->frontR[i], h->Xs[i], n, d, 0, c.n_f, B, std::min(128, c.n_f)) &&
+           map_rows3<T>(dv, &h->frontL[i], h->Xs[i], n, d, c.n_f, c.n_l, B, 32) &&
+           map_out<T>(dv, &h->frontC[i], h->Xs[i], static_cast<uint64_t>(c.n_f) * d, B, nd);
+    if (!ok) return WK_ERR_UNSUPPORTED;
+    h->front = shape;
   }
   if (h->tc_lcb) {
     h->lcbA.resize(L);
@@ -975,10 +895,61 @@ wk_status layer_front16(wk_stack* h, int l, const T* xin, const CUtensorMap& lcb
   return s;
 }
 
+// The forward of a 16-bit stack through the one-kernel layer front (front_tc.cuh). Per
+// layer l: the front reads the previous layer's output before its LayerNorm (the caller's
+// X for l = 0), writes A0 and the layer output's LCB rows and FMB-row residual into
+// Xs[l % 2]; the MLP runs on A0 and its last Linear adds its output into those FMB rows.
+// The stack's output is the last layer's output LayerNorm of Xs[(L - 1) % 2].
+template <typename T, typename IO, typename OUT>
+wk_status forward16_front(wk_stack* h, const void* X, void* out, int64_t batch, cudaStream_t st) {
+  const wk_stack_config& c = h->cfg;
+  const DevInfo* dv = h->dv;
+  const int n = c.n, d = c.d, m = c.mlp_num_linear, L = c.num_layers;
+  wk_status s = WK_OK;
+  for (int l = 0; l < L && s == WK_OK; ++l) {
+    const int o = l % 2;
+    FrontMaps fm = h->fmaps[l];
+    fm.R = h->frontR[o];
+    fm.L = h->frontL[o];
+    {
+      ProfScope ps(h, WK_KERNEL_FRONT, st);
+      if (l == 0)
+        s = run_front<IO, T>(dv, h->front, fm, static_cast<const IO*>(X), nullptr, nullptr, h->g1[l], h->b1[l],
+                             static_cast<T*>(h->A0), batch, h->eps, h->status, st);
+      else
+        s = run_front<T, T>(dv, h->front, fm, static_cast<const T*>(h->Xs[(l - 1) % 2]), h->g2[l - 1], h->b2[l - 1],
+                            h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, h->eps, h->status, st);
+    }
+    for (int j = 0; j < m && s == WK_OK; ++j) {
+      ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
+      const bool lastj = j == m - 1;
+      GemmMaps mp = h->mlp_maps[l][j];
+      if (lastj) mp.C = h->frontC[o];
+      if (h->pair) {
+        GemmParams p = mlp2_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], lastj ? 0 : 1, h->status);
+        p.reduce_out = lastj ? 1 : 0;
+        s = run_gemm_tc2<T, T>(dv, mp, p, st);
+      } else {
+        GemmParams p = mlp_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], lastj ? 0 : 1, h->status);
+        p.reduce_out = lastj ? 1 : 0;
+        s = run_gemm_tc<MODE_MLP, T, T>(dv, mp, p, st);
+      }
+    }
+  }
+  if (s != WK_OK) return s;
+  ProfScope ps(h, WK_KERNEL_RES_LN, st);
+  return run_res_ln<T, T, OUT>(dv, static_cast<const T*>(h->Xs[(L - 1) % 2]), static_cast<const T*>(nullptr),
+                               h->g2[L - 1], h->b2[L - 1], static_cast<OUT*>(out), batch * n, d, h->eps, h->status, st);
+}
+
 // The forward of a 16-bit stack with operand type T, input type IO and output type
 // OUT (the caller's type, or T when the prediction head reads the output).
 template <typename T, typename IO, typename OUT = IO>
 wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaStream_t st) {
+  constexpr bool kFrontTypes = std::is_same<T, f16>::value;
+  if constexpr (kFrontTypes) {
+    if (h->front >= 0) return forward16_front<T, IO, OUT>(h, X, out, batch, st);
+  }
   const wk_stack_config& c = h->cfg;
   const DevInfo* dv = h->dv;
   const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers;
@@ -996,65 +967,11 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
   } else if (h->tc_lcb && !map_lcb_x<T>(dv, &lcb_x0, X, n, d, batch)) {
     return WK_ERR_CUDA;
   }
-  CUtensorMap out_last, out_lcb;  // the caller's output as the fused epilogues' destination
-  if (h->fused && (!map_out<OUT>(dv, &out_last, out, static_cast<uint64_t>(c.n_f) * d, batch, nd) ||
-                   !map_lcb_out<OUT>(dv, &out_lcb, out, n, d, c.n_f, c.n_l, batch)))
-    return WK_ERR_CUDA;
   for (int l = 0; l < L && s == WK_OK; ++l) {
     const bool last = l == L - 1;
     const T* xin = static_cast<const T*>(l == 0 ? x0 : h->Xs[(l - 1) % 2]);
-    if (!h->fused) {
-      s = layer_front16<T>(h, l, xin, (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2], batch, st);
-      if (s != WK_OK) break;
-    } else {
-      {  // 1. FM + LN
-        ProfScope ps(h, WK_KERNEL_FM_LN, st);
-        s = run_fm16<T>(dv, xin, static_cast<const T*>(h->Y[l]), h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, n,
-                        d, k, h->eps, h->status, st);
-      }
-      for (int j = 0; j < m - 1 && s == WK_OK; ++j) {  // 2. MLP Linears but the last
-        ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
-        s = run_gemm_tc2<T, T>(dv, h->mlp_maps[l][j], mlp2_params(batch, h->dims[j], h->dims[j + 1], h->b[l][j], 1,
-                                                                  h->status), st);
-      }
-      if (s != WK_OK) break;
-      // 2'. last Linear + residual + LN -> rows 0..n_f-1 of X_{i+1};
-      // 3'. LCB + residual + LN -> rows n_f..n-1 of X_{i+1}
-      {
-        ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
-        const GemmParams p = mlp2_rowln_params(batch, h->dims[m - 1], n, d, c.n_f, h->b[l][m - 1], xin, h->g2[l],
-                                               h->b2[l], h->eps, h->status);
-        GemmMaps mp = h->last_maps[l];
-        if (last) {
-          mp.C = out_last;
-          s = run_gemm_tc2<T, OUT, true>(dv, mp, p, st);
-        } else {
-          s = run_gemm_tc2<T, T, true>(dv, mp, p, st);
-        }
-      }
-      if (s != WK_OK) break;
-      {
-        ProfScope ps(h, WK_KERNEL_LCB, st);
-        GemmParams p = lcb_params(batch, n, d, c.n_l, h->status);
-        p.resid = xin;
-        p.ln_g = h->g2[l];
-        p.ln_b = h->b2[l];
-        p.ln_eps = h->eps;
-        p.ln_n = n;
-        p.ln_row0 = c.n_f;
-        GemmMaps mp;
-        mp.A = h->lcbA[l];
-        mp.B = (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2];
-        if (last) {
-          mp.C = out_lcb;
-          s = run_gemm_tc<MODE_LCB, T, OUT, true>(dv, mp, p, st);
-        } else {
-          mp.C = h->lcbC_x[l % 2];
-          s = run_gemm_tc<MODE_LCB, T, T, true>(dv, mp, p, st);
-        }
-      }
-      continue;
-    }
+    s = layer_front16<T>(h, l, xin, (l == 0) ? lcb_x0 : h->lcbB_ws[(l - 1) % 2], batch, st);
+    if (s != WK_OK) break;
     {  // 4. residual + LN
       ProfScope ps(h, WK_KERNEL_RES_LN, st);
       const T* cat = static_cast<const T*>(h->cat);
@@ -1385,13 +1302,8 @@ wk_status bw_gemm_mn(wk_stack* h, const void* A, int64_t lda, const void* W, int
   ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
   // The weight gradient (K = the batch, fp32 tiles) runs persistent: its two TMEM accumulators
   // overlap a tile's epilogue with the next tile's main loop, which a short K leaves exposed in
-  // the streaming shape's one accumulator. WK_WGRAD_STREAM=1 in the environment streams it.
-  static const int wgrad_stream = [] {
-    const char* e = getenv("WK_WGRAD_STREAM");
-    return (e && e[0] == '1') ? 1 : 0;
-  }();
-  return run_gemm_tc2<T, TO, false, A_MN, B_MN>(dv, mp, mlp2_params(M, K, N, nullptr, 0, h->status), st,
-                                                (A_MN && B_MN) ? wgrad_stream : -1);
+  // the streaming shape's one accumulator.
+  return run_gemm_tc2<T, TO, A_MN, B_MN>(dv, mp, mlp2_params(M, K, N, nullptr, 0, h->status), st, !(A_MN && B_MN));
 }
 
 template <typename T>
@@ -1709,6 +1621,7 @@ wk_status read_status_word(unsigned* word, cudaStream_t st) {
     cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice);
   }
   if (v & kFlagTimeout) return WK_ERR_TIMEOUT;
+  if (v & kFlagNonFinite) return WK_ERR_NONFINITE;
   if (v) return WK_ERR_DEVICE;
   return WK_OK;
 }
@@ -1878,6 +1791,7 @@ const char* wk_status_string(wk_status s) {
     case WK_ERR_CUDA: return "CUDA runtime error";
     case WK_ERR_TIMEOUT: return "a kernel gave up waiting (device pipeline timeout)";
     case WK_ERR_DEVICE: return "device-side error flag";
+    case WK_ERR_NONFINITE: return "non-finite value (a 16-bit intermediate overflowed, or inf / NaN in the input)";
   }
   return "unknown status";
 }
@@ -2194,7 +2108,7 @@ wk_status wk_stack_backward_events(wk_stack* h, const void* X, const float* dOut
   // the fp16-operand path (first Linear folded), at most three Linears (both hidden
   // activations stay in the workspace), a batch that is a multiple of 8 (the weight
   // gradients' GEMMs contract over it), embedding rows of at most 256
-  if (h->op != WK_F16 || h->front_only || h->fused || c.mlp_num_linear > 3 || batch % 8 != 0 || c.d > 256 ||
+  if (h->op != WK_F16 || h->front_only || c.mlp_num_linear > 3 || batch % 8 != 0 || c.d > 256 ||
       c.d % 32 != 0)
     return WK_ERR_UNSUPPORTED;
   int dev = -1;
@@ -2343,12 +2257,22 @@ wk_status wk_layer_forward_noalloc(const wk_stack_config* cfg, const wk_layer_we
   if (!X || !out || !al16(X) || !al16(out) || !w->Y || !w->W || !w->W_L || !w->fmb_ln_gamma || !w->fmb_ln_beta ||
       !w->out_ln_gamma || !w->out_ln_beta)
     return WK_ERR_INVALID_ARG;
+  // the same alignment rules as wk_stack_create: the kernels read every weight, bias and
+  // LayerNorm vector with 16-byte loads or TMA
+  if (!al16(w->Y) || !al16(w->W_L) || !al16(w->fmb_ln_gamma) || !al16(w->fmb_ln_beta) || !al16(w->out_ln_gamma) ||
+      !al16(w->out_ln_beta))
+    return WK_ERR_INVALID_ARG;
   std::vector<int32_t> dims;
   dims.push_back(cfg->n * cfg->k);
   for (int j = 0; j + 1 < cfg->mlp_num_linear; ++j) dims.push_back(cfg->mlp_hidden[j]);
   dims.push_back(cfg->n_f * cfg->d);
-  for (int j = 0; j < cfg->mlp_num_linear; ++j)
-    if (!w->W[j]) return WK_ERR_INVALID_ARG;
+  for (int j = 0; j < cfg->mlp_num_linear; ++j) {
+    if (!w->W[j] || !al16(w->W[j])) return WK_ERR_INVALID_ARG;
+    if (w->b && w->b[j] && !al16(w->b[j])) return WK_ERR_INVALID_ARG;
+  }
+  // No product below can wrap: the largest per-example region (n*max(k, d, hidden) values
+  // of at most 4 bytes, under 2^33 for int32 dims) times a batch below the scratch size.
+  if (batch > static_cast<int64_t>(WK_NOALLOC_SCRATCH_BYTES)) return WK_ERR_INVALID_ARG;
   if (noalloc_bytes(cfg, dims, batch) > WK_NOALLOC_SCRATCH_BYTES) return WK_ERR_INVALID_ARG;
   const size_t bytes = static_cast<size_t>(batch) * cfg->n * cfg->d * (cfg->dtype == WK_F32 ? 4 : 2);
   const uint8_t* xa = static_cast<const uint8_t*>(X);

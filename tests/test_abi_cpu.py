@@ -36,8 +36,8 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for s in range(7):
-        assert len(wk.wk_status_string(s)) >= 2
+    for s in range(8):
+        assert len(wk.wk_status_string(s)) >= 2 and wk.wk_status_string(s) != "unknown status"
     assert wk.wk_status_string(99) == "unknown status"
 
 
@@ -162,3 +162,25 @@ def test_whale_argument_errors_without_a_device(L):
                                  None) == wk.WK_ERR_UNSUPPORTED
     assert L.wk_whale_fusion_ffn(FAKE, FAKE, ctypes.byref(w), FAKE, 0, 128, 512, wk.WK_BF16, ctypes.c_float(0),
                                  None) == wk.WK_OK
+
+
+def _noalloc_status(L, layer, batch):
+    c, hid, m = wk._config(_cfg(dtype="bf16"), 1, None, 0.0, None)
+    keep = [hid]
+    arr = wk._layer_array([layer], m, keep)
+    return L.wk_layer_forward_noalloc(ctypes.byref(c), arr, FAKE, FAKE * 4, batch, None)
+
+
+@pytest.mark.parametrize("key", ["Y", "W0", "b0", "W1", "W_L", "fmb_gamma", "fmb_beta", "out_gamma", "out_beta"])
+def test_noalloc_rejects_misaligned_weights_before_any_launch(L, key):
+    """wk_layer_forward_noalloc checks every weight, bias and LayerNorm pointer for the
+    16-byte alignment its kernels' vector loads and TMA need, on the host, before it looks
+    up a device: on a machine without a GPU the answer is still the argument error."""
+    layer = dict(_fake_layers(2)[0])
+    layer[key] = FAKE + 4
+    assert _noalloc_status(L, layer, 8) == wk.WK_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_batches_that_would_overflow_the_size_arithmetic(L):
+    for batch in (1 << 40, (1 << 62) + 1):
+        assert _noalloc_status(L, _fake_layers(2)[0], batch) == wk.WK_ERR_INVALID_ARG

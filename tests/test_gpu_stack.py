@@ -135,9 +135,10 @@ def test_profiling_counts_launches():
         st.run(X)
         t = wk.wk_stack_kernel_times(st.h)
         m = len(cfg["hidden"]) + 1
-        assert t["fm_ln"][1] == cfg["layers"] and t["mlp_gemm"][1] == cfg["layers"] * m
-        # the residual + LayerNorm runs in its own kernel, or inside the last Linear and LCB epilogues
-        assert t["lcb"][1] == cfg["layers"] and t["res_ln"][1] in (0, cfg["layers"])
+        # per layer one front kernel (input LayerNorm, FM + LayerNorm, LCB, residual) and the
+        # MLP Linears; one output LayerNorm for the stack
+        assert t["front"][1] == cfg["layers"] and t["mlp_gemm"][1] == cfg["layers"] * m
+        assert t["res_ln"][1] == 1 and t["fm_ln"][1] == 0 and t["lcb"][1] == 0 and t["convert"][1] == 0
         assert all(ms > 0 for ms, count in t.values() if count)
     finally:
         st.close()
@@ -145,3 +146,59 @@ def test_profiling_counts_launches():
 
 def test_parity_c4_bf16_full_size():
     _parity("c4_bf16", 16)
+
+
+@pytest.mark.parametrize("name,batch", [("c2_bf16", 100), ("c2_bf16", 7), ("c3_bf16", 149), ("c5_bf16", 37),
+                                        ("c4_bf16", 3)])
+def test_parity_small_and_ragged_batches(name, batch):
+    """Batches below one CTA per SM, not a multiple of the grid, and at most one 128-row MLP
+    tile (the one-CTA GEMM with its reduce-add epilogue): every example against the oracle."""
+    cfg = C.CONFIGS[name]
+    st = DevStack(name, max_batch=batch)
+    try:
+        X = C.make_x_dev(cfg, batch)
+        out = st.run(X)
+        ex = list(range(batch)) if batch <= 16 else _sample(batch, 16)
+        got = f64(out[ex])
+        assert np.isfinite(got).all()
+        err = max_scaled_err(got, _oracle(cfg, ex))
+        print("%s batch %d: max |gpu-ref|/(1+|ref|) = %.3g" % (name, batch, err))
+        assert err <= TOL[cfg["dtype"]]
+    finally:
+        st.close()
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("what", ["input", "hidden"])
+def test_fp16_overflow_is_reported(what):
+    """The default 16-bit path keeps its intermediates in fp16 (range |v| <= 65504), where the
+    pages' bf16 has the range of fp32. A value past that range must come back as
+    WK_ERR_NONFINITE from the status call, not as silent inf / NaN in the output: an input
+    scaled by 1e5 (representable in the caller's bf16, not in fp16), or a first Linear scaled
+    by 1e5 (its hidden activations overflow). A normal forward afterwards reports WK_OK."""
+    cfg = dict(C.CONFIGS["c2_bf16"], layers=1)
+    layer = C.make_layer_dev(cfg, 0)
+    X = C.make_x_dev(cfg, 64)
+    if what == "input":
+        Xb = (X.float() * 1e5).to(X.dtype)
+        assert torch.isfinite(Xb).all()
+        layers = [layer]
+    else:
+        Xb = X
+        layers = [dict(layer, W0=(layer["W0"].float() * 1e5).to(layer["W0"].dtype))]
+    h = wk.wk_stack_create(cfg, layers, max_batch=64)
+    try:
+        out = torch.empty_like(X)
+        wk.wk_stack_forward(h, Xb, out)
+        assert wk.wk_stack_sync_status(h) == wk.WK_ERR_NONFINITE
+        assert "non-finite" in wk.wk_status_string(wk.WK_ERR_NONFINITE)
+    finally:
+        wk.wk_stack_destroy(h)
+    h = wk.wk_stack_create(cfg, [layer], max_batch=64)
+    try:
+        out = torch.empty_like(X)
+        wk.wk_stack_forward(h, X, out)
+        assert wk.wk_stack_sync_status(h) == wk.WK_OK
+        assert torch.isfinite(out.float()).all()
+    finally:
+        wk.wk_stack_destroy(h)
