@@ -41,14 +41,15 @@ BACKWARD_METRIC = ("examples/sec and achieved TFLOP/s (% of bf16 peak), Wukong s
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM traffic of the CTA-pair MLP GEMM per launch (streaming launch shape), from one ncu
-# capture of each of the three Linears of the workload (dram__bytes_read.sum +
-# dram__bytes_write.sum, averaged over the three launches). It describes the kernel sources it
-# was taken on: when their hash differs, the bench reports null.
+# DRAM traffic of the CTA-pair MLP GEMM per launch, from one ncu capture of the three Linears
+# of the first layer inside the bench's own step (dram__bytes_read.sum + dram__bytes_write.sum,
+# averaged over the three launches; the last Linear reduce-adds into the layer output, so its
+# output is read as well as written). It describes the kernel sources it was taken on: when
+# their hash differs, the bench reports null.
 GEMM_TRAFFIC = {
     "sources": ["recsys_feature_interaction_b200/csrc/gemm_tc2.cuh", "recsys_feature_interaction_b200/csrc/common.cuh"],
-    "sha256": "1e7902e5ecfd65ca1140976e864c705496a8ae5e69df45f56b752cf70b0f7a36",
-    "bytes_per_launch": 3183891712,
+    "sha256": "c5d76cd63c37947785bb77b92b43359c5a3e9b9f076ba31087abab135dce9d9b",
+    "bytes_per_launch": 3338665301,
 }
 
 
