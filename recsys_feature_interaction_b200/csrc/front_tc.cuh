@@ -565,65 +565,60 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         }
         named_bar(1, 128);  // every epilogue warp is past its reads of red[]
       } else {
-        // three passes over F in TMEM: mean, variance, output
+        // two passes over F in TMEM: statistics, output. The statistics in one pass: each
+        // thread sums (x - s) and (x - s)^2 around its first value s (no cancellation for
+        // data far from 0); the mean is reduced first, then each thread's share of the sum of
+        // squared deviations follows from its sums exactly, sum (x - mean)^2 =
+        // Q - 2 (mean - s) S + n (mean - s)^2, and is reduced second.
         if (ok) ok = mbar_wait(ffull, par, status);
         tc_fence_after();
-        float part = 0.f;
+        float sh = 0.f, sx = 0.f, sq = 0.f, cnt = 0.f;
 #pragma unroll 1
         for (int c = 0; c < C::NCH; ++c) {
           const int row = c * C::R + q * 32 + lane;
+          uint32_t r[C::KP / 32][32];
 #pragma unroll
-          for (int h = 0; h < C::KP / 32; ++h) {
-            uint32_t r[32];
-            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r);
-            tmem_ld_wait();
-            if (row < C::N) {
+          for (int h = 0; h < C::KP / 32; ++h)
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r[h]);
+          tmem_ld_wait();
+          if (c == 0) sh = __uint_as_float(r[0][0]);
+          if (row < C::N) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (h * 32 + j < C::K) part += __uint_as_float(r[j]);
-            }
-          }
-        }
-        part = warp_sum(part);
-        if (lane == 0) red[ew] = part;
-        named_bar(1, 128);
-        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
-        float qs = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < C::NCH; ++c) {
-          const int row = c * C::R + q * 32 + lane;
-#pragma unroll
-          for (int h = 0; h < C::KP / 32; ++h) {
-            uint32_t r[32];
-            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r);
-            tmem_ld_wait();
-            if (row < C::N) {
+            for (int h = 0; h < C::KP / 32; ++h)
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (h * 32 + j < C::K) {
-                  const float dv = __uint_as_float(r[j]) - mean;
-                  qs = fmaf(dv, dv, qs);
+                  const float dv = __uint_as_float(r[h][j]) - sh;
+                  sx += dv;
+                  sq = fmaf(dv, dv, sq);
                 }
-            }
+            cnt += static_cast<float>(C::K);
           }
         }
-        qs = warp_sum(qs);
+        float part = warp_sum(sx + cnt * sh);
+        if (lane == 0) red[ew] = part;
+        named_bar(1, 128);
+        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+        const float dm = mean - sh;
+        float qs = warp_sum(sq - 2.f * dm * sx + cnt * dm * dm);
         if (lane == 0) red[4 + ew] = qs;
         named_bar(1, 128);
-        const float var = (red[4] + red[5] + red[6] + red[7]) * inv_cnt;
+        const float var = fmaxf((red[4] + red[5] + red[6] + red[7]) * inv_cnt, 0.f);
         const float rstd = rsqrtf(var + eps);
         if (threadIdx.x == 32 * FRONT_EPI_WARP0 && !(isfinite(mean) && isfinite(var))) flag_error(status, kFlagNonFinite);
 #pragma unroll 1
         for (int c = 0; c < C::NCH; ++c) {
           const int row = c * C::R + q * 32 + lane;
+          uint32_t rr[C::KP / 32][32];
+#pragma unroll
+          for (int h = 0; h < C::KP / 32; ++h)
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), rr[h]);
+          tmem_ld_wait();
 #pragma unroll
           for (int h = 0; h < C::KP / 32; ++h) {
-            uint32_t r[32];
-            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r);
-            tmem_ld_wait();
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = (__uint_as_float(r[e]) - mean) * rstd;
+            for (int e = 0; e < 32; ++e) v[e] = (__uint_as_float(rr[h][e]) - mean) * rstd;
             if (affine && row < C::N) {
               const float* gp = fg + row * C::K + h * 32;
               const float* bp = fb + row * C::K + h * 32;

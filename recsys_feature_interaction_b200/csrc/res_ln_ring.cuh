@@ -44,8 +44,9 @@ struct ResLnRing {
   static_assert(TILE_B % 16 == 0, "bulk copy granularity");
 };
 
-// TC, TR: 16-bit concat and residual types; TO: output type.
-template <int D, typename TC, typename TR, typename TO>
+// TC, TR: 16-bit concat and residual types; TO: output type; RESID = false: x is not read
+// (the output LayerNorm alone).
+template <int D, typename TC, typename TR, typename TO, bool RESID = true>
 __global__ void __launch_bounds__(ResLnRing<D>::THREADS, 1)
     res_ln_ring_kernel(const TC* __restrict__ cat, const TR* __restrict__ x, const float* __restrict__ gamma,
                        const float* __restrict__ beta, TO* __restrict__ out, int64_t rows, float eps,
@@ -81,9 +82,9 @@ __global__ void __launch_bounds__(ResLnRing<D>::THREADS, 1)
         const int64_t nr = rows - r0 < C::R ? rows - r0 : C::R;
         const uint32_t bytes = static_cast<uint32_t>(nr) * C::ROW_B;
         uint8_t* dst = smem + slot * 2 * C::TILE_B;
-        mbar_arrive_expect_tx(&full[slot], (x ? 2u : 1u) * bytes);
+        mbar_arrive_expect_tx(&full[slot], (RESID ? 2u : 1u) * bytes);
         bulk_load(dst, cat + r0 * D, bytes, &full[slot]);
-        if (x) bulk_load(dst + C::TILE_B, x + r0 * D, bytes, &full[slot]);
+        if constexpr (RESID) bulk_load(dst + C::TILE_B, x + r0 * D, bytes, &full[slot]);
         if (++slot == C::STAGES) {
           slot = 0;
           phase ^= 1u;
@@ -129,11 +130,17 @@ __global__ void __launch_bounds__(ResLnRing<D>::THREADS, 1)
 #pragma unroll
       for (int k = 0; k < C::VPL; ++k) {
         const int off = lr * C::ROW_B + (v0 + k * C::G) * 16;
-        float c8[8], x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float c8[8];
         Vec8<TC>::load_shared(tc + off, c8);
-        if (x) Vec8<TR>::load_shared(tx + off, x8);
+        if constexpr (RESID) {
+          float x8[8];
+          Vec8<TR>::load_shared(tx + off, x8);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) y[k][j] = ok ? c8[j] + x8[j] : 0.f;
+          for (int j = 0; j < 8; ++j) y[k][j] = ok ? c8[j] + x8[j] : 0.f;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) y[k][j] = ok ? c8[j] : 0.f;
+        }
       }
       float s = 0.f;
 #pragma unroll

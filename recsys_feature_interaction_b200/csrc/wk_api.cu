@@ -452,14 +452,21 @@ wk_status run_res_ln_d(const DevInfo* dv, const TC* cat, const TR* x, const floa
   if constexpr (sizeof(TC) == 2 && sizeof(TR) == 2) {
     if (al16(cat) && al16(x)) {
       using C = ResLnRing<D>;
-      wk_status s = smem_attr(dv, reinterpret_cast<const void*>(res_ln_ring_kernel<D, TC, TR, TO>), C::SMEM);
-      if (s != WK_OK) return s;
       const int64_t tiles = (rows + C::R - 1) / C::R;
       const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, dv->sms)));
+      if (x == nullptr) {
+        wk_status s = smem_attr(dv, reinterpret_cast<const void*>(res_ln_ring_kernel<D, TC, TR, TO, false>), C::SMEM);
+        if (s != WK_OK) return s;
+        res_ln_ring_kernel<D, TC, TR, TO, false><<<grid, C::THREADS, C::SMEM, st>>>(cat, x, g, b, out, rows, eps, status);
+        return launch_status();
+      }
+      wk_status s = smem_attr(dv, reinterpret_cast<const void*>(res_ln_ring_kernel<D, TC, TR, TO>), C::SMEM);
+      if (s != WK_OK) return s;
       res_ln_ring_kernel<D, TC, TR, TO><<<grid, C::THREADS, C::SMEM, st>>>(cat, x, g, b, out, rows, eps, status);
       return launch_status();
     }
   }
+  if (x == nullptr) return WK_ERR_UNSUPPORTED;  // the output LayerNorm alone runs on the ring only
   constexpr int VPR = D / 8;
   constexpr int G = res_ln_lanes(VPR);
   constexpr int rows_per_block = (256 / 32) * (32 / G) * ((VPR / G) >= 4 ? 2 : 4);
