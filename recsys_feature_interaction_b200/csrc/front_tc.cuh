@@ -61,7 +61,11 @@ struct FrontCfg {
   static constexpr int LCOL = MTZ * KP;                      // first TMEM column of the LCB / F
   static constexpr int LCOLS = MTL * D;
   static constexpr int FCOLS = NCH * KP;
-  static constexpr int UCOLS = LCOLS > FCOLS ? LCOLS : FCOLS;
+  // F in its own TMEM columns after the LCB's when they fit (pass B then need not wait for
+  // the LCB rows to be read out), else F reuses the LCB's columns
+  static constexpr bool SEPF = LCOL + LCOLS + FCOLS <= 512;
+  static constexpr int FCOL = SEPF ? LCOL + LCOLS : LCOL;
+  static constexpr int UCOLS = SEPF ? LCOLS + FCOLS : (LCOLS > FCOLS ? LCOLS : FCOLS);
   static constexpr int TCOLS = LCOL + UCOLS;
   static constexpr int TMEM_COLS = TCOLS <= 32 ? 32 : TCOLS <= 64 ? 64 : TCOLS <= 128 ? 128 : TCOLS <= 256 ? 256 : 512;
   static constexpr int ZB = ((D + 15) / 16) * 16 * YRB;      // Z operand
@@ -69,7 +73,11 @@ struct FrontCfg {
   static constexpr int STG = WB > YB ? WB : YB;              // ring stage
   static constexpr int EPI = 4 * 2048;                       // a 32 x 32 16-bit staging tile per epilogue warp
   static constexpr int TAIL = 2 * D * 4 + 1024;              // input LN affine, partial sums, barriers
-  static constexpr int FIXED = 1024 + NCH * CHB + ZB + EPI + TAIL;
+  // examples in flight: two sets of chunk slots (the next example loads while this one
+  // computes) where shared memory keeps a 2-stage ring beside them and TMEM holds F apart
+  static constexpr int ES = (SEPF && 1024 + 2 * NCH * CHB + ZB + EPI + TAIL + 2 * (WB > YB ? WB : YB) <=
+                             FRONT_SMEM_LIMIT) ? 2 : 1;
+  static constexpr int FIXED = 1024 + ES * NCH * CHB + ZB + EPI + TAIL;
   static constexpr int NSTG_RAW = (FRONT_SMEM_LIMIT - FIXED) / STG;
   static constexpr int NSTG = NSTG_RAW > 4 ? 4 : NSTG_RAW;
   // pass A's last Z tile reads 4 * MTZ boxes from a chunk's base: past the last chunk that
@@ -158,18 +166,18 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
                     T* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* slots = smem;                                     // [NCH] chunks of the layer input
-  uint8_t* zb = slots + C::NCH * C::CHB;                     // Z operand
+  uint8_t* slots = smem;                                     // [ES][NCH] chunks of the layer inputs
+  uint8_t* zb = slots + C::ES * C::NCH * C::CHB;             // Z operand
   uint8_t* ring = zb + C::ZB;                                // [NSTG] Y / W_L stages
   uint8_t* epi = ring + C::NSTG * C::STG;                    // [4] staging tiles
   float* sg = reinterpret_cast<float*>(epi + C::EPI + C::PAD);
   float* sb = sg + C::D;
   float* red = sb + C::D;                                    // [8] FMB LayerNorm partial sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(red + 8);
-  uint64_t* full = bars;                                     // [NCH] chunk landed
-  uint64_t* xready = full + C::NCH;                          // [NCH] chunk normalised
-  uint64_t* empty = xready + C::NCH;                         // [NCH] chunk slot free (2 arrivals)
-  uint64_t* wfull = empty + C::NCH;                          // [NSTG]
+  uint64_t* full = bars;                                     // [ES * NCH] chunk landed
+  uint64_t* xready = full + C::ES * C::NCH;                  // [ES * NCH] chunk normalised
+  uint64_t* empty = xready + C::ES * C::NCH;                 // [ES * NCH] chunk slot free (6 arrivals)
+  uint64_t* wfull = empty + C::ES * C::NCH;                  // [NSTG]
   uint64_t* wempty = wfull + C::NSTG;                        // [NSTG]
   uint64_t* zfull = wempty + C::NSTG;                        // MMA -> epilogue: Z in TMEM
   uint64_t* ffull = zfull + 1;                               // MMA -> epilogue: F in TMEM
@@ -189,10 +197,13 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
     prefetch_tmap(&tmR);
     prefetch_tmap(&tmL);
     prefetch_tmap(&tmA);
-    for (int c = 0; c < C::NCH; ++c) {
+    // a slot is free once pass B has read it (the MMA's commit), its residual stores have
+    // read it (the normalising warps) and the LCB rows' residual has been read from it (one
+    // arrival per epilogue warp)
+    for (int c = 0; c < C::ES * C::NCH; ++c) {
       mbar_init(&full[c], 1);
       mbar_init(&xready[c], 1);
-      mbar_init(&empty[c], 2);
+      mbar_init(&empty[c], 6);
     }
     for (int s = 0; s < C::NSTG; ++s) {
       mbar_init(&wfull[s], 1);
@@ -229,23 +240,25 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       int64_t i = 0;
       bool ok = true;
       for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x, ++i) {
-        const uint32_t par = static_cast<uint32_t>(i & 1);
-        for (int c = 0; c < C::NCH; ++c) {
-          if (!mbar_wait(&empty[c], par ^ 1u, status)) {
+        const int es = static_cast<int>(i % C::ES);                // slot set and its phase
+        const uint32_t sp = static_cast<uint32_t>((i / C::ES) & 1);
+        for (int cc = 0; cc < C::NCH; ++cc) {
+          const int c = es * C::NCH + cc;
+          if (!mbar_wait(&empty[c], sp ^ 1u, status)) {
             ok = false;
             break;
           }
           // the chunk's rows are one contiguous range of the input: one bulk copy
-          const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
+          const int rows = (C::N - cc * C::R) < C::R ? (C::N - cc * C::R) : C::R;
           const uint32_t bytes = static_cast<uint32_t>(rows * C::D * 2);
           mbar_arrive_expect_tx(&full[c], bytes);
-          bulk_load(slots + c * C::CHB, xin + (b * C::N + c * C::R) * C::D, bytes, &full[c]);
+          bulk_load(slots + c * C::CHB, xin + (b * C::N + cc * C::R) * C::D, bytes, &full[c]);
           issued |= 1u << c;
-          lastpar = (lastpar & ~(1u << c)) | (par << c);
+          lastpar = (lastpar & ~(1u << c)) | (sp << c);
         }
       }
       // every copy issued lands before the CTA's shared memory is released
-      for (int c = 0; c < C::NCH; ++c)
+      for (int c = 0; c < C::ES * C::NCH; ++c)
         if (issued & (1u << c)) mbar_drain(&full[c], (lastpar >> c) & 1u, status);
     }
   } else if (warp == 2) {
@@ -305,6 +318,8 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       bool issued = false;
       for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x, ++i) {
         const uint32_t par = static_cast<uint32_t>(i & 1);
+        const int es = static_cast<int>(i % C::ES);
+        const uint32_t sp = static_cast<uint32_t>((i / C::ES) & 1);
         // Chunk by chunk as they are normalised: pass A, Z += X_c^T Y_c (the previous example's Z
         // has been turned into its pass-B operand first), and the LCB, D_m += W_L[m, c] X_c for
         // every tile m (once the previous example's F, which shares D's TMEM columns, is read),
@@ -314,14 +329,14 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           break;
         }
         for (int c = 0; ok && c < C::NCH; ++c) {
-          if (!mbar_wait(&xready[c], par, status) || !mbar_wait(&wfull[s], ph, status)) {
+          if (!mbar_wait(&xready[es * C::NCH + c], sp, status) || !mbar_wait(&wfull[s], ph, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
           const int nkb = (rows + 63) / 64;
-          const uint32_t xs = slot0 + c * C::CHB;
+          const uint32_t xs = slot0 + (es * C::NCH + c) * C::CHB;
           const uint32_t ys = smem_u32(ring + s * C::STG);
           for (int ks = 0; ks < rows / 16; ++ks) {
             const uint64_t bdesc = smem_desc(ys + ks * 16 * C::YRB, C::YB, 8 * C::YRB, ysw);
@@ -339,7 +354,9 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
             ph ^= 1u;
           }
           if (c == C::NCH - 1) umma_commit(zfull);
-          if (c == 0 && i > 0 && !mbar_wait(fempty, par ^ 1u, status)) {
+          // the LCB's TMEM columns are free once the previous example's LCB rows (and, when F
+          // shares them, its F) have been read
+          if (c == 0 && i > 0 && !mbar_wait(C::SEPF ? ldone : fempty, par ^ 1u, status)) {
             ok = false;
             break;
           }
@@ -367,22 +384,24 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         }
         if (!ok) break;
         for (int m = 0; m < C::MTL; ++m) umma_commit(&lfull[m]);
-        // pass B: F = X Z into the LCB's columns, once Z is in shared memory and the LCB
-        // accumulators have been read
-        if (!mbar_wait(zready, par, status) || !mbar_wait(ldone, par, status)) {
+        // pass B: F = X Z, once Z is in shared memory and F's TMEM columns are free: the
+        // previous example's F has been read (F apart) or this example's LCB rows have been
+        // read (F in the LCB's columns)
+        if (!mbar_wait(zready, par, status) ||
+            !(C::SEPF ? (i == 0 || mbar_wait(fempty, par ^ 1u, status)) : mbar_wait(ldone, par, status))) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int c = 0; c < C::NCH; ++c) {
-          const uint32_t xs = slot0 + c * C::CHB;
+          const uint32_t xs = slot0 + (es * C::NCH + c) * C::CHB;
 #pragma unroll
           for (int ks = 0; ks < C::D / 16; ++ks) {
             const uint64_t adesc = smem_desc(xs + (ks >> 1) * C::XBOXB + (ks & 1) * 32, 16, 512, 4);
             const uint64_t bdesc = smem_desc(smem_u32(zb) + ks * 16 * C::YRB, C::ZB, 8 * C::YRB, ysw);
-            umma_f16kind(tmem_base + C::LCOL + c * C::KP, adesc, bdesc, idB, ks != 0 ? 1u : 0u);
+            umma_f16kind(tmem_base + C::FCOL + c * C::KP, adesc, bdesc, idB, ks != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[c]);  // the chunk's slot is free once pass B has read it
+          umma_commit(&empty[es * C::NCH + c]);  // pass B has read the chunk's slot
         }
         umma_commit(ffull);
       }
@@ -403,6 +422,8 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
     bool ok = true;
     for (int64_t b = blockIdx.x; b < batch; b += gridDim.x, ++i) {
       const uint32_t par = static_cast<uint32_t>(i & 1);
+      const int es = static_cast<int>(i % C::ES);
+      const uint32_t sp = static_cast<uint32_t>((i / C::ES) & 1);
       // Z (TMEM, fp32) -> 16-bit MN-major operand in shared memory (once the previous
       // example's A0 stores staged there have read it)
       if (C::A0_TMA && lane == 0) bulk_wait_read<0>();
@@ -440,7 +461,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       // LCB rows: accumulator + the residual X row (from the chunk in shared memory), staged
       // 32 columns at a time and stored by TMA (rows past n_l are clipped), through this warp's
       // own staging tile and its quarter of the Y / W_L ring, idle until the drain is done
-      for (int c = C::NF / C::R; ok && c < C::NCH; ++c) ok = mbar_wait(&xready[c], par, status);
+      for (int c = C::NF / C::R; ok && c < C::NCH; ++c) ok = mbar_wait(&xready[es * C::NCH + c], sp, status);
 #pragma unroll 1
       for (int m = 0; m < C::MTL; ++m) {
         if (ok) ok = mbar_wait(&lfull[m], par, status);
@@ -449,7 +470,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         const bool valid = r < C::NL;
         const bool any = m * C::R + q * 32 < C::NL;
         const int rho = C::NF + r;                // its residual row
-        const uint8_t* xres = slots + (rho / C::R) * C::CHB;
+        const uint8_t* xres = slots + (es * C::NCH + rho / C::R) * C::CHB;
         const int rl = rho % C::R;
 #pragma unroll 1
         for (int j = 0; j < C::XBOXES; ++j) {
@@ -485,7 +506,10 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       tc_fence_before();
       if (lane == 0) bulk_wait_read<0>();  // the ring is the producer's again
       __syncwarp();
-      if (lane == 0) mbar_arrive(ldone);
+      if (lane == 0) {
+        mbar_arrive(ldone);
+        for (int c = 0; c < C::NCH; ++c) mbar_arrive(&empty[es * C::NCH + c]);  // residual rows read
+      }
 
       // the FMB LayerNorm over the n*k values of F
       T* ab = A0 + b * (C::N * C::K);
@@ -498,7 +522,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         uint32_t fr[C::NCH][C::K];
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          const uint32_t ta = tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP);
+          const uint32_t ta = tmem_base + lane_base + static_cast<uint32_t>(C::FCOL + c * C::KP);
           if constexpr (C::K == 32) {
             tmem_ld32(ta, reinterpret_cast<uint32_t(&)[32]>(fr[c][0]));
           } else if constexpr (C::K == 24) {
@@ -579,7 +603,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           uint32_t r[C::KP / 32][32];
 #pragma unroll
           for (int h = 0; h < C::KP / 32; ++h)
-            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), r[h]);
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::FCOL + c * C::KP + h * 32), r[h]);
           tmem_ld_wait();
           if (c == 0) sh = __uint_as_float(r[0][0]);
           if (row < C::N) {
@@ -612,7 +636,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           uint32_t rr[C::KP / 32][32];
 #pragma unroll
           for (int h = 0; h < C::KP / 32; ++h)
-            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + c * C::KP + h * 32), rr[h]);
+            tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::FCOL + c * C::KP + h * 32), rr[h]);
           tmem_ld_wait();
 #pragma unroll
           for (int h = 0; h < C::KP / 32; ++h) {
@@ -668,11 +692,13 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
     int64_t i = 0;
     bool ok = true;
     for (int64_t b = blockIdx.x; b < batch; b += gridDim.x, ++i) {
-      const uint32_t par = static_cast<uint32_t>(i & 1);
+      const int es = static_cast<int>(i % C::ES);
+      const uint32_t sp = static_cast<uint32_t>((i / C::ES) & 1);
       for (int c = 0; c < C::NCH; ++c) {
-        if (ok) ok = mbar_wait(&full[c], par, status);
+        const int sc = es * C::NCH + c;
+        if (ok) ok = mbar_wait(&full[sc], sp, status);
         const int rows = (C::N - c * C::R) < C::R ? (C::N - c * C::R) : C::R;
-        uint8_t* base = slots + c * C::CHB;
+        uint8_t* base = slots + sc * C::CHB;
         const bool act = ok && row < rows;
         // the row as loaded (row-major, d values), into registers; every thread reads before
         // any thread writes the operand layout over the same bytes
@@ -684,28 +710,29 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         }
         named_bar(2, FRONT_NORM_THREADS);
         if (ln_in) {
-          float s = 0.f;
-#pragma unroll
-          for (int k = 0; k < UPT; ++k) {
-            float v[8];
-            front_unpack8<TIN>(w[k], v);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) s += v[e];
-          }
-          s += __shfl_xor_sync(0xffffffffu, s, 1);
-          const float mean = s * (1.0f / C::D);
-          float qv = 0.f;
+          // one pass over the row for its statistics: sums of (x - s) and (x - s)^2 around the
+          // row's first value s (both threads of the row use it), no cancellation for rows far
+          // from 0
+          float v0[8];
+          front_unpack8<TIN>(w[0], v0);
+          const float sh = __shfl_sync(0xffffffffu, v0[0], lane & ~1);
+          float sx = 0.f, sq = 0.f;
 #pragma unroll
           for (int k = 0; k < UPT; ++k) {
             float v[8];
             front_unpack8<TIN>(w[k], v);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float dv = v[e] - mean;
-              qv = fmaf(dv, dv, qv);
+              const float dv = v[e] - sh;
+              sx += dv;
+              sq = fmaf(dv, dv, sq);
             }
           }
-          qv += __shfl_xor_sync(0xffffffffu, qv, 1);
+          sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+          sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+          const float dmean = sx * (1.0f / C::D);
+          const float mean = sh + dmean;
+          const float qv = fmaxf(sq - sx * dmean, 0.f);  // sum of (x - mean)^2
           const float rstd = rsqrtf(qv * (1.0f / C::D) + eps);
           if (act && half == 0 && !(isfinite(mean) && isfinite(qv))) flag_error(status, kFlagNonFinite);
           if (act) {
@@ -739,7 +766,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         fence_proxy_async_smem();  // the tensor core and the TMA store read the chunk
         named_bar(2, FRONT_NORM_THREADS);
         if (tid == 0) {
-          mbar_arrive(&xready[c]);
+          mbar_arrive(&xready[sc]);
           // The FMB rows' residual (rows past n_f are clipped). The slot is released (one of
           // its two arrivals) once its stores have read it: the previous chunk's is released
           // here, after this chunk's stores are issued, so no chunk waits for its own.
@@ -755,7 +782,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
             else bulk_wait_read<0>();
             mbar_arrive(&empty[pending]);
           }
-          pending = c;
+          pending = sc;
         }
       }
       if (tid == 0 && pending >= 0) {
