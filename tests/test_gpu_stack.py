@@ -202,3 +202,37 @@ def test_fp16_overflow_is_reported(what):
         assert torch.isfinite(out.float()).all()
     finally:
         wk.wk_stack_destroy(h)
+
+
+def test_parity_fp16_caller_stack():
+    """A caller whose tensors are fp16 (the operand type): the first layer's front copies the
+    input into the operand layout without a conversion, and the output is written in fp16.
+    The bf16 workload's values rounded to fp16 on the device; the oracle reads the same fp16
+    values (exact in float32)."""
+    cfg = dict(C.CONFIGS["c2_bf16"], dtype="f16")
+    batch = 300
+    host_layers, dev_layers = [], []
+    for l in range(cfg["layers"]):
+        d = C.make_layer_dev(C.CONFIGS["c2_bf16"], l)
+        h = C.make_layer_host(C.CONFIGS["c2_bf16"], l)
+        for key in ["Y", "W_L"] + ["W%d" % j for j in range(len(cfg["hidden"]) + 1)]:
+            d[key] = d[key].to(torch.float16)
+            h[key] = d[key].float().cpu().numpy()
+        dev_layers.append(d)
+        host_layers.append(h)
+    X = C.make_x_dev(C.CONFIGS["c2_bf16"], batch).to(torch.float16)
+    h = wk.wk_stack_create(cfg, dev_layers, max_batch=batch)
+    try:
+        out = torch.empty_like(X)
+        wk.wk_stack_forward(h, X, out)
+        torch.cuda.synchronize()
+        assert wk.wk_stack_sync_status(h) == wk.WK_OK
+        assert out.dtype == torch.float16
+        ex = _sample(batch, 16)
+        got = f64(out[ex])
+        ref = oracle.stack_forward(cfg, lambda l: host_layers[l], f64(X[ex]))
+        err = max_scaled_err(got, ref)
+        print("c2 shape, fp16 caller: max |gpu-ref|/(1+|ref|) = %.3g" % err)
+        assert err <= TOL["bf16"]
+    finally:
+        wk.wk_stack_destroy(h)
