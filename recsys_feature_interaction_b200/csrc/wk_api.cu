@@ -959,9 +959,8 @@ wk_status forward16(wk_stack* h, const void* X, void* out, int64_t batch, cudaSt
   }
   const wk_stack_config& c = h->cfg;
   const DevInfo* dv = h->dv;
-  const int n = c.n, d = c.d, k = c.k, m = c.mlp_num_linear, L = c.num_layers;
+  const int n = c.n, d = c.d, L = c.num_layers;
   const int64_t rows = batch * n;
-  const size_t nd = static_cast<size_t>(n) * d;
   wk_status s = WK_OK;
   const void* x0 = X;
   CUtensorMap lcb_x0;
