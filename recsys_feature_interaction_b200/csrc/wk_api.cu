@@ -809,7 +809,8 @@ wk_status build_maps(wk_stack* h) {
   // against d = 32, reads 11x its input's bytes of W_L and keeps the four-kernel layer, whose
   // LCB shares each W_L load among several examples)
   const bool front_lcb = c.n_l <= 2 * d;
-  if (h->tc_mlp && !h->front_only && shape >= 0 && front_types && front_lcb) {
+  const bool front_rows = static_cast<int64_t>(B) * n < (1ll << 31);  // A0 row coordinates are int32
+  if (h->tc_mlp && !h->front_only && shape >= 0 && front_types && front_lcb && front_rows) {
     const int KP = c.k <= 32 ? 32 : 64;
     h->fmaps.resize(L);
     bool ok = true;
