@@ -14,9 +14,13 @@ independent, so there is no collective in the forward): weak scaling.
 Rank 0 prints one JSON line. `value` is examples/s of the whole job with the
 inputs resident in HBM (CUDA events on the launch stream, max over ranks);
 `e2e` is the same metric through the public forward with pinned host buffers
-(host-to-device copy of X and device-to-host copy of the output inside the timed
-region; wk_stack_forward_host for a stack); `roofline` reports the MLP GEMM kernel (the dominant one) against the
-measured bf16 peak; `cpu_baseline` times the fp64 oracle on a bounded sample.
+(every step's host-to-device copy of X and device-to-host copy of the output inside
+the timed region): for a stack, the streamed host forward
+(wk_stack_forward_host_async, a serving loop that waits for step i-1's result after
+issuing step i), with the synchronous wk_stack_forward_host beside it in
+`e2e.synchronous_call`; `roofline` reports the MLP GEMM kernel (the dominant one)
+against the measured bf16 peak; `cpu_baseline` times the fp64 oracle on a bounded
+sample.
 """
 import argparse
 import json
@@ -591,6 +595,7 @@ def main():
         replicas.finish()
         return
     moe = "experts" in cfg
+    host_stream = None
     B = cfg["batch"]
     # rank r works on examples [r*B, (r+1)*B) of the synthetic stream (no collective on the data path)
     first, _ = replicas.example_range(rank, world, B)
@@ -647,6 +652,20 @@ def main():
         def fwd_host(xh, oh):
             wk.wk_stack_forward_host(h, xh, oh)
         e2e_api = "wk_stack_forward_host (chunked copies overlapped with compute)"
+
+        def host_stream(xhs, ohs, steps):
+            # a serving loop: step i's input copy, forward and output copy are enqueued,
+            # then step i-1's result is waited for on the host
+            prev = None
+            for i in range(steps):
+                t = wk.wk_stack_forward_host_async(h, xhs[i % 2], ohs[i % 2])
+                if prev is not None:
+                    wk.wk_stack_host_wait(h, prev)
+                prev = t
+            wk.wk_stack_host_wait(h)
+        stream_api = ("wk_stack_forward_host_async + wk_stack_host_wait, a serving loop over two pairs of "
+                      "page-locked host buffers: step i+1's input copy and step i-1's output copy run while "
+                      "step i's forward computes, the whole batch per forward")
 
     barrier = replicas.barrier
 
@@ -724,6 +743,20 @@ def main():
         fwd_host(xh, oh)
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     e2e_value = world * B * args.steps / e2e_s
+    e2e_sync = None
+    if host_stream is not None:
+        # the next batch of this rank's examples as the second host input
+        x2 = C.make_x_dev(cfg, B, device=dev, first_example=first + world * B)
+        xhs = [xh, x2.cpu().pin_memory()]
+        del x2
+        ohs = [oh, torch.empty_like(oh).pin_memory()]
+        host_stream(xhs, ohs, 2)  # warm the slots
+        barrier()
+        t0 = time.perf_counter()
+        host_stream(xhs, ohs, args.steps)
+        s_s = max_over_ranks(time.perf_counter() - t0)
+        e2e_sync = {"value": e2e_value, "api": e2e_api}
+        e2e_value, e2e_api = world * B * args.steps / s_s, stream_api
     step_bytes = B * cfg["n"] * cfg["d"] * X.element_size()
     out_bytes = oh.numel() * oh.element_size()
 
@@ -775,6 +808,8 @@ def main():
                     "d2h_bytes_per_step": out_bytes, "api": e2e_api},
             "gpu_launches": launches_per_step * args.steps,
         }
+        if e2e_sync is not None:
+            line["e2e"]["synchronous_call"] = e2e_sync
         if world == 1 and not args.no_cpu_baseline:
             ns = ORACLE_SAMPLE[args.workload]
             v, dt, thr = oracle_sample(cfg, ns)

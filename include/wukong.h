@@ -34,7 +34,9 @@
  *   - Calls that take a stream are asynchronous and stream-ordered: they only
  *     validate their arguments on the host and enqueue kernels. They never
  *     synchronise and never copy between host and device, except
- *     wk_stack_forward_host, which is synchronous by design.
+ *     wk_stack_forward_host, which is synchronous by design, and
+ *     wk_stack_forward_host_async / wk_stack_host_wait, whose copies are waited
+ *     for by the second.
  *   - Every call returns a wk_status and never aborts the process. A kernel
  *     that detects a problem on the device (a pipeline wait that ran past its
  *     limit) records it in a device status word and returns early; read it with
@@ -146,6 +148,33 @@ WK_API wk_status wk_stack_forward(wk_stack* h, const void* X, void* out, int64_t
  * the full copy bandwidth; pageable ones work but copy slower. Chunks use the
  * handle's workspace and two staging buffers allocated on first use. */
 WK_API wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host, int64_t batch, wk_stream_t stream);
+
+/* The host-buffer forward for a stream of batches, as a serving loop issues them. The
+ * Wukong paper has no counterpart: it specifies the layer, not how batches reach the GPU.
+ * Enqueues the copy of X_host into one of two device input slots, one wk_stack_forward
+ * of the whole batch on `stream`, and the copy of its result into out_host, then returns
+ * without waiting. Successive calls alternate the slots, so the input copy of call i+1
+ * and the output copy of call i-1 run on internal copy streams while the forward of
+ * call i computes; each forward keeps the full batch (no chunking of the GEMMs).
+ * *ticket (may be NULL) receives the call's sequence number for wk_stack_host_wait.
+ * Ownership: the caller keeps X_host unchanged and does not touch out_host until
+ * wk_stack_host_wait has returned for this ticket or a later one; both must be
+ * page-locked for the copies to overlap (pageable buffers give the same result with
+ * copies that block the host). Successive calls on one handle use one stream (they
+ * share the workspace). The slots, 4 * max_batch * n * d elements of cfg->dtype, are
+ * allocated on the first call. batch == 0 is a no-op (*ticket = the last ticket, -1 if
+ * none). Errors: as wk_stack_forward, WK_ERR_OOM, WK_ERR_CUDA; on an error nothing of
+ * the call is left to wait for. */
+WK_API wk_status wk_stack_forward_host_async(wk_stack* h, const void* X_host, void* out_host, int64_t batch,
+                                             wk_stream_t stream, int64_t* ticket);
+
+/* Blocks the host until the output copy of wk_stack_forward_host_async call `ticket` has
+ * landed in its out_host, and with it the copies of every earlier call (ticket < 0: of
+ * every call made so far). A ticket more than two calls old may also wait for a later
+ * call's copy. WK_OK, WK_ERR_INVALID_ARG (NULL handle, a ticket not issued yet),
+ * WK_ERR_CUDA (a copy or a kernel it waited for failed). Device-side errors of the
+ * forwards are read with wk_stack_sync_status. */
+WK_API wk_status wk_stack_host_wait(wk_stack* h, int64_t ticket);
 
 /* Waits for `stream`, then reads and clears the device status word.
  * WK_OK, WK_ERR_TIMEOUT, WK_ERR_NONFINITE, WK_ERR_DEVICE or WK_ERR_CUDA.

@@ -86,6 +86,8 @@ def lib():
             "wk_stack_create": [ctypes.POINTER(WkStackConfig), ctypes.POINTER(WkLayerWeights), ctypes.POINTER(vp)],
             "wk_stack_forward": [vp, vp, vp, i64, vp],
             "wk_stack_forward_host": [vp, vp, vp, i64, vp],
+            "wk_stack_forward_host_async": [vp, vp, vp, i64, vp, ctypes.POINTER(i64)],
+            "wk_stack_host_wait": [vp, i64],
             "wk_stack_sync_status": [vp, vp],
             "wk_stack_set_profiling": [vp, ci],
             "wk_stack_kernel_times": [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)],
@@ -236,6 +238,21 @@ def wk_stack_forward_host(h, X_host, out_host, batch=None, stream=None):
     b = X_host.shape[0] if batch is None else batch
     _check(lib().wk_stack_forward_host(h.ptr, _addr(X_host), _addr(out_host), int(b), _stream(stream)),
            "wk_stack_forward_host")
+
+
+def wk_stack_forward_host_async(h, X_host, out_host, batch=None, stream=None):
+    """Enqueues input copy, forward and output copy; returns the call's ticket. X_host and
+    out_host (page-locked CPU tensors) must stay alive and untouched until
+    wk_stack_host_wait(h, ticket) returns."""
+    b = X_host.shape[0] if batch is None else batch
+    t = ctypes.c_int64(-1)
+    _check(lib().wk_stack_forward_host_async(h.ptr, _addr(X_host), _addr(out_host), int(b), _stream(stream),
+                                             ctypes.byref(t)), "wk_stack_forward_host_async")
+    return t.value
+
+
+def wk_stack_host_wait(h, ticket=-1):
+    _check(lib().wk_stack_host_wait(h.ptr, int(ticket)), "wk_stack_host_wait")
 
 
 def wk_stack_sync_status(h, stream=None):

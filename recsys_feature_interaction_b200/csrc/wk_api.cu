@@ -650,6 +650,11 @@ struct wk_stack {
   uint8_t* stage = nullptr;
   int64_t stage_chunk = 0;
   cudaStream_t s_in = nullptr, s_out = nullptr;
+  // streamed host-buffer forward: two input and two output slots of max_batch examples,
+  // per slot the events of its input copy, forward and output copy, and the calls issued
+  uint8_t* astage = nullptr;
+  cudaEvent_t a_in[2] = {nullptr, nullptr}, a_done[2] = {nullptr, nullptr}, a_out[2] = {nullptr, nullptr};
+  int64_t a_seq = 0;
   // profiling
   bool prof = false;
   struct Rec {
@@ -739,6 +744,12 @@ void free_stack(wk_stack* h) {
   if (h->head_ws) cudaFree(h->head_ws);
   if (h->stage) cudaFree(h->stage);
   if (h->bws) cudaFree(h->bws);
+  if (h->astage) cudaFree(h->astage);
+  for (int i = 0; i < 2; ++i) {
+    if (h->a_in[i]) cudaEventDestroy(h->a_in[i]);
+    if (h->a_done[i]) cudaEventDestroy(h->a_done[i]);
+    if (h->a_out[i]) cudaEventDestroy(h->a_out[i]);
+  }
   if (h->s_in) cudaStreamDestroy(h->s_in);
   if (h->s_out) cudaStreamDestroy(h->s_out);
   for (auto& r : h->recs) {
@@ -2086,6 +2097,76 @@ wk_status wk_stack_forward_host(wk_stack* h, const void* X_host, void* out_host,
   }
   cudaGetLastError();
   return s;
+}
+
+wk_status wk_stack_forward_host_async(wk_stack* h, const void* X_host, void* out_host, int64_t batch,
+                                      wk_stream_t stream, int64_t* ticket) {
+  if (!h || batch < 0 || batch > h->maxb) return WK_ERR_INVALID_ARG;
+  if (batch == 0) {
+    if (ticket) *ticket = h->a_seq - 1;
+    return WK_OK;
+  }
+  if (!X_host || !out_host) return WK_ERR_INVALID_ARG;
+  const size_t ex_bytes = static_cast<size_t>(h->cfg.n) * h->cfg.d * dtype_bytes(h->io);
+  const size_t slot = static_cast<size_t>(h->maxb) * ex_bytes;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!h->astage) {
+    if (cudaMalloc(&h->astage, 4 * slot) != cudaSuccess) {
+      cudaGetLastError();
+      h->astage = nullptr;
+      return WK_ERR_OOM;
+    }
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&h->a_in[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h->a_done[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h->a_out[i], cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        return WK_ERR_CUDA;
+      }
+  }
+  if (!h->s_in && cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking) != cudaSuccess) return WK_ERR_CUDA;
+  if (!h->s_out && cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking) != cudaSuccess) return WK_ERR_CUDA;
+  // Call i uses slot p = i % 2. Its input copy waits for the forward of call i-2 (the last
+  // reader of din); its forward waits for its input copy and for the output copy of call
+  // i-2 (the last reader of dout); its output copy waits for its forward. The caller's
+  // stream is not waited for by the copies, so the next call's input copy runs under this
+  // call's forward.
+  const int64_t i = h->a_seq;
+  const int p = static_cast<int>(i & 1);
+  uint8_t* din = h->astage + p * slot;
+  uint8_t* dout = h->astage + (2 + p) * slot;
+  const size_t nbytes = static_cast<size_t>(batch) * ex_bytes;
+  if (i >= 2 && cudaStreamWaitEvent(h->s_in, h->a_done[p], 0) != cudaSuccess) return WK_ERR_CUDA;
+  if (cudaMemcpyAsync(din, X_host, nbytes, cudaMemcpyHostToDevice, h->s_in) != cudaSuccess ||
+      cudaEventRecord(h->a_in[p], h->s_in) != cudaSuccess || cudaStreamWaitEvent(st, h->a_in[p], 0) != cudaSuccess ||
+      (i >= 2 && cudaStreamWaitEvent(st, h->a_out[p], 0) != cudaSuccess)) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  const wk_status s = wk_stack_forward(h, din, dout, batch, stream);
+  if (s != WK_OK) return s;
+  if (cudaEventRecord(h->a_done[p], st) != cudaSuccess || cudaStreamWaitEvent(h->s_out, h->a_done[p], 0) != cudaSuccess ||
+      cudaMemcpyAsync(out_host, dout, nbytes, cudaMemcpyDeviceToHost, h->s_out) != cudaSuccess ||
+      cudaEventRecord(h->a_out[p], h->s_out) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  h->a_seq = i + 1;
+  if (ticket) *ticket = i;
+  return WK_OK;
+}
+
+wk_status wk_stack_host_wait(wk_stack* h, int64_t ticket) {
+  if (!h || ticket >= h->a_seq) return WK_ERR_INVALID_ARG;
+  if (h->a_seq == 0) return WK_OK;
+  const int64_t t = ticket < 0 ? h->a_seq - 1 : ticket;
+  // the slot's event marks call t, or a later call of the same slot whose copy follows
+  // call t's on the output stream
+  if (cudaEventSynchronize(h->a_out[t & 1]) != cudaSuccess) {
+    cudaGetLastError();
+    return WK_ERR_CUDA;
+  }
+  return WK_OK;
 }
 
 wk_status wk_stack_sync_status(wk_stack* h, wk_stream_t stream) {

@@ -92,6 +92,10 @@ def test_create_without_device_reports_cuda_error(L):
 def test_null_handle_and_stand_alone_argument_checks(L):
     assert L.wk_stack_forward(None, FAKE, FAKE * 2, 1, None) == wk.WK_ERR_INVALID_ARG
     assert L.wk_stack_sync_status(None, None) == wk.WK_ERR_INVALID_ARG
+    t = ctypes.c_int64(7)
+    assert L.wk_stack_forward_host_async(None, FAKE, FAKE * 2, 1, None, ctypes.byref(t)) == wk.WK_ERR_INVALID_ARG
+    assert t.value == 7  # untouched on an error
+    assert L.wk_stack_host_wait(None, -1) == wk.WK_ERR_INVALID_ARG
     assert L.wk_stack_backward(None, FAKE, FAKE, FAKE, None, 8, None) == wk.WK_ERR_INVALID_ARG
     L.wk_stack_destroy(None)
     # misaligned pointers and bad sizes are rejected before any launch

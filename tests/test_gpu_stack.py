@@ -126,6 +126,38 @@ def test_batch_split_is_bitwise_and_host_path_matches():
         st.close()
 
 
+def test_streamed_host_forward_matches_the_device_forward():
+    # a serving loop: each call enqueues its input copy, forward and output copy; the
+    # previous call's result is waited for after the next call is issued, with two
+    # alternating pairs of page-locked host buffers and ragged batch sizes
+    cfg = C.CONFIGS["c2_bf16"]
+    st = DevStack("c2_bf16")
+    try:
+        B = cfg["batch"]
+        sizes = [B, 1000, B, 17, 2048, B]
+        xs = [C.make_x_dev(cfg, B, first_example=7 * B * j) for j in range(len(sizes))]
+        want = [st.run(x[:nb].contiguous()).cpu() for x, nb in zip(xs, sizes)]
+        xh = [torch.empty_like(xs[0], device="cpu").pin_memory() for _ in range(2)]
+        oh = [torch.empty_like(xs[0], device="cpu").pin_memory() for _ in range(2)]
+        got, prev = [], None
+        for j, nb in enumerate(sizes):
+            xh[j % 2][:nb].copy_(xs[j][:nb].cpu())
+            t = wk.wk_stack_forward_host_async(st.h, xh[j % 2], oh[j % 2], batch=nb)
+            if prev is not None:
+                wk.wk_stack_host_wait(st.h, prev[0])
+                got.append(oh[prev[1] % 2][:sizes[prev[1]]].clone())
+            prev = (t, j)
+        with pytest.raises(wk.WkError):
+            wk.wk_stack_host_wait(st.h, prev[0] + 1)  # not issued yet
+        wk.wk_stack_host_wait(st.h)
+        got.append(oh[prev[1] % 2][:sizes[prev[1]]].clone())
+        assert wk.wk_stack_sync_status(st.h) == wk.WK_OK
+        for j, (g, w) in enumerate(zip(got, want)):
+            assert torch.equal(g, w), "call %d" % j
+    finally:
+        st.close()
+
+
 def test_profiling_counts_launches():
     cfg = C.CONFIGS["c2_bf16"]
     st = DevStack("c2_bf16")
