@@ -45,7 +45,7 @@ constexpr int FRONT_NORM_WARP0 = 7;   // warps 7..14: normalisation
 constexpr int FRONT_NORM_THREADS = 256;
 constexpr int FRONT_SMEM_LIMIT = 232448;
 
-template <int N_, int D_, int K_, int NF_>
+template <int N_, int D_, int K_, int NF_, bool LCB_DIRECT_>
 struct FrontCfg {
   static constexpr int N = N_, D = D_, K = K_, NF = NF_, NL = N_ - NF_;
   static constexpr int R = 128;                              // rows per chunk = MMA M
@@ -96,6 +96,11 @@ struct FrontCfg {
   // A0 leaves through TMA stores of 32 x 32 tiles in the three-pass LayerNorm (k = 64, whole
   // chunks), staged in three 2 KB tiles per epilogue warp: its own and two in the Z region
   static constexpr bool A0_TMA = !REGLN && K == 64 && N % R == 0 && ZB >= 4 * 4096;
+  // the LCB rows leave by 16-byte stores of the epilogue warps, each box transposed through
+  // the warp's own staging tile (the Y / W_L ring is not borrowed, so it streams the next
+  // example's stages while the rows are read out), else by TMA stores staged in the
+  // warp's tile and its quarter of the ring; chosen per shape by measurement
+  static constexpr bool LCB_DIRECT = LCB_DIRECT_;
   static_assert(D % 32 == 0 && D <= 256 && N % 16 == 0 && K % 4 == 0 && K <= 64, "shape");
   static_assert(NSTG >= 2 && SMEM <= FRONT_SMEM_LIMIT, "shared memory");
   static_assert(TCOLS <= 512, "TMEM columns");
@@ -131,6 +136,50 @@ __device__ __forceinline__ void front_tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
                : "memory");
 }
 
+// Two fp32 values in one 64-bit register pair, for the packed fp32 instructions of sm_100
+// (add / mul / fma .f32x2: one instruction for two lanes of the per-element LayerNorm work,
+// each lane rounded as its scalar instruction would be).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ float f2_sum(uint64_t r) {
+  float lo, hi;
+  f2_unpack(r, lo, hi);
+  return lo + hi;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// The two 16-bit values of type TI in a 32-bit word as an fp32 pair.
+template <typename TI>
+__device__ __forceinline__ uint64_t f2_from16(uint32_t w) {
+  return f2_pack(Half16<TI>::lo(w), Half16<TI>::hi(w));
+}
+// An fp32 pair rounded to two 16-bit values of type TO in a 32-bit word.
+template <typename TO>
+__device__ __forceinline__ uint32_t f2_to16(uint64_t r) {
+  float lo, hi;
+  f2_unpack(r, lo, hi);
+  return Half16<TO>::pack2(lo, hi);
+}
+
 // Eight 16-bit values of type TI (one 16-byte unit) as floats.
 template <typename TI>
 __device__ __forceinline__ void front_unpack8(const uint4& a, float (&v)[8]) {
@@ -145,6 +194,16 @@ __device__ __forceinline__ uint4 front_pack8(const float (&v)[8]) {
   a.z = Half16<TO>::pack2(v[4], v[5]);
   a.w = Half16<TO>::pack2(v[6], v[7]);
   return a;
+}
+
+// Row `row` of a 32 x 32 16-bit staging tile (64-byte rows, 64-byte swizzle) from 16 words
+// of two packed 16-bit values each.
+__device__ __forceinline__ void front_stage16(uint8_t* buf, int row, const uint32_t (&o)[16]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int pc = c ^ ((row >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + row * 64 + pc * 16) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+  }
 }
 
 // xin: the layer input [batch, n, d] of type TIN (16-byte aligned). Tensor maps:
@@ -163,7 +222,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmA,
                     const float* __restrict__ in_g,
                     const float* __restrict__ in_b, const float* __restrict__ fg, const float* __restrict__ fb,
-                    T* __restrict__ A0, int64_t batch, float eps, unsigned* status) {
+                    T* __restrict__ A0, T* __restrict__ yout, int64_t batch, float eps, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* slots = smem;                                     // [ES][NCH] chunks of the layer inputs
@@ -186,7 +245,9 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
   uint64_t* fempty = zfull + 4;                              // epilogue -> MMA: F read
   uint64_t* fin = zfull + 5;                                 // MMA: its last operations completed
   uint64_t* lfull = zfull + 6;                               // [MTL] MMA -> epilogue: LCB tile m in TMEM
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lfull + C::MTL);
+  uint64_t* fcfree = lfull + C::MTL;                         // [NCH] epilogue -> MMA: the LCB
+                                                             // columns F chunk c reuses are read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fcfree + C::NCH);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -211,6 +272,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
     }
     mbar_init(zfull, 1);
     for (int m = 0; m < C::MTL; ++m) mbar_init(&lfull[m], 1);
+    for (int c = 0; c < C::NCH; ++c) mbar_init(&fcfree[c], 4);
     mbar_init(ffull, 1);
     mbar_init(zready, 4);
     mbar_init(ldone, 4);
@@ -270,7 +332,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       bool ok = true;
       for (int64_t b = blockIdx.x; ok && b < batch; b += gridDim.x, ++i) {
         // the epilogue stages the previous example's LCB rows in the ring: wait until it is done
-        if (i > 0 && !mbar_wait(ldone, static_cast<uint32_t>((i - 1) & 1), status)) {
+        if (!C::LCB_DIRECT && i > 0 && !mbar_wait(ldone, static_cast<uint32_t>((i - 1) & 1), status)) {
           ok = false;
           break;
         }
@@ -385,15 +447,22 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         if (!ok) break;
         for (int m = 0; m < C::MTL; ++m) umma_commit(&lfull[m]);
         // pass B: F = X Z, once Z is in shared memory and F's TMEM columns are free: the
-        // previous example's F has been read (F apart) or this example's LCB rows have been
-        // read (F in the LCB's columns)
-        if (!mbar_wait(zready, par, status) ||
-            !(C::SEPF ? (i == 0 || mbar_wait(fempty, par ^ 1u, status)) : mbar_wait(ldone, par, status))) {
+        // previous example's F has been read (F apart), or, chunk by chunk, the LCB columns
+        // that F_c reuses have been read out (F in the LCB's columns), so pass B runs while
+        // the rest of the LCB rows are read out
+        if (!mbar_wait(zready, par, status) || !(!C::SEPF || i == 0 || mbar_wait(fempty, par ^ 1u, status))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int c = 0; c < C::NCH; ++c) {
+        for (int c = 0; ok && c < C::NCH; ++c) {
+          if constexpr (!C::SEPF) {
+            if (!mbar_wait(&fcfree[c], par, status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
           const uint32_t xs = slot0 + (es * C::NCH + c) * C::CHB;
 #pragma unroll
           for (int ks = 0; ks < C::D / 16; ++ks) {
@@ -403,6 +472,7 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           }
           umma_commit(&empty[es * C::NCH + c]);  // pass B has read the chunk's slot
         }
+        if (!ok) break;
         umma_commit(ffull);
       }
       if (issued) {  // no MMA may still read shared memory or write TMEM when the CTA exits
@@ -461,7 +531,13 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       // LCB rows: accumulator + the residual X row (from the chunk in shared memory), staged
       // 32 columns at a time and stored by TMA (rows past n_l are clipped), through this warp's
       // own staging tile and its quarter of the Y / W_L ring, idle until the drain is done
+      // chunks holding no LCB row's residual are not read here: with one example in flight
+      // (the next one's loads wait for these slots) they are released now, else with the rest
+      constexpr int EARLY = C::ES == 1 ? C::NF / C::R : 0;
+      if (lane == 0)
+        for (int c = 0; c < EARLY; ++c) mbar_arrive(&empty[es * C::NCH + c]);
       for (int c = C::NF / C::R; ok && c < C::NCH; ++c) ok = mbar_wait(&xready[es * C::NCH + c], sp, status);
+      int fsig = 0;  // F chunks whose LCB columns this warp has read (F in the LCB's columns)
 #pragma unroll 1
       for (int m = 0; m < C::MTL; ++m) {
         if (ok) ok = mbar_wait(&lfull[m], par, status);
@@ -477,38 +553,72 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           uint32_t acc[32];
           tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::LCOL + m * C::D + j * 32), acc);
           tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(acc[e]);
+          if constexpr (!C::SEPF) {
+            const int read = m * C::D + 32 * (j + 1);  // LCB columns read so far
+            if (fsig < C::NCH && (fsig + 1) * C::KP <= read) {
+              tc_fence_before();
+              __syncwarp();
+              while (fsig < C::NCH && (fsig + 1) * C::KP <= read) {
+                if (lane == 0) mbar_arrive(&fcfree[fsig]);
+                ++fsig;
+              }
+            }
+          }
+          uint32_t o[16];
           if (valid) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const uint4 xr = *reinterpret_cast<const uint4*>(xres + j * C::XBOXB + sw64_off(rl, u));
-              float x8[8];
-              front_unpack8<T>(xr, x8);
+              const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
-              for (int e = 0; e < 8; ++e) v[8 * u + e] += x8[e];
+              for (int p = 0; p < 4; ++p)
+                o[4 * u + p] = f2_to16<T>(f2_add(f2_pack(__uint_as_float(acc[8 * u + 2 * p]),
+                                                         __uint_as_float(acc[8 * u + 2 * p + 1])),
+                                                 f2_from16<T>(xw[p])));
             }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = Half16<T>::pack2(__uint_as_float(acc[2 * e]), __uint_as_float(acc[2 * e + 1]));
           }
-          const int nb = (m * C::XBOXES + j) % C::NBUF;
-          uint8_t* stage = nb == 0 ? epi + ew * 2048 : ring + ew * (C::NBUF - 1) * 2048 + (nb - 1) * 2048;
-          if (lane == 0 && nb == 0) bulk_wait_read<0>();  // the tiles' last stores have read them
-          __syncwarp();
-          stage_row<T>(stage, lane, v);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && any) {
-            tma_store_3d(&tmL, stage, 32 * j, m * C::R + q * 32, static_cast<int32_t>(b));
-            bulk_commit();
+          if constexpr (C::LCB_DIRECT) {
+            // through the warp's own 2 KB tile: each lane writes its row, then each store
+            // instruction of the warp covers 8 whole 64-byte row segments (lane = 16 bytes)
+            uint8_t* tile = epi + ew * 2048;
+            front_stage16(tile, lane, o);
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int tr = it * 8 + (lane >> 2);  // tile row
+              const int u = lane & 3;               // its 16-byte unit
+              const uint4 val = *reinterpret_cast<const uint4*>(tile + sw64_off(tr, u));
+              const int r2 = m * C::R + q * 32 + tr;  // LCB row
+              if (r2 < C::NL)
+                *reinterpret_cast<uint4*>(yout + (b * C::N + C::NF + r2) * C::D + 32 * j + 8 * u) = val;
+            }
+            __syncwarp();  // the tile is read before the next box is written into it
+          } else {
+            const int nb = (m * C::XBOXES + j) % C::NBUF;
+            uint8_t* stage = nb == 0 ? epi + ew * 2048 : ring + ew * (C::NBUF - 1) * 2048 + (nb - 1) * 2048;
+            if (lane == 0 && nb == 0) bulk_wait_read<0>();  // the tiles' last stores have read them
+            __syncwarp();
+            front_stage16(stage, lane, o);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && any) {
+              tma_store_3d(&tmL, stage, 32 * j, m * C::R + q * 32, static_cast<int32_t>(b));
+              bulk_commit();
+            }
           }
         }
       }
       tc_fence_before();
-      if (lane == 0) bulk_wait_read<0>();  // the ring is the producer's again
+      if (!C::LCB_DIRECT && lane == 0) bulk_wait_read<0>();  // the ring is the producer's again
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(ldone);
-        for (int c = 0; c < C::NCH; ++c) mbar_arrive(&empty[es * C::NCH + c]);  // residual rows read
+        for (int c = EARLY; c < C::NCH; ++c) mbar_arrive(&empty[es * C::NCH + c]);  // residual rows read
+        if constexpr (!C::SEPF)
+          for (; fsig < C::NCH; ++fsig) mbar_arrive(&fcfree[fsig]);  // F past the LCB's columns
       }
 
       // the FMB LayerNorm over the n*k values of F
@@ -536,32 +646,38 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(fempty);
-        float part = 0.f;
+        uint64_t pa = 0, pb = 0;  // +0.0f pairs
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const int row = c * C::R + q * 32 + lane;
           if (row < C::N) {
 #pragma unroll
-            for (int j = 0; j < C::K; ++j) part += __uint_as_float(fr[c][j]);
-          }
-        }
-        part = warp_sum(part);
-        if (lane == 0) red[ew] = part;
-        named_bar(1, 128);
-        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
-        float qs = 0.f;
-#pragma unroll
-        for (int c = 0; c < C::NCH; ++c) {
-          const int row = c * C::R + q * 32 + lane;
-          if (row < C::N) {
-#pragma unroll
-            for (int j = 0; j < C::K; ++j) {
-              const float dv = __uint_as_float(fr[c][j]) - mean;
-              qs = fmaf(dv, dv, qs);
+            for (int j = 0; j < C::K; j += 4) {
+              pa = f2_add(pa, f2_pack(__uint_as_float(fr[c][j]), __uint_as_float(fr[c][j + 1])));
+              pb = f2_add(pb, f2_pack(__uint_as_float(fr[c][j + 2]), __uint_as_float(fr[c][j + 3])));
             }
           }
         }
-        qs = warp_sum(qs);
+        float part = warp_sum(f2_sum(pa) + f2_sum(pb));
+        if (lane == 0) red[ew] = part;
+        named_bar(1, 128);
+        const float mean = (red[0] + red[1] + red[2] + red[3]) * inv_cnt;
+        const uint64_t nm2 = f2_pack(-mean, -mean);
+        uint64_t qa = 0, qb = 0;
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int row = c * C::R + q * 32 + lane;
+          if (row < C::N) {
+#pragma unroll
+            for (int j = 0; j < C::K; j += 4) {
+              const uint64_t da = f2_add(f2_pack(__uint_as_float(fr[c][j]), __uint_as_float(fr[c][j + 1])), nm2);
+              const uint64_t db = f2_add(f2_pack(__uint_as_float(fr[c][j + 2]), __uint_as_float(fr[c][j + 3])), nm2);
+              qa = f2_fma(da, da, qa);
+              qb = f2_fma(db, db, qb);
+            }
+          }
+        }
+        float qs = warp_sum(f2_sum(qa) + f2_sum(qb));
         if (lane == 0) red[4 + ew] = qs;
         named_bar(1, 128);
         const float var = (red[4] + red[5] + red[6] + red[7]) * inv_cnt;
@@ -572,18 +688,24 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           const int row = c * C::R + q * 32 + lane;
           if (row < C::N) {
             T* o = ab + row * C::K;
+            const uint64_t rs2 = f2_pack(rstd, rstd);
 #pragma unroll
             for (int j = 0; j < C::K; j += 8) {
-              float v[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = (__uint_as_float(fr[c][j + e]) - mean) * rstd;
               if (affine) {
+                float v[8];
                 const float* gp = fg + row * C::K + j;
                 const float* bp = fb + row * C::K + j;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = v[e] * __ldg(gp + e) + __ldg(bp + e);
+                for (int e = 0; e < 8; ++e) v[e] = (__uint_as_float(fr[c][j + e]) - mean) * rstd * __ldg(gp + e) + __ldg(bp + e);
+                *reinterpret_cast<uint4*>(o + j) = front_pack8<T>(v);
+              } else {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  w4[e] = f2_to16<T>(f2_mul(f2_add(f2_pack(__uint_as_float(fr[c][j + 2 * e]),
+                                                           __uint_as_float(fr[c][j + 2 * e + 1])), nm2), rs2));
+                *reinterpret_cast<uint4*>(o + j) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
               }
-              *reinterpret_cast<uint4*>(o + j) = front_pack8<T>(v);
             }
           }
         }
@@ -596,7 +718,8 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         // Q - 2 (mean - s) S + n (mean - s)^2, and is reduced second.
         if (ok) ok = mbar_wait(ffull, par, status);
         tc_fence_after();
-        float sh = 0.f, sx = 0.f, sq = 0.f, cnt = 0.f;
+        float sh = 0.f, cnt = 0.f;
+        uint64_t nsh = 0, sxa = 0, sxb = 0, sqa = 0, sqb = 0;  // +0.0f pairs
 #pragma unroll 1
         for (int c = 0; c < C::NCH; ++c) {
           const int row = c * C::R + q * 32 + lane;
@@ -605,20 +728,27 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           for (int h = 0; h < C::KP / 32; ++h)
             tmem_ld32(tmem_base + lane_base + static_cast<uint32_t>(C::FCOL + c * C::KP + h * 32), r[h]);
           tmem_ld_wait();
-          if (c == 0) sh = __uint_as_float(r[0][0]);
+          if (c == 0) {
+            sh = __uint_as_float(r[0][0]);
+            nsh = f2_pack(-sh, -sh);
+          }
           if (row < C::N) {
 #pragma unroll
             for (int h = 0; h < C::KP / 32; ++h)
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (h * 32 + j < C::K) {
-                  const float dv = __uint_as_float(r[h][j]) - sh;
-                  sx += dv;
-                  sq = fmaf(dv, dv, sq);
+              for (int j = 0; j < 32; j += 4)
+                if (h * 32 + j < C::K) {  // K % 4 == 0
+                  const uint64_t da = f2_add(f2_pack(__uint_as_float(r[h][j]), __uint_as_float(r[h][j + 1])), nsh);
+                  const uint64_t db = f2_add(f2_pack(__uint_as_float(r[h][j + 2]), __uint_as_float(r[h][j + 3])), nsh);
+                  sxa = f2_add(sxa, da);
+                  sqa = f2_fma(da, da, sqa);
+                  sxb = f2_add(sxb, db);
+                  sqb = f2_fma(db, db, sqb);
                 }
             cnt += static_cast<float>(C::K);
           }
         }
+        const float sx = f2_sum(sxa) + f2_sum(sxb), sq = f2_sum(sqa) + f2_sum(sqb);
         float part = warp_sum(sx + cnt * sh);
         if (lane == 0) red[ew] = part;
         named_bar(1, 128);
@@ -640,22 +770,31 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int h = 0; h < C::KP / 32; ++h) {
-            float v[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = (__uint_as_float(rr[h][e]) - mean) * rstd;
+            uint32_t o[16];
             if (affine && row < C::N) {
+              float v[32];
               const float* gp = fg + row * C::K + h * 32;
               const float* bp = fb + row * C::K + h * 32;
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
+              for (int e = 0; e < 32; ++e) {
+                v[e] = (__uint_as_float(rr[h][e]) - mean) * rstd;
                 if (h * 32 + e < C::K) v[e] = v[e] * __ldg(gp + e) + __ldg(bp + e);
+              }
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = Half16<T>::pack2(v[2 * e], v[2 * e + 1]);
+            } else {
+              const uint64_t nm2 = f2_pack(-mean, -mean), rs2 = f2_pack(rstd, rstd);
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                o[e] = f2_to16<T>(f2_mul(f2_add(f2_pack(__uint_as_float(rr[h][2 * e]), __uint_as_float(rr[h][2 * e + 1])),
+                                                nm2), rs2));
             }
             if constexpr (C::A0_TMA) {
               const int t = c * 2 + h;  // tile, three staging buffers in turn
               uint8_t* buf = (t % 3 == 0) ? epi + ew * 2048 : zb + ew * 4096 + (t % 3 - 1) * 2048;
               if (lane == 0) bulk_wait_read<2>();  // the store that last used this buffer has read it
               __syncwarp();
-              stage_row<T>(buf, lane, v);
+              front_stage16(buf, lane, o);
               fence_proxy_async_smem();
               __syncwarp();
               if (lane == 0) {
@@ -663,11 +802,11 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
                 bulk_commit();
               }
             } else if (row < C::N) {
-              T* o = ab + row * C::K + h * 32;
+              T* op = ab + row * C::K + h * 32;
 #pragma unroll
               for (int j = 0; j < 32; j += 8)
                 if (h * 32 + j < C::K)
-                  *reinterpret_cast<uint4*>(o + j) = front_pack8<T>(reinterpret_cast<const float(&)[8]>(v[j]));
+                  *reinterpret_cast<uint4*>(op + j) = make_uint4(o[j / 2], o[j / 2 + 1], o[j / 2 + 2], o[j / 2 + 3]);
             }
           }
         }
@@ -712,22 +851,24 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
         if (ln_in) {
           // one pass over the row for its statistics: sums of (x - s) and (x - s)^2 around the
           // row's first value s (both threads of the row use it), no cancellation for rows far
-          // from 0
-          float v0[8];
-          front_unpack8<TIN>(w[0], v0);
-          const float sh = __shfl_sync(0xffffffffu, v0[0], lane & ~1);
-          float sx = 0.f, sq = 0.f;
+          // from 0; fp32 pairs in two accumulator sets, so no chain is longer than UPT * 2
+          const float sh = __shfl_sync(0xffffffffu, Half16<TIN>::lo(w[0].x), lane & ~1);
+          const uint64_t nsh = f2_pack(-sh, -sh);
+          uint64_t sxa = 0, sxb = 0, sqa = 0, sqb = 0;  // +0.0f pairs
 #pragma unroll
           for (int k = 0; k < UPT; ++k) {
-            float v[8];
-            front_unpack8<TIN>(w[k], v);
+            const uint32_t ww[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float dv = v[e] - sh;
-              sx += dv;
-              sq = fmaf(dv, dv, sq);
+            for (int p = 0; p < 4; p += 2) {
+              const uint64_t da = f2_add(f2_from16<TIN>(ww[p]), nsh);
+              const uint64_t db = f2_add(f2_from16<TIN>(ww[p + 1]), nsh);
+              sxa = f2_add(sxa, da);
+              sqa = f2_fma(da, da, sqa);
+              sxb = f2_add(sxb, db);
+              sqb = f2_fma(db, db, sqb);
             }
           }
+          float sx = f2_sum(sxa) + f2_sum(sxb), sq = f2_sum(sqa) + f2_sum(sqb);
           sx += __shfl_xor_sync(0xffffffffu, sx, 1);
           sq += __shfl_xor_sync(0xffffffffu, sq, 1);
           const float dmean = sx * (1.0f / C::D);
@@ -736,18 +877,25 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
           const float rstd = rsqrtf(qv * (1.0f / C::D) + eps);
           if (act && half == 0 && !(isfinite(mean) && isfinite(qv))) flag_error(status, kFlagNonFinite);
           if (act) {
+            const uint64_t nm2 = f2_pack(-mean, -mean), rs2 = f2_pack(rstd, rstd);
 #pragma unroll
             for (int k = 0; k < UPT; ++k) {
               const int g = half * UPT + k;
-              float v[8];
-              front_unpack8<TIN>(w[k], v);
-              const float4 g0 = reinterpret_cast<const float4*>(sg)[2 * g], g1 = reinterpret_cast<const float4*>(sg)[2 * g + 1];
-              const float4 b0 = reinterpret_cast<const float4*>(sb)[2 * g], b1 = reinterpret_cast<const float4*>(sb)[2 * g + 1];
-              const float ga[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-              const float be[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              const uint32_t ww[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+              const ulonglong2 g0 = reinterpret_cast<const ulonglong2*>(sg)[2 * g];
+              const ulonglong2 g1 = reinterpret_cast<const ulonglong2*>(sg)[2 * g + 1];
+              const ulonglong2 b0 = reinterpret_cast<const ulonglong2*>(sb)[2 * g];
+              const ulonglong2 b1 = reinterpret_cast<const ulonglong2*>(sb)[2 * g + 1];
+              const uint64_t ga[4] = {g0.x, g0.y, g1.x, g1.y};
+              const uint64_t be[4] = {b0.x, b0.y, b1.x, b1.y};
+              uint32_t o[4];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = (v[e] - mean) * rstd * ga[e] + be[e];
-              *reinterpret_cast<uint4*>(base + (g >> 2) * C::XBOXB + sw64_off(row, g & 3)) = front_pack8<T>(v);
+              for (int p = 0; p < 4; ++p) {
+                // ((x - mean) * rstd) * gamma + beta, lane by lane
+                const uint64_t t = f2_mul(f2_add(f2_from16<TIN>(ww[p]), nm2), rs2);
+                o[p] = f2_to16<T>(f2_fma(t, ga[p], be[p]));
+              }
+              *reinterpret_cast<uint4*>(base + (g >> 2) * C::XBOXB + sw64_off(row, g & 3)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
           }
         } else if (act) {  // the first layer: the input in the operand type, in the operand layout
@@ -802,8 +950,11 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
   }
 }
 
-using FrontC2 = FrontCfg<64, 128, 16, 32>;
-using FrontC3 = FrontCfg<256, 160, 32, 128>;
-using FrontC4 = FrontCfg<512, 160, 64, 256>;
+// LCB rows by direct stores where that measured faster (the 2- and 8-layer shapes: 0.100 ->
+// 0.087 ms and 0.522 -> 0.506 ms per launch; the 4-layer shape: 0.686 -> 0.711 ms, so it keeps
+// the TMA stores)
+using FrontC2 = FrontCfg<64, 128, 16, 32, true>;
+using FrontC3 = FrontCfg<256, 160, 32, 128, false>;
+using FrontC4 = FrontCfg<512, 160, 64, 256, true>;
 
 }  // namespace wk

@@ -414,24 +414,24 @@ struct FrontMaps {
 
 template <class C, typename TIN, typename T>
 wk_status run_front_c(const DevInfo* dv, const FrontMaps& mp, const TIN* xin, const float* in_g, const float* in_b,
-                      const float* fg, const float* fb, T* A0, int64_t batch, float eps, unsigned* status,
+                      const float* fg, const float* fb, T* A0, T* yout, int64_t batch, float eps, unsigned* status,
                       cudaStream_t st) {
   wk_status s = smem_attr(dv, reinterpret_cast<const void*>(front_tc_kernel<C, TIN, T>), C::SMEM);
   if (s != WK_OK) return s;
   const int grid = static_cast<int>(std::min<int64_t>(batch, dv->sms));
   front_tc_kernel<C, TIN, T><<<grid, FRONT_THREADS, C::SMEM, st>>>(xin, mp.Y, mp.W, mp.R, mp.L, mp.A, in_g, in_b, fg,
-                                                                   fb, A0, batch, eps, status);
+                                                                   fb, A0, yout, batch, eps, status);
   return launch_status();
 }
 
 template <typename TIN, typename T>
 wk_status run_front(const DevInfo* dv, int shape, const FrontMaps& mp, const TIN* xin, const float* in_g,
-                    const float* in_b, const float* fg, const float* fb, T* A0, int64_t batch, float eps,
+                    const float* in_b, const float* fg, const float* fb, T* A0, T* yout, int64_t batch, float eps,
                     unsigned* status, cudaStream_t st) {
   switch (shape) {
-    case 0: return run_front_c<FrontC2, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, batch, eps, status, st);
-    case 1: return run_front_c<FrontC3, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, batch, eps, status, st);
-    case 2: return run_front_c<FrontC4, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, batch, eps, status, st);
+    case 0: return run_front_c<FrontC2, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, yout, batch, eps, status, st);
+    case 1: return run_front_c<FrontC3, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, yout, batch, eps, status, st);
+    case 2: return run_front_c<FrontC4, TIN, T>(dv, mp, xin, in_g, in_b, fg, fb, A0, yout, batch, eps, status, st);
     default: return WK_ERR_UNSUPPORTED;
   }
 }
@@ -934,10 +934,11 @@ wk_status forward16_front(wk_stack* h, const void* X, void* out, int64_t batch, 
       ProfScope ps(h, WK_KERNEL_FRONT, st);
       if (l == 0)
         s = run_front<IO, T>(dv, h->front, fm, static_cast<const IO*>(X), nullptr, nullptr, h->g1[l], h->b1[l],
-                             static_cast<T*>(h->A0), batch, h->eps, h->status, st);
+                             static_cast<T*>(h->A0), static_cast<T*>(h->Xs[o]), batch, h->eps, h->status, st);
       else
         s = run_front<T, T>(dv, h->front, fm, static_cast<const T*>(h->Xs[(l - 1) % 2]), h->g2[l - 1], h->b2[l - 1],
-                            h->g1[l], h->b1[l], static_cast<T*>(h->A0), batch, h->eps, h->status, st);
+                            h->g1[l], h->b1[l], static_cast<T*>(h->A0), static_cast<T*>(h->Xs[o]), batch, h->eps,
+                            h->status, st);
     }
     for (int j = 0; j < m && s == WK_OK; ++j) {
       ProfScope ps(h, WK_KERNEL_MLP_GEMM, st);
