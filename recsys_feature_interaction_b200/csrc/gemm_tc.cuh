@@ -33,6 +33,17 @@ namespace wk {
 
 enum { MODE_MLP = 0, MODE_LCB = 1 };
 
+// 4-D tiled TMA load (the LCB's X operand: 32 columns x 64 rows x d/32 column chunks x E
+// examples in one copy, landing as E * d/32 consecutive 64-row blocks of 32 columns).
+__device__ __forceinline__ void tma_load_4d(const CUtensorMap* m, uint64_t* bar, void* dst, int32_t c0, int32_t c1,
+                                            int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BN = 256;
 constexpr int GEMM_BK = 64;
@@ -195,11 +206,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if (MODE == MODE_MLP) {
             tma_load_2d(&tmB, &full[s], sB + s * GEMM_B_STAGE, kb * GEMM_BK, nt * GEMM_BN);
           } else {
-            uint8_t* dst = sB + s * GEMM_B_STAGE;
-            for (int e = 0; e < p.E; ++e)
-              for (int c = 0; c < p.dchunks; ++c)
-                tma_load_3d(&tmB, &full[s], dst + (e * p.dchunks + c) * 4096, c * 32, kb * GEMM_BK,
-                            nt * p.E + e);
+            // the E examples' 64-row K slices, every 32-column chunk, in one copy
+            tma_load_4d(&tmB, &full[s], sB + s * GEMM_B_STAGE, 0, kb * GEMM_BK, 0, nt * p.E);
           }
           if (++s == GEMM_STAGES) {
             s = 0;

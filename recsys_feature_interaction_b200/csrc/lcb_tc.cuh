@@ -13,7 +13,8 @@
 // need the same example's X run side by side and share it through L2.
 //
 // Warp roles as in gemm_tc.cuh (192 threads): warp 0 TMA producer (X as an MN-major
-// operand, 3-D boxes of 32 columns x 64 rows x one example, 64B swizzle), warp 1
+// operand, one 4-D box per K step: 32 columns x 64 rows x d/32 chunks x E examples, 64B
+// swizzle), warp 1
 // TMEM allocation + the single MMA-issuing thread (tcgen05.mma M = 128, N = E*d,
 // K = 16; two TMEM accumulators), warps 2..5 the epilogue (tcgen05.ld, 16-bit pack,
 // 3-D TMA store into the concat rows). Every wait is bounded.
@@ -110,10 +111,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], b_stage);
-          uint8_t* dst = sB + s * b_stage;
-          for (int e = 0; e < p.E; ++e)
-            for (int c = 0; c < p.dchunks; ++c)
-              tma_load_3d(&tmB, &full[s], dst + (e * p.dchunks + c) * 4096, c * 32, kb * GEMM_BK, nt * p.E + e);
+          // the E examples' 64-row K slices, every 32-column chunk, in one copy
+          tma_load_4d(&tmB, &full[s], sB + s * b_stage, 0, kb * GEMM_BK, 0, nt * p.E);
           if (++s == stages) {
             s = 0;
             ph ^= 1u;

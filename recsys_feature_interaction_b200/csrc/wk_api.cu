@@ -187,10 +187,13 @@ bool map_out(const DevInfo* dv, CUtensorMap* m, const void* p, uint64_t N, uint6
 // X [batch, n, d] as the LCB's MN-major operand: box (32 t, 64 i, 1 b), 64B swizzle.
 template <typename T>
 bool map_lcb_x(const DevInfo* dv, CUtensorMap* m, const void* X, uint64_t n, uint64_t d, uint64_t batch) {
-  const uint64_t dims[3] = {d, n, batch};
-  const uint64_t str[2] = {d * 2, n * d * 2};
-  const uint32_t box[3] = {32, 64, 1};
-  return make_map(dv, m, tmap_dtype<T>(), 3, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  // X [batch, n, d] as (32 columns, n rows, d/32 column chunks, batch): one box is a K step of
+  // E = GEMM_BN / d examples, landing as E x d/32 blocks of 64 rows x 32 columns in that order
+  // (the B operand layout of the LCB kernels)
+  const uint64_t dims[4] = {32, n, d / 32, batch};
+  const uint64_t str[3] = {d * 2, 64, n * d * 2};
+  const uint32_t box[4] = {32, 64, static_cast<uint32_t>(d / 32), static_cast<uint32_t>(GEMM_BN / d)};
+  return make_map(dv, m, tmap_dtype<T>(), 4, X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // Rows n_f..n_f+n_l-1 of a [batch, rows, d] concat buffer as a (t, r, b) tensor: box (32, 32, 1).
