@@ -22,6 +22,10 @@ int main(void) {
   expect(wk_status_string(WK_ERR_UNSUPPORTED) != NULL, "status string of WK_ERR_UNSUPPORTED");
   /* null handles and null arguments are rejected without a device */
   expect(wk_stack_forward(NULL, dummy, dummy, 1, NULL) == WK_ERR_INVALID_ARG, "forward, null handle");
+  int64_t ticket = 7;
+  expect(wk_stack_forward_host_async(NULL, dummy, dummy, 1, NULL, &ticket) == WK_ERR_INVALID_ARG && ticket == 7,
+         "streamed host forward, null handle");
+  expect(wk_stack_host_wait(NULL, -1) == WK_ERR_INVALID_ARG, "host wait, null handle");
   expect(wk_stack_backward(NULL, dummy, dummy, dummy, NULL, 8, NULL) == WK_ERR_INVALID_ARG, "backward, null handle");
   expect(wk_stack_backward_events(NULL, dummy, dummy, dummy, NULL, 8, NULL, NULL) == WK_ERR_INVALID_ARG,
          "backward with events, null handle");
