@@ -367,9 +367,10 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
     // After a failed wait (status flagged) a warp stops waiting but keeps walking
     // the same control flow, so every named barrier still sees all four warps.
     bool ok = true;
-    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
-      // Z (TMEM, fp32) -> 16-bit MN-major operand in shared memory
-      if (ok) ok = mbar_wait(zfull, eph, status);
+    // Z (TMEM, fp32) -> 16-bit MN-major operand in shared memory, for the example whose
+    // zfull / zready phase has parity zpar
+    auto z_convert = [&](uint32_t zpar) {
+      if (ok) ok = mbar_wait(zfull, zpar, status);
       tc_fence_after();
 #pragma unroll
       for (int mz = 0; mz < C::MTZ; ++mz) {
@@ -398,6 +399,13 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(zready);
+    };
+    // With the LayerNorm in registers, the next example's Z is converted as soon as this
+    // example's F is in registers (pass B has read the Z operand by then), so the next
+    // pass B runs while this LayerNorm is computed; else each example's Z first.
+    if (C::REGLN && blockIdx.x < batch) z_convert(0u);
+    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
+      if (!C::REGLN) z_convert(eph);
 
       if constexpr (C::REGLN) {
         // The LayerNorm from registers: each thread's F values (one row per chunk, k
@@ -423,6 +431,7 @@ __global__ void __launch_bounds__(FMTC_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(fempty);  // F is in registers: the next pass B may overwrite it
+        if (b + gridDim.x < batch) z_convert(eph ^ 1u);
         float part = 0.f;
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
