@@ -23,12 +23,15 @@
 //                           small ring of 16 KB stages from L2);
 //   pass B  F = X Z         M = n (one tile per chunk), N = KP, K = d (Z written back to
 //                           shared memory as a 16-bit operand by the epilogue warps).
-// TMEM holds Z at column 0 and, from column LCOL, first the LCB accumulators and then F.
+// TMEM holds Z at column 0 and, from column LCOL, the LCB accumulators; F follows them where
+// TMEM has room (the 2- and 4-layer shapes) or reuses their columns chunk by chunk as the LCB
+// rows are read out (the 8-layer shape).
 //
 // Warps (480 threads): 0 loads input chunks; 1 allocates TMEM and issues the MMAs; 2 streams
 // Y and W_L; 3..6 are the epilogue (one TMEM lane quarter each: Z to shared memory, the LCB
-// rows plus residual out through TMA stores, the FMB LayerNorm of F into A0); 7..14
-// normalise each chunk as it lands (two threads per row) and store the FMB-row residual.
+// rows plus residual out, the FMB LayerNorm of F into A0); 7..14 normalise each chunk as it
+// lands (two threads per row) and store the FMB-row residual. The per-element passes (both
+// LayerNorms, the residual add) use the packed fp32x2 instructions.
 // Every mbarrier wait is bounded; after a failed wait each role stops, every copy in flight
 // lands and TMEM is freed before the CTA exits.
 #pragma once
@@ -528,9 +531,10 @@ __global__ void __launch_bounds__(FRONT_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(zready);
 
-      // LCB rows: accumulator + the residual X row (from the chunk in shared memory), staged
-      // 32 columns at a time and stored by TMA (rows past n_l are clipped), through this warp's
-      // own staging tile and its quarter of the Y / W_L ring, idle until the drain is done
+      // LCB rows: accumulator + the residual X row (from the chunk in shared memory), 32
+      // columns at a time: with LCB_DIRECT transposed through this warp's own tile and stored
+      // by the warp, else staged in that tile and its quarter of the Y / W_L ring (idle until
+      // the drain is done) and stored by TMA (rows past n_l are clipped)
       // chunks holding no LCB row's residual are not read here: with one example in flight
       // (the next one's loads wait for these slots) they are released now, else with the rest
       constexpr int EARLY = C::ES == 1 ? C::NF / C::R : 0;
