@@ -75,6 +75,8 @@ def test_mlp_linear_f32_simt():
     (5, 512, 160, 256, 256),   # one example per tile (E = 1), two W_L tiles
     (13, 720, 32, 360, 360),   # E = 8 with a ragged group, K tail (720 = 11*64 + 16), M tail (360)
     (7, 64, 128, 32, 32),      # E = 2, ragged group
+    (9, 128, 64, 64, 64),      # E = 4 examples x 2 column chunks per copy, ragged group
+    (11, 96, 96, 48, 48),      # E = 2 examples x 3 column chunks per copy, K and M tails
     (301, 512, 160, 256, 256),  # resident W_L: several example groups per CTA, the X ring wraps
     (1000, 256, 160, 128, 128),  # resident W_L, one m tile for every CTA
     (97, 200, 160, 100, 100),  # resident W_L with a K tail (200 = 3*64 + 8) and an M tail (100 rows)
