@@ -2120,11 +2120,13 @@ wk_status wk_stack_forward_host_async(wk_stack* h, const void* X_host, void* out
       h->astage = nullptr;
       return WK_ERR_OOM;
     }
-    for (int i = 0; i < 2; ++i)
-      if (cudaEventCreateWithFlags(&h->a_in[i], cudaEventDisableTiming) != cudaSuccess ||
-          cudaEventCreateWithFlags(&h->a_done[i], cudaEventDisableTiming) != cudaSuccess ||
-          cudaEventCreateWithFlags(&h->a_out[i], cudaEventDisableTiming) != cudaSuccess) {
+  }
+  for (int i = 0; i < 2; ++i) {
+    cudaEvent_t* evs[3] = {&h->a_in[i], &h->a_done[i], &h->a_out[i]};
+    for (cudaEvent_t* e : evs)
+      if (!*e && cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) {
         cudaGetLastError();
+        *e = nullptr;
         return WK_ERR_CUDA;
       }
   }
